@@ -1,0 +1,144 @@
+"""CPU reference for the sparse-attention metadata (selection -> per-unit KV lists, transposed
+lists, per-page lists and the balanced per-SM work list).
+
+TEST INFRASTRUCTURE.  Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg may
+import this module; it shares no code with the CUDA path.
+
+The SparseAttnSharedkvMetadata page describes an operator that, ahead of the attention call,
+writes a task list giving each compute core the start and end (batch, head, Q block, K block) of
+its share of the work.  The reference here defines the integer products our device metadata
+must reproduce bit-exactly:
+
+  * BSA KV lists (BlockSparseAttentionGrad page: "BlockSparseMask specifies the KV block
+    selected by each Q block"): units in (b, h, qb) order; each unit's KV block ids ascending.
+  * BSA transposed lists (needed by dK/dV, backward formulas dV = P^T dOut, dK = dS^T Q scale):
+    per (b, kv head g, kv block kb) the ascending entries h_local * nqb + qb of the query blocks
+    (of the group's query heads) that selected kb.
+  * NSA lists (NsaSelectedAttention page, Gather(key, topk_indices[i])): per (token, kv head) the
+    valid ids ascending (duplicates kept, -1 dropped, ids past the batch's block count dropped
+    and flagged); per (b, g, kb) the ascending global token indices that selected kb (a token
+    appears once per time it lists kb).
+  * SFA page lists (SparseFlashAttention page: sparse_block_size is a multiple of block_size):
+    per (b, kv head) the physical pages of the selected sparse blocks, in list order.
+  * Work list: see `work_cuts`.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BAD_INDEX = 1  # device status bit: an index at or past the sequence's block count was dropped
+
+
+def csr_from_lists(lists):
+    row_ptr = np.zeros(len(lists) + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum([len(x) for x in lists])
+    col = np.array([c for x in lists for c in x], dtype=np.int32)
+    return row_ptr, col
+
+
+def bsa_kv_csr(mask: np.ndarray):
+    """mask uint8 [B, N1, nqb, nkb] -> (row_ptr [B*N1*nqb+1], col) ascending per unit."""
+    B, N1, nqb, nkb = mask.shape
+    lists = []
+    for b in range(B):
+        for h in range(N1):
+            for qb in range(nqb):
+                lists.append([kb for kb in range(nkb) if mask[b, h, qb, kb] != 0])
+    return csr_from_lists(lists)
+
+
+def bsa_q_csr(mask: np.ndarray, N2: int):
+    """Transposed lists: rows (b, g, kb); entries h_local * nqb + qb ascending."""
+    B, N1, nqb, nkb = mask.shape
+    G = N1 // N2
+    lists = []
+    for b in range(B):
+        for g in range(N2):
+            for kb in range(nkb):
+                lst = []
+                for hl in range(G):
+                    for qb in range(nqb):
+                        if mask[b, g * G + hl, qb, kb] != 0:
+                            lst.append(hl * nqb + qb)
+                lists.append(lst)
+    return csr_from_lists(lists)
+
+
+def nsa_blocks_per_batch(cu_seqlens, sel_block):
+    lens = np.diff(np.asarray(cu_seqlens, dtype=np.int64))
+    return (lens + sel_block - 1) // sel_block
+
+
+def nsa_kv_lists(topk: np.ndarray, cu_seqlens, sel_block: int):
+    """topk int32 [T, N2, K] -> (ids [T, N2, K] valid ids ascending then -1 padding,
+    count [T, N2] int32, status bits)."""
+    T, N2, K = topk.shape
+    nblk = nsa_blocks_per_batch(cu_seqlens, sel_block)
+    batch_of = np.zeros(T, dtype=np.int64)
+    for b in range(len(nblk)):
+        batch_of[cu_seqlens[b]:cu_seqlens[b + 1]] = b
+    ids = np.full((T, N2, K), -1, dtype=np.int32)
+    cnt = np.zeros((T, N2), dtype=np.int32)
+    status = 0
+    for t in range(T):
+        nb = nblk[batch_of[t]]
+        for g in range(N2):
+            row = [int(x) for x in topk[t, g] if x >= 0]
+            if any(x >= nb for x in row):
+                status |= BAD_INDEX
+            row = sorted(x for x in row if x < nb)
+            ids[t, g, :len(row)] = row
+            cnt[t, g] = len(row)
+    return ids, cnt, status
+
+
+def nsa_token_csr(ids: np.ndarray, cnt: np.ndarray, cu_seqlens, sel_block: int):
+    """Rows (b, g, kb) with kb < nblk(b): ascending global token indices that selected kb."""
+    T, N2, _ = ids.shape
+    nblk = nsa_blocks_per_batch(cu_seqlens, sel_block)
+    lists = []
+    for b in range(len(nblk)):
+        t0, t1 = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
+        for g in range(N2):
+            per = [[] for _ in range(int(nblk[b]))]
+            for t in range(t0, t1):
+                for i in range(int(cnt[t, g])):
+                    per[int(ids[t, g, i])].append(t)
+            lists.extend(per)
+    return csr_from_lists(lists)
+
+
+def sfa_page_lists(sparse_indices: np.ndarray, block_table: np.ndarray, seqused_kv,
+                   sparse_block: int, page_size: int):
+    """sparse_indices [B, Sq, N2, K] (row 0 of Sq used) -> (pages [B, N2, K*ppb] physical pages
+    in list order with -1 for empty slots, status).  ppb = sparse_block / page_size."""
+    B, _, N2, K = sparse_indices.shape
+    ppb = sparse_block // page_size
+    pages = np.full((B, N2, K * ppb), -1, dtype=np.int32)
+    status = 0
+    for b in range(B):
+        nsb = (int(seqused_kv[b]) + sparse_block - 1) // sparse_block
+        for g in range(N2):
+            for i in range(K):
+                j = int(sparse_indices[b, 0, g, i])
+                if j < 0:
+                    continue
+                if j >= nsb:
+                    status |= BAD_INDEX
+                    continue
+                for p in range(ppb):
+                    lp = j * ppb + p
+                    if lp * page_size < int(seqused_kv[b]):
+                        pages[b, g, i * ppb + p] = block_table[b, lp]
+    return pages, status
+
+
+def work_cuts(weights: np.ndarray, n_parts: int) -> np.ndarray:
+    """Balanced split of a sequence of work items (SparseAttnSharedkvMetadata page: each core
+    gets the start and end of its share of the task list).
+
+    weights: int [U] per-unit cost.  Returns cuts int32 [n_parts + 1] in units of the
+    linearised item index: part s covers prefix positions [ceil(s*W/n), ceil((s+1)*W/n)) of the
+    total weight W, so cut[s] = ceil(s * W / n_parts)."""
+    W = int(np.sum(weights))
+    return np.array([-(-(s * W) // n_parts) for s in range(n_parts + 1)], dtype=np.int64)
