@@ -1,0 +1,184 @@
+/*
+ * selected_attention.h — C ABI of the B200 (sm_100a) block-sparse attention library.
+ *
+ * Operations (each cites the page that defines what it computes):
+ *   bsa_fwd / bsa_bwd           block-sparse attention, KV blocks chosen per Q block by a
+ *                               BlockSparseMask bitmap ("aclnnBlockSparseAttentionGrad" page,
+ *                               forward formula and backward formulas).
+ *   nsa_selected_fwd / _bwd     NSA selected attention: per-token topk_indices gather, TND
+ *                               varlen, GQA ("aclnnNsaSelectedAttention" page, forward formula;
+ *                               the backward applies the BlockSparseAttentionGrad formulas to the
+ *                               gathered blocks).
+ *   sfa_sparse_decode           sparse flash attention decode over a paged KV cache with a rope
+ *                               sub-head ("aclnnSparseFlashAttention" page, formula and
+ *                               constraints).
+ *   sparse_attn_metadata        selection -> per-unit KV lists, transposed lists and per-page
+ *                               lists, consumed by the ops above ("SparseAttnSharedkvMetadata"
+ *                               page, function description: a task list built ahead of the
+ *                               attention call).
+ *
+ * Conventions
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library allocates
+ *     nothing, never synchronises (except bsa_get_status), and launches only on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - Dtypes: Q, K, V, dOut, Out, dQ, dK, dV are bf16 (uint16 storage); LSE is fp32 natural-log
+ *     log-sum-exp of the scaled scores; masks are uint8; indices, tables, cu_seqlens are int32.
+ *   - Layouts (row-major, last dimension contiguous):
+ *       BNSD  q/dout/out/dq [B, N1, S_q, D], k/v/dk/dv [B, N2, S_kv, D], lse [B, N1, S_q]
+ *       TND   q/dout/out/dq [T, N1, D],      k/v/dk/dv [T, N2, D],       lse [T, N1]
+ *       PA_ND caches [num_pages, page_size, N2, D]; q [B, 1, N1, D]; out [B, 1, N1, Dv];
+ *             lse [B, 1, N1]
+ *   - GQA: query head h uses kv head h / (N1 / N2); N1 % N2 == 0 is required.
+ *   - Two-phase use, as on the pages: *_workspace_size() validates the problem on the host and
+ *     returns the scratch size; the op call re-validates, then launches.  Host validation
+ *     errors return before any launch.  Device-side problems (an index past the sequence, a
+ *     non-monotone cu_seqlens, a wait that exceeded its limit) set bits in a status word at the
+ *     start of the workspace; the offending block is skipped and the call still returns
+ *     BSA_OK.  bsa_get_status() reads the word.
+ *   - The workspace must be 256-byte aligned and is overwritten by every call.  Calls that
+ *     share one workspace must be ordered on the GPU (same stream or synchronised).
+ */
+#ifndef SELECTED_ATTENTION_H_
+#define SELECTED_ATTENTION_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "status_bits.h"
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_NULLPTR = 1,            /* a required pointer is NULL */
+  BSA_ERR_INVALID_ARG = 2,        /* a size, layout or rule from the pages is violated */
+  BSA_ERR_UNSUPPORTED = 3,        /* valid on the pages, not implemented by this library */
+  BSA_ERR_WORKSPACE_TOO_SMALL = 4,
+  BSA_ERR_CUDA = 5                /* a CUDA runtime call failed (launch, attribute, ...) */
+} bsa_status;
+
+typedef enum { BSA_LAYOUT_BNSD = 0, BSA_LAYOUT_TND = 1, BSA_LAYOUT_BSND = 2, BSA_LAYOUT_PA_ND = 3 } bsa_layout;
+
+/* Mask modes: 0 = no mask (all selected keys computed; NsaSelectedAttention sparseMode 0),
+ * 2 = causal, key position <= query position (sparseMode 2), 3 = right-down causal and
+ * 4 = band [q' - win_left, q' + win_right] with q' = q + S_kv - S_q (SparseAttnSharedkvMetadata
+ * cmp_mask_mode / ori_mask_mode). */
+typedef enum { BSA_MASK_NONE = 0, BSA_MASK_CAUSAL = 2, BSA_MASK_RIGHT_DOWN_CAUSAL = 3, BSA_MASK_BAND = 4 } bsa_mask_mode;
+
+typedef struct bsa_params {
+  int32_t q_layout, kv_layout; /* bsa_layout */
+  int32_t B, N1, N2;           /* batch, query heads, kv heads */
+  int32_t S_q, S_kv;           /* BNSD: sequence lengths.  TND: ignored (see T_q / cu_seqlens) */
+  int32_t T_q, T_kv;           /* TND: total tokens (host-side sizes) */
+  int32_t D, Dv, D_rope;       /* head dims of Q/K, V, and the rope part (SFA) */
+  const int32_t* cu_seqlens_q; /* TND: device int32 [B+1] prefix sums */
+  const int32_t* cu_seqlens_kv;
+  const int32_t* seqused_kv;   /* PA_ND: device int32 [B], tokens of each sequence in use */
+  /* BSA: BlockSparseMask, device uint8 [B, N1, ceil(S_q/block_x), ceil(S_kv/block_y)] */
+  int32_t block_x, block_y;
+  const uint8_t* block_mask;
+  /* NSA: topk_indices, device int32 [T, N2, sel_block_count]; ids count sel_block_size-token
+   * blocks from the batch's start; -1 = empty slot */
+  int32_t sel_block_size, sel_block_count;
+  const int32_t* topk_indices;
+  /* SFA: paged cache.  block_table device int32 [B, max_pages_per_seq]; sparse_indices device
+   * int32 [B, 1, N2, sparse_count] (logical sparse-block ids, -1 = empty) */
+  int32_t page_size, max_pages_per_seq, num_pages;
+  const int32_t* block_table;
+  int32_t sparse_block_size, sparse_count;
+  const int32_t* sparse_indices;
+  int32_t mask_mode, win_left, win_right; /* bsa_mask_mode */
+  float scale;                            /* multiplies q.k (SFA: the whole q.k + q_r.k_r) */
+} bsa_params;
+
+/* ---- workspace sizing (phase 1: host validation, no launch) ------------------------------ */
+BSA_API bsa_status bsa_fwd_workspace_size(const bsa_params* p, size_t* bytes);
+BSA_API bsa_status bsa_bwd_workspace_size(const bsa_params* p, size_t* bytes);
+BSA_API bsa_status nsa_selected_fwd_workspace_size(const bsa_params* p, size_t* bytes);
+BSA_API bsa_status nsa_selected_bwd_workspace_size(const bsa_params* p, size_t* bytes);
+BSA_API bsa_status sfa_sparse_decode_workspace_size(const bsa_params* p, size_t* bytes);
+
+/* ---- BSA (BlockSparseAttentionGrad page), BNSD, D = Dv = 128 -------------------------------
+ * Forward: Out = softmax(Mask(scale * Q K_sparse^T, atten_mask)) V_sparse, LSE per row.
+ * Rows with no visible key produce Out = 0 and LSE = -inf. */
+BSA_API bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
+                   void* workspace, size_t workspace_bytes, void* stream);
+/* Backward: softmax_grad = rowsum(dOut o Out); dP = dOut V^T; dS = P o (dP - softmax_grad);
+ * dV = P^T dOut; dQ = dS K scale; dK = dS^T Q scale.  `out` and `lse` are the forward's
+ * outputs.  dK/dV are accumulated in a fixed order (run-to-run bit identical, no atomics). */
+BSA_API bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void* v, const void* out,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* ---- NSA selected attention (NsaSelectedAttention page), TND, GQA, D = Dv = 128 ----------- */
+BSA_API bsa_status nsa_selected_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream);
+BSA_API bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ---- SFA sparse decode (SparseFlashAttention page), PA_ND caches, D = Dv = 512, D_rope = 64 -
+ * Out = softmax((q k~^T + q_rope k_rope~^T) * scale) v~ over the selected sparse blocks. */
+BSA_API bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_rope, const void* k_cache,
+                             const void* k_rope_cache, const void* v_cache, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- metadata (SparseAttnSharedkvMetadata page) -------------------------------------------
+ * Writes the integer plan the attention kernels consume into `plan` (device, plan_bytes from
+ * sparse_attn_metadata_size).  op selects the product:
+ *   BSA_META_BSA_KV     int32 row_ptr[U+1] then col[...]: per (b, h, qb) unit, ascending KV
+ *                       block ids of its BlockSparseMask row (U = B*N1*nqb).
+ *   BSA_META_BSA_Q      transposed lists: per (b, g, kb) row, ascending h_local*nqb + qb.
+ *   BSA_META_NSA_KV     int32 ids[T, N2, K] (valid ids ascending, then -1) and cnt[T, N2].
+ *   BSA_META_NSA_TOKENS per (b, g, kb) row, ascending global token indices that listed kb.
+ *   BSA_META_SFA_PAGES  int32 pages[B, N2, sparse_count * sparse_block_size / page_size].
+ * The plan layout for each op is given by sparse_attn_metadata_layout(). */
+typedef enum {
+  BSA_META_BSA_KV = 0,
+  BSA_META_BSA_Q = 1,
+  BSA_META_NSA_KV = 2,
+  BSA_META_NSA_TOKENS = 3,
+  BSA_META_SFA_PAGES = 4
+} bsa_meta_op;
+
+/* Offsets (bytes from `plan`) of the arrays an op writes: offsets[0] = status word,
+ * offsets[1..4] = op-specific arrays (see bsa_meta_op), count = number used. */
+typedef struct bsa_meta_layout {
+  size_t total_bytes;
+  size_t offsets[6];
+  int32_t count;
+} bsa_meta_layout;
+
+BSA_API bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta_layout* layout);
+BSA_API bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, size_t plan_bytes, void* stream);
+
+/* ---- status --------------------------------------------------------------------------------
+ * Copies the device status word at the start of `workspace` (or of a metadata plan) to
+ * *dev_bits after synchronising `stream`.  Bits: SA_DEV_BAD_INDEX, SA_DEV_BAD_SEQLEN,
+ * SA_DEV_TIMEOUT (status_bits.h). */
+BSA_API bsa_status bsa_get_status(const void* workspace, void* stream, uint32_t* dev_bits);
+
+/* Library version string. */
+BSA_API const char* bsa_version(void);
+
+/* ---- diagnostics ---------------------------------------------------------------------------
+ * One 128x128x128 tcgen05 tile: c[128][128] (fp32, device) = A B^T with A bf16 [128 rows][128 K]
+ * and B bf16 [128 N][128 K] (b_mn_major = 0) or [128 K][128 N] (b_mn_major = 1).  Runs the same
+ * TMA / shared-memory-descriptor / TMEM machinery as the attention kernels, so a tile-level
+ * fault can be told apart from an attention-level one.  workspace: >= 256 bytes (status word).
+ * Not part of the pages' operations. */
+BSA_API bsa_status bsa_diag_mma_tile(const void* a, const void* b, float* c, int32_t b_mn_major, void* workspace,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SELECTED_ATTENTION_H_ */

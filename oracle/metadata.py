@@ -37,31 +37,25 @@ def csr_from_lists(lists):
 
 
 def bsa_kv_csr(mask: np.ndarray):
-    """mask uint8 [B, N1, nqb, nkb] -> (row_ptr [B*N1*nqb+1], col) ascending per unit."""
+    """mask uint8 [B, N1, nqb, nkb] -> (row_ptr [B*N1*nqb+1], col) ascending per unit.
+
+    Units are the rows of the mask in (b, h, qb) order; a row's list is the positions of its
+    nonzero bytes, which np.nonzero returns in ascending row-major order."""
     B, N1, nqb, nkb = mask.shape
-    lists = []
-    for b in range(B):
-        for h in range(N1):
-            for qb in range(nqb):
-                lists.append([kb for kb in range(nkb) if mask[b, h, qb, kb] != 0])
-    return csr_from_lists(lists)
+    rows = mask.reshape(B * N1 * nqb, nkb) != 0
+    row_ptr = np.zeros(rows.shape[0] + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum(rows.sum(axis=1))
+    col = np.nonzero(rows)[1].astype(np.int32)
+    return row_ptr, col
 
 
 def bsa_q_csr(mask: np.ndarray, N2: int):
-    """Transposed lists: rows (b, g, kb); entries h_local * nqb + qb ascending."""
+    """Transposed lists: rows (b, g, kb); entries h_local * nqb + qb ascending, i.e. the nonzero
+    positions of the mask rearranged to [B, N2, nkb, G, nqb]."""
     B, N1, nqb, nkb = mask.shape
     G = N1 // N2
-    lists = []
-    for b in range(B):
-        for g in range(N2):
-            for kb in range(nkb):
-                lst = []
-                for hl in range(G):
-                    for qb in range(nqb):
-                        if mask[b, g * G + hl, qb, kb] != 0:
-                            lst.append(hl * nqb + qb)
-                lists.append(lst)
-    return csr_from_lists(lists)
+    t = mask.reshape(B, N2, G, nqb, nkb).transpose(0, 1, 4, 2, 3).reshape(B * N2 * nkb, G * nqb)
+    return bsa_kv_csr(t.reshape(B * N2 * nkb, 1, 1, G * nqb))
 
 
 def nsa_blocks_per_batch(cu_seqlens, sel_block):

@@ -1,0 +1,235 @@
+"""Python binding of the sm_100a block-sparse attention library (libselected_attention.so).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
+Torch supplies device memory (outputs, workspaces) and the current stream.  The functions carry
+the C ABI's names (include/selected_attention.h).  If the library is missing or fails to load,
+every call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libselected_attention.so")
+
+BSA_OK, BSA_ERR_NULLPTR, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_WORKSPACE_TOO_SMALL, BSA_ERR_CUDA = range(6)
+STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_NULLPTR", 2: "BSA_ERR_INVALID_ARG", 3: "BSA_ERR_UNSUPPORTED",
+                4: "BSA_ERR_WORKSPACE_TOO_SMALL", 5: "BSA_ERR_CUDA"}
+LAYOUT_BNSD, LAYOUT_TND, LAYOUT_BSND, LAYOUT_PA_ND = 0, 1, 2, 3
+MASK_NONE, MASK_CAUSAL, MASK_RIGHT_DOWN_CAUSAL, MASK_BAND = 0, 2, 3, 4
+META_BSA_KV, META_BSA_Q, META_NSA_KV, META_NSA_TOKENS, META_SFA_PAGES = range(5)
+DEV_BAD_INDEX, DEV_BAD_SEQLEN, DEV_TIMEOUT = 1, 2, 4
+
+EXPORTED = [
+    "bsa_fwd_workspace_size", "bsa_bwd_workspace_size", "nsa_selected_fwd_workspace_size",
+    "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size", "bsa_fwd", "bsa_bwd",
+    "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
+    "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
+]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    _fields_ = [
+        ("q_layout", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
+        ("B", ctypes.c_int32), ("N1", ctypes.c_int32), ("N2", ctypes.c_int32),
+        ("S_q", ctypes.c_int32), ("S_kv", ctypes.c_int32),
+        ("T_q", ctypes.c_int32), ("T_kv", ctypes.c_int32),
+        ("D", ctypes.c_int32), ("Dv", ctypes.c_int32), ("D_rope", ctypes.c_int32),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_kv", ctypes.c_void_p),
+        ("seqused_kv", ctypes.c_void_p),
+        ("block_x", ctypes.c_int32), ("block_y", ctypes.c_int32),
+        ("block_mask", ctypes.c_void_p),
+        ("sel_block_size", ctypes.c_int32), ("sel_block_count", ctypes.c_int32),
+        ("topk_indices", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("block_table", ctypes.c_void_p),
+        ("sparse_block_size", ctypes.c_int32), ("sparse_count", ctypes.c_int32),
+        ("sparse_indices", ctypes.c_void_p),
+        ("mask_mode", ctypes.c_int32), ("win_left", ctypes.c_int32), ("win_right", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+    ]
+
+
+class MetaLayout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("offsets", ctypes.c_size_t * 6), ("count", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it is missing: there is no CPU path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with python -m selected_attention_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(Params)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        for name in ("bsa_fwd_workspace_size", "bsa_bwd_workspace_size", "nsa_selected_fwd_workspace_size",
+                     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size"):
+            getattr(L, name).argtypes = [P, ctypes.POINTER(sz)]
+        L.bsa_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.nsa_selected_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.bsa_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.nsa_selected_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sfa_sparse_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sparse_attn_metadata_layout.argtypes = [P, ctypes.c_int32, ctypes.POINTER(MetaLayout)]
+        L.sparse_attn_metadata.argtypes = [P, ctypes.c_int32, vp, sz, vp]
+        L.bsa_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.bsa_diag_mma_tile.argtypes = [vp, vp, vp, ctypes.c_int32, vp, vp]
+        L.bsa_version.restype = ctypes.c_char_p
+        for name in EXPORTED:
+            if name != "bsa_version":
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn, code):
+    if code != BSA_OK:
+        raise BsaError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (the library has no CPU path)")
+
+
+def _workspace(nbytes, device):
+    return torch.empty(max(256, int(nbytes)), dtype=torch.uint8, device=device)
+
+
+def version() -> str:
+    return lib().bsa_version().decode()
+
+
+# ---------------------------------------------------------------------------------------------
+# BSA (BNSD)
+# ---------------------------------------------------------------------------------------------
+def bsa_params(q, k, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
+               win_right=0) -> Params:
+    B, N1, S_q, D = q.shape
+    _, N2, S_kv, _ = k.shape
+    p = Params()
+    p.q_layout = p.kv_layout = LAYOUT_BNSD
+    p.B, p.N1, p.N2, p.S_q, p.S_kv = B, N1, N2, S_q, S_kv
+    p.D = D
+    p.Dv = D
+    p.block_x, p.block_y = block_x, block_y
+    p.block_mask = block_mask.data_ptr()
+    p.mask_mode, p.win_left, p.win_right = mask_mode, win_left, win_right
+    p.scale = 1.0 / math.sqrt(D) if scale is None else scale
+    return p
+
+
+def bsa_fwd_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check("bsa_fwd_workspace_size", lib().bsa_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def bsa_fwd(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
+            win_right=0, out=None, lse=None, workspace=None, stream=None):
+    """Out, LSE = softmax(Mask(scale Q K_sel^T)) V_sel for BNSD bf16 tensors and a uint8
+    BlockSparseMask [B, N1, ceil(S_q/block_x), ceil(S_kv/block_y)]."""
+    _need_cuda(q, k, v, block_mask)
+    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right)
+    B, N1, S_q, _ = q.shape
+    if out is None:
+        out = torch.empty(B, N1, S_q, v.shape[-1], dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, N1, S_q, dtype=torch.float32, device=q.device)
+    need = bsa_fwd_workspace_size(p)
+    if workspace is None:
+        workspace = _workspace(need, q.device)
+    _check("bsa_fwd", lib().bsa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                    _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def bsa_bwd_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check("bsa_bwd_workspace_size", lib().bsa_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def bsa_bwd(q, k, v, out, dout, lse, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None,
+            win_left=0, win_right=0, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of block-sparse attention (BNSD)."""
+    _need_cuda(q, k, v, out, dout, lse, block_mask)
+    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bsa_bwd_workspace_size(p)
+    if workspace is None:
+        workspace = _workspace(need, q.device)
+    _check("bsa_bwd", lib().bsa_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)))
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------------------------
+# metadata
+# ---------------------------------------------------------------------------------------------
+def sparse_attn_metadata_layout(p: Params, op: int) -> MetaLayout:
+    L = MetaLayout()
+    _check("sparse_attn_metadata_layout", lib().sparse_attn_metadata_layout(ctypes.byref(p), op, ctypes.byref(L)))
+    return L
+
+
+def sparse_attn_metadata(p: Params, op: int, device, stream=None):
+    """Runs the metadata kernels for `op`; returns (plan tensor, layout)."""
+    L = sparse_attn_metadata_layout(p, op)
+    plan = _workspace(L.total_bytes, device)
+    _check("sparse_attn_metadata", lib().sparse_attn_metadata(ctypes.byref(p), op, _ptr(plan), plan.numel(),
+                                                              _stream(stream)))
+    return plan, L
+
+
+def plan_array(plan, layout: MetaLayout, index: int, count: int, dtype=torch.int32):
+    """View `count` elements of array `index` of a metadata plan."""
+    off = layout.offsets[index]
+    itemsize = torch.empty(0, dtype=dtype).element_size()
+    return plan[off:off + count * itemsize].view(dtype)
+
+
+def bsa_get_status(workspace, stream=None) -> int:
+    v = ctypes.c_uint32()
+    _check("bsa_get_status", lib().bsa_get_status(_ptr(workspace), _stream(stream), ctypes.byref(v)))
+    return v.value
+
+
+# ---------------------------------------------------------------------------------------------
+# diagnostics
+# ---------------------------------------------------------------------------------------------
+def bsa_diag_mma_tile(a, b, b_mn_major: bool, stream=None):
+    """c = a @ b.T (b K-major [N][K]) or a @ b (b MN-major [K][N]) on one tcgen05 tile."""
+    _need_cuda(a, b)
+    c = torch.empty(128, 128, dtype=torch.float32, device=a.device)
+    ws = _workspace(256, a.device)
+    _check("bsa_diag_mma_tile", lib().bsa_diag_mma_tile(_ptr(a), _ptr(b), _ptr(c), int(b_mn_major), _ptr(ws),
+                                                        _stream(stream)))
+    return c, ws

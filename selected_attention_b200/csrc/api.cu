@@ -1,0 +1,203 @@
+// C ABI entry points: host validation (the pages' constraints), workspace layout, launches.
+// Nothing here allocates memory or synchronises, except bsa_get_status.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "internal.h"
+
+using namespace sa;
+
+namespace {
+
+inline int div_up(int a, int b) { return (a + b - 1) / b; }
+
+// ---- BSA (BlockSparseAttentionGrad page constraints) -------------------------------------------
+// "N1 must be greater than or equal to N2, and N1 % N2 must be equal to 0"; "headdim=128";
+// layouts BNSD.  Block shape: block_x <= 128 (one 128-row MMA tile per Q block), block_y 64 or 128.
+bsa_status check_bsa(const bsa_params* p) {
+  if (!p) return BSA_ERR_NULLPTR;
+  if (p->q_layout != BSA_LAYOUT_BNSD || p->kv_layout != BSA_LAYOUT_BNSD) return BSA_ERR_UNSUPPORTED;
+  if (p->B <= 0 || p->N1 <= 0 || p->N2 <= 0 || p->S_q <= 0 || p->S_kv <= 0) return BSA_ERR_INVALID_ARG;
+  if (p->N1 < p->N2 || p->N1 % p->N2 != 0) return BSA_ERR_INVALID_ARG;
+  if (p->D != 128 || p->Dv != 128) return BSA_ERR_UNSUPPORTED;
+  if (p->block_x <= 0 || p->block_y <= 0) return BSA_ERR_INVALID_ARG;
+  if (p->block_x > 128 || (p->block_y != 64 && p->block_y != 128)) return BSA_ERR_UNSUPPORTED;
+  if (p->mask_mode != BSA_MASK_NONE && p->mask_mode != BSA_MASK_CAUSAL && p->mask_mode != BSA_MASK_RIGHT_DOWN_CAUSAL &&
+      p->mask_mode != BSA_MASK_BAND)
+    return BSA_ERR_INVALID_ARG;
+  if (p->mask_mode == BSA_MASK_BAND && (p->win_left < 0 || p->win_right < 0)) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return BSA_ERR_INVALID_ARG;
+  const long long rows_q = 1LL * p->B * p->N1 * p->S_q, rows_kv = 1LL * p->B * p->N2 * p->S_kv;
+  if (rows_q + 256 >= (1LL << 31) || rows_kv + 256 >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  const long long nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+  if (1LL * p->B * p->N1 * nqb * nkb >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  if (1LL * p->B * p->N1 > 65535) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+struct BsaFwdWs {
+  uint32_t* status;
+  int32_t *counts, *row_ptr, *col;
+};
+
+size_t carve_bsa_fwd(const bsa_params* p, void* ws, BsaFwdWs* w) {
+  Carver c(ws);
+  const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+  const size_t units = static_cast<size_t>(p->B) * p->N1 * nqb;
+  w->status = static_cast<uint32_t*>(ws);
+  w->counts = c.take<int32_t>(units);
+  w->row_ptr = c.take<int32_t>(units + 1);
+  w->col = c.take<int32_t>(units * nkb);
+  return c.bytes();
+}
+
+bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+bsa_status check_ws(void* ws, size_t have, size_t need) {
+  if (!ws) return BSA_ERR_NULLPTR;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return BSA_ERR_INVALID_ARG;
+  if (have < need) return BSA_ERR_WORKSPACE_TOO_SMALL;
+  return BSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bsa_version(void) { return "selected_attention_b200 0.1 (sm_100a)"; }
+
+bsa_status bsa_fwd_workspace_size(const bsa_params* p, size_t* bytes) {
+  if (!bytes) return BSA_ERR_NULLPTR;
+  bsa_status s = check_bsa(p);
+  if (s != BSA_OK) return s;
+  BsaFwdWs w;
+  *bytes = carve_bsa_fwd(p, nullptr, &w);
+  return BSA_OK;
+}
+
+bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  bsa_status s = check_bsa(p);
+  if (s != BSA_OK) return s;
+  if (!q || !k || !v || !out || !lse || !p->block_mask) return BSA_ERR_NULLPTR;
+  BsaFwdWs w;
+  const size_t need = carve_bsa_fwd(p, nullptr, &w);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != BSA_OK) return s;
+  carve_bsa_fwd(p, workspace, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+  const int units = p->B * p->N1 * nqb;
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = bsa_kv_lists(p->block_mask, units, nkb, w.counts, w.row_ptr, w.col, st);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  BsaFwdArgs a;
+  a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.S_q = p->S_q; a.S_kv = p->S_kv;
+  a.bx = p->block_x; a.by = p->block_y; a.nqb = nqb; a.nkb = nkb;
+  a.mask_mode = p->mask_mode; a.win_left = p->win_left; a.win_right = p->win_right; a.scale = p->scale;
+  a.row_ptr = w.row_ptr; a.col = w.col; a.out = out; a.lse = lse; a.status = w.status;
+  return cuda_status(bsa_fwd_launch(a, q, k, v, st));
+}
+
+bsa_status bsa_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
+  (void)p; (void)bytes;
+  return BSA_ERR_UNSUPPORTED;
+}
+bsa_status bsa_bwd(const bsa_params* p, const void*, const void*, const void*, const void*, const void*, const float*,
+                   void*, void*, void*, void*, size_t, void*) {
+  (void)p;
+  return BSA_ERR_UNSUPPORTED;
+}
+bsa_status nsa_selected_fwd_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
+bsa_status nsa_selected_bwd_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
+bsa_status nsa_selected_fwd(const bsa_params*, const void*, const void*, const void*, void*, float*, void*, size_t,
+                            void*) {
+  return BSA_ERR_UNSUPPORTED;
+}
+bsa_status nsa_selected_bwd(const bsa_params*, const void*, const void*, const void*, const void*, const void*,
+                            const float*, void*, void*, void*, void*, size_t, void*) {
+  return BSA_ERR_UNSUPPORTED;
+}
+bsa_status sfa_sparse_decode_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
+bsa_status sfa_sparse_decode(const bsa_params*, const void*, const void*, const void*, const void*, const void*,
+                             void*, float*, void*, size_t, void*) {
+  return BSA_ERR_UNSUPPORTED;
+}
+
+// ---- metadata -------------------------------------------------------------------------------------
+bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta_layout* layout) {
+  if (!layout) return BSA_ERR_NULLPTR;
+  std::memset(layout, 0, sizeof(*layout));
+  if (op == BSA_META_BSA_KV || op == BSA_META_BSA_Q) {
+    bsa_status s = check_bsa(p);
+    if (s != BSA_OK) return s;
+    const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+    Carver c(nullptr);
+    const size_t rows = op == BSA_META_BSA_KV ? static_cast<size_t>(p->B) * p->N1 * nqb
+                                              : static_cast<size_t>(p->B) * p->N2 * nkb;
+    const size_t ents = static_cast<size_t>(p->B) * p->N1 * nqb * nkb;
+    layout->offsets[0] = 0;
+    c.take<int32_t>(0);
+    layout->offsets[1] = c.off;  // row_ptr
+    c.take<int32_t>(rows + 1);
+    c.off = align_up(c.off, 256);
+    layout->offsets[2] = c.off;  // col
+    c.take<int32_t>(ents);
+    c.off = align_up(c.off, 256);
+    layout->offsets[3] = c.off;  // counts (scratch)
+    c.take<int32_t>(rows);
+    if (op == BSA_META_BSA_Q) {
+      c.off = align_up(c.off, 256);
+      layout->offsets[4] = c.off;  // transposed mask (scratch)
+      c.take<uint8_t>(ents);
+    }
+    layout->count = op == BSA_META_BSA_Q ? 5 : 4;
+    layout->total_bytes = c.bytes();
+    return BSA_OK;
+  }
+  return BSA_ERR_UNSUPPORTED;
+}
+
+bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, size_t plan_bytes, void* stream) {
+  bsa_meta_layout L;
+  bsa_status s = sparse_attn_metadata_layout(p, op, &L);
+  if (s != BSA_OK) return s;
+  if ((s = check_ws(plan, plan_bytes, L.total_bytes)) != BSA_OK) return s;
+  if (!p->block_mask) return BSA_ERR_NULLPTR;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(plan);
+  const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+  cudaError_t e = cudaMemsetAsync(plan, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  int32_t* row_ptr = reinterpret_cast<int32_t*>(base + L.offsets[1]);
+  int32_t* col = reinterpret_cast<int32_t*>(base + L.offsets[2]);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + L.offsets[3]);
+  if (op == BSA_META_BSA_KV)
+    e = bsa_kv_lists(p->block_mask, p->B * p->N1 * nqb, nkb, counts, row_ptr, col, st);
+  else
+    e = bsa_q_lists(p->block_mask, p->B, p->N1, p->N2, nqb, nkb, reinterpret_cast<uint8_t*>(base + L.offsets[4]),
+                    counts, row_ptr, col, st);
+  return cuda_status(e);
+}
+
+bsa_status bsa_get_status(const void* workspace, void* stream, uint32_t* dev_bits) {
+  if (!workspace || !dev_bits) return BSA_ERR_NULLPTR;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return BSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
+  *dev_bits = v;
+  return BSA_OK;
+}
+
+// ---- diagnostics ------------------------------------------------------------------------------------
+bsa_status bsa_diag_mma_tile(const void* a, const void* b, float* c, int32_t b_mn_major, void* workspace,
+                             void* stream) {
+  if (!a || !b || !c || !workspace) return BSA_ERR_NULLPTR;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+  return cuda_status(diag_mma_tile_launch(a, b, c, 128, b_mn_major, static_cast<uint32_t*>(workspace), st));
+}
+
+}  // extern "C"

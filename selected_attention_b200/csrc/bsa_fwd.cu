@@ -1,0 +1,318 @@
+// Block-sparse attention forward on tcgen05 (BlockSparseAttentionGrad page, forward formula):
+//   Out = softmax(Mask(scale * Q K_sparse^T, atten_mask)) V_sparse,   LSE = m + ln(l)
+// One CTA per unit (b, h, q block): 128 query rows against the KV blocks the unit's
+// BlockSparseMask row selects (CSR lists from metadata.cu).
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S, masks, keeps the running
+//              max/sum, writes P (bf16) into shared memory, rescales O in TMEM, epilogue.
+//   warp 4     TMA producer: Q once, then K/V tiles of the selected blocks into a 2-stage ring.
+//   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
+//              O += P_j V_j into the TMEM O accumulator.  S_{j+1} is issued before waiting for
+//              P_j, so the tensor core computes the next scores while softmax runs.
+// Every wait is bounded (sa_common.cuh); on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "sa_common.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kBM = 128;  // query rows per CTA tile (the MMA M)
+constexpr int kD = 128;   // head dim of Q/K and V
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int BN>
+struct __align__(1024) FwdSmem {
+  uint8_t q[2][kBM * 128];        // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
+  uint8_t k[2][2][BN * 128];      // [stage][sub-tile] K rows of one KV block
+  uint8_t v[2][2][BN * 128];      // [stage][sub-tile] V rows
+  uint8_t p[BN / 64][kBM * 128];  // P (bf16) sub-tiles of 64 keys, K-major 128B swizzle
+  uint64_t bar_q;
+  uint64_t bar_k[2], bar_v[2], bar_kv_empty[2], bar_s_full[2];
+  uint64_t bar_p_full, bar_o_done;
+  uint32_t tmem_base;
+};
+
+struct FwdParams {
+  int B, N1, N2, S_q, S_kv, bx, by, nqb, mask_mode, win_left, win_right;
+  float scale_log2;
+  const int32_t* row_ptr;
+  const int32_t* col;
+  __nv_bfloat16* out;
+  float* lse;
+  uint32_t* status;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
+  constexpr uint32_t kTmemCols = (2 * BN + kD) <= 256 ? 256 : 512;
+  constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<BN>& s = *reinterpret_cast<FwdSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // head-major, longest (latest) Q blocks first
+  const int bh = blockIdx.x / prm.nqb;
+  const int qb = prm.nqb - 1 - static_cast<int>(blockIdx.x % prm.nqb);
+  const int b = bh / prm.N1, h = bh % prm.N1;
+  const int g = h / (prm.N1 / prm.N2);
+  const int unit = bh * prm.nqb + qb;
+  const int rp = prm.row_ptr[unit];
+  const int n = prm.row_ptr[unit + 1] - rp;
+  const int q_row0 = bh * prm.S_q + qb * prm.bx;
+  const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
+
+  if (tid == 0) {
+    mbar_init(&s.bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.bar_k[i], 1);
+      mbar_init(&s.bar_v[i], 1);
+      mbar_init(&s.bar_kv_empty[i], 1);
+      mbar_init(&s.bar_s_full[i], 1);
+    }
+    mbar_init(&s.bar_p_full, kBM);
+    mbar_init(&s.bar_o_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&s.bar_q, 2 * kBM * 128);
+      tma_load_2d(s.q[0], &tm_q, &s.bar_q, 0, q_row0);
+      tma_load_2d(s.q[1], &tm_q, &s.bar_q, 64, q_row0);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(&s.bar_kv_empty[st], ((j - 2) >> 1) & 1, prm.status)) break;
+        const int row = kv_row0 + prm.col[rp + j] * prm.by;
+        mbar_arrive_expect_tx(&s.bar_k[st], 2 * BN * 128);
+        tma_load_2d(s.k[st][0], &tm_k, &s.bar_k[st], 0, row);
+        tma_load_2d(s.k[st][1], &tm_k, &s.bar_k[st], 64, row);
+        mbar_arrive_expect_tx(&s.bar_v[st], 2 * BN * 128);
+        tma_load_2d(s.v[st][0], &tm_v, &s.bar_v[st], 0, row);
+        tma_load_2d(s.v[st][1], &tm_v, &s.bar_v[st], 64, row);
+        issued = j + 1;
+      }
+      // do not leave the CTA with copies in flight
+      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
+        mbar_wait(&s.bar_k[j & 1], (j >> 1) & 1, prm.status);
+        mbar_wait(&s.bar_v[j & 1], (j >> 1) & 1, prm.status);
+      }
+      mbar_wait(&s.bar_q, 0, prm.status);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
+      const uint32_t idesc_o = idesc_bf16_f32(kBM, kD, false, true);
+      auto issue_s = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&s.bar_k[st], (j >> 1) & 1, prm.status)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + (st ? kColS1 : kColS0);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint64_t ad = sdesc_sw128(smem_u32(s.q[ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(s.k[st][ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          mma_bf16_ss(d, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(&s.bar_s_full[st]);
+        return true;
+      };
+      bool ok = mbar_wait(&s.bar_q, 0, prm.status);
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
+        if (!(ok = mbar_wait(&s.bar_p_full, j & 1, prm.status))) break;
+        const int st = j & 1;
+        if (!(ok = mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint64_t ad = sdesc_sw128(smem_u32(s.p[ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(s.v[st][0]) + ks * 2048, BN * 128, 1024);
+          mma_bf16_ss(tmem + kColO, ad, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc_commit(&s.bar_o_done);
+        tc_commit(&s.bar_kv_empty[st]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroup
+    const int r = tid;  // query row within the tile == TMEM lane
+    const int qpos = qb * prm.bx + r;
+    const bool row_valid = r < prm.bx && qpos < prm.S_q;
+    // visible key interval [lo, hi] for this row (mask modes 0/2/3/4)
+    int lo = 0, hi = prm.S_kv - 1;
+    const int qq = qpos + prm.S_kv - prm.S_q;
+    if (prm.mask_mode == 2) hi = min(hi, qpos);
+    else if (prm.mask_mode == 3) hi = min(hi, qq);
+    else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
+    if (!row_valid) { lo = 1; hi = 0; }
+
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int st = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (j >> 1) & 1, prm.status));
+      if (!ok) break;
+      tc_fence_after();
+      const int kpos0 = prm.col[rp + j] * prm.by;
+      float x[BN];
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + (st ? kColS1 : kColS0) + c, rr);
+        tmem_ld_wait(rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(rr[i]) * prm.scale_log2;
+      }
+      const bool full = kpos0 >= lo && kpos0 + BN - 1 <= hi;
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int kp = kpos0 + c;
+          if (kp < lo || kp > hi) x[c] = -INFINITY;
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m, mx);
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (j - 1) & 1, prm.status));
+        if (!ok) break;
+        tc_fence_after();
+        // tcgen05.ld/st are warp-collective: rescale when any row of the warp needs it
+        const bool need = m_new > m && m != -INFINITY;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2(m - m_new) : 1.f;
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < kD; c += 32) {
+            uint32_t rr[32];
+            tmem_ld32(tmem + lane_base + kColO + c, rr);
+            tmem_ld_wait(rr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+            tmem_st32(tmem + lane_base + kColO + c, rr);
+          }
+          tmem_st_wait();
+        }
+      }
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      float rowsum = 0.f;
+#pragma unroll
+      for (int t = 0; t < BN / 64; ++t) {
+        uint8_t* prow = s.p[t];
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float e[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            e[i] = ex2(x[t * 64 + c8 * 8 + i] - m_use);
+            rowsum += e[i];
+          }
+          uint4 pk;
+          pk.x = pack_bf16(e[0], e[1]);
+          pk.y = pack_bf16(e[2], e[3]);
+          pk.z = pack_bf16(e[4], e[5]);
+          pk.w = pack_bf16(e[6], e[7]);
+          *reinterpret_cast<uint4*>(prow + sw128_offset(r, c8 * 8)) = pk;
+        }
+      }
+      l += rowsum;
+      m = m_new;
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&s.bar_p_full);
+    }
+    // ---- epilogue
+    bool have_o = ok && n > 0;
+    if (have_o) {
+      have_o = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (n - 1) & 1, prm.status));
+      tc_fence_after();
+    }
+    const bool any = have_o && l > 0.f;
+    const float inv_l = any ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = prm.out + static_cast<size_t>(q_row0 + r) * kD;
+#pragma unroll
+    for (int c = 0; c < kD; c += 32) {
+      uint32_t rr[32];
+      if (have_o) {  // warp-uniform: every lane joins the collective load
+        tmem_ld32(tmem + lane_base + kColO + c, rr);
+        tmem_ld_wait(rr);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rr[i] = 0u;
+      }
+      if (row_valid) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 pk;
+          pk.x = pack_bf16(__uint_as_float(rr[i + 0]) * inv_l, __uint_as_float(rr[i + 1]) * inv_l);
+          pk.y = pack_bf16(__uint_as_float(rr[i + 2]) * inv_l, __uint_as_float(rr[i + 3]) * inv_l);
+          pk.z = pack_bf16(__uint_as_float(rr[i + 4]) * inv_l, __uint_as_float(rr[i + 5]) * inv_l);
+          pk.w = pack_bf16(__uint_as_float(rr[i + 6]) * inv_l, __uint_as_float(rr[i + 7]) * inv_l);
+          *reinterpret_cast<uint4*>(orow + c + i) = pk;
+        }
+      }
+    }
+    if (row_valid) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int BN>
+cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t q_rows = static_cast<uint64_t>(a.B) * a.N1 * a.S_q;
+  const uint64_t kv_rows = static_cast<uint64_t>(a.B) * a.N2 * a.S_kv;
+  if (!make_tmap_2d_bf16(&tq, q, q_rows, kD, kD, kBM)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tk, k, kv_rows, kD, kD, BN)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tv, v, kv_rows, kD, kD, BN)) return cudaErrorInvalidValue;
+  FwdParams p;
+  p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.S_q = a.S_q; p.S_kv = a.S_kv; p.bx = a.bx; p.by = a.by;
+  p.nqb = a.nqb; p.mask_mode = a.mask_mode; p.win_left = a.win_left; p.win_right = a.win_right;
+  p.scale_log2 = a.scale * kLog2e;
+  p.row_ptr = a.row_ptr; p.col = a.col;
+  p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse; p.status = a.status;
+  const size_t smem = sizeof(FwdSmem<BN>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = a.B * a.N1 * a.nqb;
+  if (grid == 0) return cudaSuccess;
+  bsa_fwd_kernel<BN><<<grid, 192, smem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t bsa_fwd_launch(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st) {
+  if (a.by == 128) return launch_fwd<128>(a, q, k, v, st);
+  if (a.by == 64) return launch_fwd<64>(a, q, k, v, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sa

@@ -1,0 +1,100 @@
+// Diagnostic: one 128 x 128 x 128 tcgen05 tile, C = A B^T with A K-major and B either K-major
+// ([N][K]) or MN-major ([K][N]).  Exercises exactly the building blocks the attention kernels use
+// (TMA 128B-swizzled loads, smem descriptors of both majors, TMEM accumulate, tcgen05.ld), so a
+// parity failure in attention can be narrowed to the tile machinery or the attention logic.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "sa_common.cuh"
+
+namespace sa {
+namespace {
+
+struct __align__(1024) DiagSmem {
+  uint8_t a[2][128 * 128];  // two 64-column sub-tiles of A: [128 rows][64] each
+  uint8_t b[2][128 * 128];  // two sub-tiles of B
+  uint64_t bar_load;
+  uint64_t bar_mma;
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                       const __grid_constant__ CUtensorMap tm_b, float* c,
+                                                       int b_mn_major, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  DiagSmem& s = *reinterpret_cast<DiagSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  if (tid == 0) {
+    mbar_init(&s.bar_load, 1);
+    mbar_init(&s.bar_mma, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  bool ok = true;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&s.bar_load, 4 * 128 * 128);
+    tma_load_2d(s.a[0], &tm_a, &s.bar_load, 0, 0);
+    tma_load_2d(s.a[1], &tm_a, &s.bar_load, 64, 0);
+    tma_load_2d(s.b[0], &tm_b, &s.bar_load, 0, 0);
+    tma_load_2d(s.b[1], &tm_b, &s.bar_load, 64, 0);
+    ok = mbar_wait(&s.bar_load, 0, status);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, 128, false, b_mn_major != 0);
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = sdesc_sw128(smem_u32(s.a[ks / 4]) + (ks % 4) * 32, 0, 1024);
+        uint64_t bd;
+        if (b_mn_major)  // B tile is [K rows][N cols]: sub-tile = N chunk, K step = 16 rows
+          bd = sdesc_sw128(smem_u32(s.b[0]) + ks * 2048, 128 * 128, 1024);
+        else
+          bd = sdesc_sw128(smem_u32(s.b[ks / 4]) + (ks % 4) * 32, 0, 1024);
+        mma_bf16_ss(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+      }
+      tc_commit(&s.bar_mma);
+    }
+  }
+  __syncwarp();
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncthreads();
+  if (!aborted(status)) ok = mbar_wait(&s.bar_mma, 0, status);
+  else ok = false;
+  tc_fence_after();
+  if (ok) {
+    const int row = warp * 32 + lane;
+    for (int cc = 0; cc < 128; cc += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem_addr(tmem, warp * 32, cc), r);
+      tmem_ld_wait(r);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) c[row * 128 + cc + i] = __uint_as_float(r[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+}  // namespace
+
+cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,
+                                 cudaStream_t st) {
+  if (n != 128) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d_bf16(&ta, a, 128, 128, 128, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tb, b, 128, 128, 128, 128)) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(DiagSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(diag_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  diag_mma_kernel<<<1, 128, smem, st>>>(ta, tb, c, b_mn_major, status);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

@@ -1,0 +1,66 @@
+// Internal (non-ABI) declarations shared by the .cu files of the library.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "selected_attention.h"
+
+namespace sa {
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Carves a caller workspace into aligned arrays, in a fixed order, so the size query and the
+// op call agree.  With base == nullptr it only measures.
+struct Carver {
+  char* base;
+  size_t off = 256;  // bytes [0, 256) hold the status word
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t n) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+  size_t bytes() const { return align_up(off, 256); }
+};
+
+// ---- metadata (metadata.cu) -------------------------------------------------------------------
+// BSA KV lists: units (b, h, qb) -> ascending kv block ids.
+cudaError_t bsa_kv_lists(const uint8_t* mask, int units, int nkb, int32_t* counts, int32_t* row_ptr, int32_t* col,
+                         cudaStream_t st);
+// BSA transposed lists: rows (b, g, kb) -> ascending h_local*nqb + qb.  maskT is scratch of
+// B*N1*nqb*nkb bytes.
+cudaError_t bsa_q_lists(const uint8_t* mask, int B, int N1, int N2, int nqb, int nkb, uint8_t* maskT,
+                        int32_t* counts, int32_t* row_ptr, int32_t* col, cudaStream_t st);
+// Exclusive scan of n counts into row_ptr[n+1].
+cudaError_t exclusive_scan(const int32_t* counts, int n, int32_t* row_ptr, cudaStream_t st);
+
+// ---- tensor maps (tma.cpp) ---------------------------------------------------------------------
+// 2D bf16 map over rows x cols (cols contiguous), row stride in elements, box {64, box_rows},
+// 128-byte swizzle.
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride,
+                       uint32_t box_rows);
+// 3D bf16 map over [d2][d1][d0] (d0 contiguous) with strides in elements, box {64, box1, box2}.
+bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2);
+
+// ---- BSA forward (bsa_fwd.cu) --------------------------------------------------------------------
+struct BsaFwdArgs {
+  int B, N1, N2, S_q, S_kv, bx, by, nqb, nkb, mask_mode, win_left, win_right;
+  float scale;
+  const int32_t* row_ptr;
+  const int32_t* col;
+  void* out;
+  float* lse;
+  uint32_t* status;
+};
+cudaError_t bsa_fwd_launch(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st);
+
+// ---- diagnostics (diag.cu) -----------------------------------------------------------------------
+cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,
+                                 cudaStream_t st);
+
+}  // namespace sa

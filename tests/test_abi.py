@@ -1,0 +1,79 @@
+"""The C-ABI library loads, exports every symbol include/*.h declares, and its host-side
+validation rejects problems the pages rule out, all without a GPU (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selected_attention_b200 as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            txt = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"^BSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", txt, flags=re.M))
+    return names
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from selected_attention_b200 import build
+    build.build()
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 15
+    L = sa.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(sa.EXPORTED) <= names
+    assert "sm_100a" in sa.version()
+
+
+def _bsa(**kw):
+    p = sa.Params()
+    p.q_layout = p.kv_layout = sa.LAYOUT_BNSD
+    p.B, p.N1, p.N2, p.S_q, p.S_kv, p.D, p.Dv = 2, 4, 2, 1000, 1000, 128, 128
+    p.block_x, p.block_y, p.mask_mode, p.scale = 128, 128, 2, 0.088
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def _ws(fn, p):
+    n = ctypes.c_size_t()
+    return getattr(sa.lib(), fn)(ctypes.byref(p), ctypes.byref(n)), n.value
+
+
+def test_bsa_host_validation():
+    code, n = _ws("bsa_fwd_workspace_size", _bsa())
+    assert code == sa.BSA_OK and n > 0 and n % 256 == 0
+    assert _ws("bsa_fwd_workspace_size", _bsa(N2=3))[0] == sa.BSA_ERR_INVALID_ARG      # N1 % N2
+    assert _ws("bsa_fwd_workspace_size", _bsa(N1=1, N2=2))[0] == sa.BSA_ERR_INVALID_ARG  # N1 < N2
+    assert _ws("bsa_fwd_workspace_size", _bsa(D=64, Dv=64))[0] == sa.BSA_ERR_UNSUPPORTED  # headdim=128
+    assert _ws("bsa_fwd_workspace_size", _bsa(q_layout=sa.LAYOUT_TND))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws("bsa_fwd_workspace_size", _bsa(block_y=96))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws("bsa_fwd_workspace_size", _bsa(mask_mode=1))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws("bsa_fwd_workspace_size", _bsa(S_q=0))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws("bsa_fwd_workspace_size", _bsa(scale=float("nan")))[0] == sa.BSA_ERR_INVALID_ARG
+    L = sa.lib()
+    assert L.bsa_fwd_workspace_size(None, None) == sa.BSA_ERR_NULLPTR
+    # op call with NULL tensors fails validation before any launch
+    p = _bsa()
+    assert L.bsa_fwd(ctypes.byref(p), None, None, None, None, None, None, 0, None) == sa.BSA_ERR_NULLPTR
+
+
+def test_workspace_size_matches_layout():
+    p = _bsa(B=1, N1=2, N2=2, S_q=512, S_kv=512, block_x=64, block_y=64)
+    code, n = _ws("bsa_fwd_workspace_size", p)
+    units, nkb = 1 * 2 * 8, 8
+    assert code == sa.BSA_OK and n >= 4 * (units + units + 1 + units * nkb)
+    lay = sa.sparse_attn_metadata_layout(p, sa.META_BSA_KV)
+    assert lay.count == 4 and lay.total_bytes >= lay.offsets[3] + 4 * units
