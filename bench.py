@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Throughput of block-sparse attention forward + backward on B200 (sm_100a).
+
+One step = one pass of the whole hot path over one batch: metadata (KV lists, transposed
+lists) + forward (Out, LSE) + backward (dQ, dK, dV), all in the library's CUDA kernels.  The
+default workload is block-sparse attention at B=2, N=16, S=8192, D=128 with 128x128 blocks
+and a causal Bernoulli(0.25) BlockSparseMask (synthetic, seeded).
+
+The metric is effective TFLOP/s: credited FLOPs / time, with forward 4*D*V and backward
+10*D*V for V visible (query, key) pairs (the diagonal block counts only its visible half).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1|2|5]
+
+With N > 1 (launched by torchrun, one process per GPU) every rank runs its own copy of the
+workload (independent batches: weak scaling, no collective on the data path); time is the max
+over ranks.  --impl reference times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import synth  # noqa: E402
+
+METRIC = "effective block-sparse attn fwd+bwd TFLOP/s (bf16)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
+# kernel's source file is unchanged (sha1 prefix of the file recorded at capture time).
+NCU_TRAFFIC = {}
+
+
+def visible_pairs_bsa(mask: np.ndarray, bx: int, by: int, s_q: int, s_kv: int) -> int:
+    """Exact number of (query, key) pairs that are selected and causal-visible."""
+    nqb, nkb = mask.shape[-2:]
+    per_block = np.zeros((nqb, nkb), dtype=np.int64)
+    for qb in range(nqb):
+        rows = np.arange(qb * bx, min(s_q, (qb + 1) * bx))
+        for kb in range(nkb):
+            k0, k1 = kb * by, min(s_kv, (kb + 1) * by)
+            if k0 > rows[-1]:
+                continue
+            per_block[qb, kb] = np.clip(np.minimum(rows, k1 - 1) - k0 + 1, 0, None).sum()
+    sel = (mask != 0).reshape(-1, nqb, nkb).sum(axis=0)
+    return int((sel * per_block).sum())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bsa_workload(config: int):
+    w = synth.workload(config)
+    assert isinstance(w, synth.BsaWorkload), "bench supports the BSA workloads (1, 2, 5)"
+    return w
+
+
+def cpu_oracle_sample(w, mask, budget_s: float):
+    """Time the fp64 oracle (forward + backward) on whole (b, h) head slices until budget_s has
+    passed; returns (credited FLOPs done, seconds, description)."""
+    from oracle import attention as A
+    flops, heads, t0 = 0, [], time.perf_counter()
+    for b in range(w.B):
+        for h in range(w.N1):
+            q = A.bf16_to_f64(w.tensor("q", b, h))[None]
+            k = A.bf16_to_f64(w.tensor("k", b, h))
+            v = A.bf16_to_f64(w.tensor("v", b, h))
+            do = A.bf16_to_f64(w.tensor("dout", b, h))[None]
+            A.bsa_slice_backward(q, k, v, do, mask[b, h][None], w.block, w.block, w.mask_mode, w.scale,
+                                 out_storage="bf16")
+            vp = visible_pairs_bsa(mask[b, h][None, None], w.block, w.block, w.S, w.S)
+            flops += 14 * w.D * vp
+            heads.append((b, h))
+            if time.perf_counter() - t0 >= budget_s:
+                dt = time.perf_counter() - t0
+                return flops, dt, f"oracle fwd+bwd on {len(heads)} of {w.B * w.N1} (b,h) head slices {heads}"
+    dt = time.perf_counter() - t0
+    return flops, dt, f"oracle fwd+bwd on all {len(heads)} (b,h) head slices"
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((x.get("num_threads", 1) for x in info), default=1)
+        return int(n)
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    w = bsa_workload(args.config)
+    mask = w.block_mask()
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are a no-op
+    total_f, total_t, desc = 0, 0.0, ""
+    for _ in range(args.steps):
+        f, t, desc = cpu_oracle_sample(w, mask, budget_s=args.ref_step_seconds)
+        total_f += f
+        total_t += t
+    value = total_f / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def config_dict(w, args):
+    return {
+        "workload": f"{w.name}: block-sparse attention fwd+bwd, BNSD B={w.B} N={w.N1} S={w.S} D={w.D}, "
+                    f"{w.block}x{w.block} blocks, selection={w.selection} {w.sel_args}, causal",
+        "B": w.B, "N": w.N1, "S": w.S, "D": w.D, "block": w.block, "seed": w.seed,
+        "l2": "no flush: inputs (Q,K,V,dOut) exceed the 126 MB L2" if 4 * w.B * w.N1 * w.S * w.D * 2 > 126e6
+        else "inputs fit in L2 (small parity workload)",
+        "parallelism": f"replicas x{args.gpus} (independent batches)",
+    }
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import selected_attention_b200 as sa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = bsa_workload(args.config)
+    mask = w.block_mask()
+    vpairs = visible_pairs_bsa(mask, w.block, w.block, w.S, w.S)
+    flops_step = 14 * w.D * vpairs
+
+    host = {t: torch.from_numpy(w.tensor(t)).view(torch.bfloat16) for t in ("q", "k", "v", "dout")}
+    q, k, v, do = (host[t].to(dev) for t in ("q", "k", "v", "dout"))
+    dmask = torch.from_numpy(mask).to(dev)
+    bx = by = w.block
+    out = torch.empty_like(q)
+    lse = torch.empty(w.B, w.N1, w.S, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    p = sa.bsa_params(q, k, dmask, bx, by, w.mask_mode, w.scale)
+    ws_f = torch.empty(sa.bsa_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(sa.bsa_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(qq=q, kk=k, vv=v, dd=do, mm=dmask):
+        sa.bsa_fwd(qq, kk, vv, mm, bx, by, w.mask_mode, w.scale, out=out, lse=lse, workspace=ws_f)
+        sa.bsa_bwd(qq, kk, vv, out, dd, lse, mm, bx, by, w.mask_mode, w.scale, dq=dq, dk=dk, dv=dv,
+                   workspace=ws_b)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x):
+        if world > 1:
+            t = torch.tensor([x], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            return float(t.item())
+        return x
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert sa.bsa_get_status(ws_f) == 0 and sa.bsa_get_status(ws_b) == 0, "device status bits set"
+
+    # ---- device-timed region: inputs resident in HBM
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        sa.bsa_profile_enable(True)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        prof = sa.bsa_profile_collect()
+        sa.bsa_profile_enable(False)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
+    value = world * flops_step / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    pin = {t: host[t].pin_memory() for t in host}
+    pin_mask = torch.from_numpy(mask).pin_memory()
+    h_out = {n: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n, x in
+             (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    d_in = {t: torch.empty_like(x) for t, x in (("q", q), ("k", k), ("v", v), ("dout", do))}
+    d_mask = torch.empty_like(dmask)
+    h2d = sum(x.numel() * x.element_size() for x in pin.values()) + pin_mask.numel()
+    d2h = sum(x.numel() * x.element_size() for x in h_out.values())
+
+    def e2e_step():
+        for t in d_in:
+            d_in[t].copy_(pin[t], non_blocking=True)
+        d_mask.copy_(pin_mask, non_blocking=True)
+        step(d_in["q"], d_in["k"], d_in["v"], d_in["dout"], d_mask)
+        for n, x in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            h_out[n].copy_(x, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = measured_peaks()
+    alg = {"bsa_fwd": 4 * w.D * vpairs, "bsa_bwd_kv": 8 * w.D * vpairs, "bsa_bwd_q": 6 * w.D * vpairs}
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roof = None
+    if dom in alg:
+        launches, total = prof[dom]
+        avg_ms = total / launches
+        achieved = alg[dom] / (avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        traffic = None
+        tr = NCU_TRAFFIC.get(dom)
+        if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config:
+            traffic = tr["bytes"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic,
+                "avg_launch_ms": avg_ms}
+    kernels = {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in prof.items()}
+    launches_total = sum(c for c, _ in prof.values())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, t, desc = cpu_oracle_sample(w, mask, budget_s=args.cpu_seconds)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, args),
+            "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_total, "kernels": kernels, "roofline": roof, "cpu_baseline": cpu,
+            "clocks": clocks.summary(), "visible_pairs": vpairs, "credited_flops_per_step": flops_step,
+        }
+        print(json.dumps(line))
+
+
+def source_sha1(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 5])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=5.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -166,12 +166,27 @@ BSA_API bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* p
  * SA_DEV_TIMEOUT (status_bits.h). */
 BSA_API bsa_status bsa_get_status(const void* workspace, void* stream, uint32_t* dev_bits);
 
+/* ---- kernel timing (for benchmarks; off by default) ---------------------------------------
+ * bsa_profile_enable(1) starts recording a pair of CUDA events around every kernel launch the
+ * library makes (events come from a pool the library creates on first use; 0 stops and clears).
+ * bsa_profile_collect() synchronises on the recorded events and returns, per kernel name, the
+ * number of launches and their summed device time in milliseconds; it then clears the records.
+ * *n_entries receives the number of names (entries beyond max_entries are not written). */
+typedef struct bsa_kernel_time {
+  char name[32];
+  int32_t launches;
+  double total_ms;
+} bsa_kernel_time;
+BSA_API bsa_status bsa_profile_enable(int32_t on);
+BSA_API bsa_status bsa_profile_collect(bsa_kernel_time* out, int32_t max_entries, int32_t* n_entries);
+
 /* Library version string. */
 BSA_API const char* bsa_version(void);
 
 /* ---- diagnostics ---------------------------------------------------------------------------
  * One 128x128x128 tcgen05 tile: c[128][128] (fp32, device) = A B^T with A bf16 [128 rows][128 K]
- * and B bf16 [128 N][128 K] (b_mn_major = 0) or [128 K][128 N] (b_mn_major = 1).  Runs the same
+ * and B bf16 [128 N][128 K] (b_mn_major = 0 or 2) or [128 K][128 N] (b_mn_major = 1 or 3); modes 2
+ * and 3 stage A in tensor memory instead of shared memory.  Runs the same
  * TMA / shared-memory-descriptor / TMEM machinery as the attention kernels, so a tile-level
  * fault can be told apart from an attention-level one.  workspace: >= 256 bytes (status word).
  * Not part of the pages' operations. */

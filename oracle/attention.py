@@ -25,6 +25,10 @@ Readings of points the pages leave open (each also listed in the design notes):
   * topk ids count sel_block_size-token blocks from the batch's own start; -1 marks an empty slot;
     a duplicated id is gathered twice (literal Gather).
   * Masked scores are -inf; a row with no visible key gives Out = 0, LSE = -inf, zero gradients.
+  * softmax_grad = softmaxGrad(dOut, attentionOut) uses attentionOut as the backward operator
+    receives it: the forward output stored in the input dtype.  With bf16 inputs (uint16 bit
+    patterns) the oracle rounds its own fp64 Out to bf16 before the rowsum; with float inputs it
+    uses Out unrounded.
   * Mask modes: 0 = none, 2 = causal (key pos <= query pos), 3 = right-down causal
     (key pos <= query pos + Skv - Sq), 4 = band [q' - win_left, q' + win_right] with
     q' = query pos + Skv - Sq.  Keys at or past the sequence's kv length are never visible.
@@ -44,6 +48,18 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """Widen bf16 bit patterns (uint16) to float64 exactly."""
     b = np.ascontiguousarray(bits, dtype=np.uint16)
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """float64 -> nearest bf16 value (via float32, ties to even), returned as float64."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    u = ((u + (((u >> 16) & np.uint32(1)) + np.uint32(0x7FFF))) >> 16) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def stored_out(o: np.ndarray, out_storage) -> np.ndarray:
+    """attentionOut as the backward operator receives it (see module notes)."""
+    return round_to_bf16(o) if out_storage == "bf16" else o
 
 
 # ----------------------------------------------------------------------------------------------
@@ -142,7 +158,7 @@ def bsa_slice_forward(q_g, k_g, v_g, mask_g, bx, by, mode, scale, win_left=0, wi
 
 
 def bsa_slice_backward(q_g, k_g, v_g, dout_g, mask_g, bx, by, mode, scale, win_left=0,
-                       win_right=0, q_blocks=None, kv_blocks=None):
+                       win_right=0, q_blocks=None, kv_blocks=None, out_storage=None):
     """One (batch, kv-head) slice of the backward pass.  Returns dQ [G,Sq,D], dK [Skv,D],
     dV [Skv,Dv], Out, LSE.  Units (h, qb) are skipped only when they contribute neither to a
     requested dQ block nor to a requested KV block, so every requested entry is exact."""
@@ -168,7 +184,7 @@ def bsa_slice_backward(q_g, k_g, v_g, dout_g, mask_g, bx, by, mode, scale, win_l
             vis = visible(rows, keys, mode, s_q, s_kv, s_kv, win_left, win_right)
             qr, kr, vr = q_g[h, rows], k_g[keys], v_g[keys]
             o, l, p = attend(qr, kr, vr, vis, scale)
-            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[h, rows], o, p, scale)
+            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[h, rows], stored_out(o, out_storage), p, scale)
             out[h, rows] = o
             lse[h, rows] = l
             dq[h, rows] = g_q
@@ -200,6 +216,7 @@ def bsa_forward(q, k, v, block_mask, bx, by, mode, scale, win_left=0, win_right=
 
 def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win_right=0):
     """Full BNSD backward; returns dQ, dK, dV, Out, LSE."""
+    out_storage = "bf16" if np.asarray(q).dtype == np.uint16 else None
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, N1, s_q, _ = q.shape
     N2 = k.shape[1]
@@ -213,7 +230,7 @@ def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win
         for g in range(N2):
             hs = slice(g * G, (g + 1) * G)
             r = bsa_slice_backward(q[b, hs], k[b, g], v[b, g], dout[b, hs], block_mask[b, hs],
-                                   bx, by, mode, scale, win_left, win_right)
+                                   bx, by, mode, scale, win_left, win_right, out_storage=out_storage)
             dq[b, hs], dk[b, g], dv[b, g], out[b, hs], lse[b, hs] = r
     return dq, dk, dv, out, lse
 
@@ -229,7 +246,8 @@ def nsa_token_keys(ids: np.ndarray, sel_block: int, seq_len: int) -> np.ndarray:
     return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
 
-def nsa_slice(q_g, k_g, v_g, topk_g, sel_block, mode, scale, dout_g=None, tokens=None):
+def nsa_slice(q_g, k_g, v_g, topk_g, sel_block, mode, scale, dout_g=None, tokens=None,
+              out_storage=None):
     """One (batch, kv-head) slice: q_g [S, G, D], k_g [S, D], v_g [S, Dv], topk_g [S, K].
     Forward for every listed token (all by default); with dout_g also the backward pass.
     Returns Out [S,G,Dv], LSE [S,G] (+ dQ [S,G,D], dK [S,D], dV [S,Dv]); unlisted tokens are NaN
@@ -248,7 +266,7 @@ def nsa_slice(q_g, k_g, v_g, topk_g, sel_block, mode, scale, dout_g=None, tokens
         o, l, p = attend(qr, kr, vr, vis, scale)
         out[t], lse[t] = o, l
         if dout_g is not None:
-            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[t], o, p, scale)
+            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[t], stored_out(o, out_storage), p, scale)
             dq[t] = g_q
             np.add.at(dk, keys, g_k)
             np.add.at(dv, keys, g_v)
@@ -277,6 +295,7 @@ def nsa_forward(q, k, v, topk, cu_seqlens, sel_block, mode, scale):
 
 def nsa_backward(q, k, v, dout, topk, cu_seqlens, sel_block, mode, scale):
     """Full TND backward; returns dQ, dK, dV, Out, LSE."""
+    out_storage = "bf16" if np.asarray(q).dtype == np.uint16 else None
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     T, N1, _ = q.shape
     N2 = k.shape[1]
@@ -291,7 +310,8 @@ def nsa_backward(q, k, v, dout, topk, cu_seqlens, sel_block, mode, scale):
         for g in range(N2):
             hs = slice(g * G, (g + 1) * G)
             o, l, gq, gk, gv = nsa_slice(q[t0:t1, hs], k[t0:t1, g], v[t0:t1, g], topk[t0:t1, g],
-                                         sel_block, mode, scale, dout_g=dout[t0:t1, hs])
+                                         sel_block, mode, scale, dout_g=dout[t0:t1, hs],
+                                         out_storage=out_storage)
             out[t0:t1, hs], lse[t0:t1, hs], dq[t0:t1, hs] = o, l, gq
             dk[t0:t1, g], dv[t0:t1, g] = gk, gv
     return dq, dk, dv, out, lse

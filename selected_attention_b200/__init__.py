@@ -29,6 +29,7 @@ EXPORTED = [
     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size", "bsa_fwd", "bsa_bwd",
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
+    "bsa_profile_enable", "bsa_profile_collect",
 ]
 
 
@@ -60,6 +61,10 @@ class Params(ctypes.Structure):
     ]
 
 
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double)]
+
+
 class MetaLayout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t), ("offsets", ctypes.c_size_t * 6), ("count", ctypes.c_int32)]
 
@@ -88,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_metadata.argtypes = [P, ctypes.c_int32, vp, sz, vp]
         L.bsa_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.bsa_diag_mma_tile.argtypes = [vp, vp, vp, ctypes.c_int32, vp, vp]
+        L.bsa_profile_enable.argtypes = [ctypes.c_int32]
+        L.bsa_profile_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
         L.bsa_version.restype = ctypes.c_char_p
         for name in EXPORTED:
             if name != "bsa_version":
@@ -220,6 +227,19 @@ def bsa_get_status(workspace, stream=None) -> int:
     v = ctypes.c_uint32()
     _check("bsa_get_status", lib().bsa_get_status(_ptr(workspace), _stream(stream), ctypes.byref(v)))
     return v.value
+
+
+def bsa_profile_enable(on: bool = True) -> None:
+    """Start (or stop) timing every kernel launch the library makes."""
+    _check("bsa_profile_enable", lib().bsa_profile_enable(1 if on else 0))
+
+
+def bsa_profile_collect() -> dict:
+    """{kernel name: (launches, total ms)} for the launches recorded since enabling (synchronises)."""
+    buf = (KernelTime * 64)()
+    n = ctypes.c_int32()
+    _check("bsa_profile_collect", lib().bsa_profile_collect(buf, 64, ctypes.byref(n)))
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(min(n.value, 64))}
 
 
 # ---------------------------------------------------------------------------------------------

@@ -53,6 +53,32 @@ size_t carve_bsa_fwd(const bsa_params* p, void* ws, BsaFwdWs* w) {
   return c.bytes();
 }
 
+struct BsaBwdWs {
+  uint32_t* status;
+  int32_t *counts, *row_ptr, *col;
+  uint8_t* maskT;
+  int32_t *t_counts, *t_row_ptr, *t_col;
+  float *dvec, *lse2;
+};
+
+size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
+  Carver c(ws);
+  const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+  const size_t units = static_cast<size_t>(p->B) * p->N1 * nqb;
+  const size_t t_rows = static_cast<size_t>(p->B) * p->N2 * nkb;
+  w->status = static_cast<uint32_t*>(ws);
+  w->counts = c.take<int32_t>(units);
+  w->row_ptr = c.take<int32_t>(units + 1);
+  w->col = c.take<int32_t>(units * nkb);
+  w->maskT = c.take<uint8_t>(units * nkb);
+  w->t_counts = c.take<int32_t>(t_rows);
+  w->t_row_ptr = c.take<int32_t>(t_rows + 1);
+  w->t_col = c.take<int32_t>(units * nkb);
+  w->dvec = c.take<float>(units * 128);
+  w->lse2 = c.take<float>(units * 128);
+  return c.bytes();
+}
+
 bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
 bsa_status check_ws(void* ws, size_t have, size_t need) {
@@ -101,13 +127,38 @@ bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void
 }
 
 bsa_status bsa_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
-  (void)p; (void)bytes;
-  return BSA_ERR_UNSUPPORTED;
+  if (!bytes) return BSA_ERR_NULLPTR;
+  bsa_status s = check_bsa(p);
+  if (s != BSA_OK) return s;
+  BsaBwdWs w;
+  *bytes = carve_bsa_bwd(p, nullptr, &w);
+  return BSA_OK;
 }
-bsa_status bsa_bwd(const bsa_params* p, const void*, const void*, const void*, const void*, const void*, const float*,
-                   void*, void*, void*, void*, size_t, void*) {
-  (void)p;
-  return BSA_ERR_UNSUPPORTED;
+
+bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void* v, const void* out,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  bsa_status s = check_bsa(p);
+  if (s != BSA_OK) return s;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !p->block_mask) return BSA_ERR_NULLPTR;
+  BsaBwdWs w;
+  const size_t need = carve_bsa_bwd(p, nullptr, &w);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != BSA_OK) return s;
+  carve_bsa_bwd(p, workspace, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = bsa_kv_lists(p->block_mask, p->B * p->N1 * nqb, nkb, w.counts, w.row_ptr, w.col, st);
+  if (e == cudaSuccess)
+    e = bsa_q_lists(p->block_mask, p->B, p->N1, p->N2, nqb, nkb, w.maskT, w.t_counts, w.t_row_ptr, w.t_col, st);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  BsaBwdArgs a;
+  a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.S_q = p->S_q; a.S_kv = p->S_kv;
+  a.bx = p->block_x; a.by = p->block_y; a.nqb = nqb; a.nkb = nkb;
+  a.mask_mode = p->mask_mode; a.win_left = p->win_left; a.win_right = p->win_right; a.scale = p->scale;
+  a.row_ptr = w.row_ptr; a.col = w.col; a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;
+  a.dvec = w.dvec; a.lse2 = w.lse2; a.dq = dq; a.dk = dk; a.dv = dv; a.status = w.status;
+  return cuda_status(bsa_bwd_launch(a, q, k, v, out, dout, lse, st));
 }
 bsa_status nsa_selected_fwd_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
 bsa_status nsa_selected_bwd_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }

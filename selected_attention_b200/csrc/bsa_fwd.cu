@@ -5,11 +5,12 @@
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S, masks, keeps the running
-//              max/sum, writes P (bf16) into shared memory, rescales O in TMEM, epilogue.
+//              max/sum, rescales O in TMEM, writes P back over the consumed S columns as two bf16
+//              parts (hi + lo, ~16 significant bits) that feed O += P V as the MMA's A operand.
 //   warp 4     TMA producer: Q once, then K/V tiles of the selected blocks into a 2-stage ring.
 //   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
-//              O += P_j V_j into the TMEM O accumulator.  S_{j+1} is issued before waiting for
-//              P_j, so the tensor core computes the next scores while softmax runs.
+//              O += P_j,hi V_j + P_j,lo V_j into the TMEM O accumulator.  S_{j+1} is issued before
+//              waiting for P_j, so the tensor core computes the next scores while softmax runs.
 // Every wait is bounded (sa_common.cuh); on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -30,7 +31,6 @@ struct __align__(1024) FwdSmem {
   uint8_t q[2][kBM * 128];        // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
   uint8_t k[2][2][BN * 128];      // [stage][sub-tile] K rows of one KV block
   uint8_t v[2][2][BN * 128];      // [stage][sub-tile] V rows
-  uint8_t p[BN / 64][kBM * 128];  // P (bf16) sub-tiles of 64 keys, K-major 128B swizzle
   uint64_t bar_q;
   uint64_t bar_k[2], bar_v[2], bar_kv_empty[2], bar_s_full[2];
   uint64_t bar_p_full, bar_o_done;
@@ -145,12 +145,15 @@ __global__ void __launch_bounds__(192, 1)
         const int st = j & 1;
         if (!(ok = mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status))) break;
         tc_fence_after();
+        const uint32_t p_col = st ? kColS1 : kColS0;
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(s.p[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.v[st][0]) + ks * 2048, BN * 128, 1024);
-          mma_bf16_ss(tmem + kColO, ad, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t bd = sdesc_sw128(smem_u32(s.v[st][0]) + ks * 2048, BN * 128, 1024);
+            mma_bf16_ts(tmem + kColO, tmem + p_col + half * (BN / 2) + ks * 8, bd, idesc_o,
+                        (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
+          }
         tc_commit(&s.bar_o_done);
         tc_commit(&s.bar_kv_empty[st]);
       }
@@ -197,52 +200,51 @@ __global__ void __launch_bounds__(192, 1)
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m, mx);
-      if (j > 0) {
+      // Lazy rescaling: the exponent reference m only moves when the row max exceeds it by more
+      // than 8 (p <= 2^8 otherwise); numerator and l share the same reference, so the final
+      // O / l is unchanged.  Only then must the previous O += P V have landed.
+      float m_new = m;
+      bool need = false;
+      if (mx > m + 8.f) {
+        need = (m != -INFINITY);
+        m_new = mx;
+      }
+      if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (j - 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
-        // tcgen05.ld/st are warp-collective: rescale when any row of the warp needs it
-        const bool need = m_new > m && m != -INFINITY;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2(m - m_new) : 1.f;
-          l *= alpha;
+        const float alpha = need ? ex2(m - m_new) : 1.f;
+        l *= alpha;
 #pragma unroll
-          for (int c = 0; c < kD; c += 32) {
-            uint32_t rr[32];
-            tmem_ld32(tmem + lane_base + kColO + c, rr);
-            tmem_ld_wait(rr);
+        for (int c = 0; c < kD; c += 32) {
+          uint32_t rr[32];
+          tmem_ld32(tmem + lane_base + kColO + c, rr);
+          tmem_ld_wait(rr);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-            tmem_st32(tmem + lane_base + kColO + c, rr);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          tmem_st32(tmem + lane_base + kColO + c, rr);
         }
+        tmem_st_wait();
       }
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const uint32_t s_col = st ? kColS1 : kColS0;
       float rowsum = 0.f;
 #pragma unroll
-      for (int t = 0; t < BN / 64; ++t) {
-        uint8_t* prow = s.p[t];
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t hv[16], lv[16];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float e[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            e[i] = ex2(x[t * 64 + c8 * 8 + i] - m_use);
-            rowsum += e[i];
-          }
-          uint4 pk;
-          pk.x = pack_bf16(e[0], e[1]);
-          pk.y = pack_bf16(e[2], e[3]);
-          pk.z = pack_bf16(e[4], e[5]);
-          pk.w = pack_bf16(e[6], e[7]);
-          *reinterpret_cast<uint4*>(prow + sw128_offset(r, c8 * 8)) = pk;
+        for (int i = 0; i < 16; ++i) {
+          const float e0 = ex2(x[c + 2 * i] - m_use), e1 = ex2(x[c + 2 * i + 1] - m_use);
+          rowsum += e0 + e1;
+          hv[i] = pack_bf16(e0, e1);
+          lv[i] = pack_bf16(e0 - bf16lo(hv[i]), e1 - bf16hi(hv[i]));
         }
+        tmem_st16(tmem + lane_base + s_col + c / 2, hv);
+        tmem_st16(tmem + lane_base + s_col + BN / 2 + c / 2, lv);
       }
+      tmem_st_wait();
       l += rowsum;
       m = m_new;
-      fence_async_smem();
       tc_fence_before();
       mbar_arrive(&s.bar_p_full);
     }
@@ -303,7 +305,9 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   if (e != cudaSuccess) return e;
   const int grid = a.B * a.N1 * a.nqb;
   if (grid == 0) return cudaSuccess;
+  prof_begin("bsa_fwd", st);
   bsa_fwd_kernel<BN><<<grid, 192, smem, st>>>(tq, tk, tv, p);
+  prof_end(st);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
 // Diagnostic: one 128 x 128 x 128 tcgen05 tile, C = A B^T with A K-major and B either K-major
-// ([N][K]) or MN-major ([K][N]).  Exercises exactly the building blocks the attention kernels use
+// ([N][K]) or MN-major ([K][N]); modes 2 and 3 take A from tensor memory (written with
+// tcgen05.st) with B K-major (2) or MN-major (3).  Exercises exactly the building blocks the attention kernels use
 // (TMA 128B-swizzled loads, smem descriptors of both majors, TMEM accumulate, tcgen05.ld), so a
 // parity failure in attention can be narrowed to the tile machinery or the attention logic.
 #include <cuda.h>
@@ -21,7 +22,7 @@ struct __align__(1024) DiagSmem {
 
 __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ CUtensorMap tm_a,
                                                        const __grid_constant__ CUtensorMap tm_b, float* c,
-                                                       int b_mn_major, uint32_t* status) {
+                                                       int b_mn_major, uint32_t* status, const void* a_ptr) {
   extern __shared__ uint8_t smem_raw[];
   DiagSmem& s = *reinterpret_cast<DiagSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -31,7 +32,7 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&s.tmem_base, 128);
+    tmem_alloc(&s.tmem_base, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -39,6 +40,19 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   bool ok = true;
+  if (b_mn_major >= 2) {
+    // A row (warp*32 + lane) from global into TMEM columns [128, 192): 64 packed bf16 pairs
+    const uint32_t* arow = reinterpret_cast<const uint32_t*>(a_ptr) + (warp * 32 + lane) * 64;
+    uint32_t r[16];
+    for (int c = 0; c < 64; c += 16) {
+      for (int i = 0; i < 16; ++i) r[i] = arow[c + i];
+      tmem_st16(tmem_addr(tmem, warp * 32, 128 + c), r);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   if (tid == 0) {
     mbar_arrive_expect_tx(&s.bar_load, 4 * 128 * 128);
     tma_load_2d(s.a[0], &tm_a, &s.bar_load, 0, 0);
@@ -48,10 +62,16 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
     ok = mbar_wait(&s.bar_load, 0, status);
     if (ok) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, 128, false, b_mn_major != 0);
+      const uint32_t idesc = idesc_bf16_f32(128, 128, false, b_mn_major == 1 || b_mn_major == 3);
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t ad = sdesc_sw128(smem_u32(s.a[ks / 4]) + (ks % 4) * 32, 0, 1024);
         uint64_t bd;
+        if (b_mn_major >= 2) {  // A from TMEM; B K-major (2) or MN-major (3)
+          bd = b_mn_major == 3 ? sdesc_sw128(smem_u32(s.b[0]) + ks * 2048, 128 * 128, 1024)
+                               : sdesc_sw128(smem_u32(s.b[ks / 4]) + (ks % 4) * 32, 0, 1024);
+          mma_bf16_ts(tmem, tmem + 128 + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
+          continue;
+        }
         if (b_mn_major)  // B tile is [K rows][N cols]: sub-tile = N chunk, K step = 16 rows
           bd = sdesc_sw128(smem_u32(s.b[0]) + ks * 2048, 128 * 128, 1024);
         else
@@ -79,7 +99,7 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace
@@ -93,7 +113,9 @@ cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, 
   const size_t smem = sizeof(DiagSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(diag_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  diag_mma_kernel<<<1, 128, smem, st>>>(ta, tb, c, b_mn_major, status);
+  prof_begin("diag_mma", st);
+  diag_mma_kernel<<<1, 128, smem, st>>>(ta, tb, c, b_mn_major, status, a);
+  prof_end(st);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,10 @@ struct Carver {
   size_t bytes() const { return align_up(off, 256); }
 };
 
+// ---- kernel timing (profile.cu): brackets a launch with events when timing is enabled ----------
+void prof_begin(const char* name, cudaStream_t st);
+void prof_end(cudaStream_t st);
+
 // ---- metadata (metadata.cu) -------------------------------------------------------------------
 // BSA KV lists: units (b, h, qb) -> ascending kv block ids.
 cudaError_t bsa_kv_lists(const uint8_t* mask, int units, int nkb, int32_t* counts, int32_t* row_ptr, int32_t* col,
@@ -58,6 +62,24 @@ struct BsaFwdArgs {
   uint32_t* status;
 };
 cudaError_t bsa_fwd_launch(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st);
+
+// ---- BSA backward (bsa_bwd.cu) -------------------------------------------------------------------
+struct BsaBwdArgs {
+  int B, N1, N2, S_q, S_kv, bx, by, nqb, nkb, mask_mode, win_left, win_right;
+  float scale;
+  const int32_t* row_ptr;    // KV lists per (b, h, qb)
+  const int32_t* col;
+  const int32_t* t_row_ptr;  // transposed lists per (b, g, kb)
+  const int32_t* t_col;
+  float* dvec;               // scratch [B*N1*nqb*128]
+  float* lse2;               // scratch [B*N1*nqb*128]
+  void* dq;
+  void* dk;
+  void* dv;
+  uint32_t* status;
+};
+cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, const void* v, const void* out,
+                           const void* dout, const float* lse, cudaStream_t st);
 
 // ---- diagnostics (diag.cu) -----------------------------------------------------------------------
 cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,

@@ -116,7 +116,9 @@ inline int div_up(int a, int b) { return (a + b - 1) / b; }
 }  // namespace
 
 cudaError_t exclusive_scan(const int32_t* counts, int n, int32_t* row_ptr, cudaStream_t st) {
+  prof_begin("meta_scan", st);
   scan_kernel<<<1, 1024, 0, st>>>(counts, n, row_ptr);
+  prof_end(st);
   return cudaGetLastError();
 }
 
@@ -124,11 +126,15 @@ cudaError_t bsa_kv_lists(const uint8_t* mask, int units, int nkb, int32_t* count
                          cudaStream_t st) {
   if (units <= 0) return cudaSuccess;
   const int grid = div_up(units, kWarps);
+  prof_begin("meta_count", st);
   count_rows_kernel<<<grid, kWarps * 32, 0, st>>>(mask, units, nkb, counts);
+  prof_end(st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if ((e = exclusive_scan(counts, units, row_ptr, st)) != cudaSuccess) return e;
+  prof_begin("meta_fill", st);
   fill_rows_kernel<<<grid, kWarps * 32, 0, st>>>(mask, units, nkb, row_ptr, col);
+  prof_end(st);
   return cudaGetLastError();
 }
 
@@ -136,7 +142,9 @@ cudaError_t bsa_q_lists(const uint8_t* mask, int B, int N1, int N2, int nqb, int
                         int32_t* counts, int32_t* row_ptr, int32_t* col, cudaStream_t st) {
   const int G = N1 / N2;
   dim3 grid(div_up(nkb, 32), div_up(nqb, 32), B * N1);
+  prof_begin("meta_transpose", st);
   transpose_mask_kernel<<<grid, dim3(32, 8), 0, st>>>(mask, N1, N2, nqb, nkb, maskT);
+  prof_end(st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return bsa_kv_lists(maskT, B * N2 * nkb, G * nqb, counts, row_ptr, col, st);

@@ -7,22 +7,12 @@ import torch
 import selected_attention_b200 as sa
 from oracle import attention as A
 from oracle import metadata as M
+from parity import LSE_ATOL, check_close, dev_bf16
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
-ATOL, RTOL_L2, LSE_ATOL = 1e-2, 1e-2, 1e-3
-
-
-def _dev(bits):
-    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).cuda()
-
-
-def _close(got, ref, what, atol=ATOL):
-    got = np.asarray(got, np.float64)
-    ref = np.asarray(ref, np.float64)
-    err = np.abs(got - ref)
-    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    assert err.max() <= atol and rel <= RTOL_L2, f"{what}: max abs {err.max():.3e} rel L2 {rel:.3e}"
+_dev = dev_bf16
+_close = check_close
 
 
 def test_diag_mma_tile(cuda_ok):
@@ -35,6 +25,13 @@ def test_diag_mma_tile(cuda_ok):
     assert sa.bsa_get_status(ws) == 0
     assert np.abs(c.cpu().numpy() - fa @ fb.T).max() < 1e-3
     c, ws = sa.bsa_diag_mma_tile(_dev(a), _dev(b), True)
+    torch.cuda.synchronize()
+    assert np.abs(c.cpu().numpy() - fa @ fb).max() < 1e-3
+    # A staged in tensor memory, B K-major then MN-major
+    c, ws = sa.bsa_diag_mma_tile(_dev(a), _dev(b), 2)
+    torch.cuda.synchronize()
+    assert np.abs(c.cpu().numpy() - fa @ fb.T).max() < 1e-3
+    c, ws = sa.bsa_diag_mma_tile(_dev(a), _dev(b), 3)
     torch.cuda.synchronize()
     assert np.abs(c.cpu().numpy() - fa @ fb).max() < 1e-3
 

@@ -369,3 +369,31 @@ def test_planted_mistakes_are_caught(monkeypatch):
         assert not (np.allclose(dq, r_dq, atol=1e-9) and np.allclose(dk, r_dk, atol=1e-9)
                     and np.allclose(dv, r_dv, atol=1e-9))
     monkeypatch.setattr(A, "attend_grad", good)
+
+
+def test_stored_out_softmax_grad_correction():
+    """softmax_grad taken from the bf16-stored attentionOut: since dS = P o (dP - D) is linear in D,
+    dQ_i moves by exactly -scale * dD_i * (P K)_i and dK_k by -scale * sum_i dD_i P_ik q_i, with
+    dD_i = dOut_i . (bf16(O_i) - O_i); dV does not move.  P, O and the base gradients come from
+    torch (float64) here, not from the oracle."""
+    rng = np.random.default_rng(10)
+    B, N, S, D, bs = 1, 1, 32, 16, 8
+    bits = [synth.f32_to_bf16_bits(rng.standard_normal((B, N, S, D), dtype=np.float32)) for _ in range(4)]
+    q, k, v, do = (A.bf16_to_f64(x) for x in bits)
+    mask = np.tril(np.ones((4, 4), np.uint8))[None, None]
+    sc = 0.25
+    dq_b, dk_b, dv_b, _, _ = A.bsa_backward(*bits, mask, bs, bs, 2, sc)   # bf16 inputs: stored Out
+    dense = _dense_mask_bsa(mask, bs, bs, S, S, 2)
+    _, _, r_dq, r_dk, r_dv = _torch_sdpa(q, k, v, dense, sc, do)          # exact D
+    s = sc * np.einsum("bhid,bhjd->bhij", q, k)
+    s = np.where(dense, s, -np.inf)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    o = p @ v
+    dD = np.sum(do * (A.round_to_bf16(o) - o), axis=-1)                  # [B, N, S]
+    exp_dq = r_dq - sc * dD[..., None] * (p @ k)
+    exp_dk = r_dk - sc * np.einsum("bhi,bhij,bhid->bhjd", dD, p, q)
+    assert np.abs(dD).max() > 0                                          # the reading matters here
+    assert np.allclose(dq_b, exp_dq, atol=1e-11)
+    assert np.allclose(dk_b, exp_dk, atol=1e-11)
+    assert np.allclose(dv_b, r_dv, atol=1e-11)
