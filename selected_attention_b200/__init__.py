@@ -29,7 +29,7 @@ EXPORTED = [
     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size", "bsa_fwd", "bsa_bwd",
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
-    "bsa_profile_enable", "bsa_profile_collect",
+    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc",
 ]
 
 
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).argtypes = [P, ctypes.POINTER(sz)]
         L.bsa_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nsa_selected_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.bsa_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
         L.bsa_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nsa_selected_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sfa_sparse_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -172,6 +173,23 @@ def bsa_fwd(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=
         workspace = _workspace(need, q.device)
     _check("bsa_fwd", lib().bsa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                     _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def bsa_fwd_noalloc(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
+                    win_right=0, out=None, lse=None, stream=None):
+    """bsa_fwd without a workspace, for callers that cannot allocate device memory: the library
+    keeps the scratch in a fixed 8 MiB device array (shared by all calls on a device; calls that
+    overlap on the GPU race).  Out and LSE are still the caller's tensors."""
+    _need_cuda(q, k, v, block_mask)
+    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right)
+    B, N1, S_q, _ = q.shape
+    if out is None:
+        out = torch.empty(B, N1, S_q, v.shape[-1], dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, N1, S_q, dtype=torch.float32, device=q.device)
+    _check("bsa_fwd_noalloc", lib().bsa_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                                    _ptr(lse), _stream(stream)))
     return out, lse
 
 
