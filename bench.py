@@ -174,8 +174,9 @@ def run_reference(args, rank, world):
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; warm-up steps are a no-op
     total_f, total_t, desc = 0, 0.0, ""
+    step_budget = min(args.ref_step_seconds, 150.0 / max(1, args.steps))  # whole run ~2.5 min at most
     for _ in range(args.steps):
-        f, t, desc = cpu_oracle_sample(w, mask, budget_s=args.ref_step_seconds)
+        f, t, desc = cpu_oracle_sample(w, mask, budget_s=step_budget)
         total_f += f
         total_t += t
     value = total_f / total_t / 1e12

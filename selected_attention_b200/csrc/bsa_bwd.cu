@@ -22,6 +22,8 @@ namespace {
 
 constexpr int kT = 128;  // rows of a Q tile and of a KV tile in the MMAs (M and N)
 constexpr int kD = 128;
+constexpr int kVecWarps = 8;  // element-wise warps: lane quarter = warp % 4, column half = warp / 4
+constexpr int kThreads = (kVecWarps + 2) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------------------------------------
@@ -94,6 +96,17 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
   }
 }
 
+// Exchange point of the two element-wise warps that share a TMEM lane quarter (64 arrivals,
+// bounded wait).  Orders each side's tensor-memory reads before the other side's writes.
+__device__ __forceinline__ bool pair_sync(uint64_t* bar, int& exchanges, uint32_t* status) {
+  tc_fence_before();
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, exchanges & 1, status);
+  ++exchanges;
+  tc_fence_after();
+  return ok;
+}
+
 // Split x into bf16 hi + lo (x ~= hi + lo to about 2^-17 relative): the dK and dQ products run as
 // two MMAs, hi then lo, so dS enters the tensor cores with ~16 significant bits.
 __device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
@@ -117,10 +130,11 @@ struct __align__(1024) KvSmem {
   uint64_t bar_kv, bar_q[2], bar_do[2];
   uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_done;
   uint64_t bar_q_empty[2], bar_do_empty[2];
+  uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const BwdParams prm) {
@@ -147,9 +161,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&s.bar_s_full, 1);
     mbar_init(&s.bar_dp_full, 1);
-    mbar_init(&s.bar_p_ready, kT);
-    mbar_init(&s.bar_ds_ready, kT);
+    mbar_init(&s.bar_p_ready, kVecWarps * 32);
+    mbar_init(&s.bar_ds_ready, kVecWarps * 32);
     mbar_init(&s.bar_done, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -170,7 +185,7 @@ __global__ void __launch_bounds__(192, 1)
     qpos0 = qb * prm.bx;
   };
 
-  if (warp == 4) {
+  if (warp == kVecWarps) {
     // ------------------------------------------------------------------ producer
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(&s.bar_kv, 4 * kT * 128);
@@ -204,7 +219,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = (ndo > 2 ? ndo - 2 : 0); i < ndo; ++i) mbar_wait(&s.bar_do[i & 1], (i >> 1) & 1, prm.status);
       mbar_wait(&s.bar_kv, 0, prm.status);
     }
-  } else if (warp == 5) {
+  } else if (warp == kVecWarps + 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
       const uint32_t id_kmaj = idesc_bf16_f32(kT, kT, false, false);  // S^T, dP^T
@@ -262,8 +277,10 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) tc_commit(&s.bar_done);
     }
   } else {
-    // ------------------------------------------------------------------ P / dS warpgroup
-    const int r = tid;  // key row within the KV tile == TMEM lane
+    // ------------------------------------------------------------------ P / dS warps
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // key row within the KV tile == TMEM lane
+    const int c0 = hf * (kT / 2);       // this thread's query columns [c0, c0 + 64)
     const int kpos = kb * prm.by + r;
     const bool key_valid = r < prm.by && kpos < prm.S_kv;
     // query positions that see this key: [qlo, qhi]
@@ -273,7 +290,8 @@ __global__ void __launch_bounds__(192, 1)
     else if (prm.mask_mode == 3) qlo = kpos - shift;
     else if (prm.mask_mode == 4) { qlo = kpos - shift - prm.win_right; qhi = kpos - shift + prm.win_left; }
     if (!key_valid) { qlo = 1; qhi = 0; }
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int exchanges = 0;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int st = i & 1;
@@ -283,32 +301,35 @@ __global__ void __launch_bounds__(192, 1)
                                        mbar_wait(&s.bar_s_full, i & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
-      const bool full = qpos0 >= qlo && qpos0 + kT - 1 <= qhi;
-      const float* l2 = s.lse2[st];
-      float p[kT];
+      const bool full = qpos0 + c0 >= qlo && qpos0 + c0 + kT / 2 - 1 <= qhi;
+      const float* l2 = s.lse2[st] + c0;
+      float p[kT / 2];
 #pragma unroll
-      for (int c = 0; c < kT; c += 32) {
+      for (int c = 0; c < kT / 2; c += 32) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColS + c, rr);
+        tmem_ld32(tmem + lane_base + kColS + c0 + c, rr);
         tmem_ld_wait(rr);
 #pragma unroll
         for (int k2 = 0; k2 < 32; ++k2) p[c + k2] = ex2(__uint_as_float(rr[k2]) * prm.scale_log2 - l2[c + k2]);
       }
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < kT; ++c) {
-          const int qp = qpos0 + c;
+        for (int c = 0; c < kT / 2; ++c) {
+          const int qp = qpos0 + c0 + c;
           if (qp < qlo || qp > qhi) p[c] = 0.f;
         }
       }
-      // P^T hi/lo -> S^T[0,64) / S^T[64,128): A operands of dV += P^T dO
+      // both halves have read S^T before either overwrites it:
+      // P^T hi -> S^T[c0/2, +32), P^T lo -> S^T[64 + c0/2, +32): A operands of dV += P^T dO
+      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+      if (!ok) break;
 #pragma unroll
-      for (int c = 0; c < kT; c += 32) {
+      for (int c = 0; c < kT / 2; c += 32) {
         uint32_t hv[16], lv[16];
 #pragma unroll
         for (int k2 = 0; k2 < 16; ++k2) split_pack(p[c + 2 * k2], p[c + 2 * k2 + 1], hv[k2], lv[k2]);
-        tmem_st16(tmem + lane_base + kColS + c / 2, hv);
-        tmem_st16(tmem + lane_base + kColS + 64 + c / 2, lv);
+        tmem_st16(tmem + lane_base + kColS + (c0 + c) / 2, hv);
+        tmem_st16(tmem + lane_base + kColS + 64 + (c0 + c) / 2, lv);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -316,66 +337,45 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, i & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
-      const float* dvv = s.dvec[st];
-      uint32_t lo01[32];
-      // dS^T = P^T o (dP^T - D): the hi part of chunk c (32 columns) goes to dP^T[c/2, c/2+16),
-      // already read.  The lo part goes to dP^T[64 + c/2, ...), which is only free once chunk
-      // 2 + c/64 has been read: lo of chunks 0,1 is written after chunk 2 is read, lo of chunks
-      // 2,3 after chunk 3.
-      uint32_t lo_held[32];
+      const float* dvv = s.dvec[st] + c0;
+      // dS^T = P^T o (dP^T - D); hi -> dP^T[c0/2, +32), lo -> dP^T[64 + c0/2, +32)
+      uint32_t hv[32], lv[32];
 #pragma unroll
-      for (int c = 0; c < kT; c += 32) {
+      for (int c = 0; c < kT / 2; c += 32) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColDP + c, rr);
+        tmem_ld32(tmem + lane_base + kColDP + c0 + c, rr);
         tmem_ld_wait(rr);
-        uint32_t hv[16], lv[16];
 #pragma unroll
         for (int k2 = 0; k2 < 16; ++k2) {
           const int cc = c + 2 * k2;
           split_pack(p[cc] * (__uint_as_float(rr[2 * k2]) - dvv[cc]),
-                     p[cc + 1] * (__uint_as_float(rr[2 * k2 + 1]) - dvv[cc + 1]), hv[k2], lv[k2]);
-        }
-        tmem_st16(tmem + lane_base + kColDP + c / 2, hv);
-        if (c == 0 || c == 64) {
-#pragma unroll
-          for (int k2 = 0; k2 < 16; ++k2) lo_held[k2] = lv[k2];
-        } else {  // c == 32 or 96: chunks (c-32, c) complete a pair
-#pragma unroll
-          for (int k2 = 0; k2 < 16; ++k2) lo_held[16 + k2] = lv[k2];
-          if (c == 96) {
-            // chunk 3 read: pair (2,3) may go to [96,128); pair (0,1) went out at c == 64 below
-            tmem_st16(tmem + lane_base + kColDP + 96, lo_held);
-            tmem_st16(tmem + lane_base + kColDP + 112, lo_held + 16);
-          }
-        }
-        if (c == 64) {
-          // chunk 2 read: the held pair (0,1) goes to [64,96)
-          tmem_st16(tmem + lane_base + kColDP + 64, lo01);
-          tmem_st16(tmem + lane_base + kColDP + 80, lo01 + 16);
-        }
-        if (c == 32) {
-#pragma unroll
-          for (int k2 = 0; k2 < 32; ++k2) lo01[k2] = lo_held[k2];
+                     p[cc + 1] * (__uint_as_float(rr[2 * k2 + 1]) - dvv[cc + 1]), hv[cc / 2], lv[cc / 2]);
         }
       }
+      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+      if (!ok) break;
+      tmem_st16(tmem + lane_base + kColDP + c0 / 2, hv);
+      tmem_st16(tmem + lane_base + kColDP + c0 / 2 + 16, hv + 16);
+      tmem_st16(tmem + lane_base + kColDP + 64 + c0 / 2, lv);
+      tmem_st16(tmem + lane_base + kColDP + 64 + c0 / 2 + 16, lv + 16);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&s.bar_ds_ready);
     }
-    // ---- epilogue: dK = scale * acc, dV = acc
+    // ---- epilogue: dK = scale * acc, dV = acc (this thread: head-dim columns [c0, c0 + 64))
     bool have = ok && n > 0;
     if (have) {
       have = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, 0, prm.status));
       tc_fence_after();
     }
-    __nv_bfloat16* dkrow = prm.dk + static_cast<size_t>(kv_row0 + r) * kD;
-    __nv_bfloat16* dvrow = prm.dv + static_cast<size_t>(kv_row0 + r) * kD;
+    __nv_bfloat16* dkrow = prm.dk + static_cast<size_t>(kv_row0 + r) * kD + c0;
+    __nv_bfloat16* dvrow = prm.dv + static_cast<size_t>(kv_row0 + r) * kD + c0;
 #pragma unroll
-    for (int c = 0; c < kD; c += 32) {
+    for (int c = 0; c < kD / 2; c += 32) {
       uint32_t rk[32], rv[32];
       if (have) {
-        tmem_ld32(tmem + lane_base + kColDK + c, rk);
-        tmem_ld32(tmem + lane_base + kColDV + c, rv);
+        tmem_ld32(tmem + lane_base + kColDK + c0 + c, rk);
+        tmem_ld32(tmem + lane_base + kColDV + c0 + c, rv);
         tmem_ld_wait(rk);
 #pragma unroll
         for (int i = 0; i < 32; ++i) reg_fence(rv[i]);
@@ -407,11 +407,12 @@ struct __align__(1024) QSmem {
   uint8_t k[2][2][BN * 128];  // [stage][sub-tile] [BN keys][64 d]
   uint8_t v[2][2][BN * 128];
   uint64_t bar_qdo, bar_k[2], bar_v[2], bar_kv_empty[2], bar_s_full[2], bar_dp_full, bar_ds_ready, bar_done;
+  uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     bsa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const BwdParams prm) {
@@ -438,8 +439,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&s.bar_s_full[i], 1);
     }
     mbar_init(&s.bar_dp_full, 1);
-    mbar_init(&s.bar_ds_ready, kT);
+    mbar_init(&s.bar_ds_ready, kVecWarps * 32);
     mbar_init(&s.bar_done, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -451,7 +453,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 4) {
+  if (warp == kVecWarps) {
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(&s.bar_qdo, 4 * kT * 128);
       tma_load_2d(s.q[0], &tm_q, &s.bar_qdo, 0, q_row0);
@@ -477,7 +479,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       mbar_wait(&s.bar_qdo, 0, prm.status);
     }
-  } else if (warp == 5) {
+  } else if (warp == kVecWarps + 1) {
     if (lane == 0 && n > 0) {
       const uint32_t id_s = idesc_bf16_f32(kT, BN, false, false);
       const uint32_t id_dq = idesc_bf16_f32(kT, kD, false, true);
@@ -530,7 +532,10 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) tc_commit(&s.bar_done);
     }
   } else {
-    const int r = tid;
+    constexpr int kHalf = BN / 2;
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // query row == TMEM lane
+    const int c0 = hf * kHalf;          // this thread's key columns [c0, c0 + BN/2)
     const int qpos = qb * prm.bx + r;
     const bool row_valid = r < prm.bx && qpos < prm.S_q;
     int lo = 0, hi = prm.S_kv - 1;
@@ -542,7 +547,8 @@ __global__ void __launch_bounds__(192, 1)
     const size_t trow = static_cast<size_t>(unit) * kT + r;
     const float l2 = prm.lse2[trow];
     const float dval = prm.dvec[trow];
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int exchanges = 0;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j & 1;
@@ -550,20 +556,20 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (j >> 1) & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
-      const int kpos0 = prm.col[rp + j] * prm.by;
-      const bool full = kpos0 >= lo && kpos0 + BN - 1 <= hi;
-      float p[BN];
+      const int kpos0 = prm.col[rp + j] * prm.by + c0;
+      const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
+      float p[kHalf];
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < kHalf; c += 32) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + s_col + c, rr);
+        tmem_ld32(tmem + lane_base + s_col + c0 + c, rr);
         tmem_ld_wait(rr);
 #pragma unroll
         for (int i = 0; i < 32; ++i) p[c + i] = ex2(__uint_as_float(rr[i]) * prm.scale_log2 - l2);
       }
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
+        for (int c = 0; c < kHalf; ++c) {
           const int kp = kpos0 + c;
           if (kp < lo || kp > hi) p[c] = 0.f;
         }
@@ -571,18 +577,25 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, j & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t hv[kHalf / 2], lv[kHalf / 2];
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < kHalf; c += 32) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColDP + c, rr);
+        tmem_ld32(tmem + lane_base + kColDP + c0 + c, rr);
         tmem_ld_wait(rr);
-        uint32_t hv[16], lv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           split_pack(p[c + 2 * i] * (__uint_as_float(rr[2 * i]) - dval),
-                     p[c + 2 * i + 1] * (__uint_as_float(rr[2 * i + 1]) - dval), hv[i], lv[i]);
-        tmem_st16(tmem + lane_base + s_col + c / 2, hv);
-        tmem_st16(tmem + lane_base + s_col + BN / 2 + c / 2, lv);
+                     p[c + 2 * i + 1] * (__uint_as_float(rr[2 * i + 1]) - dval), hv[c / 2 + i], lv[c / 2 + i]);
+      }
+      // both halves have read S_j before either writes dS over it:
+      // hi -> S_j[c0/2, +BN/4), lo -> S_j[BN/2 + c0/2, +BN/4)
+      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+      if (!ok) break;
+#pragma unroll
+      for (int c = 0; c < kHalf / 2; c += 16) {
+        tmem_st16(tmem + lane_base + s_col + c0 / 2 + c, hv + c);
+        tmem_st16(tmem + lane_base + s_col + BN / 2 + c0 / 2 + c, lv + c);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -593,12 +606,13 @@ __global__ void __launch_bounds__(192, 1)
       have = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, 0, prm.status));
       tc_fence_after();
     }
-    __nv_bfloat16* dqrow = prm.dq + static_cast<size_t>(q_row0 + r) * kD;
+    const int d0 = hf * (kD / 2);  // this thread's head-dim columns of dQ
+    __nv_bfloat16* dqrow = prm.dq + static_cast<size_t>(q_row0 + r) * kD + d0;
 #pragma unroll
-    for (int c = 0; c < kD; c += 32) {
+    for (int c = 0; c < kD / 2; c += 32) {
       uint32_t rr[32];
       if (have) {
-        tmem_ld32(tmem + lane_base + kColDQ + c, rr);
+        tmem_ld32(tmem + lane_base + kColDQ + d0 + c, rr);
         tmem_ld_wait(rr);
       } else {
 #pragma unroll
@@ -619,7 +633,7 @@ cudaError_t launch_q(const BwdParams& p, const CUtensorMap& tq, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(bsa_bwd_q_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   prof_begin("bsa_bwd_q", st);
-  bsa_bwd_q_kernel<BN><<<grid, 192, smem, st>>>(tq, tk, tv, tdo, p);
+  bsa_bwd_q_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, p);
   prof_end(st);
   return cudaGetLastError();
 }
@@ -666,7 +680,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     if (e != cudaSuccess) return e;
     const int grid = a.B * a.N2 * a.nkb;
     prof_begin("bsa_bwd_kv", st);
-    bsa_bwd_kv_kernel<<<grid, 192, smem, st>>>(tq, tk128, tv128, tdo, pk);
+    bsa_bwd_kv_kernel<<<grid, kThreads, smem, st>>>(tq, tk128, tv128, tdo, pk);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

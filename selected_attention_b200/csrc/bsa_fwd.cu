@@ -3,12 +3,15 @@
 // One CTA per unit (b, h, q block): 128 query rows against the KV blocks the unit's
 // BlockSparseMask row selects (CSR lists from metadata.cu).
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S, masks, keeps the running
-//              max/sum, rescales O in TMEM, writes P back over the consumed S columns as two bf16
-//              parts (hi + lo, ~16 significant bits) that feed O += P V as the MMA's A operand.
-//   warp 4     TMA producer: Q once, then K/V tiles of the selected blocks into a 2-stage ring.
-//   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
+// Warp roles (320 threads):
+//   warps 0-7  softmax: warp w reads TMEM lane quarter w % 4 (query rows 32*(w%4) .. +31) and the
+//              column half w / 4 of each S tile, so each row is shared by two threads that
+//              exchange their partial row max through shared memory.  They mask, keep the
+//              running max/sum, rescale their half of O in TMEM when needed, and write P back
+//              over the consumed S columns as two bf16 parts (hi + lo, ~16 significant bits)
+//              that feed O += P V as the MMA's A operand.
+//   warp 8     TMA producer: Q once, then K/V tiles of the selected blocks into a 2-stage ring.
+//   warp 9     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
 //              O += P_j,hi V_j + P_j,lo V_j into the TMEM O accumulator.  S_{j+1} is issued before
 //              waiting for P_j, so the tensor core computes the next scores while softmax runs.
 // Every wait is bounded (sa_common.cuh); on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
@@ -23,6 +26,8 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per CTA tile (the MMA M)
 constexpr int kD = 128;   // head dim of Q/K and V
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -31,9 +36,12 @@ struct __align__(1024) FwdSmem {
   uint8_t q[2][kBM * 128];        // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
   uint8_t k[2][2][BN * 128];      // [stage][sub-tile] K rows of one KV block
   uint8_t v[2][2][BN * 128];      // [stage][sub-tile] V rows
+  float red[2][2][kBM];           // [tile parity][column half][row]: partial row max / row sum
   uint64_t bar_q;
   uint64_t bar_k[2], bar_v[2], bar_kv_empty[2], bar_s_full[2];
   uint64_t bar_p_full, bar_o_done;
+  uint64_t bar_done;              // one phase: the last O += P V has completed
+  uint64_t bar_pair[4];           // the two softmax warps of each TMEM lane quarter
   uint32_t tmem_base;
 };
 
@@ -47,12 +55,25 @@ struct FwdParams {
   uint32_t* status;
 };
 
+// Exchange point of the two softmax warps that share a TMEM lane quarter: an mbarrier of 64
+// arrivals with a bounded wait (a plain bar.sync could not give up if the partner stopped early).
+// The tcgen05 fences order each side's tensor-memory reads before the other side's writes.
+__device__ __forceinline__ bool pair_sync(uint64_t* bar, int& exchanges, uint32_t* status) {
+  tc_fence_before();
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, exchanges & 1, status);
+  ++exchanges;
+  tc_fence_after();
+  return ok;
+}
+
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
   constexpr uint32_t kTmemCols = (2 * BN + kD) <= 256 ? 256 : 512;
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
+  constexpr int kHalf = BN / 2;  // S columns per softmax thread
   extern __shared__ uint8_t smem_raw[];
   FwdSmem<BN>& s = *reinterpret_cast<FwdSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -76,8 +97,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&s.bar_kv_empty[i], 1);
       mbar_init(&s.bar_s_full[i], 1);
     }
-    mbar_init(&s.bar_p_full, kBM);
+    mbar_init(&s.bar_p_full, kSoftmaxWarps * 32);
     mbar_init(&s.bar_o_done, 1);
+    mbar_init(&s.bar_done, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -89,7 +112,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 4) {
+  if (warp == kSoftmaxWarps) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_q);
@@ -118,7 +141,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       mbar_wait(&s.bar_q, 0, prm.status);
     }
-  } else if (warp == 5) {
+  } else if (warp == kSoftmaxWarps + 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
@@ -157,10 +180,12 @@ __global__ void __launch_bounds__(192, 1)
         tc_commit(&s.bar_o_done);
         tc_commit(&s.bar_kv_empty[st]);
       }
+      if (ok) tc_commit(&s.bar_done);
     }
   } else {
-    // ------------------------------------------------------------------ softmax warpgroup
-    const int r = tid;  // query row within the tile == TMEM lane
+    // ------------------------------------------------------------------ softmax warps
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
     const int qpos = qb * prm.bx + r;
     const bool row_valid = r < prm.bx && qpos < prm.S_q;
     // visible key interval [lo, hi] for this row (mask modes 0/2/3/4)
@@ -171,35 +196,44 @@ __global__ void __launch_bounds__(192, 1)
     else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
     if (!row_valid) { lo = 1; hi = 0; }
 
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t o_col = kColO + hf * (kD / 2);  // this thread's half of the O row
+    float m = -INFINITY, l = 0.f;                  // l: partial sum over this thread's columns
+    int exchanges = 0;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (j >> 1) & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
-      const int kpos0 = prm.col[rp + j] * prm.by;
-      float x[BN];
+      const uint32_t s_col = st ? kColS1 : kColS0;
+      const int kpos0 = prm.col[rp + j] * prm.by + hf * kHalf;
+      float x[kHalf];
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < kHalf; c += 32) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + (st ? kColS1 : kColS0) + c, rr);
+        tmem_ld32(tmem + lane_base + s_col + hf * kHalf + c, rr);
         tmem_ld_wait(rr);
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(rr[i]) * prm.scale_log2;
       }
-      const bool full = kpos0 >= lo && kpos0 + BN - 1 <= hi;
+      const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
+        for (int c = 0; c < kHalf; ++c) {
           const int kp = kpos0 + c;
           if (kp < lo || kp > hi) x[c] = -INFINITY;
         }
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      for (int c = 0; c < kHalf; ++c) mx = fmaxf(mx, x[c]);
+      // row max = max of the two halves; the barrier also orders both threads' S reads before
+      // either writes P over the S columns
+      s.red[st][hf][r] = mx;
+      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+      if (!ok) break;
+      mx = fmaxf(mx, s.red[st][hf ^ 1][r]);
       // Lazy rescaling: the exponent reference m only moves when the row max exceeds it by more
       // than 8 (p <= 2^8 otherwise); numerator and l share the same reference, so the final
       // O / l is unchanged.  Only then must the previous O += P V have landed.
@@ -210,27 +244,29 @@ __global__ void __launch_bounds__(192, 1)
         m_new = mx;
       }
       if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
+        // O += P_{j-1} V_{j-1} is o_done phase j-1.  S_j landed after every earlier MMA (one
+        // commit covers all prior MMAs), so phase j-2 is complete and j cannot be: the barrier is
+        // in phase j-1 or j, which a parity wait tells apart.
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (j - 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
         const float alpha = need ? ex2(m - m_new) : 1.f;
         l *= alpha;
 #pragma unroll
-        for (int c = 0; c < kD; c += 32) {
+        for (int c = 0; c < kD / 2; c += 32) {
           uint32_t rr[32];
-          tmem_ld32(tmem + lane_base + kColO + c, rr);
+          tmem_ld32(tmem + lane_base + o_col + c, rr);
           tmem_ld_wait(rr);
 #pragma unroll
           for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(tmem + lane_base + kColO + c, rr);
+          tmem_st32(tmem + lane_base + o_col + c, rr);
         }
         tmem_st_wait();
       }
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const uint32_t s_col = st ? kColS1 : kColS0;
       float rowsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < kHalf; c += 32) {
         uint32_t hv[16], lv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -239,8 +275,9 @@ __global__ void __launch_bounds__(192, 1)
           hv[i] = pack_bf16(e0, e1);
           lv[i] = pack_bf16(e0 - bf16lo(hv[i]), e1 - bf16hi(hv[i]));
         }
-        tmem_st16(tmem + lane_base + s_col + c / 2, hv);
-        tmem_st16(tmem + lane_base + s_col + BN / 2 + c / 2, lv);
+        // packed pairs: element column e -> column e/2 (hi) and BN/2 + e/2 (lo)
+        tmem_st16(tmem + lane_base + s_col + (hf * kHalf + c) / 2, hv);
+        tmem_st16(tmem + lane_base + s_col + BN / 2 + (hf * kHalf + c) / 2, lv);
       }
       tmem_st_wait();
       l += rowsum;
@@ -248,20 +285,26 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&s.bar_p_full);
     }
-    // ---- epilogue
+    // ---- epilogue.  Not a parity wait on o_done: with lazy rescaling this thread may not have
+    // observed the earlier o_done phases, and a parity wait can only tell one phase from the next.
     bool have_o = ok && n > 0;
     if (have_o) {
-      have_o = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (n - 1) & 1, prm.status));
+      have_o = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, 0, prm.status));
       tc_fence_after();
     }
+    // full row sum from the two halves, through the reduction slot of parity n & 1 (the last
+    // max exchange used parity (n - 1) & 1, and both threads passed the exchange before it)
+    s.red[n & 1][hf][r] = l;
+    if (ok) have_o = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status)) && have_o;
+    l += s.red[n & 1][hf ^ 1][r];
     const bool any = have_o && l > 0.f;
     const float inv_l = any ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = prm.out + static_cast<size_t>(q_row0 + r) * kD;
+    __nv_bfloat16* orow = prm.out + static_cast<size_t>(q_row0 + r) * kD + hf * (kD / 2);
 #pragma unroll
-    for (int c = 0; c < kD; c += 32) {
+    for (int c = 0; c < kD / 2; c += 32) {
       uint32_t rr[32];
       if (have_o) {  // warp-uniform: every lane joins the collective load
-        tmem_ld32(tmem + lane_base + kColO + c, rr);
+        tmem_ld32(tmem + lane_base + o_col + c, rr);
         tmem_ld_wait(rr);
       } else {
 #pragma unroll
@@ -279,7 +322,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
-    if (row_valid) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
+    if (row_valid && hf == 0) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
   }
   tc_fence_before();
   __syncthreads();
@@ -306,7 +349,7 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   const int grid = a.B * a.N1 * a.nqb;
   if (grid == 0) return cudaSuccess;
   prof_begin("bsa_fwd", st);
-  bsa_fwd_kernel<BN><<<grid, 192, smem, st>>>(tq, tk, tv, p);
+  bsa_fwd_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
   prof_end(st);
   return cudaGetLastError();
 }

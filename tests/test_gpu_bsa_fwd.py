@@ -107,6 +107,22 @@ def test_bsa_fwd_cases(cuda_ok, case):
     _run_case(**case, mask=mask, seed=3, wl=wl, wr=wr)
 
 
+@pytest.mark.parametrize("case", [
+    dict(B=2, N1=4, N2=4, S_q=300, S_kv=300, bx=128, by=128, mode=2),
+    dict(B=1, N1=4, N2=1, S_q=328, S_kv=328, bx=64, by=64, mode=2),
+])
+def test_bsa_fwd_short_lists(cuda_ok, case):
+    """Units with one or two KV tiles and no diagonal block: the epilogue must wait for the last
+    O += P V even when softmax finishes long before it."""
+    rng = np.random.default_rng(11)
+    nqb = -(-case["S_q"] // case["bx"])
+    nkb = -(-case["S_kv"] // case["by"])
+    mask = (rng.random((case["B"], case["N1"], nqb, nkb)) < 0.6).astype(np.uint8)
+    mask[..., 1, :] = 0
+    mask[..., :, -1] = 0
+    _run_case(**case, mask=mask, seed=4)
+
+
 def test_bsa_fwd_full_size_sampled(cuda_ok):
     """BSA S=8192 workload at full size in one launch; two heads checked against the oracle."""
     w = synth.workload(2)
