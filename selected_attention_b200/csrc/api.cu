@@ -28,7 +28,7 @@ bsa_status check_bsa(const bsa_params* p) {
       p->mask_mode != BSA_MASK_BAND)
     return BSA_ERR_INVALID_ARG;
   if (p->mask_mode == BSA_MASK_BAND && (p->win_left < 0 || p->win_right < 0)) return BSA_ERR_INVALID_ARG;
-  if (!std::isfinite(p->scale)) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale) || p->scale <= 0.f) return BSA_ERR_INVALID_ARG;  // a positive softmax scale
   const long long rows_q = 1LL * p->B * p->N1 * p->S_q, rows_kv = 1LL * p->B * p->N2 * p->S_kv;
   if (rows_q + 256 >= (1LL << 31) || rows_kv + 256 >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
   const long long nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);

@@ -400,13 +400,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dS for tile j is written back as bf16 hi -> S_j[0,BN/2) and lo -> S_j[BN/2,BN), the A operands
 // of dQ += dS K.
 // ------------------------------------------------------------------------------------------------
+constexpr int kQKStages = 3, kQVStages = 2;  // K is held by S and dQ, V only by dP
+
 template <int BN>
 struct __align__(1024) QSmem {
   uint8_t q[2][kT * 128];
   uint8_t dout[2][kT * 128];
-  uint8_t k[2][2][BN * 128];  // [stage][sub-tile] [BN keys][64 d]
-  uint8_t v[2][2][BN * 128];
-  uint64_t bar_qdo, bar_k[2], bar_v[2], bar_kv_empty[2], bar_s_full[2], bar_dp_full, bar_ds_ready, bar_done;
+  uint8_t k[kQKStages][2][BN * 128];  // [stage][sub-tile] [BN keys][64 d]
+  uint8_t v[kQVStages][2][BN * 128];
+  uint64_t bar_qdo, bar_k[kQKStages], bar_k_empty[kQKStages], bar_v[kQVStages], bar_v_empty[kQVStages];
+  uint64_t bar_s_full[2], bar_dp_full, bar_ds_ready, bar_done;
   uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
@@ -432,12 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&s.bar_qdo, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQKStages; ++i) {
       mbar_init(&s.bar_k[i], 1);
-      mbar_init(&s.bar_v[i], 1);
-      mbar_init(&s.bar_kv_empty[i], 1);
-      mbar_init(&s.bar_s_full[i], 1);
+      mbar_init(&s.bar_k_empty[i], 1);
     }
+    for (int i = 0; i < kQVStages; ++i) {
+      mbar_init(&s.bar_v[i], 1);
+      mbar_init(&s.bar_v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_s_full[i], 1);
     mbar_init(&s.bar_dp_full, 1);
     mbar_init(&s.bar_ds_ready, kVecWarps * 32);
     mbar_init(&s.bar_done, 1);
@@ -460,23 +466,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(s.q[1], &tm_q, &s.bar_qdo, 64, q_row0);
       tma_load_2d(s.dout[0], &tm_do, &s.bar_qdo, 0, q_row0);
       tma_load_2d(s.dout[1], &tm_do, &s.bar_qdo, 64, q_row0);
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&s.bar_kv_empty[st], ((j - 2) >> 1) & 1, prm.status)) break;
+      int issued_k = 0, issued_v = 0;
+      bool ok = true;
+      auto load_v = [&](int jv) -> bool {
+        const int sv = jv % kQVStages, uv = jv / kQVStages;
+        if (jv >= kQVStages && !mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status)) return false;
+        const int vrow = kv_row0 + prm.col[rp + jv] * prm.by;
+        mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
+        tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
+        tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
+        issued_v = jv + 1;
+        return true;
+      };
+      for (int j = 0; ok && j < n; ++j) {
+        const int sk = j % kQKStages, uk = j / kQKStages;
+        if (j >= kQKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
         const int row = kv_row0 + prm.col[rp + j] * prm.by;
-        mbar_arrive_expect_tx(&s.bar_k[st], 2 * BN * 128);
-        tma_load_2d(s.k[st][0], &tm_k, &s.bar_k[st], 0, row);
-        tma_load_2d(s.k[st][1], &tm_k, &s.bar_k[st], 64, row);
-        mbar_arrive_expect_tx(&s.bar_v[st], 2 * BN * 128);
-        tma_load_2d(s.v[st][0], &tm_v, &s.bar_v[st], 0, row);
-        tma_load_2d(s.v[st][1], &tm_v, &s.bar_v[st], 64, row);
-        issued = j + 1;
+        mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
+        tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
+        tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
+        issued_k = j + 1;
+        const int jv = j - (kQKStages - kQVStages);  // V trails K by one tile
+        if (jv >= 0) ok = load_v(jv);
       }
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
-        mbar_wait(&s.bar_k[j & 1], (j >> 1) & 1, prm.status);
-        mbar_wait(&s.bar_v[j & 1], (j >> 1) & 1, prm.status);
-      }
+      for (int jv = issued_v; ok && jv < n; ++jv) ok = load_v(jv);
+      for (int j = (issued_k > kQKStages ? issued_k - kQKStages : 0); j < issued_k; ++j)
+        mbar_wait(&s.bar_k[j % kQKStages], (j / kQKStages) & 1, prm.status);
+      for (int j = (issued_v > kQVStages ? issued_v - kQVStages : 0); j < issued_v; ++j)
+        mbar_wait(&s.bar_v[j % kQVStages], (j / kQVStages) & 1, prm.status);
       mbar_wait(&s.bar_qdo, 0, prm.status);
     }
   } else if (warp == kVecWarps + 1) {
@@ -484,29 +501,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_s = idesc_bf16_f32(kT, BN, false, false);
       const uint32_t id_dq = idesc_bf16_f32(kT, kD, false, true);
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&s.bar_k[st], (j >> 1) & 1, prm.status)) return false;
+        const int st = j & 1, sk = j % kQKStages;
+        if (!mbar_wait(&s.bar_k[sk], (j / kQKStages) & 1, prm.status)) return false;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint64_t ad = sdesc_sw128(smem_u32(s.q[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.k[st][ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(s.k[sk][ks >> 2]) + (ks & 3) * 32, 0, 1024);
           mma_bf16_ss(tmem + (st ? kColS1 : kColS0), ad, bd, id_s, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_s_full[st]);
         return true;
       };
       auto issue_dp = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status)) return false;
+        const int sv = j % kQVStages;
+        if (!mbar_wait(&s.bar_v[sv], (j / kQVStages) & 1, prm.status)) return false;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint64_t ad = sdesc_sw128(smem_u32(s.dout[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.v[st][ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(s.v[sv][ks >> 2]) + (ks & 3) * 32, 0, 1024);
           mma_bf16_ss(tmem + kColDP, ad, bd, id_s, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_dp_full);
+        tc_commit(&s.bar_v_empty[sv]);
         return true;
       };
       bool ok = mbar_wait(&s.bar_qdo, 0, prm.status);
@@ -518,15 +536,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(&s.bar_ds_ready, j & 1, prm.status))) break;
         tc_fence_after();
         const uint32_t s_col = st ? kColS1 : kColS0;
+        const int sk = j % kQKStages;
 #pragma unroll
         for (int half = 0; half < 2; ++half)
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t bd = sdesc_sw128(smem_u32(s.k[st][0]) + ks * 2048, BN * 128, 1024);
+            const uint64_t bd = sdesc_sw128(smem_u32(s.k[sk][0]) + ks * 2048, BN * 128, 1024);
             mma_bf16_ts(tmem + kColDQ, tmem + s_col + half * (BN / 2) + ks * 8, bd, id_dq,
                         (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
           }
-        tc_commit(&s.bar_kv_empty[st]);
+        tc_commit(&s.bar_k_empty[sk]);
         if (j + 1 < n && !(ok = issue_dp(j + 1))) break;
       }
       if (ok) tc_commit(&s.bar_done);

@@ -7,13 +7,16 @@
 //   warps 0-7  softmax: warp w reads TMEM lane quarter w % 4 (query rows 32*(w%4) .. +31) and the
 //              column half w / 4 of each S tile, so each row is shared by two threads that
 //              exchange their partial row max through shared memory.  They mask, keep the
-//              running max/sum, rescale their half of O in TMEM when needed, and write P back
-//              over the consumed S columns as two bf16 parts (hi + lo, ~16 significant bits)
-//              that feed O += P V as the MMA's A operand.
-//   warp 8     TMA producer: Q once, then K/V tiles of the selected blocks into a 2-stage ring.
+//              running max/sum, rescale their half of O in TMEM when needed, and write P (bf16)
+//              back over the consumed S columns, where it feeds O += P V as the MMA's A operand.
+//   warp 8     TMA producer: Q once, then the K tiles of the selected blocks into a 3-stage ring
+//              and the V tiles into a 2-stage ring.  A K stage is released as soon as its
+//              S = Q K^T has run, a V stage after its O += P V, so the next loads start early.
 //   warp 9     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
-//              O += P_j,hi V_j + P_j,lo V_j into the TMEM O accumulator.  S_{j+1} is issued before
-//              waiting for P_j, so the tensor core computes the next scores while softmax runs.
+//              O += P_j V_j into the TMEM O accumulator.  S_{j+1} is issued before waiting for
+//              P_j, so the tensor core computes the next scores while softmax runs.
+// The row max is taken on the raw scores (scale > 0 is required by the host checks), so each
+// probability costs one fused multiply-add (packed in pairs) and one exp2.
 // Every wait is bounded (sa_common.cuh); on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -31,14 +34,16 @@ constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+constexpr int kKStages = 3, kVStages = 2;
+
 template <int BN>
 struct __align__(1024) FwdSmem {
-  uint8_t q[2][kBM * 128];        // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
-  uint8_t k[2][2][BN * 128];      // [stage][sub-tile] K rows of one KV block
-  uint8_t v[2][2][BN * 128];      // [stage][sub-tile] V rows
-  float red[2][2][kBM];           // [tile parity][column half][row]: partial row max / row sum
+  uint8_t q[2][kBM * 128];            // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
+  uint8_t k[kKStages][2][BN * 128];   // [stage][sub-tile] K rows of one KV block
+  uint8_t v[kVStages][2][BN * 128];   // [stage][sub-tile] V rows
+  float red[2][2][kBM];               // [tile parity][column half][row]: partial row max / row sum
   uint64_t bar_q;
-  uint64_t bar_k[2], bar_v[2], bar_kv_empty[2], bar_s_full[2];
+  uint64_t bar_k[kKStages], bar_k_empty[kKStages], bar_v[kVStages], bar_v_empty[kVStages], bar_s_full[2];
   uint64_t bar_p_full, bar_o_done;
   uint64_t bar_done;              // one phase: the last O += P V has completed
   uint64_t bar_pair[4];           // the two softmax warps of each TMEM lane quarter
@@ -91,12 +96,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&s.bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&s.bar_k[i], 1);
-      mbar_init(&s.bar_v[i], 1);
-      mbar_init(&s.bar_kv_empty[i], 1);
-      mbar_init(&s.bar_s_full[i], 1);
+      mbar_init(&s.bar_k_empty[i], 1);
     }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&s.bar_v[i], 1);
+      mbar_init(&s.bar_v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_s_full[i], 1);
     mbar_init(&s.bar_p_full, kSoftmaxWarps * 32);
     mbar_init(&s.bar_o_done, 1);
     mbar_init(&s.bar_done, 1);
@@ -121,24 +129,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&s.bar_q, 2 * kBM * 128);
       tma_load_2d(s.q[0], &tm_q, &s.bar_q, 0, q_row0);
       tma_load_2d(s.q[1], &tm_q, &s.bar_q, 64, q_row0);
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&s.bar_kv_empty[st], ((j - 2) >> 1) & 1, prm.status)) break;
+      // K runs up to kKStages tiles ahead, V up to kVStages; each waits only for its own stage.
+      int issued_k = 0, issued_v = 0;
+      bool ok = true;
+      for (int j = 0; ok && j < n; ++j) {
         const int row = kv_row0 + prm.col[rp + j] * prm.by;
-        mbar_arrive_expect_tx(&s.bar_k[st], 2 * BN * 128);
-        tma_load_2d(s.k[st][0], &tm_k, &s.bar_k[st], 0, row);
-        tma_load_2d(s.k[st][1], &tm_k, &s.bar_k[st], 64, row);
-        mbar_arrive_expect_tx(&s.bar_v[st], 2 * BN * 128);
-        tma_load_2d(s.v[st][0], &tm_v, &s.bar_v[st], 0, row);
-        tma_load_2d(s.v[st][1], &tm_v, &s.bar_v[st], 64, row);
-        issued = j + 1;
+        const int sk = j % kKStages, uk = j / kKStages;
+        if (j >= kKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
+        mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
+        tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
+        tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
+        issued_k = j + 1;
+        // V of tile j - (kKStages - kVStages) so that V trails K by one stage
+        const int jv = j - (kKStages - kVStages);
+        if (jv >= 0) {
+          const int sv = jv % kVStages, uv = jv / kVStages;
+          if (jv >= kVStages && !(ok = mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status))) break;
+          const int vrow = kv_row0 + prm.col[rp + jv] * prm.by;
+          mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
+          tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
+          tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
+          issued_v = jv + 1;
+        }
+      }
+      for (int jv = issued_v; ok && jv < n; ++jv) {
+        const int sv = jv % kVStages, uv = jv / kVStages;
+        if (jv >= kVStages && !(ok = mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status))) break;
+        const int vrow = kv_row0 + prm.col[rp + jv] * prm.by;
+        mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
+        tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
+        tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
+        issued_v = jv + 1;
       }
       // do not leave the CTA with copies in flight
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
-        mbar_wait(&s.bar_k[j & 1], (j >> 1) & 1, prm.status);
-        mbar_wait(&s.bar_v[j & 1], (j >> 1) & 1, prm.status);
-      }
+      for (int j = (issued_k > kKStages ? issued_k - kKStages : 0); j < issued_k; ++j)
+        mbar_wait(&s.bar_k[j % kKStages], (j / kKStages) & 1, prm.status);
+      for (int j = (issued_v > kVStages ? issued_v - kVStages : 0); j < issued_v; ++j)
+        mbar_wait(&s.bar_v[j % kVStages], (j / kVStages) & 1, prm.status);
       mbar_wait(&s.bar_q, 0, prm.status);
     }
   } else if (warp == kSoftmaxWarps + 1) {
@@ -147,17 +174,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
       const uint32_t idesc_o = idesc_bf16_f32(kBM, kD, false, true);
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&s.bar_k[st], (j >> 1) & 1, prm.status)) return false;
+        const int st = j & 1, sk = j % kKStages;
+        if (!mbar_wait(&s.bar_k[sk], (j / kKStages) & 1, prm.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + (st ? kColS1 : kColS0);
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint64_t ad = sdesc_sw128(smem_u32(s.q[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.k[st][ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(s.k[sk][ks >> 2]) + (ks & 3) * 32, 0, 1024);
           mma_bf16_ss(d, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_s_full[st]);
+        tc_commit(&s.bar_k_empty[sk]);
         return true;
       };
       bool ok = mbar_wait(&s.bar_q, 0, prm.status);
@@ -165,20 +193,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < n; ++j) {
         if (j + 1 < n && !(ok = issue_s(j + 1))) break;
         if (!(ok = mbar_wait(&s.bar_p_full, j & 1, prm.status))) break;
-        const int st = j & 1;
-        if (!(ok = mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status))) break;
+        const int st = j & 1, sv = j % kVStages;
+        if (!(ok = mbar_wait(&s.bar_v[sv], (j / kVStages) & 1, prm.status))) break;
         tc_fence_after();
         const uint32_t p_col = st ? kColS1 : kColS0;
 #pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t bd = sdesc_sw128(smem_u32(s.v[st][0]) + ks * 2048, BN * 128, 1024);
-            mma_bf16_ts(tmem + kColO, tmem + p_col + half * (BN / 2) + ks * 8, bd, idesc_o,
-                        (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
-          }
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint64_t bd = sdesc_sw128(smem_u32(s.v[sv][0]) + ks * 2048, BN * 128, 1024);
+          mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+        }
         tc_commit(&s.bar_o_done);
-        tc_commit(&s.bar_kv_empty[st]);
+        tc_commit(&s.bar_v_empty[sv]);
       }
       if (ok) tc_commit(&s.bar_done);
     }
@@ -208,14 +233,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t s_col = st ? kColS1 : kColS0;
       const int kpos0 = prm.col[rp + j] * prm.by + hf * kHalf;
-      float x[kHalf];
+      float x[kHalf];  // raw scores
 #pragma unroll
       for (int c = 0; c < kHalf; c += 32) {
         uint32_t rr[32];
         tmem_ld32(tmem + lane_base + s_col + hf * kHalf + c, rr);
         tmem_ld_wait(rr);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(rr[i]) * prm.scale_log2;
+        for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(rr[i]);
       }
       const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
       if (!full) {
@@ -225,15 +250,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kp < lo || kp > hi) x[c] = -INFINITY;
         }
       }
-      float mx = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kHalf; ++c) mx = fmaxf(mx, x[c]);
+      for (int c = 0; c < kHalf; c += 4) {
+        mx4[0] = fmaxf(mx4[0], x[c]);
+        mx4[1] = fmaxf(mx4[1], x[c + 1]);
+        mx4[2] = fmaxf(mx4[2], x[c + 2]);
+        mx4[3] = fmaxf(mx4[3], x[c + 3]);
+      }
+      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       // row max = max of the two halves; the barrier also orders both threads' S reads before
       // either writes P over the S columns
       s.red[st][hf][r] = mx;
       ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
       if (!ok) break;
-      mx = fmaxf(mx, s.red[st][hf ^ 1][r]);
+      mx = fmaxf(mx, s.red[st][hf ^ 1][r]) * prm.scale_log2;  // log2 units of the scaled score
       // Lazy rescaling: the exponent reference m only moves when the row max exceeds it by more
       // than 8 (p <= 2^8 otherwise); numerator and l share the same reference, so the final
       // O / l is unchanged.  Only then must the previous O += P V have landed.
@@ -264,23 +295,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
       }
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      float rowsum = 0.f;
+      // p = 2^(s * scale * log2(e) - m): one packed fma per pair, one exp2 per element
+      const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2), nm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc0 = 0, acc1 = 0;  // packed partial row sums (0 bits == 0.0f, 0.0f)
 #pragma unroll
       for (int c = 0; c < kHalf; c += 32) {
-        uint32_t hv[16], lv[16];
+        uint32_t hv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float e0 = ex2(x[c + 2 * i] - m_use), e1 = ex2(x[c + 2 * i + 1] - m_use);
-          rowsum += e0 + e1;
+          float t0, t1;
+          f2_unpack(f2_fma(f2_pack(x[c + 2 * i], x[c + 2 * i + 1]), sc2, nm2), t0, t1);
+          const float e0 = ex2(t0), e1 = ex2(t1);
+          if (i & 1) acc1 = f2_add(acc1, f2_pack(e0, e1));
+          else acc0 = f2_add(acc0, f2_pack(e0, e1));
           hv[i] = pack_bf16(e0, e1);
-          lv[i] = pack_bf16(e0 - bf16lo(hv[i]), e1 - bf16hi(hv[i]));
         }
-        // packed pairs: element column e -> column e/2 (hi) and BN/2 + e/2 (lo)
+        // packed pairs: element column e -> TMEM column e/2 of the S buffer
         tmem_st16(tmem + lane_base + s_col + (hf * kHalf + c) / 2, hv);
-        tmem_st16(tmem + lane_base + s_col + BN / 2 + (hf * kHalf + c) / 2, lv);
       }
       tmem_st_wait();
-      l += rowsum;
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       m = m_new;
       tc_fence_before();
       mbar_arrive(&s.bar_p_full);

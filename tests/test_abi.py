@@ -63,6 +63,7 @@ def test_bsa_host_validation():
     assert _ws("bsa_fwd_workspace_size", _bsa(mask_mode=1))[0] == sa.BSA_ERR_INVALID_ARG
     assert _ws("bsa_fwd_workspace_size", _bsa(S_q=0))[0] == sa.BSA_ERR_INVALID_ARG
     assert _ws("bsa_fwd_workspace_size", _bsa(scale=float("nan")))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws("bsa_fwd_workspace_size", _bsa(scale=-0.1))[0] == sa.BSA_ERR_INVALID_ARG
     L = sa.lib()
     assert L.bsa_fwd_workspace_size(None, None) == sa.BSA_ERR_NULLPTR
     # op call with NULL tensors fails validation before any launch
