@@ -241,6 +241,53 @@ def plan_array(plan, layout: MetaLayout, index: int, count: int, dtype=torch.int
     return plan[off:off + count * itemsize].view(dtype)
 
 
+# ---------------------------------------------------------------------------------------------
+# SFA: sparse decode over a paged KV cache
+# ---------------------------------------------------------------------------------------------
+def sfa_params(q, k_cache, block_table, sparse_indices, seqused_kv, sparse_block_size, scale=None) -> Params:
+    """q [B, 1, N1, 512]; caches [num_pages, page_size, N2, D]; block_table [B, max_pages];
+    sparse_indices [B, 1, N2, K] int32; seqused_kv [B] int32 (all device tensors)."""
+    B, Sq, N1, D = q.shape
+    num_pages, page_size, N2, _ = k_cache.shape
+    p = Params()
+    p.q_layout = LAYOUT_BSND
+    p.kv_layout = LAYOUT_PA_ND
+    p.B, p.N1, p.N2, p.S_q = B, N1, N2, Sq
+    p.D, p.Dv, p.D_rope = D, D, 64
+    p.seqused_kv = seqused_kv.data_ptr()
+    p.page_size, p.max_pages_per_seq, p.num_pages = page_size, block_table.shape[1], num_pages
+    p.block_table = block_table.data_ptr()
+    p.sparse_block_size, p.sparse_count = sparse_block_size, sparse_indices.shape[-1]
+    p.sparse_indices = sparse_indices.data_ptr()
+    p.mask_mode = MASK_NONE
+    p.scale = 1.0 / math.sqrt(D + 64) if scale is None else scale
+    return p
+
+
+def sfa_sparse_decode_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check("sfa_sparse_decode_workspace_size", lib().sfa_sparse_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def sfa_sparse_decode(q, q_rope, k_cache, k_rope_cache, v_cache, block_table, sparse_indices, seqused_kv,
+                      sparse_block_size, scale=None, out=None, lse=None, workspace=None, stream=None):
+    """Out [B, 1, N1, 512] bf16, LSE [B, 1, N1] fp32 of sparse decode attention."""
+    _need_cuda(q, q_rope, k_cache, k_rope_cache, v_cache, block_table, sparse_indices, seqused_kv)
+    p = sfa_params(q, k_cache, block_table, sparse_indices, seqused_kv, sparse_block_size, scale)
+    B, Sq, N1, D = q.shape
+    if out is None:
+        out = torch.empty(B, Sq, N1, v_cache.shape[-1], dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, Sq, N1, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(sfa_sparse_decode_workspace_size(p), q.device)
+    _check("sfa_sparse_decode", lib().sfa_sparse_decode(ctypes.byref(p), _ptr(q), _ptr(q_rope), _ptr(k_cache),
+                                                        _ptr(k_rope_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                                        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
 def bsa_get_status(workspace, stream=None) -> int:
     v = ctypes.c_uint32()
     _check("bsa_get_status", lib().bsa_get_status(_ptr(workspace), _stream(stream), ctypes.byref(v)))

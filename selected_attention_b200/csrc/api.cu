@@ -79,6 +79,63 @@ size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
   return c.bytes();
 }
 
+// ---- SFA (SparseFlashAttention page constraints) ----------------------------------------------------
+// "D in query, key and value is 512; Dr of query_rope and key_rope is 64"; "block_size must be a
+// multiple of 16, at most 1024" (this library's 32-token tiles need a multiple of 32);
+// "sparse_block_size must be exactly divisible by block_size"; decode: one query row per batch.
+bsa_status check_sfa(const bsa_params* p) {
+  if (!p) return BSA_ERR_NULLPTR;
+  if (p->kv_layout != BSA_LAYOUT_PA_ND) return BSA_ERR_UNSUPPORTED;
+  if (p->B <= 0 || p->N1 <= 0 || p->N2 <= 0) return BSA_ERR_INVALID_ARG;
+  if (p->N1 < p->N2 || p->N1 % p->N2 != 0) return BSA_ERR_INVALID_ARG;
+  if (p->N1 / p->N2 > 128) return BSA_ERR_UNSUPPORTED;
+  if (p->S_q != 1) return BSA_ERR_UNSUPPORTED;
+  if (p->D != 512 || p->Dv != 512 || p->D_rope != 64) return BSA_ERR_UNSUPPORTED;
+  if (p->page_size <= 0 || p->page_size % 16 != 0 || p->page_size > 1024) return BSA_ERR_INVALID_ARG;
+  if (p->page_size % 32 != 0) return BSA_ERR_UNSUPPORTED;
+  if (p->sparse_block_size <= 0 || p->sparse_block_size % p->page_size != 0) return BSA_ERR_INVALID_ARG;
+  if (p->sparse_count <= 0 || p->max_pages_per_seq <= 0 || p->num_pages <= 0) return BSA_ERR_INVALID_ARG;
+  if (1LL * p->num_pages * p->page_size * p->N2 >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  if (!std::isfinite(p->scale) || p->scale <= 0.f) return BSA_ERR_INVALID_ARG;
+  return BSA_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+struct SfaWs {
+  uint32_t* status;
+  int32_t *pages, *tokens, *count, *piece_unit, *piece_begin, *piece_len, *unit_first, *unit_pieces, *n_pieces;
+  float *part_o, *part_m, *part_l;
+  int cap, units, max_pieces;
+};
+
+size_t carve_sfa(const bsa_params* p, void* ws, SfaWs* w) {
+  Carver c(ws);
+  const int ppb = p->sparse_block_size / p->page_size;
+  w->cap = p->sparse_count * ppb;
+  w->units = p->B * p->N2 * 2;
+  w->max_pieces = sm_count() + w->units;
+  const size_t lists = static_cast<size_t>(p->B) * p->N2 * w->cap;
+  w->status = static_cast<uint32_t*>(ws);
+  w->pages = c.take<int32_t>(lists);
+  w->tokens = c.take<int32_t>(lists);
+  w->count = c.take<int32_t>(static_cast<size_t>(p->B) * p->N2);
+  w->piece_unit = c.take<int32_t>(w->max_pieces);
+  w->piece_begin = c.take<int32_t>(w->max_pieces);
+  w->piece_len = c.take<int32_t>(w->max_pieces);
+  w->unit_first = c.take<int32_t>(w->units);
+  w->unit_pieces = c.take<int32_t>(w->units);
+  w->n_pieces = c.take<int32_t>(1);
+  w->part_o = c.take<float>(static_cast<size_t>(w->max_pieces) * 128 * 256);
+  w->part_m = c.take<float>(static_cast<size_t>(w->max_pieces) * 128);
+  w->part_l = c.take<float>(static_cast<size_t>(w->max_pieces) * 128);
+  return c.bytes();
+}
+
 bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
 bsa_status check_ws(void* ws, size_t have, size_t need) {
@@ -170,10 +227,47 @@ bsa_status nsa_selected_bwd(const bsa_params*, const void*, const void*, const v
                             const float*, void*, void*, void*, void*, size_t, void*) {
   return BSA_ERR_UNSUPPORTED;
 }
-bsa_status sfa_sparse_decode_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
-bsa_status sfa_sparse_decode(const bsa_params*, const void*, const void*, const void*, const void*, const void*,
-                             void*, float*, void*, size_t, void*) {
-  return BSA_ERR_UNSUPPORTED;
+bsa_status sfa_sparse_decode_workspace_size(const bsa_params* p, size_t* bytes) {
+  if (!bytes) return BSA_ERR_NULLPTR;
+  bsa_status s = check_sfa(p);
+  if (s != BSA_OK) return s;
+  SfaWs w;
+  *bytes = carve_sfa(p, nullptr, &w);
+  return BSA_OK;
+}
+
+bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_rope, const void* k_cache,
+                             const void* k_rope_cache, const void* v_cache, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  bsa_status s = check_sfa(p);
+  if (s != BSA_OK) return s;
+  if (!q || !q_rope || !k_cache || !k_rope_cache || !v_cache || !out || !lse || !p->block_table ||
+      !p->sparse_indices || !p->seqused_kv)
+    return BSA_ERR_NULLPTR;
+  SfaWs w;
+  const size_t need = carve_sfa(p, nullptr, &w);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != BSA_OK) return s;
+  carve_sfa(p, workspace, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  SfaMetaArgs m;
+  m.sparse_indices = p->sparse_indices; m.block_table = p->block_table; m.seqused_kv = p->seqused_kv;
+  m.B = p->B; m.N2 = p->N2; m.K = p->sparse_count; m.ppb = p->sparse_block_size / p->page_size;
+  m.page_size = p->page_size; m.max_pages_per_seq = p->max_pages_per_seq; m.num_pages = p->num_pages;
+  m.pages = w.pages; m.tokens = w.tokens; m.count = w.count; m.status = w.status;
+  if ((e = sfa_page_list(m, st)) != cudaSuccess) return BSA_ERR_CUDA;
+  if ((e = sfa_work_list(w.count, w.units, w.max_pieces - w.units, w.piece_unit, w.piece_begin, w.piece_len,
+                         w.unit_first, w.unit_pieces, w.n_pieces, st)) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  SfaDecodeArgs a;
+  a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.page_size = p->page_size; a.num_pages = p->num_pages;
+  a.cap = w.cap; a.units = w.units; a.max_pieces = w.max_pieces; a.scale = p->scale;
+  a.q = q; a.q_rope = q_rope; a.k_cache = k_cache; a.k_rope_cache = k_rope_cache; a.v_cache = v_cache;
+  a.pages = w.pages; a.tokens = w.tokens; a.piece_unit = w.piece_unit; a.piece_begin = w.piece_begin;
+  a.piece_len = w.piece_len; a.unit_first = w.unit_first; a.unit_pieces = w.unit_pieces; a.n_pieces = w.n_pieces;
+  a.out = out; a.lse = lse; a.part_o = w.part_o; a.part_m = w.part_m; a.part_l = w.part_l; a.status = w.status;
+  return cuda_status(sfa_decode_launch(a, st));
 }
 
 // ---- metadata -------------------------------------------------------------------------------------
@@ -207,6 +301,25 @@ bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta
     layout->total_bytes = c.bytes();
     return BSA_OK;
   }
+  if (op == BSA_META_SFA_PAGES) {
+    bsa_status s = check_sfa(p);
+    if (s != BSA_OK) return s;
+    const size_t lists = static_cast<size_t>(p->B) * p->N2 * p->sparse_count * (p->sparse_block_size / p->page_size);
+    Carver c(nullptr);
+    layout->offsets[0] = 0;
+    c.off = align_up(c.off, 256);
+    layout->offsets[1] = c.off;  // pages [B*N2][cap], compacted
+    c.take<int32_t>(lists);
+    c.off = align_up(c.off, 256);
+    layout->offsets[2] = c.off;  // tokens [B*N2][cap]
+    c.take<int32_t>(lists);
+    c.off = align_up(c.off, 256);
+    layout->offsets[3] = c.off;  // count [B*N2]
+    c.take<int32_t>(static_cast<size_t>(p->B) * p->N2);
+    layout->count = 4;
+    layout->total_bytes = c.bytes();
+    return BSA_OK;
+  }
   return BSA_ERR_UNSUPPORTED;
 }
 
@@ -215,9 +328,22 @@ bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, siz
   bsa_status s = sparse_attn_metadata_layout(p, op, &L);
   if (s != BSA_OK) return s;
   if ((s = check_ws(plan, plan_bytes, L.total_bytes)) != BSA_OK) return s;
-  if (!p->block_mask) return BSA_ERR_NULLPTR;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(plan);
+  if (op == BSA_META_SFA_PAGES) {
+    if (!p->block_table || !p->sparse_indices || !p->seqused_kv) return BSA_ERR_NULLPTR;
+    if (cudaMemsetAsync(plan, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+    SfaMetaArgs m;
+    m.sparse_indices = p->sparse_indices; m.block_table = p->block_table; m.seqused_kv = p->seqused_kv;
+    m.B = p->B; m.N2 = p->N2; m.K = p->sparse_count; m.ppb = p->sparse_block_size / p->page_size;
+    m.page_size = p->page_size; m.max_pages_per_seq = p->max_pages_per_seq; m.num_pages = p->num_pages;
+    m.pages = reinterpret_cast<int32_t*>(base + L.offsets[1]);
+    m.tokens = reinterpret_cast<int32_t*>(base + L.offsets[2]);
+    m.count = reinterpret_cast<int32_t*>(base + L.offsets[3]);
+    m.status = static_cast<uint32_t*>(plan);
+    return cuda_status(sfa_page_list(m, st));
+  }
+  if (!p->block_mask) return BSA_ERR_NULLPTR;
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
   cudaError_t e = cudaMemsetAsync(plan, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return BSA_ERR_CUDA;

@@ -81,6 +81,33 @@ struct BsaBwdArgs {
 cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, const void* v, const void* out,
                            const void* dout, const float* lse, cudaStream_t st);
 
+// ---- sparse decode (sfa_meta.cu, sfa_decode.cu) ------------------------------------------------
+struct SfaMetaArgs {
+  const int32_t* sparse_indices;  // [B, 1, N2, K] (row 0 used)
+  const int32_t* block_table;     // [B, max_pages_per_seq]
+  const int32_t* seqused_kv;      // [B]
+  int B, N2, K, ppb, page_size, max_pages_per_seq, num_pages;
+  int32_t* pages;   // [B*N2][K*ppb] compacted physical pages
+  int32_t* tokens;  // valid tokens of each listed page
+  int32_t* count;   // [B*N2]
+  uint32_t* status;
+};
+cudaError_t sfa_page_list(const SfaMetaArgs& a, cudaStream_t st);
+cudaError_t sfa_work_list(const int32_t* count, int units, int G, int32_t* piece_unit, int32_t* piece_begin,
+                          int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces, int32_t* n_pieces,
+                          cudaStream_t st);
+struct SfaDecodeArgs {
+  int B, N1, N2, page_size, num_pages, cap, units, max_pieces;
+  float scale;
+  const void *q, *q_rope, *k_cache, *k_rope_cache, *v_cache;
+  const int32_t *pages, *tokens, *piece_unit, *piece_begin, *piece_len, *unit_first, *unit_pieces, *n_pieces;
+  void* out;
+  float* lse;
+  float *part_o, *part_m, *part_l;
+  uint32_t* status;
+};
+cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st);
+
 // ---- diagnostics (diag.cu) -----------------------------------------------------------------------
 cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,
                                  cudaStream_t st);

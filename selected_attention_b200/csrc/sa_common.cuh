@@ -258,6 +258,7 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) reg_fence(r[i]);
 }
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Byte offset of element (row, col) inside a [rows][64] bf16 tile stored with the 128-byte
