@@ -362,41 +362,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the pieces of each unit in piece order:  M = max m_p, L = sum l_p 2^(m_p - M),
-// Out = sum O_p 2^(m_p - M) / L,  LSE = (M + log2 L) ln 2.
+// Out = sum O_p 2^(m_p - M) / L,  LSE = (M + log2 L) ln 2.  One warp per (unit, head row); each
+// lane owns 8 of the 256 Dv columns, so every partial row is read with coalesced 16-byte loads.
 __global__ void __launch_bounds__(256) sfa_combine_kernel(const DecParams prm, const int32_t* __restrict__ unit_first) {
   const int u = blockIdx.x;
+  const int r = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= prm.G) return;
   const int pcs = prm.unit_pieces[u];
   if (pcs == 1) return;  // written by its single piece
   const int bg = u >> 1, dvh = u & 1;
   const int b = bg / prm.N2, g = bg % prm.N2;
   const int p0 = unit_first[u];
-  const int qrow0 = b * prm.N1 + g * prm.G;
-  if (pcs == 0) {  // no selected key: Out = 0, LSE = -inf
-    for (int r = 0; r < prm.G; ++r) {
-      prm.out[static_cast<size_t>(qrow0 + r) * kDQ + dvh * kDVH + threadIdx.x] = __float2bfloat16_rn(0.f);
-      if (threadIdx.x == 0 && dvh == 0) prm.lse[qrow0 + r] = -INFINITY;
-    }
-    return;
+  const size_t orow = static_cast<size_t>(b * prm.N1 + g * prm.G + r);
+  __nv_bfloat16* dst = prm.out + orow * kDQ + dvh * kDVH + lane * 8;
+  float M = -INFINITY;
+  for (int p = 0; p < pcs; ++p) M = fmaxf(M, prm.part_m[static_cast<size_t>(p0 + p) * kM + r]);
+  float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int p = 0; p < pcs; ++p) {
+    const float mp = prm.part_m[static_cast<size_t>(p0 + p) * kM + r];
+    if (mp == -INFINITY) continue;
+    const float wgt = ex2(mp - M);
+    L += prm.part_l[static_cast<size_t>(p0 + p) * kM + r] * wgt;
+    const float4* src = reinterpret_cast<const float4*>(prm.part_o + (static_cast<size_t>(p0 + p) * kM + r) * kDVH +
+                                                        lane * 8);
+    const float4 a = src[0], c = src[1];
+    acc[0] += a.x * wgt; acc[1] += a.y * wgt; acc[2] += a.z * wgt; acc[3] += a.w * wgt;
+    acc[4] += c.x * wgt; acc[5] += c.y * wgt; acc[6] += c.z * wgt; acc[7] += c.w * wgt;
   }
-  for (int r = 0; r < prm.G; ++r) {
-    float M = -INFINITY;
-    for (int p = 0; p < pcs; ++p) M = fmaxf(M, prm.part_m[static_cast<size_t>(p0 + p) * kM + r]);
-    float L = 0.f;
-    for (int p = 0; p < pcs; ++p) {
-      const float mp = prm.part_m[static_cast<size_t>(p0 + p) * kM + r];
-      if (mp != -INFINITY) L += prm.part_l[static_cast<size_t>(p0 + p) * kM + r] * ex2(mp - M);
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    const int d = threadIdx.x;  // 256 threads = the Dv half
-    float acc = 0.f;
-    for (int p = 0; p < pcs; ++p) {
-      const float mp = prm.part_m[static_cast<size_t>(p0 + p) * kM + r];
-      if (mp == -INFINITY) continue;
-      acc += prm.part_o[(static_cast<size_t>(p0 + p) * kM + r) * kDVH + d] * ex2(mp - M);
-    }
-    prm.out[static_cast<size_t>(qrow0 + r) * kDQ + dvh * kDVH + d] = __float2bfloat16_rn(acc * inv);
-    if (d == 0 && dvh == 0) prm.lse[qrow0 + r] = L > 0.f ? (M * kLn2 + logf(L)) : -INFINITY;
-  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;  // pcs == 0 (no selected key): Out = 0, LSE = -inf
+  uint4 pk;
+  pk.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+  pk.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+  pk.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(dst) = pk;
+  if (lane == 0 && dvh == 0) prm.lse[orow] = L > 0.f ? (M * kLn2 + logf(L)) : -INFINITY;
 }
 
 }  // namespace
@@ -426,7 +427,7 @@ cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st) {
   prof_end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prof_begin("sfa_combine", st);
-  sfa_combine_kernel<<<a.units, kDVH, 0, st>>>(p, a.unit_first);
+  sfa_combine_kernel<<<dim3(a.units, (p.G + 7) / 8), 256, 0, st>>>(p, a.unit_first);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -17,12 +17,15 @@
 namespace sa {
 namespace {
 
+// One warp per (b, g): each lane takes a slot of the sparse-index row, counts its valid pages,
+// and a warp scan places them, so the compacted list keeps the row's order.
 __global__ void sfa_page_list_kernel(const int32_t* __restrict__ sparse_indices, const int32_t* __restrict__ block_table,
                                      const int32_t* __restrict__ seqused_kv, int B, int N2, int K, int ppb,
                                      int page_size, int max_pages_per_seq, int num_pages, int32_t* __restrict__ pages,
                                      int32_t* __restrict__ tokens, int32_t* __restrict__ count,
                                      uint32_t* __restrict__ status) {
-  const int bg = blockIdx.x * blockDim.x + threadIdx.x;  // one thread per (b, g): lists are short
+  const int bg = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (bg >= B * N2) return;
   const int b = bg / N2;
   const int used = seqused_kv[b];
@@ -30,25 +33,41 @@ __global__ void sfa_page_list_kernel(const int32_t* __restrict__ sparse_indices,
   const int n_sb = used > 0 ? (used + sbs - 1) / sbs : 0;
   const int32_t* idx = sparse_indices + static_cast<size_t>(bg) * K;  // row 0 of Sq
   const int cap = K * ppb;
-  int n = 0;
+  int base = 0;
   uint32_t bad = 0;
-  for (int i = 0; i < K; ++i) {
-    const int j = idx[i];
-    if (j < 0) continue;
-    if (j >= n_sb) { bad |= SA_DEV_BAD_INDEX; continue; }
-    for (int p = 0; p < ppb; ++p) {
-      const int lp = j * ppb + p;
-      const int t0 = lp * page_size;
-      if (t0 >= used) break;
-      const int phys = (lp < max_pages_per_seq) ? block_table[static_cast<size_t>(b) * max_pages_per_seq + lp] : -1;
-      if (phys < 0 || phys >= num_pages) { bad |= SA_DEV_BAD_INDEX; continue; }
-      pages[static_cast<size_t>(bg) * cap + n] = phys;
-      tokens[static_cast<size_t>(bg) * cap + n] = min(page_size, used - t0);
-      ++n;
+  for (int s0 = 0; s0 < K; s0 += 32) {
+    const int i = s0 + lane;
+    const int j = i < K ? idx[i] : -1;
+    // valid pages of this slot: logical pages j*ppb .. j*ppb+ppb-1 that start below `used`
+    int nvalid = 0;
+    if (j >= n_sb) bad |= SA_DEV_BAD_INDEX;
+    if (j >= 0 && j < n_sb) {
+      for (int p = 0; p < ppb; ++p) {
+        const int lp = j * ppb + p;
+        if (lp * page_size >= used) break;
+        const int phys = lp < max_pages_per_seq ? block_table[static_cast<size_t>(b) * max_pages_per_seq + lp] : -1;
+        if (phys < 0 || phys >= num_pages) { bad |= SA_DEV_BAD_INDEX; break; }
+        ++nvalid;
+      }
     }
+    int incl = nvalid;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = base + incl - nvalid;
+    for (int p = 0; p < nvalid; ++p) {
+      const int lp = j * ppb + p;
+      pages[static_cast<size_t>(bg) * cap + pos] = block_table[static_cast<size_t>(b) * max_pages_per_seq + lp];
+      tokens[static_cast<size_t>(bg) * cap + pos] = min(page_size, used - lp * page_size);
+      ++pos;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  count[bg] = n;
-  if (bad) raise_status(status, bad);
+  if (lane == 0) count[bg] = base;
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  if (lane == 0 && bad) raise_status(status, bad);
 }
 
 // One CTA: choose the piece size and lay out the pieces.
@@ -127,7 +146,7 @@ cudaError_t sfa_page_list(const SfaMetaArgs& a, cudaStream_t st) {
   const int n = a.B * a.N2;
   if (n == 0) return cudaSuccess;
   prof_begin("sfa_page_list", st);
-  sfa_page_list_kernel<<<(n + 127) / 128, 128, 0, st>>>(a.sparse_indices, a.block_table, a.seqused_kv, a.B, a.N2,
+  sfa_page_list_kernel<<<(n + 3) / 4, 128, 0, st>>>(a.sparse_indices, a.block_table, a.seqused_kv, a.B, a.N2,
                                                         a.K, a.ppb, a.page_size, a.max_pages_per_seq, a.num_pages,
                                                         a.pages, a.tokens, a.count, a.status);
   prof_end(st);
