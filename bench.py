@@ -9,7 +9,11 @@ and a causal Bernoulli(0.25) BlockSparseMask (synthetic, seeded).
 The metric is effective TFLOP/s: credited FLOPs / time, with forward 4*D*V and backward
 10*D*V for V visible (query, key) pairs (the diagonal block counts only its visible half).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1|2|5]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1|2|3|4|5]
+
+--config 3 runs the NSA selected-attention workload (TND, 4 batches of 4096..32768 tokens, GQA
+64/4, 16 blocks of 64 tokens per token) forward + backward under the same metric; --config 4
+runs the paged sparse decode workload (gathered-KV bandwidth).
 
 With N > 1 (launched by torchrun, one process per GPU) every rank runs its own copy of the
 workload (independent batches: weak scaling, no collective on the data path); time is the max
@@ -155,6 +159,62 @@ def cpu_oracle_sample(w, mask, budget_s: float):
     return flops, dt, f"oracle fwd+bwd on all {len(heads)} (b,h) head slices"
 
 
+def visible_pairs_nsa(w, topk: np.ndarray) -> int:
+    """(token, query head, key) triples the NSA mask keeps: per listed block id j (duplicates
+    counted), keys j*bs .. min((j+1)*bs, len) - 1, and under the causal mask only keys <= pos."""
+    total = 0
+    cu = w.cu_seqlens()
+    for b in range(w.B):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        pos = np.arange(t1 - t0)[:, None, None]
+        ids = topk[t0:t1].astype(np.int64)
+        hi = np.minimum((ids + 1) * w.sel_block, t1 - t0)
+        if w.mask_mode == 2:
+            hi = np.minimum(hi, pos + 1)
+        n = np.clip(hi - ids * w.sel_block, 0, None)
+        total += int(np.where(ids >= 0, n, 0).sum())
+    return total * (w.N1 // w.N2)
+
+
+def cpu_oracle_sample_nsa(w, topk, budget_s: float, chunk: int = 32):
+    """Time the fp64 oracle (forward + backward) on chunks of `chunk` tokens of each (b, kv head)
+    slice, round robin over the slices, until budget_s has passed."""
+    from oracle import attention as A
+    cu = w.cu_seqlens()
+    G = w.N1 // w.N2
+    f = A.bf16_to_f64
+    flops, done, t_start = 0, [], time.perf_counter()
+    slices = {}
+    for b in range(w.B):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        q, do = w.tensor("q", t0, t1), w.tensor("dout", t0, t1)
+        k, v = w.tensor("k", t0, t1), w.tensor("v", t0, t1)
+        for g in range(w.N2):
+            hs = slice(g * G, (g + 1) * G)
+            slices[(b, g)] = (f(q[:, hs]), f(k[:, g]), f(v[:, g]), topk[t0:t1, g], f(do[:, hs]), t1 - t0)
+        if b == 0:  # the first batch's slices are enough for a bounded sample
+            break
+    t_start = time.perf_counter()
+    rnd = 0
+    while True:
+        for (b, g), (q, k, v, tk, do, S) in slices.items():
+            toks = list(range(rnd * chunk, min(S, (rnd + 1) * chunk)))
+            A.nsa_slice(q, k, v, tk, w.sel_block, w.mask_mode, w.scale, dout_g=do, tokens=toks, out_storage="bf16")
+            sub = tk[toks]
+            pos = np.asarray(toks)[:, None]
+            hi = np.minimum((sub.astype(np.int64) + 1) * w.sel_block, S)
+            if w.mask_mode == 2:
+                hi = np.minimum(hi, pos + 1)
+            vis = int(np.where(sub >= 0, np.clip(hi - sub.astype(np.int64) * w.sel_block, 0, None), 0).sum())
+            flops += 14 * w.D * vis * G
+            done.append((b, g, len(toks)))
+            if time.perf_counter() - t_start >= budget_s:
+                n = sum(x[2] for x in done)
+                return flops, time.perf_counter() - t_start, \
+                    f"oracle fwd+bwd on {n} (token, kv head) rows of batch 0 ({chunk}-token chunks)"
+        rnd += 1
+
+
 def cpu_threads():
     try:
         import threadpoolctl
@@ -169,14 +229,21 @@ def run_reference(args, rank, world):
     """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
     if rank != 0:
         return
-    w = bsa_workload(args.config)
-    mask = w.block_mask()
+    w = synth.workload(args.config)
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; warm-up steps are a no-op
     total_f, total_t, desc = 0, 0.0, ""
     step_budget = min(args.ref_step_seconds, 150.0 / max(1, args.steps))  # whole run ~2.5 min at most
+    if isinstance(w, synth.NsaWorkload):
+        topk = w.topk()
+        sample = lambda: cpu_oracle_sample_nsa(w, topk, budget_s=step_budget)  # noqa: E731
+        cfg = config_dict_nsa(w, args)
+    else:
+        mask = w.block_mask()
+        sample = lambda: cpu_oracle_sample(w, mask, budget_s=step_budget)  # noqa: E731
+        cfg = config_dict(w, args)
     for _ in range(args.steps):
-        f, t, desc = cpu_oracle_sample(w, mask, budget_s=step_budget)
+        f, t, desc = sample()
         total_f += f
         total_t += t
     value = total_f / total_t / 1e12
@@ -184,7 +251,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(w, args),
+        "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"each step: {desc}"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -201,6 +268,145 @@ def config_dict(w, args):
         else "inputs fit in L2 (small parity workload)",
         "parallelism": f"replicas x{args.gpus} (independent batches)",
     }
+
+
+def config_dict_nsa(w, args):
+    return {
+        "workload": f"{w.name}: NSA selected attention fwd+bwd, TND seqlens={w.seqlens} (T={w.T}), N1={w.N1} "
+                    f"N2={w.N2} D={w.D}, {w.sel_count} blocks of {w.sel_block} per (token, kv head), causal",
+        "T": w.T, "N1": w.N1, "N2": w.N2, "D": w.D, "sel_block": w.sel_block, "sel_count": w.sel_count,
+        "seed": w.seed, "l2": "no flush: inputs (Q, dOut 1 GiB each) exceed the 126 MB L2",
+        "parallelism": f"replicas x{args.gpus} (independent batches)",
+    }
+
+
+def _dist_helpers(world, dev):
+    import torch
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x):
+        if world > 1:
+            t = torch.tensor([x], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            return float(t.item())
+        return x
+    return barrier, max_over_ranks
+
+
+def run_nsa(args, rank, world, local_rank):
+    """NSA selected attention (TND varlen, GQA) forward + backward: one step = metadata + forward
+    + backward over the whole 61440-token batch."""
+    import torch
+
+    import selected_attention_b200 as sa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.workload(3)
+    topk = w.topk()
+    cu = w.cu_seqlens()
+    vpairs = visible_pairs_nsa(w, topk)
+    flops_step = 14 * w.D * vpairs
+    S = max(w.seqlens)
+    host = {t: torch.from_numpy(w.tensor(t)).view(torch.bfloat16) for t in ("q", "k", "v", "dout")}
+    host["topk"], host["cu"] = torch.from_numpy(topk), torch.from_numpy(cu)
+    d = {t: x.to(dev) for t, x in host.items()}
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(w.T, w.N1, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+    p = sa.nsa_params(d["q"], d["k"], d["topk"], d["cu"], S, w.sel_block, w.mask_mode, w.scale)
+    ws_f = torch.empty(sa.nsa_selected_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(sa.nsa_selected_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    barrier, max_over_ranks = _dist_helpers(world, dev)
+
+    def step(x=d):
+        sa.nsa_selected_fwd(x["q"], x["k"], x["v"], x["topk"], x["cu"], S, w.sel_block, w.mask_mode, w.scale,
+                            out=out, lse=lse, workspace=ws_f)
+        sa.nsa_selected_bwd(x["q"], x["k"], x["v"], out, x["dout"], lse, x["topk"], x["cu"], S, w.sel_block,
+                            w.mask_mode, w.scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert sa.bsa_get_status(ws_f) == 0 and sa.bsa_get_status(ws_b) == 0, "device status bits set"
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        sa.bsa_profile_enable(True)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        prof = sa.bsa_profile_collect()
+        sa.bsa_profile_enable(False)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
+    value = world * flops_step / (ms * 1e-3) / 1e12
+
+    # end to end: pinned host inputs in, all outputs back, every step
+    pin = {t: x.pin_memory() for t, x in host.items()}
+    outs = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    h_out = {n_: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n_, x in outs.items()}
+    d_in = {t: torch.empty_like(x) for t, x in d.items()}
+    h2d = sum(x.numel() * x.element_size() for x in pin.values())
+    d2h = sum(x.numel() * x.element_size() for x in h_out.values())
+
+    def e2e_step():
+        for t in d_in:
+            d_in[t].copy_(pin[t], non_blocking=True)
+        step(d_in)
+        for n_, x in outs.items():
+            h_out[n_].copy_(x, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    peaks, peak_src = measured_peaks()
+    # forward 4*D per visible pair; dK/dV pass 8*D (S^T, dP^T, dV, dK); dQ pass 6*D (S, dP, dQ)
+    alg = {"nsa_fwd": 4 * w.D * vpairs, "nsa_bwd_dkdv": 8 * w.D * vpairs, "nsa_bwd_dq": 6 * w.D * vpairs}
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roof = None
+    if dom in alg:
+        launches, total = prof[dom]
+        avg_ms = total / launches
+        achieved = alg[dom] / (avg_ms * 1e-3) / 1e12
+        tr = NCU_TRAFFIC.get(dom)
+        traffic = tr["bytes"] if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) else None
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic, "avg_launch_ms": avg_ms}
+    kernels = {n_: {"launches": c, "ms_per_step": t / args.steps} for n_, (c, t) in prof.items()}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, t, desc = cpu_oracle_sample_nsa(w, topk, budget_s=args.cpu_seconds)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps({
+            "metric": "effective NSA selected attn fwd+bwd TFLOP/s (bf16)", "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_dict_nsa(w, args),
+            "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": sum(c for c, _ in prof.values()), "kernels": kernels, "roofline": roof,
+            "cpu_baseline": cpu, "clocks": clocks.summary(), "visible_pairs": vpairs,
+            "credited_flops_per_step": flops_step,
+        }))
 
 
 def run_decode(args, rank, world, local_rank):
@@ -426,7 +632,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 4, 5])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -451,6 +657,8 @@ def main():
     try:
         if args.config == 4:
             run_decode(args, rank, world, local_rank)
+        elif args.config == 3:
+            run_nsa(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)
     finally:

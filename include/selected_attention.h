@@ -130,7 +130,25 @@ BSA_API bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, co
                    const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
                    size_t workspace_bytes, void* stream);
 
-/* ---- NSA selected attention (NsaSelectedAttention page), TND, GQA, D = Dv = 128 ----------- */
+/* ---- NSA selected attention (NsaSelectedAttention page), TND, GQA, D = Dv = 128 -----------
+ * Forward formula of the page: for token t and kv head g, selected_key/value = Gather(key/value,
+ * topk_indices[t, g, i]) for the listed blocks; Out = softmax(Mask(scale q K_sel^T)) V_sel for
+ * each of the group's G = N1/N2 query heads (heads g*G .. g*G+G-1); LSE per (t, head).
+ *   p->q_layout = p->kv_layout = BSA_LAYOUT_TND; q/out/dout/dq [T, N1, 128], k/v/dk/dv
+ *   [T, N2, 128], lse [T, N1]; T_q = T_kv = T; cu_seqlens_q (= cu_seqlens_kv) [B+1] device int32
+ *   with per-batch lengths (query and key lengths equal); S_q = the longest batch's length.
+ *   topk_indices [T, N2, sel_block_count] int32: block ids of sel_block_size tokens, counted
+ *   from the batch's first token; -1 = empty slot; a duplicated id is gathered twice.
+ *   mask_mode BSA_MASK_NONE or BSA_MASK_CAUSAL (key position <= query position in the batch).
+ *   Host errors (INVALID_ARG / UNSUPPORTED): sel_block_size not a multiple of 16 in [16, 128],
+ *   sel_block_count not in [1, 128] or count * size > 8192, N1 % N2 != 0, N2 > 32, N1 > 128,
+ *   D != 128, S_q > 128K, T_q != T_kv, scale <= 0.
+ *   Device status bits: SA_DEV_BAD_INDEX for an id at or past the batch's block count (the id
+ *   is skipped); SA_DEV_BAD_SEQLEN if cu_seqlens is not a non-decreasing 0..T sequence or a
+ *   batch is longer than S_q (nothing is computed).
+ *   Rows with no visible key produce Out = 0 and LSE = -inf.  The backward produces dK/dV rows
+ *   of unselected keys as zeros, accumulates dK/dV in a fixed order (no atomics), and counts a
+ *   duplicated id once per occurrence. */
 BSA_API bsa_status nsa_selected_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream);
 BSA_API bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const void* k, const void* v, const void* out,
@@ -150,7 +168,9 @@ BSA_API bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const v
  *                       block ids of its BlockSparseMask row (U = B*N1*nqb).
  *   BSA_META_BSA_Q      transposed lists: per (b, g, kb) row, ascending h_local*nqb + qb.
  *   BSA_META_NSA_KV     int32 ids[T, N2, K] (valid ids ascending, then -1) and cnt[T, N2].
- *   BSA_META_NSA_TOKENS per (b, g, kb) row, ascending global token indices that listed kb.
+ *   BSA_META_NSA_TOKENS also, per (b, g, kb) row (kb < ceil(S_q / sel_block_size)), the
+ *                       ascending global token indices whose list holds kb, each token once:
+ *                       int32 row_ptr[B*N2*nblk+1] and col[...].
  *   BSA_META_SFA_PAGES  int32 pages[B, N2, sparse_count * sparse_block_size / page_size].
  * The plan layout for each op is given by sparse_attn_metadata_layout(). */
 typedef enum {

@@ -16,8 +16,9 @@ must reproduce bit-exactly:
     (of the group's query heads) that selected kb.
   * NSA lists (NsaSelectedAttention page, Gather(key, topk_indices[i])): per (token, kv head) the
     valid ids ascending (duplicates kept, -1 dropped, ids past the batch's block count dropped
-    and flagged); per (b, g, kb) the ascending global token indices that selected kb (a token
-    appears once per time it lists kb).
+    and flagged); per (b, g, kb), kb < the longest batch's block count, the ascending global
+    token indices whose list holds kb, each token once (a duplicated id is weighted by its
+    multiplicity in the dK/dV computation instead).
   * SFA page lists (SparseFlashAttention page: sparse_block_size is a multiple of block_size):
     per (b, kv head) the physical pages of the selected sparse blocks, in list order.
   * Work list: see `work_cuts`.
@@ -86,18 +87,19 @@ def nsa_kv_lists(topk: np.ndarray, cu_seqlens, sel_block: int):
     return ids, cnt, status
 
 
-def nsa_token_csr(ids: np.ndarray, cnt: np.ndarray, cu_seqlens, sel_block: int):
-    """Rows (b, g, kb) with kb < nblk(b): ascending global token indices that selected kb."""
+def nsa_token_csr(ids: np.ndarray, cnt: np.ndarray, cu_seqlens, sel_block: int, nblk_max: int):
+    """Rows (b, g, kb) for kb < nblk_max (rows past the batch's own block count are empty):
+    ascending global token indices whose valid list holds kb, each token once."""
     T, N2, _ = ids.shape
-    nblk = nsa_blocks_per_batch(cu_seqlens, sel_block)
+    B = len(cu_seqlens) - 1
     lists = []
-    for b in range(len(nblk)):
+    for b in range(B):
         t0, t1 = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
         for g in range(N2):
-            per = [[] for _ in range(int(nblk[b]))]
+            per = [[] for _ in range(nblk_max)]
             for t in range(t0, t1):
-                for i in range(int(cnt[t, g])):
-                    per[int(ids[t, g, i])].append(t)
+                for kb in sorted(set(int(x) for x in ids[t, g, :int(cnt[t, g])])):
+                    per[kb].append(t)
             lists.extend(per)
     return csr_from_lists(lists)
 

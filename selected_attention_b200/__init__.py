@@ -242,6 +242,70 @@ def plan_array(plan, layout: MetaLayout, index: int, count: int, dtype=torch.int
 
 
 # ---------------------------------------------------------------------------------------------
+# NSA selected attention (TND)
+# ---------------------------------------------------------------------------------------------
+def nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode=MASK_CAUSAL,
+               scale=None) -> Params:
+    """q [T, N1, 128], k [T, N2, 128], topk_indices [T, N2, K] int32, cu_seqlens [B+1] int32 (device)."""
+    T, N1, D = q.shape
+    _, N2, _ = k.shape
+    p = Params()
+    p.q_layout = p.kv_layout = LAYOUT_TND
+    p.B, p.N1, p.N2 = cu_seqlens.shape[0] - 1, N1, N2
+    p.S_q = p.S_kv = int(max_seqlen)
+    p.T_q = p.T_kv = T
+    p.D = p.Dv = D
+    p.cu_seqlens_q = p.cu_seqlens_kv = cu_seqlens.data_ptr()
+    p.sel_block_size, p.sel_block_count = sel_block_size, topk_indices.shape[-1]
+    p.topk_indices = topk_indices.data_ptr()
+    p.mask_mode = mask_mode
+    p.scale = 1.0 / math.sqrt(D) if scale is None else scale
+    return p
+
+
+def nsa_selected_fwd_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check("nsa_selected_fwd_workspace_size", lib().nsa_selected_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def nsa_selected_bwd_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check("nsa_selected_bwd_workspace_size", lib().nsa_selected_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def nsa_selected_fwd(q, k, v, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode=MASK_CAUSAL,
+                     scale=None, out=None, lse=None, workspace=None, stream=None):
+    """Out [T, N1, 128] bf16, LSE [T, N1] fp32 of NSA selected attention."""
+    _need_cuda(q, k, v, topk_indices, cu_seqlens)
+    p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = _workspace(nsa_selected_fwd_workspace_size(p), q.device)
+    _check("nsa_selected_fwd", lib().nsa_selected_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                                      _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def nsa_selected_bwd(q, k, v, out, dout, lse, topk_indices, cu_seqlens, max_seqlen, sel_block_size,
+                     mask_mode=MASK_CAUSAL, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of NSA selected attention."""
+    _need_cuda(q, k, v, out, dout, lse, topk_indices, cu_seqlens)
+    p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = _workspace(nsa_selected_bwd_workspace_size(p), q.device)
+    _check("nsa_selected_bwd", lib().nsa_selected_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                                      _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                                      workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------------------------
 # SFA: sparse decode over a paged KV cache
 # ---------------------------------------------------------------------------------------------
 def sfa_params(q, k_cache, block_table, sparse_indices, seqused_kv, sparse_block_size, scale=None) -> Params:

@@ -100,6 +100,88 @@ bsa_status check_sfa(const bsa_params* p) {
   return BSA_OK;
 }
 
+// ---- NSA (NsaSelectedAttention page constraints) -------------------------------------------------
+// TND only; sparseMode 0 or 2; selected_block_size <= 128 and a multiple of 16; selected block
+// count in [1, 128] with count * size <= 8K; B in [1, 1024], N1 in [1, 128], N2 in [1, 32]; each
+// batch's length up to 128K (S_q carries the longest one); query and key lengths equal.
+bsa_status check_nsa(const bsa_params* p) {
+  if (!p) return BSA_ERR_NULLPTR;
+  if (p->q_layout != BSA_LAYOUT_TND || p->kv_layout != BSA_LAYOUT_TND) return BSA_ERR_UNSUPPORTED;
+  if (p->B < 1 || p->B > 1024 || p->N1 < 1 || p->N1 > 128 || p->N2 < 1 || p->N2 > 32) return BSA_ERR_INVALID_ARG;
+  if (p->N1 < p->N2 || p->N1 % p->N2 != 0) return BSA_ERR_INVALID_ARG;
+  if (p->D != 128 || p->Dv != 128) return BSA_ERR_UNSUPPORTED;
+  if (p->T_q <= 0 || p->T_q != p->T_kv) return BSA_ERR_INVALID_ARG;
+  if (p->S_q <= 0 || p->S_q > 128 * 1024 || p->S_q > p->T_q) return BSA_ERR_INVALID_ARG;
+  if (p->sel_block_size <= 0 || p->sel_block_size > 128 || p->sel_block_size % 16 != 0) return BSA_ERR_INVALID_ARG;
+  if (p->sel_block_count < 1 || p->sel_block_count > 128 || p->sel_block_count * p->sel_block_size > 8192)
+    return BSA_ERR_INVALID_ARG;
+  if (p->mask_mode != BSA_MASK_NONE && p->mask_mode != BSA_MASK_CAUSAL) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale) || p->scale <= 0.f) return BSA_ERR_INVALID_ARG;
+  if (1LL * p->T_q * p->N1 * 128 >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+struct NsaWs {
+  uint32_t* status;
+  int32_t *ok_flag, *ids, *cnt;
+  uint32_t* bitmap;
+  int32_t *t_counts, *t_row_ptr, *t_col;
+  float *lse2, *dvec;
+  int nblk_max, words;
+  size_t off_ids, off_cnt, off_t_row_ptr, off_t_col;  // byte offsets, for the metadata layout
+};
+
+size_t carve_nsa(const bsa_params* p, void* ws, NsaWs* w, bool bwd) {
+  Carver c(ws);
+  w->nblk_max = div_up(p->S_q, p->sel_block_size);
+  w->words = div_up(p->T_q, 32);
+  const size_t rows = static_cast<size_t>(p->T_q) * p->N2;
+  w->status = static_cast<uint32_t*>(ws);
+  w->ok_flag = c.take<int32_t>(1);
+  w->off_ids = c.next();
+  w->ids = c.take<int32_t>(rows * p->sel_block_count);
+  w->off_cnt = c.next();
+  w->cnt = c.take<int32_t>(rows);
+  w->bitmap = nullptr;
+  w->off_t_row_ptr = w->off_t_col = 0;
+  w->t_counts = w->t_row_ptr = w->t_col = nullptr;
+  w->lse2 = w->dvec = nullptr;
+  if (bwd) {
+    w->bitmap = c.take<uint32_t>(static_cast<size_t>(p->N2) * w->nblk_max * w->words);
+    const size_t trows = static_cast<size_t>(p->B) * p->N2 * w->nblk_max;
+    w->t_counts = c.take<int32_t>(trows);
+    w->off_t_row_ptr = c.next();
+    w->t_row_ptr = c.take<int32_t>(trows + 1);
+    w->off_t_col = c.next();
+    w->t_col = c.take<int32_t>(rows * p->sel_block_count);
+    w->lse2 = c.take<float>(static_cast<size_t>(p->T_q) * p->N1);
+    w->dvec = c.take<float>(static_cast<size_t>(p->T_q) * p->N1);
+  }
+  return c.bytes();
+}
+
+NsaMetaArgs nsa_meta_args(const bsa_params* p, const NsaWs& w, bool token_lists) {
+  NsaMetaArgs m;
+  m.topk = p->topk_indices; m.cu_seqlens = p->cu_seqlens_q;
+  m.B = p->B; m.T = p->T_q; m.N2 = p->N2; m.K = p->sel_block_count; m.sel_block = p->sel_block_size;
+  m.max_len = p->S_q; m.nblk_max = w.nblk_max; m.words = w.words; m.token_lists = token_lists;
+  m.ok_flag = w.ok_flag; m.ids = w.ids; m.cnt = w.cnt; m.bitmap = w.bitmap;
+  m.t_counts = w.t_counts; m.t_row_ptr = w.t_row_ptr; m.t_col = w.t_col; m.status = w.status;
+  return m;
+}
+
+NsaArgs nsa_args(const bsa_params* p, const NsaWs& w) {
+  NsaArgs a;
+  a.B = p->B; a.T = p->T_q; a.N1 = p->N1; a.N2 = p->N2; a.K = p->sel_block_count; a.sel_block = p->sel_block_size;
+  a.nblk_max = w.nblk_max; a.mask_mode = p->mask_mode; a.scale = p->scale;
+  a.cu_seqlens = p->cu_seqlens_q; a.ok_flag = w.ok_flag; a.ids = w.ids; a.cnt = w.cnt;
+  a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;
+  a.q = a.k = a.v = a.out_in = a.dout = nullptr;
+  a.lse_in = nullptr; a.lse2 = w.lse2; a.dvec = w.dvec;
+  a.out = a.dq = a.dk = a.dv = nullptr; a.lse_out = nullptr; a.status = w.status;
+  return a;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -217,15 +299,60 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
   a.dvec = w.dvec; a.lse2 = w.lse2; a.dq = dq; a.dk = dk; a.dv = dv; a.status = w.status;
   return cuda_status(bsa_bwd_launch(a, q, k, v, out, dout, lse, st));
 }
-bsa_status nsa_selected_fwd_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
-bsa_status nsa_selected_bwd_workspace_size(const bsa_params*, size_t*) { return BSA_ERR_UNSUPPORTED; }
-bsa_status nsa_selected_fwd(const bsa_params*, const void*, const void*, const void*, void*, float*, void*, size_t,
-                            void*) {
-  return BSA_ERR_UNSUPPORTED;
+bsa_status nsa_selected_fwd_workspace_size(const bsa_params* p, size_t* bytes) {
+  if (!bytes) return BSA_ERR_NULLPTR;
+  bsa_status s = check_nsa(p);
+  if (s != BSA_OK) return s;
+  NsaWs w;
+  *bytes = carve_nsa(p, nullptr, &w, false);
+  return BSA_OK;
 }
-bsa_status nsa_selected_bwd(const bsa_params*, const void*, const void*, const void*, const void*, const void*,
-                            const float*, void*, void*, void*, void*, size_t, void*) {
-  return BSA_ERR_UNSUPPORTED;
+
+bsa_status nsa_selected_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
+  if (!bytes) return BSA_ERR_NULLPTR;
+  bsa_status s = check_nsa(p);
+  if (s != BSA_OK) return s;
+  NsaWs w;
+  *bytes = carve_nsa(p, nullptr, &w, true);
+  return BSA_OK;
+}
+
+bsa_status nsa_selected_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  bsa_status s = check_nsa(p);
+  if (s != BSA_OK) return s;
+  if (!q || !k || !v || !out || !lse || !p->topk_indices || !p->cu_seqlens_q) return BSA_ERR_NULLPTR;
+  NsaWs w;
+  const size_t need = carve_nsa(p, nullptr, &w, false);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != BSA_OK) return s;
+  carve_nsa(p, workspace, &w, false);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+  cudaError_t e = nsa_metadata(nsa_meta_args(p, w, false), st);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  NsaArgs a = nsa_args(p, w);
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse_out = lse;
+  return cuda_status(nsa_fwd_launch(a, st));
+}
+
+bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  bsa_status s = check_nsa(p);
+  if (s != BSA_OK) return s;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !p->topk_indices || !p->cu_seqlens_q)
+    return BSA_ERR_NULLPTR;
+  NsaWs w;
+  const size_t need = carve_nsa(p, nullptr, &w, true);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != BSA_OK) return s;
+  carve_nsa(p, workspace, &w, true);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+  cudaError_t e = nsa_metadata(nsa_meta_args(p, w, true), st);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  NsaArgs a = nsa_args(p, w);
+  a.q = q; a.k = k; a.v = v; a.out_in = out; a.dout = dout; a.lse_in = lse; a.dq = dq; a.dk = dk; a.dv = dv;
+  return cuda_status(nsa_bwd_launch(a, st));
 }
 bsa_status sfa_sparse_decode_workspace_size(const bsa_params* p, size_t* bytes) {
   if (!bytes) return BSA_ERR_NULLPTR;
@@ -301,6 +428,20 @@ bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta
     layout->total_bytes = c.bytes();
     return BSA_OK;
   }
+  if (op == BSA_META_NSA_KV || op == BSA_META_NSA_TOKENS) {
+    bsa_status s = check_nsa(p);
+    if (s != BSA_OK) return s;
+    NsaWs w;
+    const bool tok = op == BSA_META_NSA_TOKENS;
+    layout->total_bytes = carve_nsa(p, nullptr, &w, tok);
+    layout->offsets[1] = w.off_ids;
+    layout->offsets[2] = w.off_cnt;
+    layout->offsets[3] = w.off_t_row_ptr;
+    layout->offsets[4] = w.off_t_col;
+    layout->offsets[0] = 0;
+    layout->count = tok ? 5 : 3;
+    return BSA_OK;
+  }
   if (op == BSA_META_SFA_PAGES) {
     bsa_status s = check_sfa(p);
     if (s != BSA_OK) return s;
@@ -330,6 +471,13 @@ bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, siz
   if ((s = check_ws(plan, plan_bytes, L.total_bytes)) != BSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(plan);
+  if (op == BSA_META_NSA_KV || op == BSA_META_NSA_TOKENS) {
+    if (!p->topk_indices || !p->cu_seqlens_q) return BSA_ERR_NULLPTR;
+    if (cudaMemsetAsync(plan, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+    NsaWs w;
+    carve_nsa(p, plan, &w, op == BSA_META_NSA_TOKENS);
+    return cuda_status(nsa_metadata(nsa_meta_args(p, w, op == BSA_META_NSA_TOKENS), st));
+  }
   if (op == BSA_META_SFA_PAGES) {
     if (!p->block_table || !p->sparse_indices || !p->seqused_kv) return BSA_ERR_NULLPTR;
     if (cudaMemsetAsync(plan, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;

@@ -25,6 +25,7 @@ struct Carver {
     return p;
   }
   size_t bytes() const { return align_up(off, 256); }
+  size_t next() const { return align_up(off, 256); }  // offset of the next take
 };
 
 // ---- kernel timing (profile.cu): brackets a launch with events when timing is enabled ----------
@@ -107,6 +108,34 @@ struct SfaDecodeArgs {
   uint32_t* status;
 };
 cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st);
+
+// ---- NSA selected attention (nsa_meta.cu, nsa.cu) ----------------------------------------------
+struct NsaMetaArgs {
+  const int32_t* topk;        // [T, N2, K]
+  const int32_t* cu_seqlens;  // [B+1]
+  int B, T, N2, K, sel_block, max_len, nblk_max, words;  // words = ceil(T / 32)
+  bool token_lists;           // also build the transposed lists (backward)
+  int32_t* ok_flag;           // 1 if cu_seqlens is valid
+  int32_t* ids;               // [T, N2, K]
+  int32_t* cnt;               // [T, N2]
+  uint32_t* bitmap;           // [N2, nblk_max, words] (backward only)
+  int32_t *t_counts, *t_row_ptr, *t_col;  // rows (b, g, kb) with kb < nblk_max
+  uint32_t* status;
+};
+cudaError_t nsa_metadata(const NsaMetaArgs& a, cudaStream_t st);
+struct NsaArgs {
+  int B, T, N1, N2, K, sel_block, nblk_max, mask_mode;
+  float scale;
+  const int32_t *cu_seqlens, *ok_flag, *ids, *cnt, *t_row_ptr, *t_col;
+  const void *q, *k, *v, *out_in, *dout;
+  const float* lse_in;
+  float *lse2, *dvec;
+  void *out, *dq, *dk, *dv;
+  float* lse_out;
+  uint32_t* status;
+};
+cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st);
+cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st);
 
 // ---- diagnostics (diag.cu) -----------------------------------------------------------------------
 cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,

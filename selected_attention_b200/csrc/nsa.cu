@@ -1,0 +1,586 @@
+// NSA selected attention, forward and backward (NsaSelectedAttention page, forward formula:
+// selected_key/value = Gather(key/value, topk_indices[i]); Out = Softmax(Mask(scale q K_sel^T))
+// V_sel; the backward applies the BlockSparseAttentionGrad formulas to the gathered blocks).
+//
+// A query tile here is one token's heads of one kv-head group: 16 rows.  That is below the 64-row
+// minimum of tcgen05, and the path moves ~16 bytes of gathered K/V per 16x16 MMA step, so the
+// kernels use warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate): one warp owns one
+// (token, kv head, 16-head tile) and streams its selected blocks through shared memory in 16-key
+// chunks with cp.async (2 stages).  The dK/dV pass is block-major: one CTA per (b, g, kv block)
+// walks the ascending token list of that block (nsa_meta.cu), four warps each owning 16 of the
+// block's 64 keys; a block listed twice by a token (literal Gather) counts twice.
+// P and dS enter the products that accumulate dV, dK and dQ as two bf16 parts (hi + lo).
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "sa_common.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kChunk = 16;       // keys per shared-memory chunk
+constexpr int kWarpsFwd = 8;     // warps per CTA in the token-major kernels
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------------------------------------
+// warp-level MMA and shared-memory helpers
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // zero-fill rows past the sequence
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// A [rows][128] bf16 tile in shared memory, rows of 256 B, 16-byte chunks XOR-swizzled by row % 8
+// (ldmatrix reads 8 rows of one chunk column conflict-free).
+__device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
+  return static_cast<uint32_t>(row * 256 + (((chunk ^ row) & 7) | (chunk & 8)) * 16);
+}
+
+// Copy `rows` rows of 128 bf16 (row stride `stride` elements) into a swizzled tile, one warp.
+__device__ __forceinline__ void warp_load_rows(uint32_t tile, const __nv_bfloat16* src, size_t stride, int rows,
+                                               int valid_rows, int lane) {
+  for (int i = lane; i < rows * 16; i += 32) {
+    const int r = i >> 4, c = i & 15;
+    cp_async16(tile + tile_off(r, c), src + static_cast<size_t>(r < valid_rows ? r : 0) * stride + c * 8,
+               r < valid_rows);
+  }
+}
+
+// B fragments for n = 16 rows of the tile, k = 16 columns starting at k0 (tile rows = n):
+// non-transposed ldmatrix, two n8 tiles: {b0,b1} of rows 0-7 and of rows 8-15.
+__device__ __forceinline__ void ldsm_b_rows(uint32_t (&r)[4], uint32_t tile, int k0, int lane) {
+  const int row = (lane & 7) + ((lane >> 4) << 3);
+  const int chunk = (k0 >> 3) + ((lane >> 3) & 1);
+  ldsm_x4(r, tile + tile_off(row, chunk));  // r0,r1: rows 0-7 (k lo, k hi); r2,r3: rows 8-15
+}
+// B fragments for k = 16 rows of the tile (keys), n = 16 columns starting at n0: transposed
+// ldmatrix; r0,r1 = {b0,b1} of columns n0..n0+7, r2,r3 = of columns n0+8..n0+15.
+__device__ __forceinline__ void ldsm_b_cols(uint32_t (&r)[4], uint32_t tile, int n0, int lane) {
+  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+  const int chunk = (n0 >> 3) + (lane >> 4);
+  ldsm_x4_t(r, tile + tile_off(row, chunk));
+}
+// A fragment (16 rows x 16 columns from k0) of a tile.
+__device__ __forceinline__ void ldsm_a(uint32_t (&r)[4], uint32_t tile, int row0, int k0, int lane) {
+  const int row = row0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+  const int chunk = (k0 >> 3) + (lane >> 4);
+  ldsm_x4(r, tile + tile_off(row, chunk));
+}
+
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(x0, x1);
+  lo = pack_bf16(x0 - bf16lo(hi), x1 - bf16hi(hi));
+}
+
+struct NsaParams {
+  int B, T, N1, N2, G, K, sel_block, mask_mode, head_tiles;
+  float scale, scale_log2;
+  const int32_t* cu;
+  const int32_t* ok_flag;
+  const int32_t* ids;  // [T][N2][K] ascending, -1 padded
+  const int32_t* cnt;  // [T][N2]
+  const int32_t* t_row_ptr;
+  const int32_t* t_col;
+  int nblk_max;
+  const __nv_bfloat16 *q, *k, *v, *out, *dout;
+  const float* lse;
+  const float* lse2;   // [T][N1] LSE * log2(e), +inf for rows without keys
+  const float* dvec;   // [T][N1] rowsum(dOut o Out)
+  __nv_bfloat16 *o, *dq, *dk, *dv;
+  float* lse_out;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ int batch_of_token(const int32_t* __restrict__ cu, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------------------------------------
+// token-major kernels: forward (kDq = false) and dQ (kDq = true)
+// ---------------------------------------------------------------------------------------------
+template <bool kDq>
+__global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaParams prm) {
+  extern __shared__ __align__(128) uint8_t tsm[];  // [warp][stage][K, V][16 keys x 256 B]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long item = static_cast<long long>(blockIdx.x) * kWarpsFwd + warp;  // (g, token, head tile)
+  const long long items = static_cast<long long>(prm.N2) * prm.T * prm.head_tiles;
+  if (item >= items || !*prm.ok_flag) return;
+  const int ht = static_cast<int>(item % prm.head_tiles);
+  const int t = static_cast<int>((item / prm.head_tiles) % prm.T);
+  const int g = static_cast<int>(item / (static_cast<long long>(prm.head_tiles) * prm.T));
+  const int b = batch_of_token(prm.cu, prm.B, t);
+  const int t0 = prm.cu[b], len = prm.cu[b + 1] - t0;
+  const int pos = t - t0;
+  const int h0 = g * prm.G + ht * 16;   // first query head of this tile
+  const int rows = min(16, prm.G - ht * 16);
+  const int n_sel = prm.cnt[static_cast<size_t>(t) * prm.N2 + g];
+  const int32_t* sel = prm.ids + (static_cast<size_t>(t) * prm.N2 + g) * prm.K;
+  const int r0 = lane >> 2, cq = (lane & 3) * 2;  // fragment row and column pair
+
+  // Q (and dO for dQ) as A fragments: 8 k-steps x 4 registers, rows = heads
+  uint32_t qa[8][4], da[8][4];
+  {
+    const __nv_bfloat16* qb = prm.q + (static_cast<size_t>(t) * prm.N1 + h0) * kD;
+    const __nv_bfloat16* db = kDq ? prm.dout + (static_cast<size_t>(t) * prm.N1 + h0) * kD : nullptr;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rr = r0 + (i & 1) * 8, cc = ks * 16 + cq + (i >> 1) * 8;
+        qa[ks][i] = rr < rows ? *reinterpret_cast<const uint32_t*>(qb + rr * kD + cc) : 0u;
+        if (kDq) da[ks][i] = rr < rows ? *reinterpret_cast<const uint32_t*>(db + rr * kD + cc) : 0u;
+      }
+  }
+  // per-row state (rows r0 and r0 + 8 of the tile)
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  float l2r[2] = {0.f, 0.f}, dr[2] = {0.f, 0.f};
+  if (kDq) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int rr = r0 + i * 8;
+      l2r[i] = rr < rows ? prm.lse2[static_cast<size_t>(t) * prm.N1 + h0 + rr] : INFINITY;
+      dr[i] = rr < rows ? prm.dvec[static_cast<size_t>(t) * prm.N1 + h0 + rr] : 0.f;
+    }
+  }
+  float acc[16][4];  // O or dQ: 16 n-tiles of 8 columns
+#pragma unroll
+  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+
+  // chunk list: each selected block contributes sel_block / 16 chunks; a chunk whose first key is
+  // past the last visible position (the sequence end, or the query under the causal mask) holds
+  // no visible key and is skipped, so every copied row lies inside the batch
+  const int cpb = prm.sel_block / kChunk;
+  const int n_chunks = n_sel * cpb;
+  const int last_key = prm.mask_mode == 2 ? pos : len - 1;
+  const uint32_t base = smem_u32(tsm) + warp * (2 * 2 * kChunk * 256);
+  auto first_key = [&](int c) { return sel[c / cpb] * prm.sel_block + (c % cpb) * kChunk; };
+  auto next_chunk = [&](int c) {
+    while (c < n_chunks && first_key(c) > last_key) ++c;
+    return c;
+  };
+  auto issue = [&](int c, int stage) {
+    const int kp0 = first_key(c);
+    const int valid = min(kChunk, len - kp0);
+    const uint32_t st = base + stage * 2 * kChunk * 256;
+    const size_t row = static_cast<size_t>(t0 + kp0) * prm.N2 + g;
+    warp_load_rows(st, prm.k + row * kD, static_cast<size_t>(prm.N2) * kD, kChunk, valid, lane);
+    warp_load_rows(st + kChunk * 256, prm.v + row * kD, static_cast<size_t>(prm.N2) * kD, kChunk, valid, lane);
+    cp_commit();
+  };
+  int c = next_chunk(0), stage = 0;
+  if (c < n_chunks) issue(c, 0);
+  while (c < n_chunks) {
+    const int cn = next_chunk(c + 1);
+    if (cn < n_chunks) {
+      issue(cn, stage ^ 1);
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
+    __syncwarp();
+    const int kp0 = first_key(c);
+    const int valid = min(kChunk, len - kp0);
+    const uint32_t kt = base + stage * 2 * kChunk * 256, vt = kt + kChunk * 256;
+    // S = Q K^T (16 rows x 16 keys): two n8 tiles
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t bk[4];
+      ldsm_b_rows(bk, kt, ks * 16, lane);
+      mma16816(s[0], qa[ks], bk[0], bk[1]);
+      mma16816(s[1], qa[ks], bk[2], bk[3]);
+    }
+    // mask: key position kp0 + column < len, and causal key <= query position
+    const int lim = prm.mask_mode == 2 ? min(valid - 1, pos - kp0) : valid - 1;
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = n * 8 + cq + (i & 1);
+        const int rr = r0 + (i >> 1) * 8;
+        if (col > lim || rr >= rows) s[n][i] = -INFINITY;
+      }
+    uint32_t pa_hi[4], pa_lo[4];  // P (or dS) as the A operand over the 16 keys
+    if (!kDq) {
+      // online softmax (lazy rescale by 2^8), rows r0 and r0 + 8
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float mx = fmaxf(fmaxf(s[0][2 * i], s[0][2 * i + 1]), fmaxf(s[1][2 * i], s[1][2 * i + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx *= prm.scale_log2;
+        if (mx > m[i] + 8.f) {
+          const float alpha = m[i] == -INFINITY ? 0.f : ex2(m[i] - mx);
+          l[i] *= alpha;
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            acc[n][2 * i] *= alpha;
+            acc[n][2 * i + 1] *= alpha;
+          }
+          m[i] = mx;
+        }
+        const float mu = m[i] == -INFINITY ? 0.f : m[i];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          s[n][2 * i] = ex2(fmaf(s[n][2 * i], prm.scale_log2, -mu));
+          s[n][2 * i + 1] = ex2(fmaf(s[n][2 * i + 1], prm.scale_log2, -mu));
+          l[i] += s[n][2 * i] + s[n][2 * i + 1];
+        }
+      }
+      pa_hi[0] = pack_bf16(s[0][0], s[0][1]);
+      pa_hi[1] = pack_bf16(s[0][2], s[0][3]);
+      pa_hi[2] = pack_bf16(s[1][0], s[1][1]);
+      pa_hi[3] = pack_bf16(s[1][2], s[1][3]);
+    } else {
+      // P = 2^(s scale log2e - LSE log2e); dP = dO V^T; dS = P (dP - D)
+      float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t bv[4];
+        ldsm_b_rows(bv, vt, ks * 16, lane);
+        mma16816(dp[0], da[ks], bv[0], bv[1]);
+        mma16816(dp[1], da[ks], bv[2], bv[3]);
+      }
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float p = ex2(fmaf(s[n][i], prm.scale_log2, -l2r[i >> 1]));
+          s[n][i] = p * (dp[n][i] - dr[i >> 1]);
+        }
+      split2(s[0][0], s[0][1], pa_hi[0], pa_lo[0]);
+      split2(s[0][2], s[0][3], pa_hi[1], pa_lo[1]);
+      split2(s[1][0], s[1][1], pa_hi[2], pa_lo[2]);
+      split2(s[1][2], s[1][3], pa_hi[3], pa_lo[3]);
+    }
+    // acc += P V (forward) or dS K (dQ): B = [16 keys][128 columns] from the V or K tile
+    const uint32_t bt = kDq ? kt : vt;
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+      uint32_t bb[4];
+      ldsm_b_cols(bb, bt, n * 8, lane);
+      mma16816(acc[n], pa_hi, bb[0], bb[1]);
+      mma16816(acc[n + 1], pa_hi, bb[2], bb[3]);
+      if (kDq) {
+        mma16816(acc[n], pa_lo, bb[0], bb[1]);
+        mma16816(acc[n + 1], pa_lo, bb[2], bb[3]);
+      }
+    }
+    __syncwarp();
+    c = cn;
+    stage ^= 1;
+  }
+  // epilogue
+  if (!kDq) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      l[i] += __shfl_xor_sync(0xffffffffu, l[i], 1);
+      l[i] += __shfl_xor_sync(0xffffffffu, l[i], 2);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int rr = r0 + i * 8;
+    if (rr >= rows) continue;
+    const size_t orow = static_cast<size_t>(t) * prm.N1 + h0 + rr;
+    const float mul = kDq ? prm.scale : (l[i] > 0.f ? 1.f / l[i] : 0.f);
+    __nv_bfloat16* dst = (kDq ? prm.dq : prm.o) + orow * kD;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<uint32_t*>(dst + n * 8 + cq) = pack_bf16(acc[n][2 * i] * mul, acc[n][2 * i + 1] * mul);
+    if (!kDq && (lane & 3) == 0) prm.lse_out[orow] = l[i] > 0.f ? (m[i] * kLn2 + logf(l[i])) : -INFINITY;
+  }
+}
+
+// softmax_grad D = rowsum(dOut o Out) and LSE * log2(e) per (token, head); 8 threads per row
+__global__ void nsa_prep_kernel(const NsaParams prm) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gid >> 3;
+  const int part = static_cast<int>(gid & 7);
+  const long long n_rows = static_cast<long long>(prm.T) * prm.N1;
+  const bool live = row < n_rows;  // whole warps stay for the shuffles below
+  const uint4* po = reinterpret_cast<const uint4*>(prm.out + (live ? row : 0) * kD + part * 16);
+  const uint4* pd = reinterpret_cast<const uint4*>(prm.dout + (live ? row : 0) * kD + part * 16);
+  float d = 0.f;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint4 a = po[k], b = pd[k];
+    d += bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x);
+    d += bf16lo(a.y) * bf16lo(b.y) + bf16hi(a.y) * bf16hi(b.y);
+    d += bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z);
+    d += bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+  }
+  d += __shfl_xor_sync(0xffffffffu, d, 1);
+  d += __shfl_xor_sync(0xffffffffu, d, 2);
+  d += __shfl_xor_sync(0xffffffffu, d, 4);
+  if (live && part == 0) {
+    const_cast<float*>(prm.dvec)[row] = d;
+    const float l = prm.lse[row];
+    const_cast<float*>(prm.lse2)[row] = l == -INFINITY ? INFINITY : l * kLog2e;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// block-major dK / dV
+// ---------------------------------------------------------------------------------------------
+// one warp per 16 keys of the block (sel_block / 16 warps, at most 8)
+__global__ void __launch_bounds__(256) nsa_dkdv_kernel(const NsaParams prm) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x;  // (b, g, kb)
+  const int kb = r % prm.nblk_max;
+  const int bg = r / prm.nblk_max;
+  const int b = bg / prm.N2, g = bg % prm.N2;
+  if (!*prm.ok_flag) return;
+  const int t0 = prm.cu[b], len = prm.cu[b + 1] - t0;
+  const int nkeys = min(prm.sel_block, len - kb * prm.sel_block);  // keys of this block in the batch
+  if (nkeys <= 0) return;
+  const int nb = prm.sel_block;  // block tile rows (rows past nkeys are zero)
+  const int rp = prm.t_row_ptr[r], n_tok = prm.t_row_ptr[r + 1] - rp;
+  // shared memory: K, V of the block [64][128]; Q, dO tiles of one token's 16 heads x 2 stages
+  const uint32_t k_t = smem_u32(dsm), v_t = k_t + nb * 256;
+  const uint32_t qd0 = v_t + nb * 256;  // stage s: Q at qd0 + s*8192, dO at + 4096
+  float* vec = reinterpret_cast<float*>(dsm + 2 * nb * 256 + 2 * 8192);  // [stage][lse2 16 | dvec 16]
+  const int r0 = lane >> 2, cq = (lane & 3) * 2;
+  const int key0 = warp * 16;  // this warp's keys within the block
+  {
+    const size_t row = static_cast<size_t>(t0 + kb * prm.sel_block) * prm.N2 + g;
+    // every warp loads a quarter of K and V
+    for (int i = threadIdx.x; i < nb * 16; i += blockDim.x) {
+      const int rr = i >> 4, c = i & 15;
+      const bool ok = rr < nkeys;
+      cp_async16(k_t + tile_off(rr, c), prm.k + (row + static_cast<size_t>(ok ? rr : 0) * prm.N2) * kD + c * 8, ok);
+      cp_async16(v_t + tile_off(rr, c), prm.v + (row + static_cast<size_t>(ok ? rr : 0) * prm.N2) * kD + c * 8, ok);
+    }
+    cp_commit();
+  }
+  const int items = n_tok * prm.head_tiles;
+  auto issue = [&](int it) {
+    const int tok = prm.t_col[rp + it / prm.head_tiles];
+    const int ht = it % prm.head_tiles;
+    const int h0 = g * prm.G + ht * 16;
+    const int rows = min(16, prm.G - ht * 16);
+    const uint32_t qs = qd0 + (it & 1) * 8192;
+    for (int i = threadIdx.x; i < 16 * 16; i += blockDim.x) {
+      const int rr = i >> 4, c = i & 15;
+      const bool ok = rr < rows;
+      const size_t off = (static_cast<size_t>(tok) * prm.N1 + h0 + (ok ? rr : 0)) * kD + c * 8;
+      cp_async16(qs + tile_off(rr, c), prm.q + off, ok);
+      cp_async16(qs + 4096 + tile_off(rr, c), prm.dout + off, ok);
+    }
+    if (threadIdx.x < 16) {
+      const bool ok = threadIdx.x < rows;
+      const size_t o = static_cast<size_t>(tok) * prm.N1 + h0 + threadIdx.x;
+      vec[(it & 1) * 32 + threadIdx.x] = ok ? prm.lse2[o] : INFINITY;
+      vec[(it & 1) * 32 + 16 + threadIdx.x] = ok ? prm.dvec[o] : 0.f;
+    }
+    cp_commit();
+  };
+  float dk[16][4], dv[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dk[n][i] = dv[n][i] = 0.f;
+  if (items > 0) issue(0);
+  for (int it = 0; it < items; ++it) {
+    if (it + 1 < items) {
+      __syncthreads();  // stage (it+1)&1 was last read in iteration it-1
+      issue(it + 1);
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
+    __syncthreads();
+    const int tok = prm.t_col[rp + it / prm.head_tiles];
+    const int qpos = tok - t0;
+    // multiplicity of this block in the token's list (literal Gather counts duplicates)
+    int mult = 0;
+    {
+      const int32_t* sl = prm.ids + (static_cast<size_t>(tok) * prm.N2 + g) * prm.K;
+      const int nsl = prm.cnt[static_cast<size_t>(tok) * prm.N2 + g];
+      for (int i = 0; i < nsl; ++i) mult += sl[i] == kb;
+    }
+    const uint32_t qs = qd0 + (it & 1) * 8192, ds = qs + 4096;
+    const float* l2 = vec + (it & 1) * 32;
+    const float* dvv = l2 + 16;
+    // S^T = K Q^T and dP^T = V dO^T: this warp's 16 keys x the token's 16 heads
+    float st[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t ka[4], va[4], bq[4], bd[4];
+      ldsm_a(ka, k_t, key0, ks * 16, lane);
+      ldsm_a(va, v_t, key0, ks * 16, lane);
+      ldsm_b_rows(bq, qs, ks * 16, lane);
+      ldsm_b_rows(bd, ds, ks * 16, lane);
+      mma16816(st[0], ka, bq[0], bq[1]);
+      mma16816(st[1], ka, bq[2], bq[3]);
+      mma16816(dpt[0], va, bd[0], bd[1]);
+      mma16816(dpt[1], va, bd[2], bd[3]);
+    }
+    // P^T, dS^T: rows = keys (key0 + r0 (+8)), columns = heads (n*8 + cq (+1))
+    uint32_t p_hi[4], p_lo[4], s_hi[4], s_lo[4];
+    float pv[2][4], sv[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int kr = key0 + r0 + (i >> 1) * 8;   // key row within the block
+        const int hc = n * 8 + cq + (i & 1);       // head column
+        const bool vis = kr < nkeys && (prm.mask_mode != 2 || kb * prm.sel_block + kr <= qpos);
+        const float p = vis ? ex2(fmaf(st[n][i], prm.scale_log2, -l2[hc])) * static_cast<float>(mult) : 0.f;
+        pv[n][i] = p;
+        sv[n][i] = p * (dpt[n][i] - dvv[hc]);
+      }
+    split2(pv[0][0], pv[0][1], p_hi[0], p_lo[0]);
+    split2(pv[0][2], pv[0][3], p_hi[1], p_lo[1]);
+    split2(pv[1][0], pv[1][1], p_hi[2], p_lo[2]);
+    split2(pv[1][2], pv[1][3], p_hi[3], p_lo[3]);
+    split2(sv[0][0], sv[0][1], s_hi[0], s_lo[0]);
+    split2(sv[0][2], sv[0][3], s_hi[1], s_lo[1]);
+    split2(sv[1][0], sv[1][1], s_hi[2], s_lo[2]);
+    split2(sv[1][2], sv[1][3], s_hi[3], s_lo[3]);
+    // dV += P^T dO, dK += dS^T Q  (B = [16 heads][128 dims], transposed loads)
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+      uint32_t bdo[4], bqq[4];
+      ldsm_b_cols(bdo, ds, n * 8, lane);
+      ldsm_b_cols(bqq, qs, n * 8, lane);
+      mma16816(dv[n], p_hi, bdo[0], bdo[1]);
+      mma16816(dv[n + 1], p_hi, bdo[2], bdo[3]);
+      mma16816(dv[n], p_lo, bdo[0], bdo[1]);
+      mma16816(dv[n + 1], p_lo, bdo[2], bdo[3]);
+      mma16816(dk[n], s_hi, bqq[0], bqq[1]);
+      mma16816(dk[n + 1], s_hi, bqq[2], bqq[3]);
+      mma16816(dk[n], s_lo, bqq[0], bqq[1]);
+      mma16816(dk[n + 1], s_lo, bqq[2], bqq[3]);
+    }
+  }
+  if (items == 0) cp_wait<0>();
+  // write dK (scaled) and dV for this warp's keys
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int kr = key0 + r0 + i * 8;
+    if (kr >= nkeys) continue;
+    const size_t row = (static_cast<size_t>(t0 + kb * prm.sel_block + kr) * prm.N2 + g) * kD;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      *reinterpret_cast<uint32_t*>(prm.dk + row + n * 8 + cq) =
+          pack_bf16(dk[n][2 * i] * prm.scale, dk[n][2 * i + 1] * prm.scale);
+      *reinterpret_cast<uint32_t*>(prm.dv + row + n * 8 + cq) = pack_bf16(dv[n][2 * i], dv[n][2 * i + 1]);
+    }
+  }
+}
+
+// dK/dV rows of keys that no token selected stay zero: clear everything first
+__global__ void nsa_zero_kernel(__nv_bfloat16* __restrict__ a, __nv_bfloat16* __restrict__ b, long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n8) {
+    reinterpret_cast<uint4*>(a)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(b)[i] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+NsaParams make_params(const NsaArgs& a) {
+  NsaParams p;
+  p.B = a.B; p.T = a.T; p.N1 = a.N1; p.N2 = a.N2; p.G = a.N1 / a.N2; p.K = a.K; p.sel_block = a.sel_block;
+  p.mask_mode = a.mask_mode; p.head_tiles = (p.G + 15) / 16;
+  p.scale = a.scale; p.scale_log2 = a.scale * kLog2e;
+  p.cu = a.cu_seqlens; p.ok_flag = a.ok_flag; p.ids = a.ids; p.cnt = a.cnt;
+  p.t_row_ptr = a.t_row_ptr; p.t_col = a.t_col; p.nblk_max = a.nblk_max;
+  p.q = static_cast<const __nv_bfloat16*>(a.q); p.k = static_cast<const __nv_bfloat16*>(a.k);
+  p.v = static_cast<const __nv_bfloat16*>(a.v); p.out = static_cast<const __nv_bfloat16*>(a.out_in);
+  p.dout = static_cast<const __nv_bfloat16*>(a.dout);
+  p.lse = a.lse_in; p.lse2 = a.lse2; p.dvec = a.dvec;
+  p.o = static_cast<__nv_bfloat16*>(a.out); p.dq = static_cast<__nv_bfloat16*>(a.dq);
+  p.dk = static_cast<__nv_bfloat16*>(a.dk); p.dv = static_cast<__nv_bfloat16*>(a.dv);
+  p.lse_out = a.lse_out; p.status = a.status;
+  return p;
+}
+
+}  // namespace
+
+cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st) {
+  const NsaParams p = make_params(a);
+  const long long items = static_cast<long long>(a.N2) * a.T * p.head_tiles;
+  if (items == 0) return cudaSuccess;
+  const int smem = kWarpsFwd * 2 * 2 * kChunk * 256;
+  cudaError_t e = cudaFuncSetAttribute(nsa_token_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  prof_begin("nsa_fwd", st);
+  nsa_token_kernel<false><<<static_cast<unsigned>((items + kWarpsFwd - 1) / kWarpsFwd), kWarpsFwd * 32, smem, st>>>(p);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st) {
+  const NsaParams p = make_params(a);
+  cudaError_t e;
+  const long long rows = static_cast<long long>(a.T) * a.N1;
+  if (rows > 0) {
+    prof_begin("nsa_bwd_prep", st);
+    nsa_prep_kernel<<<static_cast<unsigned>((rows * 8 + 255) / 256), 256, 0, st>>>(p);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const long long n8 = static_cast<long long>(a.T) * a.N2 * kD / 8;
+  if (n8 > 0) {
+    nsa_zero_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, st>>>(p.dk, p.dv, n8);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const int kv_rows = a.B * a.N2 * a.nblk_max;
+  if (kv_rows > 0) {
+    const size_t smem = 2 * a.sel_block * 256 + 2 * 8192 + 2 * 32 * sizeof(float);
+    if ((e = cudaFuncSetAttribute(nsa_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+      return e;
+    prof_begin("nsa_bwd_dkdv", st);
+    nsa_dkdv_kernel<<<kv_rows, (a.sel_block / 16) * 32, smem, st>>>(p);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const long long items = static_cast<long long>(a.N2) * a.T * p.head_tiles;
+  if (items > 0) {
+    const int smem = kWarpsFwd * 2 * 2 * kChunk * 256;
+    if ((e = cudaFuncSetAttribute(nsa_token_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    prof_begin("nsa_bwd_dq", st);
+    nsa_token_kernel<true><<<static_cast<unsigned>((items + kWarpsFwd - 1) / kWarpsFwd), kWarpsFwd * 32, smem, st>>>(p);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace sa

@@ -3,7 +3,9 @@
 Floating-point outputs (bf16 Out, dQ, dK, dV) must be within 1e-2 max-abs and 1e-2 relative L2 of
 the fp64 oracle.  Where a reference value is so large that 1e-2 is below bf16 resolution
 (|x| > 2.56, where one bf16 ulp exceeds 1e-2), an element also passes within one bf16 ulp of the
-reference.  LSE (fp32) must be within 1e-3 max-abs.
+reference.  The relative-L2 denominator is floored at 1e-2 * sqrt(n): a reference that is exactly
+zero (a token that sees only its own key has dQ = 0 in closed form) then needs an RMS error of at
+most 1e-4 instead of a ratio over zero.  LSE (fp32) must be within 1e-3 max-abs.
 """
 import numpy as np
 import torch
@@ -22,7 +24,7 @@ def check_close(got, ref, what):
     err = np.abs(got - ref)
     tol = np.maximum(ATOL, bf16_ulp(ref))
     bad = err > tol
-    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), ATOL * np.sqrt(ref.size))
     assert not bad.any() and rel <= RTOL_L2, (
         f"{what}: {bad.sum()} elements over tolerance, max abs {err.max():.3e}, rel L2 {rel:.3e}")
     return float(err.max()), float(rel)

@@ -61,16 +61,18 @@ def test_nsa_lists_properties():
                 want = sorted(int(x) for x in topk[t, g] if 0 <= x < nblk[b])
                 assert ids[t, g, :cnt[t, g]].tolist() == want
                 assert np.all(ids[t, g, cnt[t, g]:] == -1)
-    rp, col = M.nsa_token_csr(ids, cnt, cu, bs)
-    assert rp[-1] == cnt.sum()
-    # every (token, g, id) occurrence appears exactly once per time it is listed
+    nmax = int(nblk.max())
+    rp, col = M.nsa_token_csr(ids, cnt, cu, bs, nmax)
+    distinct = sum(len(set(ids[t, g, :cnt[t, g]].tolist())) for t in range(T) for g in range(N2))
+    assert rp[-1] == distinct and len(rp) == len(seqlens) * N2 * nmax + 1
+    # every (token, g, id) pair appears exactly once, tokens ascending
     r = 0
     for b in range(len(seqlens)):
         for g in range(N2):
-            for kb in range(nblk[b]):
+            for kb in range(nmax):
                 toks = col[rp[r]:rp[r + 1]]
-                assert np.all(np.diff(toks) >= 0)
-                want = [t for t in range(cu[b], cu[b + 1]) for x in ids[t, g, :cnt[t, g]] if x == kb]
+                assert np.all(np.diff(toks) > 0)
+                want = [t for t in range(cu[b], cu[b + 1]) if kb in set(ids[t, g, :cnt[t, g]].tolist())]
                 assert toks.tolist() == want
                 r += 1
 
