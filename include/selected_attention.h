@@ -217,8 +217,9 @@ BSA_API const char* bsa_version(void);
 
 /* ---- diagnostics ---------------------------------------------------------------------------
  * One 128x128x128 tcgen05 tile: c[128][128] (fp32, device) = A B^T with A bf16 [128 rows][128 K]
- * and B bf16 [128 N][128 K] (b_mn_major = 0 or 2) or [128 K][128 N] (b_mn_major = 1 or 3); modes 2
- * and 3 stage A in tensor memory instead of shared memory.  Runs the same
+ * and B bf16 [128 N][128 K] (b_mn_major = 0, 2, 4) or [128 K][128 N] (b_mn_major = 1, 3, 5); modes 2
+ * and 3 stage A in tensor memory instead of shared memory; modes 4 and 5 read `a` as A^T
+ * ([128 K][128 M], the MN-major A operand).  Other modes return BSA_ERR_INVALID_ARG.  Runs the same
  * TMA / shared-memory-descriptor / TMEM machinery as the attention kernels, so a tile-level
  * fault can be told apart from an attention-level one.  workspace: >= 256 bytes (status word).
  * Not part of the pages' operations. */

@@ -374,11 +374,12 @@ def bsa_profile_collect() -> dict:
 # ---------------------------------------------------------------------------------------------
 # diagnostics
 # ---------------------------------------------------------------------------------------------
-def bsa_diag_mma_tile(a, b, b_mn_major: bool, stream=None):
-    """c = a @ b.T (b K-major [N][K]) or a @ b (b MN-major [K][N]) on one tcgen05 tile."""
+def bsa_diag_mma_tile(a, b, mode, stream=None):
+    """One tcgen05 tile.  mode 0/2: c = a @ b.T; 1/3: c = a @ b (2, 3 stage a in tensor memory);
+    4: c = a.T @ b.T; 5: c = a.T @ b (a read as the MN-major A operand)."""
     _need_cuda(a, b)
     c = torch.empty(128, 128, dtype=torch.float32, device=a.device)
     ws = _workspace(256, a.device)
-    _check("bsa_diag_mma_tile", lib().bsa_diag_mma_tile(_ptr(a), _ptr(b), _ptr(c), int(b_mn_major), _ptr(ws),
+    _check("bsa_diag_mma_tile", lib().bsa_diag_mma_tile(_ptr(a), _ptr(b), _ptr(c), int(mode), _ptr(ws),
                                                         _stream(stream)))
     return c, ws

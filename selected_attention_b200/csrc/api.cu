@@ -123,7 +123,7 @@ bsa_status check_nsa(const bsa_params* p) {
 
 struct NsaWs {
   uint32_t* status;
-  int32_t *ok_flag, *ids, *cnt;
+  int32_t *ok_flag, *ids, *cnt, *dup;
   uint32_t* bitmap;
   int32_t *t_counts, *t_row_ptr, *t_col;
   float *lse2, *dvec;
@@ -142,6 +142,7 @@ size_t carve_nsa(const bsa_params* p, void* ws, NsaWs* w, bool bwd) {
   w->ids = c.take<int32_t>(rows * p->sel_block_count);
   w->off_cnt = c.next();
   w->cnt = c.take<int32_t>(rows);
+  w->dup = c.take<int32_t>(rows);
   w->bitmap = nullptr;
   w->off_t_row_ptr = w->off_t_col = 0;
   w->t_counts = w->t_row_ptr = w->t_col = nullptr;
@@ -165,7 +166,7 @@ NsaMetaArgs nsa_meta_args(const bsa_params* p, const NsaWs& w, bool token_lists)
   m.topk = p->topk_indices; m.cu_seqlens = p->cu_seqlens_q;
   m.B = p->B; m.T = p->T_q; m.N2 = p->N2; m.K = p->sel_block_count; m.sel_block = p->sel_block_size;
   m.max_len = p->S_q; m.nblk_max = w.nblk_max; m.words = w.words; m.token_lists = token_lists;
-  m.ok_flag = w.ok_flag; m.ids = w.ids; m.cnt = w.cnt; m.bitmap = w.bitmap;
+  m.ok_flag = w.ok_flag; m.ids = w.ids; m.cnt = w.cnt; m.dup = w.dup; m.bitmap = w.bitmap;
   m.t_counts = w.t_counts; m.t_row_ptr = w.t_row_ptr; m.t_col = w.t_col; m.status = w.status;
   return m;
 }
@@ -174,7 +175,7 @@ NsaArgs nsa_args(const bsa_params* p, const NsaWs& w) {
   NsaArgs a;
   a.B = p->B; a.T = p->T_q; a.N1 = p->N1; a.N2 = p->N2; a.K = p->sel_block_count; a.sel_block = p->sel_block_size;
   a.nblk_max = w.nblk_max; a.mask_mode = p->mask_mode; a.scale = p->scale;
-  a.cu_seqlens = p->cu_seqlens_q; a.ok_flag = w.ok_flag; a.ids = w.ids; a.cnt = w.cnt;
+  a.cu_seqlens = p->cu_seqlens_q; a.ok_flag = w.ok_flag; a.ids = w.ids; a.cnt = w.cnt; a.dup = w.dup;
   a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;
   a.q = a.k = a.v = a.out_in = a.dout = nullptr;
   a.lse_in = nullptr; a.lse2 = w.lse2; a.dvec = w.dvec;
@@ -520,6 +521,7 @@ bsa_status bsa_get_status(const void* workspace, void* stream, uint32_t* dev_bit
 bsa_status bsa_diag_mma_tile(const void* a, const void* b, float* c, int32_t b_mn_major, void* workspace,
                              void* stream) {
   if (!a || !b || !c || !workspace) return BSA_ERR_NULLPTR;
+  if (b_mn_major < 0 || b_mn_major > 5) return BSA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
   return cuda_status(diag_mma_tile_launch(a, b, c, 128, b_mn_major, static_cast<uint32_t*>(workspace), st));

@@ -1,6 +1,7 @@
 // Diagnostic: one 128 x 128 x 128 tcgen05 tile, C = A B^T with A K-major and B either K-major
 // ([N][K]) or MN-major ([K][N]); modes 2 and 3 take A from tensor memory (written with
-// tcgen05.st) with B K-major (2) or MN-major (3).  Exercises exactly the building blocks the attention kernels use
+// tcgen05.st) with B K-major (2) or MN-major (3); modes 4 and 5 give A MN-major (the buffer holds
+// A^T, [K][M]) with B K-major (4) or MN-major (5).  Exercises exactly the building blocks the attention kernels use
 // (TMA 128B-swizzled loads, smem descriptors of both majors, TMEM accumulate, tcgen05.ld), so a
 // parity failure in attention can be narrowed to the tile machinery or the attention logic.
 #include <cuda.h>
@@ -40,7 +41,7 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   bool ok = true;
-  if (b_mn_major >= 2) {
+  if (b_mn_major == 2 || b_mn_major == 3) {
     // A row (warp*32 + lane) from global into TMEM columns [128, 192): 64 packed bf16 pairs
     const uint32_t* arow = reinterpret_cast<const uint32_t*>(a_ptr) + (warp * 32 + lane) * 64;
     uint32_t r[16];
@@ -62,17 +63,21 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
     ok = mbar_wait(&s.bar_load, 0, status);
     if (ok) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, 128, false, b_mn_major == 1 || b_mn_major == 3);
+      const bool a_mn = b_mn_major >= 4;
+      const uint32_t idesc =
+          idesc_bf16_f32(128, 128, a_mn, b_mn_major == 1 || b_mn_major == 3 || b_mn_major == 5);
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = sdesc_sw128(smem_u32(s.a[ks / 4]) + (ks % 4) * 32, 0, 1024);
+        // A MN-major: sub-tile = M chunk of 64, K step = 16 rows
+        const uint64_t ad = a_mn ? sdesc_sw128(smem_u32(s.a[0]) + ks * 2048, 128 * 128, 1024)
+                                 : sdesc_sw128(smem_u32(s.a[ks / 4]) + (ks % 4) * 32, 0, 1024);
         uint64_t bd;
-        if (b_mn_major >= 2) {  // A from TMEM; B K-major (2) or MN-major (3)
+        if (b_mn_major == 2 || b_mn_major == 3) {  // A from TMEM; B K-major (2) or MN-major (3)
           bd = b_mn_major == 3 ? sdesc_sw128(smem_u32(s.b[0]) + ks * 2048, 128 * 128, 1024)
                                : sdesc_sw128(smem_u32(s.b[ks / 4]) + (ks % 4) * 32, 0, 1024);
           mma_bf16_ts(tmem, tmem + 128 + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
           continue;
         }
-        if (b_mn_major)  // B tile is [K rows][N cols]: sub-tile = N chunk, K step = 16 rows
+        if (b_mn_major == 1 || b_mn_major == 5)  // B tile is [K rows][N cols]: sub-tile = N chunk, K step = 16 rows
           bd = sdesc_sw128(smem_u32(s.b[0]) + ks * 2048, 128 * 128, 1024);
         else
           bd = sdesc_sw128(smem_u32(s.b[ks / 4]) + (ks % 4) * 32, 0, 1024);

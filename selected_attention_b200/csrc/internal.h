@@ -118,6 +118,7 @@ struct NsaMetaArgs {
   int32_t* ok_flag;           // 1 if cu_seqlens is valid
   int32_t* ids;               // [T, N2, K]
   int32_t* cnt;               // [T, N2]
+  int32_t* dup;               // [T, N2] 1 if the valid list holds an id twice
   uint32_t* bitmap;           // [N2, nblk_max, words] (backward only)
   int32_t *t_counts, *t_row_ptr, *t_col;  // rows (b, g, kb) with kb < nblk_max
   uint32_t* status;
@@ -126,7 +127,7 @@ cudaError_t nsa_metadata(const NsaMetaArgs& a, cudaStream_t st);
 struct NsaArgs {
   int B, T, N1, N2, K, sel_block, nblk_max, mask_mode;
   float scale;
-  const int32_t *cu_seqlens, *ok_flag, *ids, *cnt, *t_row_ptr, *t_col;
+  const int32_t *cu_seqlens, *ok_flag, *ids, *cnt, *dup, *t_row_ptr, *t_col;
   const void *q, *k, *v, *out_in, *dout;
   const float* lse_in;
   float *lse2, *dvec;
@@ -136,6 +137,10 @@ struct NsaArgs {
 };
 cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st);
 cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st);
+// dK/dV on tcgen05 (nsa_dkdv.cu) for 64-token blocks and G in {8, 16, 32, 64, 128};
+// cudaErrorNotSupported for other shapes.  Needs lse2/dvec from the backward preprocess.
+bool nsa_dkdv_tc_supported(const NsaArgs& a);
+cudaError_t nsa_dkdv_tc_launch(const NsaArgs& a, cudaStream_t st);
 
 // ---- diagnostics (diag.cu) -----------------------------------------------------------------------
 cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,

@@ -559,12 +559,14 @@ cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int kv_rows = a.B * a.N2 * a.nblk_max;
-  if (kv_rows > 0) {
+  if (kv_rows > 0 && nsa_dkdv_tc_supported(a)) {
+    if ((e = nsa_dkdv_tc_launch(a, st)) != cudaSuccess) return e;
+  } else if (kv_rows > 0) {
     const size_t smem = 2 * a.sel_block * 256 + 2 * 8192 + 2 * 32 * sizeof(float);
     if ((e = cudaFuncSetAttribute(nsa_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
       return e;
-    prof_begin("nsa_bwd_dkdv", st);
+    prof_begin("nsa_bwd_dkdv_warp", st);
     nsa_dkdv_kernel<<<kv_rows, (a.sel_block / 16) * 32, smem, st>>>(p);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

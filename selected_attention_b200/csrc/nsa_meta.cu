@@ -6,8 +6,9 @@
 //                      and every kernel skips all work.
 //   nsa_kv_lists       per (token, kv head): the valid block ids ascending (-1 dropped; ids at or
 //                      past the batch's block count dropped and flagged SA_DEV_BAD_INDEX;
-//                      duplicates kept) and their count.  For the backward it also sets bit t of
-//                      the bit-row (g, kb) of a bitmap [N2][nblk_max][ceil(T/32)] words.
+//                      duplicates kept), their count and whether an id repeats.  For the
+//                      backward it also sets bit t of the bit-row (g, kb) of a bitmap
+//                      [N2][nblk_max][ceil(T/32)] words.
 //   nsa_token_lists    per (b, g, kb) (kb padded to the longest batch): the tokens whose list holds
 //                      kb, ascending, each once.  One warp per (b, g, kb) reads the batch's span of
 //                      the bit-row, a word per lane, so the order is fixed without sorting.
@@ -44,7 +45,7 @@ __device__ __forceinline__ int batch_of(const int32_t* __restrict__ cu, int B, i
 __global__ void nsa_kv_lists_kernel(const int32_t* __restrict__ topk, const int32_t* __restrict__ cu, int B, int T,
                                     int N2, int K, int sel_block, int nblk_max, int words,
                                     const int32_t* __restrict__ ok_flag,
-                                    int32_t* __restrict__ ids, int32_t* __restrict__ cnt,
+                                    int32_t* __restrict__ ids, int32_t* __restrict__ cnt, int32_t* __restrict__ dup,
                                     uint32_t* __restrict__ bitmap, uint32_t* __restrict__ status) {
   const int row = blockIdx.x * blockDim.x + threadIdx.x;  // (t, g)
   if (row >= T * N2) return;
@@ -53,6 +54,7 @@ __global__ void nsa_kv_lists_kernel(const int32_t* __restrict__ topk, const int3
   if (!*ok_flag) {
     for (int i = 0; i < K; ++i) out[i] = -1;
     cnt[row] = 0;
+    dup[row] = 0;
     return;
   }
   const int b = batch_of(cu, B, t);
@@ -77,8 +79,11 @@ __global__ void nsa_kv_lists_kernel(const int32_t* __restrict__ topk, const int3
     if (bitmap)  // v < nblk <= nblk_max: the batch is no longer than the maximum length
       atomicOr(&bitmap[(static_cast<size_t>(g) * nblk_max + v) * words + (t >> 5)], 1u << (t & 31));
   }
+  int d = 0;
+  for (int i = 1; i < n; ++i) d |= out[i] == out[i - 1];
   for (int i = n; i < K; ++i) out[i] = -1;
   cnt[row] = n;
+  dup[row] = d;
   if (bad) raise_status(status, SA_DEV_BAD_INDEX);
 }
 
@@ -141,7 +146,7 @@ cudaError_t nsa_metadata(const NsaMetaArgs& a, cudaStream_t st) {
   if (rows > 0) {
     prof_begin("nsa_kv_lists", st);
     nsa_kv_lists_kernel<<<(rows + 127) / 128, 128, 0, st>>>(a.topk, a.cu_seqlens, a.B, a.T, a.N2, a.K, a.sel_block,
-                                                            a.nblk_max, a.words, a.ok_flag, a.ids, a.cnt, bitmap,
+                                                            a.nblk_max, a.words, a.ok_flag, a.ids, a.cnt, a.dup, bitmap,
                                                             a.status);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -34,6 +34,14 @@ def test_diag_mma_tile(cuda_ok):
     c, ws = sa.bsa_diag_mma_tile(_dev(a), _dev(b), 3)
     torch.cuda.synchronize()
     assert np.abs(c.cpu().numpy() - fa @ fb).max() < 1e-3
+    # A MN-major (the buffer holds A^T), B K-major then MN-major
+    c, ws = sa.bsa_diag_mma_tile(_dev(a), _dev(b), 4)
+    torch.cuda.synchronize()
+    assert np.abs(c.cpu().numpy() - fa.T @ fb.T).max() < 1e-3
+    c, ws = sa.bsa_diag_mma_tile(_dev(a), _dev(b), 5)
+    torch.cuda.synchronize()
+    assert sa.bsa_get_status(ws) == 0
+    assert np.abs(c.cpu().numpy() - fa.T @ fb).max() < 1e-3
 
 
 @pytest.mark.parametrize("config", [1, 2, 5])
