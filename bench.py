@@ -229,7 +229,7 @@ def run_reference(args, rank, world):
     """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
     if rank != 0:
         return
-    w = synth.workload(args.config)
+    w = nsa_workload(args) if args.config == 3 else synth.workload(args.config)
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; warm-up steps are a no-op
     total_f, total_t, desc = 0, 0.0, ""
@@ -280,6 +280,17 @@ def config_dict_nsa(w, args):
     }
 
 
+def nsa_workload(args):
+    """The NSA workload; --nsa-seqlens swaps in other batch lengths (same seed and shapes), a
+    smaller problem for profiler captures."""
+    import dataclasses
+    w = synth.workload(3)
+    if args.nsa_seqlens:
+        lens = [int(x) for x in args.nsa_seqlens.split(",")]
+        w = dataclasses.replace(w, seqlens=lens, name=f"{w.name}_seqlens_{'_'.join(map(str, lens))}")
+    return w
+
+
 def _dist_helpers(world, dev):
     import torch
 
@@ -305,7 +316,7 @@ def run_nsa(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = synth.workload(3)
+    w = nsa_workload(args)
     topk = w.topk()
     cu = w.cu_seqlens()
     vpairs = visible_pairs_nsa(w, topk)
@@ -636,6 +647,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nsa-seqlens", default="", help="config 3 only: comma-separated batch lengths")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

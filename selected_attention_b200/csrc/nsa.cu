@@ -6,7 +6,7 @@
 // minimum of tcgen05, and the path moves ~16 bytes of gathered K/V per 16x16 MMA step, so the
 // kernels use warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate): one warp owns one
 // (token, kv head, 16-head tile) and streams its selected blocks through shared memory in 16-key
-// chunks with cp.async (2 stages).  The dK/dV pass is block-major: one CTA per (b, g, kv block)
+// chunks (TMA, three stages per warp).  The dK/dV pass is block-major: one CTA per (b, g, kv block)
 // walks the ascending token list of that block (nsa_meta.cu), four warps each owning 16 of the
 // block's 64 keys; a block listed twice by a token (literal Gather) counts twice.
 // P and dS enter the products that accumulate dV, dK and dQ as two bf16 parts (hi + lo).
@@ -20,7 +20,6 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kChunk = 16;       // keys per shared-memory chunk
-constexpr int kWarpsFwd = 8;     // warps per CTA in the token-major kernels
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -58,16 +57,6 @@ __device__ __forceinline__ void cp_wait() {
 // (ldmatrix reads 8 rows of one chunk column conflict-free).
 __device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
   return static_cast<uint32_t>(row * 256 + (((chunk ^ row) & 7) | (chunk & 8)) * 16);
-}
-
-// Copy `rows` rows of 128 bf16 (row stride `stride` elements) into a swizzled tile, one warp.
-__device__ __forceinline__ void warp_load_rows(uint32_t tile, const __nv_bfloat16* src, size_t stride, int rows,
-                                               int valid_rows, int lane) {
-  for (int i = lane; i < rows * 16; i += 32) {
-    const int r = i >> 4, c = i & 15;
-    cp_async16(tile + tile_off(r, c), src + static_cast<size_t>(r < valid_rows ? r : 0) * stride + c * 8,
-               r < valid_rows);
-  }
 }
 
 // B fragments for n = 16 rows of the tile, k = 16 columns starting at k0 (tile rows = n):
@@ -127,12 +116,60 @@ __device__ __forceinline__ int batch_of_token(const int32_t* __restrict__ cu, in
 
 // ---------------------------------------------------------------------------------------------
 // token-major kernels: forward (kDq = false) and dQ (kDq = true)
+//
+// Each warp owns one (token, kv head, 16-head tile) item and a private ring of kTokStages chunk
+// stages.  Lane 0 copies a chunk's 16 K rows and 16 V rows with four TMA loads (the rows of one kv
+// head are 256 B apart in TND, one box of {64 dims, 1 head, 16 tokens} per head-dim half), into
+// 128-byte-swizzled [16 rows][64 dims] halves; all lanes wait on the stage's mbarrier.
 // ---------------------------------------------------------------------------------------------
+constexpr int kTokStages = 3;
+// warps per CTA: the forward fits 168 registers (9 warps); dQ holds dO fragments too (8 warps)
 template <bool kDq>
-__global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaParams prm) {
-  extern __shared__ __align__(128) uint8_t tsm[];  // [warp][stage][K, V][16 keys x 256 B]
+__host__ __device__ constexpr int tok_warps() { return kDq ? 8 : 9; }
+constexpr int kHalfBytes = kChunk * 128;        // [16 rows][64 dims]
+constexpr int kTileBytes = 2 * kHalfBytes;      // [16 rows][128 dims]
+constexpr int kTokStageBytes = 2 * kTileBytes;  // K and V tiles of one chunk
+template <bool kDq>
+__host__ __device__ constexpr int tok_smem() { return tok_warps<kDq>() * kTokStages * (kTokStageBytes + 8) + 1024; }
+
+// byte address of (row, 16-byte column c16 of the 128 dims) in a chunk tile
+__device__ __forceinline__ uint32_t tok_swz(uint32_t tile, int row, int c16) {
+  return tile + (c16 >> 3) * kHalfBytes + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
+}
+// B fragments of X^T for k = dims [16 ks, 16 ks + 16) and n = the 16 rows (two n8 tiles)
+__device__ __forceinline__ void ldsm_rows_k(uint32_t (&r)[4], uint32_t tile, int ks, int lane) {
+  const int row = (lane & 7) + ((lane >> 4) << 3);
+  ldsm_x4(r, tok_swz(tile, row, ks * 2 + ((lane >> 3) & 1)));
+}
+// B fragments of X for k = the 16 rows and n = dims [n0, n0 + 16) (transposed load)
+__device__ __forceinline__ void ldsm_rows_n(uint32_t (&r)[4], uint32_t tile, int n0, int lane) {
+  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+  ldsm_x4_t(r, tok_swz(tile, row, (n0 >> 3) + (lane >> 4)));
+}
+
+// wait on a warp-private stage barrier (bounded; does not give up early when another CTA has
+// timed out, so a warp can always drain its own copies)
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      raise_status(status, SA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+template <bool kDq>
+__global__ void __launch_bounds__(tok_warps<kDq>() * 32)
+    nsa_token_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const NsaParams prm) {
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kTokWarps = tok_warps<kDq>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long item = static_cast<long long>(blockIdx.x) * kWarpsFwd + warp;  // (g, token, head tile)
+  const long long item = static_cast<long long>(blockIdx.x) * kTokWarps + warp;  // (g, token, head tile)
   const long long items = static_cast<long long>(prm.N2) * prm.T * prm.head_tiles;
   if (item >= items || !*prm.ok_flag) return;
   const int ht = static_cast<int>(item % prm.head_tiles);
@@ -146,6 +183,13 @@ __global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaPara
   const int n_sel = prm.cnt[static_cast<size_t>(t) * prm.N2 + g];
   const int32_t* sel = prm.ids + (static_cast<size_t>(t) * prm.N2 + g) * prm.K;
   const int r0 = lane >> 2, cq = (lane & 3) * 2;  // fragment row and column pair
+  uint8_t* wst = tsm + warp * kTokStages * kTokStageBytes;  // this warp's stages
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(tsm + kTokWarps * kTokStages * kTokStageBytes) + warp * kTokStages;
+  if (lane == 0) {
+    for (int i = 0; i < kTokStages; ++i) mbar_init(&wbar[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
 
   // Q (and dO for dQ) as A fragments: 8 k-steps x 4 registers, rows = heads
   uint32_t qa[8][4], da[8][4];
@@ -178,48 +222,61 @@ __global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaPara
 
   // chunk list: each selected block contributes sel_block / 16 chunks; a chunk whose first key is
   // past the last visible position (the sequence end, or the query under the causal mask) holds
-  // no visible key and is skipped, so every copied row lies inside the batch
+  // no visible key and is skipped.  Rows of a loaded chunk past the batch are masked below.
   const int cpb = prm.sel_block / kChunk;
   const int n_chunks = n_sel * cpb;
   const int last_key = prm.mask_mode == 2 ? pos : len - 1;
-  const uint32_t base = smem_u32(tsm) + warp * (2 * 2 * kChunk * 256);
   auto first_key = [&](int c) { return sel[c / cpb] * prm.sel_block + (c % cpb) * kChunk; };
-  auto next_chunk = [&](int c) {
+  int cand = 0;
+  // the next visible chunk (or n_chunks) into `stage`
+  auto take = [&](int stage) {
+    int c = cand;
     while (c < n_chunks && first_key(c) > last_key) ++c;
+    if (c < n_chunks) {
+      cand = c + 1;
+      if (lane == 0) {
+        const int tk = t0 + first_key(c);
+        uint8_t* st = wst + stage * kTokStageBytes;
+        mbar_arrive_expect_tx(&wbar[stage], kTokStageBytes);
+        tma_load_3d(st, &tm_k, &wbar[stage], 0, g, tk);
+        tma_load_3d(st + kHalfBytes, &tm_k, &wbar[stage], 64, g, tk);
+        tma_load_3d(st + kTileBytes, &tm_v, &wbar[stage], 0, g, tk);
+        tma_load_3d(st + kTileBytes + kHalfBytes, &tm_v, &wbar[stage], 64, g, tk);
+      }
+    }
     return c;
   };
-  auto issue = [&](int c, int stage) {
-    const int kp0 = first_key(c);
-    const int valid = min(kChunk, len - kp0);
-    const uint32_t st = base + stage * 2 * kChunk * 256;
-    const size_t row = static_cast<size_t>(t0 + kp0) * prm.N2 + g;
-    warp_load_rows(st, prm.k + row * kD, static_cast<size_t>(prm.N2) * kD, kChunk, valid, lane);
-    warp_load_rows(st + kChunk * 256, prm.v + row * kD, static_cast<size_t>(prm.N2) * kD, kChunk, valid, lane);
-    cp_commit();
-  };
-  int c = next_chunk(0), stage = 0;
-  if (c < n_chunks) issue(c, 0);
-  while (c < n_chunks) {
-    const int cn = next_chunk(c + 1);
-    if (cn < n_chunks) {
-      issue(cn, stage ^ 1);
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
+  int c = take(0), c1 = take(1);
+  int it = 0;
+  for (; c < n_chunks; ++it) {
+    const int c2 = take((it + 2) % kTokStages);  // the stage consumed in the previous iteration
+    const int stage = it % kTokStages;
+    if (!__all_sync(0xffffffffu, stage_wait(&wbar[stage], (it / kTokStages) & 1, prm.status))) {
+      c = c1;   // leave the loop; the copies still in flight are drained below
+      c1 = c2;
+      ++it;
+      break;
     }
-    __syncwarp();
     const int kp0 = first_key(c);
     const int valid = min(kChunk, len - kp0);
-    const uint32_t kt = base + stage * 2 * kChunk * 256, vt = kt + kChunk * 256;
-    // S = Q K^T (16 rows x 16 keys): two n8 tiles
+    const uint32_t kt = smem_u32(wst + stage * kTokStageBytes), vt = kt + kTileBytes;
+    // S = Q K^T (16 rows x 16 keys): two n8 tiles, each as two independent k-halves
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t bk[4];
-      ldsm_b_rows(bk, kt, ks * 16, lane);
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t bk[4], bk2[4];
+      ldsm_rows_k(bk, kt, ks, lane);
+      ldsm_rows_k(bk2, kt, ks + 4, lane);
       mma16816(s[0], qa[ks], bk[0], bk[1]);
       mma16816(s[1], qa[ks], bk[2], bk[3]);
+      mma16816(s2[0], qa[ks + 4], bk2[0], bk2[1]);
+      mma16816(s2[1], qa[ks + 4], bk2[2], bk2[3]);
     }
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[n][i] += s2[n][i];
     // mask: key position kp0 + column < len, and causal key <= query position
     const int lim = prm.mask_mode == 2 ? min(valid - 1, pos - kp0) : valid - 1;
 #pragma unroll
@@ -264,19 +321,23 @@ __global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaPara
     } else {
       // P = 2^(s scale log2e - LSE log2e); dP = dO V^T; dS = P (dP - D)
       float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float dp2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t bv[4];
-        ldsm_b_rows(bv, vt, ks * 16, lane);
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t bv[4], bv2[4];
+        ldsm_rows_k(bv, vt, ks, lane);
+        ldsm_rows_k(bv2, vt, ks + 4, lane);
         mma16816(dp[0], da[ks], bv[0], bv[1]);
         mma16816(dp[1], da[ks], bv[2], bv[3]);
+        mma16816(dp2[0], da[ks + 4], bv2[0], bv2[1]);
+        mma16816(dp2[1], da[ks + 4], bv2[2], bv2[3]);
       }
 #pragma unroll
       for (int n = 0; n < 2; ++n)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float p = ex2(fmaf(s[n][i], prm.scale_log2, -l2r[i >> 1]));
-          s[n][i] = p * (dp[n][i] - dr[i >> 1]);
+          s[n][i] = p * (dp[n][i] + dp2[n][i] - dr[i >> 1]);
         }
       split2(s[0][0], s[0][1], pa_hi[0], pa_lo[0]);
       split2(s[0][2], s[0][3], pa_hi[1], pa_lo[1]);
@@ -288,7 +349,7 @@ __global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaPara
 #pragma unroll
     for (int n = 0; n < 16; n += 2) {
       uint32_t bb[4];
-      ldsm_b_cols(bb, bt, n * 8, lane);
+      ldsm_rows_n(bb, bt, n * 8, lane);
       mma16816(acc[n], pa_hi, bb[0], bb[1]);
       mma16816(acc[n + 1], pa_hi, bb[2], bb[3]);
       if (kDq) {
@@ -296,10 +357,16 @@ __global__ void __launch_bounds__(kWarpsFwd * 32) nsa_token_kernel(const NsaPara
         mma16816(acc[n + 1], pa_lo, bb[2], bb[3]);
       }
     }
-    __syncwarp();
-    c = cn;
-    stage ^= 1;
+    __syncwarp();  // every lane has read the stage before lane 0 refills it
+    c = c1;
+    c1 = c2;
   }
+  // drain copies still in flight after an early exit (none after a complete pass)
+  for (int k = 0; k < 2; ++k) {
+    const int ck = k == 0 ? c : c1;
+    if (ck < n_chunks) stage_wait(&wbar[(it + k) % kTokStages], ((it + k) / kTokStages) & 1, prm.status);
+  }
+  if (aborted(prm.status)) return;
   // epilogue
   if (!kDq) {
 #pragma unroll
@@ -530,17 +597,30 @@ NsaParams make_params(const NsaArgs& a) {
 
 }  // namespace
 
-cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st) {
-  const NsaParams p = make_params(a);
+// K and V as [T][N2][128] with a {64 dims, 1 head, 16 tokens} box (rows past T read as zero)
+bool nsa_kv_maps(const NsaArgs& a, CUtensorMap* tk, CUtensorMap* tv) {
+  const uint64_t hs = static_cast<uint64_t>(a.N2) * kD;
+  return make_tmap_3d_bf16(tk, a.k, kD, a.N2, a.T, kD, hs, 1, kChunk) &&
+         make_tmap_3d_bf16(tv, a.v, kD, a.N2, a.T, kD, hs, 1, kChunk);
+}
+
+template <bool kDq>
+cudaError_t nsa_token_launch(const NsaArgs& a, const NsaParams& p, const char* name, cudaStream_t st) {
   const long long items = static_cast<long long>(a.N2) * a.T * p.head_tiles;
   if (items == 0) return cudaSuccess;
-  const int smem = kWarpsFwd * 2 * 2 * kChunk * 256;
-  cudaError_t e = cudaFuncSetAttribute(nsa_token_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  CUtensorMap tk, tv;
+  if (!nsa_kv_maps(a, &tk, &tv)) return cudaErrorInvalidValue;
+  constexpr int warps = tok_warps<kDq>(), smem = tok_smem<kDq>();
+  cudaError_t e = cudaFuncSetAttribute(nsa_token_kernel<kDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  prof_begin("nsa_fwd", st);
-  nsa_token_kernel<false><<<static_cast<unsigned>((items + kWarpsFwd - 1) / kWarpsFwd), kWarpsFwd * 32, smem, st>>>(p);
+  prof_begin(name, st);
+  nsa_token_kernel<kDq><<<static_cast<unsigned>((items + warps - 1) / warps), warps * 32, smem, st>>>(tk, tv, p);
   prof_end(st);
   return cudaGetLastError();
+}
+
+cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st) {
+  return nsa_token_launch<false>(a, make_params(a), "nsa_fwd", st);
 }
 
 cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st) {
@@ -571,17 +651,7 @@ cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st) {
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const long long items = static_cast<long long>(a.N2) * a.T * p.head_tiles;
-  if (items > 0) {
-    const int smem = kWarpsFwd * 2 * 2 * kChunk * 256;
-    if ((e = cudaFuncSetAttribute(nsa_token_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-        cudaSuccess)
-      return e;
-    prof_begin("nsa_bwd_dq", st);
-    nsa_token_kernel<true><<<static_cast<unsigned>((items + kWarpsFwd - 1) / kWarpsFwd), kWarpsFwd * 32, smem, st>>>(p);
-    prof_end(st);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+  if ((e = nsa_token_launch<true>(a, p, "nsa_bwd_dq", st)) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
