@@ -255,10 +255,11 @@ bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
   const int units = p->B * p->N1 * nqb;
-  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(WsHeader), st);
   if (e == cudaSuccess) e = bsa_kv_lists(p->block_mask, units, nkb, w.counts, w.row_ptr, w.col, st);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   BsaFwdArgs a;
+  a.next_unit = &reinterpret_cast<WsHeader*>(w.status)->next_fwd;
   a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.S_q = p->S_q; a.S_kv = p->S_kv;
   a.bx = p->block_x; a.by = p->block_y; a.nqb = nqb; a.nkb = nkb;
   a.mask_mode = p->mask_mode; a.win_left = p->win_left; a.win_right = p->win_right; a.scale = p->scale;

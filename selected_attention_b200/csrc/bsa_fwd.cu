@@ -1,20 +1,27 @@
 // Block-sparse attention forward on tcgen05 (BlockSparseAttentionGrad page, forward formula):
 //   Out = softmax(Mask(scale * Q K_sparse^T, atten_mask)) V_sparse,   LSE = m + ln(l)
-// One CTA per unit (b, h, q block): 128 query rows against the KV blocks the unit's
-// BlockSparseMask row selects (CSR lists from metadata.cu).
+// A unit is (b, h, q block): 128 query rows against the KV blocks its BlockSparseMask row selects
+// (CSR lists from metadata.cu).  The kernel is persistent: one CTA per SM takes units from a
+// device counter (head-major, longest q block of each head first) until none is left, so the
+// next unit's Q load and first score tiles overlap the current unit's epilogue.  Every unit is
+// computed whole by one CTA in list order, so results do not depend on the assignment.
 //
 // Warp roles (320 threads):
 //   warps 0-7  softmax: warp w reads TMEM lane quarter w % 4 (query rows 32*(w%4) .. +31) and the
 //              column half w / 4 of each S tile, so each row is shared by two threads that
 //              exchange their partial row max through shared memory.  They mask, keep the
-//              running max/sum, rescale their half of O in TMEM when needed, and write P (bf16)
-//              back over the consumed S columns, where it feeds O += P V as the MMA's A operand.
-//   warp 8     TMA producer: Q once, then the K tiles of the selected blocks into a 3-stage ring
-//              and the V tiles into a 2-stage ring.  A K stage is released as soon as its
-//              S = Q K^T has run, a V stage after its O += P V, so the next loads start early.
+//              running max/sum, rescale their half of O in TMEM when needed, write P (bf16)
+//              back over the consumed S columns (the A operand of O += P V), and write the
+//              unit's Out and LSE.
+//   warp 8     scheduler and TMA producer: takes the next unit, hands it to the other warps
+//              through a small ring in shared memory, then loads Q (once the previous unit's
+//              last S has read the old Q), the K tiles into a 3-stage ring and the V tiles into
+//              a 2-stage ring.  A K stage is released when its S = Q K^T has run, a V stage
+//              after its O += P V.
 //   warp 9     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
-//              O += P_j V_j into the TMEM O accumulator.  S_{j+1} is issued before waiting for
-//              P_j, so the tensor core computes the next scores while softmax runs.
+//              O += P_j V_j into the TMEM O accumulator.  Within a unit S_{j+1} is issued before
+//              waiting for P_j; the next unit's first S is issued right after the last O += P V.
+// Tile counters run across units, so rings, S buffers and barrier phases carry over.
 // The row max is taken on the raw scores (scale > 0 is required by the host checks), so each
 // probability costs one fused multiply-add (packed in pairs) and one exp2.
 // Every wait is bounded (sa_common.cuh); on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
@@ -35,30 +42,49 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr int kKStages = 3, kVStages = 2;
+constexpr int kSched = 4;  // unit ring between the scheduler and the other warps
 
 template <int BN>
 struct __align__(1024) FwdSmem {
   uint8_t q[2][kBM * 128];            // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
   uint8_t k[kKStages][2][BN * 128];   // [stage][sub-tile] K rows of one KV block
   uint8_t v[kVStages][2][BN * 128];   // [stage][sub-tile] V rows
-  float red[2][2][kBM];               // [tile parity][column half][row]: partial row max / row sum
-  uint64_t bar_q;
+  float red[2][2][kBM];               // [tile parity][column half][row]: partial row max
+  float red_l[2][2][kBM];             // [unit parity][column half][row]: partial row sum
+  int32_t sched[kSched];              // unit ring (-1: no more units)
+  uint64_t bar_q, bar_q_empty;
   uint64_t bar_k[kKStages], bar_k_empty[kKStages], bar_v[kVStages], bar_v_empty[kVStages], bar_s_full[2];
   uint64_t bar_p_full, bar_o_done;
-  uint64_t bar_done;              // one phase: the last O += P V has completed
-  uint64_t bar_pair[4];           // the two softmax warps of each TMEM lane quarter
+  uint64_t bar_done;                  // one phase per non-empty unit: its last O += P V has completed
+  uint64_t bar_sched_full[kSched], bar_sched_empty[kSched];
+  uint64_t bar_pair[4];               // the two softmax warps of each TMEM lane quarter
   uint32_t tmem_base;
 };
 
 struct FwdParams {
-  int B, N1, N2, S_q, S_kv, bx, by, nqb, mask_mode, win_left, win_right;
+  int B, N1, N2, S_q, S_kv, bx, by, nqb, mask_mode, win_left, win_right, units;
   float scale_log2;
   const int32_t* row_ptr;
   const int32_t* col;
   __nv_bfloat16* out;
   float* lse;
+  int32_t* next_unit;  // scheduler counter, zero at launch
   uint32_t* status;
 };
+
+// Unit number i of the schedule -> (b*N1 + h, q block): head-major, latest q block first.
+struct UnitInfo {
+  int bh, qb, rp, n;
+};
+__device__ __forceinline__ UnitInfo unit_info(const FwdParams& prm, int i) {
+  UnitInfo u;
+  u.bh = i / prm.nqb;
+  u.qb = prm.nqb - 1 - i % prm.nqb;
+  const int unit = u.bh * prm.nqb + u.qb;
+  u.rp = prm.row_ptr[unit];
+  u.n = prm.row_ptr[unit + 1] - u.rp;
+  return u;
+}
 
 // Exchange point of the two softmax warps that share a TMEM lane quarter: an mbarrier of 64
 // arrivals with a bounded wait (a plain bar.sync could not give up if the partner stopped early).
@@ -81,21 +107,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kHalf = BN / 2;  // S columns per softmax thread
   extern __shared__ uint8_t smem_raw[];
   FwdSmem<BN>& s = *reinterpret_cast<FwdSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // head-major, longest (latest) Q blocks first
-  const int bh = blockIdx.x / prm.nqb;
-  const int qb = prm.nqb - 1 - static_cast<int>(blockIdx.x % prm.nqb);
-  const int b = bh / prm.N1, h = bh % prm.N1;
-  const int g = h / (prm.N1 / prm.N2);
-  const int unit = bh * prm.nqb + qb;
-  const int rp = prm.row_ptr[unit];
-  const int n = prm.row_ptr[unit + 1] - rp;
-  const int q_row0 = bh * prm.S_q + qb * prm.bx;
-  const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
 
   if (tid == 0) {
     mbar_init(&s.bar_q, 1);
+    mbar_init(&s.bar_q_empty, 1);
     for (int i = 0; i < kKStages; ++i) {
       mbar_init(&s.bar_k[i], 1);
       mbar_init(&s.bar_k_empty[i], 1);
@@ -108,6 +124,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.bar_p_full, kSoftmaxWarps * 32);
     mbar_init(&s.bar_o_done, 1);
     mbar_init(&s.bar_done, 1);
+    for (int i = 0; i < kSched; ++i) {
+      mbar_init(&s.bar_sched_full[i], 1);
+      mbar_init(&s.bar_sched_empty[i], 1 + kSoftmaxWarps * 32);
+    }
     for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
@@ -120,62 +140,82 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
+  // the k-th unit of this CTA from the ring (consumers); -1 when the work is done or on timeout
+  auto next_from_ring = [&](int k) -> int {
+    const int slot = k % kSched;
+    if (!mbar_wait(&s.bar_sched_full[slot], (k / kSched) & 1, prm.status)) return -1;
+    const int u = *reinterpret_cast<volatile int32_t*>(&s.sched[slot]);
+    mbar_arrive(&s.bar_sched_empty[slot]);
+    return u;
+  };
+
   if (warp == kSoftmaxWarps) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && n > 0) {
+    // ------------------------------------------------------------------ scheduler + TMA producer
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&s.bar_q, 2 * kBM * 128);
-      tma_load_2d(s.q[0], &tm_q, &s.bar_q, 0, q_row0);
-      tma_load_2d(s.q[1], &tm_q, &s.bar_q, 64, q_row0);
-      // K runs up to kKStages tiles ahead, V up to kVStages; each waits only for its own stage.
-      int issued_k = 0, issued_v = 0;
+      int jk = 0, jv = 0, qcount = 0;  // K / V tiles issued, Q loads issued (this CTA)
       bool ok = true;
-      for (int j = 0; ok && j < n; ++j) {
-        const int row = kv_row0 + prm.col[rp + j] * prm.by;
-        const int sk = j % kKStages, uk = j / kKStages;
-        if (j >= kKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
-        mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
-        tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
-        tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
-        issued_k = j + 1;
-        // V of tile j - (kKStages - kVStages) so that V trails K by one stage
-        const int jv = j - (kKStages - kVStages);
-        if (jv >= 0) {
-          const int sv = jv % kVStages, uv = jv / kVStages;
-          if (jv >= kVStages && !(ok = mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status))) break;
-          const int vrow = kv_row0 + prm.col[rp + jv] * prm.by;
-          mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
-          tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
-          tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
-          issued_v = jv + 1;
-        }
-      }
-      for (int jv = issued_v; ok && jv < n; ++jv) {
+      auto load_v = [&](int rp, int kv_row0, int j) -> bool {  // V of the unit's tile j (global jv)
         const int sv = jv % kVStages, uv = jv / kVStages;
-        if (jv >= kVStages && !(ok = mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status))) break;
-        const int vrow = kv_row0 + prm.col[rp + jv] * prm.by;
+        if (jv >= kVStages && !mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status)) return false;
+        const int vrow = kv_row0 + prm.col[rp + j] * prm.by;
         mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
         tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
         tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
-        issued_v = jv + 1;
+        ++jv;
+        return true;
+      };
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kSched;
+        if (k >= kSched && !(ok = mbar_wait(&s.bar_sched_empty[slot], ((k / kSched) - 1) & 1, prm.status))) break;
+        int i = atomicAdd(prm.next_unit, 1);
+        if (i >= prm.units) i = -1;
+        s.sched[slot] = i;
+        mbar_arrive(&s.bar_sched_full[slot]);  // release: the ring entry is visible to its readers
+        if (i < 0) break;
+        const UnitInfo u = unit_info(prm, i);
+        if (u.n == 0) continue;
+        const int b = u.bh / prm.N1, h = u.bh % prm.N1;
+        const int g = h / (prm.N1 / prm.N2);
+        const int q_row0 = u.bh * prm.S_q + u.qb * prm.bx;
+        const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
+        // Q: the previous unit's last S = Q K^T must have read the old Q
+        if (qcount > 0 && !(ok = mbar_wait(&s.bar_q_empty, (qcount - 1) & 1, prm.status))) break;
+        mbar_arrive_expect_tx(&s.bar_q, 2 * kBM * 128);
+        tma_load_2d(s.q[0], &tm_q, &s.bar_q, 0, q_row0);
+        tma_load_2d(s.q[1], &tm_q, &s.bar_q, 64, q_row0);
+        ++qcount;
+        // K runs up to kKStages tiles ahead, V trails K by one tile
+        for (int j = 0; ok && j < u.n; ++j) {
+          const int row = kv_row0 + prm.col[u.rp + j] * prm.by;
+          const int sk = jk % kKStages, uk = jk / kKStages;
+          if (jk >= kKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
+          mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
+          tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
+          tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
+          ++jk;
+          if (j >= kKStages - kVStages) ok = load_v(u.rp, kv_row0, j - (kKStages - kVStages));
+        }
+        for (int j = u.n - (kKStages - kVStages); ok && j < u.n; ++j)
+          if (j >= 0) ok = load_v(u.rp, kv_row0, j);
       }
       // do not leave the CTA with copies in flight
-      for (int j = (issued_k > kKStages ? issued_k - kKStages : 0); j < issued_k; ++j)
+      for (int j = (jk > kKStages ? jk - kKStages : 0); j < jk; ++j)
         mbar_wait(&s.bar_k[j % kKStages], (j / kKStages) & 1, prm.status);
-      for (int j = (issued_v > kVStages ? issued_v - kVStages : 0); j < issued_v; ++j)
+      for (int j = (jv > kVStages ? jv - kVStages : 0); j < jv; ++j)
         mbar_wait(&s.bar_v[j % kVStages], (j / kVStages) & 1, prm.status);
-      mbar_wait(&s.bar_q, 0, prm.status);
+      if (qcount > 0) mbar_wait(&s.bar_q, (qcount - 1) & 1, prm.status);
     }
   } else if (warp == kSoftmaxWarps + 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
       const uint32_t idesc_o = idesc_bf16_f32(kBM, kD, false, true);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1, sk = j % kKStages;
-        if (!mbar_wait(&s.bar_k[sk], (j / kKStages) & 1, prm.status)) return false;
+      auto issue_s = [&](int J) -> bool {  // global tile J
+        const int st = J & 1, sk = J % kKStages;
+        if (!mbar_wait(&s.bar_k[sk], (J / kKStages) & 1, prm.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + (st ? kColS1 : kColS0);
 #pragma unroll
@@ -188,180 +228,208 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(&s.bar_k_empty[sk]);
         return true;
       };
-      bool ok = mbar_wait(&s.bar_q, 0, prm.status);
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(&s.bar_p_full, j & 1, prm.status))) break;
-        const int st = j & 1, sv = j % kVStages;
-        if (!(ok = mbar_wait(&s.bar_v[sv], (j / kVStages) & 1, prm.status))) break;
-        tc_fence_after();
-        const uint32_t p_col = st ? kColS1 : kColS0;
+      int J0 = 0, qcount = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int i = next_from_ring(k);
+        if (i < 0) break;
+        const UnitInfo u = unit_info(prm, i);
+        if (u.n == 0) continue;
+        if (!(ok = mbar_wait(&s.bar_q, qcount & 1, prm.status))) break;
+        ++qcount;
+        if (!(ok = issue_s(J0))) break;
+        if (u.n == 1) tc_commit(&s.bar_q_empty);
+        for (int j = 0; ok && j < u.n; ++j) {
+          const int J = J0 + j;
+          if (j + 1 < u.n) {
+            if (!(ok = issue_s(J + 1))) break;
+            if (j + 2 == u.n) tc_commit(&s.bar_q_empty);  // the unit's last read of Q
+          }
+          if (!(ok = mbar_wait(&s.bar_p_full, J & 1, prm.status))) break;
+          const int st = J & 1, sv = J % kVStages;
+          if (!(ok = mbar_wait(&s.bar_v[sv], (J / kVStages) & 1, prm.status))) break;
+          tc_fence_after();
+          const uint32_t p_col = st ? kColS1 : kColS0;
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(smem_u32(s.v[sv][0]) + ks * 2048, BN * 128, 1024);
-          mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t bd = sdesc_sw128(smem_u32(s.v[sv][0]) + ks * 2048, BN * 128, 1024);
+            mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(&s.bar_o_done);
+          tc_commit(&s.bar_v_empty[sv]);
         }
-        tc_commit(&s.bar_o_done);
-        tc_commit(&s.bar_v_empty[sv]);
+        if (ok) tc_commit(&s.bar_done);
+        J0 += u.n;
       }
-      if (ok) tc_commit(&s.bar_done);
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
     const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
-    const int qpos = qb * prm.bx + r;
-    const bool row_valid = r < prm.bx && qpos < prm.S_q;
-    // visible key interval [lo, hi] for this row (mask modes 0/2/3/4)
-    int lo = 0, hi = prm.S_kv - 1;
-    const int qq = qpos + prm.S_kv - prm.S_q;
-    if (prm.mask_mode == 2) hi = min(hi, qpos);
-    else if (prm.mask_mode == 3) hi = min(hi, qq);
-    else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
-    if (!row_valid) { lo = 1; hi = 0; }
-
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t o_col = kColO + hf * (kD / 2);  // this thread's half of the O row
-    float m = -INFINITY, l = 0.f;                  // l: partial sum over this thread's columns
-    int exchanges = 0;
+    int exchanges = 0, J0 = 0, done_count = 0;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int st = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (j >> 1) & 1, prm.status));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t s_col = st ? kColS1 : kColS0;
-      const int kpos0 = prm.col[rp + j] * prm.by + hf * kHalf;
-      float x[kHalf];  // raw scores
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + s_col + hf * kHalf + c, rr);
-        tmem_ld_wait(rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(rr[i]);
-      }
-      const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
-      if (!full) {
-#pragma unroll
-        for (int c = 0; c < kHalf; ++c) {
-          const int kp = kpos0 + c;
-          if (kp < lo || kp > hi) x[c] = -INFINITY;
-        }
-      }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 4) {
-        mx4[0] = fmaxf(mx4[0], x[c]);
-        mx4[1] = fmaxf(mx4[1], x[c + 1]);
-        mx4[2] = fmaxf(mx4[2], x[c + 2]);
-        mx4[3] = fmaxf(mx4[3], x[c + 3]);
-      }
-      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      // row max = max of the two halves; the barrier also orders both threads' S reads before
-      // either writes P over the S columns
-      s.red[st][hf][r] = mx;
-      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
-      if (!ok) break;
-      mx = fmaxf(mx, s.red[st][hf ^ 1][r]) * prm.scale_log2;  // log2 units of the scaled score
-      // Lazy rescaling: the exponent reference m only moves when the row max exceeds it by more
-      // than 8 (p <= 2^8 otherwise); numerator and l share the same reference, so the final
-      // O / l is unchanged.  Only then must the previous O += P V have landed.
-      float m_new = m;
-      bool need = false;
-      if (mx > m + 8.f) {
-        need = (m != -INFINITY);
-        m_new = mx;
-      }
-      if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
-        // O += P_{j-1} V_{j-1} is o_done phase j-1.  S_j landed after every earlier MMA (one
-        // commit covers all prior MMAs), so phase j-2 is complete and j cannot be: the barrier is
-        // in phase j-1 or j, which a parity wait tells apart.
-        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (j - 1) & 1, prm.status));
+    for (int k = 0; ok; ++k) {
+      const int i = __shfl_sync(0xffffffffu, next_from_ring(k), 0);
+      if (i < 0) break;
+      const UnitInfo u = unit_info(prm, i);
+      const int n = u.n, rp = u.rp, qb = u.qb;
+      const int q_row0 = u.bh * prm.S_q + qb * prm.bx;
+      const int qpos = qb * prm.bx + r;
+      const bool row_valid = r < prm.bx && qpos < prm.S_q;
+      // visible key interval [lo, hi] for this row (mask modes 0/2/3/4)
+      int lo = 0, hi = prm.S_kv - 1;
+      const int qq = qpos + prm.S_kv - prm.S_q;
+      if (prm.mask_mode == 2) hi = min(hi, qpos);
+      else if (prm.mask_mode == 3) hi = min(hi, qq);
+      else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
+      if (!row_valid) { lo = 1; hi = 0; }
+      float m = -INFINITY, l = 0.f;  // l: partial sum over this thread's columns
+      for (int j = 0; j < n; ++j) {
+        const int J = J0 + j;
+        const int st = J & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (J >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
-        const float alpha = need ? ex2(m - m_new) : 1.f;
-        l *= alpha;
+        const uint32_t s_col = st ? kColS1 : kColS0;
+        const int kpos0 = prm.col[rp + j] * prm.by + hf * kHalf;
+        float x[kHalf];  // raw scores
 #pragma unroll
-        for (int c = 0; c < kD / 2; c += 32) {
+        for (int c = 0; c < kHalf; c += 32) {
           uint32_t rr[32];
-          tmem_ld32(tmem + lane_base + o_col + c, rr);
+          tmem_ld32(tmem + lane_base + s_col + hf * kHalf + c, rr);
           tmem_ld_wait(rr);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(tmem + lane_base + o_col + c, rr);
+          for (int i2 = 0; i2 < 32; ++i2) x[c + i2] = __uint_as_float(rr[i2]);
+        }
+        const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
+        if (!full) {
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c) {
+            const int kp = kpos0 + c;
+            if (kp < lo || kp > hi) x[c] = -INFINITY;
+          }
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 4) {
+          mx4[0] = fmaxf(mx4[0], x[c]);
+          mx4[1] = fmaxf(mx4[1], x[c + 1]);
+          mx4[2] = fmaxf(mx4[2], x[c + 2]);
+          mx4[3] = fmaxf(mx4[3], x[c + 3]);
+        }
+        float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        // row max = max of the two halves; the barrier also orders both threads' S reads before
+        // either writes P over the S columns
+        s.red[st][hf][r] = mx;
+        ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+        if (!ok) break;
+        mx = fmaxf(mx, s.red[st][hf ^ 1][r]) * prm.scale_log2;  // log2 units of the scaled score
+        // Lazy rescaling: the exponent reference m only moves when the row max exceeds it by
+        // more than 8 (p <= 2^8 otherwise); numerator and l share the same reference, so the
+        // final O / l is unchanged.  Only then must the previous O += P V have landed.
+        float m_new = m;
+        bool need = false;
+        if (mx > m + 8.f) {
+          need = (m != -INFINITY);
+          m_new = mx;
+        }
+        if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
+          // O += P_{J-1} V_{J-1} is o_done phase J-1 (need implies j > 0).  S_J landed after every
+          // earlier MMA, so phase J-2 is complete and J cannot be: a parity wait tells them apart.
+          ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (J - 1) & 1, prm.status));
+          if (!ok) break;
+          tc_fence_after();
+          const float alpha = need ? ex2(m - m_new) : 1.f;
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < kD / 2; c += 32) {
+            uint32_t rr[32];
+            tmem_ld32(tmem + lane_base + o_col + c, rr);
+            tmem_ld_wait(rr);
+#pragma unroll
+            for (int i2 = 0; i2 < 32; ++i2) rr[i2] = __float_as_uint(__uint_as_float(rr[i2]) * alpha);
+            tmem_st32(tmem + lane_base + o_col + c, rr);
+          }
+          tmem_st_wait();
+        }
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        // p = 2^(s * scale * log2(e) - m): one packed fma per pair, one exp2 per element
+        const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2), nm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc0 = 0, acc1 = 0;  // packed partial row sums (0 bits == 0.0f, 0.0f)
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 32) {
+          uint32_t hv[16];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) {
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(x[c + 2 * i2], x[c + 2 * i2 + 1]), sc2, nm2), t0, t1);
+            const float e0 = ex2(t0), e1 = ex2(t1);
+            if (i2 & 1) acc1 = f2_add(acc1, f2_pack(e0, e1));
+            else acc0 = f2_add(acc0, f2_pack(e0, e1));
+            hv[i2] = pack_bf16(e0, e1);
+          }
+          // packed pairs: element column e -> TMEM column e/2 of the S buffer
+          tmem_st16(tmem + lane_base + s_col + (hf * kHalf + c) / 2, hv);
         }
         tmem_st_wait();
-      }
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      // p = 2^(s * scale * log2(e) - m): one packed fma per pair, one exp2 per element
-      const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2), nm2 = f2_pack(-m_use, -m_use);
-      uint64_t acc0 = 0, acc1 = 0;  // packed partial row sums (0 bits == 0.0f, 0.0f)
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 32) {
-        uint32_t hv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float t0, t1;
-          f2_unpack(f2_fma(f2_pack(x[c + 2 * i], x[c + 2 * i + 1]), sc2, nm2), t0, t1);
-          const float e0 = ex2(t0), e1 = ex2(t1);
-          if (i & 1) acc1 = f2_add(acc1, f2_pack(e0, e1));
-          else acc0 = f2_add(acc0, f2_pack(e0, e1));
-          hv[i] = pack_bf16(e0, e1);
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(acc0, a0, a1);
+          f2_unpack(acc1, b0, b1);
+          l += (a0 + a1) + (b0 + b1);
         }
-        // packed pairs: element column e -> TMEM column e/2 of the S buffer
-        tmem_st16(tmem + lane_base + s_col + (hf * kHalf + c) / 2, hv);
+        m = m_new;
+        tc_fence_before();
+        mbar_arrive(&s.bar_p_full);
       }
-      tmem_st_wait();
-      {
-        float a0, a1, b0, b1;
-        f2_unpack(acc0, a0, a1);
-        f2_unpack(acc1, b0, b1);
-        l += (a0 + a1) + (b0 + b1);
+      if (!ok) break;
+      // ---- epilogue.  bar_done has one phase per non-empty unit and this thread has waited on
+      // every earlier one, so a parity wait is exact (o_done is not: lazy rescaling skips phases).
+      bool have_o = n > 0;
+      if (have_o) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, done_count & 1, prm.status));
+        ++done_count;
+        if (!ok) break;
+        tc_fence_after();
       }
-      m = m_new;
+      // full row sum from the two halves (slot by unit parity: the partner may still be reading
+      // the previous unit's entry when this thread writes the next one)
+      s.red_l[k & 1][hf][r] = l;
+      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+      if (!ok) break;
+      l += s.red_l[k & 1][hf ^ 1][r];
+      const bool any = have_o && l > 0.f;
+      const float inv_l = any ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = prm.out + static_cast<size_t>(q_row0 + r) * kD + hf * (kD / 2);
+#pragma unroll
+      for (int c = 0; c < kD / 2; c += 32) {
+        uint32_t rr[32];
+        if (have_o) {  // warp-uniform: every lane joins the collective load
+          tmem_ld32(tmem + lane_base + o_col + c, rr);
+          tmem_ld_wait(rr);
+        } else {
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2) rr[i2] = 0u;
+        }
+        if (row_valid) {
+#pragma unroll
+          for (int i2 = 0; i2 < 32; i2 += 8) {
+            uint4 pk;
+            pk.x = pack_bf16(__uint_as_float(rr[i2 + 0]) * inv_l, __uint_as_float(rr[i2 + 1]) * inv_l);
+            pk.y = pack_bf16(__uint_as_float(rr[i2 + 2]) * inv_l, __uint_as_float(rr[i2 + 3]) * inv_l);
+            pk.z = pack_bf16(__uint_as_float(rr[i2 + 4]) * inv_l, __uint_as_float(rr[i2 + 5]) * inv_l);
+            pk.w = pack_bf16(__uint_as_float(rr[i2 + 6]) * inv_l, __uint_as_float(rr[i2 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + c + i2) = pk;
+          }
+        }
+      }
+      if (row_valid && hf == 0) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
+      // O has been read: the next unit's first O += P V waits for P, which comes after this
       tc_fence_before();
-      mbar_arrive(&s.bar_p_full);
+      J0 += n;
     }
-    // ---- epilogue.  Not a parity wait on o_done: with lazy rescaling this thread may not have
-    // observed the earlier o_done phases, and a parity wait can only tell one phase from the next.
-    bool have_o = ok && n > 0;
-    if (have_o) {
-      have_o = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, 0, prm.status));
-      tc_fence_after();
-    }
-    // full row sum from the two halves, through the reduction slot of parity n & 1 (the last
-    // max exchange used parity (n - 1) & 1, and both threads passed the exchange before it)
-    s.red[n & 1][hf][r] = l;
-    if (ok) have_o = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status)) && have_o;
-    l += s.red[n & 1][hf ^ 1][r];
-    const bool any = have_o && l > 0.f;
-    const float inv_l = any ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = prm.out + static_cast<size_t>(q_row0 + r) * kD + hf * (kD / 2);
-#pragma unroll
-    for (int c = 0; c < kD / 2; c += 32) {
-      uint32_t rr[32];
-      if (have_o) {  // warp-uniform: every lane joins the collective load
-        tmem_ld32(tmem + lane_base + o_col + c, rr);
-        tmem_ld_wait(rr);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rr[i] = 0u;
-      }
-      if (row_valid) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 pk;
-          pk.x = pack_bf16(__uint_as_float(rr[i + 0]) * inv_l, __uint_as_float(rr[i + 1]) * inv_l);
-          pk.y = pack_bf16(__uint_as_float(rr[i + 2]) * inv_l, __uint_as_float(rr[i + 3]) * inv_l);
-          pk.z = pack_bf16(__uint_as_float(rr[i + 4]) * inv_l, __uint_as_float(rr[i + 5]) * inv_l);
-          pk.w = pack_bf16(__uint_as_float(rr[i + 6]) * inv_l, __uint_as_float(rr[i + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(orow + c + i) = pk;
-        }
-      }
-    }
-    if (row_valid && hf == 0) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
   }
   tc_fence_before();
   __syncthreads();
@@ -379,14 +447,18 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   FwdParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.S_q = a.S_q; p.S_kv = a.S_kv; p.bx = a.bx; p.by = a.by;
   p.nqb = a.nqb; p.mask_mode = a.mask_mode; p.win_left = a.win_left; p.win_right = a.win_right;
+  p.units = a.B * a.N1 * a.nqb;
   p.scale_log2 = a.scale * kLog2e;
   p.row_ptr = a.row_ptr; p.col = a.col;
-  p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse; p.status = a.status;
+  p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse; p.next_unit = a.next_unit; p.status = a.status;
   const size_t smem = sizeof(FwdSmem<BN>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int grid = a.B * a.N1 * a.nqb;
-  if (grid == 0) return cudaSuccess;
+  if (p.units == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.units < sms ? p.units : sms;  // persistent: one CTA per SM
   prof_begin("bsa_fwd", st);
   bsa_fwd_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
   prof_end(st);

@@ -60,7 +60,15 @@ struct BsaFwdArgs {
   const int32_t* col;
   void* out;
   float* lse;
+  int32_t* next_unit;  // persistent-kernel work counter, zeroed before the launch
   uint32_t* status;
+};
+
+// The first 256 bytes of every workspace: the device status word, then the work counters of the
+// persistent kernels (zeroed with the status word before each call).
+struct WsHeader {
+  uint32_t status;
+  int32_t next_fwd, next_bwd_kv, next_bwd_q;
 };
 cudaError_t bsa_fwd_launch(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st);
 
