@@ -288,7 +288,7 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
   carve_bsa_bwd(p, workspace, &w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
-  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(WsHeader), st);
   if (e == cudaSuccess) e = bsa_kv_lists(p->block_mask, p->B * p->N1 * nqb, nkb, w.counts, w.row_ptr, w.col, st);
   if (e == cudaSuccess)
     e = bsa_q_lists(p->block_mask, p->B, p->N1, p->N2, nqb, nkb, w.maskT, w.t_counts, w.t_row_ptr, w.t_col, st);
@@ -299,6 +299,8 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
   a.mask_mode = p->mask_mode; a.win_left = p->win_left; a.win_right = p->win_right; a.scale = p->scale;
   a.row_ptr = w.row_ptr; a.col = w.col; a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;
   a.dvec = w.dvec; a.lse2 = w.lse2; a.dq = dq; a.dk = dk; a.dv = dv; a.status = w.status;
+  a.next_kv = &reinterpret_cast<WsHeader*>(w.status)->next_bwd_kv;
+  a.next_q = &reinterpret_cast<WsHeader*>(w.status)->next_bwd_q;
   return cuda_status(bsa_bwd_launch(a, q, k, v, out, dout, lse, st));
 }
 bsa_status nsa_selected_fwd_workspace_size(const bsa_params* p, size_t* bytes) {

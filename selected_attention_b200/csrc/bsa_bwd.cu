@@ -27,8 +27,9 @@ constexpr int kThreads = (kVecWarps + 2) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------------------------------------
-// preprocess: D_i = sum_d dOut_id Out_id ; L2_i = LSE_i * log2(e)  (+inf where the row has no key
-// or the tile row is padding, which makes exp2(s - L2) = 0 there)
+// preprocess: -D_i = -sum_d dOut_id Out_id ; -L2_i = -LSE_i * log2(e)  (-inf where the row has no
+// key or the tile row is padding, which makes exp2(s + (-L2)) = 0 there).  Stored negated so that
+// P = exp2(s * scale * log2(e) + (-L2)) is one fused multiply-add and dS = P * (dP + (-D)).
 // ------------------------------------------------------------------------------------------------
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
                                 const float* __restrict__ lse, int S_q, int bx, int nqb, long long n_rows,
@@ -61,11 +62,11 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __n
   d += __shfl_xor_sync(0xffffffffu, d, 2);
   d += __shfl_xor_sync(0xffffffffu, d, 4);
   if (part == 0) {
-    dvec[row] = valid ? d : 0.f;
-    float l2 = INFINITY;
+    dvec[row] = valid ? -d : 0.f;
+    float l2 = -INFINITY;
     if (valid) {
       const float l = lse[static_cast<size_t>(bh) * S_q + qpos];
-      l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;
+      l2 = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     }
     lse2[row] = l2;
   }
@@ -74,10 +75,11 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __n
 struct BwdParams {
   int B, N1, N2, S_q, S_kv, bx, by, nqb, nkb, mask_mode, win_left, win_right;
   float scale, scale_log2;
+  int32_t* next_unit;      // persistent-kernel work counter, zero at launch
   const int32_t* row_ptr;  // KV lists (Q-major pass) or transposed lists (KV-major pass)
   const int32_t* col;
-  const float* dvec;       // [B*N1*nqb*128]
-  const float* lse2;
+  const float* dvec;       // [B*N1*nqb*128]: -softmax_grad per padded query row
+  const float* lse2;       // -LSE*log2(e) per padded query row (-inf: no key or padding)
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -107,63 +109,86 @@ __device__ __forceinline__ bool pair_sync(uint64_t* bar, int& exchanges, uint32_
   return ok;
 }
 
-// Split x into bf16 hi + lo (x ~= hi + lo to about 2^-17 relative): the dK and dQ products run as
-// two MMAs, hi then lo, so dS enters the tensor cores with ~16 significant bits.
-__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  hi = pack_bf16(x0, x1);
-  lo = pack_bf16(x0 - bf16lo(hi), x1 - bf16hi(hi));
+// Split a packed pair x into bf16 hi + lo (x ~= hi + lo to about 2^-17 relative; lo = x - hi by
+// one packed fused multiply-add): the products that take P and dS run as two MMAs, hi then lo,
+// so those operands enter the tensor cores with ~16 significant bits.
+__device__ __forceinline__ void split_pack2(uint64_t x, uint32_t& hi, uint32_t& lo) {
+  float a, b;
+  f2_unpack(x, a, b);
+  hi = pack_bf16(a, b);
+  float la, lb;
+  f2_unpack(f2_fma(f2_pack(bf16lo(hi), bf16hi(hi)), f2_pack(-1.f, -1.f), x), la, lb);
+  lo = pack_bf16(la, lb);
 }
 
 // ------------------------------------------------------------------------------------------------
-// KV-major pass: dK, dV
-// TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,384) | dK [384,512).
-// After the P/dS warpgroup has read S^T and dP^T, it writes back the bf16 MMA A operands over
-// the consumed columns: P^T hi/lo -> S^T[0,64)/[64,128), dS^T hi/lo -> dP^T[0,64)/[64,128).
+// KV-major pass: dK, dV.  Persistent: one CTA per SM takes KV blocks (b, g, kb) from a device
+// counter (head-major, earliest block first: with causal masks those have the longest lists) and
+// walks each block's transposed list.  Every entry (a 128-row Q tile of one of the group's heads)
+// runs as two 64-row halves, so the element-wise work on one half overlaps the tensor-core work of
+// the neighbouring halves:
+//   TMEM columns: half buffers 0 [0,128) and 1 [128,256), each S^T [0,64) | dP^T [64,128) of one
+//   half (128 keys x 64 query rows); dV [256,384), dK [384,512).  After the 8 element-wise warps
+//   have read S^T and dP^T of a half they write the bf16 A operands over them: P^T hi -> [0,32),
+//   lo -> [32,64), dS^T hi -> [64,96), lo -> [96,128) (64 query rows -> 32 packed columns).
+//   Shared memory: the block's K and V tiles, and a 4-stage ring of half entries (64 rows of Q
+//   and dO with their D and LSE*log2e values), so loads run two half-steps ahead.
+//   MMA order per half x: dV += P^T dO, dK += dS^T Q (hi, lo), then S^T / dP^T of half x + 2
+//   into the buffer just consumed.
 // ------------------------------------------------------------------------------------------------
+constexpr int kHalfRows = 64;
+constexpr int kKvRing = 4;
+constexpr int kSchedKv = 4;
+// warps: 0-7 element-wise, 8 scheduler + TMA, 9 issues dV / dK products, 10 issues S^T / dP^T.
+// Two issuing threads: tcgen05.mma issue blocks while the tensor pipe's queue is full, so with one
+// thread the next half's products would wait behind the previous half's score MMAs.
+constexpr int kKvThreads = (kVecWarps + 3) * 32;
+
 struct __align__(1024) KvSmem {
-  uint8_t k[2][kT * 128];        // K tile [128 keys][64 d] x 2
+  uint8_t k[2][kT * 128];                 // K tile [128 keys][64 d] x 2
   uint8_t v[2][kT * 128];
-  uint8_t q[2][2][kT * 128];     // [stage][sub-tile] Q tile [128 queries][64 d]
-  uint8_t dout[2][2][kT * 128];  // [stage][sub-tile] dO tile
-  float lse2[2][kT];             // per Q stage
-  float dvec[2][kT];
-  uint64_t bar_kv, bar_q[2], bar_do[2];
-  uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_done;
-  uint64_t bar_q_empty[2], bar_do_empty[2];
+  uint8_t q[kKvRing][2][kHalfRows * 128];     // [stage][d half] [64 query rows][64 d]
+  uint8_t dout[kKvRing][2][kHalfRows * 128];
+  float lse2[kKvRing][kHalfRows];
+  float dvec[kKvRing][kHalfRows];
+  int32_t sched[kSchedKv];
+  uint64_t bar_kv, bar_kv_empty;
+  uint64_t bar_qdo[kKvRing], bar_qdo_empty[kKvRing];
+  uint64_t bar_sdp_full[2], bar_pds_ready[2], bar_done;
+  uint64_t bar_grads_done[2];  // per half buffer: its products have completed (buffer reusable)
+  uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
   uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
-    bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+__global__ void __launch_bounds__(kKvThreads, 1)
+    bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
                       const BwdParams prm) {
-  constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+  constexpr uint32_t kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   KvSmem& s = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bg = blockIdx.x / prm.nkb;
-  const int kb = static_cast<int>(blockIdx.x % prm.nkb);  // early KV blocks have the longest lists
-  const int b = bg / prm.N2, g = bg % prm.N2;
   const int G = prm.N1 / prm.N2;
-  const int unit = bg * prm.nkb + kb;
-  const int rp = prm.row_ptr[unit];
-  const int n = prm.row_ptr[unit + 1] - rp;
-  const int kv_row0 = bg * prm.S_kv + kb * prm.by;
+  const int units = prm.B * prm.N2 * prm.nkb;
 
   if (tid == 0) {
     mbar_init(&s.bar_kv, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.bar_q[i], 1);
-      mbar_init(&s.bar_do[i], 1);
-      mbar_init(&s.bar_q_empty[i], 1);
-      mbar_init(&s.bar_do_empty[i], 1);
+    mbar_init(&s.bar_kv_empty, 1);
+    for (int i = 0; i < kKvRing; ++i) {
+      mbar_init(&s.bar_qdo[i], 1);
+      mbar_init(&s.bar_qdo_empty[i], 1);
     }
-    mbar_init(&s.bar_s_full, 1);
-    mbar_init(&s.bar_dp_full, 1);
-    mbar_init(&s.bar_p_ready, kVecWarps * 32);
-    mbar_init(&s.bar_ds_ready, kVecWarps * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.bar_sdp_full[i], 1);
+      mbar_init(&s.bar_pds_ready[i], kVecWarps * 32);
+    }
     mbar_init(&s.bar_done, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_grads_done[i], 1);
+    for (int i = 0; i < kSchedKv; ++i) {
+      mbar_init(&s.bar_sched_full[i], 1);
+      mbar_init(&s.bar_sched_empty[i], 2 + kVecWarps * 32);
+    }
     for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
@@ -176,217 +201,274 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  auto entry_rows = [&](int i, int& qrow, int& tile, int& qpos0) {
-    const int e = prm.col[rp + i];
-    const int hl = e / prm.nqb, qb = e % prm.nqb;
+  // unit i -> (b*N2 + g, kv block), its transposed list [rp, rp + n)
+  auto unit_of = [&](int i, int& bg, int& kb, int& rp, int& n) {
+    bg = i / prm.nkb;
+    kb = i % prm.nkb;
+    const int unit = bg * prm.nkb + kb;
+    rp = prm.row_ptr[unit];
+    n = prm.row_ptr[unit + 1] - rp;
+  };
+  // list entry -> first row of its Q tile in the [B*N1*S_q, 128] view, its padded tile index and
+  // the position of its first query row
+  auto entry_rows = [&](int bg, int e_code, int& qrow, int& tile, int& qpos0) {
+    const int b = bg / prm.N2, g = bg % prm.N2;
+    const int hl = e_code / prm.nqb, qb = e_code % prm.nqb;
     const int bh = b * prm.N1 + g * G + hl;
     qrow = bh * prm.S_q + qb * prm.bx;
     tile = bh * prm.nqb + qb;
     qpos0 = qb * prm.bx;
   };
+  auto next_from_ring = [&](int k) -> int {
+    const int slot = k % kSchedKv;
+    if (!mbar_wait(&s.bar_sched_full[slot], (k / kSchedKv) & 1, prm.status)) return -1;
+    const int u = *reinterpret_cast<volatile int32_t*>(&s.sched[slot]);
+    mbar_arrive(&s.bar_sched_empty[slot]);
+    return u;
+  };
 
   if (warp == kVecWarps) {
-    // ------------------------------------------------------------------ producer
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(&s.bar_kv, 4 * kT * 128);
-      tma_load_2d(s.k[0], &tm_k, &s.bar_kv, 0, kv_row0);
-      tma_load_2d(s.k[1], &tm_k, &s.bar_kv, 64, kv_row0);
-      tma_load_2d(s.v[0], &tm_v, &s.bar_kv, 0, kv_row0);
-      tma_load_2d(s.v[1], &tm_v, &s.bar_kv, 64, kv_row0);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int st = i & 1;
-        int qrow, tile, qpos0;
-        entry_rows(i, qrow, tile, qpos0);
-        if (i >= 2 && !mbar_wait(&s.bar_q_empty[st], ((i - 2) >> 1) & 1, prm.status)) break;
-        mbar_arrive_expect_tx(&s.bar_q[st], 2 * kT * 128 + 2 * kT * 4);
-        tma_load_2d(s.q[st][0], &tm_q, &s.bar_q[st], 0, qrow);
-        tma_load_2d(s.q[st][1], &tm_q, &s.bar_q[st], 64, qrow);
-        bulk_load(s.lse2[st], prm.lse2 + static_cast<size_t>(tile) * kT, kT * 4, &s.bar_q[st]);
-        bulk_load(s.dvec[st], prm.dvec + static_cast<size_t>(tile) * kT, kT * 4, &s.bar_q[st]);
-        if (i >= 2 && !mbar_wait(&s.bar_do_empty[st], ((i - 2) >> 1) & 1, prm.status)) {
-          issued = -(i + 1);  // Q issued, dO not
+    // ------------------------------------------------------------------ scheduler + TMA producer
+    if (lane == 0) {
+      int hq = 0, ucount = 0;  // half entries loaded, K/V loads (this CTA)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kSchedKv;
+        if (k >= kSchedKv && !(ok = mbar_wait(&s.bar_sched_empty[slot], ((k / kSchedKv) - 1) & 1, prm.status)))
           break;
+        int i = atomicAdd(prm.next_unit, 1);
+        if (i >= units) i = -1;
+        s.sched[slot] = i;
+        mbar_arrive(&s.bar_sched_full[slot]);
+        if (i < 0) break;
+        int bg, kb, rp, n;
+        unit_of(i, bg, kb, rp, n);
+        if (n == 0) continue;
+        const int kv_row0 = bg * prm.S_kv + kb * prm.by;
+        if (ucount > 0 && !(ok = mbar_wait(&s.bar_kv_empty, (ucount - 1) & 1, prm.status))) break;
+        mbar_arrive_expect_tx(&s.bar_kv, 4 * kT * 128);
+        tma_load_2d(s.k[0], &tm_k, &s.bar_kv, 0, kv_row0);
+        tma_load_2d(s.k[1], &tm_k, &s.bar_kv, 64, kv_row0);
+        tma_load_2d(s.v[0], &tm_v, &s.bar_kv, 0, kv_row0);
+        tma_load_2d(s.v[1], &tm_v, &s.bar_kv, 64, kv_row0);
+        ++ucount;
+        for (int e = 0; ok && e < 2 * n; ++e) {
+          const int h = e & 1;
+          int qrow, tile, qpos0;
+          entry_rows(bg, prm.col[rp + (e >> 1)], qrow, tile, qpos0);
+          const int hs = hq % kKvRing;
+          if (hq >= kKvRing && !(ok = mbar_wait(&s.bar_qdo_empty[hs], ((hq / kKvRing) - 1) & 1, prm.status))) break;
+          mbar_arrive_expect_tx(&s.bar_qdo[hs], 4 * kHalfRows * 128 + 2 * kHalfRows * 4);
+          const int row = qrow + h * kHalfRows;
+          tma_load_2d(s.q[hs][0], &tm_q64, &s.bar_qdo[hs], 0, row);
+          tma_load_2d(s.q[hs][1], &tm_q64, &s.bar_qdo[hs], 64, row);
+          tma_load_2d(s.dout[hs][0], &tm_do64, &s.bar_qdo[hs], 0, row);
+          tma_load_2d(s.dout[hs][1], &tm_do64, &s.bar_qdo[hs], 64, row);
+          const size_t voff = static_cast<size_t>(tile) * kT + h * kHalfRows;
+          bulk_load(s.lse2[hs], prm.lse2 + voff, kHalfRows * 4, &s.bar_qdo[hs]);
+          bulk_load(s.dvec[hs], prm.dvec + voff, kHalfRows * 4, &s.bar_qdo[hs]);
+          ++hq;
         }
-        mbar_arrive_expect_tx(&s.bar_do[st], 2 * kT * 128);
-        tma_load_2d(s.dout[st][0], &tm_do, &s.bar_do[st], 0, qrow);
-        tma_load_2d(s.dout[st][1], &tm_do, &s.bar_do[st], 64, qrow);
-        issued = i + 1;
       }
-      const int nq = issued < 0 ? -issued : issued;
-      const int ndo = issued < 0 ? -issued - 1 : issued;
-      for (int i = (nq > 2 ? nq - 2 : 0); i < nq; ++i) mbar_wait(&s.bar_q[i & 1], (i >> 1) & 1, prm.status);
-      for (int i = (ndo > 2 ? ndo - 2 : 0); i < ndo; ++i) mbar_wait(&s.bar_do[i & 1], (i >> 1) & 1, prm.status);
-      mbar_wait(&s.bar_kv, 0, prm.status);
+      // do not leave the CTA with copies in flight
+      for (int j = (hq > kKvRing ? hq - kKvRing : 0); j < hq; ++j)
+        mbar_wait(&s.bar_qdo[j % kKvRing], (j / kKvRing) & 1, prm.status);
+      if (ucount > 0) mbar_wait(&s.bar_kv, (ucount - 1) & 1, prm.status);
     }
-  } else if (warp == kVecWarps + 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
-      const uint32_t id_kmaj = idesc_bf16_f32(kT, kT, false, false);  // S^T, dP^T
-      const uint32_t id_mnb = idesc_bf16_f32(kT, kD, false, true);    // dV, dK (B = [queries][d])
-      auto mma_ss = [&](uint32_t d, const uint8_t (*a)[kT * 128], const uint8_t (*bm)[kT * 128]) {
+  } else if (warp == kVecWarps + 1 || warp == kVecWarps + 2) {
+    // ------------------------------------------------------------------ MMA issuers
+    if (lane == 0) {
+      const bool grads_thread = warp == kVecWarps + 1;
+      const uint32_t id_sdp = idesc_bf16_f32(kT, kHalfRows, false, false);  // S^T, dP^T of a half
+      const uint32_t id_mnb = idesc_bf16_f32(kT, kD, false, true);          // dV, dK (B = [queries][d])
+      int G0 = 0, ucount = 0;
+      bool ok = true;
+      // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
+      const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0]), 0, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0]), 0, 1024);
+      const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0][0]), 0, 1024);
+      const uint64_t ddo0 = sdesc_sw128(smem_u32(s.dout[0][0]), 0, 1024);
+      const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0][0]), kHalfRows * 128, 1024);      // MN-major
+      const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0][0]), kHalfRows * 128, 1024);
+      constexpr uint32_t kStage16 = (2 * kHalfRows * 128) >> 4;  // one ring stage, in 16-byte units
+      // S^T = K Q_h^T and dP^T = V dO_h^T of global half hx into half buffer hx & 1
+      auto sdp = [&](int hx) -> bool {
+        const int hs = hx % kKvRing, buf = hx & 1;
+        if (!mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * 128;
+        const uint64_t dq = dq0 + static_cast<uint64_t>(hs) * kStage16;
+        const uint64_t ddo = ddo0 + static_cast<uint64_t>(hs) * kStage16;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(a[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(bm[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          mma_bf16_ss(d, ad, bd, id_kmaj, ks > 0 ? 1u : 0u);
+          const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
+          mma_bf16_ss(d, sdesc_add(dk0, ko), sdesc_add(dq, qo), id_sdp, ks > 0 ? 1u : 0u);
         }
-      };
-      auto mma_ts = [&](uint32_t d, uint32_t a_col, const uint8_t (*bm)[kT * 128], bool acc) {
 #pragma unroll
-        for (int ks = 0; ks < kT / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(smem_u32(bm[0]) + ks * 2048, kT * 128, 1024);
-          mma_bf16_ts(d, tmem + a_col + ks * 8, bd, id_mnb, (acc || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
+          mma_bf16_ss(d + 64, sdesc_add(dv0, ko), sdesc_add(ddo, qo), id_sdp, ks > 0 ? 1u : 0u);
         }
+        tc_commit(&s.bar_sdp_full[buf]);
+        return true;
       };
-      bool ok = mbar_wait(&s.bar_kv, 0, prm.status) && mbar_wait(&s.bar_q[0], 0, prm.status);
-      if (ok) {
-        tc_fence_after();
-        mma_ss(tmem + kColS, s.k, s.q[0]);
-        tc_commit(&s.bar_s_full);
-        ok = mbar_wait(&s.bar_do[0], 0, prm.status);
-      }
-      if (ok) {
-        tc_fence_after();
-        mma_ss(tmem + kColDP, s.v, s.dout[0]);
-        tc_commit(&s.bar_dp_full);
-      }
-      for (int i = 0; ok && i < n; ++i) {
-        const int st = i & 1;
-        if (!(ok = mbar_wait(&s.bar_p_ready, i & 1, prm.status))) break;
-        tc_fence_after();
-        mma_ts(tmem + kColDV, kColS, s.dout[st], i > 0);       // dV += P^T_hi dO
-        mma_ts(tmem + kColDV, kColS + 64, s.dout[st], true);   // dV += P^T_lo dO
-        tc_commit(&s.bar_do_empty[st]);
-        if (!(ok = mbar_wait(&s.bar_ds_ready, i & 1, prm.status))) break;
-        tc_fence_after();
-        mma_ts(tmem + kColDK, kColDP, s.q[st], i > 0);       // dK += dS^T_hi Q
-        mma_ts(tmem + kColDK, kColDP + 64, s.q[st], true);   // dK += dS^T_lo Q
-        tc_commit(&s.bar_q_empty[st]);
-        if (i + 1 < n) {
-          if (!(ok = mbar_wait(&s.bar_q[st ^ 1], ((i + 1) >> 1) & 1, prm.status))) break;
-          tc_fence_after();
-          mma_ss(tmem + kColS, s.k, s.q[st ^ 1]);
-          tc_commit(&s.bar_s_full);
-          if (!(ok = mbar_wait(&s.bar_do[st ^ 1], ((i + 1) >> 1) & 1, prm.status))) break;
-          tc_fence_after();
-          mma_ss(tmem + kColDP, s.v, s.dout[st ^ 1]);
-          tc_commit(&s.bar_dp_full);
+      // acc += A (TMEM, 128 keys x 64 query rows) . B (the half's [64 rows][128 d], MN-major)
+      auto grad = [&](uint32_t d, uint32_t a_col, uint64_t bdesc, bool acc) {
+#pragma unroll
+        for (int ks = 0; ks < kHalfRows / 16; ++ks)
+          mma_bf16_ts(d, tmem + a_col + ks * 8, sdesc_add(bdesc, ks * 2048), id_mnb, (acc || ks > 0) ? 1u : 0u);
+      };
+      for (int k = 0; ok; ++k) {
+        const int i = next_from_ring(k);
+        if (i < 0) break;
+        int bg, kb, rp, n;
+        unit_of(i, bg, kb, rp, n);
+        if (n == 0) continue;
+        const int nh = 2 * n;
+        if (grads_thread) {
+          // dV += P^T dO and dK += dS^T Q (hi, lo) as soon as the element-wise warps have a half
+          for (int x = 0; ok && x < nh; ++x) {
+            const int hx = G0 + x, buf = hx & 1, hs = hx % kKvRing;
+            if (!(ok = mbar_wait(&s.bar_pds_ready[buf], (hx >> 1) & 1, prm.status))) break;
+            tc_fence_after();
+            const uint32_t b0 = buf * 128;
+            const uint64_t ddom = ddom0 + static_cast<uint64_t>(hs) * kStage16;
+            const uint64_t dqm = dqm0 + static_cast<uint64_t>(hs) * kStage16;
+            grad(tmem + kColDV, b0, ddom, x > 0);        // dV += P^T_hi dO
+            grad(tmem + kColDV, b0 + 32, ddom, true);    // dV += P^T_lo dO
+            grad(tmem + kColDK, b0 + 64, dqm, x > 0);    // dK += dS^T_hi Q
+            grad(tmem + kColDK, b0 + 96, dqm, true);     // dK += dS^T_lo Q
+            tc_commit(&s.bar_qdo_empty[hs]);
+            tc_commit(&s.bar_grads_done[buf]);          // half buffer hx & 1 may be overwritten
+          }
+          if (ok) tc_commit(&s.bar_done);
+        } else {
+          // S^T / dP^T of each half once its buffer's previous products have completed.  One
+          // barrier per buffer: its next phase needs an S^T this thread has not issued yet, so a
+          // parity wait always names the right phase (this thread may fall behind while it waits
+          // for the next block's K and V).
+          if (!(ok = mbar_wait(&s.bar_kv, ucount & 1, prm.status))) break;
+          ++ucount;
+          for (int x = 0; ok && x < nh; ++x) {
+            const int hx = G0 + x;
+            if (hx >= 2 && !(ok = mbar_wait(&s.bar_grads_done[hx & 1], ((hx >> 1) - 1) & 1, prm.status))) break;
+            if (!(ok = sdp(hx))) break;
+            if (x + 1 == nh) tc_commit(&s.bar_kv_empty);  // the block's last read of K and V
+          }
         }
+        G0 += nh;
       }
-      if (ok) tc_commit(&s.bar_done);
     }
   } else {
     // ------------------------------------------------------------------ P / dS warps
     const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // key row within the KV tile == TMEM lane
-    const int c0 = hf * (kT / 2);       // this thread's query columns [c0, c0 + 64)
-    const int kpos = kb * prm.by + r;
-    const bool key_valid = r < prm.by && kpos < prm.S_kv;
-    // query positions that see this key: [qlo, qhi]
-    int qlo = -0x40000000, qhi = 0x3fffffff;
-    const int shift = prm.S_kv - prm.S_q;
-    if (prm.mask_mode == 2) qlo = kpos;
-    else if (prm.mask_mode == 3) qlo = kpos - shift;
-    else if (prm.mask_mode == 4) { qlo = kpos - shift - prm.win_right; qhi = kpos - shift + prm.win_left; }
-    if (!key_valid) { qlo = 1; qhi = 0; }
+    const int c0 = hf * 32;             // this thread's query columns [c0, c0 + 32) of a half
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int exchanges = 0;
+    const int shift = prm.S_kv - prm.S_q;
+    int exchanges = 0, G0 = 0, done_count = 0;
     bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      const int st = i & 1;
-      int qrow, tile, qpos0;
-      entry_rows(i, qrow, tile, qpos0);
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_q[st], (i >> 1) & 1, prm.status) &&
-                                       mbar_wait(&s.bar_s_full, i & 1, prm.status));
-      if (!ok) break;
-      tc_fence_after();
-      const bool full = qpos0 + c0 >= qlo && qpos0 + c0 + kT / 2 - 1 <= qhi;
-      const float* l2 = s.lse2[st] + c0;
-      float p[kT / 2];
+    for (int k = 0; ok; ++k) {
+      const int i = __shfl_sync(0xffffffffu, next_from_ring(k), 0);
+      if (i < 0) break;
+      int bg, kb, rp, n;
+      unit_of(i, bg, kb, rp, n);
+      const int kpos = kb * prm.by + r;
+      const bool key_valid = r < prm.by && kpos < prm.S_kv;
+      // query positions that see this key: [qlo, qhi]
+      int qlo = -0x40000000, qhi = 0x3fffffff;
+      if (prm.mask_mode == 2) qlo = kpos;
+      else if (prm.mask_mode == 3) qlo = kpos - shift;
+      else if (prm.mask_mode == 4) { qlo = kpos - shift - prm.win_right; qhi = kpos - shift + prm.win_left; }
+      if (!key_valid) { qlo = 1; qhi = 0; }
+      for (int x = 0; x < 2 * n; ++x) {
+        const int hx = G0 + x, buf = hx & 1, hs = hx % kKvRing;
+        int qrow, tile, qpos0;
+        entry_rows(bg, prm.col[rp + (x >> 1)], qrow, tile, qpos0);
+        const int qp0 = qpos0 + (x & 1) * kHalfRows + c0;  // query position of column c0
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status) &&
+                                         mbar_wait(&s.bar_sdp_full[buf], (hx >> 1) & 1, prm.status));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tmem + lane_base + buf * 128 + c0, sr);
+        tmem_ld32(tmem + lane_base + buf * 128 + 64 + c0, dr);
+        tmem_ld_wait(sr);
 #pragma unroll
-      for (int c = 0; c < kT / 2; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColS + c0 + c, rr);
-        tmem_ld_wait(rr);
+        for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
+        const float4* nl2 = reinterpret_cast<const float4*>(s.lse2[hs] + c0);  // -LSE*log2e per query row
+        const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D per query row
+        const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
+        const bool full = qp0 >= qlo && qp0 + 31 <= qhi;
+        uint32_t ph[16], pl[16], dh[16], dl[16];
 #pragma unroll
-        for (int k2 = 0; k2 < 32; ++k2) p[c + k2] = ex2(__uint_as_float(rr[k2]) * prm.scale_log2 - l2[c + k2]);
-      }
-      if (!full) {
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 L = nl2[c4], Dn = nd[c4];
 #pragma unroll
-        for (int c = 0; c < kT / 2; ++c) {
-          const int qp = qpos0 + c0 + c;
-          if (qp < qlo || qp > qhi) p[c] = 0.f;
+          for (int hp = 0; hp < 2; ++hp) {
+            const int c = c4 * 4 + hp * 2;
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2,
+                             hp ? f2_pack(L.z, L.w) : f2_pack(L.x, L.y)),
+                      t0, t1);
+            float p0 = ex2(t0), p1 = ex2(t1);
+            if (!full) {
+              if (qp0 + c < qlo || qp0 + c > qhi) p0 = 0.f;
+              if (qp0 + c + 1 < qlo || qp0 + c + 1 > qhi) p1 = 0.f;
+            }
+            const uint64_t p2 = f2_pack(p0, p1);
+            const uint64_t g2 = f2_mul(p2, f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                                                  hp ? f2_pack(Dn.z, Dn.w) : f2_pack(Dn.x, Dn.y)));
+            split_pack2(p2, ph[c / 2], pl[c / 2]);
+            split_pack2(g2, dh[c / 2], dl[c / 2]);
+          }
         }
+        // both warps of the quarter have read S^T and dP^T before either overwrites them
+        ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+        if (!ok) break;
+        const uint32_t base = tmem + lane_base + buf * 128 + hf * 16;
+        tmem_st16(base, ph);
+        tmem_st16(base + 32, pl);
+        tmem_st16(base + 64, dh);
+        tmem_st16(base + 96, dl);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&s.bar_pds_ready[buf]);
       }
-      // both halves have read S^T before either overwrites it:
-      // P^T hi -> S^T[c0/2, +32), P^T lo -> S^T[64 + c0/2, +32): A operands of dV += P^T dO
-      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
       if (!ok) break;
-#pragma unroll
-      for (int c = 0; c < kT / 2; c += 32) {
-        uint32_t hv[16], lv[16];
-#pragma unroll
-        for (int k2 = 0; k2 < 16; ++k2) split_pack(p[c + 2 * k2], p[c + 2 * k2 + 1], hv[k2], lv[k2]);
-        tmem_st16(tmem + lane_base + kColS + (c0 + c) / 2, hv);
-        tmem_st16(tmem + lane_base + kColS + 64 + (c0 + c) / 2, lv);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&s.bar_p_ready);
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, i & 1, prm.status));
-      if (!ok) break;
-      tc_fence_after();
-      const float* dvv = s.dvec[st] + c0;
-      // dS^T = P^T o (dP^T - D); hi -> dP^T[c0/2, +32), lo -> dP^T[64 + c0/2, +32)
-      uint32_t hv[32], lv[32];
-#pragma unroll
-      for (int c = 0; c < kT / 2; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColDP + c0 + c, rr);
-        tmem_ld_wait(rr);
-#pragma unroll
-        for (int k2 = 0; k2 < 16; ++k2) {
-          const int cc = c + 2 * k2;
-          split_pack(p[cc] * (__uint_as_float(rr[2 * k2]) - dvv[cc]),
-                     p[cc + 1] * (__uint_as_float(rr[2 * k2 + 1]) - dvv[cc + 1]), hv[cc / 2], lv[cc / 2]);
-        }
-      }
-      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
-      if (!ok) break;
-      tmem_st16(tmem + lane_base + kColDP + c0 / 2, hv);
-      tmem_st16(tmem + lane_base + kColDP + c0 / 2 + 16, hv + 16);
-      tmem_st16(tmem + lane_base + kColDP + 64 + c0 / 2, lv);
-      tmem_st16(tmem + lane_base + kColDP + 64 + c0 / 2 + 16, lv + 16);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&s.bar_ds_ready);
-    }
-    // ---- epilogue: dK = scale * acc, dV = acc (this thread: head-dim columns [c0, c0 + 64))
-    bool have = ok && n > 0;
-    if (have) {
-      have = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, 0, prm.status));
-      tc_fence_after();
-    }
-    __nv_bfloat16* dkrow = prm.dk + static_cast<size_t>(kv_row0 + r) * kD + c0;
-    __nv_bfloat16* dvrow = prm.dv + static_cast<size_t>(kv_row0 + r) * kD + c0;
-#pragma unroll
-    for (int c = 0; c < kD / 2; c += 32) {
-      uint32_t rk[32], rv[32];
+      // ---- epilogue: dK = scale * acc, dV = acc (this thread: head-dim columns [hf*64, +64))
+      bool have = n > 0;
       if (have) {
-        tmem_ld32(tmem + lane_base + kColDK + c0 + c, rk);
-        tmem_ld32(tmem + lane_base + kColDV + c0 + c, rv);
-        tmem_ld_wait(rk);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) reg_fence(rv[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rk[i] = rv[i] = 0u;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, done_count & 1, prm.status));
+        ++done_count;
+        if (!ok) break;
+        tc_fence_after();
       }
-      if (key_valid) {
-        store_row_bf16(dkrow + c, rk, prm.scale);
-        store_row_bf16(dvrow + c, rv, 1.f);
+      const int kv_row0 = bg * prm.S_kv + kb * prm.by;
+      __nv_bfloat16* dkrow = prm.dk + static_cast<size_t>(kv_row0 + r) * kD + hf * 64;
+      __nv_bfloat16* dvrow = prm.dv + static_cast<size_t>(kv_row0 + r) * kD + hf * 64;
+#pragma unroll
+      for (int c = 0; c < kD / 2; c += 32) {
+        uint32_t rk[32], rv[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + kColDK + hf * 64 + c, rk);
+          tmem_ld32(tmem + lane_base + kColDV + hf * 64 + c, rv);
+          tmem_ld_wait(rk);
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2) reg_fence(rv[i2]);
+        } else {
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2) rk[i2] = rv[i2] = 0u;
+        }
+        if (key_valid) {
+          store_row_bf16(dkrow + c, rk, prm.scale);
+          store_row_bf16(dvrow + c, rv, 1.f);
+        }
       }
+      // dK / dV have been read: the next block's first products wait for its P / dS, which come
+      // after this
+      tc_fence_before();
+      G0 += 2 * n;
     }
   }
   tc_fence_before();
@@ -500,16 +582,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n > 0) {
       const uint32_t id_s = idesc_bf16_f32(kT, BN, false, false);
       const uint32_t id_dq = idesc_bf16_f32(kT, kD, false, true);
+      // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
+      const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0]), 0, 1024);
+      const uint64_t ddo0 = sdesc_sw128(smem_u32(s.dout[0]), 0, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0][0]), 0, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), 0, 1024);
+      const uint64_t dkm0 = sdesc_sw128(smem_u32(s.k[0][0]), BN * 128, 1024);  // K as MN-major B of dQ
+      constexpr uint32_t kKv16 = (2 * BN * 128) >> 4;  // one K or V stage, in 16-byte units
       auto issue_s = [&](int j) -> bool {
         const int st = j & 1, sk = j % kQKStages;
         if (!mbar_wait(&s.bar_k[sk], (j / kQKStages) & 1, prm.status)) return false;
         tc_fence_after();
+        const uint64_t dk = dk0 + static_cast<uint64_t>(sk) * kKv16;
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(s.q[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.k[sk][ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          mma_bf16_ss(tmem + (st ? kColS1 : kColS0), ad, bd, id_s, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kD / 16; ++ks)
+          mma_bf16_ss(tmem + (st ? kColS1 : kColS0), sdesc_add(dq0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
+                      sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
         tc_commit(&s.bar_s_full[st]);
         return true;
       };
@@ -517,12 +605,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sv = j % kQVStages;
         if (!mbar_wait(&s.bar_v[sv], (j / kQVStages) & 1, prm.status)) return false;
         tc_fence_after();
+        const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * kKv16;
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(s.dout[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.v[sv][ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          mma_bf16_ss(tmem + kColDP, ad, bd, id_s, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kD / 16; ++ks)
+          mma_bf16_ss(tmem + kColDP, sdesc_add(ddo0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
+                      sdesc_add(dv, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
         tc_commit(&s.bar_dp_full);
         tc_commit(&s.bar_v_empty[sv]);
         return true;
@@ -537,14 +624,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t s_col = st ? kColS1 : kColS0;
         const int sk = j % kQKStages;
+        const uint64_t dkm = dkm0 + static_cast<uint64_t>(sk) * kKv16;
 #pragma unroll
         for (int half = 0; half < 2; ++half)
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t bd = sdesc_sw128(smem_u32(s.k[sk][0]) + ks * 2048, BN * 128, 1024);
-            mma_bf16_ts(tmem + kColDQ, tmem + s_col + half * (BN / 2) + ks * 8, bd, id_dq,
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_bf16_ts(tmem + kColDQ, tmem + s_col + half * (BN / 2) + ks * 8, sdesc_add(dkm, ks * 2048), id_dq,
                         (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
-          }
         tc_commit(&s.bar_k_empty[sk]);
         if (j + 1 < n && !(ok = issue_dp(j + 1))) break;
       }
@@ -564,8 +650,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
     if (!row_valid) { lo = 1; hi = 0; }
     const size_t trow = static_cast<size_t>(unit) * kT + r;
-    const float l2 = prm.lse2[trow];
-    const float dval = prm.dvec[trow];
+    const uint64_t nl2 = f2_pack(prm.lse2[trow], prm.lse2[trow]);  // -LSE*log2e of the row, twice
+    const uint64_t nd2 = f2_pack(prm.dvec[trow], prm.dvec[trow]);  // -D of the row, twice
+    const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     int exchanges = 0;
     bool ok = true;
@@ -584,7 +671,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + s_col + c0 + c, rr);
         tmem_ld_wait(rr);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) p[c + i] = ex2(__uint_as_float(rr[i]) * prm.scale_log2 - l2);
+        for (int i = 0; i < 32; i += 2) {
+          float t0, t1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(rr[i]), __uint_as_float(rr[i + 1])), sc2, nl2), t0, t1);
+          p[c + i] = ex2(t0);
+          p[c + i + 1] = ex2(t1);
+        }
       }
       if (!full) {
 #pragma unroll
@@ -604,8 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait(rr);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          split_pack(p[c + 2 * i] * (__uint_as_float(rr[2 * i]) - dval),
-                     p[c + 2 * i + 1] * (__uint_as_float(rr[2 * i + 1]) - dval), hv[c / 2 + i], lv[c / 2 + i]);
+          split_pack2(f2_mul(f2_pack(p[c + 2 * i], p[c + 2 * i + 1]),
+                             f2_add(f2_pack(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1])), nd2)),
+                      hv[c / 2 + i], lv[c / 2 + i]);
       }
       // both halves have read S_j before either writes dS over it:
       // hi -> S_j[c0/2, +BN/4), lo -> S_j[BN/2 + c0/2, +BN/4)
@@ -673,12 +766,14 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tq, tk, tv, tdo, tk128, tv128;
+  CUtensorMap tq, tk, tv, tdo, tk128, tv128, tq64, tdo64;
   const uint64_t q_rows = static_cast<uint64_t>(a.B) * a.N1 * a.S_q;
   const uint64_t kv_rows = static_cast<uint64_t>(a.B) * a.N2 * a.S_kv;
   if (!make_tmap_2d_bf16(&tq, q, q_rows, kD, kD, kT) || !make_tmap_2d_bf16(&tdo, dout, q_rows, kD, kD, kT) ||
       !make_tmap_2d_bf16(&tk, k, kv_rows, kD, kD, a.by) || !make_tmap_2d_bf16(&tv, v, kv_rows, kD, kD, a.by) ||
-      !make_tmap_2d_bf16(&tk128, k, kv_rows, kD, kD, kT) || !make_tmap_2d_bf16(&tv128, v, kv_rows, kD, kD, kT))
+      !make_tmap_2d_bf16(&tk128, k, kv_rows, kD, kD, kT) || !make_tmap_2d_bf16(&tv128, v, kv_rows, kD, kD, kT) ||
+      !make_tmap_2d_bf16(&tq64, q, q_rows, kD, kD, kHalfRows) ||
+      !make_tmap_2d_bf16(&tdo64, dout, q_rows, kD, kD, kHalfRows))
     return cudaErrorInvalidValue;
   BwdParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.S_q = a.S_q; p.S_kv = a.S_kv; p.bx = a.bx; p.by = a.by;
@@ -694,12 +789,17 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     BwdParams pk = p;
     pk.row_ptr = a.t_row_ptr;
     pk.col = a.t_col;
+    pk.next_unit = a.next_kv;
     const size_t smem = sizeof(KvSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(bsa_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = a.B * a.N2 * a.nkb;
+    const int units = a.B * a.N2 * a.nkb;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = units < sms ? units : sms;  // persistent: one CTA per SM
     prof_begin("bsa_bwd_kv", st);
-    bsa_bwd_kv_kernel<<<grid, kThreads, smem, st>>>(tq, tk128, tv128, tdo, pk);
+    if (grid > 0) bsa_bwd_kv_kernel<<<grid, kKvThreads, smem, st>>>(tq64, tk128, tv128, tdo64, pk);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

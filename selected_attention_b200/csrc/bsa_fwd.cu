@@ -213,15 +213,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
       const uint32_t idesc_o = idesc_bf16_f32(kBM, kD, false, true);
+      // descriptors of stage 0 / sub-tile 0; other stages, sub-tiles and K steps are added offsets
+      const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0]), 0, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0][0]), 0, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), BN * 128, 1024);
       auto issue_s = [&](int J) -> bool {  // global tile J
         const int st = J & 1, sk = J % kKStages;
         if (!mbar_wait(&s.bar_k[sk], (J / kKStages) & 1, prm.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + (st ? kColS1 : kColS0);
+        const uint64_t dk = dk0 + static_cast<uint64_t>(sk) * ((2 * BN * 128) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(s.q[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.k[sk][ks >> 2]) + (ks & 3) * 32, 0, 1024);
+          const uint64_t ad = sdesc_add(dq0, (ks >> 2) * (kBM * 128) + (ks & 3) * 32);
+          const uint64_t bd = sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32);
           mma_bf16_ss(d, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_s_full[st]);
@@ -250,11 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&s.bar_v[sv], (J / kVStages) & 1, prm.status))) break;
           tc_fence_after();
           const uint32_t p_col = st ? kColS1 : kColS0;
+          const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * ((2 * BN * 128) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t bd = sdesc_sw128(smem_u32(s.v[sv][0]) + ks * 2048, BN * 128, 1024);
-            mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, sdesc_add(dv, ks * 2048), idesc_o,
+                        (j > 0 || ks > 0) ? 1u : 0u);
           tc_commit(&s.bar_o_done);
           tc_commit(&s.bar_v_empty[sv]);
         }

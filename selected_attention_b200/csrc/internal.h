@@ -82,6 +82,8 @@ struct BsaBwdArgs {
   const int32_t* t_col;
   float* dvec;               // scratch [B*N1*nqb*128]
   float* lse2;               // scratch [B*N1*nqb*128]
+  int32_t* next_kv;          // work counters of the persistent passes, zeroed before the launch
+  int32_t* next_q;
   void* dq;
   void* dk;
   void* dv;

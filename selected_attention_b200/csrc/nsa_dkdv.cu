@@ -149,47 +149,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(kRows, kKeys, false, false);  // S, dP
       const uint32_t id_g = idesc_bf16_f32(kD, kKeys, true, true);       // dV^T, dK^T
+      // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
+      const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0][0]), 0, 1024);
+      const uint64_t ddo0 = sdesc_sw128(smem_u32(s.dout[0][0]), 0, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 0, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 0, 1024);
+      const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0][0]), kRows * 128, 1024);    // MN-major A
+      const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0][0]), kRows * 128, 1024);
+      const uint64_t dph = sdesc_sw128(smem_u32(s.p[0]), kRows * 128, 1024), dpl = sdesc_add(dph, kRows * 128);
+      const uint64_t dsh = sdesc_sw128(smem_u32(s.ds[0]), kRows * 128, 1024), dsl = sdesc_add(dsh, kRows * 128);
+      constexpr uint32_t kStage16 = (2 * kRows * 128) >> 4;  // one Q / dO stage, in 16-byte units
       // [128 rows] x [64 keys] += A [128 rows][128 d] . B [64 keys][128 d]^T, both K-major
-      auto mma_s = [&](uint32_t d, const uint8_t (*a)[kRows * 128], const uint8_t (*bk)[kKeys * 128]) {
+      auto mma_s = [&](uint32_t d, uint64_t a, uint64_t b) {
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(a[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(bk[ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          mma_bf16_ss(d, ad, bd, id_s, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kD / 16; ++ks)
+          mma_bf16_ss(d, sdesc_add(a, (ks >> 2) * (kRows * 128) + (ks & 3) * 32),
+                      sdesc_add(b, (ks >> 2) * (kKeys * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
       };
       // [128 d] x [64 keys] += A^T . B with A the [128 rows][128 d] tile (MN-major, two 64-d
       // chunks 16 KB apart) and B the [128 rows][64 keys] tile (MN-major, one chunk)
-      auto mma_g = [&](uint32_t d, const uint8_t (*a)[kRows * 128], const uint8_t* bm, bool acc) {
+      auto mma_g = [&](uint32_t d, uint64_t a, uint64_t b, bool acc) {
 #pragma unroll
-        for (int ks = 0; ks < kRows / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(smem_u32(a[0]) + ks * 2048, kRows * 128, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(bm) + ks * 2048, kRows * 128, 1024);
-          mma_bf16_ss(d, ad, bd, id_g, (acc || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kRows / 16; ++ks)
+          mma_bf16_ss(d, sdesc_add(a, ks * 2048), sdesc_add(b, ks * 2048), id_g, (acc || ks > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&s.bar_kv, 0, prm.status) && mbar_wait(&s.bar_qdo[0], 0, prm.status);
       if (ok) {
         tc_fence_after();
-        mma_s(tmem + kColS, s.q[0], s.k);
-        mma_s(tmem + kColDP, s.dout[0], s.v);
+        mma_s(tmem + kColS, dq0, dk);
+        mma_s(tmem + kColDP, ddo0, dv);
         tc_commit(&s.bar_s_full);
       }
       for (int i = 0; ok && i < steps; ++i) {
         const int st = i & 1;
         if (!(ok = mbar_wait(&s.bar_p_ready, i & 1, prm.status))) break;
         tc_fence_after();
-        mma_g(tmem + kColDV, s.dout[st], s.p[0], i > 0);   // dV^T += dO^T P_hi
-        mma_g(tmem + kColDV, s.dout[st], s.p[1], true);    // dV^T += dO^T P_lo
-        mma_g(tmem + kColDK, s.q[st], s.ds[0], i > 0);     // dK^T += Q^T dS_hi
-        mma_g(tmem + kColDK, s.q[st], s.ds[1], true);      // dK^T += Q^T dS_lo
+        const uint64_t ddom = ddom0 + static_cast<uint64_t>(st) * kStage16;
+        const uint64_t dqm = dqm0 + static_cast<uint64_t>(st) * kStage16;
+        mma_g(tmem + kColDV, ddom, dph, i > 0);   // dV^T += dO^T P_hi
+        mma_g(tmem + kColDV, ddom, dpl, true);    // dV^T += dO^T P_lo
+        mma_g(tmem + kColDK, dqm, dsh, i > 0);    // dK^T += Q^T dS_hi
+        mma_g(tmem + kColDK, dqm, dsl, true);     // dK^T += Q^T dS_lo
         tc_commit(&s.bar_p_free);
         tc_commit(&s.bar_qdo_empty[st]);
         if (i + 1 < steps) {
           if (!(ok = mbar_wait(&s.bar_qdo[st ^ 1], ((i + 1) >> 1) & 1, prm.status))) break;
           tc_fence_after();
-          mma_s(tmem + kColS, s.q[st ^ 1], s.k);
-          mma_s(tmem + kColDP, s.dout[st ^ 1], s.v);
+          mma_s(tmem + kColS, dq0 + static_cast<uint64_t>(st ^ 1) * kStage16, dk);
+          mma_s(tmem + kColDP, ddo0 + static_cast<uint64_t>(st ^ 1) * kStage16, dv);
           tc_commit(&s.bar_s_full);
         }
       }

@@ -53,6 +53,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 
 // Register barrier: makes later uses of `r` depend on an asm that sits after a wait instruction.
 __device__ __forceinline__ void reg_fence(uint32_t& r) { asm volatile("" : "+r"(r)); }
@@ -223,6 +228,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
+
+// The start-address field holds (shared address >> 4) in bits [0,14), and shared addresses stay
+// below 256 KB, so the descriptor of (base + off) is the descriptor of base plus off / 16.  The MMA
+// issuers build one descriptor per buffer up front and step it with these adds: a single thread
+// issues every MMA of a CTA, and per-MMA descriptor arithmetic would cost more cycles than the
+// MMA itself takes on the tensor core.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t off_bytes) { return desc + (off_bytes >> 4); }
 
 // TMEM address: lane in bits [16,32), column in [0,16).  A warp may only touch the 32-lane
 // subpartition (warp_id % 4).

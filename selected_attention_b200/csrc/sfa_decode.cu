@@ -165,23 +165,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_tiles > 0) {
       const uint32_t id_s = idesc_bf16_f32(kM, kTile, false, false);
       const uint32_t id_o = idesc_bf16_f32(kM, kDVH, false, true);
+      // descriptors of stage 0 / box 0; stages, boxes and K steps are added offsets
+      const uint64_t dqh = sdesc_sw128(smem_u32(s.qhi[0]), 0, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0][0]), 0, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), kTile * 128, 1024);
+      constexpr uint32_t kK16 = (kKBoxes * kTile * 128) >> 4, kV16 = (kVBoxes * kTile * 128) >> 4;
       auto issue_s = [&](int j) -> bool {
         const int st = j & 1;
         if (!mbar_wait(&s.bar_k[st], (j >> 1) & 1, prm.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + (st ? kColS1 : kColS0);
+        const uint64_t dk = dk0 + static_cast<uint64_t>(st) * kK16;
         // dims 0-255: A = Q from tensor memory; dims 256-575: A = Q from shared memory
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(smem_u32(s.k[st][ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          mma_bf16_ts(d, tmem + kColQ + ks * 8, bd, id_s, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < 16; ++ks)
+          mma_bf16_ts(d, tmem + kColQ + ks * 8, sdesc_add(dk, (ks >> 2) * (kTile * 128) + (ks & 3) * 32), id_s,
+                      ks > 0 ? 1u : 0u);
 #pragma unroll
         for (int ks = 16; ks < 36; ++ks) {
           const int qs = ks - 16;
-          const uint64_t ad = sdesc_sw128(smem_u32(s.qhi[qs >> 2]) + (qs & 3) * 32, 0, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(s.k[st][ks >> 2]) + (ks & 3) * 32, 0, 1024);
-          mma_bf16_ss(d, ad, bd, id_s, 1u);
+          mma_bf16_ss(d, sdesc_add(dqh, (qs >> 2) * (kM * 128) + (qs & 3) * 32),
+                      sdesc_add(dk, (ks >> 2) * (kTile * 128) + (ks & 3) * 32), id_s, 1u);
         }
         tc_commit(&s.bar_s_full[st]);
         tc_commit(&s.bar_k_empty[st]);
@@ -196,11 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status))) break;
         tc_fence_after();
         const uint32_t p_col = st ? kColS1 : kColS0;
+        const uint64_t dv = dv0 + static_cast<uint64_t>(st) * kV16;
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(smem_u32(s.v[st][0]) + ks * 2048, kTile * 128, 1024);
-          mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, bd, id_o, (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, sdesc_add(dv, ks * 2048), id_o, (j > 0 || ks > 0) ? 1u : 0u);
         tc_commit(&s.bar_o_done);
         tc_commit(&s.bar_v_empty[st]);
       }
