@@ -226,6 +226,12 @@ BSA_API const char* bsa_version(void);
 BSA_API bsa_status bsa_diag_mma_tile(const void* a, const void* b, float* c, int32_t b_mn_major, void* workspace,
                              void* stream);
 
+/* Diagnostic: y[i] = 2^x[i] (device arrays of n floats) by the polynomial the softmax loops use
+ * on the FMA pipe for part of their exponentials (Cody-Waite reduction to [-1/2, 1/2], fitted
+ * polynomial of degree 3 or 4, exponent add).  x must lie in [-126, 128).  Not part of the pages'
+ * operations.  Returns BSA_ERR_INVALID_ARG for another degree or n < 0. */
+BSA_API bsa_status bsa_diag_exp2(const float* x, float* y, int32_t n, int32_t degree, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

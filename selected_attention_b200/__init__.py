@@ -29,7 +29,7 @@ EXPORTED = [
     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size", "bsa_fwd", "bsa_bwd",
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
-    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc",
+    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_diag_exp2",
 ]
 
 
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_metadata.argtypes = [P, ctypes.c_int32, vp, sz, vp]
         L.bsa_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.bsa_diag_mma_tile.argtypes = [vp, vp, vp, ctypes.c_int32, vp, vp]
+        L.bsa_diag_exp2.argtypes = [vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
         L.bsa_profile_enable.argtypes = [ctypes.c_int32]
         L.bsa_profile_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
         L.bsa_version.restype = ctypes.c_char_p
@@ -383,3 +384,11 @@ def bsa_diag_mma_tile(a, b, mode, stream=None):
     _check("bsa_diag_mma_tile", lib().bsa_diag_mma_tile(_ptr(a), _ptr(b), _ptr(c), int(mode), _ptr(ws),
                                                         _stream(stream)))
     return c, ws
+
+
+def bsa_diag_exp2(x, degree, stream=None):
+    """2^x by the device polynomial of the given degree (3 or 4); x a CUDA float32 tensor."""
+    _need_cuda(x)
+    y = torch.empty_like(x)
+    _check("bsa_diag_exp2", lib().bsa_diag_exp2(_ptr(x), _ptr(y), x.numel(), degree, _stream(stream)))
+    return y

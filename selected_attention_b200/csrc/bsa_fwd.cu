@@ -18,9 +18,11 @@
 //              last S has read the old Q), the K tiles into a 3-stage ring and the V tiles into
 //              a 2-stage ring.  A K stage is released when its S = Q K^T has run, a V stage
 //              after its O += P V.
-//   warp 9     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers, and
-//              O += P_j V_j into the TMEM O accumulator.  Within a unit S_{j+1} is issued before
-//              waiting for P_j; the next unit's first S is issued right after the last O += P V.
+//   warp 9     issues O += P_j V_j into the TMEM O accumulator as soon as P_j is ready.
+//   warp 10    issues S_j = Q K_j^T into TMEM S buffer j % 2 as soon as K_j is loaded and the
+//              buffer's previous O += P V has completed.  Two issuing threads: tcgen05.mma issue
+//              blocks while the tensor pipe's queue is full, so one thread would hold each
+//              O += P V back behind the next tile's score MMAs.
 // Tile counters run across units, so rings, S buffers and barrier phases carry over.
 // The row max is taken on the raw scores (scale > 0 is required by the host checks), so each
 // probability costs one fused multiply-add (packed in pairs) and one exp2.
@@ -37,11 +39,11 @@ namespace {
 constexpr int kBM = 128;  // query rows per CTA tile (the MMA M)
 constexpr int kD = 128;   // head dim of Q/K and V
 constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kKStages = 3, kVStages = 2;
+constexpr int kKStages = 2, kVStages = 2;
 constexpr int kSched = 4;  // unit ring between the scheduler and the other warps
 
 template <int BN>
@@ -49,15 +51,20 @@ struct __align__(1024) FwdSmem {
   uint8_t q[2][kBM * 128];            // Q sub-tiles (head-dim columns 0-63, 64-127), 128B swizzle
   uint8_t k[kKStages][2][BN * 128];   // [stage][sub-tile] K rows of one KV block
   uint8_t v[kVStages][2][BN * 128];   // [stage][sub-tile] V rows
+  uint8_t ostage[2][kBM * 128];       // Out tile staged for the TMA store (head-dim halves)
   float red[2][2][kBM];               // [tile parity][column half][row]: partial row max
   float red_l[2][2][kBM];             // [unit parity][column half][row]: partial row sum
   int32_t sched[kSched];              // unit ring (-1: no more units)
   uint64_t bar_q, bar_q_empty;
   uint64_t bar_k[kKStages], bar_k_empty[kKStages], bar_v[kVStages], bar_v_empty[kVStages], bar_s_full[2];
-  uint64_t bar_p_full, bar_o_done;
+  uint64_t bar_p_full[2];             // per S buffer: P of its tile is written (256 arrivals)
+  uint64_t bar_o_done;
+  uint64_t bar_pv_done[2];            // per S buffer: the O += P V that read it has completed
   uint64_t bar_done;                  // one phase per non-empty unit: its last O += P V has completed
   uint64_t bar_sched_full[kSched], bar_sched_empty[kSched];
   uint64_t bar_pair[4];               // the two softmax warps of each TMEM lane quarter
+  uint64_t bar_epi;                   // the unit's Out tile is staged (256 arrivals)
+  uint64_t bar_stage_free;            // the previous store has read the staging buffer
   uint32_t tmem_base;
 };
 
@@ -101,7 +108,8 @@ __device__ __forceinline__ bool pair_sync(uint64_t* bar, int& exchanges, uint32_
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const FwdParams prm) {
   constexpr uint32_t kTmemCols = (2 * BN + kD) <= 256 ? 256 : 512;
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
   constexpr int kHalf = BN / 2;  // S columns per softmax thread
@@ -121,14 +129,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&s.bar_s_full[i], 1);
-    mbar_init(&s.bar_p_full, kSoftmaxWarps * 32);
+    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_p_full[i], kSoftmaxWarps * 32);
     mbar_init(&s.bar_o_done, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_pv_done[i], 1);
     mbar_init(&s.bar_done, 1);
     for (int i = 0; i < kSched; ++i) {
       mbar_init(&s.bar_sched_full[i], 1);
-      mbar_init(&s.bar_sched_empty[i], 1 + kSoftmaxWarps * 32);
+      mbar_init(&s.bar_sched_empty[i], 2 + kSoftmaxWarps * 32);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
+    mbar_init(&s.bar_epi, kSoftmaxWarps * 32);
+    mbar_init(&s.bar_stage_free, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -208,31 +219,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&s.bar_v[j % kVStages], (j / kVStages) & 1, prm.status);
       if (qcount > 0) mbar_wait(&s.bar_q, (qcount - 1) & 1, prm.status);
     }
-  } else if (warp == kSoftmaxWarps + 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kSoftmaxWarps + 1 || warp == kSoftmaxWarps + 2) {
+    // ------------------------------------------------------------------ MMA issuers
     if (lane == 0) {
+      const bool pv_thread = warp == kSoftmaxWarps + 1;
       const uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
       const uint32_t idesc_o = idesc_bf16_f32(kBM, kD, false, true);
       // descriptors of stage 0 / sub-tile 0; other stages, sub-tiles and K steps are added offsets
       const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0]), 0, 1024);
       const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0][0]), 0, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), BN * 128, 1024);
-      auto issue_s = [&](int J) -> bool {  // global tile J
-        const int st = J & 1, sk = J % kKStages;
-        if (!mbar_wait(&s.bar_k[sk], (J / kKStages) & 1, prm.status)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + (st ? kColS1 : kColS0);
-        const uint64_t dk = dk0 + static_cast<uint64_t>(sk) * ((2 * BN * 128) >> 4);
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t ad = sdesc_add(dq0, (ks >> 2) * (kBM * 128) + (ks & 3) * 32);
-          const uint64_t bd = sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32);
-          mma_bf16_ss(d, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-        }
-        tc_commit(&s.bar_s_full[st]);
-        tc_commit(&s.bar_k_empty[sk]);
-        return true;
-      };
       int J0 = 0, qcount = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
@@ -240,30 +236,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i < 0) break;
         const UnitInfo u = unit_info(prm, i);
         if (u.n == 0) continue;
-        if (!(ok = mbar_wait(&s.bar_q, qcount & 1, prm.status))) break;
-        ++qcount;
-        if (!(ok = issue_s(J0))) break;
-        if (u.n == 1) tc_commit(&s.bar_q_empty);
-        for (int j = 0; ok && j < u.n; ++j) {
-          const int J = J0 + j;
-          if (j + 1 < u.n) {
-            if (!(ok = issue_s(J + 1))) break;
-            if (j + 2 == u.n) tc_commit(&s.bar_q_empty);  // the unit's last read of Q
-          }
-          if (!(ok = mbar_wait(&s.bar_p_full, J & 1, prm.status))) break;
-          const int st = J & 1, sv = J % kVStages;
-          if (!(ok = mbar_wait(&s.bar_v[sv], (J / kVStages) & 1, prm.status))) break;
-          tc_fence_after();
-          const uint32_t p_col = st ? kColS1 : kColS0;
-          const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * ((2 * BN * 128) >> 4);
+        if (pv_thread) {
+          for (int j = 0; ok && j < u.n; ++j) {
+            const int J = J0 + j, st = J & 1, sv = J % kVStages;
+            // one barrier per S buffer: its next phase needs S_{J+2}, which waits for this PV
+            if (!(ok = mbar_wait(&s.bar_p_full[st], (J >> 1) & 1, prm.status))) break;
+            if (!(ok = mbar_wait(&s.bar_v[sv], (J / kVStages) & 1, prm.status))) break;
+            tc_fence_after();
+            const uint32_t p_col = st ? kColS1 : kColS0;
+            const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * ((2 * BN * 128) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, sdesc_add(dv, ks * 2048), idesc_o,
-                        (j > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(&s.bar_o_done);
-          tc_commit(&s.bar_v_empty[sv]);
+            for (int ks = 0; ks < BN / 16; ++ks)
+              mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, sdesc_add(dv, ks * 2048), idesc_o,
+                          (j > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(&s.bar_o_done);
+            tc_commit(&s.bar_v_empty[sv]);
+            tc_commit(&s.bar_pv_done[st]);
+          }
+          if (ok) tc_commit(&s.bar_done);
+        } else {
+          if (!(ok = mbar_wait(&s.bar_q, qcount & 1, prm.status))) break;
+          ++qcount;
+          for (int j = 0; ok && j < u.n; ++j) {
+            const int J = J0 + j, st = J & 1, sk = J % kKStages;
+            // S buffer st last held P_{J-2}; one barrier per buffer keeps the parity wait exact
+            if (J >= 2 && !(ok = mbar_wait(&s.bar_pv_done[st], ((J >> 1) - 1) & 1, prm.status))) break;
+            if (!(ok = mbar_wait(&s.bar_k[sk], (J / kKStages) & 1, prm.status))) break;
+            tc_fence_after();
+            const uint32_t d = tmem + (st ? kColS1 : kColS0);
+            const uint64_t dk = dk0 + static_cast<uint64_t>(sk) * ((2 * BN * 128) >> 4);
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks)
+              mma_bf16_ss(d, sdesc_add(dq0, (ks >> 2) * (kBM * 128) + (ks & 3) * 32),
+                          sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
+            tc_commit(&s.bar_s_full[st]);
+            tc_commit(&s.bar_k_empty[sk]);
+            if (j + 1 == u.n) tc_commit(&s.bar_q_empty);  // the unit's last read of Q
+          }
         }
-        if (ok) tc_commit(&s.bar_done);
         J0 += u.n;
       }
     }
@@ -341,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_new = mx;
         }
         if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
-          // O += P_{J-1} V_{J-1} is o_done phase J-1 (need implies j > 0).  S_J landed after every
-          // earlier MMA, so phase J-2 is complete and J cannot be: a parity wait tells them apart.
+          // O += P_{J-1} V_{J-1} is o_done phase J-1 (need implies j > 0).  S_J was issued after
+          // O += P_{J-2} V_{J-2} completed (the S buffer's pv_done), so phase J-2 is complete,
+          // and phase J needs this thread's P_J: a parity wait tells J-1 from J.
           ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (J - 1) & 1, prm.status));
           if (!ok) break;
           tc_fence_after();
@@ -387,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         m = m_new;
         tc_fence_before();
-        mbar_arrive(&s.bar_p_full);
+        mbar_arrive(&s.bar_p_full[st]);
       }
       if (!ok) break;
       // ---- epilogue.  bar_done has one phase per non-empty unit and this thread has waited on
@@ -407,7 +418,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       l += s.red_l[k & 1][hf ^ 1][r];
       const bool any = have_o && l > 0.f;
       const float inv_l = any ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = prm.out + static_cast<size_t>(q_row0 + r) * kD + hf * (kD / 2);
+      // Out goes through a 128-byte-swizzled staging tile and two TMA stores (one per head-dim
+      // half), so global writes are whole rows; the box of block_x rows of a [B*N1][S_q][128] map
+      // stops at the q block and at the head's end.  The previous unit's store must have read
+      // the staging tile first.
+      if (k > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_stage_free, (k - 1) & 1, prm.status));
+        if (!ok) break;
+      }
+      uint8_t* ost = s.ostage[hf];
 #pragma unroll
       for (int c = 0; c < kD / 2; c += 32) {
         uint32_t rr[32];
@@ -418,24 +437,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i2 = 0; i2 < 32; ++i2) rr[i2] = 0u;
         }
-        if (row_valid) {
 #pragma unroll
-          for (int i2 = 0; i2 < 32; i2 += 8) {
-            uint4 pk;
-            pk.x = pack_bf16(__uint_as_float(rr[i2 + 0]) * inv_l, __uint_as_float(rr[i2 + 1]) * inv_l);
-            pk.y = pack_bf16(__uint_as_float(rr[i2 + 2]) * inv_l, __uint_as_float(rr[i2 + 3]) * inv_l);
-            pk.z = pack_bf16(__uint_as_float(rr[i2 + 4]) * inv_l, __uint_as_float(rr[i2 + 5]) * inv_l);
-            pk.w = pack_bf16(__uint_as_float(rr[i2 + 6]) * inv_l, __uint_as_float(rr[i2 + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + c + i2) = pk;
-          }
+        for (int i2 = 0; i2 < 32; i2 += 8) {
+          uint4 pk;
+          pk.x = pack_bf16(__uint_as_float(rr[i2 + 0]) * inv_l, __uint_as_float(rr[i2 + 1]) * inv_l);
+          pk.y = pack_bf16(__uint_as_float(rr[i2 + 2]) * inv_l, __uint_as_float(rr[i2 + 3]) * inv_l);
+          pk.z = pack_bf16(__uint_as_float(rr[i2 + 4]) * inv_l, __uint_as_float(rr[i2 + 5]) * inv_l);
+          pk.w = pack_bf16(__uint_as_float(rr[i2 + 6]) * inv_l, __uint_as_float(rr[i2 + 7]) * inv_l);
+          const int chunk = (c + i2) >> 3;  // 16-byte chunk of this row's 64 columns
+          *reinterpret_cast<uint4*>(ost + r * 128 + ((chunk ^ (r & 7)) << 4)) = pk;
         }
       }
+      fence_async_smem();
+      mbar_arrive(&s.bar_epi);
+      if (warp == 0 && lane == 0) {
+        ok = mbar_wait(&s.bar_epi, k & 1, prm.status);
+        if (ok) {
+          tma_store_3d(&tm_o, s.ostage[0], 0, qb * prm.bx, u.bh);
+          tma_store_3d(&tm_o, s.ostage[1], 64, qb * prm.bx, u.bh);
+          bulk_commit();
+          bulk_wait_read_all();
+          mbar_arrive(&s.bar_stage_free);
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
       if (row_valid && hf == 0) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
       // O has been read: the next unit's first O += P V waits for P, which comes after this
       tc_fence_before();
       J0 += n;
     }
   }
+  if (warp == 0 && lane == 0) bulk_wait_all();  // the last Out stores have completed
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
@@ -449,6 +482,10 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   if (!make_tmap_2d_bf16(&tq, q, q_rows, kD, kD, kBM)) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tk, k, kv_rows, kD, kD, BN)) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tv, v, kv_rows, kD, kD, BN)) return cudaErrorInvalidValue;
+  CUtensorMap to;  // Out as [B*N1][S_q][128], box {64, block_x, 1}
+  if (!make_tmap_3d_bf16(&to, a.out, kD, a.S_q, static_cast<uint64_t>(a.B) * a.N1, kD,
+                         static_cast<uint64_t>(a.S_q) * kD, a.bx, 1))
+    return cudaErrorInvalidValue;
   FwdParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.S_q = a.S_q; p.S_kv = a.S_kv; p.bx = a.bx; p.by = a.by;
   p.nqb = a.nqb; p.mask_mode = a.mask_mode; p.win_left = a.win_left; p.win_right = a.win_right;
@@ -465,7 +502,7 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.units < sms ? p.units : sms;  // persistent: one CTA per SM
   prof_begin("bsa_fwd", st);
-  bsa_fwd_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
+  bsa_fwd_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, to, p);
   prof_end(st);
   return cudaGetLastError();
 }

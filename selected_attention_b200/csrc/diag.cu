@@ -107,7 +107,25 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+__global__ void diag_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int degree) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float y0, y1;
+  if (degree == 3) ex2_poly_pair<3>(x0, x1, y0, y1);
+  else ex2_poly_pair<4>(x0, x1, y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
+
+cudaError_t diag_exp2_launch(const float* x, float* y, int n, int degree, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int pairs = (n + 1) / 2;
+  diag_exp2_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n, degree);
+  return cudaGetLastError();
+}
 
 cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,
                                  cudaStream_t st) {

@@ -59,6 +59,44 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x for a pair of floats on the FMA pipe instead of the special-function unit, which the
+// softmax loops saturate.  Cody-Waite argument reduction: n = round(x) by adding 1.5 * 2^23 (n
+// lands in the low mantissa bits), f = x - n in [-1/2, 1/2]; 2^f by a polynomial whose
+// coefficients were fitted by weighted least squares to minimise the relative error on
+// [-1/2, 1/2] (max relative error in fp32 Horner form: 7.5e-5 for degree 3, 2.7e-6 for degree 4);
+// 2^n enters as an add of n << 23 to the exponent field.  x is clamped below at -126 (the result
+// is then about 2^-126, not 0): callers use it only where every x is finite, or select 0 for
+// x < -126 themselves.  x must be below 128.
+template <int DEG>
+__device__ __forceinline__ void ex2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  static_assert(DEG == 3 || DEG == 4, "fitted degrees");
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));       // 1.5 * 2^23 + round(x)
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));     // round(x), exact
+  const uint64_t fr = f2_fma(n, f2_pack(-1.f, -1.f), x);               // x - round(x)
+  uint64_t p;
+  if (DEG == 3) {
+    p = f2_fma(f2_pack(0.055171627551317215f, 0.055171627551317215f), fr,
+               f2_pack(0.2426111400127411f, 0.2426111400127411f));
+    p = f2_fma(p, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  } else {
+    p = f2_fma(f2_pack(0.009570096619427204f, 0.009570096619427204f), fr,
+               f2_pack(0.05591786280274391f, 0.05591786280274391f));
+    p = f2_fma(p, fr, f2_pack(0.240247443318367f, 0.240247443318367f));
+    p = f2_fma(p, fr, f2_pack(0.6931217908859253f, 0.6931217908859253f));
+    p = f2_fma(p, fr, f2_pack(0.9999992847442627f, 0.9999992847442627f));
+  }
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // the low 9 bits of t's pattern hold n (two's complement); << 23 moves them to the exponent
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Register barrier: makes later uses of `r` depend on an asm that sits after a wait instruction.
 __device__ __forceinline__ void reg_fence(uint32_t& r) { asm volatile("" : "+r"(r)); }
 
@@ -147,6 +185,20 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// TMA tiled store shared -> global, completion tracked per thread by bulk groups.  Coordinates
+// are never negative and the innermost one is a multiple of 64 bf16 elements.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until this thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until this thread's committed bulk stores have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (MMA, TMA).

@@ -7,8 +7,9 @@
 //                   number of valid tokens of each page.  A sparse block id at or past the
 //                   sequence's block count sets SA_DEV_BAD_INDEX and is skipped.
 //   sfa_work_list   units (b, g, Dv half) each own a page list; one CTA computes a piece of at
-//                   most `chunk` consecutive pages of one unit, with chunk chosen so that the
-//                   number of pieces fits one wave of CTAs.  Pieces are numbered unit by unit.
+//                   most `chunk` consecutive pages of one unit, with chunk the smallest size whose
+//                   pieces fit one wave of CTAs (so the longest piece is as short as possible).
+//                   Pieces are numbered unit by unit.
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -72,7 +73,8 @@ __global__ void sfa_page_list_kernel(const int32_t* __restrict__ sparse_indices,
 
 // One CTA: choose the piece size and lay out the pieces.
 //   units u = (b * N2 + g) * 2 + dv_half; n_u = count[b, g]
-//   chunk = ceil(W / max(1, G - U)) pages, where W = sum n_u, so sum ceil(n_u / chunk) <= G
+//   chunk = the smallest c >= 1 with sum_u ceil(n_u / c) <= G (binary search; c = max n_u always
+//   qualifies when units <= G, and the host never launches more units than that)
 //   piece records: unit, first page, page count; unit_first[u], unit_pieces[u]
 __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __restrict__ count, int units, int G,
                                                              int32_t* __restrict__ piece_unit,
@@ -81,21 +83,36 @@ __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __re
                                                              int32_t* __restrict__ unit_first,
                                                              int32_t* __restrict__ unit_pieces,
                                                              int32_t* __restrict__ n_pieces) {
-  __shared__ long long s_w;
+  __shared__ int s_pieces, s_max;
   __shared__ int s_chunk;
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  if (tid == 0) s_w = 0;
+  if (tid == 0) s_max = 1;
   __syncthreads();
-  long long loc = 0;
-  for (int u = tid; u < units; u += blockDim.x) loc += count[u >> 1];
-  atomicAdd(reinterpret_cast<unsigned long long*>(&s_w), static_cast<unsigned long long>(loc));  // integer sum
+  int mx = 1;
+  for (int u = tid; u < units; u += blockDim.x) mx = max(mx, count[u >> 1]);
+  atomicMax(&s_max, mx);
   __syncthreads();
+  int lo = 1, hi = s_max;  // pieces(hi) = units <= G
+  while (lo < hi) {        // uniform across the block
+    const int mid = (lo + hi) >> 1;
+    if (tid == 0) s_pieces = 0;
+    __syncthreads();
+    int loc = 0;
+    for (int u = tid; u < units; u += blockDim.x) {
+      const int n = count[u >> 1];
+      loc += n > 0 ? (n + mid - 1) / mid : 0;
+    }
+    atomicAdd(&s_pieces, loc);  // integer sum: order does not matter
+    __syncthreads();
+    const int total = s_pieces;
+    __syncthreads();
+    if (total <= G) hi = mid;
+    else lo = mid + 1;
+  }
   if (tid == 0) {
-    const long long slots = G > units ? G - units : 1;
-    const long long c = (s_w + slots - 1) / slots;
-    s_chunk = static_cast<int>(c < 1 ? 1 : c);
+    s_chunk = lo;
     carry = 0;
   }
   __syncthreads();
