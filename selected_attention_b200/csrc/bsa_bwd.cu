@@ -490,14 +490,20 @@ struct __align__(1024) QSmem {
   uint8_t dout[2][kT * 128];
   uint8_t k[kQKStages][2][BN * 128];  // [stage][sub-tile] [BN keys][64 d]
   uint8_t v[kQVStages][2][BN * 128];
-  uint64_t bar_qdo, bar_k[kQKStages], bar_k_empty[kQKStages], bar_v[kQVStages], bar_v_empty[kQVStages];
-  uint64_t bar_s_full[2], bar_dp_full, bar_ds_ready, bar_done;
+  int32_t sched[kSchedKv];
+  uint64_t bar_qdo, bar_qdo_empty, bar_k[kQKStages], bar_k_empty[kQKStages], bar_v[kQVStages], bar_v_empty[kQVStages];
+  uint64_t bar_s_full[2], bar_dp_full, bar_ds_ready[2], bar_dq_done[2], bar_done;
+  uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
   uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
 
+// Persistent: one CTA per SM takes Q tiles (b, h, qb) from a device counter (head-major, latest
+// q block first).  Warps: 0-7 element-wise, 8 scheduler + TMA, 9 issues dQ += dS K (hi, lo),
+// 10 issues S = Q K^T and dP = dO V^T.  Per-buffer barriers (ds_ready, dq_done per S buffer) keep
+// every parity wait exact with two issuing threads.
 template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     bsa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const BwdParams prm) {
@@ -505,18 +511,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   QSmem<BN>& s = *reinterpret_cast<QSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / prm.nqb;
-  const int qb = prm.nqb - 1 - static_cast<int>(blockIdx.x % prm.nqb);
-  const int b = bh / prm.N1, h = bh % prm.N1;
-  const int g = h / (prm.N1 / prm.N2);
-  const int unit = bh * prm.nqb + qb;
-  const int rp = prm.row_ptr[unit];
-  const int n = prm.row_ptr[unit + 1] - rp;
-  const int q_row0 = bh * prm.S_q + qb * prm.bx;
-  const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
+  const int units = prm.B * prm.N1 * prm.nqb;
 
   if (tid == 0) {
     mbar_init(&s.bar_qdo, 1);
+    mbar_init(&s.bar_qdo_empty, 1);
     for (int i = 0; i < kQKStages; ++i) {
       mbar_init(&s.bar_k[i], 1);
       mbar_init(&s.bar_k_empty[i], 1);
@@ -525,10 +524,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_v[i], 1);
       mbar_init(&s.bar_v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_s_full[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.bar_s_full[i], 1);
+      mbar_init(&s.bar_ds_ready[i], kVecWarps * 32);
+      mbar_init(&s.bar_dq_done[i], 1);
+    }
     mbar_init(&s.bar_dp_full, 1);
-    mbar_init(&s.bar_ds_ready, kVecWarps * 32);
     mbar_init(&s.bar_done, 1);
+    for (int i = 0; i < kSchedKv; ++i) {
+      mbar_init(&s.bar_sched_full[i], 1);
+      mbar_init(&s.bar_sched_empty[i], 2 + kVecWarps * 32);
+    }
     for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
@@ -541,45 +547,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
+  // schedule number i -> (b*N1 + h, q block), its KV list [rp, rp + n)
+  auto unit_of = [&](int i, int& bh, int& qb, int& rp, int& n) {
+    bh = i / prm.nqb;
+    qb = prm.nqb - 1 - i % prm.nqb;
+    const int unit = bh * prm.nqb + qb;
+    rp = prm.row_ptr[unit];
+    n = prm.row_ptr[unit + 1] - rp;
+  };
+  auto next_from_ring = [&](int k) -> int {
+    const int slot = k % kSchedKv;
+    if (!mbar_wait(&s.bar_sched_full[slot], (k / kSchedKv) & 1, prm.status)) return -1;
+    const int u = *reinterpret_cast<volatile int32_t*>(&s.sched[slot]);
+    mbar_arrive(&s.bar_sched_empty[slot]);
+    return u;
+  };
+
   if (warp == kVecWarps) {
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(&s.bar_qdo, 4 * kT * 128);
-      tma_load_2d(s.q[0], &tm_q, &s.bar_qdo, 0, q_row0);
-      tma_load_2d(s.q[1], &tm_q, &s.bar_qdo, 64, q_row0);
-      tma_load_2d(s.dout[0], &tm_do, &s.bar_qdo, 0, q_row0);
-      tma_load_2d(s.dout[1], &tm_do, &s.bar_qdo, 64, q_row0);
-      int issued_k = 0, issued_v = 0;
+    // ------------------------------------------------------------------ scheduler + TMA producer
+    if (lane == 0) {
+      int jk = 0, jv = 0, ucount = 0;
       bool ok = true;
-      auto load_v = [&](int jv) -> bool {
+      auto load_v = [&](int rp, int kv_row0, int j) -> bool {
         const int sv = jv % kQVStages, uv = jv / kQVStages;
         if (jv >= kQVStages && !mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status)) return false;
-        const int vrow = kv_row0 + prm.col[rp + jv] * prm.by;
+        const int vrow = kv_row0 + prm.col[rp + j] * prm.by;
         mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
         tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
         tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
-        issued_v = jv + 1;
+        ++jv;
         return true;
       };
-      for (int j = 0; ok && j < n; ++j) {
-        const int sk = j % kQKStages, uk = j / kQKStages;
-        if (j >= kQKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
-        const int row = kv_row0 + prm.col[rp + j] * prm.by;
-        mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
-        tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
-        tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
-        issued_k = j + 1;
-        const int jv = j - (kQKStages - kQVStages);  // V trails K by one tile
-        if (jv >= 0) ok = load_v(jv);
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kSchedKv;
+        if (k >= kSchedKv && !(ok = mbar_wait(&s.bar_sched_empty[slot], ((k / kSchedKv) - 1) & 1, prm.status)))
+          break;
+        int i = atomicAdd(prm.next_unit, 1);
+        if (i >= units) i = -1;
+        s.sched[slot] = i;
+        mbar_arrive(&s.bar_sched_full[slot]);
+        if (i < 0) break;
+        int bh, qb, rp, n;
+        unit_of(i, bh, qb, rp, n);
+        if (n == 0) continue;
+        const int b = bh / prm.N1, g = (bh % prm.N1) / (prm.N1 / prm.N2);
+        const int q_row0 = bh * prm.S_q + qb * prm.bx;
+        const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
+        if (ucount > 0 && !(ok = mbar_wait(&s.bar_qdo_empty, (ucount - 1) & 1, prm.status))) break;
+        mbar_arrive_expect_tx(&s.bar_qdo, 4 * kT * 128);
+        tma_load_2d(s.q[0], &tm_q, &s.bar_qdo, 0, q_row0);
+        tma_load_2d(s.q[1], &tm_q, &s.bar_qdo, 64, q_row0);
+        tma_load_2d(s.dout[0], &tm_do, &s.bar_qdo, 0, q_row0);
+        tma_load_2d(s.dout[1], &tm_do, &s.bar_qdo, 64, q_row0);
+        ++ucount;
+        for (int j = 0; ok && j < n; ++j) {
+          const int sk = jk % kQKStages, uk = jk / kQKStages;
+          if (jk >= kQKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
+          const int row = kv_row0 + prm.col[rp + j] * prm.by;
+          mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
+          tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
+          tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
+          ++jk;
+          if (j >= kQKStages - kQVStages) ok = load_v(rp, kv_row0, j - (kQKStages - kQVStages));  // V trails K
+        }
+        for (int j = n - (kQKStages - kQVStages); ok && j < n; ++j)
+          if (j >= 0) ok = load_v(rp, kv_row0, j);
       }
-      for (int jv = issued_v; ok && jv < n; ++jv) ok = load_v(jv);
-      for (int j = (issued_k > kQKStages ? issued_k - kQKStages : 0); j < issued_k; ++j)
+      // do not leave the CTA with copies in flight
+      for (int j = (jk > kQKStages ? jk - kQKStages : 0); j < jk; ++j)
         mbar_wait(&s.bar_k[j % kQKStages], (j / kQKStages) & 1, prm.status);
-      for (int j = (issued_v > kQVStages ? issued_v - kQVStages : 0); j < issued_v; ++j)
+      for (int j = (jv > kQVStages ? jv - kQVStages : 0); j < jv; ++j)
         mbar_wait(&s.bar_v[j % kQVStages], (j / kQVStages) & 1, prm.status);
-      mbar_wait(&s.bar_qdo, 0, prm.status);
+      if (ucount > 0) mbar_wait(&s.bar_qdo, (ucount - 1) & 1, prm.status);
     }
-  } else if (warp == kVecWarps + 1) {
-    if (lane == 0 && n > 0) {
+  } else if (warp == kVecWarps + 1 || warp == kVecWarps + 2) {
+    // ------------------------------------------------------------------ MMA issuers
+    if (lane == 0) {
+      const bool dq_thread = warp == kVecWarps + 1;
       const uint32_t id_s = idesc_bf16_f32(kT, BN, false, false);
       const uint32_t id_dq = idesc_bf16_f32(kT, kD, false, true);
       // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
@@ -589,148 +633,174 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), 0, 1024);
       const uint64_t dkm0 = sdesc_sw128(smem_u32(s.k[0][0]), BN * 128, 1024);  // K as MN-major B of dQ
       constexpr uint32_t kKv16 = (2 * BN * 128) >> 4;  // one K or V stage, in 16-byte units
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1, sk = j % kQKStages;
-        if (!mbar_wait(&s.bar_k[sk], (j / kQKStages) & 1, prm.status)) return false;
-        tc_fence_after();
-        const uint64_t dk = dk0 + static_cast<uint64_t>(sk) * kKv16;
+      int J0 = 0, ucount = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int i = next_from_ring(k);
+        if (i < 0) break;
+        int bh, qb, rp, n;
+        unit_of(i, bh, qb, rp, n);
+        if (n == 0) continue;
+        if (dq_thread) {
+          for (int j = 0; ok && j < n; ++j) {
+            const int J = J0 + j, st = J & 1, sk = J % kQKStages;
+            if (!(ok = mbar_wait(&s.bar_ds_ready[st], (J >> 1) & 1, prm.status))) break;
+            tc_fence_after();
+            const uint32_t s_col = st ? kColS1 : kColS0;
+            const uint64_t dkm = dkm0 + static_cast<uint64_t>(sk) * kKv16;
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks)
-          mma_bf16_ss(tmem + (st ? kColS1 : kColS0), sdesc_add(dq0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
-                      sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
-        tc_commit(&s.bar_s_full[st]);
-        return true;
-      };
-      auto issue_dp = [&](int j) -> bool {
-        const int sv = j % kQVStages;
-        if (!mbar_wait(&s.bar_v[sv], (j / kQVStages) & 1, prm.status)) return false;
-        tc_fence_after();
-        const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * kKv16;
+            for (int half = 0; half < 2; ++half)
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks)
-          mma_bf16_ss(tmem + kColDP, sdesc_add(ddo0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
-                      sdesc_add(dv, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
-        tc_commit(&s.bar_dp_full);
-        tc_commit(&s.bar_v_empty[sv]);
-        return true;
-      };
-      bool ok = mbar_wait(&s.bar_qdo, 0, prm.status);
-      if (ok) ok = issue_s(0);
-      if (ok) ok = issue_dp(0);
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1;
-        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(&s.bar_ds_ready, j & 1, prm.status))) break;
-        tc_fence_after();
-        const uint32_t s_col = st ? kColS1 : kColS0;
-        const int sk = j % kQKStages;
-        const uint64_t dkm = dkm0 + static_cast<uint64_t>(sk) * kKv16;
+              for (int ks = 0; ks < BN / 16; ++ks)
+                mma_bf16_ts(tmem + kColDQ, tmem + s_col + half * (BN / 2) + ks * 8, sdesc_add(dkm, ks * 2048),
+                            id_dq, (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(&s.bar_k_empty[sk]);
+            tc_commit(&s.bar_dq_done[st]);
+          }
+          if (ok) tc_commit(&s.bar_done);
+        } else {
+          if (!(ok = mbar_wait(&s.bar_qdo, ucount & 1, prm.status))) break;
+          ++ucount;
+          for (int j = 0; ok && j < n; ++j) {
+            const int J = J0 + j, st = J & 1, sk = J % kQKStages, sv = J % kQVStages;
+            // S buffer st last held dS_{J-2}, read by dQ_{J-2}
+            if (J >= 2 && !(ok = mbar_wait(&s.bar_dq_done[st], ((J >> 1) - 1) & 1, prm.status))) break;
+            if (!(ok = mbar_wait(&s.bar_k[sk], (J / kQKStages) & 1, prm.status))) break;
+            tc_fence_after();
+            const uint64_t dk = dk0 + static_cast<uint64_t>(sk) * kKv16;
 #pragma unroll
-        for (int half = 0; half < 2; ++half)
+            for (int ks = 0; ks < kD / 16; ++ks)
+              mma_bf16_ss(tmem + (st ? kColS1 : kColS0), sdesc_add(dq0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
+                          sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
+            tc_commit(&s.bar_s_full[st]);
+            // dP has one buffer: dP_{J-1} has been read once dS_{J-1} is written
+            if (J >= 1 && !(ok = mbar_wait(&s.bar_ds_ready[(J - 1) & 1], ((J - 1) >> 1) & 1, prm.status))) break;
+            if (!(ok = mbar_wait(&s.bar_v[sv], (J / kQVStages) & 1, prm.status))) break;
+            tc_fence_after();
+            const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * kKv16;
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_bf16_ts(tmem + kColDQ, tmem + s_col + half * (BN / 2) + ks * 8, sdesc_add(dkm, ks * 2048), id_dq,
-                        (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
-        tc_commit(&s.bar_k_empty[sk]);
-        if (j + 1 < n && !(ok = issue_dp(j + 1))) break;
+            for (int ks = 0; ks < kD / 16; ++ks)
+              mma_bf16_ss(tmem + kColDP, sdesc_add(ddo0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
+                          sdesc_add(dv, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
+            tc_commit(&s.bar_dp_full);
+            tc_commit(&s.bar_v_empty[sv]);
+            if (j + 1 == n) tc_commit(&s.bar_qdo_empty);  // the unit's last read of Q and dO
+          }
+        }
+        J0 += n;
       }
-      if (ok) tc_commit(&s.bar_done);
     }
   } else {
+    // ------------------------------------------------------------------ P / dS warps
     constexpr int kHalf = BN / 2;
     const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // query row == TMEM lane
     const int c0 = hf * kHalf;          // this thread's key columns [c0, c0 + BN/2)
-    const int qpos = qb * prm.bx + r;
-    const bool row_valid = r < prm.bx && qpos < prm.S_q;
-    int lo = 0, hi = prm.S_kv - 1;
-    const int qq = qpos + prm.S_kv - prm.S_q;
-    if (prm.mask_mode == 2) hi = min(hi, qpos);
-    else if (prm.mask_mode == 3) hi = min(hi, qq);
-    else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
-    if (!row_valid) { lo = 1; hi = 0; }
-    const size_t trow = static_cast<size_t>(unit) * kT + r;
-    const uint64_t nl2 = f2_pack(prm.lse2[trow], prm.lse2[trow]);  // -LSE*log2e of the row, twice
-    const uint64_t nd2 = f2_pack(prm.dvec[trow], prm.dvec[trow]);  // -D of the row, twice
     const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int exchanges = 0;
+    int exchanges = 0, J0 = 0, done_count = 0;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int st = j & 1;
-      const uint32_t s_col = st ? kColS1 : kColS0;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (j >> 1) & 1, prm.status));
-      if (!ok) break;
-      tc_fence_after();
-      const int kpos0 = prm.col[rp + j] * prm.by + c0;
-      const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
-      float p[kHalf];
+    for (int k = 0; ok; ++k) {
+      const int i = __shfl_sync(0xffffffffu, next_from_ring(k), 0);
+      if (i < 0) break;
+      int bh, qb, rp, n;
+      unit_of(i, bh, qb, rp, n);
+      const int q_row0 = bh * prm.S_q + qb * prm.bx;
+      const int qpos = qb * prm.bx + r;
+      const bool row_valid = r < prm.bx && qpos < prm.S_q;
+      int lo = 0, hi = prm.S_kv - 1;
+      const int qq = qpos + prm.S_kv - prm.S_q;
+      if (prm.mask_mode == 2) hi = min(hi, qpos);
+      else if (prm.mask_mode == 3) hi = min(hi, qq);
+      else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
+      if (!row_valid) { lo = 1; hi = 0; }
+      const size_t trow = static_cast<size_t>(bh * prm.nqb + qb) * kT + r;
+      const uint64_t nl2 = f2_pack(prm.lse2[trow], prm.lse2[trow]);  // -LSE*log2e of the row, twice
+      const uint64_t nd2 = f2_pack(prm.dvec[trow], prm.dvec[trow]);  // -D of the row, twice
+      for (int j = 0; j < n; ++j) {
+        const int J = J0 + j, st = J & 1;
+        const uint32_t s_col = st ? kColS1 : kColS0;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (J >> 1) & 1, prm.status));
+        if (!ok) break;
+        tc_fence_after();
+        const int kpos0 = prm.col[rp + j] * prm.by + c0;
+        const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
+        float p[kHalf];
 #pragma unroll
-      for (int c = 0; c < kHalf; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + s_col + c0 + c, rr);
-        tmem_ld_wait(rr);
+        for (int c = 0; c < kHalf; c += 32) {
+          uint32_t rr[32];
+          tmem_ld32(tmem + lane_base + s_col + c0 + c, rr);
+          tmem_ld_wait(rr);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float t0, t1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(rr[i]), __uint_as_float(rr[i + 1])), sc2, nl2), t0, t1);
-          p[c + i] = ex2(t0);
-          p[c + i + 1] = ex2(t1);
+          for (int i2 = 0; i2 < 32; i2 += 2) {
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(rr[i2]), __uint_as_float(rr[i2 + 1])), sc2, nl2), t0, t1);
+            p[c + i2] = ex2(t0);
+            p[c + i2 + 1] = ex2(t1);
+          }
         }
-      }
-      if (!full) {
+        if (!full) {
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c) {
-          const int kp = kpos0 + c;
-          if (kp < lo || kp > hi) p[c] = 0.f;
+          for (int c = 0; c < kHalf; ++c) {
+            const int kp = kpos0 + c;
+            if (kp < lo || kp > hi) p[c] = 0.f;
+          }
         }
+        // dp_full has one phase per tile; its next phase needs dS_J from this thread
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, J & 1, prm.status));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t hv[kHalf / 2], lv[kHalf / 2];
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 32) {
+          uint32_t rr[32];
+          tmem_ld32(tmem + lane_base + kColDP + c0 + c, rr);
+          tmem_ld_wait(rr);
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2)
+            split_pack2(f2_mul(f2_pack(p[c + 2 * i2], p[c + 2 * i2 + 1]),
+                               f2_add(f2_pack(__uint_as_float(rr[2 * i2]), __uint_as_float(rr[2 * i2 + 1])), nd2)),
+                        hv[c / 2 + i2], lv[c / 2 + i2]);
+        }
+        // both halves have read S_J before either writes dS over it:
+        // hi -> S_J[c0/2, +BN/4), lo -> S_J[BN/2 + c0/2, +BN/4)
+        ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
+        if (!ok) break;
+#pragma unroll
+        for (int c = 0; c < kHalf / 2; c += 16) {
+          tmem_st16(tmem + lane_base + s_col + c0 / 2 + c, hv + c);
+          tmem_st16(tmem + lane_base + s_col + BN / 2 + c0 / 2 + c, lv + c);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&s.bar_ds_ready[st]);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, j & 1, prm.status));
       if (!ok) break;
-      tc_fence_after();
-      uint32_t hv[kHalf / 2], lv[kHalf / 2];
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColDP + c0 + c, rr);
-        tmem_ld_wait(rr);
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          split_pack2(f2_mul(f2_pack(p[c + 2 * i], p[c + 2 * i + 1]),
-                             f2_add(f2_pack(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1])), nd2)),
-                      hv[c / 2 + i], lv[c / 2 + i]);
-      }
-      // both halves have read S_j before either writes dS over it:
-      // hi -> S_j[c0/2, +BN/4), lo -> S_j[BN/2 + c0/2, +BN/4)
-      ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
-      if (!ok) break;
-#pragma unroll
-      for (int c = 0; c < kHalf / 2; c += 16) {
-        tmem_st16(tmem + lane_base + s_col + c0 / 2 + c, hv + c);
-        tmem_st16(tmem + lane_base + s_col + BN / 2 + c0 / 2 + c, lv + c);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&s.bar_ds_ready);
-    }
-    bool have = ok && n > 0;
-    if (have) {
-      have = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, 0, prm.status));
-      tc_fence_after();
-    }
-    const int d0 = hf * (kD / 2);  // this thread's head-dim columns of dQ
-    __nv_bfloat16* dqrow = prm.dq + static_cast<size_t>(q_row0 + r) * kD + d0;
-#pragma unroll
-    for (int c = 0; c < kD / 2; c += 32) {
-      uint32_t rr[32];
+      // ---- epilogue: dQ = scale * acc (this thread: head-dim columns [hf*64, +64))
+      const bool have = n > 0;
       if (have) {
-        tmem_ld32(tmem + lane_base + kColDQ + d0 + c, rr);
-        tmem_ld_wait(rr);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rr[i] = 0u;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_done, done_count & 1, prm.status));
+        ++done_count;
+        if (!ok) break;
+        tc_fence_after();
       }
-      if (row_valid) store_row_bf16(dqrow + c, rr, prm.scale);
+      const int d0 = hf * (kD / 2);
+      __nv_bfloat16* dqrow = prm.dq + static_cast<size_t>(q_row0 + r) * kD + d0;
+#pragma unroll
+      for (int c = 0; c < kD / 2; c += 32) {
+        uint32_t rr[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + kColDQ + d0 + c, rr);
+          tmem_ld_wait(rr);
+        } else {
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2) rr[i2] = 0u;
+        }
+        if (row_valid) store_row_bf16(dqrow + c, rr, prm.scale);
+      }
+      // dQ has been read: the next unit's first dQ product waits for its dS, which comes after
+      tc_fence_before();
+      J0 += n;
     }
   }
   tc_fence_before();
@@ -745,7 +815,7 @@ cudaError_t launch_q(const BwdParams& p, const CUtensorMap& tq, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(bsa_bwd_q_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   prof_begin("bsa_bwd_q", st);
-  bsa_bwd_q_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, p);
+  if (grid > 0) bsa_bwd_q_kernel<BN><<<grid, kKvThreads, smem, st>>>(tq, tk, tv, tdo, p);
   prof_end(st);
   return cudaGetLastError();
 }
@@ -803,10 +873,15 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // Q-major pass
+  // Q-major pass (persistent)
   p.row_ptr = a.row_ptr;
   p.col = a.col;
-  const int grid = a.B * a.N1 * a.nqb;
+  p.next_unit = a.next_q;
+  const int q_units = a.B * a.N1 * a.nqb;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = q_units < sms ? q_units : sms;
   if (a.by == 128) return launch_q<128>(p, tq, tk, tv, tdo, grid, st);
   return launch_q<64>(p, tq, tk, tv, tdo, grid, st);
 }
