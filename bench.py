@@ -44,11 +44,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
 # kernel's source file is unchanged (sha1 prefix of the file recorded at capture time).
 NCU_TRAFFIC = {
-    # profiles/bsa_S8192_fwd_bwd_v1.md (dram__bytes_read.sum + dram__bytes_write.sum)
-    "bsa_bwd_kv": {"bytes": 270701056 + 106852864, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                   "src_sha1": "2c7caf740969"},
-    "bsa_fwd": {"bytes": 201472768 + 49305344, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
-                "src_sha1": "42bb769e5322"},
+    # profiles/bsa_S8192_fwd_bwd.md (dram__bytes_read.sum + dram__bytes_write.sum, one launch)
+    "bsa_bwd_kv": {"bytes": 270780160 + 104547328, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                   "src_sha1": "c2bcda8c6f15"},
+    "bsa_bwd_q": {"bytes": 270909696 + 51656192, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                  "src_sha1": "c2bcda8c6f15"},
+    "bsa_fwd": {"bytes": 201515008 + 51768320, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+                "src_sha1": "d34d6d9c1339"},
 }
 
 
