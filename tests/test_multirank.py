@@ -1,0 +1,60 @@
+"""The multi-process plumbing bench.py uses for N > 1 (one process per GPU on the GPUs): a barrier,
+the max over ranks of the measured time, and rank 0 alone printing, run here as two gloo ranks
+on the CPU."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        barrier, max_over_ranks = bench._dist_helpers(world, torch.device("cpu"))
+        barrier()
+        results[rank] = max_over_ranks(1.5 + rank)  # each rank's "time"; all must see the max
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        results = mgr.dict()
+        mp.spawn(_rank_main, args=(world, port, results), nprocs=world, join=True)
+        assert dict(results) == {0: 2.5, 1: 2.5}
+
+
+def test_single_rank_helpers_are_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    barrier, max_over_ranks = bench._dist_helpers(1, torch.device("cpu"))
+    barrier()
+    assert max_over_ranks(3.25) == 3.25
+
+
+def test_reference_arm_other_ranks_print_nothing(capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Args:
+        config, steps, warmup, ref_step_seconds, nsa_seqlens = 1, 1, 3, 1.0, ""
+
+    bench.run_reference(Args(), rank=1, world=2)
+    assert capsys.readouterr().out == ""
