@@ -58,6 +58,7 @@ def _run(pb, scale=None):
     dict(B=2, N1=64, N2=1, page=64, n_logical=20, K=9, sbs=128, seqused=[1280, 1250]),   # G = 64, 2 pages/block
     dict(B=2, N1=128, N2=2, page=32, n_logical=24, K=5, sbs=64, seqused=[768, 600]),     # two kv heads, 32-token pages
     dict(B=1, N1=128, N2=1, page=64, n_logical=8, K=8, sbs=64, seqused=[512]),           # every block selected
+    dict(B=3, N1=128, N2=1, page=64, n_logical=8, K=4, sbs=64, seqused=[512, 0, 130]),   # an empty batch
 ])
 def test_sfa_decode_cases(cuda_ok, case):
     pb = _problem(**case, seed=21)
