@@ -127,14 +127,14 @@ __device__ __forceinline__ void split_pack2(uint64_t x, uint32_t& hi, uint32_t& 
 // walks each block's transposed list.  Every entry (a 128-row Q tile of one of the group's heads)
 // runs as two 64-row halves, so the element-wise work on one half overlaps the tensor-core work of
 // the neighbouring halves:
-//   TMEM columns: half buffers 0 [0,128) and 1 [128,256), each S^T [0,64) | dP^T [64,128) of one
-//   half (128 keys x 64 query rows); dV [256,384), dK [384,512).  After the 8 element-wise warps
-//   have read S^T and dP^T of a half they write the bf16 A operands over them: P^T hi -> [0,32),
-//   lo -> [32,64), dS^T hi -> [64,96), lo -> [96,128) (64 query rows -> 32 packed columns).
+//   TMEM columns: scores S^T [0,64) | dP^T [64,128) of one half (128 keys x 64 query rows); the
+//   bf16 A operands of the products P^T hi [128,160), lo [160,192), dS^T hi [192,224), lo
+//   [224,256) (64 query rows -> 32 packed columns); dV [256,384), dK [384,512).
+//   The score buffer is released as soon as the 8 element-wise warps have loaded it into
+//   registers, so S^T / dP^T of half x + 1 run on the tensor cores while the warps turn half x into
+//   P and dS; those go to the operand buffer once the products of half x - 1 have read it.
 //   Shared memory: the block's K and V tiles, and a 4-stage ring of half entries (64 rows of Q
 //   and dO with their D and LSE*log2e values), so loads run two half-steps ahead.
-//   MMA order per half x: dV += P^T dO, dK += dS^T Q (hi, lo), then S^T / dP^T of half x + 2
-//   into the buffer just consumed.
 // ------------------------------------------------------------------------------------------------
 constexpr int kHalfRows = 64;
 constexpr int kKvRing = 4;
@@ -154,10 +154,12 @@ struct __align__(1024) KvSmem {
   int32_t sched[kSchedKv];
   uint64_t bar_kv, bar_kv_empty;
   uint64_t bar_qdo[kKvRing], bar_qdo_empty[kKvRing];
-  uint64_t bar_sdp_full[2], bar_pds_ready[2], bar_done;
-  uint64_t bar_grads_done[2];  // per half buffer: its products have completed (buffer reusable)
+  uint64_t bar_sdp_full;    // S^T / dP^T of the current half are in the score buffer
+  uint64_t bar_sdp_free;    // the element-wise warps have loaded them (256 arrivals)
+  uint64_t bar_pds_ready;   // P^T / dS^T of the half are in the operand buffer (256 arrivals)
+  uint64_t bar_grads_done;  // the products of the half have completed (operand buffer reusable)
+  uint64_t bar_done;
   uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
-  uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
 
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
                       const BwdParams prm) {
-  constexpr uint32_t kColDV = 256, kColDK = 384;
+  constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   KvSmem& s = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -179,17 +181,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&s.bar_qdo[i], 1);
       mbar_init(&s.bar_qdo_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.bar_sdp_full[i], 1);
-      mbar_init(&s.bar_pds_ready[i], kVecWarps * 32);
-    }
+    mbar_init(&s.bar_sdp_full, 1);
+    mbar_init(&s.bar_sdp_free, kVecWarps * 32);
+    mbar_init(&s.bar_pds_ready, kVecWarps * 32);
+    mbar_init(&s.bar_grads_done, 1);
     mbar_init(&s.bar_done, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&s.bar_grads_done[i], 1);
     for (int i = 0; i < kSchedKv; ++i) {
       mbar_init(&s.bar_sched_full[i], 1);
       mbar_init(&s.bar_sched_empty[i], 2 + kVecWarps * 32);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -291,12 +291,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0][0]), kHalfRows * 128, 1024);      // MN-major
       const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0][0]), kHalfRows * 128, 1024);
       constexpr uint32_t kStage16 = (2 * kHalfRows * 128) >> 4;  // one ring stage, in 16-byte units
-      // S^T = K Q_h^T and dP^T = V dO_h^T of global half hx into half buffer hx & 1
+      // S^T = K Q_h^T and dP^T = V dO_h^T of global half hx into the score buffer
       auto sdp = [&](int hx) -> bool {
-        const int hs = hx % kKvRing, buf = hx & 1;
+        const int hs = hx % kKvRing;
         if (!mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status)) return false;
         tc_fence_after();
-        const uint32_t d = tmem + buf * 128;
+        const uint32_t d = tmem + kColS;
         const uint64_t dq = dq0 + static_cast<uint64_t>(hs) * kStage16;
         const uint64_t ddo = ddo0 + static_cast<uint64_t>(hs) * kStage16;
 #pragma unroll
@@ -307,9 +307,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
-          mma_bf16_ss(d + 64, sdesc_add(dv0, ko), sdesc_add(ddo, qo), id_sdp, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(d + (kColDP - kColS), sdesc_add(dv0, ko), sdesc_add(ddo, qo), id_sdp, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&s.bar_sdp_full[buf]);
+        tc_commit(&s.bar_sdp_full);
         return true;
       };
       // acc += A (TMEM, 128 keys x 64 query rows) . B (the half's [64 rows][128 d], MN-major)
@@ -328,30 +328,29 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (grads_thread) {
           // dV += P^T dO and dK += dS^T Q (hi, lo) as soon as the element-wise warps have a half
           for (int x = 0; ok && x < nh; ++x) {
-            const int hx = G0 + x, buf = hx & 1, hs = hx % kKvRing;
-            if (!(ok = mbar_wait(&s.bar_pds_ready[buf], (hx >> 1) & 1, prm.status))) break;
+            const int hx = G0 + x, hs = hx % kKvRing;
+            // exact parity: the next phase needs the warps' P / dS of half hx + 1, which wait for
+            // the grads_done commit below
+            if (!(ok = mbar_wait(&s.bar_pds_ready, hx & 1, prm.status))) break;
             tc_fence_after();
-            const uint32_t b0 = buf * 128;
             const uint64_t ddom = ddom0 + static_cast<uint64_t>(hs) * kStage16;
             const uint64_t dqm = dqm0 + static_cast<uint64_t>(hs) * kStage16;
-            grad(tmem + kColDV, b0, ddom, x > 0);        // dV += P^T_hi dO
-            grad(tmem + kColDV, b0 + 32, ddom, true);    // dV += P^T_lo dO
-            grad(tmem + kColDK, b0 + 64, dqm, x > 0);    // dK += dS^T_hi Q
-            grad(tmem + kColDK, b0 + 96, dqm, true);     // dK += dS^T_lo Q
+            grad(tmem + kColDV, kColP, ddom, x > 0);        // dV += P^T_hi dO
+            grad(tmem + kColDV, kColP + 32, ddom, true);    // dV += P^T_lo dO
+            grad(tmem + kColDK, kColP + 64, dqm, x > 0);    // dK += dS^T_hi Q
+            grad(tmem + kColDK, kColP + 96, dqm, true);     // dK += dS^T_lo Q
             tc_commit(&s.bar_qdo_empty[hs]);
-            tc_commit(&s.bar_grads_done[buf]);          // half buffer hx & 1 may be overwritten
+            tc_commit(&s.bar_grads_done);                   // the operand buffer may be rewritten
           }
           if (ok) tc_commit(&s.bar_done);
         } else {
-          // S^T / dP^T of each half once its buffer's previous products have completed.  One
-          // barrier per buffer: its next phase needs an S^T this thread has not issued yet, so a
-          // parity wait always names the right phase (this thread may fall behind while it waits
-          // for the next block's K and V).
+          // S^T / dP^T of each half once the warps have loaded the previous half's scores.  Exact
+          // parity: the next phase of sdp_free needs the scores of half hx, issued after the wait.
           if (!(ok = mbar_wait(&s.bar_kv, ucount & 1, prm.status))) break;
           ++ucount;
           for (int x = 0; ok && x < nh; ++x) {
             const int hx = G0 + x;
-            if (hx >= 2 && !(ok = mbar_wait(&s.bar_grads_done[hx & 1], ((hx >> 1) - 1) & 1, prm.status))) break;
+            if (hx >= 1 && !(ok = mbar_wait(&s.bar_sdp_free, (hx - 1) & 1, prm.status))) break;
             if (!(ok = sdp(hx))) break;
             if (x + 1 == nh) tc_commit(&s.bar_kv_empty);  // the block's last read of K and V
           }
@@ -366,7 +365,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int c0 = hf * 32;             // this thread's query columns [c0, c0 + 32) of a half
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int shift = prm.S_kv - prm.S_q;
-    int exchanges = 0, G0 = 0, done_count = 0;
+    int G0 = 0, done_count = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int i = __shfl_sync(0xffffffffu, next_from_ring(k), 0);
@@ -382,20 +381,24 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       else if (prm.mask_mode == 4) { qlo = kpos - shift - prm.win_right; qhi = kpos - shift + prm.win_left; }
       if (!key_valid) { qlo = 1; qhi = 0; }
       for (int x = 0; x < 2 * n; ++x) {
-        const int hx = G0 + x, buf = hx & 1, hs = hx % kKvRing;
+        const int hx = G0 + x, hs = hx % kKvRing;
         int qrow, tile, qpos0;
         entry_rows(bg, prm.col[rp + (x >> 1)], qrow, tile, qpos0);
         const int qp0 = qpos0 + (x & 1) * kHalfRows + c0;  // query position of column c0
+        // exact parity: the next phase of sdp_full needs the sdp_free arrival below
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status) &&
-                                         mbar_wait(&s.bar_sdp_full[buf], (hx >> 1) & 1, prm.status));
+                                         mbar_wait(&s.bar_sdp_full, hx & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
         uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_base + buf * 128 + c0, sr);
-        tmem_ld32(tmem + lane_base + buf * 128 + 64 + c0, dr);
+        tmem_ld32(tmem + lane_base + kColS + c0, sr);
+        tmem_ld32(tmem + lane_base + kColDP + c0, dr);
         tmem_ld_wait(sr);
 #pragma unroll
         for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
+        // the score buffer is free for the next half's S^T / dP^T
+        tc_fence_before();
+        mbar_arrive(&s.bar_sdp_free);
         const float4* nl2 = reinterpret_cast<const float4*>(s.lse2[hs] + c0);  // -LSE*log2e per query row
         const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D per query row
         const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
@@ -423,17 +426,21 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             split_pack2(g2, dh[c / 2], dl[c / 2]);
           }
         }
-        // both warps of the quarter have read S^T and dP^T before either overwrites them
-        ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
-        if (!ok) break;
-        const uint32_t base = tmem + lane_base + buf * 128 + hf * 16;
+        // the operand buffer is free once the previous half's products have completed (exact
+        // parity: grads_done's next phase needs the pds_ready arrival below)
+        if (hx >= 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_grads_done, (hx - 1) & 1, prm.status));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint32_t base = tmem + lane_base + kColP + hf * 16;
         tmem_st16(base, ph);
         tmem_st16(base + 32, pl);
         tmem_st16(base + 64, dh);
         tmem_st16(base + 96, dl);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&s.bar_pds_ready[buf]);
+        mbar_arrive(&s.bar_pds_ready);
       }
       if (!ok) break;
       // ---- epilogue: dK = scale * acc, dV = acc (this thread: head-dim columns [hf*64, +64))
@@ -493,6 +500,7 @@ struct __align__(1024) QSmem {
   int32_t sched[kSchedKv];
   uint64_t bar_qdo, bar_qdo_empty, bar_k[kQKStages], bar_k_empty[kQKStages], bar_v[kQVStages], bar_v_empty[kQVStages];
   uint64_t bar_s_full[2], bar_dp_full, bar_ds_ready[2], bar_dq_done[2], bar_done;
+  uint64_t bar_dp_free;  // the element-wise warps have loaded dP of the current tile (256 arrivals)
   uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
   uint64_t bar_pair[4];
   uint32_t tmem_base;
@@ -530,6 +538,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&s.bar_dq_done[i], 1);
     }
     mbar_init(&s.bar_dp_full, 1);
+    mbar_init(&s.bar_dp_free, kVecWarps * 32);
     mbar_init(&s.bar_done, 1);
     for (int i = 0; i < kSchedKv; ++i) {
       mbar_init(&s.bar_sched_full[i], 1);
@@ -673,8 +682,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
               mma_bf16_ss(tmem + (st ? kColS1 : kColS0), sdesc_add(dq0, (ks >> 2) * (kT * 128) + (ks & 3) * 32),
                           sdesc_add(dk, (ks >> 2) * (BN * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
             tc_commit(&s.bar_s_full[st]);
-            // dP has one buffer: dP_{J-1} has been read once dS_{J-1} is written
-            if (J >= 1 && !(ok = mbar_wait(&s.bar_ds_ready[(J - 1) & 1], ((J - 1) >> 1) & 1, prm.status))) break;
+            // dP has one buffer: the warps have loaded dP_{J-1} (exact parity: the next phase of
+            // dp_free needs dP_J, issued after the wait)
+            if (J >= 1 && !(ok = mbar_wait(&s.bar_dp_free, (J - 1) & 1, prm.status))) break;
             if (!(ok = mbar_wait(&s.bar_v[sv], (J / kQVStages) & 1, prm.status))) break;
             tc_fence_after();
             const uint64_t dv = dv0 + static_cast<uint64_t>(sv) * kKv16;
@@ -746,7 +756,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             if (kp < lo || kp > hi) p[c] = 0.f;
           }
         }
-        // dp_full has one phase per tile; its next phase needs dS_J from this thread
+        // dp_full has one phase per tile; its next phase needs the dp_free arrival below
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, J & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
@@ -762,6 +772,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                                f2_add(f2_pack(__uint_as_float(rr[2 * i2]), __uint_as_float(rr[2 * i2 + 1])), nd2)),
                         hv[c / 2 + i2], lv[c / 2 + i2]);
         }
+        tc_fence_before();
+        mbar_arrive(&s.bar_dp_free);  // dP of tile J has been read: the next dP may overwrite it
         // both halves have read S_J before either writes dS over it:
         // hi -> S_J[c0/2, +BN/4), lo -> S_J[BN/2 + c0/2, +BN/4)
         ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
