@@ -79,7 +79,10 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks / throttle reasons, sampled every 50 ms from just before the timed region to
+    just after it.  Entering waits (at most 3 s) for the first sample, so sampling is live when the
+    timed steps start; summary() uses the samples taken inside the block, or, when the block was
+    shorter than the sampling period, the nearest sample on each side of it."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -88,25 +91,32 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (host time, csv line)
+        self.t_in = self.t_out = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            deadline = time.monotonic() + 3.0
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except (OSError, ValueError):
             self.proc = None
+        self.t_in = time.monotonic()
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def __exit__(self, *a):
+        self.t_out = time.monotonic()
         if self.proc is not None:
+            time.sleep(0.06)  # one more sample after the block
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -114,9 +124,15 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        inside = [ln for t, ln in self.lines if self.t_in <= t <= self.t_out]
+        window = "timed region"
+        if not inside:
+            before = [ln for t, ln in self.lines if t < self.t_in][-1:]
+            after = [ln for t, ln in self.lines if t > self.t_out][:1]
+            inside, window = before + after, "nearest samples around a timed region shorter than 50 ms"
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in inside:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -129,7 +145,7 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
 
 
 def bsa_workload(config: int):
