@@ -10,7 +10,8 @@
 // Shared memory: Q dims 256-511 and the rope part (5 x 16 KB), K tiles of 32 tokens x 576 dims
 // (2 stages x 9 boxes of 4 KB) and V tiles of 32 tokens x 256 dims (2 stages x 4 boxes).
 // Warps 0-7 softmax (lane quarter = head rows, half = 16 of the tile's 32 keys), warp 8 TMA
-// producer, warp 9 MMA issuer.  A piece covering a whole unit writes Out and LSE; otherwise it
+// producer, warp 9 issues O += P V, warp 10 issues S (tcgen05.mma issue blocks while the tensor
+// pipe's queue is full, so with one thread O += P_t V_t would wait behind the issue of S_{t+1}).  A piece covering a whole unit writes Out and LSE; otherwise it
 // writes (O, m, l) partials that sfa_combine merges in piece order.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -29,7 +30,7 @@ constexpr int kDVH = 256;     // Dv half per CTA
 constexpr int kKBoxes = 9;    // 8 boxes of k (64 dims) + 1 of k_rope
 constexpr int kVBoxes = 4;    // 4 boxes of v (64 dims) per Dv half
 constexpr int kVecWarps = 8;
-constexpr int kThreads = (kVecWarps + 2) * 32;
+constexpr int kThreads = (kVecWarps + 3) * 32;
 constexpr uint32_t kColO = 0, kColQ = 256, kColS0 = 384, kColS1 = 416;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -40,7 +41,9 @@ struct __align__(1024) DecSmem {
   uint8_t v[2][kVBoxes][kTile * 128];
   float red[2][2][kM];
   uint64_t bar_q, bar_qlo, bar_k[2], bar_k_empty[2], bar_v[2], bar_v_empty[2], bar_s_full[2];
-  uint64_t bar_p_full, bar_o_done, bar_done, bar_pair[4];
+  uint64_t bar_p_full[2];   // per S buffer: P of its tile is written (256 arrivals)
+  uint64_t bar_pv_done[2];  // per S buffer: the O += P V that read it has completed
+  uint64_t bar_o_done, bar_done, bar_pair[4];
   uint32_t tmem_base;
 };
 
@@ -102,7 +105,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_v_empty[i], 1);
       mbar_init(&s.bar_s_full[i], 1);
     }
-    mbar_init(&s.bar_p_full, kVecWarps * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.bar_p_full[i], kVecWarps * 32);
+      mbar_init(&s.bar_pv_done[i], 1);
+    }
     mbar_init(&s.bar_o_done, 1);
     mbar_init(&s.bar_done, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
@@ -147,54 +153,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) mbar_wait(&s.bar_v[j & 1], (j >> 1) & 1, prm.status);
       mbar_wait(&s.bar_q, 0, prm.status);
     }
-  } else if (warp == kVecWarps + 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kVecWarps + 1 || warp == kVecWarps + 2) {
+    // ------------------------------------------------------------------ MMA issuers
     if (lane == 0 && n_tiles > 0) {
-      const uint32_t id_s = idesc_bf16_f32(kM, kTile, false, false);
-      const uint32_t id_o = idesc_bf16_f32(kM, kDVH, false, true);
-      // descriptors of stage 0 / box 0; stages, boxes and K steps are added offsets
-      const uint64_t dqh = sdesc_sw128(smem_u32(s.qhi[0]), 0, 1024);
-      const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0][0]), 0, 1024);
-      const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), kTile * 128, 1024);
-      constexpr uint32_t kK16 = (kKBoxes * kTile * 128) >> 4, kV16 = (kVBoxes * kTile * 128) >> 4;
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&s.bar_k[st], (j >> 1) & 1, prm.status)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + (st ? kColS1 : kColS0);
-        const uint64_t dk = dk0 + static_cast<uint64_t>(st) * kK16;
-        // dims 0-255: A = Q from tensor memory; dims 256-575: A = Q from shared memory
+      const bool pv_thread = warp == kVecWarps + 1;
+      bool ok = true;
+      if (pv_thread) {
+        const uint32_t id_o = idesc_bf16_f32(kM, kDVH, false, true);
+        const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0][0]), kTile * 128, 1024);
+        constexpr uint32_t kV16 = (kVBoxes * kTile * 128) >> 4;
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int st = j & 1;
+          // one barrier per S buffer: its next phase needs S_{j+2}, which waits for this product
+          if (!(ok = mbar_wait(&s.bar_p_full[st], (j >> 1) & 1, prm.status))) break;
+          if (!(ok = mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status))) break;
+          tc_fence_after();
+          const uint32_t p_col = st ? kColS1 : kColS0;
+          const uint64_t dv = dv0 + static_cast<uint64_t>(st) * kV16;
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks)
-          mma_bf16_ts(d, tmem + kColQ + ks * 8, sdesc_add(dk, (ks >> 2) * (kTile * 128) + (ks & 3) * 32), id_s,
-                      ks > 0 ? 1u : 0u);
-#pragma unroll
-        for (int ks = 16; ks < 36; ++ks) {
-          const int qs = ks - 16;
-          mma_bf16_ss(d, sdesc_add(dqh, (qs >> 2) * (kM * 128) + (qs & 3) * 32),
-                      sdesc_add(dk, (ks >> 2) * (kTile * 128) + (ks & 3) * 32), id_s, 1u);
+          for (int ks = 0; ks < kTile / 16; ++ks)
+            mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, sdesc_add(dv, ks * 2048), id_o,
+                        (j > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(&s.bar_o_done);
+          tc_commit(&s.bar_v_empty[st]);
+          tc_commit(&s.bar_pv_done[st]);
         }
-        tc_commit(&s.bar_s_full[st]);
-        tc_commit(&s.bar_k_empty[st]);
-        return true;
-      };
-      bool ok = mbar_wait(&s.bar_q, 0, prm.status) && mbar_wait(&s.bar_qlo, 0, prm.status);
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(&s.bar_p_full, j & 1, prm.status))) break;
-        const int st = j & 1;
-        if (!(ok = mbar_wait(&s.bar_v[st], (j >> 1) & 1, prm.status))) break;
-        tc_fence_after();
-        const uint32_t p_col = st ? kColS1 : kColS0;
-        const uint64_t dv = dv0 + static_cast<uint64_t>(st) * kV16;
+        if (ok) tc_commit(&s.bar_done);
+      } else {
+        const uint32_t id_s = idesc_bf16_f32(kM, kTile, false, false);
+        // descriptors of stage 0 / box 0; stages, boxes and K steps are added offsets
+        const uint64_t dqh = sdesc_sw128(smem_u32(s.qhi[0]), 0, 1024);
+        const uint64_t dk0 = sdesc_sw128(smem_u32(s.k[0][0]), 0, 1024);
+        constexpr uint32_t kK16 = (kKBoxes * kTile * 128) >> 4;
+        ok = mbar_wait(&s.bar_q, 0, prm.status) && mbar_wait(&s.bar_qlo, 0, prm.status);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int st = j & 1;
+          // S buffer st last held P_{j-2}; exact parity: pv_done's next phase needs P_j
+          if (j >= 2 && !(ok = mbar_wait(&s.bar_pv_done[st], ((j >> 1) - 1) & 1, prm.status))) break;
+          if (!(ok = mbar_wait(&s.bar_k[st], (j >> 1) & 1, prm.status))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + (st ? kColS1 : kColS0);
+          const uint64_t dk = dk0 + static_cast<uint64_t>(st) * kK16;
+          // dims 0-255: A = Q from tensor memory; dims 256-575: A = Q from shared memory
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_bf16_ts(tmem + kColO, tmem + p_col + ks * 8, sdesc_add(dv, ks * 2048), id_o, (j > 0 || ks > 0) ? 1u : 0u);
-        tc_commit(&s.bar_o_done);
-        tc_commit(&s.bar_v_empty[st]);
+          for (int ks = 0; ks < 16; ++ks)
+            mma_bf16_ts(d, tmem + kColQ + ks * 8, sdesc_add(dk, (ks >> 2) * (kTile * 128) + (ks & 3) * 32), id_s,
+                        ks > 0 ? 1u : 0u);
+#pragma unroll
+          for (int ks = 16; ks < 36; ++ks) {
+            const int qs = ks - 16;
+            mma_bf16_ss(d, sdesc_add(dqh, (qs >> 2) * (kM * 128) + (qs & 3) * 32),
+                        sdesc_add(dk, (ks >> 2) * (kTile * 128) + (ks & 3) * 32), id_s, 1u);
+          }
+          tc_commit(&s.bar_s_full[st]);
+          tc_commit(&s.bar_k_empty[st]);
+        }
       }
-      if (ok) tc_commit(&s.bar_done);
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
@@ -259,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_new = mx;
       }
       if (__any_sync(0xffffffffu, need)) {
-        // o_done phase j-1 (O += P_{j-1} V_{j-1}); phase j-2 is complete (S_j committed after it)
+        // o_done phase j-1 (O += P_{j-1} V_{j-1}); phase j-2 is complete (S_j waited for it)
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_o_done, (j - 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
@@ -291,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l += rs;
       m = m_new;
       tc_fence_before();
-      mbar_arrive(&s.bar_p_full);
+      mbar_arrive(&s.bar_p_full[st]);
     }
     // ---- epilogue
     bool have = ok && n_tiles > 0;
