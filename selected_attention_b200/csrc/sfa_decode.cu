@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sfa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
                       const __grid_constant__ CUtensorMap tm_v, const DecParams prm) {
+  griddep_launch_dependents();  // the combine may launch now; it waits for this grid's results
+  griddep_wait();               // launched early: the work list must be complete
   const int piece = blockIdx.x;
   if (piece >= *prm.n_pieces) return;  // uniform for the whole CTA
   extern __shared__ uint8_t smem_raw[];
@@ -369,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Out = sum O_p 2^(m_p - M) / L,  LSE = (M + log2 L) ln 2.  One warp per (unit, head row); each
 // lane owns 8 of the 256 Dv columns, so every partial row is read with coalesced 16-byte loads.
 __global__ void __launch_bounds__(256) sfa_combine_kernel(const DecParams prm, const int32_t* __restrict__ unit_first) {
+  griddep_wait();  // launched early: the decode pieces must be complete
   const int u = blockIdx.x;
   const int r = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -427,13 +430,13 @@ cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(sfa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   prof_begin("sfa_decode", st);
-  sfa_decode_kernel<<<a.max_pieces, kThreads, smem, st>>>(tq, tqr, tk, tkr, tv, p);
+  e = launch_pdl(sfa_decode_kernel, dim3(a.max_pieces), dim3(kThreads), smem, st, tq, tqr, tk, tkr, tv, p);
   prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
   prof_begin("sfa_combine", st);
-  sfa_combine_kernel<<<dim3(a.units, (p.G + 7) / 8), 256, 0, st>>>(p, a.unit_first);
+  e = launch_pdl(sfa_combine_kernel, dim3(a.units, (p.G + 7) / 8), dim3(256), 0, st, p, a.unit_first);
   prof_end(st);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sa

@@ -25,6 +25,7 @@ __global__ void sfa_page_list_kernel(const int32_t* __restrict__ sparse_indices,
                                      int page_size, int max_pages_per_seq, int num_pages, int32_t* __restrict__ pages,
                                      int32_t* __restrict__ tokens, int32_t* __restrict__ count,
                                      uint32_t* __restrict__ status) {
+  griddep_launch_dependents();  // the work list may launch now; it waits for this grid's results
   const int bg = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (bg >= B * N2) return;
@@ -87,6 +88,8 @@ __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __re
   __shared__ int s_chunk;
   __shared__ int warp_tot[32];
   __shared__ int carry;
+  griddep_launch_dependents();
+  griddep_wait();  // launched early (programmatic dependent launch): the page counts must be complete
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   if (tid == 0) s_max = 1;
   __syncthreads();
@@ -174,10 +177,10 @@ cudaError_t sfa_work_list(const int32_t* count, int units, int G, int32_t* piece
                           int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces, int32_t* n_pieces,
                           cudaStream_t st) {
   prof_begin("sfa_work_list", st);
-  sfa_work_list_kernel<<<1, 1024, 0, st>>>(count, units, G, piece_unit, piece_begin, piece_len, unit_first,
-                                           unit_pieces, n_pieces);
+  cudaError_t e = launch_pdl(sfa_work_list_kernel, dim3(1), dim3(1024), 0, st, count, units, G, piece_unit,
+                             piece_begin, piece_len, unit_first, unit_pieces, n_pieces);
   prof_end(st);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sa
