@@ -98,17 +98,6 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
   }
 }
 
-// Exchange point of the two element-wise warps that share a TMEM lane quarter (64 arrivals,
-// bounded wait).  Orders each side's tensor-memory reads before the other side's writes.
-__device__ __forceinline__ bool pair_sync(uint64_t* bar, int& exchanges, uint32_t* status) {
-  tc_fence_before();
-  mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, exchanges & 1, status);
-  ++exchanges;
-  tc_fence_after();
-  return ok;
-}
-
 // Split a packed pair x into bf16 hi + lo (x ~= hi + lo to about 2^-17 relative; lo = x - hi by
 // one packed fused multiply-add): the products that take P and dS run as two MMAs, hi then lo,
 // so those operands enter the tensor cores with ~16 significant bits.
@@ -486,8 +475,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // ------------------------------------------------------------------------------------------------
 // Q-major pass: dQ
 // TMEM columns: S0 [0,BN) | S1 [BN,2BN) | dP [2BN,3BN) | dQ [3BN, 3BN+128).
-// dS for tile j is written back as bf16 hi -> S_j[0,BN/2) and lo -> S_j[BN/2,BN), the A operands
-// of dQ += dS K.
+// dS for tile j is written back as packed bf16 over the S_j columns its warp has read: the warp of
+// key half h (columns [h*BN/2, +BN/2)) puts dS hi of its keys at [h*BN/2, +BN/4) and lo at
+// [h*BN/2 + BN/4, +BN/4); these are the A operands of dQ += dS K (one MMA per 16 keys, so the A
+// columns of each K step are addressed individually).
 // ------------------------------------------------------------------------------------------------
 constexpr int kQKStages = 3, kQVStages = 2;  // K is held by S and dQ, V only by dP
 
@@ -502,7 +493,6 @@ struct __align__(1024) QSmem {
   uint64_t bar_s_full[2], bar_dp_full, bar_ds_ready[2], bar_dq_done[2], bar_done;
   uint64_t bar_dp_free;  // the element-wise warps have loaded dP of the current tile (256 arrivals)
   uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
-  uint64_t bar_pair[4];
   uint32_t tmem_base;
 };
 
@@ -544,7 +534,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&s.bar_sched_full[i], 1);
       mbar_init(&s.bar_sched_empty[i], 2 + kVecWarps * 32);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&s.bar_pair[i], 64);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -657,12 +646,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc_fence_after();
             const uint32_t s_col = st ? kColS1 : kColS0;
             const uint64_t dkm = dkm0 + static_cast<uint64_t>(sk) * kKv16;
+            constexpr int kStepsPerHalf = BN / 32;  // 16-key K steps in a warp's key half
 #pragma unroll
-            for (int half = 0; half < 2; ++half)
+            for (int part = 0; part < 2; ++part)  // hi, then lo
 #pragma unroll
-              for (int ks = 0; ks < BN / 16; ++ks)
-                mma_bf16_ts(tmem + kColDQ, tmem + s_col + half * (BN / 2) + ks * 8, sdesc_add(dkm, ks * 2048),
-                            id_dq, (j > 0 || half > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < BN / 16; ++ks) {
+                const uint32_t a_col = s_col + (ks / kStepsPerHalf) * (BN / 2) + part * (BN / 4) +
+                                       (ks % kStepsPerHalf) * 8;
+                mma_bf16_ts(tmem + kColDQ, tmem + a_col, sdesc_add(dkm, ks * 2048), id_dq,
+                            (j > 0 || part > 0 || ks > 0) ? 1u : 0u);
+              }
             tc_commit(&s.bar_k_empty[sk]);
             tc_commit(&s.bar_dq_done[st]);
           }
@@ -708,7 +701,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int c0 = hf * kHalf;          // this thread's key columns [c0, c0 + BN/2)
     const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int exchanges = 0, J0 = 0, done_count = 0;
+    int J0 = 0, done_count = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int i = __shfl_sync(0xffffffffu, next_from_ring(k), 0);
@@ -774,14 +767,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&s.bar_dp_free);  // dP of tile J has been read: the next dP may overwrite it
-        // both halves have read S_J before either writes dS over it:
-        // hi -> S_J[c0/2, +BN/4), lo -> S_J[BN/2 + c0/2, +BN/4)
-        ok = __all_sync(0xffffffffu, pair_sync(&s.bar_pair[quarter], exchanges, prm.status));
-        if (!ok) break;
+        // dS over the S_J columns this warp has read: hi -> [c0, +BN/4), lo -> [c0 + BN/4, +BN/4)
 #pragma unroll
         for (int c = 0; c < kHalf / 2; c += 16) {
-          tmem_st16(tmem + lane_base + s_col + c0 / 2 + c, hv + c);
-          tmem_st16(tmem + lane_base + s_col + BN / 2 + c0 / 2 + c, lv + c);
+          tmem_st16(tmem + lane_base + s_col + c0 + c, hv + c);
+          tmem_st16(tmem + lane_base + s_col + c0 + BN / 4 + c, lv + c);
         }
         tmem_st_wait();
         tc_fence_before();
