@@ -117,20 +117,24 @@ __device__ __forceinline__ int batch_of_token(const int32_t* __restrict__ cu, in
 // ---------------------------------------------------------------------------------------------
 // token-major kernels: forward (kDq = false) and dQ (kDq = true)
 //
-// Each warp owns one (token, kv head, 16-head tile) item and a private ring of kTokStages chunk
+// Each warp owns one (token, kv head, 16-head tile) item and a private ring of tok_stages() chunk
 // stages.  Lane 0 copies a chunk's 16 K rows and 16 V rows with four TMA loads (the rows of one kv
 // head are 256 B apart in TND, one box of {64 dims, 1 head, 16 tokens} per head-dim half), into
 // 128-byte-swizzled [16 rows][64 dims] halves; all lanes wait on the stage's mbarrier.
 // ---------------------------------------------------------------------------------------------
-constexpr int kTokStages = 3;
-// warps per CTA: the forward fits 168 registers (9 warps); dQ holds dO fragments too (8 warps)
+// Warps per CTA and ring depth: the forward fits 168 registers, so 12 warps with 2-stage rings fill
+// the register file; dQ also holds dO fragments (222 registers: 8 warps) and keeps 3 stages.
 template <bool kDq>
-__host__ __device__ constexpr int tok_warps() { return kDq ? 8 : 9; }
+__host__ __device__ constexpr int tok_warps() { return kDq ? 8 : 12; }
+template <bool kDq>
+__host__ __device__ constexpr int tok_stages() { return kDq ? 3 : 2; }
 constexpr int kHalfBytes = kChunk * 128;        // [16 rows][64 dims]
 constexpr int kTileBytes = 2 * kHalfBytes;      // [16 rows][128 dims]
 constexpr int kTokStageBytes = 2 * kTileBytes;  // K and V tiles of one chunk
 template <bool kDq>
-__host__ __device__ constexpr int tok_smem() { return tok_warps<kDq>() * kTokStages * (kTokStageBytes + 8) + 1024; }
+__host__ __device__ constexpr int tok_smem() {
+  return tok_warps<kDq>() * tok_stages<kDq>() * (kTokStageBytes + 8) + 1024;
+}
 
 // byte address of (row, 16-byte column c16 of the 128 dims) in a chunk tile
 __device__ __forceinline__ uint32_t tok_swz(uint32_t tile, int row, int c16) {
@@ -168,6 +172,7 @@ __global__ void __launch_bounds__(tok_warps<kDq>() * 32)
   extern __shared__ uint8_t tsm_raw[];
   uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
   constexpr int kTokWarps = tok_warps<kDq>();
+  constexpr int kTokStages = tok_stages<kDq>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long item = static_cast<long long>(blockIdx.x) * kTokWarps + warp;  // (g, token, head tile)
   const long long items = static_cast<long long>(prm.N2) * prm.T * prm.head_tiles;
@@ -246,17 +251,23 @@ __global__ void __launch_bounds__(tok_warps<kDq>() * 32)
     }
     return c;
   };
-  int c = take(0), c1 = take(1);
-  int it = 0;
-  for (; c < n_chunks; ++it) {
-    const int c2 = take((it + 2) % kTokStages);  // the stage consumed in the previous iteration
+  // chunks in flight, oldest first: load k goes to stage k % kTokStages
+  int fifo[kTokStages - 1];
+#pragma unroll
+  for (int i = 0; i < kTokStages - 1; ++i) fifo[i] = take(i);
+  int loaded = 0, waited = 0;
+#pragma unroll
+  for (int i = 0; i < kTokStages - 1; ++i) loaded += fifo[i] < n_chunks ? 1 : 0;
+  for (int it = 0; fifo[0] < n_chunks; ++it) {
+    const int c = fifo[0];
+#pragma unroll
+    for (int i = 0; i + 1 < kTokStages - 1; ++i) fifo[i] = fifo[i + 1];
+    fifo[kTokStages - 2] = take((it + kTokStages - 1) % kTokStages);  // the stage consumed last iteration
+    loaded += fifo[kTokStages - 2] < n_chunks ? 1 : 0;
     const int stage = it % kTokStages;
-    if (!__all_sync(0xffffffffu, stage_wait(&wbar[stage], (it / kTokStages) & 1, prm.status))) {
-      c = c1;   // leave the loop; the copies still in flight are drained below
-      c1 = c2;
-      ++it;
-      break;
-    }
+    if (!__all_sync(0xffffffffu, stage_wait(&wbar[stage], (it / kTokStages) & 1, prm.status)))
+      break;  // the copies still in flight are drained below
+    ++waited;
     const int kp0 = first_key(c);
     const int valid = min(kChunk, len - kp0);
     const uint32_t kt = smem_u32(wst + stage * kTokStageBytes), vt = kt + kTileBytes;
@@ -358,14 +369,9 @@ __global__ void __launch_bounds__(tok_warps<kDq>() * 32)
       }
     }
     __syncwarp();  // every lane has read the stage before lane 0 refills it
-    c = c1;
-    c1 = c2;
   }
   // drain copies still in flight after an early exit (none after a complete pass)
-  for (int k = 0; k < 2; ++k) {
-    const int ck = k == 0 ? c : c1;
-    if (ck < n_chunks) stage_wait(&wbar[(it + k) % kTokStages], ((it + k) / kTokStages) & 1, prm.status);
-  }
+  for (int k = waited; k < loaded; ++k) stage_wait(&wbar[k % kTokStages], (k / kTokStages) & 1, prm.status);
   if (aborted(prm.status)) return;
   // epilogue
   if (!kDq) {
