@@ -125,9 +125,9 @@ __device__ __forceinline__ int batch_of_token(const int32_t* __restrict__ cu, in
 // Warps per CTA and ring depth: the forward fits 168 registers, so 12 warps with 2-stage rings fill
 // the register file; dQ also holds dO fragments (222 registers: 8 warps) and keeps 3 stages.
 template <bool kDq>
-__host__ __device__ constexpr int tok_warps() { return kDq ? 8 : 12; }
+__host__ __device__ constexpr int tok_warps() { return kDq ? 12 : 12; }
 template <bool kDq>
-__host__ __device__ constexpr int tok_stages() { return kDq ? 3 : 2; }
+__host__ __device__ constexpr int tok_stages() { return kDq ? 2 : 2; }
 constexpr int kHalfBytes = kChunk * 128;        // [16 rows][64 dims]
 constexpr int kTileBytes = 2 * kHalfBytes;      // [16 rows][128 dims]
 constexpr int kTokStageBytes = 2 * kTileBytes;  // K and V tiles of one chunk
