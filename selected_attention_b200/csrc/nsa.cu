@@ -271,23 +271,34 @@ __global__ void __launch_bounds__(tok_warps<kDq>() * 32)
     const int kp0 = first_key(c);
     const int valid = min(kChunk, len - kp0);
     const uint32_t kt = smem_u32(wst + stage * kTokStageBytes), vt = kt + kTileBytes;
-    // S = Q K^T (16 rows x 16 keys): two n8 tiles, each as two independent k-halves
+    // S = Q K^T (16 rows x 16 keys): two n8 tiles.  The forward runs each as two independent
+    // k-halves (shorter dependency chains); dQ, short of registers, as one chain.
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    if (!kDq) {
+      float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t bk[4], bk2[4];
-      ldsm_rows_k(bk, kt, ks, lane);
-      ldsm_rows_k(bk2, kt, ks + 4, lane);
-      mma16816(s[0], qa[ks], bk[0], bk[1]);
-      mma16816(s[1], qa[ks], bk[2], bk[3]);
-      mma16816(s2[0], qa[ks + 4], bk2[0], bk2[1]);
-      mma16816(s2[1], qa[ks + 4], bk2[2], bk2[3]);
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t bk[4], bk2[4];
+        ldsm_rows_k(bk, kt, ks, lane);
+        ldsm_rows_k(bk2, kt, ks + 4, lane);
+        mma16816(s[0], qa[ks], bk[0], bk[1]);
+        mma16816(s[1], qa[ks], bk[2], bk[3]);
+        mma16816(s2[0], qa[ks + 4], bk2[0], bk2[1]);
+        mma16816(s2[1], qa[ks + 4], bk2[2], bk2[3]);
+      }
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[n][i] += s2[n][i];
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t bk[4];
+        ldsm_rows_k(bk, kt, ks, lane);
+        mma16816(s[0], qa[ks], bk[0], bk[1]);
+        mma16816(s[1], qa[ks], bk[2], bk[3]);
+      }
     }
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) s[n][i] += s2[n][i];
     // mask: key position kp0 + column < len, and causal key <= query position
     const int lim = prm.mask_mode == 2 ? min(valid - 1, pos - kp0) : valid - 1;
 #pragma unroll
@@ -332,23 +343,19 @@ __global__ void __launch_bounds__(tok_warps<kDq>() * 32)
     } else {
       // P = 2^(s scale log2e - LSE log2e); dP = dO V^T; dS = P (dP - D)
       float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      float dp2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t bv[4], bv2[4];
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t bv[4];
         ldsm_rows_k(bv, vt, ks, lane);
-        ldsm_rows_k(bv2, vt, ks + 4, lane);
         mma16816(dp[0], da[ks], bv[0], bv[1]);
         mma16816(dp[1], da[ks], bv[2], bv[3]);
-        mma16816(dp2[0], da[ks + 4], bv2[0], bv2[1]);
-        mma16816(dp2[1], da[ks + 4], bv2[2], bv2[3]);
       }
 #pragma unroll
       for (int n = 0; n < 2; ++n)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float p = ex2(fmaf(s[n][i], prm.scale_log2, -l2r[i >> 1]));
-          s[n][i] = p * (dp[n][i] + dp2[n][i] - dr[i >> 1]);
+          s[n][i] = p * (dp[n][i] - dr[i >> 1]);
         }
       split2(s[0][0], s[0][1], pa_hi[0], pa_lo[0]);
       split2(s[0][2], s[0][3], pa_hi[1], pa_lo[1]);
