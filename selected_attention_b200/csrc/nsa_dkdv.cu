@@ -116,30 +116,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kEw) {
     // ------------------------------------------------------------------ TMA producer
+    // Lane j < tps loads the token of slot j and issues that slot's four row copies, so the token
+    // reads of a step are one round trip, not tps dependent ones.
     if (lane == 0) {
       mbar_arrive_expect_tx(&s.bar_kv, 4 * kKeys * 128);
       tma_load_3d(s.k[0], &tm_k, &s.bar_kv, 0, g, key_tok0);
       tma_load_3d(s.k[1], &tm_k, &s.bar_kv, 64, g, key_tok0);
       tma_load_3d(s.v[0], &tm_v, &s.bar_kv, 0, g, key_tok0);
       tma_load_3d(s.v[1], &tm_v, &s.bar_kv, 64, g, key_tok0);
-      int issued = 0;
-      for (int i = 0; i < steps; ++i) {
-        const int st = i & 1;
-        if (i >= 2 && !mbar_wait(&s.bar_qdo_empty[st], ((i - 2) >> 1) & 1, prm.status)) break;
-        mbar_arrive_expect_tx(&s.bar_qdo[st], 4 * kRows * 128);
-        for (int j = 0; j < tps; ++j) {
-          // slots past the list repeat its last token (finite data; their rows are masked)
-          const int idx = min(i * tps + j, n_tok - 1);
-          const int qrow = prm.t_col[rp + idx] * prm.N1 + g * prm.G;
-          const uint32_t off = static_cast<uint32_t>(j * prm.G * 128);
-          tma_load_2d(s.q[st][0] + off, &tm_q, &s.bar_qdo[st], 0, qrow);
-          tma_load_2d(s.q[st][1] + off, &tm_q, &s.bar_qdo[st], 64, qrow);
-          tma_load_2d(s.dout[st][0] + off, &tm_do, &s.bar_qdo[st], 0, qrow);
-          tma_load_2d(s.dout[st][1] + off, &tm_do, &s.bar_qdo[st], 64, qrow);
-        }
-        issued = i + 1;
+    }
+    int issued = 0;
+    for (int i = 0; i < steps; ++i) {
+      const int st = i & 1;
+      // slots past the list repeat its last token (finite data; their rows are masked)
+      const int qrow = lane < tps ? prm.t_col[rp + min(i * tps + lane, n_tok - 1)] * prm.N1 + g * prm.G : 0;
+      bool ok = true;
+      if (lane == 0) {
+        if (i >= 2) ok = mbar_wait(&s.bar_qdo_empty[st], ((i - 2) >> 1) & 1, prm.status);
+        if (ok) mbar_arrive_expect_tx(&s.bar_qdo[st], 4 * kRows * 128);
       }
-      // wait for this CTA's own copies still in flight before it may exit
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // the expected bytes are set before any copy
+      if (lane < tps) {
+        const uint32_t off = static_cast<uint32_t>(lane * prm.G * 128);
+        tma_load_2d(s.q[st][0] + off, &tm_q, &s.bar_qdo[st], 0, qrow);
+        tma_load_2d(s.q[st][1] + off, &tm_q, &s.bar_qdo[st], 64, qrow);
+        tma_load_2d(s.dout[st][0] + off, &tm_do, &s.bar_qdo[st], 0, qrow);
+        tma_load_2d(s.dout[st][1] + off, &tm_do, &s.bar_qdo[st], 64, qrow);
+      }
+      issued = i + 1;
+    }
+    // wait for this CTA's own copies still in flight before it may exit
+    if (lane == 0) {
       for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
         mbar_wait(&s.bar_qdo[i & 1], (i >> 1) & 1, prm.status);
       mbar_wait(&s.bar_kv, 0, prm.status);
