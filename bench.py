@@ -44,13 +44,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
 # kernel's source file is unchanged (sha1 prefix of the file recorded at capture time).
 NCU_TRAFFIC = {
-    # profiles/bsa_S8192_fwd_bwd.md (dram__bytes_read.sum + dram__bytes_write.sum, one launch)
-    "bsa_bwd_kv": {"bytes": 270780160 + 104547328, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                   "src_sha1": "c2bcda8c6f15"},
-    "bsa_bwd_q": {"bytes": 270909696 + 51656192, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                  "src_sha1": "c2bcda8c6f15"},
-    "bsa_fwd": {"bytes": 201515008 + 51768320, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+    # profiles/bsa_S8192_fwd_bwd.md and profiles/sfa_decode_B32.md
+    # (dram__bytes_read.sum + dram__bytes_write.sum of one launch; null once the source has changed)
+    "bsa_bwd_kv": {"bytes": 270705920 + 104391424, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                   "src_sha1": "53e9353b2603"},
+    "bsa_bwd_q": {"bytes": 270712832 + 52873728, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                  "src_sha1": "53e9353b2603"},
+    "bsa_fwd": {"bytes": 201467648 + 51852288, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
                 "src_sha1": "d34d6d9c1339"},
+    "sfa_decode": {"bytes": 147432192 + 3553536, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
+                   "src_sha1": "274bce18f713"},
 }
 
 
@@ -505,6 +508,8 @@ def run_decode(args, rank, world, local_rank):
     value = world * gathered / (ms * 1e-3) / 1e9  # every rank decodes its own copy of the batch
     dec_ms = prof["sfa_decode"][1] / prof["sfa_decode"][0] if "sfa_decode" in prof else None
     dec_gbs = gathered / (dec_ms * 1e-3) / 1e9 if dec_ms else None
+    tr = NCU_TRAFFIC["sfa_decode"]
+    dec_traffic = tr["bytes"] if tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config else None
     line = {
         "metric": "sparse decode gathered-KV bandwidth (paged, bf16)", "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -517,7 +522,7 @@ def run_decode(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": "sfa_decode", "achieved": dec_gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": dec_gbs / peaks["hbm_gbs"] if dec_gbs else None,
-                     "peak_source": f"{src} hbm_gbs (burst)", "traffic": None, "avg_launch_ms": dec_ms},
+                     "peak_source": f"{src} hbm_gbs (burst)", "traffic": dec_traffic, "avg_launch_ms": dec_ms},
         "kernels": {n: {"launches": c, "ms_per_call": t / c} for n, (c, t) in prof.items()},
         "clocks": clocks.summary(), "gathered_bytes_per_step": gathered,
     }
