@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
 # kernel's source file is unchanged (sha1 prefix of the file recorded at capture time).
 NCU_TRAFFIC = {
-    # profiles/bsa_S8192_fwd_bwd.md and profiles/sfa_decode_B32.md
+    # profiles/bsa_S8192_fwd_bwd.md, profiles/sfa_decode_B32.md, profiles/nsa_token_kernels_T16384.md
     # (dram__bytes_read.sum + dram__bytes_write.sum of one launch; null once the source has changed)
     "bsa_bwd_kv": {"bytes": 270705920 + 104391424, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
                    "src_sha1": "53e9353b2603"},
@@ -54,6 +54,9 @@ NCU_TRAFFIC = {
                 "src_sha1": "d34d6d9c1339"},
     "sfa_decode": {"bytes": 147432192 + 3553536, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
                    "src_sha1": "274bce18f713"},
+    # profiles/nsa_token_kernels_T16384.md (full-size launch, T = 61440)
+    "nsa_bwd_dq": {"bytes": 2239617536 + 985623296, "config": 3, "src": "selected_attention_b200/csrc/nsa.cu",
+                   "src_sha1": "ea904e4aa7c6"},
 }
 
 
