@@ -6,7 +6,7 @@ import this module.  It shares no code with the CUDA path and must never serve a
 Everything is computed in float64 on the bf16 inputs widened exactly.  The arithmetic is the
 plain definition, with no blocking, online rescaling or reordering:
 
-  * Forward (BlockSparseAttentionGrad page, "known forward computation formula"; the
+  * Forward (BlockSparseAttentionGrad page, section stating the forward formula; the
     NsaSelectedAttention page's forward formula is the same after its Gather step):
         S = Mask(scale * Q K_sel^T, atten_mask);  P = softmax(S);  Out = P V_sel
     The softmax is the two-pass form m = max S, l = sum exp(S - m), P = exp(S - m) / l.

@@ -34,6 +34,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
                                 const float* __restrict__ lse, int S_q, int bx, int nqb, long long n_rows,
                                 float* __restrict__ dvec, float* __restrict__ lse2) {
+  griddep_wait();  // launched with programmatic dependent launch: the lists before it must be complete
+  griddep_launch_dependents();
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long row = gid >> 3;  // 8 threads per row, 16 elements each
   const int part = static_cast<int>(gid & 7);
@@ -76,6 +78,8 @@ struct BwdParams {
   int B, N1, N2, S_q, S_kv, bx, by, nqb, nkb, mask_mode, win_left, win_right;
   float scale, scale_log2;
   int32_t* next_unit;      // persistent-kernel work counter, zero at launch
+  int pdl_wait;            // wait for the previous grid (0: the dQ pass right after the KV pass,
+                           // which it does not read: it may fill the KV pass's tail)
   const int32_t* row_ptr;  // KV lists (Q-major pass) or transposed lists (KV-major pass)
   const int32_t* col;
   const float* dvec;       // [B*N1*nqb*128]: -softmax_grad per padded query row
@@ -156,6 +160,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
                       const BwdParams prm) {
+  griddep_wait();  // the D / LSE tiles of the preprocess must be complete
+  griddep_launch_dependents();  // after the wait: the dQ pass then starts only once its inputs exist
   constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   KvSmem& s = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -505,6 +511,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     bsa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const BwdParams prm) {
+  if (prm.pdl_wait) griddep_wait();
+  griddep_launch_dependents();
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColDP = 2 * BN, kColDQ = 3 * BN;
   extern __shared__ uint8_t smem_raw[];
   QSmem<BN>& s = *reinterpret_cast<QSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -817,9 +825,9 @@ cudaError_t launch_q(const BwdParams& p, const CUtensorMap& tq, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(bsa_bwd_q_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   prof_begin("bsa_bwd_q", st);
-  if (grid > 0) bsa_bwd_q_kernel<BN><<<grid, kKvThreads, smem, st>>>(tq, tk, tv, tdo, p);
+  if (grid > 0) e = launch_pdl(bsa_bwd_q_kernel<BN>, dim3(grid), dim3(kKvThreads), smem, st, tq, tk, tv, tdo, p);
   prof_end(st);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -831,11 +839,11 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     const long long threads = n_rows * 8;
     const int blk = 256;
     prof_begin("bsa_bwd_prep", st);
-    bwd_prep_kernel<<<static_cast<unsigned>((threads + blk - 1) / blk), blk, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, a.S_q, a.bx, a.nqb,
-        n_rows, a.dvec, a.lse2);
+    cudaError_t e = launch_pdl(bwd_prep_kernel, dim3(static_cast<unsigned>((threads + blk - 1) / blk)), dim3(blk), 0,
+                               st, static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout),
+                               lse, a.S_q, a.bx, a.nqb, n_rows, a.dvec, a.lse2);
     prof_end(st);
-    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   CUtensorMap tq, tk, tv, tdo, tk128, tv128, tq64, tdo64;
@@ -848,6 +856,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
       !make_tmap_2d_bf16(&tdo64, dout, q_rows, kD, kD, kHalfRows))
     return cudaErrorInvalidValue;
   BwdParams p;
+  bool kv_launched = false;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.S_q = a.S_q; p.S_kv = a.S_kv; p.bx = a.bx; p.by = a.by;
   p.nqb = a.nqb; p.nkb = a.nkb; p.mask_mode = a.mask_mode; p.win_left = a.win_left; p.win_right = a.win_right;
   p.scale = a.scale; p.scale_log2 = a.scale * kLog2e;
@@ -871,14 +880,20 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = units < sms ? units : sms;  // persistent: one CTA per SM
     prof_begin("bsa_bwd_kv", st);
-    if (grid > 0) bsa_bwd_kv_kernel<<<grid, kKvThreads, smem, st>>>(tq64, tk128, tv128, tdo64, pk);
+    pk.pdl_wait = 1;
+    if (grid > 0) e = launch_pdl(bsa_bwd_kv_kernel, dim3(grid), dim3(kKvThreads), smem, st, tq64, tk128, tv128, tdo64, pk);
     prof_end(st);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
+    kv_launched = grid > 0;
   }
   // Q-major pass (persistent)
   p.row_ptr = a.row_ptr;
   p.col = a.col;
   p.next_unit = a.next_q;
+  // The dQ pass reads the preprocess and the KV lists, not the KV pass: launched right after a KV
+  // pass (which signals dependents only after its own wait on the preprocess), it need not wait
+  // and its CTAs take the SMs the KV pass leaves; otherwise it waits for the preprocess.
+  p.pdl_wait = kv_launched ? 0 : 1;
   const int q_units = a.B * a.N1 * a.nqb;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -110,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams prm) {
+  griddep_wait();  // launched with programmatic dependent launch: the KV lists must be complete
+  griddep_launch_dependents();
   constexpr uint32_t kTmemCols = (2 * BN + kD) <= 256 ? 256 : 512;
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
   constexpr int kHalf = BN / 2;  // S columns per softmax thread
@@ -423,6 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stops at the q block and at the head's end.  The previous unit's store must have read
       // the staging tile first.
       if (k > 0) {
+        if (warp == 0 && lane == 0) {  // the thread that issued the previous unit's stores
+          bulk_wait_read_all();
+          mbar_arrive(&s.bar_stage_free);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_stage_free, (k - 1) & 1, prm.status));
         if (!ok) break;
       }
@@ -455,9 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           tma_store_3d(&tm_o, s.ostage[0], 0, qb * prm.bx, u.bh);
           tma_store_3d(&tm_o, s.ostage[1], 64, qb * prm.bx, u.bh);
-          bulk_commit();
-          bulk_wait_read_all();
-          mbar_arrive(&s.bar_stage_free);
+          bulk_commit();  // read completion is awaited at the next unit's epilogue, off the critical path
         }
       }
       ok = __all_sync(0xffffffffu, ok);
@@ -502,9 +506,9 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.units < sms ? p.units : sms;  // persistent: one CTA per SM
   prof_begin("bsa_fwd", st);
-  bsa_fwd_kernel<BN><<<grid, kThreads, smem, st>>>(tq, tk, tv, to, p);
+  e = launch_pdl(bsa_fwd_kernel<BN>, dim3(grid), dim3(kThreads), smem, st, tq, tk, tv, to, p);
   prof_end(st);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

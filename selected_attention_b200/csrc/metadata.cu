@@ -3,14 +3,15 @@
 // SparseAttnSharedkvMetadata page (function description): an operator run ahead of the
 // attention call that lays out each core's share of the work.  Here the products are CSR lists:
 //   * BSA: for unit (b, h, qb), the KV blocks its BlockSparseMask row selects, ascending
-//     (BlockSparseAttentionGrad page: "BlockSparseMask specifies the KV block selected by each
-//     Q block").
+//     (BlockSparseAttentionGrad page, parameter description of the mask: one row of selected KV
+//     blocks per Q block).
 //   * BSA transposed: for (b, g, kb), ascending h_local * nqb + qb over the group's query heads
 //     that selected kb; the dK/dV pass (dV = P^T dOut, dK = dS^T Q scale) walks these.
 // All products are integers and deterministic (no atomics decide an order).
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "sa_common.cuh"
 
 namespace sa {
 namespace {
@@ -20,6 +21,8 @@ constexpr int kWarps = 8;
 // One warp per row: count nonzero bytes.
 __global__ void count_rows_kernel(const uint8_t* __restrict__ rows, int n_rows, int row_len,
                                   int32_t* __restrict__ counts) {
+  griddep_wait();  // launched with programmatic dependent launch: the predecessor must be complete
+  griddep_launch_dependents();
   const int warp = blockIdx.x * kWarps + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (warp >= n_rows) return;
@@ -34,6 +37,8 @@ __global__ void count_rows_kernel(const uint8_t* __restrict__ rows, int n_rows, 
 // One warp per row: write the indices of nonzero bytes, ascending, at col[row_ptr[row]...].
 __global__ void fill_rows_kernel(const uint8_t* __restrict__ rows, int n_rows, int row_len,
                                  const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int warp = blockIdx.x * kWarps + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (warp >= n_rows) return;
@@ -54,6 +59,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
                                                     int32_t* __restrict__ row_ptr) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
+  griddep_wait();
+  griddep_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   if (tid == 0) carry = 0;
   __syncthreads();
@@ -92,6 +99,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 __global__ void transpose_mask_kernel(const uint8_t* __restrict__ mask, int N1, int N2, int nqb, int nkb,
                                       uint8_t* __restrict__ maskT) {
   __shared__ uint8_t tile[32][33];
+  griddep_wait();
+  griddep_launch_dependents();
   const int bh = blockIdx.z;  // b * N1 + h
   const int b = bh / N1, h = bh % N1;
   const int G = N1 / N2, g = h / G, hl = h % G;
@@ -117,9 +126,9 @@ inline int div_up(int a, int b) { return (a + b - 1) / b; }
 
 cudaError_t exclusive_scan(const int32_t* counts, int n, int32_t* row_ptr, cudaStream_t st) {
   prof_begin("meta_scan", st);
-  scan_kernel<<<1, 1024, 0, st>>>(counts, n, row_ptr);
+  cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, counts, n, row_ptr);
   prof_end(st);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t bsa_kv_lists(const uint8_t* mask, int units, int nkb, int32_t* counts, int32_t* row_ptr, int32_t* col,
@@ -127,15 +136,16 @@ cudaError_t bsa_kv_lists(const uint8_t* mask, int units, int nkb, int32_t* count
   if (units <= 0) return cudaSuccess;
   const int grid = div_up(units, kWarps);
   prof_begin("meta_count", st);
-  count_rows_kernel<<<grid, kWarps * 32, 0, st>>>(mask, units, nkb, counts);
+  cudaError_t e = launch_pdl(count_rows_kernel, dim3(grid), dim3(kWarps * 32), 0, st, mask, units, nkb, counts);
   prof_end(st);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if ((e = exclusive_scan(counts, units, row_ptr, st)) != cudaSuccess) return e;
   prof_begin("meta_fill", st);
-  fill_rows_kernel<<<grid, kWarps * 32, 0, st>>>(mask, units, nkb, row_ptr, col);
+  e = launch_pdl(fill_rows_kernel, dim3(grid), dim3(kWarps * 32), 0, st, mask, units, nkb,
+                 static_cast<const int32_t*>(row_ptr), col);
   prof_end(st);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t bsa_q_lists(const uint8_t* mask, int B, int N1, int N2, int nqb, int nkb, uint8_t* maskT,
@@ -143,9 +153,9 @@ cudaError_t bsa_q_lists(const uint8_t* mask, int B, int N1, int N2, int nqb, int
   const int G = N1 / N2;
   dim3 grid(div_up(nkb, 32), div_up(nqb, 32), B * N1);
   prof_begin("meta_transpose", st);
-  transpose_mask_kernel<<<grid, dim3(32, 8), 0, st>>>(mask, N1, N2, nqb, nkb, maskT);
+  cudaError_t e = launch_pdl(transpose_mask_kernel, grid, dim3(32, 8), 0, st, mask, N1, N2, nqb, nkb, maskT);
   prof_end(st);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return bsa_kv_lists(maskT, B * N2 * nkb, G * nqb, counts, row_ptr, col, st);
 }
