@@ -46,12 +46,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # profiles/bsa_S8192_fwd_bwd.md, profiles/sfa_decode_B32.md, profiles/nsa_token_kernels_T16384.md
     # (dram__bytes_read.sum + dram__bytes_write.sum of one launch; null once the source has changed)
-    "bsa_bwd_kv": {"bytes": 270705920 + 104391424, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                   "src_sha1": "53e9353b2603"},
-    "bsa_bwd_q": {"bytes": 270712832 + 52873728, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                  "src_sha1": "53e9353b2603"},
-    "bsa_fwd": {"bytes": 201467648 + 51852288, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
-                "src_sha1": "d34d6d9c1339"},
+    "bsa_bwd_kv": {"bytes": 270692864 + 105957888, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                   "src_sha1": "1b48ca31dc53"},
+    "bsa_bwd_q": {"bytes": 270671872 + 53610752, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                  "src_sha1": "1b48ca31dc53"},
+    "bsa_fwd": {"bytes": 201541888 + 51276544, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+                "src_sha1": "90fa1eb3e002"},
     "sfa_decode": {"bytes": 147432192 + 3553536, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
                    "src_sha1": "274bce18f713"},
     # profiles/nsa_token_kernels_T16384.md (full-size launch, T = 61440)
