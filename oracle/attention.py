@@ -63,7 +63,7 @@ def stored_out(o: np.ndarray, out_storage) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------------------
-# mask rule (BlockSparseAttentionGrad formula "Mask(., atten_mask)"; NsaSelectedAttention
+# mask rule (BlockSparseAttentionGrad forward formula, its Mask(., atten_mask) step; NsaSelectedAttention
 # sparseMode 0 / 2; SparseAttnSharedkvMetadata mask modes 3 and 4 with ori_win_left/right)
 # ----------------------------------------------------------------------------------------------
 def visible(pos_q: np.ndarray, pos_k: np.ndarray, mode: int, s_q: int, s_kv: int,

@@ -14,8 +14,8 @@ namespace {
 inline int div_up(int a, int b) { return (a + b - 1) / b; }
 
 // ---- BSA (BlockSparseAttentionGrad page constraints) -------------------------------------------
-// "N1 must be greater than or equal to N2, and N1 % N2 must be equal to 0"; "headdim=128";
-// layouts BNSD.  Block shape: block_x <= 128 (one 128-row MMA tile per Q block), block_y 64 or 128.
+// N1 at least N2 and a multiple of it (the GQA rule), head dim 128; layouts BNSD.  Block shape:
+// block_x <= 128 (one 128-row MMA tile per Q block), block_y 64 or 128.
 bsa_status check_bsa(const bsa_params* p) {
   if (!p) return BSA_ERR_NULLPTR;
   if (p->q_layout != BSA_LAYOUT_BNSD || p->kv_layout != BSA_LAYOUT_BNSD) return BSA_ERR_UNSUPPORTED;
@@ -80,9 +80,9 @@ size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
 }
 
 // ---- SFA (SparseFlashAttention page constraints) ----------------------------------------------------
-// "D in query, key and value is 512; Dr of query_rope and key_rope is 64"; "block_size must be a
-// multiple of 16, at most 1024" (this library's 32-token tiles need a multiple of 32);
-// "sparse_block_size must be exactly divisible by block_size"; decode: one query row per batch.
+// query / key / value dims 512 with a 64-dim rope part; the page size a multiple of 16 up to 1024
+// (this library's 32-token tiles need a multiple of 32);
+// the sparse block size must be a whole number of pages; decode: one query row per batch.
 bsa_status check_sfa(const bsa_params* p) {
   if (!p) return BSA_ERR_NULLPTR;
   if (p->kv_layout != BSA_LAYOUT_PA_ND) return BSA_ERR_UNSUPPORTED;

@@ -74,8 +74,9 @@ __global__ void sfa_page_list_kernel(const int32_t* __restrict__ sparse_indices,
 
 // One CTA: choose the piece size and lay out the pieces.
 //   units u = (b * N2 + g) * 2 + dv_half; n_u = count[b, g]
-//   chunk = the smallest c >= 1 with sum_u ceil(n_u / c) <= G (binary search; c = max n_u always
-//   qualifies when units <= G, and the host never launches more units than that)
+//   chunk = the smallest c >= 1 with sum_u ceil(n_u / c) <= G (binary search; with more units
+//   than G it ends at c = max n_u, one piece per unit, and the piece arrays, sized G + units,
+//   still hold them)
 //   piece records: unit, first page, page count; unit_first[u], unit_pieces[u]
 __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __restrict__ count, int units, int G,
                                                              int32_t* __restrict__ piece_unit,
