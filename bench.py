@@ -39,6 +39,8 @@ sys.path.insert(0, ROOT)
 from workloads import synth  # noqa: E402
 
 METRIC = "effective block-sparse attn fwd+bwd TFLOP/s (bf16)"
+METRIC_NSA = "effective NSA selected attn fwd+bwd TFLOP/s (bf16)"
+METRIC_DEC = "sparse decode gathered-KV bandwidth (paged, bf16)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
@@ -160,27 +162,57 @@ def bsa_workload(config: int):
     return w
 
 
-def cpu_oracle_sample(w, mask, budget_s: float):
-    """Time the fp64 oracle (forward + backward) on whole (b, h) head slices until budget_s has
-    passed; returns (credited FLOPs done, seconds, description)."""
+def cpu_oracle_sample(w, mask, budget_s: float, chunk: int = 64):
+    """Time the fp64 oracle (forward + backward) on runs of about `chunk` Q blocks spread over each
+    (b, h) head slice in turn (every unit's full contribution: its dQ rows and its share of dK /
+    dV), until budget_s of oracle time has passed; returns (credited FLOPs, seconds, description)."""
     from oracle import attention as A
-    flops, heads, t0 = 0, [], time.perf_counter()
+    flops, dt, units, t_wall = 0, 0.0, 0, time.perf_counter()
+    nqb = mask.shape[2]
     for b in range(w.B):
         for h in range(w.N1):
             q = A.bf16_to_f64(w.tensor("q", b, h))[None]
             k = A.bf16_to_f64(w.tensor("k", b, h))
             v = A.bf16_to_f64(w.tensor("v", b, h))
             do = A.bf16_to_f64(w.tensor("dout", b, h))[None]
-            A.bsa_slice_backward(q, k, v, do, mask[b, h][None], w.block, w.block, w.mask_mode, w.scale,
-                                 out_storage="bf16")
-            vp = visible_pairs_bsa(mask[b, h][None, None], w.block, w.block, w.S, w.S)
-            flops += 14 * w.D * vp
-            heads.append((b, h))
-            if time.perf_counter() - t0 >= budget_s:
-                dt = time.perf_counter() - t0
-                return flops, dt, f"oracle fwd+bwd on {len(heads)} of {w.B * w.N1} (b,h) head slices {heads}"
-    dt = time.perf_counter() - t0
-    return flops, dt, f"oracle fwd+bwd on all {len(heads)} (b,h) head slices"
+            n_runs = -(-nqb // chunk)
+            for r0 in range(n_runs):  # run r0 takes q blocks r0, r0 + n_runs, ...: spread over the head
+                qbs = list(range(r0, nqb, n_runs))
+                t0 = time.perf_counter()
+                A.bsa_slice_backward(q, k, v, do, mask[b, h][None], w.block, w.block, w.mask_mode, w.scale,
+                                     q_blocks=qbs, out_storage="bf16")
+                dt += time.perf_counter() - t0
+                sub = np.zeros_like(mask[b, h])
+                sub[qbs] = mask[b, h][qbs]
+                flops += 14 * w.D * visible_pairs_bsa(sub[None, None], w.block, w.block, w.S, w.S)
+                units += len(qbs)
+                if dt >= budget_s or time.perf_counter() - t_wall >= 4 * budget_s:
+                    return flops, dt, (f"oracle fwd+bwd on {units} of {w.B * w.N1 * nqb} (b, h, q block) units "
+                                       f"(head slices in order, {chunk} q blocks spread over the head at a time)")
+    return flops, dt, f"oracle fwd+bwd on all {units} (b, h, q block) units"
+
+
+def cpu_oracle_sample_decode(w, budget_s: float):
+    """Time the fp64 oracle decode one batch at a time until budget_s of oracle time has passed;
+    returns (gathered bytes done, seconds, description)."""
+    from oracle import attention as A
+    table, idx = w.selection()
+    seqused = np.full(w.B, w.context, np.int32)
+    q, qr = w.query("q"), w.query("q_rope")
+    per_batch = w.count * w.sparse_block * (w.D + w.Dr + w.D) * 2
+    done, dt = [], 0.0
+    for b in range(w.B):
+        pages = [int(pg) for pg in table[b, idx[b, 0, 0]]]
+        kc = {pg: w.pages("k", [pg])[0] for pg in pages}
+        krc = {pg: w.pages("k_rope", [pg])[0] for pg in pages}
+        vc = {pg: w.pages("v", [pg])[0] for pg in pages}
+        t0 = time.perf_counter()
+        A.sfa_decode(q, qr, kc, krc, vc, table, idx, seqused, w.page, w.sparse_block, w.scale, batches=[b])
+        dt += time.perf_counter() - t0
+        done.append(b)
+        if dt >= budget_s:
+            break
+    return len(done) * per_batch, dt, f"oracle decode of {len(done)} of {w.B} batches"
 
 
 def visible_pairs_nsa(w, topk: np.ndarray) -> int:
@@ -258,29 +290,42 @@ def run_reference(args, rank, world):
         pass  # the oracle has no warm-up state; warm-up steps are a no-op
     total_f, total_t, desc = 0, 0.0, ""
     step_budget = min(args.ref_step_seconds, 150.0 / max(1, args.steps))  # whole run ~2.5 min at most
+    metric, unit, scale = METRIC, "TFLOP/s", 1e12
     if isinstance(w, synth.NsaWorkload):
         topk = w.topk()
         sample = lambda: cpu_oracle_sample_nsa(w, topk, budget_s=step_budget)  # noqa: E731
         cfg = config_dict_nsa(w, args)
-    else:
+        metric = METRIC_NSA
+    elif isinstance(w, synth.BsaWorkload):
         mask = w.block_mask()
         sample = lambda: cpu_oracle_sample(w, mask, budget_s=step_budget)  # noqa: E731
         cfg = config_dict(w, args)
+    else:  # paged sparse decode: gathered bytes per second
+        sample = lambda: cpu_oracle_sample_decode(w, budget_s=step_budget)  # noqa: E731
+        cfg = config_dict_decode(w)
+        metric, unit, scale = METRIC_DEC, "GB/s", 1e9
     for _ in range(args.steps):
         f, t, desc = sample()
         total_f += f
         total_t += t
-    value = total_f / total_t / 1e12
+    value = total_f / total_t / scale
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": cfg,
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"each step: {desc}"},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+
+
+def config_dict_decode(w):
+    return {"workload": f"{w.name}: B={w.B}, N1={w.N1}, N2={w.N2}, D={w.D}+{w.Dr}, {w.context}-token "
+                        f"cache, page {w.page}, {w.count} sparse blocks of {w.sparse_block} per query",
+            "l2": "flushed (256 MiB write) before every timed rep",
+            "timing": "mean over the timed reps, each one CUDA-graph replay timed with events"}
 
 
 def config_dict(w, args):
@@ -432,7 +477,7 @@ def run_nsa(args, rank, world, local_rank):
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps({
-            "metric": "effective NSA selected attn fwd+bwd TFLOP/s (bf16)", "value": value, "unit": "TFLOP/s",
+            "metric": METRIC_NSA, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config_dict_nsa(w, args),
@@ -499,7 +544,7 @@ def run_decode(args, rank, world, local_rank):
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
         barrier()
-    ms = max_over_ranks(float(np.median(times)))
+    ms = max_over_ranks(float(np.mean(times)))
     assert sa.bsa_get_status(ws) == 0
     sa.bsa_profile_enable(True)
     for _ in range(3):
@@ -507,6 +552,43 @@ def run_decode(args, rank, world, local_rank):
         call()
     prof = sa.bsa_profile_collect()
     sa.bsa_profile_enable(False)
+    launches_per_call = sum(c for c, _ in prof.values()) // 3
+
+    # end to end through the API: each step copies the step's inputs (the query and its rope part,
+    # the block table, the sparse indices, seqused) from pinned host memory and reads Out and LSE
+    # back; the paged cache is resident device state, as in a serving loop
+    h_in = {n_: x.cpu().pin_memory() for n_, x in (("q", q), ("qr", qr), ("tb", tb), ("ti", ti), ("tu", tu))}
+    d_in = {n_: torch.empty_like(x) for n_, x in (("q", q), ("qr", qr), ("tb", tb), ("ti", ti), ("tu", tu))}
+    h_out, h_lse = torch.empty(out.shape, dtype=out.dtype).pin_memory(), torch.empty(lse.shape).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in h_in.values())
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+
+    def e2e_step():
+        for n_ in d_in:
+            d_in[n_].copy_(h_in[n_], non_blocking=True)
+        sa.sfa_sparse_decode(d_in["q"], d_in["qr"], caches["k"], caches["k_rope"], caches["v"], d_in["tb"],
+                             d_in["ti"], d_in["tu"], w.sparse_block, w.scale, out=out, lse=lse, workspace=ws)
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_times = []
+    barrier()
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_times.append(e0.elapsed_time(e1))
+    barrier()
+    e2e_ms = max_over_ranks(float(np.mean(e2e_times)))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f_, t_, desc = cpu_oracle_sample_decode(w, budget_s=args.cpu_seconds)
+        cpu = {"value": f_ / t_ / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
     peaks, src = measured_peaks()
     value = world * gathered / (ms * 1e-3) / 1e9  # every rank decodes its own copy of the batch
     dec_ms = prof["sfa_decode"][1] / prof["sfa_decode"][0] if "sfa_decode" in prof else None
@@ -514,12 +596,13 @@ def run_decode(args, rank, world, local_rank):
     tr = NCU_TRAFFIC["sfa_decode"]
     dec_traffic = tr["bytes"] if tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config else None
     line = {
-        "metric": "sparse decode gathered-KV bandwidth (paged, bf16)", "value": value, "unit": "GB/s",
+        "metric": METRIC_DEC, "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B}, N1={w.N1}, N2={w.N2}, D={w.D}+{w.Dr}, {w.context}-token "
-                               f"cache, page {w.page}, {w.count} sparse blocks of {w.sparse_block} per query",
-                   "l2": "flushed (256 MiB write) before every timed rep", "timing": "median of CUDA-graph replays"},
+        "config": config_dict_decode(w),
+        "e2e": {"value": world * gathered / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_call * args.steps,
         "effective_tflops": world * flops / (ms * 1e-3) / 1e12,
         # dominant kernel: the decode kernel alone, its gathered bytes over its mean launch time
         "roofline": {"bound": "hbm", "kernel": "sfa_decode", "achieved": dec_gbs,
@@ -527,7 +610,7 @@ def run_decode(args, rank, world, local_rank):
                      "frac": dec_gbs / peaks["hbm_gbs"] if dec_gbs else None,
                      "peak_source": f"{src} hbm_gbs (burst)", "traffic": dec_traffic, "avg_launch_ms": dec_ms},
         "kernels": {n: {"launches": c, "ms_per_call": t / c} for n, (c, t) in prof.items()},
-        "clocks": clocks.summary(), "gathered_bytes_per_step": gathered,
+        "cpu_baseline": cpu, "clocks": clocks.summary(), "gathered_bytes_per_step": gathered,
     }
     if rank == 0:
         print(json.dumps(line))
@@ -677,9 +760,6 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        if args.config == 4:
-            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the BSA workloads"}))
-            return
         run_reference(args, rank, world)
         return
     if world > 1:
