@@ -226,11 +226,19 @@ BSA_API const char* bsa_version(void);
 BSA_API bsa_status bsa_diag_mma_tile(const void* a, const void* b, float* c, int32_t b_mn_major, void* workspace,
                              void* stream);
 
-/* Diagnostic: y[i] = 2^x[i] (device arrays of n floats) by the polynomial the softmax loops use
- * on the FMA pipe for part of their exponentials (Cody-Waite reduction to [-1/2, 1/2], fitted
- * polynomial of degree 3 or 4, exponent add).  x must lie in [-126, 128).  Not part of the pages'
+/* Diagnostic: y[i] = 2^x[i] (device arrays of n floats) by an exp2 on the FMA pipe (Cody-Waite
+ * reduction to [-1/2, 1/2], fitted polynomial of degree 3 or 4, exponent add); the attention
+ * kernels use the special-function unit's exp2.  x must lie in [-126, 128).  Not part of the pages'
  * operations.  Returns BSA_ERR_INVALID_ARG for another degree or n < 0. */
 BSA_API bsa_status bsa_diag_exp2(const float* x, float* y, int32_t n, int32_t degree, void* stream);
+
+/* Diagnostic for failure detection: one warp waits on a device barrier with the bounded wait every
+ * kernel uses.  arrive = 1: the barrier is satisfied first and the status word stays 0.  arrive = 0:
+ * nothing arrives; after the wait limit (about one second) the kernel sets SA_DEV_TIMEOUT in the
+ * status word at the start of `workspace` (>= 4 bytes, device) and returns normally, so the CUDA
+ * context stays usable; read the bits with bsa_get_status.  Other values of arrive return
+ * BSA_ERR_INVALID_ARG.  Not part of the pages' operations. */
+BSA_API bsa_status bsa_diag_wait(void* workspace, int32_t arrive, void* stream);
 
 #ifdef __cplusplus
 }

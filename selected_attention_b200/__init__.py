@@ -29,7 +29,7 @@ EXPORTED = [
     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size", "bsa_fwd", "bsa_bwd",
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
-    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_diag_exp2",
+    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_diag_exp2", "bsa_diag_wait",
 ]
 
 
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
         L.bsa_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.bsa_diag_mma_tile.argtypes = [vp, vp, vp, ctypes.c_int32, vp, vp]
         L.bsa_diag_exp2.argtypes = [vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
+        L.bsa_diag_wait.argtypes = [vp, ctypes.c_int32, vp]
         L.bsa_profile_enable.argtypes = [ctypes.c_int32]
         L.bsa_profile_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
         L.bsa_version.restype = ctypes.c_char_p
@@ -384,6 +385,14 @@ def bsa_diag_mma_tile(a, b, mode, stream=None):
     _check("bsa_diag_mma_tile", lib().bsa_diag_mma_tile(_ptr(a), _ptr(b), _ptr(c), int(mode), _ptr(ws),
                                                         _stream(stream)))
     return c, ws
+
+
+def bsa_diag_wait(arrive: bool, device="cuda", stream=None) -> int:
+    """Run the bounded-wait diagnostic and return the device status bits (SA_DEV_TIMEOUT = 4 when
+    nothing arrived)."""
+    ws = _workspace(256, torch.device(device))
+    _check("bsa_diag_wait", lib().bsa_diag_wait(_ptr(ws), 1 if arrive else 0, _stream(stream)))
+    return bsa_get_status(ws, stream)
 
 
 def bsa_diag_exp2(x, degree, stream=None):

@@ -530,6 +530,14 @@ bsa_status bsa_diag_mma_tile(const void* a, const void* b, float* c, int32_t b_m
   return cuda_status(diag_mma_tile_launch(a, b, c, 128, b_mn_major, static_cast<uint32_t*>(workspace), st));
 }
 
+bsa_status bsa_diag_wait(void* workspace, int32_t arrive, void* stream) {
+  if (!workspace) return BSA_ERR_NULLPTR;
+  if (arrive != 0 && arrive != 1) return BSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+  return cuda_status(diag_wait_launch(static_cast<uint32_t*>(workspace), arrive, st));
+}
+
 bsa_status bsa_diag_exp2(const float* x, float* y, int32_t n, int32_t degree, void* stream) {
   if (!x || !y) return BSA_ERR_NULLPTR;
   if (n < 0 || (degree != 3 && degree != 4)) return BSA_ERR_INVALID_ARG;

@@ -107,6 +107,22 @@ __global__ void __launch_bounds__(128) diag_mma_kernel(const __grid_constant__ C
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// Failure detection: one warp waits on an mbarrier of one arrival with the kernels' bounded wait.
+// With `arrive` lane 0 arrives first and the wait succeeds; without it nothing ever arrives, the
+// wait gives up after kWaitLimitNs and sets SA_DEV_TIMEOUT, and the kernel returns normally, so the
+// context stays usable (no trap, no fault).
+__global__ void diag_wait_kernel(uint32_t* status, int arrive) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (arrive && threadIdx.x == 0) mbar_arrive(&bar);
+  __syncwarp();
+  mbar_wait(&bar, 0, status);
+}
+
 __global__ void diag_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int degree) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (i >= n) return;
@@ -139,6 +155,11 @@ cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, 
   prof_begin("diag_mma", st);
   diag_mma_kernel<<<1, 128, smem, st>>>(ta, tb, c, b_mn_major, status, a);
   prof_end(st);
+  return cudaGetLastError();
+}
+
+cudaError_t diag_wait_launch(uint32_t* status, int arrive, cudaStream_t st) {
+  diag_wait_kernel<<<1, 32, 0, st>>>(status, arrive);
   return cudaGetLastError();
 }
 

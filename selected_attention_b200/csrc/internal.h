@@ -156,5 +156,6 @@ cudaError_t nsa_dkdv_tc_launch(const NsaArgs& a, cudaStream_t st);
 cudaError_t diag_mma_tile_launch(const void* a, const void* b, float* c, int n, int b_mn_major, uint32_t* status,
                                  cudaStream_t st);
 cudaError_t diag_exp2_launch(const float* x, float* y, int n, int degree, cudaStream_t st);
+cudaError_t diag_wait_launch(uint32_t* status, int arrive, cudaStream_t st);
 
 }  // namespace sa
