@@ -193,14 +193,15 @@ struct SfaWs {
   uint32_t* status;
   int32_t *pages, *tokens, *count, *piece_unit, *piece_begin, *piece_len, *unit_first, *unit_pieces, *n_pieces;
   float *part_o, *part_m, *part_l;
-  int cap, units, max_pieces;
+  int cap, per, units, max_pieces;
 };
 
 size_t carve_sfa(const bsa_params* p, void* ws, SfaWs* w) {
   Carver c(ws);
   const int ppb = p->sparse_block_size / p->page_size;
   w->cap = p->sparse_count * ppb;
-  w->units = p->B * p->N2 * 2;
+  w->per = sfa_head_halves(p->N1 / p->N2);
+  w->units = p->B * p->N2 * w->per;
   w->max_pieces = sm_count() + w->units;
   const size_t lists = static_cast<size_t>(p->B) * p->N2 * w->cap;
   w->status = static_cast<uint32_t*>(ws);
@@ -213,9 +214,9 @@ size_t carve_sfa(const bsa_params* p, void* ws, SfaWs* w) {
   w->unit_first = c.take<int32_t>(w->units);
   w->unit_pieces = c.take<int32_t>(w->units);
   w->n_pieces = c.take<int32_t>(1);
-  w->part_o = c.take<float>(static_cast<size_t>(w->max_pieces) * 128 * 256);
-  w->part_m = c.take<float>(static_cast<size_t>(w->max_pieces) * 128);
-  w->part_l = c.take<float>(static_cast<size_t>(w->max_pieces) * 128);
+  w->part_o = c.take<float>(static_cast<size_t>(w->max_pieces) * 64 * 512);  // [piece][64 heads][Dv]
+  w->part_m = c.take<float>(static_cast<size_t>(w->max_pieces) * 64);
+  w->part_l = c.take<float>(static_cast<size_t>(w->max_pieces) * 64);
   return c.bytes();
 }
 
@@ -388,8 +389,8 @@ bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_r
   m.page_size = p->page_size; m.max_pages_per_seq = p->max_pages_per_seq; m.num_pages = p->num_pages;
   m.pages = w.pages; m.tokens = w.tokens; m.count = w.count; m.status = w.status;
   if ((e = sfa_page_list(m, st)) != cudaSuccess) return BSA_ERR_CUDA;
-  if ((e = sfa_work_list(w.count, w.units, w.max_pieces - w.units, w.piece_unit, w.piece_begin, w.piece_len,
-                         w.unit_first, w.unit_pieces, w.n_pieces, st)) != cudaSuccess)
+  if ((e = sfa_work_list(w.count, w.units, w.per, w.max_pieces - w.units, w.piece_unit, w.piece_begin,
+                         w.piece_len, w.unit_first, w.unit_pieces, w.n_pieces, st)) != cudaSuccess)
     return BSA_ERR_CUDA;
   SfaDecodeArgs a;
   a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.page_size = p->page_size; a.num_pages = p->num_pages;

@@ -104,9 +104,12 @@ struct SfaMetaArgs {
   uint32_t* status;
 };
 cudaError_t sfa_page_list(const SfaMetaArgs& a, cudaStream_t st);
-cudaError_t sfa_work_list(const int32_t* count, int units, int G, int32_t* piece_unit, int32_t* piece_begin,
-                          int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces, int32_t* n_pieces,
-                          cudaStream_t st);
+// units (b, g, head half), `per` head halves per (b, g); G = CTAs of one wave
+cudaError_t sfa_work_list(const int32_t* count, int units, int per, int G, int32_t* piece_unit,
+                          int32_t* piece_begin, int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces,
+                          int32_t* n_pieces, cudaStream_t st);
+// head halves of 64 per kv head: 2 when the group has more than 64 query heads
+int sfa_head_halves(int G);
 struct SfaDecodeArgs {
   int B, N1, N2, page_size, num_pages, cap, units, max_pieces;
   float scale;

@@ -6,10 +6,10 @@
 //                   order, compacted (empty slots and pages past seqused_kv dropped), with the
 //                   number of valid tokens of each page.  A sparse block id at or past the
 //                   sequence's block count sets SA_DEV_BAD_INDEX and is skipped.
-//   sfa_work_list   units (b, g, Dv half) each own a page list; one CTA computes a piece of at
-//                   most `chunk` consecutive pages of one unit, with chunk the smallest size whose
-//                   pieces fit one wave of CTAs (so the longest piece is as short as possible).
-//                   Pieces are numbered unit by unit.
+//   sfa_work_list   units (b, g, head half) share the page list of (b, g); one CTA computes a
+//                   piece of at most `chunk` consecutive pages of one unit, with chunk the smallest
+//                   size whose pieces fit one wave of CTAs (so the longest piece is as short as
+//                   possible).  Pieces are numbered unit by unit.
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -73,12 +73,13 @@ __global__ void sfa_page_list_kernel(const int32_t* __restrict__ sparse_indices,
 }
 
 // One CTA: choose the piece size and lay out the pieces.
-//   units u = (b * N2 + g) * 2 + dv_half; n_u = count[b, g]
+//   units u = (b * N2 + g) * per + head_half; n_u = count[b, g]
 //   chunk = the smallest c >= 1 with sum_u ceil(n_u / c) <= G (binary search; with more units
 //   than G it ends at c = max n_u, one piece per unit, and the piece arrays, sized G + units,
 //   still hold them)
 //   piece records: unit, first page, page count; unit_first[u], unit_pieces[u]
-__global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __restrict__ count, int units, int G,
+__global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __restrict__ count, int units, int per,
+                                                             int G,
                                                              int32_t* __restrict__ piece_unit,
                                                              int32_t* __restrict__ piece_begin,
                                                              int32_t* __restrict__ piece_len,
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __re
   if (tid == 0) s_max = 1;
   __syncthreads();
   int mx = 1;
-  for (int u = tid; u < units; u += blockDim.x) mx = max(mx, count[u >> 1]);
+  for (int u = tid; u < units; u += blockDim.x) mx = max(mx, count[u / per]);
   atomicMax(&s_max, mx);
   __syncthreads();
   int lo = 1, hi = s_max;  // pieces(hi) = units <= G
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __re
     __syncthreads();
     int loc = 0;
     for (int u = tid; u < units; u += blockDim.x) {
-      const int n = count[u >> 1];
+      const int n = count[u / per];
       loc += n > 0 ? (n + mid - 1) / mid : 0;
     }
     atomicAdd(&s_pieces, loc);  // integer sum: order does not matter
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(1024) sfa_work_list_kernel(const int32_t* __re
   // exclusive scan of pieces per unit, in unit order
   for (int base = 0; base < units; base += blockDim.x) {
     const int u = base + tid;
-    const int n = u < units ? count[u >> 1] : 0;
+    const int n = u < units ? count[u / per] : 0;
     const int pcs = u < units ? (n > 0 ? (n + chunk - 1) / chunk : 0) : 0;
     int x = pcs;
 #pragma unroll
@@ -174,11 +175,11 @@ cudaError_t sfa_page_list(const SfaMetaArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t sfa_work_list(const int32_t* count, int units, int G, int32_t* piece_unit, int32_t* piece_begin,
-                          int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces, int32_t* n_pieces,
-                          cudaStream_t st) {
+cudaError_t sfa_work_list(const int32_t* count, int units, int per, int G, int32_t* piece_unit,
+                          int32_t* piece_begin, int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces,
+                          int32_t* n_pieces, cudaStream_t st) {
   prof_begin("sfa_work_list", st);
-  cudaError_t e = launch_pdl(sfa_work_list_kernel, dim3(1), dim3(1024), 0, st, count, units, G, piece_unit,
+  cudaError_t e = launch_pdl(sfa_work_list_kernel, dim3(1), dim3(1024), 0, st, count, units, per, G, piece_unit,
                              piece_begin, piece_len, unit_first, unit_pieces, n_pieces);
   prof_end(st);
   return e != cudaSuccess ? e : cudaGetLastError();
