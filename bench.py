@@ -54,8 +54,8 @@ NCU_TRAFFIC = {
                   "src_sha1": "1b48ca31dc53"},
     "bsa_fwd": {"bytes": 201541888 + 51276544, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
                 "src_sha1": "90fa1eb3e002"},
-    "sfa_decode": {"bytes": 147432192 + 3553536, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
-                   "src_sha1": "274bce18f713"},
+    "sfa_decode": {"bytes": 147414528 + 4740864, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
+                   "src_sha1": "b6892b780a60"},
     # profiles/nsa_token_kernels_T16384.md (full-size launch, T = 61440)
     "nsa_bwd_dq": {"bytes": 2239617536 + 985623296, "config": 3, "src": "selected_attention_b200/csrc/nsa.cu",
                    "src_sha1": "ea904e4aa7c6"},

@@ -12,6 +12,8 @@
 // 256 TMEM columns and the two S^T buffers 128, so every head of the CTA keeps all 512 dv columns
 // and S is computed once per head.  K streams through a ring of [128 tokens][64 dims] slots and V
 // through a ring of [2 x 64 dv][64 tokens] slots, each ring with its own producer and consumer.
+// P^T has a single shared-memory buffer (written once O^T += V^T P^T of the previous tile has
+// completed); the 16 KB that a second one would take hold a fourth V slot instead.
 //
 // The softmax runs across tokens, i.e. across TMEM lanes: each softmax thread owns one token of a
 // tile and 32 heads.  Per tile the four warps of a head half reduce their maxima with redux.sync
@@ -39,7 +41,7 @@ constexpr int kDR = 64;       // rope dim
 constexpr int kKChunks = 9;   // 8 x 64 dims of k + 1 of k_rope
 constexpr int kVUses = 8;     // V slots per tile: 4 dv tiles of 128 x 2 token halves of 64
 constexpr int kKR = 4;        // K ring depth
-constexpr int kVR = 3;        // V ring depth
+constexpr int kVR = 4;        // V ring depth
 constexpr int kSmWarps = 8;
 constexpr int kThreads = (kSmWarps + 4) * 32;
 constexpr uint32_t kColO = 0, kColS = 256;  // O^T: 4 x 64 columns; S^T buffers at 256 and 320
@@ -52,7 +54,7 @@ struct __align__(1024) DecSmem {
   uint8_t q[kKChunks][kHeads * 128];  // Q rows (heads) x 64 dims per chunk, 128-byte swizzle
   uint8_t k[kKR][kSlot];              // [128 tokens][64 dims]
   uint8_t v[kVR][kSlot];              // [2 dv chunks][64 tokens][64 dv]
-  uint8_t p[2][kSlot];                // P^T [128 tokens][64 heads] bf16
+  uint8_t p[kSlot];                   // P^T [128 tokens][64 heads] bf16 (one buffer)
   float red_m[2][2][4][32];           // [tile parity][head half][lane quarter][head]
   float red_l[2][4][32];              // [head half][lane quarter][head]
   uint64_t bar_q, bar_k[kKR], bar_k_empty[kKR], bar_v[kVR], bar_v_empty[kVR];
@@ -161,12 +163,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  // token coordinate of box t of tile j in the cache's token dimension; a box past the piece's
-  // end repeats the tile's first box (its rows are masked, and the copy stays in bounds)
-  auto box_token = [&](int j, int t) -> int {
-    int qb = j * n_sub + t;
-    if (qb >= n_chunks) qb = j * n_sub;
-    return plist[qb / spp] * prm.page_size + (qb % spp) * sub;
+  // Box t of tile j: its page-list entry and its token offset inside the page; a box past the
+  // piece's end repeats the tile's first box (its rows are masked, and the copy stays in bounds).
+  // The producers load the entry one tile ahead and use it one iteration later, so the load's
+  // latency is not paid at the start of every tile.
+  auto box_entry = [&](int j, int t) -> int {
+    const int qb = j * n_sub + t;
+    return qb < n_chunks ? qb : j * n_sub;
   };
 
   if (warp == kSmWarps) {
@@ -179,10 +182,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) tma_load_2d(s.q[c], &tm_q, &s.bar_q, c * 64, qrow0);
         tma_load_2d(s.q[8], &tm_qr, &s.bar_q, 0, qrow0);
       }
-      int nxt = lane < n_sub ? box_token(0, lane) : 0;
+      int nxt_page = 0, nxt_off = 0;  // page id (loaded, used next iteration) and token offset
+      if (lane < n_sub) {
+        const int qb = box_entry(0, lane);
+        nxt_page = plist[qb / spp];
+        nxt_off = (qb % spp) * sub;
+      }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int tok = nxt;
-        if (j + 1 < n_tiles && lane < n_sub) nxt = box_token(j + 1, lane);
+        const int tok = nxt_page * prm.page_size + nxt_off;
+        if (j + 1 < n_tiles && lane < n_sub) {
+          const int qb = box_entry(j + 1, lane);
+          nxt_page = plist[qb / spp];
+          nxt_off = (qb % spp) * sub;
+        }
         for (int c = 0; c < kKChunks; ++c) {
           const int use = j * kKChunks + c, slot = use % kKR;
           if (lane == 0 && use >= kKR) ok = mbar_wait(&s.bar_k_empty[slot], ((use / kKR) - 1) & 1, prm.status);
@@ -211,10 +223,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     if (n_tiles > 0) {
       const int half_boxes = n_sub / 2;  // boxes per token half
-      int nxt = lane < n_sub ? box_token(0, lane) : 0;
+      int nxt_page = 0, nxt_off = 0;  // page id (loaded, used next iteration) and token offset
+      if (lane < n_sub) {
+        const int qb = box_entry(0, lane);
+        nxt_page = plist[qb / spp];
+        nxt_off = (qb % spp) * sub;
+      }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int tok = nxt;
-        if (j + 1 < n_tiles && lane < n_sub) nxt = box_token(j + 1, lane);
+        const int tok = nxt_page * prm.page_size + nxt_off;
+        if (j + 1 < n_tiles && lane < n_sub) {
+          const int qb = box_entry(j + 1, lane);
+          nxt_page = plist[qb / spp];
+          nxt_off = (qb % spp) * sub;
+        }
         for (int x = 0; x < kVUses; ++x) {
           const int mt = x >> 1, th = x & 1;
           const int use = j * kVUses + x, slot = use % kVR;
@@ -267,11 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_o = idesc_bf16_f32(kTok, kHeads, true, true);
       // A = V^T: MN-major, the two 64-dv chunks of a slot 8 KB apart; B = P^T: MN-major, one chunk
       const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0]), 64 * 128, 1024);
-      const uint64_t dp0 = sdesc_sw128(smem_u32(s.p[0]), kSlot, 1024);
+      const uint64_t dp0 = sdesc_sw128(smem_u32(s.p), kSlot, 1024);
       bool ok = true;
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j & 1;
-        // one barrier per P buffer: its next phase needs P_{j+2}, which waits for this product
+        // one barrier per tile parity: its next phase needs P_{j+2}, written after this product
         if (!(ok = mbar_wait(&s.bar_p_full[st], (j >> 1) & 1, prm.status))) break;
         for (int x = 0; x < kVUses; ++x) {
           const int mt = x >> 1, th = x & 1;
@@ -279,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&s.bar_v[slot], (use / kVR) & 1, prm.status))) break;
           tc_fence_after();
           const uint64_t dv = sdesc_add(dv0, slot * kSlot);
-          const uint64_t dp = sdesc_add(dp0, st * kSlot + th * (64 * 128));
+          const uint64_t dp = sdesc_add(dp0, th * (64 * 128));
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             mma_bf16_ss(tmem + kColO + mt * kHeads, sdesc_add(dv, ks * 2048), sdesc_add(dp, ks * 2048), id_o,
@@ -295,11 +316,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;  // token row of the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int rt = r / sub, rin = r % sub;  // box of the row, row inside the box
-    // this row holds a token in use: its box lies in the piece and the row below the page's count
-    auto row_valid = [&](int j) -> bool {
+    // the row holds a token in use when its box lies in the piece and rin + the box's offset in
+    // the page is below the page's token count; the count is loaded one tile ahead (cnt) and
+    // compared one iteration later, so the load's latency is not paid at the start of every tile
+    int cnt = 0, cnt_off = 0;
+    auto load_count = [&](int j) {
       const int qb = j * n_sub + rt;
-      if (qb >= n_chunks) return false;
-      return rin < tlist[qb / spp] - (qb % spp) * sub;
+      if (qb < n_chunks) {
+        cnt = tlist[qb / spp];
+        cnt_off = (qb % spp) * sub;
+      } else {
+        cnt = 0;
+        cnt_off = 0;
+      }
     };
     float m[32], l[32];
 #pragma unroll
@@ -308,11 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       l[i] = 0.f;
     }
     bool ok = true;
-    bool nxt_valid = n_tiles > 0 ? row_valid(0) : false;
+    if (n_tiles > 0) load_count(0);
     for (int j = 0; j < n_tiles; ++j) {
       const int st = j & 1;
-      const bool tv = nxt_valid;
-      if (j + 1 < n_tiles) nxt_valid = row_valid(j + 1);
+      const bool tv = rin + cnt_off < cnt;
+      if (j + 1 < n_tiles) load_count(j + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (j >> 1) & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
@@ -364,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // P buffer st is free once O^T += V^T P^T_{j-2} has completed
-      if (j >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[st], ((j >> 1) - 1) & 1, prm.status));
+      // the P buffer is free once O^T += V^T P^T_{j-1} has completed
+      if (j >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[st ^ 1], ((j - 1) >> 1) & 1, prm.status));
         if (!ok) break;
       }
 #pragma unroll
@@ -382,11 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           l[i + 1] += e1;
           hv[e] = pack_bf16(e0, e1);
         }
-        *reinterpret_cast<uint4*>(s.p[st] + sw128(r, hc * 4 + cc)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(s.p + sw128(r, hc * 4 + cc)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       }
       if (any && j > 0) {
-        // O^T holds P_{j-1} V_{j-1} once pv_done of buffer j-1 has its phase; the phase before it
-        // completed before P_{j-1} was written, so the parity is exact
+        // O^T holds P_{j-1} V_{j-1} once pv_done of tile j-1 has its phase (already waited for
+        // above, before P_j was written); the phase before it completed before P_{j-1} was
+        // written, so the parity is exact
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[st ^ 1], ((j - 1) >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
