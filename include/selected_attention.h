@@ -156,7 +156,24 @@ BSA_API bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const vo
                             size_t workspace_bytes, void* stream);
 
 /* ---- SFA sparse decode (SparseFlashAttention page), PA_ND caches, D = Dv = 512, D_rope = 64 -
- * Out = softmax((q k~^T + q_rope k_rope~^T) * scale) v~ over the selected sparse blocks. */
+ * Out = softmax((q k~^T + q_rope k_rope~^T) * scale) v~ over the selected sparse blocks.
+ *   p->kv_layout = BSA_LAYOUT_PA_ND, S_q = 1.  q [B, 1, N1, 512], q_rope [B, 1, N1, 64];
+ *   k_cache, v_cache [num_pages, page_size, N2, 512] and k_rope_cache [num_pages, page_size, N2,
+ *   64]; out [B, 1, N1, 512] bf16, lse [B, 1, N1] fp32.  block_table [B, max_pages_per_seq] maps
+ *   a sequence's logical page to its physical page; sparse_indices [B, 1, N2, sparse_count]
+ *   holds logical sparse-block ids (sparse_block_size tokens each, a whole number of pages;
+ *   -1 = empty slot); seqused_kv [B] is each sequence's token count: keys at or past it are not
+ *   attended.  Query head h uses kv head h / (N1 / N2).
+ *   Cache rows past seqused_kv inside a selected page are read by the tensor-core products with
+ *   weight exactly zero, so they must hold finite values (0 * NaN is NaN); rows of pages that no
+ *   selected block reaches are never read.
+ *   Host errors: UNSUPPORTED for S_q != 1, D / Dv / D_rope other than 512 / 512 / 64, N1 / N2 >
+ *   128, page_size not a multiple of 32, or num_pages * page_size * N2 >= 2^31; INVALID_ARG for
+ *   non-positive sizes, N1 % N2 != 0, page_size not a multiple of 16 in [16, 1024],
+ *   sparse_block_size not a multiple of page_size, or a non-finite or non-positive scale.
+ *   Device status bits: SA_DEV_BAD_INDEX for a sparse id at or past the sequence's block count,
+ *   or a table entry outside [0, num_pages) (the block is skipped).
+ *   A sequence with no selected key produces Out = 0 and LSE = -inf. */
 BSA_API bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_rope, const void* k_cache,
                              const void* k_rope_cache, const void* v_cache, void* out, float* lse,
                              void* workspace, size_t workspace_bytes, void* stream);

@@ -81,7 +81,7 @@ size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
 
 // ---- SFA (SparseFlashAttention page constraints) ----------------------------------------------------
 // query / key / value dims 512 with a 64-dim rope part; the page size a multiple of 16 up to 1024
-// (this library's 32-token tiles need a multiple of 32);
+// (this library's TMA boxes of 32 or 64 tokens must divide the page, hence a multiple of 32);
 // the sparse block size must be a whole number of pages; decode: one query row per batch.
 bsa_status check_sfa(const bsa_params* p) {
   if (!p) return BSA_ERR_NULLPTR;
