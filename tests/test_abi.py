@@ -78,3 +78,72 @@ def test_workspace_size_matches_layout():
     assert code == sa.BSA_OK and n >= 4 * (units + units + 1 + units * nkb)
     lay = sa.sparse_attn_metadata_layout(p, sa.META_BSA_KV)
     assert lay.count == 4 and lay.total_bytes >= lay.offsets[3] + 4 * units
+
+
+def _sfa(**kw):
+    p = sa.Params()
+    p.q_layout, p.kv_layout = sa.LAYOUT_BSND, sa.LAYOUT_PA_ND
+    p.B, p.N1, p.N2, p.S_q, p.D, p.Dv, p.D_rope = 2, 128, 1, 1, 512, 512, 64
+    p.page_size, p.sparse_block_size, p.sparse_count = 64, 64, 32
+    p.max_pages_per_seq, p.num_pages, p.scale = 1024, 2048, 576 ** -0.5
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_sfa_host_validation():
+    """SparseFlashAttention constraints: D = Dv = 512 with a 64-dim rope part, one query row,
+    a page size that is a multiple of 16 (here of 32), sparse blocks of whole pages."""
+    fn = "sfa_sparse_decode_workspace_size"
+    code, n = _ws(fn, _sfa())
+    assert code == sa.BSA_OK and n > 0
+    assert _ws(fn, _sfa(S_q=2))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws(fn, _sfa(D=256, Dv=256))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws(fn, _sfa(D_rope=0))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws(fn, _sfa(page_size=48, sparse_block_size=96))[0] == sa.BSA_ERR_UNSUPPORTED  # not a multiple of 32
+    assert _ws(fn, _sfa(page_size=40))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws(fn, _sfa(page_size=2048, sparse_block_size=2048))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws(fn, _sfa(sparse_block_size=96))[0] == sa.BSA_ERR_INVALID_ARG  # not whole pages
+    assert _ws(fn, _sfa(N2=3))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws(fn, _sfa(N1=256))[0] == sa.BSA_ERR_UNSUPPORTED  # G > 128
+    assert _ws(fn, _sfa(num_pages=1 << 25))[0] == sa.BSA_ERR_UNSUPPORTED  # token index past int32
+    assert _ws(fn, _sfa(scale=float("inf")))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws(fn, _sfa(kv_layout=sa.LAYOUT_BNSD))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws(fn, _sfa(page_size=32, sparse_block_size=64))[0] == sa.BSA_OK  # 32-token pages
+    # a group of more than 64 query heads is split into two head halves, each with its own pieces
+    n64 = _ws(fn, _sfa(N1=64))[1]
+    assert _ws(fn, _sfa(N1=96))[1] > n64
+    L = sa.lib()
+    p = _sfa()
+    assert L.sfa_sparse_decode(ctypes.byref(p), None, None, None, None, None, None, None, None, 0,
+                               None) == sa.BSA_ERR_NULLPTR
+
+
+def _nsa(**kw):
+    p = sa.Params()
+    p.q_layout = p.kv_layout = sa.LAYOUT_TND
+    p.B, p.N1, p.N2, p.T_q, p.T_kv, p.S_q, p.D, p.Dv = 2, 64, 4, 4096, 4096, 2048, 128, 128
+    p.sel_block_size, p.sel_block_count, p.mask_mode, p.scale = 64, 16, 2, 0.088
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_nsa_host_validation():
+    """NsaSelectedAttention constraints: TND, headdim 128, block size a multiple of 16 up to 128,
+    at most 128 blocks and 8K selected tokens, sparseMode 0 or 2, equal query and key lengths."""
+    for fn in ("nsa_selected_fwd_workspace_size", "nsa_selected_bwd_workspace_size"):
+        code, n = _ws(fn, _nsa())
+        assert code == sa.BSA_OK and n > 0
+        assert _ws(fn, _nsa(q_layout=sa.LAYOUT_BNSD))[0] == sa.BSA_ERR_UNSUPPORTED
+        assert _ws(fn, _nsa(D=64, Dv=64))[0] == sa.BSA_ERR_UNSUPPORTED
+        assert _ws(fn, _nsa(sel_block_size=40))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(sel_block_size=256))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(sel_block_count=129))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(sel_block_count=128, sel_block_size=128))[0] == sa.BSA_ERR_INVALID_ARG  # > 8K tokens
+        assert _ws(fn, _nsa(mask_mode=3))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(T_kv=4000))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(N2=3))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(N1=256, N2=4))[0] == sa.BSA_ERR_INVALID_ARG
+        assert _ws(fn, _nsa(S_q=5000))[0] == sa.BSA_ERR_INVALID_ARG  # longer than T
+        assert _ws(fn, _nsa(scale=0.0))[0] == sa.BSA_ERR_INVALID_ARG
