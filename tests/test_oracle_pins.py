@@ -226,6 +226,37 @@ def test_sfa_matches_dense_sdpa():
         assert np.allclose(lse[b, 0], r_lse[0, :, 0], atol=1e-12)
 
 
+def test_sfa_readings_multi_page_blocks_duplicates_and_empty():
+    """Sparse blocks of two scattered pages each, a sequence cut inside a page, a duplicated id
+    (gathered twice, the literal reading) and a row with no valid id (Out = 0, LSE = -inf), against
+    dense SDPA over an explicitly built key list."""
+    rng = np.random.default_rng(9)
+    B, N1, N2, D, Dr, page, ppb, n_logical, K = 2, 4, 1, 8, 4, 4, 2, 8, 3
+    sbs = page * ppb
+    n_pages = B * n_logical + 2
+    table = rng.permutation(n_pages)[:B * n_logical].reshape(B, n_logical).astype(np.int32)
+    kc, krc, vc = _rand(rng, n_pages, page, N2, D), _rand(rng, n_pages, page, N2, Dr), \
+        _rand(rng, n_pages, page, N2, D)
+    q, qr = _rand(rng, B, 1, N1, D), _rand(rng, B, 1, N1, Dr)
+    seqused = np.array([n_logical * page - 3, 0])        # batch 0 ends inside its last page
+    idx = np.array([[[[3, 1, 3]]], [[[-1, -1, -1]]]], np.int32)  # block 3 listed twice; batch 1 empty
+    scale = 0.4
+    out, lse = A.sfa_decode(q, qr, kc, krc, vc, table, idx, seqused, page, sbs, scale)
+    # batch 0: keys of blocks 3, 1, 3 in that order, each block = logical pages 2j, 2j + 1
+    toks = [j * sbs + t for j in (3, 1, 3) for t in range(sbs) if j * sbs + t < seqused[0]]
+    kk = np.stack([kc[table[0, t // page], t % page] for t in toks])      # [L, N2, D]
+    kr = np.stack([krc[table[0, t // page], t % page] for t in toks])
+    vv = np.stack([vc[table[0, t // page], t % page] for t in toks])
+    tr = lambda x: x.transpose(1, 0, 2)[None]  # noqa: E731
+    dense = np.ones((1, N1, 1, len(toks)), dtype=bool)
+    r_out, r_lse = _torch_sdpa(q[0].transpose(1, 0, 2)[None], tr(kk), tr(vv), dense, scale,
+                               q2=qr[0].transpose(1, 0, 2)[None], k2=tr(kr))
+    assert len(toks) == 3 * sbs - 2 * 3  # block 3 holds the cut page (3 tokens past the end), twice
+    assert np.allclose(out[0, 0], r_out[0, :, 0], atol=1e-12)
+    assert np.allclose(lse[0, 0], r_lse[0, :, 0], atol=1e-12)
+    assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1]))
+
+
 # ---------------------------------------------------------------------------------------------
 # finite differences
 # ---------------------------------------------------------------------------------------------
