@@ -13,8 +13,9 @@ from workloads import synth
 pytestmark = pytest.mark.gpu
 
 
-def _problem(B, N1, N2, page, n_logical, K, sbs, seqused, seed, fill_nan=True):
-    """Random paged problem; unselected pages are NaN so a wrong gather shows up."""
+def _problem(B, N1, N2, page, n_logical, K, sbs, seqused, seed, fill_nan=True, dup=False):
+    """Random paged problem; unselected pages are NaN so a wrong gather shows up.  dup: the last
+    slot of every row repeats the first (a duplicated id is gathered twice)."""
     rng = np.random.default_rng(seed)
     n_pages = B * n_logical + 5
     table = rng.permutation(n_pages)[:B * n_logical].reshape(B, n_logical).astype(np.int32)
@@ -25,6 +26,8 @@ def _problem(B, N1, N2, page, n_logical, K, sbs, seqused, seed, fill_nan=True):
         for g in range(N2):
             idx[b, 0, g] = rng.choice(max(nsb, K), size=K, replace=False)
             idx[b, 0, g][idx[b, 0, g] >= nsb] = -1
+    if dup:
+        idx[:, 0, :, -1] = idx[:, 0, :, 0]
     bits = lambda *s: synth.f32_to_bf16_bits(rng.standard_normal(s, dtype=np.float32))  # noqa: E731
     q, qr = bits(B, 1, N1, 512), bits(B, 1, N1, 64)
     kc, krc, vc = bits(n_pages, page, N2, 512), bits(n_pages, page, N2, 64), bits(n_pages, page, N2, 512)
@@ -61,6 +64,7 @@ def _run(pb, scale=None):
     dict(B=3, N1=128, N2=1, page=64, n_logical=8, K=4, sbs=64, seqused=[512, 0, 130]),   # an empty batch
     dict(B=2, N1=96, N2=1, page=64, n_logical=12, K=7, sbs=64, seqused=[700, 768]),      # second head half of 32
     dict(B=2, N1=16, N2=2, page=64, n_logical=10, K=6, sbs=64, seqused=[640, 500]),      # G = 8
+    dict(B=2, N1=128, N2=1, page=64, n_logical=12, K=5, sbs=64, seqused=[700, 768], dup=True),  # an id twice
 ])
 def test_sfa_decode_cases(cuda_ok, case):
     pb = _problem(**case, seed=21)
