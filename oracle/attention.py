@@ -17,7 +17,9 @@ plain definition, with no blocking, online rescaling or reordering:
     with dK/dV summed over every query row (and every query head of the GQA group) that used
     the key.
   * Sparse decode (SparseFlashAttention page, formula): softmax(Q K~^T / sqrt(d_k)) V~ with the
-    rope split scoring (q.k + q_rope.k_rope) / sqrt(D + Dr).
+    rope split scoring (q.k + q_rope.k_rope) / sqrt(D + Dr).  Its backward (no CUDA counterpart
+    yet) applies the backward formulas above to the gathered keys, the rope parts included, and
+    adds each key's gradient to the cache row it came from.
 
 Readings of points the pages leave open (each also listed in the design notes):
   * GQA: query head h uses kv head h // (N1 / N2) (contiguous groups; N1 % N2 == 0 rule).
@@ -373,3 +375,42 @@ def sfa_decode(q, q_rope, k_cache, k_rope_cache, v_cache, block_table, sparse_in
                                     pos, page_size, scale)
             out[b, :, hs], lse[b, :, hs] = o, l
     return out, lse
+
+
+def sfa_backward(q, q_rope, k_cache, k_rope_cache, v_cache, dout, block_table, sparse_indices,
+                 seqused_kv, page_size, sparse_block, scale):
+    """Backward of sfa_decode: the BlockSparseAttentionGrad backward formulas applied to the
+    gathered keys with the rope split score s = scale (q.k + q_rope.k_rope), so
+        dQ = (dS K~) scale,  dQ_rope = (dS K~_rope) scale,
+        dK~ = (dS^T Q) scale, dK~_rope = (dS^T Q_rope) scale, dV~ = P^T dOut,
+    and each gathered key's gradient is added to the cache row it was read from (a sparse block
+    listed twice adds twice; rows never read stay zero).  Arrays as in sfa_decode, caches as
+    arrays.  Returns dQ, dQ_rope, dK_cache, dK_rope_cache, dV_cache, Out, LSE."""
+    out_storage = "bf16" if np.asarray(q).dtype == np.uint16 else None
+    q, q_rope, dout = _f64(q), _f64(q_rope), _f64(dout)
+    k_cache, k_rope_cache, v_cache = _f64(k_cache), _f64(k_rope_cache), _f64(v_cache)
+    B, Sq, N1, _ = q.shape
+    N2 = sparse_indices.shape[2]
+    G = N1 // N2
+    dq, dqr = np.zeros(q.shape), np.zeros(q_rope.shape)
+    dk, dkr, dv = np.zeros(k_cache.shape), np.zeros(k_rope_cache.shape), np.zeros(v_cache.shape)
+    out = np.zeros((B, Sq, N1, v_cache.shape[-1]))
+    lse = np.zeros((B, Sq, N1))
+    for b in range(B):
+        for g in range(N2):
+            hs = slice(g * G, (g + 1) * G)
+            pos = sfa_token_positions(sparse_indices[b, 0, g], sparse_block, int(seqused_kv[b]))
+            pages = np.array([int(block_table[b, p // page_size]) for p in pos], dtype=np.int64)
+            offs = np.asarray(pos, dtype=np.int64) % page_size
+            kk, kr, vv = k_cache[pages, offs, g], k_rope_cache[pages, offs, g], v_cache[pages, offs, g]
+            for s in range(Sq):
+                vis = np.ones((G, len(pos)), dtype=bool)
+                o, l, p = attend(q[b, s, hs], kk, vv, vis, scale, q_extra=q_rope[b, s, hs], k_extra=kr)
+                gq, gk, gv, gqr, gkr = attend_grad(q[b, s, hs], kk, vv, dout[b, s, hs], stored_out(o, out_storage),
+                                                   p, scale, q_extra=q_rope[b, s, hs], k_extra=kr)
+                out[b, s, hs], lse[b, s, hs] = o, l
+                dq[b, s, hs], dqr[b, s, hs] = gq, gqr
+                np.add.at(dk, (pages, offs, g), gk)
+                np.add.at(dkr, (pages, offs, g), gkr)
+                np.add.at(dv, (pages, offs, g), gv)
+    return dq, dqr, dk, dkr, dv, out, lse

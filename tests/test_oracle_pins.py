@@ -257,6 +257,69 @@ def test_sfa_readings_multi_page_blocks_duplicates_and_empty():
     assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1]))
 
 
+def _sfa_small(rng, Sq=1):
+    B, N1, N2, D, Dr, page, ppb, n_logical, K = 2, 4, 2, 8, 4, 4, 2, 8, 3
+    n_pages = B * n_logical + 2
+    table = rng.permutation(n_pages)[:B * n_logical].reshape(B, n_logical).astype(np.int32)
+    kc, krc, vc = _rand(rng, n_pages, page, N2, D), _rand(rng, n_pages, page, N2, Dr), \
+        _rand(rng, n_pages, page, N2, D)
+    q, qr, do = _rand(rng, B, Sq, N1, D), _rand(rng, B, Sq, N1, Dr), _rand(rng, B, Sq, N1, D)
+    seqused = np.array([n_logical * page - 3, n_logical * page])
+    idx = np.array([[[[3, 1, 3], [0, -1, 2]]], [[[2, 0, -1], [1, 3, 2]]]], np.int32)  # a duplicate, empty slots
+    return dict(q=q, qr=qr, do=do, kc=kc, krc=krc, vc=vc, table=table, idx=idx, seqused=seqused,
+                page=page, sbs=page * ppb)
+
+
+def test_sfa_backward_matches_autograd():
+    """Sparse-decode backward against torch float64 autograd through an explicit gather from
+    leaf cache tensors (torch's indexing backward does the scatter-add, duplicates included)."""
+    rng = np.random.default_rng(10)
+    for Sq in (1, 2):
+        pb = _sfa_small(rng, Sq)
+        scale = 0.35
+        dq, dqr, dk, dkr, dv, out, lse = A.sfa_backward(pb["q"], pb["qr"], pb["kc"], pb["krc"], pb["vc"],
+                                                        pb["do"], pb["table"], pb["idx"], pb["seqused"],
+                                                        pb["page"], pb["sbs"], scale)
+        t = {n: torch.tensor(pb[n], dtype=torch.float64, requires_grad=True) for n in ("q", "qr", "kc", "krc", "vc")}
+        B, _, N1, _ = pb["q"].shape
+        N2 = pb["kc"].shape[2]
+        G = N1 // N2
+        loss = 0.0
+        for b in range(B):
+            for g in range(N2):
+                toks = [j * pb["sbs"] + i for j in pb["idx"][b, 0, g] if j >= 0 for i in range(pb["sbs"])
+                        if j * pb["sbs"] + i < pb["seqused"][b]]
+                pages = torch.tensor([int(pb["table"][b, x // pb["page"]]) for x in toks])
+                offs = torch.tensor([x % pb["page"] for x in toks])
+                kk = torch.cat([t["kc"][pages, offs, g], t["krc"][pages, offs, g]], dim=-1)
+                vv = t["vc"][pages, offs, g]
+                qq = torch.cat([t["q"][b, :, g * G:(g + 1) * G], t["qr"][b, :, g * G:(g + 1) * G]], dim=-1)
+                o = torch.nn.functional.scaled_dot_product_attention(qq.transpose(0, 1), kk[None], vv[None],
+                                                                     scale=scale)
+                loss = loss + (o.transpose(0, 1) * torch.tensor(pb["do"][b, :, g * G:(g + 1) * G])).sum()
+                assert np.allclose(out[b, :, g * G:(g + 1) * G], o.transpose(0, 1).detach().numpy(), atol=1e-12)
+        loss.backward()
+        for got, name in ((dq, "q"), (dqr, "qr"), (dk, "kc"), (dkr, "krc"), (dv, "vc")):
+            assert np.allclose(got, t[name].grad.numpy(), atol=1e-12), name
+
+
+def test_sfa_backward_finite_differences():
+    rng = np.random.default_rng(12)
+    pb = _sfa_small(rng)
+    scale = 0.35
+    args = lambda: (pb["table"], pb["idx"], pb["seqused"], pb["page"], pb["sbs"], scale)  # noqa: E731
+    dq, dqr, dk, dkr, dv, _, _ = A.sfa_backward(pb["q"], pb["qr"], pb["kc"], pb["krc"], pb["vc"], pb["do"], *args())
+
+    def loss():
+        return float(np.sum(pb["do"] * A.sfa_decode(pb["q"], pb["qr"], pb["kc"], pb["krc"], pb["vc"], *args())[0]))
+
+    _fd_check(loss, [pb["q"], pb["qr"]], [dq, dqr])
+    # the cache rows of one read page of each kind (a page read twice through the duplicated block)
+    page = int(pb["table"][0, 3 * 2])  # block 3 of batch 0 = logical pages 6, 7
+    for name, g in (("kc", dk), ("krc", dkr), ("vc", dv)):
+        _fd_check(loss, [pb[name][page]], [g[page]])
+
+
 # ---------------------------------------------------------------------------------------------
 # finite differences
 # ---------------------------------------------------------------------------------------------
