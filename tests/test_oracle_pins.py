@@ -127,15 +127,15 @@ def test_bsa_all_blocks_is_dense_causal():
 # ---------------------------------------------------------------------------------------------
 # NSA vs dense SDPA
 # ---------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", [2, 0])
-def test_nsa_matches_dense_sdpa(mode):
+@pytest.mark.parametrize("mode,Dv", [(2, 8), (0, 8), (2, 6)])   # Dv != D: the next scope row's split
+def test_nsa_matches_dense_sdpa(mode, Dv):
     rng = np.random.default_rng(3)
     seqlens = [40, 17, 64]
     N1, N2, D, bs, K = 4, 2, 8, 8, 3
     T = sum(seqlens)
     cu = np.concatenate([[0], np.cumsum(seqlens)])
-    q, do = _rand(rng, T, N1, D), _rand(rng, T, N1, D)
-    k, v = _rand(rng, T, N2, D), _rand(rng, T, N2, D)
+    q, do = _rand(rng, T, N1, D), _rand(rng, T, N1, Dv)
+    k, v = _rand(rng, T, N2, D), _rand(rng, T, N2, Dv)
     topk = np.full((T, N2, K), -1, np.int32)
     for b, s in enumerate(seqlens):
         for t in range(s):
