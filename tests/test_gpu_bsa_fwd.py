@@ -158,41 +158,3 @@ def test_bsa_fwd_full_size_sampled(cuda_ok):
         _close(out[b, h].float().cpu().numpy(), r_out[0], f"out[{b},{h}]")
         assert np.abs(lse[b, h].cpu().numpy() - r_lse[0]).max() <= LSE_ATOL
 
-
-def _rescale_problem(seed=13):
-    """B=1, two query heads on one kv head, S=512 in four 128-key blocks, every block selected, no
-    mask.  Every query has +16 in dim 0 and every key of block j has 14 j there, so block j's
-    scores sit ~10 j (natural units, at half the usual scale) above block 0's."""
-    rng = np.random.default_rng(seed)
-    B, N1, N2, S, D, blk = 1, 2, 1, 512, 128, 128
-    f = lambda *s: rng.standard_normal(s, dtype=np.float32)  # noqa: E731
-    q, k, v = f(B, N1, S, D), f(B, N2, S, D), f(B, N2, S, D)
-    q[..., 0] += 16.0
-    k[..., 0] = 14.0 * (np.arange(S) // blk)
-    bits = synth.f32_to_bf16_bits
-    mask = np.ones((B, N1, S // blk, S // blk), np.uint8)
-    return bits(q), bits(k), bits(v), mask, blk, 0.5 / np.sqrt(D)  # half scale: flatter within a block
-
-
-def _block_jumps(q, k, blk, scale):
-    """Smallest, over rows and KV blocks after the first, of (the block's max score) - (max over
-    the earlier blocks), in log2 units: the forward visits a unit's blocks in ascending order."""
-    qq = synth.bf16_bits_to_f32(q).astype(np.float64)[0]
-    kk = synth.bf16_bits_to_f32(k).astype(np.float64)[0, 0]
-    s = np.einsum("hsd,td->hst", qq, kk) * scale / np.log(2.0)
-    bm = s.reshape(s.shape[0], s.shape[1], -1, blk).max(-1)
-    run = np.maximum.accumulate(bm, axis=-1)
-    return float((bm[..., 1:] - run[..., :-1]).min())
-
-
-def test_bsa_fwd_lazy_rescale(cuda_ok):
-    """Each KV tile raises every row's running maximum by far more than the 2^8 a tile may exceed
-    it without a rescale (checked on the inputs), so the output accumulated in TMEM is rescaled at
-    every tile; the softmax stays spread over the last block's keys."""
-    q, k, v, mask, blk, scale = _rescale_problem()
-    assert _block_jumps(q, k, blk, scale) > 8.0
-    out, lse = sa.bsa_fwd(_dev(q), _dev(k), _dev(v), torch.from_numpy(mask).cuda(), blk, blk, 0, scale)
-    torch.cuda.synchronize()
-    r_out, r_lse = A.bsa_forward(q, k, v, mask, blk, blk, 0, scale)
-    _close(out.float().cpu().numpy(), r_out, "out")
-    assert np.abs(lse.cpu().numpy() - r_lse).max() <= LSE_ATOL

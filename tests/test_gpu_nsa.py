@@ -226,44 +226,3 @@ def test_nsa_workload_full_size_sampled(cuda_ok):
             check_close(gk[t0 + sl.start:t0 + sl.stop, g].float().cpu().numpy(), r_dk[sl], f"dk[{b},{g},{kb}]")
             check_close(gv[t0 + sl.start:t0 + sl.stop, g].float().cpu().numpy(), r_dv[sl], f"dv[{b},{g},{kb}]")
 
-
-def _rescale_problem(seed=29):
-    """One 320-token batch (five 64-token blocks), G = 16 heads on one kv head, every block
-    selected, no mask.  Every query has +16 in dim 0 and every key of block j has 14 j there, so
-    block j's scores sit ~10 j (natural units, at half the usual scale) above block 0's."""
-    pb = _problem([320], N1=16, N2=1, bs=64, K=5, mode=0, seed=seed)
-    q = synth.bf16_bits_to_f32(pb["q"])
-    k = synth.bf16_bits_to_f32(pb["k"])
-    q[..., 0] += 16.0
-    k[:, :, 0] = 14.0 * (np.arange(320) // 64)[:, None]
-    pb["q"], pb["k"] = synth.f32_to_bf16_bits(q), synth.f32_to_bf16_bits(k)
-    pb["scale"] = 0.5 / np.sqrt(D)  # flatter within a block: no single bf16 P carries a row
-    return pb
-
-
-def _block_jumps(pb):
-    """Smallest, over (token, head) and selected blocks after the first, of (the block's max
-    score) - (max over the earlier selected blocks), in log2 units: the token kernels visit a
-    token's blocks in ascending id order."""
-    q = synth.bf16_bits_to_f32(pb["q"]).astype(np.float64)
-    k = synth.bf16_bits_to_f32(pb["k"]).astype(np.float64)[:, 0]
-    worst = np.inf
-    for t in range(q.shape[0]):
-        ids = sorted(int(x) for x in pb["topk"][t, 0] if x >= 0)
-        s = q[t] @ k.T * pb["scale"] / np.log(2.0)  # [heads, keys]
-        bm = np.stack([s[:, i * 64:(i + 1) * 64].max(-1) for i in ids], -1)
-        run = np.maximum.accumulate(bm, axis=-1)
-        worst = min(worst, float((bm[:, 1:] - run[:, :-1]).min()))
-    return worst
-
-
-def test_nsa_fwd_lazy_rescale(cuda_ok):
-    """Each selected block raises every (token, head) row's running maximum by far more than the
-    2^8 a chunk may exceed it without a rescale (checked on the inputs), so the output accumulated
-    in registers is rescaled at every block; the softmax stays spread over the top block's keys."""
-    pb = _rescale_problem()
-    assert (pb["topk"] >= 0).all() and _block_jumps(pb) > 8.0
-    out, lse = _fwd(pb)
-    r_out, r_lse = A.nsa_forward(pb["q"], pb["k"], pb["v"], pb["topk"], pb["cu"], pb["bs"], pb["mode"], pb["scale"])
-    check_close(out.float().cpu().numpy(), r_out, "out")
-    check_lse(lse.cpu().numpy(), r_lse)
