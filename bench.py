@@ -42,6 +42,18 @@ METRIC = "effective block-sparse attn fwd+bwd TFLOP/s (bf16)"
 METRIC_NSA = "effective NSA selected attn fwd+bwd TFLOP/s (bf16)"
 METRIC_DEC = "sparse decode gathered-KV bandwidth (paged, bf16)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures, reported beside the measured-peak fractions: dense bf16 and HBM3e
+SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+
+
+def with_spec(roof):
+    """Add the nominal peak and the fraction of it to a roofline entry (None passes through)."""
+    if roof is None:
+        return None
+    spec = SPEC_PEAKS["hbm_gbs" if roof["unit"] == "GB/s" else "bf16_tflops"]
+    roof["spec_peak"] = spec
+    roof["frac_of_spec"] = roof["achieved"] / spec if roof["achieved"] is not None else None
+    return roof
 
 # DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
 # kernel's source file is unchanged (sha1 prefix of the file recorded at capture time).
@@ -483,7 +495,7 @@ def run_nsa(args, rank, world, local_rank):
             "data": "synthetic", "config": config_dict_nsa(w, args),
             "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": sum(c for c, _ in prof.values()), "kernels": kernels, "roofline": roof,
+            "gpu_launches": sum(c for c, _ in prof.values()), "kernels": kernels, "roofline": with_spec(roof),
             "cpu_baseline": cpu, "clocks": clocks.summary(), "visible_pairs": vpairs,
             "credited_flops_per_step": flops_step,
         }))
@@ -605,10 +617,11 @@ def run_decode(args, rank, world, local_rank):
         "gpu_launches": launches_per_call * args.steps,
         "effective_tflops": world * flops / (ms * 1e-3) / 1e12,
         # dominant kernel: the decode kernel alone, its gathered bytes over its mean launch time
-        "roofline": {"bound": "hbm", "kernel": "sfa_decode", "achieved": dec_gbs,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": dec_gbs / peaks["hbm_gbs"] if dec_gbs else None,
-                     "peak_source": f"{src} hbm_gbs (burst)", "traffic": dec_traffic, "avg_launch_ms": dec_ms},
+        "roofline": with_spec({"bound": "hbm", "kernel": "sfa_decode", "achieved": dec_gbs,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": dec_gbs / peaks["hbm_gbs"] if dec_gbs else None,
+                               "peak_source": f"{src} hbm_gbs (burst)", "traffic": dec_traffic,
+                               "avg_launch_ms": dec_ms}),
         "kernels": {n: {"launches": c, "ms_per_call": t / c} for n, (c, t) in prof.items()},
         "cpu_baseline": cpu, "clocks": clocks.summary(), "gathered_bytes_per_step": gathered,
     }
@@ -731,7 +744,7 @@ def run_ours(args, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, args),
             "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": launches_total, "kernels": kernels, "roofline": roof, "cpu_baseline": cpu,
+            "gpu_launches": launches_total, "kernels": kernels, "roofline": with_spec(roof), "cpu_baseline": cpu,
             "clocks": clocks.summary(), "visible_pairs": vpairs, "credited_flops_per_step": flops_step,
         }
         print(json.dumps(line))

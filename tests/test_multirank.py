@@ -78,3 +78,14 @@ def test_reference_arm_json_line():
     assert d["impl"] == "reference" and d["dtype"] == "f64" and d["steps"] == 1 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+
+
+def test_roofline_spec_fraction():
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.with_spec({"unit": "GB/s", "achieved": 4000.0})
+    assert r["spec_peak"] == 8000.0 and r["frac_of_spec"] == 0.5
+    r = bench.with_spec({"unit": "TFLOP/s", "achieved": 1125.0})
+    assert r["spec_peak"] == 2250.0 and r["frac_of_spec"] == 0.5
+    assert bench.with_spec(None) is None
+    assert bench.with_spec({"unit": "GB/s", "achieved": None})["frac_of_spec"] is None
