@@ -147,3 +147,23 @@ def test_nsa_host_validation():
         assert _ws(fn, _nsa(N1=256, N2=4))[0] == sa.BSA_ERR_INVALID_ARG
         assert _ws(fn, _nsa(S_q=5000))[0] == sa.BSA_ERR_INVALID_ARG  # longer than T
         assert _ws(fn, _nsa(scale=0.0))[0] == sa.BSA_ERR_INVALID_ARG
+
+
+def test_metadata_layouts_without_gpu():
+    """Plan layouts of the NSA and decode metadata ops: array offsets in order, 256-byte aligned,
+    inside the plan, sized for the problem."""
+    p = _sfa()
+    lay = sa.sparse_attn_metadata_layout(p, sa.META_SFA_PAGES)
+    lists = p.B * p.N2 * p.sparse_count * (p.sparse_block_size // p.page_size)
+    assert lay.count == 4
+    offs = [lay.offsets[i] for i in range(1, 4)]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert offs[1] - offs[0] >= 4 * lists and lay.total_bytes >= offs[2] + 4 * p.B * p.N2
+    q = _nsa()
+    kv = sa.sparse_attn_metadata_layout(q, sa.META_NSA_KV)
+    tok = sa.sparse_attn_metadata_layout(q, sa.META_NSA_TOKENS)
+    assert kv.count == 3 and tok.count == 5
+    ids_bytes = 4 * q.T_q * q.N2 * q.sel_block_count
+    assert kv.offsets[2] - kv.offsets[1] >= ids_bytes and tok.total_bytes > kv.total_bytes
+    assert sa.lib().sparse_attn_metadata_layout(ctypes.byref(q), 99, ctypes.byref(sa.MetaLayout())) \
+        == sa.BSA_ERR_UNSUPPORTED
