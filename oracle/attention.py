@@ -53,10 +53,22 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
-    """float64 -> nearest bf16 value (via float32, ties to even), returned as float64."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    u = ((u + (((u >> 16) & np.uint32(1)) + np.uint32(0x7FFF))) >> 16) << 16
-    return u.view(np.float32).astype(np.float64)
+    """float64 -> the nearest bf16 value (round half to even), returned as float64.
+
+    One rounding of the exact value: bf16 keeps 8 significant bits, so a value in the binade
+    [2^(e-1), 2^e) is rounded to a multiple of 2^(e-8); below the normal range (|x| < 2^-126) the
+    step stays 2^-133 (the subnormal spacing).  Results of magnitude 2^128 or more become +-inf;
+    zeros keep their sign, infinities and NaN pass through."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.array(x, dtype=np.float64, copy=True)
+    fin = np.isfinite(x) & (x != 0)
+    xf = x[fin]
+    _, e = np.frexp(xf)                              # xf = m * 2^e with 0.5 <= |m| < 1
+    step_exp = np.maximum(e - 8, -133)
+    y = np.ldexp(np.rint(np.ldexp(xf, -step_exp)), step_exp)   # np.rint: half to even
+    y = np.where(np.abs(y) >= 2.0 ** 128, np.copysign(np.inf, xf), y)
+    out[fin] = y
+    return out
 
 
 def stored_out(o: np.ndarray, out_storage) -> np.ndarray:
@@ -160,10 +172,13 @@ def bsa_slice_forward(q_g, k_g, v_g, mask_g, bx, by, mode, scale, win_left=0, wi
 
 
 def bsa_slice_backward(q_g, k_g, v_g, dout_g, mask_g, bx, by, mode, scale, win_left=0,
-                       win_right=0, q_blocks=None, kv_blocks=None, out_storage=None):
+                       win_right=0, q_blocks=None, kv_blocks=None, out_storage=None, out_in_g=None):
     """One (batch, kv-head) slice of the backward pass.  Returns dQ [G,Sq,D], dK [Skv,D],
     dV [Skv,Dv], Out, LSE.  Units (h, qb) are skipped only when they contribute neither to a
-    requested dQ block nor to a requested KV block, so every requested entry is exact."""
+    requested dQ block nor to a requested KV block, so every requested entry is exact.
+    out_in_g [G,Sq,Dv] (float64), when given, is the attentionOut input of the backward operator:
+    softmax_grad = rowsum(dOut o attentionOut) then uses it as given instead of the oracle's own
+    forward output."""
     G, s_q, _ = q_g.shape
     s_kv = k_g.shape[0]
     nqb = mask_g.shape[1]
@@ -186,7 +201,8 @@ def bsa_slice_backward(q_g, k_g, v_g, dout_g, mask_g, bx, by, mode, scale, win_l
             vis = visible(rows, keys, mode, s_q, s_kv, s_kv, win_left, win_right)
             qr, kr, vr = q_g[h, rows], k_g[keys], v_g[keys]
             o, l, p = attend(qr, kr, vr, vis, scale)
-            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[h, rows], stored_out(o, out_storage), p, scale)
+            o_in = stored_out(o, out_storage) if out_in_g is None else out_in_g[h, rows]
+            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[h, rows], o_in, p, scale)
             out[h, rows] = o
             lse[h, rows] = l
             dq[h, rows] = g_q
@@ -216,10 +232,13 @@ def bsa_forward(q, k, v, block_mask, bx, by, mode, scale, win_left=0, win_right=
     return out, lse
 
 
-def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win_right=0):
-    """Full BNSD backward; returns dQ, dK, dV, Out, LSE."""
+def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win_right=0, out_in=None):
+    """Full BNSD backward; returns dQ, dK, dV, Out, LSE.  out_in [B,N1,Sq,Dv] (bf16 bits or
+    floats), when given, is the backward operator's attentionOut input (softmax_grad =
+    rowsum(dOut o attentionOut)); by default the oracle's own Out, stored in the input dtype."""
     out_storage = "bf16" if np.asarray(q).dtype == np.uint16 else None
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    out_in = None if out_in is None else _f64(out_in)
     B, N1, s_q, _ = q.shape
     N2 = k.shape[1]
     G = N1 // N2
@@ -232,7 +251,8 @@ def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win
         for g in range(N2):
             hs = slice(g * G, (g + 1) * G)
             r = bsa_slice_backward(q[b, hs], k[b, g], v[b, g], dout[b, hs], block_mask[b, hs],
-                                   bx, by, mode, scale, win_left, win_right, out_storage=out_storage)
+                                   bx, by, mode, scale, win_left, win_right, out_storage=out_storage,
+                                   out_in_g=None if out_in is None else out_in[b, hs])
             dq[b, hs], dk[b, g], dv[b, g], out[b, hs], lse[b, hs] = r
     return dq, dk, dv, out, lse
 
@@ -249,11 +269,12 @@ def nsa_token_keys(ids: np.ndarray, sel_block: int, seq_len: int) -> np.ndarray:
 
 
 def nsa_slice(q_g, k_g, v_g, topk_g, sel_block, mode, scale, dout_g=None, tokens=None,
-              out_storage=None):
+              out_storage=None, out_in_g=None):
     """One (batch, kv-head) slice: q_g [S, G, D], k_g [S, D], v_g [S, Dv], topk_g [S, K].
     Forward for every listed token (all by default); with dout_g also the backward pass.
     Returns Out [S,G,Dv], LSE [S,G] (+ dQ [S,G,D], dK [S,D], dV [S,Dv]); unlisted tokens are NaN
-    in Out/LSE/dQ, and dK/dV then hold only the listed tokens' contributions."""
+    in Out/LSE/dQ, and dK/dV then hold only the listed tokens' contributions.  out_in_g [S,G,Dv]
+    (float64), when given, is the backward's attentionOut input (used for softmax_grad as given)."""
     S, G, _ = q_g.shape
     out = np.full((S, G, v_g.shape[1]), np.nan)
     lse = np.full((S, G), np.nan)
@@ -268,7 +289,8 @@ def nsa_slice(q_g, k_g, v_g, topk_g, sel_block, mode, scale, dout_g=None, tokens
         o, l, p = attend(qr, kr, vr, vis, scale)
         out[t], lse[t] = o, l
         if dout_g is not None:
-            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[t], stored_out(o, out_storage), p, scale)
+            o_in = stored_out(o, out_storage) if out_in_g is None else out_in_g[t]
+            g_q, g_k, g_v = attend_grad(qr, kr, vr, dout_g[t], o_in, p, scale)
             dq[t] = g_q
             np.add.at(dk, keys, g_k)
             np.add.at(dv, keys, g_v)
@@ -295,10 +317,12 @@ def nsa_forward(q, k, v, topk, cu_seqlens, sel_block, mode, scale):
     return out, lse
 
 
-def nsa_backward(q, k, v, dout, topk, cu_seqlens, sel_block, mode, scale):
-    """Full TND backward; returns dQ, dK, dV, Out, LSE."""
+def nsa_backward(q, k, v, dout, topk, cu_seqlens, sel_block, mode, scale, out_in=None):
+    """Full TND backward; returns dQ, dK, dV, Out, LSE.  out_in [T,N1,Dv], when given, is the
+    backward's attentionOut input (as in bsa_backward)."""
     out_storage = "bf16" if np.asarray(q).dtype == np.uint16 else None
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    out_in = None if out_in is None else _f64(out_in)
     T, N1, _ = q.shape
     N2 = k.shape[1]
     G = N1 // N2
@@ -313,7 +337,8 @@ def nsa_backward(q, k, v, dout, topk, cu_seqlens, sel_block, mode, scale):
             hs = slice(g * G, (g + 1) * G)
             o, l, gq, gk, gv = nsa_slice(q[t0:t1, hs], k[t0:t1, g], v[t0:t1, g], topk[t0:t1, g],
                                          sel_block, mode, scale, dout_g=dout[t0:t1, hs],
-                                         out_storage=out_storage)
+                                         out_storage=out_storage,
+                                         out_in_g=None if out_in is None else out_in[t0:t1, hs])
             out[t0:t1, hs], lse[t0:t1, hs], dq[t0:t1, hs] = o, l, gq
             dk[t0:t1, g], dv[t0:t1, g] = gk, gv
     return dq, dk, dv, out, lse

@@ -484,10 +484,113 @@ def test_stored_out_softmax_grad_correction():
     p = np.exp(s - s.max(-1, keepdims=True))
     p /= p.sum(-1, keepdims=True)
     o = p @ v
-    dD = np.sum(do * (A.round_to_bf16(o) - o), axis=-1)                  # [B, N, S]
+    dD = np.sum(do * (_nearest_bf16_bruteforce(o) - o), axis=-1)         # [B, N, S]
     exp_dq = r_dq - sc * dD[..., None] * (p @ k)
     exp_dk = r_dk - sc * np.einsum("bhi,bhij,bhid->bhjd", dD, p, q)
     assert np.abs(dD).max() > 0                                          # the reading matters here
     assert np.allclose(dq_b, exp_dq, atol=1e-11)
     assert np.allclose(dk_b, exp_dk, atol=1e-11)
     assert np.allclose(dv_b, r_dv, atol=1e-11)
+
+
+# ---------------------------------------------------------------------------------------------
+# round_to_bf16 (the stored-attentionOut reading rests on it): pinned against torch's float32 ->
+# bfloat16 cast, a brute-force nearest search over every finite bf16 value, and a hand-worked table
+# ---------------------------------------------------------------------------------------------
+def _all_finite_bf16():
+    """Every finite bf16 value (as float64) with its bit pattern, sorted by value."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    vals = (bits << 16).view(np.float32).astype(np.float64)
+    fin = np.isfinite(vals)
+    vals, bits = vals[fin], bits[fin]
+    order = np.lexsort((bits, vals))
+    vals, bits = vals[order], bits[order]
+    keep = np.concatenate([[True], vals[1:] != vals[:-1]])   # +0 and -0 collapse to one grid point
+    return vals[keep], bits[keep]
+
+
+def _nearest_bf16_bruteforce(x):
+    """Nearest grid point of the finite bf16 values extended by +-2^128 (standing for +-inf), ties
+    to the point whose bit pattern is even."""
+    vals, bits = _all_finite_bf16()
+    vals = np.concatenate([[-2.0 ** 128], vals, [2.0 ** 128]])
+    bits = np.concatenate([[0xFF80], bits, [0x7F80]]).astype(np.uint32)
+    i = np.clip(np.searchsorted(vals, x), 1, len(vals) - 1)
+    lo, hi = vals[i - 1], vals[i]
+    dlo, dhi = x - lo, hi - x
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (bits[i] % 2 == 0))
+    y = np.where(pick_hi, hi, lo)
+    y = np.where(np.abs(y) >= 2.0 ** 128, np.copysign(np.inf, y), y)
+    return np.where(y == 0, np.copysign(0.0, x), y)
+
+
+def test_round_to_bf16_matches_torch_on_float32_values():
+    """On float32 inputs (no rounding before the bf16 step) torch's cast is round-to-nearest-even:
+    every finite float32 exponent, ties (low 16 bits exactly 0x8000), overflow, subnormals."""
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0, 1 << 32, size=300_000, dtype=np.uint64).astype(np.uint32)
+    ties = (rng.integers(0, 1 << 16, size=50_000, dtype=np.uint64).astype(np.uint32) << 16) | np.uint32(0x8000)
+    edges = np.array([0x7F7F7FFF, 0x7F7F8000, 0x7F7F8001, 0xFF7F8000, 0x00008000, 0x00018000, 0x007FFFFF,
+                      0x00800000, 0x3F808000, 0x3F818000, 0x80000000, 0x00000000], dtype=np.uint32)
+    x = np.concatenate([bits, ties, edges]).view(np.float32)
+    x = x[np.isfinite(x)]
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).to(torch.float64).numpy()
+    got = A.round_to_bf16(x.astype(np.float64))
+    assert np.array_equal(np.signbit(got), np.signbit(ref))
+    assert np.array_equal(got, ref)
+
+
+def test_round_to_bf16_is_the_nearest_bf16_of_float64_values():
+    """For float64 inputs (between float32 values too) the result is the nearest bf16 value found
+    by brute force over the whole bf16 grid, ties to even; rounding through float32 first would
+    differ on values just above a tie, which this set contains."""
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal(200_000) * np.exp2(rng.integers(-140, 129, size=200_000))
+    vals, _ = _all_finite_bf16()
+    mids = (vals[1:] + vals[:-1]) / 2
+    near_ties = rng.choice(mids, 20_000) * (1 + rng.choice([-1, 1], 20_000) * 2.0 ** -40)
+    x = np.concatenate([x, rng.choice(mids, 20_000), near_ties])
+    x = x[np.isfinite(x)]
+    assert np.array_equal(A.round_to_bf16(x), _nearest_bf16_bruteforce(x))
+
+
+def test_round_to_bf16_golden_table():
+    with open(os.path.join(GOLDEN, "bf16_rounding.json")) as f:
+        doc = json.load(f)
+    for c in doc["cases"]:
+        x, want = float.fromhex(c["x"]), float.fromhex(c["bf16"])
+        got = float(A.round_to_bf16(np.array([x]))[0])
+        assert got == want and np.signbit(got) == np.signbit(want), (c["why"], got, want)
+
+
+def test_backward_with_given_attention_out():
+    """The backward operator's attentionOut input enters only softmax_grad = rowsum(dOut o Out):
+    with Out_in = Out + E, dQ moves by -scale (dOut.E)_i (P K)_i, dK by -scale sum_i (dOut.E)_i
+    P_ik q_i and dV not at all; P, Out and the base gradients from torch (float64).  Checked for
+    the BSA and the NSA entry points (NSA: one token per block, so its keys are a BSA block)."""
+    rng = np.random.default_rng(14)
+    B, N, S, D, bs = 1, 2, 32, 16, 8
+    q, k, v, do = (_rand(rng, B, N, S, D) for _ in range(4))
+    mask = np.tril(np.ones((4, 4), np.uint8))[None, None].repeat(N, 1)
+    sc = 0.3
+    dense = _dense_mask_bsa(mask, bs, bs, S, S, 2)
+    r_out, _, r_dq, r_dk, r_dv = _torch_sdpa(q, k, v, dense, sc, do)
+    E = _rand(rng, B, N, S, D) * 0.01
+    dq, dk, dv, _, _ = A.bsa_backward(q, k, v, do, mask, bs, bs, 2, sc, out_in=r_out + E)
+    s = sc * np.einsum("bhid,bhjd->bhij", q, k)
+    s = np.where(dense, s, -np.inf)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    dD = np.sum(do * E, axis=-1)
+    assert np.allclose(dq, r_dq - sc * dD[..., None] * (p @ k), atol=1e-11)
+    assert np.allclose(dk, r_dk - sc * np.einsum("bhi,bhij,bhid->bhjd", dD, p, q), atol=1e-11)
+    assert np.allclose(dv, r_dv, atol=1e-11)
+    # NSA: TND with N2 = N (G = 1), every token lists all causal blocks
+    qt, kt, vt, dot = (x[0].transpose(1, 0, 2) for x in (q, k, v, do))      # [S, N, D]
+    topk = np.array([[list(range(t // bs + 1)) + [-1] * (3 - t // bs) for _ in range(N)] for t in range(S)],
+                    dtype=np.int32)
+    Et = E[0].transpose(1, 0, 2)
+    ndq, ndk, ndv, _, _ = A.nsa_backward(qt, kt, vt, dot, topk, np.array([0, S]), bs, 2, sc,
+                                         out_in=r_out[0].transpose(1, 0, 2) + Et)
+    assert np.allclose(ndq, (r_dq - sc * dD[..., None] * (p @ k))[0].transpose(1, 0, 2), atol=1e-11)
+    assert np.allclose(ndv, r_dv[0].transpose(1, 0, 2), atol=1e-11)
