@@ -134,7 +134,8 @@ def test_nsa_bwd_cases(cuda_ok, case):
 
 
 def test_nsa_chained_determinism_and_invariants(cuda_ok):
-    """GPU forward -> GPU backward, twice: bit-identical; per (token, head) the softmax Jacobian
+    """GPU forward -> GPU backward, twice: bit-identical, and element by element against the
+    oracle's backward on the GPU's Out; per (token, head) the softmax Jacobian
     gives sum over keys of dS = 0, so sum_t dK[t, g] = 0 per kv head, and sum_t dV[t, g] equals
     the sum of dOut over the group's heads and the tokens that see at least one key.  The sums run
     over bf16-stored rows, each within 2^-8 relative of its fp32 value, which sets the bound."""
@@ -145,6 +146,13 @@ def test_nsa_chained_determinism_and_invariants(cuda_ok):
         runs.append((out, lse) + _bwd(pb, out, lse))
     for a, b in zip(runs[0], runs[1]):
         assert torch.equal(a, b)
+    # element by element against the oracle's backward given the GPU's Out as attentionOut
+    gpu_out = runs[0][0].view(torch.int16).cpu().numpy().view(np.uint16)
+    c_dq, c_dk, c_dv, _, _ = A.nsa_backward(pb["q"], pb["k"], pb["v"], pb["do"], pb["topk"], pb["cu"], pb["bs"],
+                                            pb["mode"], pb["scale"], out_in=gpu_out)
+    check_close(runs[0][2].float().cpu().numpy(), c_dq, "chained dq")
+    check_close(runs[0][3].float().cpu().numpy(), c_dk, "chained dk")
+    check_close(runs[0][4].float().cpu().numpy(), c_dv, "chained dv")
     _, _, _, gk, gv = runs[0]
     G = 8
     do = A.bf16_to_f64(pb["do"]).reshape(-1, 2, G, D).sum(axis=2)        # [T, N2, D]
