@@ -115,14 +115,18 @@ BSA_API bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, co
  * memory and gives its plugins no scratch, or a path where a cudaMalloc is not acceptable).  The
  * paper has no counterpart: this entry point exists for such callers only.  It needs no
  * workspace: its scratch (status word and KV lists) is a fixed 8 MiB device array inside the
- * library, held by every GPU that loads the library until the process exits.  The first call on
- * a device looks up that array's device address (cudaGetSymbolAddress) and should come before
- * any stream capture.  Problems whose bsa_fwd workspace exceeds 8 MiB return
- * BSA_ERR_WORKSPACE_TOO_SMALL.  All calls on a device share the array: calls whose GPU work
- * overlaps race and must be ordered by the caller.  Device status bits stay in the array and are
- * not reported. */
+ * library, held by every GPU that loads the library until the process exits.  The first call in a
+ * CUDA context looks up that array's device address there (cudaGetSymbolAddress) and keeps it for
+ * the context; the first call on a device should come before any stream capture.  Problems whose
+ * bsa_fwd workspace exceeds 8 MiB return BSA_ERR_WORKSPACE_TOO_SMALL before any launch.  All calls
+ * on a device share the array: calls whose GPU work overlaps race and must be ordered by the
+ * caller.  The device status bits of the last call stay in the array: read them with
+ * bsa_fwd_noalloc_get_status. */
 BSA_API bsa_status bsa_fwd_noalloc(const bsa_params* p, const void* q, const void* k, const void* v, void* out,
                                    float* lse, void* stream);
+/* Device status bits (SA_DEV_*) of the last bsa_fwd_noalloc call on the current device, after
+ * synchronising `stream` (as bsa_get_status).  No counterpart in the paper. */
+BSA_API bsa_status bsa_fwd_noalloc_get_status(void* stream, uint32_t* dev_bits);
 /* Backward: softmax_grad = rowsum(dOut o Out); dP = dOut V^T; dS = P o (dP - softmax_grad);
  * dV = P^T dOut; dQ = dS K scale; dK = dS^T Q scale.  `out` and `lse` are the forward's
  * outputs.  dK/dV are accumulated in a fixed order (run-to-run bit identical, no atomics). */

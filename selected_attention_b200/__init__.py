@@ -29,7 +29,8 @@ EXPORTED = [
     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size", "bsa_fwd", "bsa_bwd",
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
-    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_diag_exp2", "bsa_diag_wait",
+    "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_fwd_noalloc_get_status", "bsa_diag_exp2",
+    "bsa_diag_wait",
 ]
 
 
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.bsa_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nsa_selected_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         L.bsa_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
+        L.bsa_fwd_noalloc_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.bsa_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nsa_selected_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sfa_sparse_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -193,6 +195,13 @@ def bsa_fwd_noalloc(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL
     _check("bsa_fwd_noalloc", lib().bsa_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                                     _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def bsa_fwd_noalloc_get_status(stream=None) -> int:
+    """Device status bits of the last bsa_fwd_noalloc call on the current device (synchronises)."""
+    v = ctypes.c_uint32()
+    _check("bsa_fwd_noalloc_get_status", lib().bsa_fwd_noalloc_get_status(_stream(stream), ctypes.byref(v)))
+    return v.value
 
 
 def bsa_bwd_workspace_size(p: Params) -> int:
