@@ -3,11 +3,19 @@
 
 One step = one pass of the whole hot path over one batch: metadata (KV lists, transposed
 lists) + forward (Out, LSE) + backward (dQ, dK, dV), all in the library's CUDA kernels.  The
-default workload is block-sparse attention at B=2, N=16, S=8192, D=128 with 128x128 blocks
-and a causal Bernoulli(0.25) BlockSparseMask (synthetic, seeded).
+default workload is the long-context block-sparse attention: B=1, N=32, S=131072, D=128 with
+128x128 blocks, each q block selecting min(64, causal) KV blocks (diagonal, 4 previous, the
+first block, the rest uniform), causal (synthetic, seeded).  --config 2 runs the S=8192 workload
+(B=2, N=16, causal Bernoulli(0.25) mask).
 
 The metric is effective TFLOP/s: credited FLOPs / time, with forward 4*D*V and backward
-10*D*V for V visible (query, key) pairs (the diagonal block counts only its visible half).
+10*D*V for V visible (query, key) pairs (the diagonal block counts only its visible half).  Per
+kernel the credits are forward 4*D*V (S, O), KV-major pass 8*D*V (S, dP, dV, dK) and Q-major pass
+2*D*V (dQ only: its S and dP are recomputations already credited to the KV pass).
+
+The end-to-end number copies each step's inputs in from pinned host memory and every output back,
+with the host-to-device and device-to-host copies on their own streams, double-buffered against
+the compute stream (the copies of step i+1 and i-1 overlap the compute of step i).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1|2|3|4|5]
 
@@ -55,11 +63,10 @@ def with_spec(roof):
     roof["frac_of_spec"] = roof["achieved"] / spec if roof["achieved"] is not None else None
     return roof
 
-# DRAM bytes per launch from an ncu capture of each kernel (profiles/), valid only while the
-# kernel's source file is unchanged (sha1 prefix of the file recorded at capture time).
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum of one launch) from an ncu
+# capture of each kernel, valid only while the kernel's source file is unchanged (sha1 prefix of
+# the file recorded at capture time); reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # profiles/bsa_S8192_fwd_bwd.md, profiles/sfa_decode_B32.md, profiles/nsa_token_kernels_T16384.md
-    # (dram__bytes_read.sum + dram__bytes_write.sum of one launch; null once the source has changed)
     "bsa_bwd_kv": {"bytes": 270692864 + 105957888, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
                    "src_sha1": "1b48ca31dc53"},
     "bsa_bwd_q": {"bytes": 270671872 + 53610752, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
@@ -68,7 +75,7 @@ NCU_TRAFFIC = {
                 "src_sha1": "90fa1eb3e002"},
     "sfa_decode": {"bytes": 147414528 + 4740864, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
                    "src_sha1": "b6892b780a60"},
-    # profiles/nsa_token_kernels_T16384.md (full-size launch, T = 61440)
+    # full-size launch, T = 61440
     "nsa_bwd_dq": {"bytes": 2239617536 + 985623296, "config": 3, "src": "selected_attention_b200/csrc/nsa.cu",
                    "src_sha1": "ea904e4aa7c6"},
 }
@@ -293,6 +300,89 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def pipelined_e2e(steps, host_in, dev_in, dev_out, host_out, compute, barrier, max_over_ranks):
+    """End-to-end steps through the public API with host buffers: every step copies its inputs from
+    pinned host memory (host_in) into device buffer set i % 2 on a host-to-device stream, computes
+    on the current stream, and copies every output of set i % 2 back to pinned host memory
+    (host_out) on a device-to-host stream.  Events order each buffer set's reuse, so the copies of
+    neighbouring steps overlap the compute.  Returns the device-timed ms per step (max over ranks)
+    measured on the compute stream from before the first copy to after the last."""
+    import torch
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, done, out_read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def run(n):
+        for i in range(n):
+            j = i % 2
+            if i >= 2:
+                s_in.wait_event(done[j])          # compute of step i - 2 has read input set j
+            with torch.cuda.stream(s_in):
+                for t, x in dev_in[j].items():
+                    x.copy_(host_in[t], non_blocking=True)
+                in_ready[j].record(s_in)
+            main.wait_event(in_ready[j])
+            if i >= 2:
+                main.wait_event(out_read[j])      # outputs of step i - 2 have been copied back
+            compute(dev_in[j], dev_out[j])
+            done[j].record(main)
+            s_out.wait_event(done[j])
+            with torch.cuda.stream(s_out):
+                for t, x in dev_out[j].items():
+                    host_out[t].copy_(x, non_blocking=True)
+                out_read[j].record(s_out)
+        for j in range(min(n, 2)):
+            main.wait_event(out_read[j])
+
+    run(2)  # warm-up of the copy paths
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    run(steps)
+    e1.record(main)
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(e0.elapsed_time(e1) / steps)
+
+
+
+def tensor_peak(peaks, peak_src, timed_ms):
+    """The bf16 tensor denominator: the measured burst figure for a region under a second, the
+    sustained (power-capped, seconds-long loop) figure for longer timed regions."""
+    if timed_ms >= 1000.0 and "bf16_tflops_sustained" in peaks:
+        return peaks["bf16_tflops_sustained"], f"{peak_src} bf16_tflops_sustained (timed region {timed_ms:.0f} ms)"
+    return peaks["bf16_tflops"], f"{peak_src} bf16_tflops (burst; timed region {timed_ms:.0f} ms)"
+
+
+def kernel_table(prof, alg, steps, peak):
+    """Per kernel: launches and ms per step, and for the attention kernels their credited TFLOP/s
+    and its fraction of the tensor denominator."""
+    out = {}
+    for n, (c, t) in prof.items():
+        e = {"launches": c, "ms_per_step": t / steps}
+        if n in alg and t > 0:
+            tf = alg[n] * c / (t * 1e-3) / 1e12
+            e.update({"credited_tflops": tf, "frac": tf / peak})
+        out[n] = e
+    return out
+
+
+
 def run_reference(args, rank, world):
     """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
     if rank != 0:
@@ -326,8 +416,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": cfg,
-        "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"each step: {desc}"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(), "cpu_model": cpu_model(),
+                         "kind": "oracle", "sample": f"each step: {desc}"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -441,36 +531,28 @@ def run_nsa(args, rank, world, local_rank):
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
     value = world * flops_step / (ms * 1e-3) / 1e12
 
-    # end to end: pinned host inputs in, all outputs back, every step
+    # end to end: pinned host inputs in, all outputs back, every step (copies on their own streams)
     pin = {t: x.pin_memory() for t, x in host.items()}
     outs = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
     h_out = {n_: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n_, x in outs.items()}
-    d_in = {t: torch.empty_like(x) for t, x in d.items()}
+    dev_in = [d, {t: torch.empty_like(x) for t, x in d.items()}]
+    dev_out = [outs, {n_: torch.empty_like(x) for n_, x in outs.items()}]
     h2d = sum(x.numel() * x.element_size() for x in pin.values())
     d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
-    def e2e_step():
-        for t in d_in:
-            d_in[t].copy_(pin[t], non_blocking=True)
-        step(d_in)
-        for n_, x in outs.items():
-            h_out[n_].copy_(x, non_blocking=True)
+    def e2e_compute(x, o):
+        sa.nsa_selected_fwd(x["q"], x["k"], x["v"], x["topk"], x["cu"], S, w.sel_block, w.mask_mode, w.scale,
+                            out=o["out"], lse=o["lse"], workspace=ws_f)
+        sa.nsa_selected_bwd(x["q"], x["k"], x["v"], o["out"], x["dout"], o["lse"], x["topk"], x["cu"], S,
+                            w.sel_block, w.mask_mode, w.scale, dq=o["dq"], dk=o["dk"], dv=o["dv"], workspace=ws_b)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    e2e_ms = pipelined_e2e(args.steps, pin, dev_in, dev_out, h_out, e2e_compute, barrier, max_over_ranks)
 
     peaks, peak_src = measured_peaks()
-    # forward 4*D per visible pair; dK/dV pass 8*D (S^T, dP^T, dV, dK); dQ pass 6*D (S, dP, dQ)
-    alg = {"nsa_fwd": 4 * w.D * vpairs, "nsa_bwd_dkdv": 8 * w.D * vpairs, "nsa_bwd_dq": 6 * w.D * vpairs}
+    # forward 4*D per visible pair; dK/dV pass 8*D (S^T, dP^T, dV, dK); dQ pass 2*D (dQ; its S and dP
+    # recompute what the dK/dV pass is credited with)
+    alg = {"nsa_fwd": 4 * w.D * vpairs, "nsa_bwd_dkdv": 8 * w.D * vpairs, "nsa_bwd_dq": 2 * w.D * vpairs}
+    peak, peak_desc = tensor_peak(peaks, peak_src, ms * args.steps)
     dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
     roof = None
     if dom in alg:
@@ -479,14 +561,15 @@ def run_nsa(args, rank, world, local_rank):
         achieved = alg[dom] / (avg_ms * 1e-3) / 1e12
         tr = NCU_TRAFFIC.get(dom)
         traffic = tr["bytes"] if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) else None
-        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic, "avg_launch_ms": avg_ms}
-    kernels = {n_: {"launches": c, "ms_per_step": t / args.steps} for n_, (c, t) in prof.items()}
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_desc, "traffic": traffic,
+                "avg_launch_ms": avg_ms, "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    kernels = kernel_table(prof, alg, args.steps, peak)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, t, desc = cpu_oracle_sample_nsa(w, topk, budget_s=args.cpu_seconds)
-        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+               "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps({
             "metric": METRIC_NSA, "value": value, "unit": "TFLOP/s",
@@ -600,7 +683,8 @@ def run_decode(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f_, t_, desc = cpu_oracle_sample_decode(w, budget_s=args.cpu_seconds)
-        cpu = {"value": f_ / t_ / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+        cpu = {"value": f_ / t_ / 1e9, "unit": "GB/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+               "kind": "oracle", "sample": desc}
     peaks, src = measured_peaks()
     value = world * gathered / (ms * 1e-3) / 1e9  # every rank decodes its own copy of the batch
     dec_ms = prof["sfa_decode"][1] / prof["sfa_decode"][0] if "sfa_decode" in prof else None
@@ -682,60 +766,53 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
     value = world * flops_step / (ms * 1e-3) / 1e12
 
-    # ---- end to end through the public API with host buffers (pinned), copies timed
+    # ---- end to end through the public API with host buffers (pinned), copies timed, each on its
+    # own stream and double-buffered against the compute
     pin = {t: host[t].pin_memory() for t in host}
-    pin_mask = torch.from_numpy(mask).pin_memory()
-    h_out = {n: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n, x in
-             (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
-    d_in = {t: torch.empty_like(x) for t, x in (("q", q), ("k", k), ("v", v), ("dout", do))}
-    d_mask = torch.empty_like(dmask)
-    h2d = sum(x.numel() * x.element_size() for x in pin.values()) + pin_mask.numel()
+    pin["mask"] = torch.from_numpy(mask).pin_memory()
+    outs = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    h_out = {n: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n, x in outs.items()}
+    d0 = {"q": q, "k": k, "v": v, "dout": do, "mask": dmask}
+    dev_in = [d0, {t: torch.empty_like(x) for t, x in d0.items()}]
+    dev_out = [outs, {n: torch.empty_like(x) for n, x in outs.items()}]
+    h2d = sum(x.numel() * x.element_size() for x in pin.values())
     d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
-    def e2e_step():
-        for t in d_in:
-            d_in[t].copy_(pin[t], non_blocking=True)
-        d_mask.copy_(pin_mask, non_blocking=True)
-        step(d_in["q"], d_in["k"], d_in["v"], d_in["dout"], d_mask)
-        for n, x in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-            h_out[n].copy_(x, non_blocking=True)
+    def e2e_compute(x, o):
+        sa.bsa_fwd(x["q"], x["k"], x["v"], x["mask"], bx, by, w.mask_mode, w.scale, out=o["out"], lse=o["lse"],
+                   workspace=ws_f)
+        sa.bsa_bwd(x["q"], x["k"], x["v"], o["out"], x["dout"], o["lse"], x["mask"], bx, by, w.mask_mode, w.scale,
+                   dq=o["dq"], dk=o["dk"], dv=o["dv"], workspace=ws_b)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    e2e_ms = pipelined_e2e(args.steps, pin, dev_in, dev_out, h_out, e2e_compute, barrier, max_over_ranks)
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = measured_peaks()
-    alg = {"bsa_fwd": 4 * w.D * vpairs, "bsa_bwd_kv": 8 * w.D * vpairs, "bsa_bwd_q": 6 * w.D * vpairs}
+    # forward 4*D per visible pair (S, O); KV-major pass 8*D (S^T, dP^T, dV, dK); Q-major pass 2*D (dQ;
+    # its S and dP recompute what the KV pass is credited with): 14*D in all
+    alg = {"bsa_fwd": 4 * w.D * vpairs, "bsa_bwd_kv": 8 * w.D * vpairs, "bsa_bwd_q": 2 * w.D * vpairs}
+    peak, peak_desc = tensor_peak(peaks, peak_src, ms * args.steps)
     dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
     roof = None
     if dom in alg:
         launches, total = prof[dom]
         avg_ms = total / launches
         achieved = alg[dom] / (avg_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
         traffic = None
         tr = NCU_TRAFFIC.get(dom)
         if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config:
             traffic = tr["bytes"]
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic,
-                "avg_launch_ms": avg_ms}
-    kernels = {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in prof.items()}
+                "frac": achieved / peak, "peak_source": peak_desc, "traffic": traffic, "avg_launch_ms": avg_ms,
+                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    kernels = kernel_table(prof, alg, args.steps, peak)
     launches_total = sum(c for c, _ in prof.values())
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, t, desc = cpu_oracle_sample(w, mask, budget_s=args.cpu_seconds)
-        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+               "kind": "oracle", "sample": desc}
 
     if rank == 0:
         line = {
@@ -761,7 +838,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -6,7 +6,7 @@
 // next unit's Q load and first score tiles overlap the current unit's epilogue.  Every unit is
 // computed whole by one CTA in list order, so results do not depend on the assignment.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads: 11 warps):
 //   warps 0-7  softmax: warp w reads TMEM lane quarter w % 4 (query rows 32*(w%4) .. +31) and the
 //              column half w / 4 of each S tile, so each row is shared by two threads that
 //              exchange their partial row max through shared memory.  They mask, keep the
@@ -15,7 +15,7 @@
 //              unit's Out and LSE.
 //   warp 8     scheduler and TMA producer: takes the next unit, hands it to the other warps
 //              through a small ring in shared memory, then loads Q (once the previous unit's
-//              last S has read the old Q), the K tiles into a 3-stage ring and the V tiles into
+//              last S has read the old Q), the K tiles into a 2-stage ring and the V tiles into
 //              a 2-stage ring.  A K stage is released when its S = Q K^T has run, a V stage
 //              after its O += P V.
 //   warp 9     issues O += P_j V_j into the TMEM O accumulator as soon as P_j is ready.
