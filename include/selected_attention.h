@@ -192,22 +192,36 @@ BSA_API bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const v
  *   BSA_META_NSA_TOKENS also, per (b, g, kb) row (kb < ceil(S_q / sel_block_size)), the
  *                       ascending global token indices whose list holds kb, each token once:
  *                       int32 row_ptr[B*N2*nblk+1] and col[...].
- *   BSA_META_SFA_PAGES  int32 pages[B, N2, sparse_count * sparse_block_size / page_size].
+ *   BSA_META_SFA_PAGES  int32 pages[B, N2, cap] (compacted: the physical pages of the selected
+ *                       sparse blocks in list order, empty slots and pages past seqused_kv
+ *                       dropped; cap = sparse_count * sparse_block_size / page_size), tokens[B, N2,
+ *                       cap] (tokens in use of each listed page) and count[B, N2].
+ *   BSA_META_SFA_WORK   the sparse decode's split of its work (SparseAttnSharedkvMetadata page:
+ *                       each core's share of the task list): unit u = (b * N2 + g) * HH + head half
+ *                       (HH = 2 when N1 / N2 > 64, else 1) is cut into P pieces, piece u * P + p
+ *                       taking pages [floor(p n / P), floor((p + 1) n / P)) of the unit's n.  Per
+ *                       piece: int32 pages[pieces][cap] and tokens[pieces][cap] (the unit's
+ *                       compacted list, as BSA_META_SFA_PAGES) and rec[pieces][3] = (n, begin,
+ *                       len); layout.info[0] = pieces, info[1] = P.  The decode runs this same
+ *                       code in its prologue; P = min(4, max(1, SMs / units)).
  * The plan layout for each op is given by sparse_attn_metadata_layout(). */
 typedef enum {
   BSA_META_BSA_KV = 0,
   BSA_META_BSA_Q = 1,
   BSA_META_NSA_KV = 2,
   BSA_META_NSA_TOKENS = 3,
-  BSA_META_SFA_PAGES = 4
+  BSA_META_SFA_PAGES = 4,
+  BSA_META_SFA_WORK = 5
 } bsa_meta_op;
 
 /* Offsets (bytes from `plan`) of the arrays an op writes: offsets[0] = status word,
- * offsets[1..4] = op-specific arrays (see bsa_meta_op), count = number used. */
+ * offsets[1..4] = op-specific arrays (see bsa_meta_op), count = number used; info = op-specific
+ * sizes (BSA_META_SFA_WORK: pieces, pieces per unit), zero otherwise. */
 typedef struct bsa_meta_layout {
   size_t total_bytes;
   size_t offsets[6];
   int32_t count;
+  size_t info[2];
 } bsa_meta_layout;
 
 BSA_API bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta_layout* layout);
@@ -232,6 +246,14 @@ typedef struct bsa_kernel_time {
 } bsa_kernel_time;
 BSA_API bsa_status bsa_profile_enable(int32_t on);
 BSA_API bsa_status bsa_profile_collect(bsa_kernel_time* out, int32_t max_entries, int32_t* n_entries);
+
+/* Schedule record (for benchmarks; off by default).  With dev_buf set (a caller-owned device
+ * array of 3 * capacity * 2 uint64), every later launch of the three persistent block-sparse
+ * kernels writes, per CTA c < capacity, its start and finish time in ns (the GPU's global timer)
+ * to dev_buf[(slot * capacity + c) * 2 + {0, 1}], slot 0 = forward, 1 = KV-major backward pass,
+ * 2 = Q-major backward pass; each launch overwrites its slot.  Launches with more CTAs than
+ * capacity write nothing.  dev_buf = NULL stops recording.  Not part of the pages' operations. */
+BSA_API bsa_status bsa_profile_cta_clock(uint64_t* dev_buf, int32_t capacity);
 
 /* Library version string. */
 BSA_API const char* bsa_version(void);

@@ -138,3 +138,25 @@ def work_cuts(weights: np.ndarray, n_parts: int) -> np.ndarray:
     total weight W, so cut[s] = ceil(s * W / n_parts)."""
     W = int(np.sum(weights))
     return np.array([-(-(s * W) // n_parts) for s in range(n_parts + 1)], dtype=np.int64)
+
+
+def sfa_pieces_per_unit(units: int, sms: int, max_pieces: int = 4) -> int:
+    """Pieces per decode unit: as many as one wave of the GPU's SMs allows, at most `max_pieces`
+    (the pieces of a unit merge their partial results inside one thread-block cluster)."""
+    return min(max_pieces, max(1, sms // max(units, 1)))
+
+
+def sfa_pieces(count: np.ndarray, HH: int, P: int):
+    """Split of the sparse decode's work (SparseAttnSharedkvMetadata page: each core gets the start
+    and end of its share of the task list).  count [B*N2]: compacted pages per (b, kv head); a unit
+    u = bg * HH + head half shares its (b, kv head)'s list.  Unit u's n pages are cut into P
+    consecutive pieces; piece u * P + p gets pages [floor(p n / P), floor((p + 1) n / P)).
+    Returns int32 [units * P, 3] = (n, begin, len)."""
+    units = len(count) * HH
+    rec = np.zeros((units * P, 3), dtype=np.int32)
+    for u in range(units):
+        n = int(count[u // HH])
+        for p in range(P):
+            b0, b1 = (p * n) // P, ((p + 1) * n) // P
+            rec[u * P + p] = (n, b0, b1 - b0)
+    return rec

@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_NULLPTR", 2: "BSA_ERR_INVALID_ARG", 3: 
                 4: "BSA_ERR_WORKSPACE_TOO_SMALL", 5: "BSA_ERR_CUDA"}
 LAYOUT_BNSD, LAYOUT_TND, LAYOUT_BSND, LAYOUT_PA_ND = 0, 1, 2, 3
 MASK_NONE, MASK_CAUSAL, MASK_RIGHT_DOWN_CAUSAL, MASK_BAND = 0, 2, 3, 4
-META_BSA_KV, META_BSA_Q, META_NSA_KV, META_NSA_TOKENS, META_SFA_PAGES = range(5)
+META_BSA_KV, META_BSA_Q, META_NSA_KV, META_NSA_TOKENS, META_SFA_PAGES, META_SFA_WORK = range(6)
 DEV_BAD_INDEX, DEV_BAD_SEQLEN, DEV_TIMEOUT = 1, 2, 4
 
 EXPORTED = [
@@ -30,7 +30,7 @@ EXPORTED = [
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
     "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_fwd_noalloc_get_status", "bsa_diag_exp2",
-    "bsa_diag_wait",
+    "bsa_diag_wait", "bsa_profile_cta_clock",
 ]
 
 
@@ -67,7 +67,8 @@ class KernelTime(ctypes.Structure):
 
 
 class MetaLayout(ctypes.Structure):
-    _fields_ = [("total_bytes", ctypes.c_size_t), ("offsets", ctypes.c_size_t * 6), ("count", ctypes.c_int32)]
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("offsets", ctypes.c_size_t * 6), ("count", ctypes.c_int32),
+                ("info", ctypes.c_size_t * 2)]
 
 
 _lib = None
@@ -99,6 +100,7 @@ def lib() -> ctypes.CDLL:
         L.bsa_diag_exp2.argtypes = [vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
         L.bsa_diag_wait.argtypes = [vp, ctypes.c_int32, vp]
         L.bsa_profile_enable.argtypes = [ctypes.c_int32]
+        L.bsa_profile_cta_clock.argtypes = [vp, ctypes.c_int32]
         L.bsa_profile_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
         L.bsa_version.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -372,6 +374,18 @@ def bsa_get_status(workspace, stream=None) -> int:
 def bsa_profile_enable(on: bool = True) -> None:
     """Start (or stop) timing every kernel launch the library makes."""
     _check("bsa_profile_enable", lib().bsa_profile_enable(1 if on else 0))
+
+
+def bsa_profile_cta_clock(buf=None) -> None:
+    """Record per-CTA start / finish times of the persistent block-sparse kernels into `buf`, a
+    CUDA int64 tensor [3, capacity, 2] (slot 0 forward, 1 KV-major pass, 2 Q-major pass); None
+    stops recording."""
+    if buf is None:
+        _check("bsa_profile_cta_clock", lib().bsa_profile_cta_clock(None, 0))
+        return
+    _need_cuda(buf)
+    assert buf.dtype == torch.int64 and buf.dim() == 3 and buf.shape[0] == 3 and buf.shape[2] == 2
+    _check("bsa_profile_cta_clock", lib().bsa_profile_cta_clock(_ptr(buf), buf.shape[1]))
 
 
 def bsa_profile_collect() -> dict:

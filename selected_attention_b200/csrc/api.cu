@@ -189,11 +189,14 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
+// Decode workspace: per piece, the unit's compacted page list (pages, tokens; K * ppb entries
+// each) and its set-up record (n, begin, len).  The metadata op BSA_META_SFA_WORK fills the same
+// arrays with the same device code.
 struct SfaWs {
   uint32_t* status;
-  int32_t *pages, *tokens, *count, *piece_unit, *piece_begin, *piece_len, *unit_first, *unit_pieces, *n_pieces;
-  float *part_o, *part_m, *part_l;
-  int cap, per, units, max_pieces;
+  int32_t *pages, *tokens, *rec;
+  int cap, per, units, P, pieces;
+  size_t off_pages, off_tokens, off_rec;
 };
 
 size_t carve_sfa(const bsa_params* p, void* ws, SfaWs* w) {
@@ -202,22 +205,26 @@ size_t carve_sfa(const bsa_params* p, void* ws, SfaWs* w) {
   w->cap = p->sparse_count * ppb;
   w->per = sfa_head_halves(p->N1 / p->N2);
   w->units = p->B * p->N2 * w->per;
-  w->max_pieces = sm_count() + w->units;
-  const size_t lists = static_cast<size_t>(p->B) * p->N2 * w->cap;
+  w->P = sfa_pieces_per_unit(w->units, sm_count());
+  w->pieces = w->units * w->P;
   w->status = static_cast<uint32_t*>(ws);
-  w->pages = c.take<int32_t>(lists);
-  w->tokens = c.take<int32_t>(lists);
-  w->count = c.take<int32_t>(static_cast<size_t>(p->B) * p->N2);
-  w->piece_unit = c.take<int32_t>(w->max_pieces);
-  w->piece_begin = c.take<int32_t>(w->max_pieces);
-  w->piece_len = c.take<int32_t>(w->max_pieces);
-  w->unit_first = c.take<int32_t>(w->units);
-  w->unit_pieces = c.take<int32_t>(w->units);
-  w->n_pieces = c.take<int32_t>(1);
-  w->part_o = c.take<float>(static_cast<size_t>(w->max_pieces) * 64 * 512);  // [piece][64 heads][Dv]
-  w->part_m = c.take<float>(static_cast<size_t>(w->max_pieces) * 64);
-  w->part_l = c.take<float>(static_cast<size_t>(w->max_pieces) * 64);
+  w->off_pages = c.next();
+  w->pages = c.take<int32_t>(static_cast<size_t>(w->pieces) * w->cap);
+  w->off_tokens = c.next();
+  w->tokens = c.take<int32_t>(static_cast<size_t>(w->pieces) * w->cap);
+  w->off_rec = c.next();
+  w->rec = c.take<int32_t>(static_cast<size_t>(w->pieces) * 3);
   return c.bytes();
+}
+
+SfaMetaArgs sfa_meta_args(const bsa_params* p) {
+  SfaMetaArgs m;
+  m.sparse_indices = p->sparse_indices; m.block_table = p->block_table; m.seqused_kv = p->seqused_kv;
+  m.B = p->B; m.N2 = p->N2; m.K = p->sparse_count; m.ppb = p->sparse_block_size / p->page_size;
+  m.page_size = p->page_size; m.max_pages_per_seq = p->max_pages_per_seq; m.num_pages = p->num_pages;
+  m.pages = m.tokens = m.count = nullptr;
+  m.status = nullptr;
+  return m;
 }
 
 bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
@@ -383,22 +390,14 @@ bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_r
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
-  SfaMetaArgs m;
-  m.sparse_indices = p->sparse_indices; m.block_table = p->block_table; m.seqused_kv = p->seqused_kv;
-  m.B = p->B; m.N2 = p->N2; m.K = p->sparse_count; m.ppb = p->sparse_block_size / p->page_size;
-  m.page_size = p->page_size; m.max_pages_per_seq = p->max_pages_per_seq; m.num_pages = p->num_pages;
-  m.pages = w.pages; m.tokens = w.tokens; m.count = w.count; m.status = w.status;
-  if ((e = sfa_page_list(m, st)) != cudaSuccess) return BSA_ERR_CUDA;
-  if ((e = sfa_work_list(w.count, w.units, w.per, w.max_pieces - w.units, w.piece_unit, w.piece_begin,
-                         w.piece_len, w.unit_first, w.unit_pieces, w.n_pieces, st)) != cudaSuccess)
-    return BSA_ERR_CUDA;
   SfaDecodeArgs a;
-  a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.page_size = p->page_size; a.num_pages = p->num_pages;
-  a.cap = w.cap; a.units = w.units; a.max_pieces = w.max_pieces; a.scale = p->scale;
+  a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.K = p->sparse_count; a.ppb = p->sparse_block_size / p->page_size;
+  a.page_size = p->page_size; a.max_pages_per_seq = p->max_pages_per_seq; a.num_pages = p->num_pages;
+  a.units = w.units; a.P = w.P; a.scale = p->scale;
   a.q = q; a.q_rope = q_rope; a.k_cache = k_cache; a.k_rope_cache = k_rope_cache; a.v_cache = v_cache;
-  a.pages = w.pages; a.tokens = w.tokens; a.piece_unit = w.piece_unit; a.piece_begin = w.piece_begin;
-  a.piece_len = w.piece_len; a.unit_first = w.unit_first; a.unit_pieces = w.unit_pieces; a.n_pieces = w.n_pieces;
-  a.out = out; a.lse = lse; a.part_o = w.part_o; a.part_m = w.part_m; a.part_l = w.part_l; a.status = w.status;
+  a.sparse_indices = p->sparse_indices; a.block_table = p->block_table; a.seqused_kv = p->seqused_kv;
+  a.pages = w.pages; a.tokens = w.tokens; a.rec = w.rec;
+  a.out = out; a.lse = lse; a.status = w.status;
   return cuda_status(sfa_decode_launch(a, st));
 }
 
@@ -466,6 +465,20 @@ bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta
     layout->total_bytes = c.bytes();
     return BSA_OK;
   }
+  if (op == BSA_META_SFA_WORK) {
+    bsa_status s = check_sfa(p);
+    if (s != BSA_OK) return s;
+    SfaWs w;
+    layout->total_bytes = carve_sfa(p, nullptr, &w);
+    layout->offsets[0] = 0;
+    layout->offsets[1] = w.off_pages;   // pages [pieces][cap]
+    layout->offsets[2] = w.off_tokens;  // tokens [pieces][cap]
+    layout->offsets[3] = w.off_rec;     // (n, begin, len) [pieces][3]
+    layout->count = 4;
+    layout->info[0] = static_cast<size_t>(w.pieces);
+    layout->info[1] = static_cast<size_t>(w.P);
+    return BSA_OK;
+  }
   return BSA_ERR_UNSUPPORTED;
 }
 
@@ -483,18 +496,20 @@ bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, siz
     carve_nsa(p, plan, &w, op == BSA_META_NSA_TOKENS);
     return cuda_status(nsa_metadata(nsa_meta_args(p, w, op == BSA_META_NSA_TOKENS), st));
   }
-  if (op == BSA_META_SFA_PAGES) {
+  if (op == BSA_META_SFA_PAGES || op == BSA_META_SFA_WORK) {
     if (!p->block_table || !p->sparse_indices || !p->seqused_kv) return BSA_ERR_NULLPTR;
     if (cudaMemsetAsync(plan, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
-    SfaMetaArgs m;
-    m.sparse_indices = p->sparse_indices; m.block_table = p->block_table; m.seqused_kv = p->seqused_kv;
-    m.B = p->B; m.N2 = p->N2; m.K = p->sparse_count; m.ppb = p->sparse_block_size / p->page_size;
-    m.page_size = p->page_size; m.max_pages_per_seq = p->max_pages_per_seq; m.num_pages = p->num_pages;
+    SfaMetaArgs m = sfa_meta_args(p);
+    m.status = static_cast<uint32_t*>(plan);
     m.pages = reinterpret_cast<int32_t*>(base + L.offsets[1]);
     m.tokens = reinterpret_cast<int32_t*>(base + L.offsets[2]);
-    m.count = reinterpret_cast<int32_t*>(base + L.offsets[3]);
-    m.status = static_cast<uint32_t*>(plan);
-    return cuda_status(sfa_page_list(m, st));
+    if (op == BSA_META_SFA_PAGES) {
+      m.count = reinterpret_cast<int32_t*>(base + L.offsets[3]);
+      return cuda_status(sfa_page_list(m, st));
+    }
+    SfaWs w;
+    carve_sfa(p, nullptr, &w);
+    return cuda_status(sfa_pieces(m, w.P, w.per, w.pieces, reinterpret_cast<int32_t*>(base + L.offsets[3]), st));
   }
   if (!p->block_mask) return BSA_ERR_NULLPTR;
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);

@@ -31,6 +31,10 @@ struct Carver {
 // ---- kernel timing (profile.cu): brackets a launch with events when timing is enabled ----------
 void prof_begin(const char* name, cudaStream_t st);
 void prof_end(cudaStream_t st);
+// Per-CTA start / finish record of the persistent block-sparse kernels (slot 0 bsa_fwd, 1
+// bsa_bwd_kv, 2 bsa_bwd_q): the device array to write for a launch of `grid` CTAs, or nullptr
+// when recording is off or the caller's buffer is too small.
+uint64_t* prof_cta_clock(int slot, int grid);
 
 // ---- metadata (metadata.cu) -------------------------------------------------------------------
 // BSA KV lists: units (b, h, qb) -> ascending kv block ids.
@@ -104,20 +108,23 @@ struct SfaMetaArgs {
   uint32_t* status;
 };
 cudaError_t sfa_page_list(const SfaMetaArgs& a, cudaStream_t st);
-// units (b, g, head half), `per` head halves per (b, g); G = CTAs of one wave
-cudaError_t sfa_work_list(const int32_t* count, int units, int per, int G, int32_t* piece_unit,
-                          int32_t* piece_begin, int32_t* piece_len, int32_t* unit_first, int32_t* unit_pieces,
-                          int32_t* n_pieces, cudaStream_t st);
+// Decode pieces: unit u = (b * N2 + g) * HH + head half is cut into P pieces (P = the cluster size
+// of the decode launch); piece u * P + p takes pages [floor(p n / P), floor((p + 1) n / P)) of the
+// unit's n.  sfa_pieces runs the decode prologue's set-up for every piece: a.pages / a.tokens are
+// [n_pieces][K * ppb] regions, rec is int32 [n_pieces][3] = (n, begin, len).
+constexpr int kSfaMaxPieces = 4;
+int sfa_pieces_per_unit(int units, int sms);
+cudaError_t sfa_pieces(const SfaMetaArgs& a, int P, int HH, int n_pieces, int32_t* rec, cudaStream_t st);
 // head halves of 64 per kv head: 2 when the group has more than 64 query heads
 int sfa_head_halves(int G);
 struct SfaDecodeArgs {
-  int B, N1, N2, page_size, num_pages, cap, units, max_pieces;
+  int B, N1, N2, K, ppb, page_size, max_pages_per_seq, num_pages, units, P;
   float scale;
   const void *q, *q_rope, *k_cache, *k_rope_cache, *v_cache;
-  const int32_t *pages, *tokens, *piece_unit, *piece_begin, *piece_len, *unit_first, *unit_pieces, *n_pieces;
+  const int32_t *sparse_indices, *block_table, *seqused_kv;
+  int32_t *pages, *tokens, *rec;  // per-piece regions, as for sfa_pieces
   void* out;
   float* lse;
-  float *part_o, *part_m, *part_l;
   uint32_t* status;
 };
 cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st);

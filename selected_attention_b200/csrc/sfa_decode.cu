@@ -1,14 +1,16 @@
 // Sparse flash attention decode over a paged KV cache (SparseFlashAttention page, formula):
 //   Out = softmax((q k~^T + q_rope k_rope~^T) * scale) v~,  D = Dv = 512, Dr = 64, q_len = 1
-// where k~ / v~ are the tokens of the selected sparse blocks (sfa_meta.cu turns them into page
-// lists and a work list of pieces).
+// where k~ / v~ are the tokens of the selected sparse blocks.
 //
 // The query side of a decode step is small (the G = N1/N2 heads of one kv head, one row each) and
 // the key side long, so the products are taken transposed, with the tokens as the MMA's M = 128
 // rows and the heads as N:
 //   S^T [128 tokens][64 heads]  = K~ [128][576] . Q^T          (Q of 64 heads stays in shared memory)
 //   O^T [512 dv][64 heads]     += V~^T [512][128] . P^T [128][64] (four M = 128 tiles of dv)
-// One CTA per piece: a run of pages of one unit (batch, kv head, half of the G heads).  O^T takes
+// A unit is (batch, kv head, half of the G heads).  Its compacted page list (sfa_pages.cuh, the
+// code the metadata op runs too) is built in the kernel's prologue while Q is loaded, and its n
+// pages are split evenly over P pieces (P = the thread-block cluster size, up to 4): piece p takes
+// pages [floor(p n / P), floor((p + 1) n / P)).  One CTA per piece.  O^T takes
 // 256 TMEM columns and the two S^T buffers 128, so every head of the CTA keeps all 512 dv columns
 // and S is computed once per head.  K streams through a ring of [128 tokens][64 dims] slots and V
 // through a ring of [2 x 64 dv][64 tokens] slots, each ring with its own producer and consumer.
@@ -23,13 +25,17 @@
 // Per-thread partial sums l are reduced over the tokens once, in the epilogue.
 //
 // Warps: 0-7 softmax (lane quarter = TMEM lanes, warp >> 2 = head half of 32), 8 K producer,
-// 9 V producer, 10 issues S^T, 11 issues O^T += V^T P^T.  A piece covering a whole unit writes
-// Out and LSE; otherwise it writes (O, m, l) partials that sfa_combine merges in piece order.
+// 9 V producer, 10 builds the page list then issues S^T, 11 issues O^T += V^T P^T (and first zeroes
+// the V rows of a partly used page past its tokens in use: those rows get weight 0, but a
+// non-finite value there would still turn 0 * x into NaN).  With P = 1 the CTA writes Out and LSE;
+// otherwise the P CTAs of a cluster leave their (O, m, l) in shared memory and each merges a
+// 512 / P slice of the head dim from all of them over distributed shared memory, in rank order.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "internal.h"
 #include "sa_common.cuh"
+#include "sfa_pages.cuh"
 
 namespace sa {
 namespace {
@@ -60,26 +66,50 @@ struct __align__(1024) DecSmem {
   uint64_t bar_q, bar_k[kKR], bar_k_empty[kKR], bar_v[kVR], bar_v_empty[kVR];
   uint64_t bar_s_full[2], bar_s_free[2], bar_p_full[2], bar_pv_done[2];
   uint64_t bar_x[2];  // per head half: maxima (one phase per tile), then the sums
+  float cl_m[kHeads], cl_l[kHeads];        // this piece's running max (log2 units) and sum per head
+  float cl_w[kHeads][kSfaMaxPieces];       // merge weights of the cluster's pieces per head
+  int32_t setup[3];                        // n, begin, len of this piece
   uint32_t tmem_base;
 };
 
 struct DecParams {
-  int B, N1, N2, G, HH, page_size, cap, sub_rows;
+  int B, N1, N2, G, HH, P, K, ppb, page_size, max_pages_per_seq, num_pages, cap, sub_rows;
   float scale_log2;
-  const int32_t* pages;
-  const int32_t* tokens;
-  const int32_t* piece_unit;
-  const int32_t* piece_begin;
-  const int32_t* piece_len;
-  const int32_t* unit_pieces;
-  const int32_t* n_pieces;
+  const int32_t* sparse_indices;
+  const int32_t* block_table;
+  const int32_t* seqused_kv;
+  int32_t* pages;   // [piece][cap]: the unit's compacted page list, built by the piece itself
+  int32_t* tokens;  // [piece][cap]: tokens in use of each listed page
+  int32_t* rec;     // [piece][3]: n, begin, len
   __nv_bfloat16* out;
   float* lse;
-  float* part_o;  // [piece][64 heads][512]
-  float* part_m;  // [piece][64]
-  float* part_l;
   uint32_t* status;
 };
+
+// ---- thread-block cluster: distributed shared memory and the cluster barrier --------------------
+__device__ __forceinline__ uint32_t cluster_map(const void* p, int rank) {  // own smem -> rank's copy
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+// Every thread of every CTA of the cluster: shared-memory writes before it are visible to the
+// cluster's reads after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 __device__ __forceinline__ float warp_max(float v) {
   float r;
@@ -112,25 +142,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     sfa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
                       const __grid_constant__ CUtensorMap tm_v, const DecParams prm) {
-  griddep_launch_dependents();  // the combine may launch now; it waits for this grid's results
-  griddep_wait();               // launched early: the work list must be complete
-  const int piece = blockIdx.x;
-  if (piece >= *prm.n_pieces) return;  // uniform for the whole CTA
+  griddep_launch_dependents();
+  griddep_wait();  // launched early (programmatic dependent launch): the inputs must be complete
+  const int piece = blockIdx.x;  // unit * P + its rank in the cluster
   extern __shared__ uint8_t smem_raw[];
   DecSmem& s = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int u = prm.piece_unit[piece];
+  const int u = piece / prm.P, rank = piece % prm.P;
   const int bg = u / prm.HH, hh = u % prm.HH;
   const int b = bg / prm.N2, g = bg % prm.N2;
-  const int pbeg = prm.piece_begin[piece];
-  const int npages = prm.piece_len[piece];
-  const int sub = prm.sub_rows;             // tokens per TMA box (32 or 64, divides the page)
-  const int spp = prm.page_size / sub;      // boxes per page
-  const int n_sub = kTok / sub;             // boxes per tile
-  const int n_chunks = npages * spp;
-  const int n_tiles = (n_chunks + n_sub - 1) / n_sub;
-  const int32_t* plist = prm.pages + static_cast<size_t>(bg) * prm.cap + pbeg;
-  const int32_t* tlist = prm.tokens + static_cast<size_t>(bg) * prm.cap + pbeg;
   const int head0 = hh * kHeads;                       // first head of this CTA within the group
   const int nh = min(kHeads, prm.G - head0);           // heads of the group this CTA owns
   const int qrow0 = b * prm.N1 + g * prm.G + head0;    // their first query row
@@ -162,6 +182,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  // Q does not depend on the page list: its load overlaps the list's construction
+  if (warp == kSmWarps && lane == 0) {
+    mbar_arrive_expect_tx(&s.bar_q, kKChunks * kHeads * 128);
+    for (int c = 0; c < 8; ++c) tma_load_2d(s.q[c], &tm_q, &s.bar_q, c * 64, qrow0);
+    tma_load_2d(s.q[8], &tm_qr, &s.bar_q, 0, qrow0);
+  }
+  if (warp == kSmWarps + 2) {
+    int n, begin, len;
+    sfa_piece_setup(piece, prm.P, prm.HH, prm.N2, prm.K, prm.ppb, prm.page_size, prm.max_pages_per_seq,
+                    prm.num_pages, prm.sparse_indices, prm.block_table, prm.seqused_kv,
+                    prm.pages + static_cast<size_t>(piece) * prm.cap, prm.tokens + static_cast<size_t>(piece) * prm.cap,
+                    &n, &begin, &len, prm.status);
+    if (lane == 0) {
+      s.setup[0] = n;
+      s.setup[1] = begin;
+      s.setup[2] = len;
+      prm.rec[3 * piece] = n;
+      prm.rec[3 * piece + 1] = begin;
+      prm.rec[3 * piece + 2] = len;
+    }
+  }
+  __syncthreads();  // the page list (global, written by this CTA) and the piece's range are ready
+  const int pbeg = s.setup[1];
+  const int npages = s.setup[2];
+  const int sub = prm.sub_rows;             // tokens per TMA box (32 or 64, divides the page)
+  const int spp = prm.page_size / sub;      // boxes per page
+  const int n_sub = kTok / sub;             // boxes per tile
+  const int n_chunks = npages * spp;
+  const int n_tiles = (n_chunks + n_sub - 1) / n_sub;
+  const int32_t* plist = prm.pages + static_cast<size_t>(piece) * prm.cap + pbeg;
+  const int32_t* tlist = prm.tokens + static_cast<size_t>(piece) * prm.cap + pbeg;
 
   // Box t of tile j: its page-list entry and its token offset inside the page; a box past the
   // piece's end repeats the tile's first box (its rows are masked, and the copy stays in bounds).
@@ -177,11 +228,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool ok = true;
     if (n_tiles > 0) {
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&s.bar_q, kKChunks * kHeads * 128);
-        for (int c = 0; c < 8; ++c) tma_load_2d(s.q[c], &tm_q, &s.bar_q, c * 64, qrow0);
-        tma_load_2d(s.q[8], &tm_qr, &s.bar_q, 0, qrow0);
-      }
       int nxt_page = 0, nxt_off = 0;  // page id (loaded, used next iteration) and token offset
       if (lane < n_sub) {
         const int qb = box_entry(0, lane);
@@ -211,12 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // wait for this CTA's own copies still in flight before it may exit
-      if (lane == 0) {
+      if (lane == 0)
         for (int use = (issued > kKR ? issued - kKR : 0); use < issued; ++use)
           mbar_wait(&s.bar_k[use % kKR], (use / kKR) & 1, prm.status);
-        mbar_wait(&s.bar_q, 0, prm.status);
-      }
     }
+    if (lane == 0) mbar_wait(&s.bar_q, 0, prm.status);
   } else if (warp == kSmWarps + 1) {
     // ------------------------------------------------------------------ V producer
     int issued = 0;
@@ -284,30 +329,87 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kSmWarps + 3) {
     // ------------------------------------------------------------------ O^T issuer
-    if (lane == 0 && n_tiles > 0) {
+    // Lane 0 issues; the warp first zeroes the V rows of a box past its page's tokens in use (the
+    // last page of a sequence, or a box past the piece's end that repeats the tile's first box).
+    if (n_tiles > 0) {
       const uint32_t id_o = idesc_bf16_f32(kTok, kHeads, true, true);
       // A = V^T: MN-major, the two 64-dv chunks of a slot 8 KB apart; B = P^T: MN-major, one chunk
       const uint64_t dv0 = sdesc_sw128(smem_u32(s.v[0]), 64 * 128, 1024);
       const uint64_t dp0 = sdesc_sw128(smem_u32(s.p), kSlot, 1024);
+      const int half_boxes = n_sub / 2;  // boxes per token half of a tile
       bool ok = true;
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j & 1;
+        // rows in use of each box of the tile (lane t < n_sub: box t)
+        int valid = sub;
+        if (lane < n_sub) {
+          const int qb = j * n_sub + lane;
+          valid = qb < n_chunks ? max(0, min(sub, tlist[qb / spp] - (qb % spp) * sub)) : 0;
+        }
+        const uint32_t partial = __ballot_sync(0xffffffffu, lane < n_sub && valid < sub);
+        if (partial == 0) {
+          // every box of the tile is fully in use: lane 0 alone waits and issues
+          if (lane == 0) {
+            ok = mbar_wait(&s.bar_p_full[st], (j >> 1) & 1, prm.status);
+            for (int x = 0; ok && x < kVUses; ++x) {
+              const int mt = x >> 1, th = x & 1;
+              const int use = j * kVUses + x, slot = use % kVR;
+              if (!(ok = mbar_wait(&s.bar_v[slot], (use / kVR) & 1, prm.status))) break;
+              tc_fence_after();
+              const uint64_t dv = sdesc_add(dv0, slot * kSlot);
+              const uint64_t dp = sdesc_add(dp0, th * (64 * 128));
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + kColO + mt * kHeads, sdesc_add(dv, ks * 2048), sdesc_add(dp, ks * 2048), id_o,
+                            (j > 0 || th > 0 || ks > 0) ? 1u : 0u);
+              tc_commit(&s.bar_v_empty[slot]);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (ok && lane == 0) tc_commit(&s.bar_pv_done[st]);
+          continue;
+        }
         // one barrier per tile parity: its next phase needs P_{j+2}, written after this product
-        if (!(ok = mbar_wait(&s.bar_p_full[st], (j >> 1) & 1, prm.status))) break;
+        if (lane == 0) ok = mbar_wait(&s.bar_p_full[st], (j >> 1) & 1, prm.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
         for (int x = 0; x < kVUses; ++x) {
           const int mt = x >> 1, th = x & 1;
           const int use = j * kVUses + x, slot = use % kVR;
-          if (!(ok = mbar_wait(&s.bar_v[slot], (use / kVR) & 1, prm.status))) break;
-          tc_fence_after();
-          const uint64_t dv = sdesc_add(dv0, slot * kSlot);
-          const uint64_t dp = sdesc_add(dp0, th * (64 * 128));
+          if (lane == 0) ok = mbar_wait(&s.bar_v[slot], (use / kVR) & 1, prm.status);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          const uint32_t mine = (partial >> (th * half_boxes)) & ((1u << half_boxes) - 1u);
+          if (mine) {
+            // every lane observes the copy's completion itself before it overwrites part of it
+            ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_v[slot], (use / kVR) & 1, prm.status));
+            if (!ok) break;
+            for (int t = 0; t < half_boxes; ++t) {
+              if (!((mine >> t) & 1u)) continue;
+              const int v0 = __shfl_sync(0xffffffffu, valid, th * half_boxes + t);
+              uint8_t* box = s.v[slot] + t * sub * 128;
+              const int n16 = (sub - v0) * 8;  // 16-byte chunks per 64-dv chunk to clear
+              for (int c = lane; c < 2 * n16; c += 32) {
+                const int chunk = c / n16, e = c % n16;
+                *reinterpret_cast<uint4*>(box + chunk * (64 * 128) + v0 * 128 + e * 16) = make_uint4(0u, 0u, 0u, 0u);
+              }
+            }
+            fence_async_smem();
+            __syncwarp();
+          }
+          if (lane == 0) {
+            tc_fence_after();
+            const uint64_t dv = sdesc_add(dv0, slot * kSlot);
+            const uint64_t dp = sdesc_add(dp0, th * (64 * 128));
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + kColO + mt * kHeads, sdesc_add(dv, ks * 2048), sdesc_add(dp, ks * 2048), id_o,
-                        (j > 0 || th > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(&s.bar_v_empty[slot]);
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16_ss(tmem + kColO + mt * kHeads, sdesc_add(dv, ks * 2048), sdesc_add(dp, ks * 2048), id_o,
+                          (j > 0 || th > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(&s.bar_v_empty[slot]);
+          }
+          __syncwarp();
         }
-        if (ok) tc_commit(&s.bar_pv_done[st]);
+        if (ok && lane == 0) tc_commit(&s.bar_pv_done[st]);
       }
     }
   } else {
@@ -458,99 +560,98 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 1; i < 32; ++i)
       if (lane == i) mh = m[i];
-    const bool single = prm.unit_pieces[u] == 1;
     const bool any = have && L > 0.f;
-    const float inv_l = any ? 1.f / L : 0.f;
     const int hl = hc * 32;  // this warp's first head (of the CTA's 64)
+    if (prm.P == 1) {
+      const float inv_l = any ? 1.f / L : 0.f;
 #pragma unroll 1
-    for (int mt = 0; mt < 4; ++mt) {
-      uint32_t rr[32];
-      if (have) {
-        tmem_ld32(tmem + lane_base + kColO + mt * kHeads + hl, rr);
-        tmem_ld_wait(rr);
-      } else {
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t rr[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + kColO + mt * kHeads + hl, rr);
+          tmem_ld_wait(rr);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) rr[i] = 0u;
-      }
-      const int dv = mt * 128 + r;
-      if (single) {
+          for (int i = 0; i < 32; ++i) rr[i] = 0u;
+        }
+        const int dv = mt * 128 + r;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float sc = __shfl_sync(0xffffffffu, inv_l, i);
           if (hl + i < nh)
             prm.out[static_cast<size_t>(qrow0 + hl + i) * kDQ + dv] = __float2bfloat16_rn(__uint_as_float(rr[i]) * sc);
         }
-      } else {
-        float* dst = prm.part_o + (static_cast<size_t>(piece) * kHeads + hl) * kDQ + dv;
+      }
+      if (quarter == 0 && hl + lane < nh)
+        prm.lse[static_cast<size_t>(qrow0 + hl + lane)] = any ? (mh * kLn2 + logf(L)) : -INFINITY;
+    } else {
+      // O^T (unnormalised) into this CTA's shared memory as [64 heads][512 dv] fp32 over the K and
+      // V rings (all their copies and products have completed); m and l per head beside it
+      float* so = reinterpret_cast<float*>(s.k[0]);
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t rr[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + kColO + mt * kHeads + hl, rr);
+          tmem_ld_wait(rr);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (hl + i < nh) dst[static_cast<size_t>(i) * kDQ] = __uint_as_float(rr[i]);
+          for (int i = 0; i < 32; ++i) rr[i] = 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) so[(hl + i) * kDQ + mt * 128 + r] = __uint_as_float(rr[i]);
+      }
+      if (quarter == 0) {
+        s.cl_m[hl + lane] = any ? mh : -INFINITY;
+        s.cl_l[hl + lane] = any ? L : 0.f;
       }
     }
-    if (quarter == 0 && hl + lane < nh) {
-      const size_t orow = static_cast<size_t>(qrow0 + hl + lane);
-      if (single) {
-        prm.lse[orow] = any ? (mh * kLn2 + logf(L)) : -INFINITY;
-      } else {
-        prm.part_m[static_cast<size_t>(piece) * kHeads + hl + lane] = any ? mh : -INFINITY;
-        prm.part_l[static_cast<size_t>(piece) * kHeads + hl + lane] = have ? L : 0.f;
+  }
+  if (prm.P > 1) {
+    // ---- merge of the cluster's pieces (all threads of every CTA of the cluster take part)
+    const int P = prm.P;
+    cluster_sync_all();
+    if (tid < kHeads) {  // per head: M = max m_q, L = sum l_q 2^(m_q - M), weight 2^(m_q - M) / L
+      float mq[kSfaMaxPieces], lq[kSfaMaxPieces];
+      float M = -INFINITY;
+      for (int q = 0; q < P; ++q) {
+        mq[q] = ld_cluster_f32(cluster_map(&s.cl_m[tid], q));
+        lq[q] = ld_cluster_f32(cluster_map(&s.cl_l[tid], q));
+        M = fmaxf(M, mq[q]);
       }
+      float Lt = 0.f;
+      for (int q = 0; q < P; ++q)
+        if (mq[q] != -INFINITY) Lt += lq[q] * ex2(mq[q] - M);
+      const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+      for (int q = 0; q < P; ++q) s.cl_w[tid][q] = (mq[q] != -INFINITY) ? ex2(mq[q] - M) * inv : 0.f;
+      if (rank == 0 && tid < nh)
+        prm.lse[static_cast<size_t>(qrow0 + tid)] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
     }
+    __syncthreads();
+    // this CTA's slice of the head dim: float4 columns [f0, f1) of the 128 per row
+    const int f0 = rank * (kDQ / 4) / P, f1 = (rank + 1) * (kDQ / 4) / P, nf = f1 - f0;
+    const float* so = reinterpret_cast<const float*>(s.k[0]);
+    for (int idx = tid; idx < nh * nf; idx += kThreads) {
+      const int h = idx / nf, f = f0 + idx % nf;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < P; ++q) {
+        const float w = s.cl_w[h][q];
+        const float4 o = ld_cluster_f32x4(cluster_map(so + h * kDQ + 4 * f, q));
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+      }
+      uint2 pk;
+      pk.x = pack_bf16(acc.x, acc.y);
+      pk.y = pack_bf16(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(prm.out + static_cast<size_t>(qrow0 + h) * kDQ + 4 * f) = pk;
+    }
+    cluster_sync_all();  // no CTA leaves while another still reads its shared memory
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
-}
-
-// Merge the pieces of each unit in piece order:  M = max m_p, L = sum l_p 2^(m_p - M),
-// Out = sum O_p 2^(m_p - M) / L,  LSE = (M + log2 L) ln 2.  One warp per (unit, head); each lane
-// owns 16 of the 512 Dv columns, so every partial row is read with coalesced 16-byte loads.
-__global__ void __launch_bounds__(256) sfa_combine_kernel(const DecParams prm, const int32_t* __restrict__ unit_first) {
-  griddep_wait();  // launched early: the decode pieces must be complete
-  const int u = blockIdx.x;
-  const int hcol = blockIdx.y * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int bg = u / prm.HH, hh = u % prm.HH;
-  const int head = hh * kHeads + hcol;
-  if (hcol >= kHeads || head >= prm.G) return;
-  const int pcs = prm.unit_pieces[u];
-  if (pcs == 1) return;  // written by its single piece
-  const int b = bg / prm.N2, g = bg % prm.N2;
-  const int p0 = unit_first[u];
-  const size_t orow = static_cast<size_t>(b * prm.N1 + g * prm.G + head);
-  __nv_bfloat16* dst = prm.out + orow * kDQ + lane * 16;
-  float M = -INFINITY;
-  for (int p = 0; p < pcs; ++p) M = fmaxf(M, prm.part_m[static_cast<size_t>(p0 + p) * kHeads + hcol]);
-  float L = 0.f, acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int p = 0; p < pcs; ++p) {
-    const float mp = prm.part_m[static_cast<size_t>(p0 + p) * kHeads + hcol];
-    if (mp == -INFINITY) continue;
-    const float wgt = ex2(mp - M);
-    L += prm.part_l[static_cast<size_t>(p0 + p) * kHeads + hcol] * wgt;
-    const float4* src =
-        reinterpret_cast<const float4*>(prm.part_o + (static_cast<size_t>(p0 + p) * kHeads + hcol) * kDQ + lane * 16);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float4 a = src[c];
-      acc[4 * c] += a.x * wgt;
-      acc[4 * c + 1] += a.y * wgt;
-      acc[4 * c + 2] += a.z * wgt;
-      acc[4 * c + 3] += a.w * wgt;
-    }
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;  // pcs == 0 (no selected key): Out = 0, LSE = -inf
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    uint4 pk;
-    pk.x = pack_bf16(acc[8 * c] * inv, acc[8 * c + 1] * inv);
-    pk.y = pack_bf16(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-    pk.z = pack_bf16(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-    pk.w = pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-    *reinterpret_cast<uint4*>(dst + 8 * c) = pk;
-  }
-  if (lane == 0) prm.lse[orow] = L > 0.f ? (M * kLn2 + logf(L)) : -INFINITY;
 }
 
 }  // namespace
@@ -569,22 +670,34 @@ cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st) {
       !make_tmap_3d_bf16(&tv, a.v_cache, kDQ, a.N2, tokens, kDQ, static_cast<uint64_t>(a.N2) * kDQ, 1, sub))
     return cudaErrorInvalidValue;
   DecParams p;
-  p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.G = a.N1 / a.N2; p.HH = sfa_head_halves(p.G);
-  p.page_size = a.page_size; p.cap = a.cap; p.sub_rows = sub;
+  p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.G = a.N1 / a.N2; p.HH = sfa_head_halves(p.G); p.P = a.P;
+  p.K = a.K; p.ppb = a.ppb; p.page_size = a.page_size; p.max_pages_per_seq = a.max_pages_per_seq;
+  p.num_pages = a.num_pages; p.cap = a.K * a.ppb; p.sub_rows = sub;
   p.scale_log2 = a.scale * kLog2e;
-  p.pages = a.pages; p.tokens = a.tokens; p.piece_unit = a.piece_unit; p.piece_begin = a.piece_begin;
-  p.piece_len = a.piece_len; p.unit_pieces = a.unit_pieces; p.n_pieces = a.n_pieces;
-  p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse;
-  p.part_o = a.part_o; p.part_m = a.part_m; p.part_l = a.part_l; p.status = a.status;
+  p.sparse_indices = a.sparse_indices; p.block_table = a.block_table; p.seqused_kv = a.seqused_kv;
+  p.pages = a.pages; p.tokens = a.tokens; p.rec = a.rec;
+  p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse; p.status = a.status;
   const size_t smem = sizeof(DecSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(sfa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  const int grid = a.units * a.P;
+  if (grid == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = a.P;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.P > 1 ? 2 : 1;
   prof_begin("sfa_decode", st);
-  e = launch_pdl(sfa_decode_kernel, dim3(a.max_pieces), dim3(kThreads), smem, st, tq, tqr, tk, tkr, tv, p);
-  prof_end(st);
-  if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
-  prof_begin("sfa_combine", st);
-  e = launch_pdl(sfa_combine_kernel, dim3(a.units, kHeads / 8), dim3(256), 0, st, p, a.unit_first);
+  e = cudaLaunchKernelEx(&cfg, sfa_decode_kernel, tq, tqr, tk, tkr, tv, p);
   prof_end(st);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

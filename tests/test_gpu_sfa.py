@@ -125,3 +125,76 @@ def test_sfa_decode_workload_sampled(cuda_ok):
         assert np.abs(lse[b].cpu().numpy() - r_lse[b]).max() <= LSE_ATOL
     assert np.isfinite(out.float().cpu().numpy()).all()
 
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=3, N1=128, N2=2, page=32, n_logical=24, K=5, sbs=64, seqused=[768, 600, 97]),   # 12 units
+    dict(B=40, N1=64, N2=1, page=64, n_logical=6, K=4, sbs=64, seqused=[384 - 7 * (i % 5) for i in range(40)]),
+    dict(B=80, N1=128, N2=1, page=64, n_logical=6, K=3, sbs=128, seqused=[384 - 50 * (i % 7) for i in range(80)]),
+    dict(B=1, N1=64, N2=1, page=64, n_logical=40, K=19, sbs=64, seqused=[2500]),            # one unit
+])
+def test_sfa_work_split_bit_exact(cuda_ok, case):
+    """The decode's own split of its work (the prologue code, run by the metadata op): per piece
+    the unit's compacted page list and (n, begin, len), against the CPU reference, bit for bit;
+    pieces per unit as one wave of SMs allows (1 to 4 here)."""
+    pb = _problem(**case, seed=31, fill_nan=False)
+    idx = pb["idx"].copy()
+    idx[0, 0, 0, -1] = 10 ** 6  # past the sequence: dropped, flagged
+    tb, ti, tu = (torch.from_numpy(x).cuda() for x in (pb["table"], idx, pb["seqused"]))
+    q = torch.empty(case["B"], 1, case["N1"], 512, device="meta")
+    p = sa.sfa_params(q, pb["dev"]["k"], tb, ti, tu, pb["sbs"])
+    plan, lay = sa.sparse_attn_metadata(p, sa.META_SFA_WORK, "cuda")
+    torch.cuda.synchronize()
+    N2, G = case["N2"], case["N1"] // case["N2"]
+    HH = 2 if G > 64 else 1
+    units = case["B"] * N2 * HH
+    P = M.sfa_pieces_per_unit(units, _sms())
+    assert lay.info[0] == units * P and lay.info[1] == P
+    cap = case["K"] * (pb["sbs"] // pb["page"])
+    pieces = units * P
+    rec = sa.plan_array(plan, lay, 3, pieces * 3).cpu().numpy().reshape(pieces, 3)
+    pages = sa.plan_array(plan, lay, 1, pieces * cap).cpu().numpy().reshape(pieces, cap)
+    tokens = sa.plan_array(plan, lay, 2, pieces * cap).cpu().numpy().reshape(pieces, cap)
+    ref_pages, status = M.sfa_page_lists(idx, pb["table"], pb["seqused"], pb["sbs"], pb["page"])
+    count = (ref_pages >= 0).sum(axis=2).reshape(-1)
+    assert np.array_equal(rec, M.sfa_pieces(count, HH, P))
+    for piece in range(pieces):
+        bg = piece // P // HH
+        b, g = bg // N2, bg % N2
+        want = [int(x) for x in ref_pages[b, g] if x >= 0]
+        n = len(want)
+        assert pages[piece, :n].tolist() == want
+        # tokens in use of each listed page: a full page except where the sequence ends inside it
+        lp = [j * (pb["sbs"] // pb["page"]) + k for j in idx[b, 0, g] if 0 <= j < 10 ** 6
+              for k in range(pb["sbs"] // pb["page"]) if (j * (pb["sbs"] // pb["page"]) + k) * pb["page"] < pb["seqused"][b]]
+        want_tok = [min(pb["page"], int(pb["seqused"][b]) - x * pb["page"]) for x in lp]
+        assert tokens[piece, :n].tolist() == want_tok
+    assert status == M.BAD_INDEX and sa.bsa_get_status(plan) & sa.DEV_BAD_INDEX
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=3, N1=128, N2=1, page=64, n_logical=16, K=6, sbs=64, seqused=[1000, 700, 1023]),   # 4 pieces a unit
+    dict(B=40, N1=64, N2=1, page=64, n_logical=6, K=4, sbs=64, seqused=[377 - 3 * (i % 9) for i in range(40)]),
+    dict(B=80, N1=128, N2=1, page=32, n_logical=8, K=3, sbs=64, seqused=[250 - 9 * (i % 6) for i in range(80)]),
+])
+def test_sfa_decode_nan_past_seqused(cuda_ok, case):
+    """Cache rows past seqused_kv inside the last, partly used page hold NaN (an uninitialised tail,
+    as paged caches leave it): they get weight 0 and must not reach Out.  Pieces per unit from 1
+    to 4 (the cluster merge at 3 and 4 pieces, a single CTA per unit when units exceed the SMs)."""
+    pb = _problem(**case, seed=37)
+    page = pb["page"]
+    for b, used in enumerate(pb["seqused"]):
+        if used % page:
+            phys = int(pb["table"][b, used // page])
+            for name in ("k", "kr", "v"):
+                pb["dev"][name][phys, used % page:] = float("nan")
+    out, lse, r_out, r_lse = _run(pb)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    check_close(got, r_out, "out")
+    fin = np.isfinite(r_lse)
+    assert np.abs(lse.cpu().numpy()[fin] - r_lse[fin]).max() <= LSE_ATOL

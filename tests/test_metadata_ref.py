@@ -94,3 +94,24 @@ def test_work_cuts():
     cuts = M.work_cuts(w, 4)
     assert cuts[0] == 0 and cuts[-1] == w.sum()
     assert np.all(np.diff(cuts) >= 0) and np.max(np.diff(cuts)) - np.min(np.diff(cuts)) <= 1
+
+
+def test_sfa_pieces_cover_each_unit_evenly():
+    """Brute-force properties of the decode split, independent of its formula: the pieces of a
+    unit are consecutive, start at 0, end at n, and their lengths differ by at most one (the
+    most even split of n pages into P runs); units of one (b, kv head) share its count."""
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        bgs, HH, P = int(rng.integers(1, 9)), int(rng.integers(1, 3)), int(rng.integers(1, 5))
+        count = rng.integers(0, 70, size=bgs).astype(np.int32)
+        rec = M.sfa_pieces(count, HH, P)
+        assert rec.shape == (bgs * HH * P, 3)
+        for u in range(bgs * HH):
+            r = rec[u * P:(u + 1) * P]
+            n = int(count[u // HH])
+            assert (r[:, 0] == n).all()
+            assert r[0, 1] == 0 and int(r[-1, 1] + r[-1, 2]) == n
+            assert (r[1:, 1] == r[:-1, 1] + r[:-1, 2]).all()
+            assert r[:, 2].max() - r[:, 2].min() <= 1 and r[:, 2].min() >= 0
+    assert M.sfa_pieces_per_unit(64, 148) == 2 and M.sfa_pieces_per_unit(160, 148) == 1
+    assert M.sfa_pieces_per_unit(40, 148) == 3 and M.sfa_pieces_per_unit(1, 148) == 4
