@@ -383,6 +383,32 @@ def kernel_table(prof, alg, steps, peak):
 
 
 
+def schedule_balance(sa, torch, step, dev, capacity=512):
+    """One extra step with the per-CTA start / finish record on: per persistent kernel, the time
+    from the first CTA's start to the last CTA's finish (span), the spread of the CTAs' finish
+    times, and the idle tail: the fraction of CTA-time (CTAs x span) spent after a CTA finished
+    and before the last one did."""
+    buf = torch.zeros(3, capacity, 2, dtype=torch.int64, device=dev)
+    sa.bsa_profile_cta_clock(buf)
+    step()
+    torch.cuda.synchronize()
+    sa.bsa_profile_cta_clock(None)
+    t = buf.cpu().numpy()
+    out = {}
+    for slot, name in enumerate(("bsa_fwd", "bsa_bwd_kv", "bsa_bwd_q")):
+        rows = t[slot][t[slot][:, 1] > 0]
+        if len(rows) == 0:
+            continue
+        start, end = rows[:, 0], rows[:, 1]
+        span = float(end.max() - start.min())
+        out[name] = {"ctas": int(len(rows)), "span_us": span / 1e3,
+                     "finish_spread_us": float(end.max() - end.min()) / 1e3,
+                     "start_spread_us": float(start.max() - start.min()) / 1e3,
+                     "idle_tail_frac": float((end.max() - end).sum()) / (len(rows) * span) if span > 0 else 0.0}
+    return out
+
+
+
 def run_reference(args, rank, world):
     """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
     if rank != 0:
@@ -765,6 +791,7 @@ def run_ours(args, rank, world, local_rank):
         sa.bsa_profile_enable(False)
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
     value = world * flops_step / (ms * 1e-3) / 1e12
+    sched = schedule_balance(sa, torch, step, dev)  # an extra, untimed step
 
     # ---- end to end through the public API with host buffers (pinned), copies timed, each on its
     # own stream and double-buffered against the compute
@@ -823,6 +850,7 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_total, "kernels": kernels, "roofline": with_spec(roof), "cpu_baseline": cpu,
             "clocks": clocks.summary(), "visible_pairs": vpairs, "credited_flops_per_step": flops_step,
+            "schedule": sched,
         }
         print(json.dumps(line))
 

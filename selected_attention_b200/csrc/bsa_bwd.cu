@@ -88,6 +88,7 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   uint32_t* status;
+  uint64_t* cta_clock;  // optional [grid][2] start / finish times (ns), see bsa_profile_cta_clock
 };
 
 __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&rr)[32], float mul) {
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                       const BwdParams prm) {
   griddep_wait();  // the D / LSE tiles of the preprocess must be complete
   griddep_launch_dependents();  // after the wait: the dQ pass then starts only once its inputs exist
+  if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x] = globaltimer_ns();
   constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   KvSmem& s = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -476,6 +478,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+  if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x + 1] = globaltimer_ns();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -513,6 +516,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                      const BwdParams prm) {
   if (prm.pdl_wait) griddep_wait();
   griddep_launch_dependents();
+  if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x] = globaltimer_ns();
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColDP = 2 * BN, kColDQ = 3 * BN;
   extern __shared__ uint8_t smem_raw[];
   QSmem<BN>& s = *reinterpret_cast<QSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -816,6 +820,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+  if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x + 1] = globaltimer_ns();
 }
 
 template <int BN>
@@ -865,6 +870,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
   p.dk = static_cast<__nv_bfloat16*>(a.dk);
   p.dv = static_cast<__nv_bfloat16*>(a.dv);
   p.status = a.status;
+  p.cta_clock = nullptr;
   // KV-major pass
   {
     BwdParams pk = p;
@@ -881,6 +887,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     const int grid = units < sms ? units : sms;  // persistent: one CTA per SM
     prof_begin("bsa_bwd_kv", st);
     pk.pdl_wait = 1;
+    pk.cta_clock = prof_cta_clock(1, grid);
     if (grid > 0) e = launch_pdl(bsa_bwd_kv_kernel, dim3(grid), dim3(kKvThreads), smem, st, tq64, tk128, tv128, tdo64, pk);
     prof_end(st);
     if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
@@ -899,6 +906,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = q_units < sms ? q_units : sms;
+  p.cta_clock = prof_cta_clock(2, grid);
   if (a.by == 128) return launch_q<128>(p, tq, tk, tv, tdo, grid, st);
   return launch_q<64>(p, tq, tk, tv, tdo, grid, st);
 }

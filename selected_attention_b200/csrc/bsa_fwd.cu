@@ -77,6 +77,7 @@ struct FwdParams {
   float* lse;
   int32_t* next_unit;  // scheduler counter, zero at launch
   uint32_t* status;
+  uint64_t* cta_clock;  // optional [grid][2] start / finish times (ns), see bsa_profile_cta_clock
 };
 
 // Unit number i of the schedule -> (b*N1 + h, q block): head-major, latest q block first.
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams prm) {
   griddep_wait();  // launched with programmatic dependent launch: the KV lists must be complete
+  if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x] = globaltimer_ns();
   griddep_launch_dependents();
   constexpr uint32_t kTmemCols = (2 * BN + kD) <= 256 ? 256 : 512;
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
@@ -476,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x + 1] = globaltimer_ns();
 }
 
 template <int BN>
@@ -497,6 +500,7 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   p.scale_log2 = a.scale * kLog2e;
   p.row_ptr = a.row_ptr; p.col = a.col;
   p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse; p.next_unit = a.next_unit; p.status = a.status;
+  p.cta_clock = nullptr;
   const size_t smem = sizeof(FwdSmem<BN>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -505,6 +509,7 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.units < sms ? p.units : sms;  // persistent: one CTA per SM
+  p.cta_clock = prof_cta_clock(0, grid);
   prof_begin("bsa_fwd", st);
   e = launch_pdl(bsa_fwd_kernel<BN>, dim3(grid), dim3(kThreads), smem, st, tq, tk, tv, to, p);
   prof_end(st);

@@ -25,6 +25,8 @@ std::vector<cudaEvent_t> g_pool;
 size_t g_pool_next = 0;
 std::vector<Rec> g_recs;
 int g_open = -1;
+uint64_t* g_cta_buf = nullptr;  // caller-owned device array [3][g_cta_cap][2]
+int g_cta_cap = 0;
 
 cudaEvent_t take_event() {
   if (g_pool_next == g_pool.size()) {
@@ -54,9 +56,23 @@ void prof_end(cudaStream_t st) {
   g_open = -1;
 }
 
+uint64_t* prof_cta_clock(int slot, int grid) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_cta_buf || grid > g_cta_cap || slot < 0 || slot > 2) return nullptr;
+  return g_cta_buf + static_cast<size_t>(slot) * g_cta_cap * 2;
+}
+
 }  // namespace sa
 
 extern "C" {
+
+bsa_status bsa_profile_cta_clock(uint64_t* dev_buf, int32_t capacity) {
+  if (dev_buf && capacity <= 0) return BSA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(sa::g_mu);
+  sa::g_cta_buf = dev_buf;
+  sa::g_cta_cap = dev_buf ? capacity : 0;
+  return BSA_OK;
+}
 
 bsa_status bsa_profile_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(sa::g_mu);
