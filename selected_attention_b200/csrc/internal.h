@@ -56,10 +56,30 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64
 bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                        uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2);
 
+// 4D bf16 map over (d0 contiguous, d1, d2, d3) with strides in elements, box {64, 1, box2, 1}: a
+// [B][..][..][D] attention tensor seen as (head dim, head, position, batch) whatever the order of
+// head and position in memory (BNSD or BSND).  Rows past d2 read as zero and are not stored.
+bool make_tmap_4d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                       uint64_t stride1, uint64_t stride2, uint64_t stride3, uint32_t box2);
+
+// Element strides of a BSA tensor (b, head, position, d): BNSD [B][N][S][D] or BSND [B][S][N][D];
+// the LSE [b][head][position] is [B][N][S] for BNSD and [B][S][N] for BSND.
+struct BsaStrides {
+  long long b, h, s;
+};
+// Strides of a [B][heads][S][D] (BNSD) or [B][S][heads][D] (BSND) tensor, and of its [B][heads][S]
+// or [B][S][heads] LSE.
+inline BsaStrides bsa_strides(int layout, int heads, int S, int D) {
+  if (layout == BSA_LAYOUT_BSND) return {1LL * S * heads * D, D, 1LL * heads * D};
+  return {1LL * heads * S * D, 1LL * S * D, D};
+}
+
 // ---- BSA forward (bsa_fwd.cu) --------------------------------------------------------------------
 struct BsaFwdArgs {
   int B, N1, N2, S_q, S_kv, bx, by, nqb, nkb, mask_mode, win_left, win_right;
   float scale;
+  BsaStrides qs, kvs, lse_s;  // element strides of q / out, of k / v, of the LSE
+  const uint8_t* atten_mask;  // optional dense [S_q][S_kv] mask (nonzero = masked out) or nullptr
   const int32_t* row_ptr;
   const int32_t* col;
   void* out;
@@ -80,6 +100,8 @@ cudaError_t bsa_fwd_launch(const BsaFwdArgs& a, const void* q, const void* k, co
 struct BsaBwdArgs {
   int B, N1, N2, S_q, S_kv, bx, by, nqb, nkb, mask_mode, win_left, win_right;
   float scale;
+  BsaStrides qs, kvs, lse_s;  // element strides of q / out / dout / dq, of k / v / dk / dv, of the LSE
+  const uint8_t* atten_mask;  // optional dense [S_q][S_kv] mask (nonzero = masked out) or nullptr
   const int32_t* row_ptr;    // KV lists per (b, h, qb)
   const int32_t* col;
   const int32_t* t_row_ptr;  // transposed lists per (b, g, kb)
@@ -156,6 +178,10 @@ struct NsaArgs {
   uint32_t* status;
 };
 cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st);
+// token-major passes on tcgen05 (nsa_tc.cu): Out / LSE, and dQ (needs lse2 / dvec from the
+// backward preprocess)
+cudaError_t nsa_fwd_tc_launch(const NsaArgs& a, cudaStream_t st);
+cudaError_t nsa_dq_tc_launch(const NsaArgs& a, cudaStream_t st);
 cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st);
 // dK/dV on tcgen05 (nsa_dkdv.cu) for 64-token blocks and G in {8, 16, 32, 64, 128};
 // cudaErrorNotSupported for other shapes.  Needs lse2/dvec from the backward preprocess.

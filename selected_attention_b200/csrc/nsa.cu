@@ -1,15 +1,14 @@
-// NSA selected attention, forward and backward (NsaSelectedAttention page, forward formula:
-// selected_key/value = Gather(key/value, topk_indices[i]); Out = Softmax(Mask(scale q K_sel^T))
-// V_sel; the backward applies the BlockSparseAttentionGrad formulas to the gathered blocks).
+// NSA selected attention, backward preprocess and the block-major dK / dV pass for the shapes the
+// tensor-core dK / dV kernel does not cover (NsaSelectedAttention page, forward formula:
+// selected_key/value = Gather(key/value, topk_indices[i]); the backward applies the
+// BlockSparseAttentionGrad formulas to the gathered blocks).  The token-major forward and dQ
+// passes run on tcgen05 (nsa_tc.cu), dK / dV for 64-token blocks and G in {8, ..., 128} too
+// (nsa_dkdv.cu).
 //
-// A query tile here is one token's heads of one kv-head group: 16 rows.  That is below the 64-row
-// minimum of tcgen05, and the path moves ~16 bytes of gathered K/V per 16x16 MMA step, so the
-// kernels use warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate): one warp owns one
-// (token, kv head, 16-head tile) and streams its selected blocks through shared memory in 16-key
-// chunks (TMA, three stages per warp).  The dK/dV pass is block-major: one CTA per (b, g, kv block)
-// walks the ascending token list of that block (nsa_meta.cu), four warps each owning 16 of the
-// block's 64 keys; a block listed twice by a token (literal Gather) counts twice.
-// P and dS enter the products that accumulate dV, dK and dQ as two bf16 parts (hi + lo).
+// The fallback dK/dV pass here is block-major: one CTA per (b, g, kv block) walks the ascending
+// token list of that block (nsa_meta.cu), warps each owning 16 of the block's keys with warp-level
+// mma.sync (m16n8k16); a block listed twice by a token (literal Gather) counts twice.  P and dS
+// enter the products that accumulate dV and dK as two bf16 parts (hi + lo).
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -19,9 +18,7 @@ namespace sa {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kChunk = 16;       // keys per shared-memory chunk
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 // ---------------------------------------------------------------------------------------------
 // warp-level MMA and shared-memory helpers
@@ -104,303 +101,6 @@ struct NsaParams {
   uint32_t* status;
 };
 
-__device__ __forceinline__ int batch_of_token(const int32_t* __restrict__ cu, int B, int t) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (cu[mid] <= t) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
-// ---------------------------------------------------------------------------------------------
-// token-major kernels: forward (kDq = false) and dQ (kDq = true)
-//
-// Each warp owns one (token, kv head, 16-head tile) item and a private ring of tok_stages() chunk
-// stages.  Lane 0 copies a chunk's 16 K rows and 16 V rows with four TMA loads (the rows of one kv
-// head are 256 B apart in TND, one box of {64 dims, 1 head, 16 tokens} per head-dim half), into
-// 128-byte-swizzled [16 rows][64 dims] halves; all lanes wait on the stage's mbarrier.
-// ---------------------------------------------------------------------------------------------
-// Warps per CTA and ring depth: the forward fits 168 registers, so 12 warps with 2-stage rings fill
-// the register file; dQ also holds dO fragments (222 registers: 8 warps) and keeps 3 stages.
-template <bool kDq>
-__host__ __device__ constexpr int tok_warps() { return kDq ? 12 : 12; }
-template <bool kDq>
-__host__ __device__ constexpr int tok_stages() { return kDq ? 2 : 2; }
-constexpr int kHalfBytes = kChunk * 128;        // [16 rows][64 dims]
-constexpr int kTileBytes = 2 * kHalfBytes;      // [16 rows][128 dims]
-constexpr int kTokStageBytes = 2 * kTileBytes;  // K and V tiles of one chunk
-template <bool kDq>
-__host__ __device__ constexpr int tok_smem() {
-  return tok_warps<kDq>() * tok_stages<kDq>() * (kTokStageBytes + 8) + 1024;
-}
-
-// byte address of (row, 16-byte column c16 of the 128 dims) in a chunk tile
-__device__ __forceinline__ uint32_t tok_swz(uint32_t tile, int row, int c16) {
-  return tile + (c16 >> 3) * kHalfBytes + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
-}
-// B fragments of X^T for k = dims [16 ks, 16 ks + 16) and n = the 16 rows (two n8 tiles)
-__device__ __forceinline__ void ldsm_rows_k(uint32_t (&r)[4], uint32_t tile, int ks, int lane) {
-  const int row = (lane & 7) + ((lane >> 4) << 3);
-  ldsm_x4(r, tok_swz(tile, row, ks * 2 + ((lane >> 3) & 1)));
-}
-// B fragments of X for k = the 16 rows and n = dims [n0, n0 + 16) (transposed load)
-__device__ __forceinline__ void ldsm_rows_n(uint32_t (&r)[4], uint32_t tile, int n0, int lane) {
-  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
-  ldsm_x4_t(r, tok_swz(tile, row, (n0 >> 3) + (lane >> 4)));
-}
-
-// wait on a warp-private stage barrier (bounded; does not give up early when another CTA has
-// timed out, so a warp can always drain its own copies)
-__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      raise_status(status, SA_DEV_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-template <bool kDq>
-__global__ void __launch_bounds__(tok_warps<kDq>() * 32)
-    nsa_token_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const NsaParams prm) {
-  extern __shared__ uint8_t tsm_raw[];
-  uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int kTokWarps = tok_warps<kDq>();
-  constexpr int kTokStages = tok_stages<kDq>();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long item = static_cast<long long>(blockIdx.x) * kTokWarps + warp;  // (g, token, head tile)
-  const long long items = static_cast<long long>(prm.N2) * prm.T * prm.head_tiles;
-  if (item >= items || !*prm.ok_flag) return;
-  const int ht = static_cast<int>(item % prm.head_tiles);
-  const int t = static_cast<int>((item / prm.head_tiles) % prm.T);
-  const int g = static_cast<int>(item / (static_cast<long long>(prm.head_tiles) * prm.T));
-  const int b = batch_of_token(prm.cu, prm.B, t);
-  const int t0 = prm.cu[b], len = prm.cu[b + 1] - t0;
-  const int pos = t - t0;
-  const int h0 = g * prm.G + ht * 16;   // first query head of this tile
-  const int rows = min(16, prm.G - ht * 16);
-  const int n_sel = prm.cnt[static_cast<size_t>(t) * prm.N2 + g];
-  const int32_t* sel = prm.ids + (static_cast<size_t>(t) * prm.N2 + g) * prm.K;
-  const int r0 = lane >> 2, cq = (lane & 3) * 2;  // fragment row and column pair
-  uint8_t* wst = tsm + warp * kTokStages * kTokStageBytes;  // this warp's stages
-  uint64_t* wbar = reinterpret_cast<uint64_t*>(tsm + kTokWarps * kTokStages * kTokStageBytes) + warp * kTokStages;
-  if (lane == 0) {
-    for (int i = 0; i < kTokStages; ++i) mbar_init(&wbar[i], 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-
-  // Q (and dO for dQ) as A fragments: 8 k-steps x 4 registers, rows = heads
-  uint32_t qa[8][4], da[8][4];
-  {
-    const __nv_bfloat16* qb = prm.q + (static_cast<size_t>(t) * prm.N1 + h0) * kD;
-    const __nv_bfloat16* db = kDq ? prm.dout + (static_cast<size_t>(t) * prm.N1 + h0) * kD : nullptr;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int rr = r0 + (i & 1) * 8, cc = ks * 16 + cq + (i >> 1) * 8;
-        qa[ks][i] = rr < rows ? *reinterpret_cast<const uint32_t*>(qb + rr * kD + cc) : 0u;
-        if (kDq) da[ks][i] = rr < rows ? *reinterpret_cast<const uint32_t*>(db + rr * kD + cc) : 0u;
-      }
-  }
-  // per-row state (rows r0 and r0 + 8 of the tile)
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-  float l2r[2] = {0.f, 0.f}, dr[2] = {0.f, 0.f};
-  if (kDq) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int rr = r0 + i * 8;
-      l2r[i] = rr < rows ? prm.lse2[static_cast<size_t>(t) * prm.N1 + h0 + rr] : INFINITY;
-      dr[i] = rr < rows ? prm.dvec[static_cast<size_t>(t) * prm.N1 + h0 + rr] : 0.f;
-    }
-  }
-  float acc[16][4];  // O or dQ: 16 n-tiles of 8 columns
-#pragma unroll
-  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-
-  // chunk list: each selected block contributes sel_block / 16 chunks; a chunk whose first key is
-  // past the last visible position (the sequence end, or the query under the causal mask) holds
-  // no visible key and is skipped.  Rows of a loaded chunk past the batch are masked below.
-  const int cpb = prm.sel_block / kChunk;
-  const int n_chunks = n_sel * cpb;
-  const int last_key = prm.mask_mode == 2 ? pos : len - 1;
-  auto first_key = [&](int c) { return sel[c / cpb] * prm.sel_block + (c % cpb) * kChunk; };
-  int cand = 0;
-  // the next visible chunk (or n_chunks) into `stage`
-  auto take = [&](int stage) {
-    int c = cand;
-    while (c < n_chunks && first_key(c) > last_key) ++c;
-    if (c < n_chunks) {
-      cand = c + 1;
-      if (lane == 0) {
-        const int tk = t0 + first_key(c);
-        uint8_t* st = wst + stage * kTokStageBytes;
-        mbar_arrive_expect_tx(&wbar[stage], kTokStageBytes);
-        tma_load_3d(st, &tm_k, &wbar[stage], 0, g, tk);
-        tma_load_3d(st + kHalfBytes, &tm_k, &wbar[stage], 64, g, tk);
-        tma_load_3d(st + kTileBytes, &tm_v, &wbar[stage], 0, g, tk);
-        tma_load_3d(st + kTileBytes + kHalfBytes, &tm_v, &wbar[stage], 64, g, tk);
-      }
-    }
-    return c;
-  };
-  // chunks in flight, oldest first: load k goes to stage k % kTokStages
-  int fifo[kTokStages - 1];
-#pragma unroll
-  for (int i = 0; i < kTokStages - 1; ++i) fifo[i] = take(i);
-  int loaded = 0, waited = 0;
-#pragma unroll
-  for (int i = 0; i < kTokStages - 1; ++i) loaded += fifo[i] < n_chunks ? 1 : 0;
-  for (int it = 0; fifo[0] < n_chunks; ++it) {
-    const int c = fifo[0];
-#pragma unroll
-    for (int i = 0; i + 1 < kTokStages - 1; ++i) fifo[i] = fifo[i + 1];
-    fifo[kTokStages - 2] = take((it + kTokStages - 1) % kTokStages);  // the stage consumed last iteration
-    loaded += fifo[kTokStages - 2] < n_chunks ? 1 : 0;
-    const int stage = it % kTokStages;
-    if (!__all_sync(0xffffffffu, stage_wait(&wbar[stage], (it / kTokStages) & 1, prm.status)))
-      break;  // the copies still in flight are drained below
-    ++waited;
-    const int kp0 = first_key(c);
-    const int valid = min(kChunk, len - kp0);
-    const uint32_t kt = smem_u32(wst + stage * kTokStageBytes), vt = kt + kTileBytes;
-    // S = Q K^T (16 rows x 16 keys): two n8 tiles.  The forward runs each as two independent
-    // k-halves (shorter dependency chains); dQ, short of registers, as one chain.
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    if (!kDq) {
-      float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t bk[4], bk2[4];
-        ldsm_rows_k(bk, kt, ks, lane);
-        ldsm_rows_k(bk2, kt, ks + 4, lane);
-        mma16816(s[0], qa[ks], bk[0], bk[1]);
-        mma16816(s[1], qa[ks], bk[2], bk[3]);
-        mma16816(s2[0], qa[ks + 4], bk2[0], bk2[1]);
-        mma16816(s2[1], qa[ks + 4], bk2[2], bk2[3]);
-      }
-#pragma unroll
-      for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) s[n][i] += s2[n][i];
-    } else {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t bk[4];
-        ldsm_rows_k(bk, kt, ks, lane);
-        mma16816(s[0], qa[ks], bk[0], bk[1]);
-        mma16816(s[1], qa[ks], bk[2], bk[3]);
-      }
-    }
-    // mask: key position kp0 + column < len, and causal key <= query position
-    const int lim = prm.mask_mode == 2 ? min(valid - 1, pos - kp0) : valid - 1;
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = n * 8 + cq + (i & 1);
-        const int rr = r0 + (i >> 1) * 8;
-        if (col > lim || rr >= rows) s[n][i] = -INFINITY;
-      }
-    uint32_t pa_hi[4], pa_lo[4];  // P (or dS) as the A operand over the 16 keys
-    if (!kDq) {
-      // online softmax (lazy rescale by 2^8), rows r0 and r0 + 8
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        float mx = fmaxf(fmaxf(s[0][2 * i], s[0][2 * i + 1]), fmaxf(s[1][2 * i], s[1][2 * i + 1]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        mx *= prm.scale_log2;
-        if (mx > m[i] + 8.f) {
-          const float alpha = m[i] == -INFINITY ? 0.f : ex2(m[i] - mx);
-          l[i] *= alpha;
-#pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            acc[n][2 * i] *= alpha;
-            acc[n][2 * i + 1] *= alpha;
-          }
-          m[i] = mx;
-        }
-        const float mu = m[i] == -INFINITY ? 0.f : m[i];
-#pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          s[n][2 * i] = ex2(fmaf(s[n][2 * i], prm.scale_log2, -mu));
-          s[n][2 * i + 1] = ex2(fmaf(s[n][2 * i + 1], prm.scale_log2, -mu));
-          l[i] += s[n][2 * i] + s[n][2 * i + 1];
-        }
-      }
-      pa_hi[0] = pack_bf16(s[0][0], s[0][1]);
-      pa_hi[1] = pack_bf16(s[0][2], s[0][3]);
-      pa_hi[2] = pack_bf16(s[1][0], s[1][1]);
-      pa_hi[3] = pack_bf16(s[1][2], s[1][3]);
-    } else {
-      // P = 2^(s scale log2e - LSE log2e); dP = dO V^T; dS = P (dP - D)
-      float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t bv[4];
-        ldsm_rows_k(bv, vt, ks, lane);
-        mma16816(dp[0], da[ks], bv[0], bv[1]);
-        mma16816(dp[1], da[ks], bv[2], bv[3]);
-      }
-#pragma unroll
-      for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float p = ex2(fmaf(s[n][i], prm.scale_log2, -l2r[i >> 1]));
-          s[n][i] = p * (dp[n][i] - dr[i >> 1]);
-        }
-      split2(s[0][0], s[0][1], pa_hi[0], pa_lo[0]);
-      split2(s[0][2], s[0][3], pa_hi[1], pa_lo[1]);
-      split2(s[1][0], s[1][1], pa_hi[2], pa_lo[2]);
-      split2(s[1][2], s[1][3], pa_hi[3], pa_lo[3]);
-    }
-    // acc += P V (forward) or dS K (dQ): B = [16 keys][128 columns] from the V or K tile
-    const uint32_t bt = kDq ? kt : vt;
-#pragma unroll
-    for (int n = 0; n < 16; n += 2) {
-      uint32_t bb[4];
-      ldsm_rows_n(bb, bt, n * 8, lane);
-      mma16816(acc[n], pa_hi, bb[0], bb[1]);
-      mma16816(acc[n + 1], pa_hi, bb[2], bb[3]);
-      if (kDq) {
-        mma16816(acc[n], pa_lo, bb[0], bb[1]);
-        mma16816(acc[n + 1], pa_lo, bb[2], bb[3]);
-      }
-    }
-    __syncwarp();  // every lane has read the stage before lane 0 refills it
-  }
-  // drain copies still in flight after an early exit (none after a complete pass)
-  for (int k = waited; k < loaded; ++k) stage_wait(&wbar[k % kTokStages], (k / kTokStages) & 1, prm.status);
-  if (aborted(prm.status)) return;
-  // epilogue
-  if (!kDq) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      l[i] += __shfl_xor_sync(0xffffffffu, l[i], 1);
-      l[i] += __shfl_xor_sync(0xffffffffu, l[i], 2);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int rr = r0 + i * 8;
-    if (rr >= rows) continue;
-    const size_t orow = static_cast<size_t>(t) * prm.N1 + h0 + rr;
-    const float mul = kDq ? prm.scale : (l[i] > 0.f ? 1.f / l[i] : 0.f);
-    __nv_bfloat16* dst = (kDq ? prm.dq : prm.o) + orow * kD;
-#pragma unroll
-    for (int n = 0; n < 16; ++n)
-      *reinterpret_cast<uint32_t*>(dst + n * 8 + cq) = pack_bf16(acc[n][2 * i] * mul, acc[n][2 * i + 1] * mul);
-    if (!kDq && (lane & 3) == 0) prm.lse_out[orow] = l[i] > 0.f ? (m[i] * kLn2 + logf(l[i])) : -INFINITY;
-  }
-}
 
 // softmax_grad D = rowsum(dOut o Out) and LSE * log2(e) per (token, head); 8 threads per row
 __global__ void nsa_prep_kernel(const NsaParams prm) {
@@ -610,31 +310,7 @@ NsaParams make_params(const NsaArgs& a) {
 
 }  // namespace
 
-// K and V as [T][N2][128] with a {64 dims, 1 head, 16 tokens} box (rows past T read as zero)
-bool nsa_kv_maps(const NsaArgs& a, CUtensorMap* tk, CUtensorMap* tv) {
-  const uint64_t hs = static_cast<uint64_t>(a.N2) * kD;
-  return make_tmap_3d_bf16(tk, a.k, kD, a.N2, a.T, kD, hs, 1, kChunk) &&
-         make_tmap_3d_bf16(tv, a.v, kD, a.N2, a.T, kD, hs, 1, kChunk);
-}
-
-template <bool kDq>
-cudaError_t nsa_token_launch(const NsaArgs& a, const NsaParams& p, const char* name, cudaStream_t st) {
-  const long long items = static_cast<long long>(a.N2) * a.T * p.head_tiles;
-  if (items == 0) return cudaSuccess;
-  CUtensorMap tk, tv;
-  if (!nsa_kv_maps(a, &tk, &tv)) return cudaErrorInvalidValue;
-  constexpr int warps = tok_warps<kDq>(), smem = tok_smem<kDq>();
-  cudaError_t e = cudaFuncSetAttribute(nsa_token_kernel<kDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  prof_begin(name, st);
-  nsa_token_kernel<kDq><<<static_cast<unsigned>((items + warps - 1) / warps), warps * 32, smem, st>>>(tk, tv, p);
-  prof_end(st);
-  return cudaGetLastError();
-}
-
-cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st) {
-  return nsa_token_launch<false>(a, make_params(a), "nsa_fwd", st);
-}
+cudaError_t nsa_fwd_launch(const NsaArgs& a, cudaStream_t st) { return nsa_fwd_tc_launch(a, st); }
 
 cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st) {
   const NsaParams p = make_params(a);
@@ -664,8 +340,7 @@ cudaError_t nsa_bwd_launch(const NsaArgs& a, cudaStream_t st) {
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = nsa_token_launch<true>(a, p, "nsa_bwd_dq", st)) != cudaSuccess) return e;
-  return cudaSuccess;
+  return nsa_dq_tc_launch(a, st);
 }
 
 }  // namespace sa
