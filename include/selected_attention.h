@@ -97,6 +97,10 @@ typedef struct bsa_params {
   const int32_t* sparse_indices;
   int32_t mask_mode, win_left, win_right; /* bsa_mask_mode */
   float scale;                            /* multiplies q.k (SFA: the whole q.k + q_r.k_r) */
+  /* BSA only: optional dense atten_mask, device uint8 [S_q, S_kv] shared by every batch and head,
+   * nonzero = masked out; applied inside the selected blocks on top of mask_mode (the
+   * Mask(., atten_mask) step of the BlockSparseAttentionGrad formulas).  NULL = none. */
+  const uint8_t* atten_mask;
 } bsa_params;
 
 /* ---- workspace sizing (phase 1: host validation, no launch) ------------------------------ */

@@ -81,11 +81,17 @@ def stored_out(o: np.ndarray, out_storage) -> np.ndarray:
 # sparseMode 0 / 2; SparseAttnSharedkvMetadata mask modes 3 and 4 with ori_win_left/right)
 # ----------------------------------------------------------------------------------------------
 def visible(pos_q: np.ndarray, pos_k: np.ndarray, mode: int, s_q: int, s_kv: int,
-            kv_len: int, win_left: int = 0, win_right: int = 0) -> np.ndarray:
-    """Boolean [len(pos_q), len(pos_k)]: key k is visible to query q."""
+            kv_len: int, win_left: int = 0, win_right: int = 0, atten_mask=None) -> np.ndarray:
+    """Boolean [len(pos_q), len(pos_k)]: key k is visible to query q.  atten_mask, when given, is
+    the dense [S_q, S_kv] mask of the Mask(., atten_mask) step (nonzero = masked out), applied on
+    top of the mode."""
     pq = np.asarray(pos_q, dtype=np.int64)[:, None]
     pk = np.asarray(pos_k, dtype=np.int64)[None, :]
     ok = (pk >= 0) & (pk < kv_len)
+    if atten_mask is not None:
+        am = np.asarray(atten_mask)
+        inside = (pq >= 0) & (pq < am.shape[0]) & (pk >= 0) & (pk < am.shape[1])
+        ok = ok & inside & (am[np.clip(pq, 0, am.shape[0] - 1), np.clip(pk, 0, am.shape[1] - 1)] == 0)
     if mode == 0:
         return ok & np.ones_like(pq, dtype=bool)
     if mode == 2:
@@ -151,7 +157,7 @@ def bsa_unit_keys(mask_row: np.ndarray, by: int, s_kv: int) -> np.ndarray:
 
 
 def bsa_slice_forward(q_g, k_g, v_g, mask_g, bx, by, mode, scale, win_left=0, win_right=0,
-                      q_blocks=None):
+                      q_blocks=None, atten_mask=None):
     """One (batch, kv-head) slice.  q_g [G, Sq, D] (the group's query heads), k_g [Skv, D],
     v_g [Skv, Dv], mask_g [G, nqb, nkb].  Returns Out [G, Sq, Dv], LSE [G, Sq]; with q_blocks
     given, only those Q blocks are filled (the rest stay NaN)."""
@@ -164,7 +170,7 @@ def bsa_slice_forward(q_g, k_g, v_g, mask_g, bx, by, mode, scale, win_left=0, wi
         for qb in (range(nqb) if q_blocks is None else q_blocks):
             rows = np.arange(qb * bx, min(s_q, (qb + 1) * bx))
             keys = bsa_unit_keys(mask_g[h, qb], by, s_kv)
-            vis = visible(rows, keys, mode, s_q, s_kv, s_kv, win_left, win_right)
+            vis = visible(rows, keys, mode, s_q, s_kv, s_kv, win_left, win_right, atten_mask)
             o, l, _ = attend(q_g[h, rows], k_g[keys], v_g[keys], vis, scale)
             out[h, rows] = o
             lse[h, rows] = l
@@ -172,7 +178,8 @@ def bsa_slice_forward(q_g, k_g, v_g, mask_g, bx, by, mode, scale, win_left=0, wi
 
 
 def bsa_slice_backward(q_g, k_g, v_g, dout_g, mask_g, bx, by, mode, scale, win_left=0,
-                       win_right=0, q_blocks=None, kv_blocks=None, out_storage=None, out_in_g=None):
+                       win_right=0, q_blocks=None, kv_blocks=None, out_storage=None, out_in_g=None,
+                       atten_mask=None):
     """One (batch, kv-head) slice of the backward pass.  Returns dQ [G,Sq,D], dK [Skv,D],
     dV [Skv,Dv], Out, LSE.  Units (h, qb) are skipped only when they contribute neither to a
     requested dQ block nor to a requested KV block, so every requested entry is exact.
@@ -198,7 +205,7 @@ def bsa_slice_backward(q_g, k_g, v_g, dout_g, mask_g, bx, by, mode, scale, win_l
                     continue
             rows = np.arange(qb * bx, min(s_q, (qb + 1) * bx))
             keys = bsa_unit_keys(mask_g[h, qb], by, s_kv)
-            vis = visible(rows, keys, mode, s_q, s_kv, s_kv, win_left, win_right)
+            vis = visible(rows, keys, mode, s_q, s_kv, s_kv, win_left, win_right, atten_mask)
             qr, kr, vr = q_g[h, rows], k_g[keys], v_g[keys]
             o, l, p = attend(qr, kr, vr, vis, scale)
             o_in = stored_out(o, out_storage) if out_in_g is None else out_in_g[h, rows]
@@ -215,8 +222,9 @@ def _f64(x):
     return bf16_to_f64(x) if np.asarray(x).dtype == np.uint16 else np.asarray(x, dtype=np.float64)
 
 
-def bsa_forward(q, k, v, block_mask, bx, by, mode, scale, win_left=0, win_right=0):
-    """Full BNSD forward: q [B,N1,Sq,D], k/v [B,N2,Skv,D*] (bf16 bits or floats)."""
+def bsa_forward(q, k, v, block_mask, bx, by, mode, scale, win_left=0, win_right=0, atten_mask=None):
+    """Full BNSD forward: q [B,N1,Sq,D], k/v [B,N2,Skv,D*] (bf16 bits or floats); atten_mask an
+    optional dense [Sq, Skv] mask (nonzero = masked out) shared by every batch and head."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, N1, s_q, _ = q.shape
     N2 = k.shape[1]
@@ -227,12 +235,13 @@ def bsa_forward(q, k, v, block_mask, bx, by, mode, scale, win_left=0, win_right=
         for g in range(N2):
             hs = slice(g * G, (g + 1) * G)
             o, l = bsa_slice_forward(q[b, hs], k[b, g], v[b, g], block_mask[b, hs], bx, by, mode,
-                                     scale, win_left, win_right)
+                                     scale, win_left, win_right, atten_mask=atten_mask)
             out[b, hs], lse[b, hs] = o, l
     return out, lse
 
 
-def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win_right=0, out_in=None):
+def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win_right=0, out_in=None,
+                 atten_mask=None):
     """Full BNSD backward; returns dQ, dK, dV, Out, LSE.  out_in [B,N1,Sq,Dv] (bf16 bits or
     floats), when given, is the backward operator's attentionOut input (softmax_grad =
     rowsum(dOut o attentionOut)); by default the oracle's own Out, stored in the input dtype."""
@@ -252,7 +261,7 @@ def bsa_backward(q, k, v, dout, block_mask, bx, by, mode, scale, win_left=0, win
             hs = slice(g * G, (g + 1) * G)
             r = bsa_slice_backward(q[b, hs], k[b, g], v[b, g], dout[b, hs], block_mask[b, hs],
                                    bx, by, mode, scale, win_left, win_right, out_storage=out_storage,
-                                   out_in_g=None if out_in is None else out_in[b, hs])
+                                   out_in_g=None if out_in is None else out_in[b, hs], atten_mask=atten_mask)
             dq[b, hs], dk[b, g], dv[b, g], out[b, hs], lse[b, hs] = r
     return dq, dk, dv, out, lse
 

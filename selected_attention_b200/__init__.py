@@ -59,6 +59,7 @@ class Params(ctypes.Structure):
         ("sparse_indices", ctypes.c_void_p),
         ("mask_mode", ctypes.c_int32), ("win_left", ctypes.c_int32), ("win_right", ctypes.c_int32),
         ("scale", ctypes.c_float),
+        ("atten_mask", ctypes.c_void_p),
     ]
 
 
@@ -142,11 +143,17 @@ def version() -> str:
 # BSA (BNSD)
 # ---------------------------------------------------------------------------------------------
 def bsa_params(q, k, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
-               win_right=0) -> Params:
-    B, N1, S_q, D = q.shape
-    _, N2, S_kv, _ = k.shape
+               win_right=0, layout=LAYOUT_BNSD, atten_mask=None) -> Params:
+    """layout LAYOUT_BNSD: q [B, N1, S_q, D], k [B, N2, S_kv, D]; LAYOUT_BSND: q [B, S_q, N1, D],
+    k [B, S_kv, N2, D].  atten_mask: optional uint8 CUDA tensor [S_q, S_kv], nonzero = masked out."""
+    if layout == LAYOUT_BSND:
+        B, S_q, N1, D = q.shape
+        _, S_kv, N2, _ = k.shape
+    else:
+        B, N1, S_q, D = q.shape
+        _, N2, S_kv, _ = k.shape
     p = Params()
-    p.q_layout = p.kv_layout = LAYOUT_BNSD
+    p.q_layout = p.kv_layout = layout
     p.B, p.N1, p.N2, p.S_q, p.S_kv = B, N1, N2, S_q, S_kv
     p.D = D
     p.Dv = D
@@ -154,7 +161,15 @@ def bsa_params(q, k, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=
     p.block_mask = block_mask.data_ptr()
     p.mask_mode, p.win_left, p.win_right = mask_mode, win_left, win_right
     p.scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if atten_mask is not None:
+        _need_cuda(atten_mask)
+        assert atten_mask.dtype == torch.uint8 and tuple(atten_mask.shape) == (S_q, S_kv) and atten_mask.is_contiguous()
+        p.atten_mask = atten_mask.data_ptr()
     return p
+
+
+def _lse_shape(p: Params):
+    return (p.B, p.S_q, p.N1) if p.q_layout == LAYOUT_BSND else (p.B, p.N1, p.S_q)
 
 
 def bsa_fwd_workspace_size(p: Params) -> int:
@@ -164,16 +179,16 @@ def bsa_fwd_workspace_size(p: Params) -> int:
 
 
 def bsa_fwd(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
-            win_right=0, out=None, lse=None, workspace=None, stream=None):
-    """Out, LSE = softmax(Mask(scale Q K_sel^T)) V_sel for BNSD bf16 tensors and a uint8
-    BlockSparseMask [B, N1, ceil(S_q/block_x), ceil(S_kv/block_y)]."""
+            win_right=0, out=None, lse=None, workspace=None, stream=None, layout=LAYOUT_BNSD, atten_mask=None):
+    """Out, LSE = softmax(Mask(scale Q K_sel^T)) V_sel for BNSD (or BSND) bf16 tensors and a uint8
+    BlockSparseMask [B, N1, ceil(S_q/block_x), ceil(S_kv/block_y)].  Out has q's layout; LSE is
+    [B, N1, S_q] (BNSD) or [B, S_q, N1] (BSND)."""
     _need_cuda(q, k, v, block_mask)
-    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right)
-    B, N1, S_q, _ = q.shape
+    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right, layout, atten_mask)
     if out is None:
-        out = torch.empty(B, N1, S_q, v.shape[-1], dtype=torch.bfloat16, device=q.device)
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
-        lse = torch.empty(B, N1, S_q, dtype=torch.float32, device=q.device)
+        lse = torch.empty(_lse_shape(p), dtype=torch.float32, device=q.device)
     need = bsa_fwd_workspace_size(p)
     if workspace is None:
         workspace = _workspace(need, q.device)
@@ -183,17 +198,16 @@ def bsa_fwd(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=
 
 
 def bsa_fwd_noalloc(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
-                    win_right=0, out=None, lse=None, stream=None):
+                    win_right=0, out=None, lse=None, stream=None, layout=LAYOUT_BNSD):
     """bsa_fwd without a workspace, for callers that cannot allocate device memory: the library
     keeps the scratch in a fixed 8 MiB device array (shared by all calls on a device; calls that
     overlap on the GPU race).  Out and LSE are still the caller's tensors."""
     _need_cuda(q, k, v, block_mask)
-    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right)
-    B, N1, S_q, _ = q.shape
+    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right, layout)
     if out is None:
-        out = torch.empty(B, N1, S_q, v.shape[-1], dtype=torch.bfloat16, device=q.device)
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
-        lse = torch.empty(B, N1, S_q, dtype=torch.float32, device=q.device)
+        lse = torch.empty(_lse_shape(p), dtype=torch.float32, device=q.device)
     _check("bsa_fwd_noalloc", lib().bsa_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                                     _ptr(lse), _stream(stream)))
     return out, lse
@@ -213,10 +227,11 @@ def bsa_bwd_workspace_size(p: Params) -> int:
 
 
 def bsa_bwd(q, k, v, out, dout, lse, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None,
-            win_left=0, win_right=0, dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV of block-sparse attention (BNSD)."""
+            win_left=0, win_right=0, dq=None, dk=None, dv=None, workspace=None, stream=None, layout=LAYOUT_BNSD,
+            atten_mask=None):
+    """dQ, dK, dV of block-sparse attention (BNSD or BSND, the gradients in the inputs' layout)."""
     _need_cuda(q, k, v, out, dout, lse, block_mask)
-    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right)
+    p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right, layout, atten_mask)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

@@ -18,7 +18,8 @@ inline int div_up(int a, int b) { return (a + b - 1) / b; }
 // block_x <= 128 (one 128-row MMA tile per Q block), block_y 64 or 128.
 bsa_status check_bsa(const bsa_params* p) {
   if (!p) return BSA_ERR_NULLPTR;
-  if (p->q_layout != BSA_LAYOUT_BNSD || p->kv_layout != BSA_LAYOUT_BNSD) return BSA_ERR_UNSUPPORTED;
+  if (p->q_layout != BSA_LAYOUT_BNSD && p->q_layout != BSA_LAYOUT_BSND) return BSA_ERR_UNSUPPORTED;
+  if (p->kv_layout != p->q_layout) return BSA_ERR_UNSUPPORTED;
   if (p->B <= 0 || p->N1 <= 0 || p->N2 <= 0 || p->S_q <= 0 || p->S_kv <= 0) return BSA_ERR_INVALID_ARG;
   if (p->N1 < p->N2 || p->N1 % p->N2 != 0) return BSA_ERR_INVALID_ARG;
   if (p->D != 128 || p->Dv != 128) return BSA_ERR_UNSUPPORTED;
@@ -271,6 +272,10 @@ bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void
   a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.S_q = p->S_q; a.S_kv = p->S_kv;
   a.bx = p->block_x; a.by = p->block_y; a.nqb = nqb; a.nkb = nkb;
   a.mask_mode = p->mask_mode; a.win_left = p->win_left; a.win_right = p->win_right; a.scale = p->scale;
+  a.qs = bsa_strides(p->q_layout, p->N1, p->S_q, p->D);
+  a.kvs = bsa_strides(p->kv_layout, p->N2, p->S_kv, p->D);
+  a.lse_s = bsa_strides(p->q_layout, p->N1, p->S_q, 1);
+  a.atten_mask = p->atten_mask;
   a.row_ptr = w.row_ptr; a.col = w.col; a.out = out; a.lse = lse; a.status = w.status;
   return cuda_status(bsa_fwd_launch(a, q, k, v, st));
 }
@@ -305,6 +310,10 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
   a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.S_q = p->S_q; a.S_kv = p->S_kv;
   a.bx = p->block_x; a.by = p->block_y; a.nqb = nqb; a.nkb = nkb;
   a.mask_mode = p->mask_mode; a.win_left = p->win_left; a.win_right = p->win_right; a.scale = p->scale;
+  a.qs = bsa_strides(p->q_layout, p->N1, p->S_q, p->D);
+  a.kvs = bsa_strides(p->kv_layout, p->N2, p->S_kv, p->D);
+  a.lse_s = bsa_strides(p->q_layout, p->N1, p->S_q, 1);
+  a.atten_mask = p->atten_mask;
   a.row_ptr = w.row_ptr; a.col = w.col; a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;
   a.dvec = w.dvec; a.lse2 = w.lse2; a.dq = dq; a.dk = dk; a.dv = dv; a.status = w.status;
   a.next_kv = &reinterpret_cast<WsHeader*>(w.status)->next_bwd_kv;

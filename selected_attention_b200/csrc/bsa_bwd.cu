@@ -32,8 +32,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // P = exp2(s * scale * log2(e) + (-L2)) is one fused multiply-add and dS = P * (dP + (-D)).
 // ------------------------------------------------------------------------------------------------
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
-                                const float* __restrict__ lse, int S_q, int bx, int nqb, long long n_rows,
-                                float* __restrict__ dvec, float* __restrict__ lse2) {
+                                const float* __restrict__ lse, int N1, int S_q, int bx, int nqb, long long n_rows,
+                                BsaStrides qs, BsaStrides ls, float* __restrict__ dvec, float* __restrict__ lse2) {
   griddep_wait();  // launched with programmatic dependent launch: the lists before it must be complete
   griddep_launch_dependents();
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -48,7 +48,8 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __n
   const bool valid = i < bx && qpos < S_q;
   float d = 0.f;
   if (valid) {
-    const size_t g = (static_cast<size_t>(bh) * S_q + qpos) * kD + part * 16;
+    const long long b = bh / N1, h = bh % N1;
+    const size_t g = static_cast<size_t>(b * qs.b + h * qs.h + qpos * qs.s) + part * 16;
     const uint4* po = reinterpret_cast<const uint4*>(out + g);
     const uint4* pd = reinterpret_cast<const uint4*>(dout + g);
 #pragma unroll
@@ -67,7 +68,8 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __n
     dvec[row] = valid ? -d : 0.f;
     float l2 = -INFINITY;
     if (valid) {
-      const float l = lse[static_cast<size_t>(bh) * S_q + qpos];
+      const long long b = bh / N1, h = bh % N1;
+      const float l = lse[static_cast<size_t>(b * ls.b + h * ls.h + qpos * ls.s)];
       l2 = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     }
     lse2[row] = l2;
@@ -89,6 +91,8 @@ struct BwdParams {
   __nv_bfloat16* dv;
   uint32_t* status;
   uint64_t* cta_clock;  // optional [grid][2] start / finish times (ns), see bsa_profile_cta_clock
+  BsaStrides qs, kvs;   // element strides of dq (heads N1) and of dk / dv (heads N2)
+  const uint8_t* amask; // optional dense atten_mask [S_q][S_kv], nonzero = masked out
 };
 
 __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&rr)[32], float mul) {
@@ -157,6 +161,7 @@ struct __align__(1024) KvSmem {
   uint32_t tmem_base;
 };
 
+template <bool kMask>  // kMask: a dense atten_mask is applied
 __global__ void __launch_bounds__(kKvThreads, 1)
     bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
@@ -198,22 +203,31 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  // unit i -> (b*N2 + g, kv block), its transposed list [rp, rp + n)
+  // Schedule number i -> (b*N2 + g, kv block), its transposed list [rp, rp + n).  The first
+  // kLead KV blocks of every (b, g) come first, interleaved across heads (under causal selection
+  // the earliest blocks are selected by the most q blocks: the longest lists, a sink block by all
+  // of them), then each head's remaining blocks in order, so no long list starts near the end.
   auto unit_of = [&](int i, int& bg, int& kb, int& rp, int& n) {
-    bg = i / prm.nkb;
-    kb = i % prm.nkb;
+    constexpr int kLead = 16;
+    const int bgs = prm.B * prm.N2, lead = min(prm.nkb, kLead);
+    if (i < bgs * lead) {
+      kb = i / bgs;
+      bg = i % bgs;
+    } else {
+      const int j = i - bgs * lead, rest = prm.nkb - lead;
+      bg = j / rest;
+      kb = lead + j % rest;
+    }
     const int unit = bg * prm.nkb + kb;
     rp = prm.row_ptr[unit];
     n = prm.row_ptr[unit + 1] - rp;
   };
-  // list entry -> first row of its Q tile in the [B*N1*S_q, 128] view, its padded tile index and
-  // the position of its first query row
-  auto entry_rows = [&](int bg, int e_code, int& qrow, int& tile, int& qpos0) {
+  // list entry -> its query head, its padded tile index and the position of its first query row
+  auto entry_rows = [&](int bg, int e_code, int& qh, int& tile, int& qpos0) {
     const int b = bg / prm.N2, g = bg % prm.N2;
     const int hl = e_code / prm.nqb, qb = e_code % prm.nqb;
-    const int bh = b * prm.N1 + g * G + hl;
-    qrow = bh * prm.S_q + qb * prm.bx;
-    tile = bh * prm.nqb + qb;
+    qh = g * G + hl;
+    tile = (b * prm.N1 + qh) * prm.nqb + qb;
     qpos0 = qb * prm.bx;
   };
   auto next_from_ring = [&](int k) -> int {
@@ -241,26 +255,26 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         int bg, kb, rp, n;
         unit_of(i, bg, kb, rp, n);
         if (n == 0) continue;
-        const int kv_row0 = bg * prm.S_kv + kb * prm.by;
+        const int b = bg / prm.N2, g = bg % prm.N2, kpos0 = kb * prm.by;
         if (ucount > 0 && !(ok = mbar_wait(&s.bar_kv_empty, (ucount - 1) & 1, prm.status))) break;
         mbar_arrive_expect_tx(&s.bar_kv, 4 * kT * 128);
-        tma_load_2d(s.k[0], &tm_k, &s.bar_kv, 0, kv_row0);
-        tma_load_2d(s.k[1], &tm_k, &s.bar_kv, 64, kv_row0);
-        tma_load_2d(s.v[0], &tm_v, &s.bar_kv, 0, kv_row0);
-        tma_load_2d(s.v[1], &tm_v, &s.bar_kv, 64, kv_row0);
+        tma_load_4d(s.k[0], &tm_k, &s.bar_kv, 0, g, kpos0, b);
+        tma_load_4d(s.k[1], &tm_k, &s.bar_kv, 64, g, kpos0, b);
+        tma_load_4d(s.v[0], &tm_v, &s.bar_kv, 0, g, kpos0, b);
+        tma_load_4d(s.v[1], &tm_v, &s.bar_kv, 64, g, kpos0, b);
         ++ucount;
         for (int e = 0; ok && e < 2 * n; ++e) {
           const int h = e & 1;
-          int qrow, tile, qpos0;
-          entry_rows(bg, prm.col[rp + (e >> 1)], qrow, tile, qpos0);
+          int qh, tile, qpos0;  // the entry's query head (hq counts the half entries loaded)
+          entry_rows(bg, prm.col[rp + (e >> 1)], qh, tile, qpos0);
           const int hs = hq % kKvRing;
           if (hq >= kKvRing && !(ok = mbar_wait(&s.bar_qdo_empty[hs], ((hq / kKvRing) - 1) & 1, prm.status))) break;
           mbar_arrive_expect_tx(&s.bar_qdo[hs], 4 * kHalfRows * 128 + 2 * kHalfRows * 4);
-          const int row = qrow + h * kHalfRows;
-          tma_load_2d(s.q[hs][0], &tm_q64, &s.bar_qdo[hs], 0, row);
-          tma_load_2d(s.q[hs][1], &tm_q64, &s.bar_qdo[hs], 64, row);
-          tma_load_2d(s.dout[hs][0], &tm_do64, &s.bar_qdo[hs], 0, row);
-          tma_load_2d(s.dout[hs][1], &tm_do64, &s.bar_qdo[hs], 64, row);
+          const int qp = qpos0 + h * kHalfRows;
+          tma_load_4d(s.q[hs][0], &tm_q64, &s.bar_qdo[hs], 0, qh, qp, b);
+          tma_load_4d(s.q[hs][1], &tm_q64, &s.bar_qdo[hs], 64, qh, qp, b);
+          tma_load_4d(s.dout[hs][0], &tm_do64, &s.bar_qdo[hs], 0, qh, qp, b);
+          tma_load_4d(s.dout[hs][1], &tm_do64, &s.bar_qdo[hs], 64, qh, qp, b);
           const size_t voff = static_cast<size_t>(tile) * kT + h * kHalfRows;
           bulk_load(s.lse2[hs], prm.lse2 + voff, kHalfRows * 4, &s.bar_qdo[hs]);
           bulk_load(s.dvec[hs], prm.dvec + voff, kHalfRows * 4, &s.bar_qdo[hs]);
@@ -379,8 +393,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (!key_valid) { qlo = 1; qhi = 0; }
       for (int x = 0; x < 2 * n; ++x) {
         const int hx = G0 + x, hs = hx % kKvRing;
-        int qrow, tile, qpos0;
-        entry_rows(bg, prm.col[rp + (x >> 1)], qrow, tile, qpos0);
+        int qh, tile, qpos0;
+        entry_rows(bg, prm.col[rp + (x >> 1)], qh, tile, qpos0);
         const int qp0 = qpos0 + (x & 1) * kHalfRows + c0;  // query position of column c0
         // exact parity: the next phase of sdp_full needs the sdp_free arrival below
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status) &&
@@ -399,7 +413,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const float4* nl2 = reinterpret_cast<const float4*>(s.lse2[hs] + c0);  // -LSE*log2e per query row
         const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D per query row
         const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
-        const bool full = qp0 >= qlo && qp0 + 31 <= qhi;
+        // the dense atten_mask: bit c set when query column c of the chunk may not see this key
+        uint32_t mbits = 0;
+        if (kMask && key_valid) {
+#pragma unroll 4
+          for (int c = 0; c < 32; ++c) {
+            const int qp = qp0 + c;
+            if (qp < prm.S_q && prm.amask[static_cast<size_t>(qp) * prm.S_kv + kpos] != 0) mbits |= 1u << c;
+          }
+        }
+        const bool full = qp0 >= qlo && qp0 + 31 <= qhi && mbits == 0;
         uint32_t ph[16], pl[16], dh[16], dl[16];
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
@@ -413,8 +436,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                       t0, t1);
             float p0 = ex2(t0), p1 = ex2(t1);
             if (!full) {
-              if (qp0 + c < qlo || qp0 + c > qhi) p0 = 0.f;
-              if (qp0 + c + 1 < qlo || qp0 + c + 1 > qhi) p1 = 0.f;
+              if (qp0 + c < qlo || qp0 + c > qhi || ((mbits >> c) & 1u)) p0 = 0.f;
+              if (qp0 + c + 1 < qlo || qp0 + c + 1 > qhi || ((mbits >> (c + 1)) & 1u)) p1 = 0.f;
             }
             const uint64_t p2 = f2_pack(p0, p1);
             const uint64_t g2 = f2_mul(p2, f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
@@ -448,9 +471,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (!ok) break;
         tc_fence_after();
       }
-      const int kv_row0 = bg * prm.S_kv + kb * prm.by;
-      __nv_bfloat16* dkrow = prm.dk + static_cast<size_t>(kv_row0 + r) * kD + hf * 64;
-      __nv_bfloat16* dvrow = prm.dv + static_cast<size_t>(kv_row0 + r) * kD + hf * 64;
+      const size_t krow = static_cast<size_t>((bg / prm.N2) * prm.kvs.b + (bg % prm.N2) * prm.kvs.h +
+                                              static_cast<long long>(kb * prm.by + r) * prm.kvs.s);
+      __nv_bfloat16* dkrow = prm.dk + krow + hf * 64;
+      __nv_bfloat16* dvrow = prm.dv + krow + hf * 64;
 #pragma unroll
       for (int c = 0; c < kD / 2; c += 32) {
         uint32_t rk[32], rv[32];
@@ -509,7 +533,7 @@ struct __align__(1024) QSmem {
 // q block first).  Warps: 0-7 element-wise, 8 scheduler + TMA, 9 issues dQ += dS K (hi, lo),
 // 10 issues S = Q K^T and dP = dO V^T.  Per-buffer barriers (ds_ready, dq_done per S buffer) keep
 // every parity wait exact with two issuing threads.
-template <int BN>
+template <int BN, bool kMask>  // kMask: a dense atten_mask is applied
 __global__ void __launch_bounds__(kKvThreads, 1)
     bsa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -578,13 +602,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (lane == 0) {
       int jk = 0, jv = 0, ucount = 0;
       bool ok = true;
-      auto load_v = [&](int rp, int kv_row0, int j) -> bool {
+      auto load_v = [&](int rp, int b, int g, int j) -> bool {
         const int sv = jv % kQVStages, uv = jv / kQVStages;
         if (jv >= kQVStages && !mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status)) return false;
-        const int vrow = kv_row0 + prm.col[rp + j] * prm.by;
+        const int vpos = prm.col[rp + j] * prm.by;
         mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
-        tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
-        tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
+        tma_load_4d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, g, vpos, b);
+        tma_load_4d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, g, vpos, b);
         ++jv;
         return true;
       };
@@ -601,27 +625,26 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         unit_of(i, bh, qb, rp, n);
         if (n == 0) continue;
         const int b = bh / prm.N1, g = (bh % prm.N1) / (prm.N1 / prm.N2);
-        const int q_row0 = bh * prm.S_q + qb * prm.bx;
-        const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
+        const int h = bh % prm.N1, q_pos0 = qb * prm.bx;
         if (ucount > 0 && !(ok = mbar_wait(&s.bar_qdo_empty, (ucount - 1) & 1, prm.status))) break;
         mbar_arrive_expect_tx(&s.bar_qdo, 4 * kT * 128);
-        tma_load_2d(s.q[0], &tm_q, &s.bar_qdo, 0, q_row0);
-        tma_load_2d(s.q[1], &tm_q, &s.bar_qdo, 64, q_row0);
-        tma_load_2d(s.dout[0], &tm_do, &s.bar_qdo, 0, q_row0);
-        tma_load_2d(s.dout[1], &tm_do, &s.bar_qdo, 64, q_row0);
+        tma_load_4d(s.q[0], &tm_q, &s.bar_qdo, 0, h, q_pos0, b);
+        tma_load_4d(s.q[1], &tm_q, &s.bar_qdo, 64, h, q_pos0, b);
+        tma_load_4d(s.dout[0], &tm_do, &s.bar_qdo, 0, h, q_pos0, b);
+        tma_load_4d(s.dout[1], &tm_do, &s.bar_qdo, 64, h, q_pos0, b);
         ++ucount;
         for (int j = 0; ok && j < n; ++j) {
           const int sk = jk % kQKStages, uk = jk / kQKStages;
           if (jk >= kQKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
-          const int row = kv_row0 + prm.col[rp + j] * prm.by;
+          const int kpos = prm.col[rp + j] * prm.by;
           mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
-          tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
-          tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
+          tma_load_4d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, g, kpos, b);
+          tma_load_4d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, g, kpos, b);
           ++jk;
-          if (j >= kQKStages - kQVStages) ok = load_v(rp, kv_row0, j - (kQKStages - kQVStages));  // V trails K
+          if (j >= kQKStages - kQVStages) ok = load_v(rp, b, g, j - (kQKStages - kQVStages));  // V trails K
         }
         for (int j = n - (kQKStages - kQVStages); ok && j < n; ++j)
-          if (j >= 0) ok = load_v(rp, kv_row0, j);
+          if (j >= 0) ok = load_v(rp, b, g, j);
       }
       // do not leave the CTA with copies in flight
       for (int j = (jk > kQKStages ? jk - kQKStages : 0); j < jk; ++j)
@@ -720,7 +743,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (i < 0) break;
       int bh, qb, rp, n;
       unit_of(i, bh, qb, rp, n);
-      const int q_row0 = bh * prm.S_q + qb * prm.bx;
       const int qpos = qb * prm.bx + r;
       const bool row_valid = r < prm.bx && qpos < prm.S_q;
       int lo = 0, hi = prm.S_kv - 1;
@@ -761,6 +783,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             if (kp < lo || kp > hi) p[c] = 0.f;
           }
         }
+        if (kMask && row_valid) {
+          // the dense atten_mask inside the selected block: this row's bytes of the tile's columns
+          const uint64_t mbits =
+              dense_mask_bits<kHalf>(prm.amask + static_cast<size_t>(qpos) * prm.S_kv, kpos0, prm.S_kv);
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c)
+            if ((mbits >> c) & 1ull) p[c] = 0.f;
+        }
         // dp_full has one phase per tile; its next phase needs the dp_free arrival below
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, J & 1, prm.status));
         if (!ok) break;
@@ -799,7 +829,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc_fence_after();
       }
       const int d0 = hf * (kD / 2);
-      __nv_bfloat16* dqrow = prm.dq + static_cast<size_t>(q_row0 + r) * kD + d0;
+      __nv_bfloat16* dqrow =
+          prm.dq + static_cast<size_t>((bh / prm.N1) * prm.qs.b + (bh % prm.N1) * prm.qs.h +
+                                       static_cast<long long>(qpos) * prm.qs.s) + d0;
 #pragma unroll
       for (int c = 0; c < kD / 2; c += 32) {
         uint32_t rr[32];
@@ -827,10 +859,11 @@ template <int BN>
 cudaError_t launch_q(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tdo, int grid, cudaStream_t st) {
   const size_t smem = sizeof(QSmem<BN>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(bsa_bwd_q_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kernel = p.amask ? bsa_bwd_q_kernel<BN, true> : bsa_bwd_q_kernel<BN, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   prof_begin("bsa_bwd_q", st);
-  if (grid > 0) e = launch_pdl(bsa_bwd_q_kernel<BN>, dim3(grid), dim3(kKvThreads), smem, st, tq, tk, tv, tdo, p);
+  if (grid > 0) e = launch_pdl(kernel, dim3(grid), dim3(kKvThreads), smem, st, tq, tk, tv, tdo, p);
   prof_end(st);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -846,19 +879,21 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     prof_begin("bsa_bwd_prep", st);
     cudaError_t e = launch_pdl(bwd_prep_kernel, dim3(static_cast<unsigned>((threads + blk - 1) / blk)), dim3(blk), 0,
                                st, static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout),
-                               lse, a.S_q, a.bx, a.nqb, n_rows, a.dvec, a.lse2);
+                               lse, a.N1, a.S_q, a.bx, a.nqb, n_rows, a.qs, a.lse_s, a.dvec, a.lse2);
     prof_end(st);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  // Q, dO, K, V as (head dim, head, position, batch), whichever of BNSD / BSND is in memory
   CUtensorMap tq, tk, tv, tdo, tk128, tv128, tq64, tdo64;
-  const uint64_t q_rows = static_cast<uint64_t>(a.B) * a.N1 * a.S_q;
-  const uint64_t kv_rows = static_cast<uint64_t>(a.B) * a.N2 * a.S_kv;
-  if (!make_tmap_2d_bf16(&tq, q, q_rows, kD, kD, kT) || !make_tmap_2d_bf16(&tdo, dout, q_rows, kD, kD, kT) ||
-      !make_tmap_2d_bf16(&tk, k, kv_rows, kD, kD, a.by) || !make_tmap_2d_bf16(&tv, v, kv_rows, kD, kD, a.by) ||
-      !make_tmap_2d_bf16(&tk128, k, kv_rows, kD, kD, kT) || !make_tmap_2d_bf16(&tv128, v, kv_rows, kD, kD, kT) ||
-      !make_tmap_2d_bf16(&tq64, q, q_rows, kD, kD, kHalfRows) ||
-      !make_tmap_2d_bf16(&tdo64, dout, q_rows, kD, kD, kHalfRows))
+  auto qmap = [&](CUtensorMap* m, const void* base, uint32_t rows) {
+    return make_tmap_4d_bf16(m, base, kD, a.N1, a.S_q, a.B, a.qs.h, a.qs.s, a.qs.b, rows);
+  };
+  auto kvmap = [&](CUtensorMap* m, const void* base, uint32_t rows) {
+    return make_tmap_4d_bf16(m, base, kD, a.N2, a.S_kv, a.B, a.kvs.h, a.kvs.s, a.kvs.b, rows);
+  };
+  if (!qmap(&tq, q, kT) || !qmap(&tdo, dout, kT) || !kvmap(&tk, k, a.by) || !kvmap(&tv, v, a.by) ||
+      !kvmap(&tk128, k, kT) || !kvmap(&tv128, v, kT) || !qmap(&tq64, q, kHalfRows) || !qmap(&tdo64, dout, kHalfRows))
     return cudaErrorInvalidValue;
   BwdParams p;
   bool kv_launched = false;
@@ -871,6 +906,9 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
   p.dv = static_cast<__nv_bfloat16*>(a.dv);
   p.status = a.status;
   p.cta_clock = nullptr;
+  p.qs = a.qs;
+  p.kvs = a.kvs;
+  p.amask = a.atten_mask;
   // KV-major pass
   {
     BwdParams pk = p;
@@ -878,7 +916,8 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     pk.col = a.t_col;
     pk.next_unit = a.next_kv;
     const size_t smem = sizeof(KvSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(bsa_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kv_kernel = a.atten_mask ? bsa_bwd_kv_kernel<true> : bsa_bwd_kv_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int units = a.B * a.N2 * a.nkb;
     int dev = 0, sms = 148;
@@ -888,7 +927,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     prof_begin("bsa_bwd_kv", st);
     pk.pdl_wait = 1;
     pk.cta_clock = prof_cta_clock(1, grid);
-    if (grid > 0) e = launch_pdl(bsa_bwd_kv_kernel, dim3(grid), dim3(kKvThreads), smem, st, tq64, tk128, tv128, tdo64, pk);
+    if (grid > 0) e = launch_pdl(kv_kernel, dim3(grid), dim3(kKvThreads), smem, st, tq64, tk128, tv128, tdo64, pk);
     prof_end(st);
     if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
     kv_launched = grid > 0;

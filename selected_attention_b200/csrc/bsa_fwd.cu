@@ -78,6 +78,8 @@ struct FwdParams {
   int32_t* next_unit;  // scheduler counter, zero at launch
   uint32_t* status;
   uint64_t* cta_clock;  // optional [grid][2] start / finish times (ns), see bsa_profile_cta_clock
+  long long lse_sb, lse_sh, lse_ss;  // LSE element strides of (b, head, position)
+  const uint8_t* amask;  // optional dense atten_mask [S_q][S_kv], nonzero = masked out
 };
 
 // Unit number i of the schedule -> (b*N1 + h, q block): head-major, latest q block first.
@@ -106,7 +108,8 @@ __device__ __forceinline__ bool pair_sync(uint64_t* bar, int& exchanges, uint32_
   return ok;
 }
 
-template <int BN>
+// kMask: a dense atten_mask is applied (a separate instantiation keeps the mask-free loop unchanged)
+template <int BN, bool kMask>
 __global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -172,13 +175,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_v);
       int jk = 0, jv = 0, qcount = 0;  // K / V tiles issued, Q loads issued (this CTA)
       bool ok = true;
-      auto load_v = [&](int rp, int kv_row0, int j) -> bool {  // V of the unit's tile j (global jv)
+      // TMA coordinates (head dim, head, position, batch) of the 4-D maps
+      auto load_v = [&](int rp, int b, int g, int j) -> bool {  // V of the unit's tile j (global jv)
         const int sv = jv % kVStages, uv = jv / kVStages;
         if (jv >= kVStages && !mbar_wait(&s.bar_v_empty[sv], (uv - 1) & 1, prm.status)) return false;
-        const int vrow = kv_row0 + prm.col[rp + j] * prm.by;
+        const int vpos = prm.col[rp + j] * prm.by;
         mbar_arrive_expect_tx(&s.bar_v[sv], 2 * BN * 128);
-        tma_load_2d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, vrow);
-        tma_load_2d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, vrow);
+        tma_load_4d(s.v[sv][0], &tm_v, &s.bar_v[sv], 0, g, vpos, b);
+        tma_load_4d(s.v[sv][1], &tm_v, &s.bar_v[sv], 64, g, vpos, b);
         ++jv;
         return true;
       };
@@ -194,27 +198,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u.n == 0) continue;
         const int b = u.bh / prm.N1, h = u.bh % prm.N1;
         const int g = h / (prm.N1 / prm.N2);
-        const int q_row0 = u.bh * prm.S_q + u.qb * prm.bx;
-        const int kv_row0 = (b * prm.N2 + g) * prm.S_kv;
+        const int q_pos0 = u.qb * prm.bx;
         // Q: the previous unit's last S = Q K^T must have read the old Q
         if (qcount > 0 && !(ok = mbar_wait(&s.bar_q_empty, (qcount - 1) & 1, prm.status))) break;
         mbar_arrive_expect_tx(&s.bar_q, 2 * kBM * 128);
-        tma_load_2d(s.q[0], &tm_q, &s.bar_q, 0, q_row0);
-        tma_load_2d(s.q[1], &tm_q, &s.bar_q, 64, q_row0);
+        tma_load_4d(s.q[0], &tm_q, &s.bar_q, 0, h, q_pos0, b);
+        tma_load_4d(s.q[1], &tm_q, &s.bar_q, 64, h, q_pos0, b);
         ++qcount;
         // K runs up to kKStages tiles ahead, V trails K by one tile
         for (int j = 0; ok && j < u.n; ++j) {
-          const int row = kv_row0 + prm.col[u.rp + j] * prm.by;
+          const int kpos = prm.col[u.rp + j] * prm.by;
           const int sk = jk % kKStages, uk = jk / kKStages;
           if (jk >= kKStages && !(ok = mbar_wait(&s.bar_k_empty[sk], (uk - 1) & 1, prm.status))) break;
           mbar_arrive_expect_tx(&s.bar_k[sk], 2 * BN * 128);
-          tma_load_2d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, row);
-          tma_load_2d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, row);
+          tma_load_4d(s.k[sk][0], &tm_k, &s.bar_k[sk], 0, g, kpos, b);
+          tma_load_4d(s.k[sk][1], &tm_k, &s.bar_k[sk], 64, g, kpos, b);
           ++jk;
-          if (j >= kKStages - kVStages) ok = load_v(u.rp, kv_row0, j - (kKStages - kVStages));
+          if (j >= kKStages - kVStages) ok = load_v(u.rp, b, g, j - (kKStages - kVStages));
         }
         for (int j = u.n - (kKStages - kVStages); ok && j < u.n; ++j)
-          if (j >= 0) ok = load_v(u.rp, kv_row0, j);
+          if (j >= 0) ok = load_v(u.rp, b, g, j);
       }
       // do not leave the CTA with copies in flight
       for (int j = (jk > kKStages ? jk - kKStages : 0); j < jk; ++j)
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i < 0) break;
       const UnitInfo u = unit_info(prm, i);
       const int n = u.n, rp = u.rp, qb = u.qb;
-      const int q_row0 = u.bh * prm.S_q + qb * prm.bx;
+      const int ub = u.bh / prm.N1, uh = u.bh % prm.N1;
       const int qpos = qb * prm.bx + r;
       const bool row_valid = r < prm.bx && qpos < prm.S_q;
       // visible key interval [lo, hi] for this row (mask modes 0/2/3/4)
@@ -313,6 +316,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t s_col = st ? kColS1 : kColS0;
         const int kpos0 = prm.col[rp + j] * prm.by + hf * kHalf;
+        // the dense atten_mask inside the selected block: bit c = this row may not see column c
+        const uint64_t mbits = kMask && row_valid
+                                   ? dense_mask_bits<kHalf>(prm.amask + static_cast<size_t>(qpos) * prm.S_kv, kpos0,
+                                                           prm.S_kv)
+                                   : 0ull;
         float x[kHalf];  // raw scores
 #pragma unroll
         for (int c = 0; c < kHalf; c += 32) {
@@ -329,6 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kp = kpos0 + c;
             if (kp < lo || kp > hi) x[c] = -INFINITY;
           }
+        }
+        if (kMask && mbits != 0) {
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c)
+            if ((mbits >> c) & 1ull) x[c] = -INFINITY;
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -461,14 +474,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (warp == 0 && lane == 0) {
         ok = mbar_wait(&s.bar_epi, k & 1, prm.status);
         if (ok) {
-          tma_store_3d(&tm_o, s.ostage[0], 0, qb * prm.bx, u.bh);
-          tma_store_3d(&tm_o, s.ostage[1], 64, qb * prm.bx, u.bh);
+          tma_store_4d(&tm_o, s.ostage[0], 0, uh, qb * prm.bx, ub);
+          tma_store_4d(&tm_o, s.ostage[1], 64, uh, qb * prm.bx, ub);
           bulk_commit();  // read completion is awaited at the next unit's epilogue, off the critical path
         }
       }
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      if (row_valid && hf == 0) prm.lse[q_row0 + r] = any ? (m * kLn2 + logf(l)) : -INFINITY;
+      if (row_valid && hf == 0)
+        prm.lse[ub * prm.lse_sb + uh * prm.lse_sh + qpos * prm.lse_ss] = any ? (m * kLn2 + logf(l)) : -INFINITY;
       // O has been read: the next unit's first O += P V waits for P, which comes after this
       tc_fence_before();
       J0 += n;
@@ -483,15 +497,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int BN>
 cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
-  const uint64_t q_rows = static_cast<uint64_t>(a.B) * a.N1 * a.S_q;
-  const uint64_t kv_rows = static_cast<uint64_t>(a.B) * a.N2 * a.S_kv;
-  if (!make_tmap_2d_bf16(&tq, q, q_rows, kD, kD, kBM)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d_bf16(&tk, k, kv_rows, kD, kD, BN)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d_bf16(&tv, v, kv_rows, kD, kD, BN)) return cudaErrorInvalidValue;
-  CUtensorMap to;  // Out as [B*N1][S_q][128], box {64, block_x, 1}
-  if (!make_tmap_3d_bf16(&to, a.out, kD, a.S_q, static_cast<uint64_t>(a.B) * a.N1, kD,
-                         static_cast<uint64_t>(a.S_q) * kD, a.bx, 1))
+  // Q, K, V and Out as (head dim, head, position, batch), whichever of BNSD / BSND is in memory;
+  // the Out box stops at the q block (block_x rows) and the tensor's positions
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_4d_bf16(&tq, q, kD, a.N1, a.S_q, a.B, a.qs.h, a.qs.s, a.qs.b, kBM) ||
+      !make_tmap_4d_bf16(&tk, k, kD, a.N2, a.S_kv, a.B, a.kvs.h, a.kvs.s, a.kvs.b, BN) ||
+      !make_tmap_4d_bf16(&tv, v, kD, a.N2, a.S_kv, a.B, a.kvs.h, a.kvs.s, a.kvs.b, BN) ||
+      !make_tmap_4d_bf16(&to, a.out, kD, a.N1, a.S_q, a.B, a.qs.h, a.qs.s, a.qs.b, a.bx))
     return cudaErrorInvalidValue;
   FwdParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.S_q = a.S_q; p.S_kv = a.S_kv; p.bx = a.bx; p.by = a.by;
@@ -501,8 +513,11 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   p.row_ptr = a.row_ptr; p.col = a.col;
   p.out = static_cast<__nv_bfloat16*>(a.out); p.lse = a.lse; p.next_unit = a.next_unit; p.status = a.status;
   p.cta_clock = nullptr;
+  p.lse_sb = a.lse_s.b; p.lse_sh = a.lse_s.h; p.lse_ss = a.lse_s.s;
+  p.amask = a.atten_mask;
   const size_t smem = sizeof(FwdSmem<BN>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kernel = a.atten_mask ? bsa_fwd_kernel<BN, true> : bsa_fwd_kernel<BN, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (p.units == 0) return cudaSuccess;
   int dev = 0, sms = 148;
@@ -511,7 +526,7 @@ cudaError_t launch_fwd(const BsaFwdArgs& a, const void* q, const void* k, const 
   const int grid = p.units < sms ? p.units : sms;  // persistent: one CTA per SM
   p.cta_clock = prof_cta_clock(0, grid);
   prof_begin("bsa_fwd", st);
-  e = launch_pdl(bsa_fwd_kernel<BN>, dim3(grid), dim3(kThreads), smem, st, tq, tk, tv, to, p);
+  e = launch_pdl(kernel, dim3(grid), dim3(kThreads), smem, st, tq, tk, tv, to, p);
   prof_end(st);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -181,6 +181,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 // Contiguous bulk copy global -> shared (src and dst 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -194,6 +202,12 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
                "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -346,6 +360,30 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 // swizzle (16-byte chunk index XOR row % 8), tile base 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
+}
+
+// Dense atten_mask: bits of N <= 64 bytes row[kp0 .. kp0 + n) of a dense atten_mask row (bit c set: byte nonzero);
+// bytes at or past `len` count as 0.  16-byte loads when the run is aligned and inside the row.
+template <int N>
+__device__ __forceinline__ uint64_t dense_mask_bits(const uint8_t* __restrict__ row, int kp0, int len) {
+  uint64_t bits = 0;
+  if (kp0 + N <= len && (reinterpret_cast<uintptr_t>(row + kp0) & 15u) == 0) {
+#pragma unroll
+    for (int c = 0; c < N; c += 16) {
+      const uint4 w = *reinterpret_cast<const uint4*>(row + kp0 + c);
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t nz = __vcmpne4(wv[e], 0u);  // 0xFF in each nonzero byte
+        const uint32_t b4 = (nz & 1u) | ((nz >> 7) & 2u) | ((nz >> 14) & 4u) | ((nz >> 21) & 8u);
+        bits |= static_cast<uint64_t>(b4) << (c + 4 * e);
+      }
+    }
+  } else {
+    for (int c = 0; c < N; ++c)
+      if (kp0 + c < len && row[kp0 + c] != 0) bits |= 1ull << c;
+  }
+  return bits;
 }
 
 // ---- programmatic dependent launch ---------------------------------------------------------------

@@ -594,3 +594,29 @@ def test_backward_with_given_attention_out():
                                          out_in=r_out[0].transpose(1, 0, 2) + Et)
     assert np.allclose(ndq, (r_dq - sc * dD[..., None] * (p @ k))[0].transpose(1, 0, 2), atol=1e-11)
     assert np.allclose(ndv, r_dv[0].transpose(1, 0, 2), atol=1e-11)
+
+
+@pytest.mark.parametrize("mode,s_q,s_kv", [(2, 48, 48), (0, 40, 56), (3, 32, 48)])
+def test_bsa_dense_atten_mask_matches_sdpa(mode, s_q, s_kv):
+    """The dense atten_mask ([S_q, S_kv], nonzero = masked out) on top of the block selection and
+    the mode: forward and gradients equal torch SDPA (float64) under the combined boolean mask;
+    rows the mask leaves without a key give Out = 0, LSE = -inf and zero dQ."""
+    rng = np.random.default_rng(15)
+    B, N1, N2, D, bx, by = 1, 2, 1, 8, 8, 8
+    q, do = _rand(rng, B, N1, s_q, D), _rand(rng, B, N1, s_q, D)
+    k, v = _rand(rng, B, N2, s_kv, D), _rand(rng, B, N2, s_kv, D)
+    nqb, nkb = -(-s_q // bx), -(-s_kv // by)
+    mask = (rng.random((B, N1, nqb, nkb)) < 0.7).astype(np.uint8)
+    am = (rng.random((s_q, s_kv)) < 0.3).astype(np.uint8)
+    am[5] = 1  # a row with no key left
+    dense = _dense_mask_bsa(mask, bx, by, s_q, s_kv, mode) & (am == 0)[None, None]
+    dq, dk, dv, out, lse = A.bsa_backward(q, k, v, do, mask, bx, by, mode, 0.4, atten_mask=am)
+    live = dense.any(-1)                                     # [B, N1, S_q]
+    assert not live[..., 5].any()
+    r_out, r_lse, r_dq, r_dk, r_dv = _torch_sdpa(q, k, v, np.where(live[..., None], dense, True), 0.4,
+                                                 np.where(live[..., None], do, 0.0))
+    assert np.allclose(out[live], r_out[live], atol=1e-12)
+    assert np.allclose(lse[live], r_lse[live], atol=1e-12)
+    assert np.all(out[~live] == 0) and np.all(np.isneginf(lse[~live])) and np.all(dq[~live] == 0)
+    assert np.allclose(dq, np.where(live[..., None], r_dq, 0.0), atol=1e-11)
+    assert np.allclose(dk, r_dk, atol=1e-11) and np.allclose(dv, r_dv, atol=1e-11)
