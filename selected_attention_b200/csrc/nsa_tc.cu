@@ -17,10 +17,10 @@
 // memory; 8 chunks make a 128-key tile, loaded by TMA ({64 dims, 1 head, 16 tokens} boxes, 128-byte
 // swizzle) into K and V rings.  A tile's unused chunk slots repeat its first chunk and are masked.
 //
-// Warps: 0-3 softmax (TMEM lane quarter = 32 keys, or 32 rows of the accumulator in the epilogue),
-// 4 builds the item lists (up to two items ahead) and loads Q (dO), 5 and 6 load the K and V tiles
-// (each on its own ring, so K runs ahead of the V slots the later products still hold), 7 issues
-// S^T (and dP^T), 8 issues O^T (dQ^T).  Persistent CTAs take items round-robin.  Every wait is
+// Warps: 0-15 softmax (TMEM lane quarter = 32 keys, or 32 rows of the accumulator in the epilogue,
+// and a quarter of the tile's heads), 16 builds the item lists (up to two items ahead) and loads Q
+// (dO), 17 and 18 load the K and V tiles (each on its own ring, so K runs ahead of the V slots the
+// later products still hold), 19 issues S^T (and dP^T), 20 issues O^T (dQ^T).  Persistent CTAs take items round-robin.  Every wait is
 // bounded; on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -33,11 +33,14 @@ namespace {
 
 constexpr int kTok = 128;     // keys per tile: MMA M
 constexpr int kD = 128;       // head dim of q / k / v
-constexpr int kChunk = 16;    // keys per TMA box
-constexpr int kChunksPerTile = kTok / kChunk;
+// Keys per gather chunk (one TMA box per head-dim half): 64 when the selected block size is a
+// multiple of 64 (a block's visible prefix then ends inside its last chunk and is masked there),
+// else 16.  A 128-key tile holds kTok / chunk chunks.
 constexpr int kMaxChunks = 512;  // count * size <= 8192 keys per (token, kv head)
-constexpr int kSoftWarps = 4;
-// warps: 0-3 softmax, 4 item lists + Q loads, 5 K producer, 6 V producer, 7 S^T issuer, 8 O^T issuer
+constexpr int kSoftWarps = 16;
+constexpr int kHeadGroups = kSoftWarps / 4;
+// warps: 0-15 softmax (lane quarter = warp % 4, head group = warp / 4), 16 item lists + Q loads,
+// 17 K producer, 18 V producer, 19 S^T issuer, 20 O^T issuer
 constexpr int kWList = kSoftWarps, kWK = kSoftWarps + 1, kWV = kSoftWarps + 2, kWS = kSoftWarps + 3,
               kWO = kSoftWarps + 4;
 constexpr int kThreads = (kSoftWarps + 5) * 32;
@@ -73,8 +76,8 @@ struct __align__(1024) TcSmem {
   alignas(1024) uint8_t p[2][kDq ? 2 : 1][2][NH * 128];
   alignas(1024) uint8_t dout[kDq ? 2 : 1][2][kDq ? NH * 128 : 16];  // dQ pass only
   ItemDesc desc[2];
-  float red[2][kSoftWarps][NH];              // per tile parity: column maxima of each lane quarter
-  float red_l[kSoftWarps][NH];
+  float red[2][4][NH];                       // per tile parity: column maxima of each lane quarter
+  float red_l[4][NH];
   uint64_t bar_desc_full[2], bar_desc_empty[2];
   uint64_t bar_q[2], bar_q_empty[2];
   uint64_t bar_k[TcCfg<kDq, NH>::kKR], bar_k_empty[TcCfg<kDq, NH>::kKR];
@@ -88,6 +91,7 @@ struct __align__(1024) TcSmem {
 
 struct TcParams {
   int B, T, N1, N2, G, K, sel_block, mask_mode, head_tiles;
+  int chunk, chunk_shift;  // keys per gather chunk (16 or 64) and its log2
   long long items;
   float scale, scale_log2;
   const int32_t* cu;
@@ -118,15 +122,32 @@ __device__ __forceinline__ int batch_of(const int32_t* __restrict__ cu, int B, i
 }
 
 // NH consecutive 32-bit TMEM columns of this thread's lane (NH = 16 or 32)
-template <int NH>
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[NH]) {
-  if constexpr (NH == 16) tmem_ld16(taddr, r);
-  else tmem_ld32(taddr, r);
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
 }
-template <int NH>
-__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&r)[NH]) {
-  if constexpr (NH == 16) tmem_st16(taddr, r);
-  else tmem_st32(taddr, r);
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+template <int N>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 4) tmem_ld4(taddr, r);
+  else if constexpr (N == 8) tmem_ld8(taddr, r);
+  else tmem_ld16(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 4) tmem_st4(taddr, r);
+  else if constexpr (N == 8) tmem_st8(taddr, r);
+  else tmem_st16(taddr, r);
 }
 
 // byte offset of (row, 16-byte chunk) in a [rows][128 B] tile written with the 128-byte swizzle
@@ -212,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int last_key = prm.mask_mode == 2 ? pos : len - 1;
       const int n_sel = prm.cnt[static_cast<size_t>(t) * prm.N2 + g];
       const int32_t* sel = prm.ids + (static_cast<size_t>(t) * prm.N2 + g) * prm.K;
-      const int cpb = prm.sel_block / kChunk;
+      const int cpb = prm.sel_block >> prm.chunk_shift;
       ItemDesc& d = s.desc[slot];
       // visible chunks of each listed block (a prefix of its chunks), laid out in list order
       int base = 0;
@@ -220,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = i0 + lane;
         const int j = i < n_sel ? sel[i] : -1;
         const int first = j * prm.sel_block;
-        const int nc = (j >= 0 && first <= last_key) ? min(cpb, (last_key - first) / kChunk + 1) : 0;
+        const int nc = (j >= 0 && first <= last_key) ? min(cpb, ((last_key - first) >> prm.chunk_shift) + 1) : 0;
         int incl = nc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -228,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane >= o) incl += y;
         }
         const int at = base + incl - nc;
-        for (int c = 0; c < nc; ++c) d.kp0[at + c] = first + c * kChunk;
+        for (int c = 0; c < nc; ++c) d.kp0[at + c] = first + (c << prm.chunk_shift);
         base += __shfl_sync(0xffffffffu, incl, 31);
       }
       const int h0 = g * prm.G + ht * NH;
@@ -280,10 +301,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = __all_sync(0xffffffffu, desc_wait(k)))) break;
       const ItemDesc& d = s.desc[slot];
       const int n_vis = d.n_vis, t0 = d.t0, g = d.g;
-      const int n_tiles = (n_vis + kChunksPerTile - 1) / kChunksPerTile;
+      const int cpt = kTok >> prm.chunk_shift;  // chunks per tile
+      const int n_tiles = (n_vis + cpt - 1) / cpt;
       for (int j = 0; ok && j < n_tiles; ++j, ++use) {
-        const int c = j * kChunksPerTile + (lane & 7);
-        const int tok = t0 + (lane < 8 ? d.kp0[c < n_vis ? c : j * kChunksPerTile] : 0);
+        const int c = j * cpt + (lane & 7);
+        const int tok = t0 + (lane < cpt ? d.kp0[c < n_vis ? c : j * cpt] : 0);
         const int st = static_cast<int>(use % R);
         if (lane == 0 && use >= R) ok = mbar_wait(&empty[st], ((use / R) - 1) & 1, prm.status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -291,9 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = is_k ? s.k[st % kRK][0] : s.v[st % kRV][0];
         if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
         __syncwarp();
-        if (lane < 8) {
-          tma_load_3d(dst + lane * kChunk * 128, map, &full[st], 0, g, tok);
-          tma_load_3d(dst + kTileBytes + lane * kChunk * 128, map, &full[st], 64, g, tok);
+        if (lane < cpt) {
+          tma_load_3d(dst + lane * prm.chunk * 128, map, &full[st], 0, g, tok);
+          tma_load_3d(dst + kTileBytes + lane * prm.chunk * 128, map, &full[st], 64, g, tok);
         }
       }
       __syncwarp();
@@ -317,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = desc_wait(k))) break;
         const int n_vis = s.desc[slot].n_vis;
         mbar_arrive(&s.bar_desc_empty[slot]);
-        const int n_tiles = (n_vis + kChunksPerTile - 1) / kChunksPerTile;
+        const int n_tiles = (n_vis + (kTok >> prm.chunk_shift) - 1) / (kTok >> prm.chunk_shift);
         // every item's Q slot is loaded (and released below), with or without tiles
         if (!(ok = mbar_wait(&s.bar_q[slot], (k >> 1) & 1, prm.status))) break;
         const uint64_t dq = dq0 + static_cast<uint64_t>(slot) * ((2 * NH * 128) >> 4);
@@ -367,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = desc_wait(k))) break;
         const int n_vis = s.desc[slot].n_vis;
         mbar_arrive(&s.bar_desc_empty[slot]);
-        const int n_tiles = (n_vis + kChunksPerTile - 1) / kChunksPerTile;
+        const int n_tiles = (n_vis + (kTok >> prm.chunk_shift) - 1) / (kTok >> prm.chunk_shift);
         if (n_tiles == 0) continue;
         // the accumulator is overwritten by this item's first product: the epilogue of the last item
         // with tiles has read it (exact parity: acc_free's next phase needs this item's products)
@@ -397,7 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    const int quarter = warp;
+    // warp = (head group hg, lane quarter): its 32 keys of a tile (TMEM lanes) and HW = NH / 4 of
+    // the heads (TMEM columns), so each tile's chain is split over four warps per sub-partition
+    constexpr int HW = NH / kHeadGroups;
+    const int quarter = warp & 3, hg = warp >> 2;
+    const int hb = hg * HW;             // this warp's first head of the tile
     const int r = quarter * 32 + lane;  // key row of a tile == TMEM lane (and accumulator row)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     bool ok = true;
@@ -408,30 +434,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = __all_sync(0xffffffffu, desc_wait(k)))) break;
       const ItemDesc& d = s.desc[slot];
       const int n_vis = d.n_vis, pos = d.pos, len = d.len, rows = d.rows, h0 = d.h0, t = d.t;
-      const int n_tiles = (n_vis + kChunksPerTile - 1) / kChunksPerTile;
-      float m[NH], l[NH];
+      const int cpt = kTok >> prm.chunk_shift;  // chunks per tile
+      const int n_tiles = (n_vis + cpt - 1) / cpt;
+      float m[HW], l[HW];
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
+      for (int h = 0; h < HW; ++h) {
         m[h] = -INFINITY;
         l[h] = 0.f;
       }
       for (int j = 0; j < n_tiles; ++j, ++J) {
         const int st = static_cast<int>(J & 1);
-        const int c = j * kChunksPerTile + (r >> 4);
-        const int kpos = c < n_vis ? d.kp0[c] + (r & 15) : 0x7fffffff;
+        const int c = j * cpt + (r >> prm.chunk_shift);
+        const int kpos = c < n_vis ? d.kp0[c] + (r & (prm.chunk - 1)) : 0x7fffffff;
         const bool vis = kpos < len && (prm.mask_mode != 2 || kpos <= pos);
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (J >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
-        float x[NH];
-        uint32_t dpr[NH];
+        float x[HW];
+        uint32_t dpr[HW];
         {
-          uint32_t rr[NH];
-          tmem_ld_row<NH>(tmem + lane_base + kColS + st * NH, rr);
-          if constexpr (kDq) tmem_ld_row<NH>(tmem + lane_base + kColDP + st * NH, dpr);
+          uint32_t rr[HW];
+          tmem_ld_row<HW>(tmem + lane_base + kColS + st * NH + hb, rr);
+          if constexpr (kDq) tmem_ld_row<HW>(tmem + lane_base + kColDP + st * NH + hb, dpr);
           tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
+          for (int h = 0; h < HW; ++h) {
             reg_fence(rr[h]);
             if (kDq) reg_fence(dpr[h]);
             x[h] = vis ? __uint_as_float(rr[h]) * prm.scale_log2 : -INFINITY;
@@ -442,9 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!kDq) {
           // column maxima of the tile: over the warp's 32 keys, then over the four lane quarters
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
+          for (int h = 0; h < HW; ++h) {
             const float mx = warp_max(x[h]);
-            if (lane == 0) s.red[st][quarter][h] = mx;
+            if (lane == 0) s.red[st][quarter][hb + h] = mx;
           }
           mbar_arrive(&s.bar_x);
           ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_x, xph & 1, prm.status));
@@ -458,13 +485,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
         }
         bool any = false;
-        float alpha[NH];
+        float alpha[HW];
         if (!kDq) {
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            const float tm = fmaxf(fmaxf(s.red[st][0][h], s.red[st][1][h]), fmaxf(s.red[st][2][h], s.red[st][3][h]));
+          for (int h = 0; h < HW; ++h) {
+            const float tm = fmaxf(fmaxf(s.red[st][0][hb + h], s.red[st][1][hb + h]),
+                                   fmaxf(s.red[st][2][hb + h], s.red[st][3][hb + h]));
             alpha[h] = 1.f;
-            if (tm > m[h] + kLazy) {  // uniform over the CTA
+            if (tm > m[h] + kLazy) {  // uniform over the warps of this head group
               alpha[h] = ex2(m[h] - tm);
               l[h] *= alpha[h];
               m[h] = tm;
@@ -476,37 +504,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int khalf = r >> 6, kcol = r & 63;
         uint8_t* pb = s.p[st][0][khalf];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          const uint32_t off = sw128(h, kcol >> 3) + (kcol & 7) * 2;
+        for (int h = 0; h < HW; ++h) {
+          const uint32_t off = sw128(hb + h, kcol >> 3) + (kcol & 7) * 2;
           if (!kDq) {
             const float mu = m[h] == -INFINITY ? 0.f : m[h];
             const float e = ex2(x[h] - mu);
             l[h] += e;
             *reinterpret_cast<__nv_bfloat16*>(pb + off) = __float2bfloat16_rn(e);
           } else {
-            const float p = vis ? ex2(x[h] - d.lse2[h]) : 0.f;  // per-head values read from shared memory
-            const float ds = p * (__uint_as_float(dpr[h]) - d.dvec[h]);
+            const float p = vis ? ex2(x[h] - d.lse2[hb + h]) : 0.f;  // per-head values from shared memory
+            const float ds = p * (__uint_as_float(dpr[h]) - d.dvec[hb + h]);
             const __nv_bfloat16 hi = __float2bfloat16_rn(ds);
             const __nv_bfloat16 lo = __float2bfloat16_rn(ds - __bfloat162float(hi));
             *reinterpret_cast<__nv_bfloat16*>(pb + off) = hi;
             *reinterpret_cast<__nv_bfloat16*>(s.p[st][kDq ? 1 : 0][khalf] + off) = lo;
           }
         }
-        if (!kDq && any && j > 0) {
-          // rescale O^T's columns (accumulator row r) once the product of tile J-1 has completed
-          // (exact parity: that buffer's next product needs P of tile J+1, written after this)
+        if (!kDq && __any_sync(0xffffffffu, any) && j > 0) {
+          // rescale this head group's O^T columns (accumulator row r) once the product of tile J-1
+          // has completed (exact parity: that buffer's next product needs P of tile J+1)
           ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[st ^ 1], ((J - 1) >> 1) & 1, prm.status));
           if (!ok) break;
           tc_fence_after();
-          uint32_t rr[NH];
-          tmem_ld_row<NH>(tmem + lane_base + kColAcc, rr);
+          uint32_t rr[HW];
+          tmem_ld_row<HW>(tmem + lane_base + kColAcc + hb, rr);
           tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
+          for (int h = 0; h < HW; ++h) {
             reg_fence(rr[h]);
             rr[h] = __float_as_uint(__uint_as_float(rr[h]) * alpha[h]);
           }
-          tmem_st_row<NH>(tmem + lane_base + kColAcc, rr);
+          tmem_st_row<HW>(tmem + lane_base + kColAcc + hb, rr);
           tmem_st_wait();
         }
         fence_async_smem();
@@ -515,59 +543,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue of the item: accumulator row r = dv (d) index, columns = heads
-      float L[NH];
+      float L[HW];
       if (!kDq) {
         // l over the 128 keys of each head: warp sums, then the four quarters
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
+        for (int h = 0; h < HW; ++h) {
           float v = l[h];
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) s.red_l[quarter][h] = v;
+          if (lane == 0) s.red_l[quarter][hb + h] = v;
         }
         mbar_arrive(&s.bar_x);
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_x, xph & 1, prm.status));
         ++xph;
         if (!ok) break;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) L[h] = (s.red_l[0][h] + s.red_l[1][h]) + (s.red_l[2][h] + s.red_l[3][h]);
+        for (int h = 0; h < HW; ++h)
+          L[h] = (s.red_l[0][hb + h] + s.red_l[1][hb + h]) + (s.red_l[2][hb + h] + s.red_l[3][hb + h]);
       }
-      uint32_t acc[NH];
+      uint32_t acc[HW];
       if (n_tiles > 0) {
         const long long jl = J - 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[jl & 1], (jl >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
-        tmem_ld_row<NH>(tmem + lane_base + kColAcc, acc);
+        tmem_ld_row<HW>(tmem + lane_base + kColAcc + hb, acc);
         tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < NH; ++h) reg_fence(acc[h]);
+        for (int h = 0; h < HW; ++h) reg_fence(acc[h]);
         tc_fence_before();
         mbar_arrive(&s.bar_acc_free);
       } else {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) acc[h] = 0u;
+        for (int h = 0; h < HW; ++h) acc[h] = 0u;
       }
       // the descriptor slot is no longer needed
       mbar_arrive(&s.bar_desc_empty[slot]);
       __nv_bfloat16* base = prm.out + static_cast<size_t>(t) * prm.N1 * kD;
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        if (h >= rows) break;
+      for (int h = 0; h < HW; ++h) {
+        if (hb + h >= rows) break;
         float mul;
         if (kDq) mul = prm.scale;
         else mul = L[h] > 0.f ? 1.f / L[h] : 0.f;
-        base[static_cast<size_t>(h0 + h) * kD + r] = __float2bfloat16_rn(__uint_as_float(acc[h]) * mul);
+        base[static_cast<size_t>(h0 + hb + h) * kD + r] = __float2bfloat16_rn(__uint_as_float(acc[h]) * mul);
       }
-      if (!kDq && quarter == 0 && lane < rows && lane < NH) {
+      if (!kDq && quarter == 0 && lane < HW && hb + lane < rows) {
         float mh = m[0], lh = L[0];
 #pragma unroll
-        for (int h = 1; h < NH; ++h)
+        for (int h = 1; h < HW; ++h)
           if (lane == h) {
             mh = m[h];
             lh = L[h];
           }
-        prm.lse_out[static_cast<size_t>(t) * prm.N1 + h0 + lane] = lh > 0.f ? (mh * kLn2 + logf(lh)) : -INFINITY;
+        prm.lse_out[static_cast<size_t>(t) * prm.N1 + h0 + hb + lane] = lh > 0.f ? (mh * kLn2 + logf(lh)) : -INFINITY;
       }
     }
   }
@@ -583,8 +612,8 @@ cudaError_t launch_tc(const NsaArgs& a, const TcParams& p, const char* name, cud
   const uint64_t hs = static_cast<uint64_t>(a.N2) * kD;
   if (!make_tmap_2d_bf16(&tq, a.q, qrows, kD, kD, NH) ||
       !make_tmap_2d_bf16(&tdo, kDq ? a.dout : a.q, qrows, kD, kD, NH) ||
-      !make_tmap_3d_bf16(&tk, a.k, kD, a.N2, a.T, kD, hs, 1, kChunk) ||
-      !make_tmap_3d_bf16(&tv, a.v, kD, a.N2, a.T, kD, hs, 1, kChunk))
+      !make_tmap_3d_bf16(&tk, a.k, kD, a.N2, a.T, kD, hs, 1, p.chunk) ||
+      !make_tmap_3d_bf16(&tv, a.v, kD, a.N2, a.T, kD, hs, 1, p.chunk))
     return cudaErrorInvalidValue;
   static_assert(sizeof(TcSmem<kDq, NH>) + 1024 <= 227 * 1024, "shared memory of one CTA (227 KB on sm_100)");
   const size_t smem = sizeof(TcSmem<kDq, NH>) + 1024;
@@ -605,6 +634,8 @@ TcParams tc_params(const NsaArgs& a, int NH) {
   TcParams p;
   p.B = a.B; p.T = a.T; p.N1 = a.N1; p.N2 = a.N2; p.G = a.N1 / a.N2; p.K = a.K; p.sel_block = a.sel_block;
   p.mask_mode = a.mask_mode; p.head_tiles = (p.G + NH - 1) / NH;
+  p.chunk = a.sel_block % 64 == 0 ? 64 : 16;
+  p.chunk_shift = p.chunk == 64 ? 6 : 4;
   p.items = static_cast<long long>(a.T) * a.N2 * p.head_tiles;
   p.scale = a.scale; p.scale_log2 = a.scale * kLog2e;
   p.cu = a.cu_seqlens; p.ok_flag = a.ok_flag; p.ids = a.ids; p.cnt = a.cnt;
