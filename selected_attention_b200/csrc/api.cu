@@ -60,6 +60,7 @@ struct BsaBwdWs {
   uint8_t* maskT;
   int32_t *t_counts, *t_row_ptr, *t_col;
   float *dvec, *lse2;
+  uint16_t *q16, *k16, *v16, *do16;
 };
 
 size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
@@ -77,6 +78,12 @@ size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
   w->t_col = c.take<int32_t>(units * nkb);
   w->dvec = c.take<float>(units * 128);
   w->lse2 = c.take<float>(units * 128);
+  const size_t nq = static_cast<size_t>(p->B) * p->N1 * p->S_q * p->D;
+  const size_t nk = static_cast<size_t>(p->B) * p->N2 * p->S_kv * p->D;
+  w->q16 = c.take<uint16_t>(nq);
+  w->do16 = c.take<uint16_t>(nq);
+  w->k16 = c.take<uint16_t>(nk);
+  w->v16 = c.take<uint16_t>(nk);
   return c.bytes();
 }
 
@@ -316,6 +323,8 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
   a.atten_mask = p->atten_mask;
   a.row_ptr = w.row_ptr; a.col = w.col; a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;
   a.dvec = w.dvec; a.lse2 = w.lse2; a.dq = dq; a.dk = dk; a.dv = dv; a.status = w.status;
+  a.q16 = w.q16; a.k16 = w.k16; a.v16 = w.v16; a.do16 = w.do16;
+  a.amax = reinterpret_cast<WsHeader*>(w.status)->amax;
   a.next_kv = &reinterpret_cast<WsHeader*>(w.status)->next_bwd_kv;
   a.next_q = &reinterpret_cast<WsHeader*>(w.status)->next_bwd_q;
   return cuda_status(bsa_bwd_launch(a, q, k, v, out, dout, lse, st));

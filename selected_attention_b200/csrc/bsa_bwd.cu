@@ -3,8 +3,18 @@
 //   dV = P^T dOut;  dQ = (dS K) scale;  dK = (dS^T Q) scale
 // P is recomputed from the forward's LSE: P = exp(scale q.k - LSE).
 //
-// Three kernels, no atomics (run-to-run bit identical):
-//   bwd_prep     softmax_grad (D) and LSE*log2(e) per query row, written into 128-row padded
+// Operands: the passes run their products on fp16 copies of Q, K, V and dOut, each scaled by a
+// power of two s_x (1 when 2^-8 <= max|x| < 2^14, else chosen so max|x| s_x <= 2^14; bf16 values have
+// 8 significant bits, so the copies are exact unless a value falls below fp16's normal range); P (in [0, 1]) and dS (scaled by a power of
+// two from the bound |dS| <= 256 max|dOut| max|V|) enter the gradient products as single fp16
+// operands, 11 significant bits.  The scales are undone in fp32: in the exponent of P, on dP
+// before dS, and in the dQ / dK / dV epilogues (all exact, being powers of two).
+//
+// Kernels, no atomics on the results (run-to-run bit identical):
+//   bwd_to_f16   fp16 copies of Q, K, V, dOut and their max |x| (an integer atomic max on the float
+//                bits: order-free); bwd_f16_fixup re-converts, scaled, a tensor whose max lies
+//                outside [2^-8, 2^14), and returns at once otherwise.
+//   bwd_prep     softmax_grad (D, times the dS scale) and LSE*log2(e) per query row, written into 128-row padded
 //                tiles so the passes below can bulk-load a tile's vectors.
 //   bwd_kv       one CTA per KV block (b, g, kb) walking its transposed list of Q tiles (the
 //                group's query heads included, in a fixed order): S^T = K Q^T, P^T, dP^T = V dO^T,
@@ -27,13 +37,106 @@ constexpr int kThreads = (kVecWarps + 2) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------------------------------------
+// fp16 operand copies
+// ------------------------------------------------------------------------------------------------
+// The four tensors of the backward's products, blockIdx.y = 0 Q, 1 K, 2 V, 3 dOut; n8 = elements / 8.
+struct F16Copy {
+  const uint4* src[4];
+  uint4* dst[4];
+  long long n8[4];
+};
+
+__device__ __forceinline__ float bf16_pair_absmax(uint32_t w) {
+  return fmaxf(fabsf(bf16lo(w)), fabsf(bf16hi(w)));
+}
+
+// Plain conversion (scale 1) of the four tensors and their max |x| in one sweep.
+__global__ void bwd_to_f16_kernel(const F16Copy c, uint32_t* __restrict__ amax) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int t = blockIdx.y;
+  // selected by comparisons, not a dynamic index, so the parameter block is not copied to local memory
+  const uint4* __restrict__ src = t == 0 ? c.src[0] : t == 1 ? c.src[1] : t == 2 ? c.src[2] : c.src[3];
+  uint4* __restrict__ dst = t == 0 ? c.dst[0] : t == 1 ? c.dst[1] : t == 2 ? c.dst[2] : c.dst[3];
+  const long long n8 = t == 0 ? c.n8[0] : t == 1 ? c.n8[1] : t == 2 ? c.n8[2] : c.n8[3];
+  float m = 0.f;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 w = src[i];
+    m = fmaxf(m, fmaxf(fmaxf(bf16_pair_absmax(w.x), bf16_pair_absmax(w.y)),
+                       fmaxf(bf16_pair_absmax(w.z), bf16_pair_absmax(w.w))));
+    uint4 o;
+    o.x = pack_f16(bf16lo(w.x), bf16hi(w.x));
+    o.y = pack_f16(bf16lo(w.y), bf16hi(w.y));
+    o.z = pack_f16(bf16lo(w.z), bf16hi(w.z));
+    o.w = pack_f16(bf16lo(w.w), bf16hi(w.w));
+    dst[i] = o;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(&amax[t], __float_as_uint(m));  // m >= 0: bits order as values
+}
+
+// The per-tensor scales and the factors that undo them.
+struct BwdScales {
+  float s[4];    // Q, K, V, dOut copy scales
+  float s_ds;    // dS scale
+  float c_s;     // multiplies a score accumulator: scale * log2(e) / (s_Q s_K)
+  float c_dp;    // multiplies a dP accumulator: s_dS / (s_dO s_V)
+  float dq_mul;  // dQ = acc * scale / (s_dS s_K)
+  float dk_mul;  // dK = acc * scale / (s_dS s_Q)
+  float dv_mul;  // dV = acc / s_dO
+};
+
+__device__ __forceinline__ BwdScales bwd_scales(const uint32_t* __restrict__ amax, float scale, float scale_log2) {
+  BwdScales r;
+  float a[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    a[t] = __uint_as_float(amax[t]);
+    r.s[t] = copy_scale(a[t]);
+  }
+  r.s_ds = pow2_scale(256.f * a[3] * a[2]);
+  r.c_s = scale_log2 / (r.s[0] * r.s[1]);
+  r.c_dp = r.s_ds / (r.s[3] * r.s[2]);
+  r.dq_mul = scale / (r.s_ds * r.s[1]);
+  r.dk_mul = scale / (r.s_ds * r.s[0]);
+  r.dv_mul = 1.f / r.s[3];
+  return r;
+}
+
+// Re-conversion of a tensor whose max |x| asks for a scale other than 1 (very large or very small
+// values); the whole grid returns at once otherwise.
+__global__ void bwd_f16_fixup_kernel(const F16Copy c, const uint32_t* __restrict__ amax) {
+  griddep_wait();  // the conversion and its maxima must be complete
+  griddep_launch_dependents();
+  const int t = blockIdx.y;
+  const float sc = copy_scale(__uint_as_float(amax[t]));
+  if (sc == 1.f) return;
+  const uint4* __restrict__ src = t == 0 ? c.src[0] : t == 1 ? c.src[1] : t == 2 ? c.src[2] : c.src[3];
+  uint4* __restrict__ dst = t == 0 ? c.dst[0] : t == 1 ? c.dst[1] : t == 2 ? c.dst[2] : c.dst[3];
+  const long long n8 = t == 0 ? c.n8[0] : t == 1 ? c.n8[1] : t == 2 ? c.n8[2] : c.n8[3];
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 w = src[i];
+    uint4 o;
+    o.x = pack_f16(bf16lo(w.x) * sc, bf16hi(w.x) * sc);
+    o.y = pack_f16(bf16lo(w.y) * sc, bf16hi(w.y) * sc);
+    o.z = pack_f16(bf16lo(w.z) * sc, bf16hi(w.z) * sc);
+    o.w = pack_f16(bf16lo(w.w) * sc, bf16hi(w.w) * sc);
+    dst[i] = o;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // preprocess: -D_i = -sum_d dOut_id Out_id ; -L2_i = -LSE_i * log2(e)  (-inf where the row has no
 // key or the tile row is padding, which makes exp2(s + (-L2)) = 0 there).  Stored negated so that
 // P = exp2(s * scale * log2(e) + (-L2)) is one fused multiply-add and dS = P * (dP + (-D)).
 // ------------------------------------------------------------------------------------------------
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
                                 const float* __restrict__ lse, int N1, int S_q, int bx, int nqb, long long n_rows,
-                                BsaStrides qs, BsaStrides ls, float* __restrict__ dvec, float* __restrict__ lse2) {
+                                BsaStrides qs, BsaStrides ls, const uint32_t* __restrict__ amax,
+                                float* __restrict__ dvec, float* __restrict__ lse2) {
   griddep_wait();  // launched with programmatic dependent launch: the lists before it must be complete
   griddep_launch_dependents();
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -65,7 +168,9 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __n
   d += __shfl_xor_sync(0xffffffffu, d, 2);
   d += __shfl_xor_sync(0xffffffffu, d, 4);
   if (part == 0) {
-    dvec[row] = valid ? -d : 0.f;
+    // -D in the dS scale (the dP accumulators are brought to it by c_dp)
+    const float s_ds = pow2_scale(256.f * __uint_as_float(amax[3]) * __uint_as_float(amax[2]));
+    dvec[row] = valid ? -d * s_ds : 0.f;
     float l2 = -INFINITY;
     if (valid) {
       const long long b = bh / N1, h = bh % N1;
@@ -93,6 +198,7 @@ struct BwdParams {
   uint64_t* cta_clock;  // optional [grid][2] start / finish times (ns), see bsa_profile_cta_clock
   BsaStrides qs, kvs;   // element strides of dq (heads N1) and of dk / dv (heads N2)
   const uint8_t* amask; // optional dense atten_mask [S_q][S_kv], nonzero = masked out
+  const uint32_t* amax; // max |x| of Q, K, V, dOut (the fp16 copies' scales)
 };
 
 __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&rr)[32], float mul) {
@@ -107,17 +213,6 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
   }
 }
 
-// Split a packed pair x into bf16 hi + lo (x ~= hi + lo to about 2^-17 relative; lo = x - hi by
-// one packed fused multiply-add): the products that take P and dS run as two MMAs, hi then lo,
-// so those operands enter the tensor cores with ~16 significant bits.
-__device__ __forceinline__ void split_pack2(uint64_t x, uint32_t& hi, uint32_t& lo) {
-  float a, b;
-  f2_unpack(x, a, b);
-  hi = pack_bf16(a, b);
-  float la, lb;
-  f2_unpack(f2_fma(f2_pack(bf16lo(hi), bf16hi(hi)), f2_pack(-1.f, -1.f), x), la, lb);
-  lo = pack_bf16(la, lb);
-}
 
 // ------------------------------------------------------------------------------------------------
 // KV-major pass: dK, dV.  Persistent: one CTA per SM takes KV blocks (b, g, kb) from a device
@@ -126,8 +221,8 @@ __device__ __forceinline__ void split_pack2(uint64_t x, uint32_t& hi, uint32_t& 
 // runs as two 64-row halves, so the element-wise work on one half overlaps the tensor-core work of
 // the neighbouring halves:
 //   TMEM columns: scores S^T [0,64) | dP^T [64,128) of one half (128 keys x 64 query rows); the
-//   bf16 A operands of the products P^T hi [128,160), lo [160,192), dS^T hi [192,224), lo
-//   [224,256) (64 query rows -> 32 packed columns); dV [256,384), dK [384,512).
+//   fp16 A operands of the products P^T [128,160) and dS^T [192,224) (64 query rows -> 32 packed
+//   columns); dV [256,384), dK [384,512).
 //   The score buffer is released as soon as the 8 element-wise warps have loaded it into
 //   registers, so S^T / dP^T of half x + 1 run on the tensor cores while the warps turn half x into
 //   P and dS; those go to the operand buffer once the products of half x - 1 have read it.
@@ -169,6 +264,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   griddep_wait();  // the D / LSE tiles of the preprocess must be complete
   griddep_launch_dependents();  // after the wait: the dQ pass then starts only once its inputs exist
   if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x] = globaltimer_ns();
+  const BwdScales sc = bwd_scales(prm.amax, prm.scale, prm.scale_log2);
   constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   KvSmem& s = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -290,8 +386,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ------------------------------------------------------------------ MMA issuers
     if (lane == 0) {
       const bool grads_thread = warp == kVecWarps + 1;
-      const uint32_t id_sdp = idesc_bf16_f32(kT, kHalfRows, false, false);  // S^T, dP^T of a half
-      const uint32_t id_mnb = idesc_bf16_f32(kT, kD, false, true);          // dV, dK (B = [queries][d])
+      const uint32_t id_sdp = idesc_f16_f32(kT, kHalfRows, false, false);  // S^T, dP^T of a half
+      const uint32_t id_mnb = idesc_f16_f32(kT, kD, false, true);          // dV, dK (B = [queries][d])
       int G0 = 0, ucount = 0;
       bool ok = true;
       // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
@@ -337,7 +433,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (n == 0) continue;
         const int nh = 2 * n;
         if (grads_thread) {
-          // dV += P^T dO and dK += dS^T Q (hi, lo) as soon as the element-wise warps have a half
+          // dV += P^T dO and dK += dS^T Q as soon as the element-wise warps have a half
           for (int x = 0; ok && x < nh; ++x) {
             const int hx = G0 + x, hs = hx % kKvRing;
             // exact parity: the next phase needs the warps' P / dS of half hx + 1, which wait for
@@ -346,10 +442,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc_fence_after();
             const uint64_t ddom = ddom0 + static_cast<uint64_t>(hs) * kStage16;
             const uint64_t dqm = dqm0 + static_cast<uint64_t>(hs) * kStage16;
-            grad(tmem + kColDV, kColP, ddom, x > 0);        // dV += P^T_hi dO
-            grad(tmem + kColDV, kColP + 32, ddom, true);    // dV += P^T_lo dO
-            grad(tmem + kColDK, kColP + 64, dqm, x > 0);    // dK += dS^T_hi Q
-            grad(tmem + kColDK, kColP + 96, dqm, true);     // dK += dS^T_lo Q
+            grad(tmem + kColDV, kColP, ddom, x > 0);        // dV += P^T dO
+            grad(tmem + kColDK, kColP + 64, dqm, x > 0);    // dK += dS^T Q
             tc_commit(&s.bar_qdo_empty[hs]);
             tc_commit(&s.bar_grads_done);                   // the operand buffer may be rewritten
           }
@@ -411,8 +505,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc_fence_before();
         mbar_arrive(&s.bar_sdp_free);
         const float4* nl2 = reinterpret_cast<const float4*>(s.lse2[hs] + c0);  // -LSE*log2e per query row
-        const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D per query row
-        const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
+        const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D s_dS per query row
+        const uint64_t sc2 = f2_pack(sc.c_s, sc.c_s), cdp2 = f2_pack(sc.c_dp, sc.c_dp);
         // the dense atten_mask: bit c set when query column c of the chunk may not see this key
         uint32_t mbits = 0;
         if (kMask && key_valid) {
@@ -423,7 +517,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           }
         }
         const bool full = qp0 >= qlo && qp0 + 31 <= qhi && mbits == 0;
-        uint32_t ph[16], pl[16], dh[16], dl[16];
+        uint32_t ph[16], dh[16];
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
           const float4 L = nl2[c4], Dn = nd[c4];
@@ -439,11 +533,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
               if (qp0 + c < qlo || qp0 + c > qhi || ((mbits >> c) & 1u)) p0 = 0.f;
               if (qp0 + c + 1 < qlo || qp0 + c + 1 > qhi || ((mbits >> (c + 1)) & 1u)) p1 = 0.f;
             }
-            const uint64_t p2 = f2_pack(p0, p1);
-            const uint64_t g2 = f2_mul(p2, f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
-                                                  hp ? f2_pack(Dn.z, Dn.w) : f2_pack(Dn.x, Dn.y)));
-            split_pack2(p2, ph[c / 2], pl[c / 2]);
-            split_pack2(g2, dh[c / 2], dl[c / 2]);
+            // dS (in its fp16 scale) = P (dP c_dp - D s_dS)
+            float g0, g1;
+            f2_unpack(f2_mul(f2_pack(p0, p1), f2_fma(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), cdp2,
+                                                    hp ? f2_pack(Dn.z, Dn.w) : f2_pack(Dn.x, Dn.y))),
+                      g0, g1);
+            ph[c / 2] = pack_f16(p0, p1);
+            dh[c / 2] = pack_f16(g0, g1);
           }
         }
         // the operand buffer is free once the previous half's products have completed (exact
@@ -454,10 +550,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           tc_fence_after();
         }
         const uint32_t base = tmem + lane_base + kColP + hf * 16;
-        tmem_st16(base, ph);
-        tmem_st16(base + 32, pl);
-        tmem_st16(base + 64, dh);
-        tmem_st16(base + 96, dl);
+        tmem_st16(base, ph);       // P^T: columns [128, 160)
+        tmem_st16(base + 64, dh);  // dS^T: columns [192, 224)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&s.bar_pds_ready);
@@ -489,8 +583,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           for (int i2 = 0; i2 < 32; ++i2) rk[i2] = rv[i2] = 0u;
         }
         if (key_valid) {
-          store_row_bf16(dkrow + c, rk, prm.scale);
-          store_row_bf16(dvrow + c, rv, 1.f);
+          store_row_bf16(dkrow + c, rk, sc.dk_mul);
+          store_row_bf16(dvrow + c, rv, sc.dv_mul);
         }
       }
       // dK / dV have been read: the next block's first products wait for its P / dS, which come
@@ -541,6 +635,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   if (prm.pdl_wait) griddep_wait();
   griddep_launch_dependents();
   if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x] = globaltimer_ns();
+  const BwdScales sc = bwd_scales(prm.amax, prm.scale, prm.scale_log2);
   constexpr uint32_t kColS0 = 0, kColS1 = BN, kColDP = 2 * BN, kColDQ = 3 * BN;
   extern __shared__ uint8_t smem_raw[];
   QSmem<BN>& s = *reinterpret_cast<QSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -657,8 +752,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ------------------------------------------------------------------ MMA issuers
     if (lane == 0) {
       const bool dq_thread = warp == kVecWarps + 1;
-      const uint32_t id_s = idesc_bf16_f32(kT, BN, false, false);
-      const uint32_t id_dq = idesc_bf16_f32(kT, kD, false, true);
+      const uint32_t id_s = idesc_f16_f32(kT, BN, false, false);
+      const uint32_t id_dq = idesc_f16_f32(kT, kD, false, true);
       // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
       const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0]), 0, 1024);
       const uint64_t ddo0 = sdesc_sw128(smem_u32(s.dout[0]), 0, 1024);
@@ -683,14 +778,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const uint64_t dkm = dkm0 + static_cast<uint64_t>(sk) * kKv16;
             constexpr int kStepsPerHalf = BN / 32;  // 16-key K steps in a warp's key half
 #pragma unroll
-            for (int part = 0; part < 2; ++part)  // hi, then lo
 #pragma unroll
-              for (int ks = 0; ks < BN / 16; ++ks) {
-                const uint32_t a_col = s_col + (ks / kStepsPerHalf) * (BN / 2) + part * (BN / 4) +
-                                       (ks % kStepsPerHalf) * 8;
-                mma_bf16_ts(tmem + kColDQ, tmem + a_col, sdesc_add(dkm, ks * 2048), id_dq,
-                            (j > 0 || part > 0 || ks > 0) ? 1u : 0u);
-              }
+            for (int ks = 0; ks < BN / 16; ++ks) {
+              const uint32_t a_col = s_col + (ks / kStepsPerHalf) * (BN / 2) + (ks % kStepsPerHalf) * 8;
+              mma_bf16_ts(tmem + kColDQ, tmem + a_col, sdesc_add(dkm, ks * 2048), id_dq, (j > 0 || ks > 0) ? 1u : 0u);
+            }
             tc_commit(&s.bar_k_empty[sk]);
             tc_commit(&s.bar_dq_done[st]);
           }
@@ -734,7 +826,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // query row == TMEM lane
     const int c0 = hf * kHalf;          // this thread's key columns [c0, c0 + BN/2)
-    const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
+    const uint64_t sc2 = f2_pack(sc.c_s, sc.c_s), cdp2 = f2_pack(sc.c_dp, sc.c_dp);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     int J0 = 0, done_count = 0;
     bool ok = true;
@@ -753,7 +845,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (!row_valid) { lo = 1; hi = 0; }
       const size_t trow = static_cast<size_t>(bh * prm.nqb + qb) * kT + r;
       const uint64_t nl2 = f2_pack(prm.lse2[trow], prm.lse2[trow]);  // -LSE*log2e of the row, twice
-      const uint64_t nd2 = f2_pack(prm.dvec[trow], prm.dvec[trow]);  // -D of the row, twice
+      const uint64_t nd2 = f2_pack(prm.dvec[trow], prm.dvec[trow]);  // -D s_dS of the row, twice
       for (int j = 0; j < n; ++j) {
         const int J = J0 + j, st = J & 1;
         const uint32_t s_col = st ? kColS1 : kColS0;
@@ -795,26 +887,27 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full, J & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
-        uint32_t hv[kHalf / 2], lv[kHalf / 2];
+        uint32_t hv[kHalf / 2];
 #pragma unroll
         for (int c = 0; c < kHalf; c += 32) {
           uint32_t rr[32];
           tmem_ld32(tmem + lane_base + kColDP + c0 + c, rr);
           tmem_ld_wait(rr);
 #pragma unroll
-          for (int i2 = 0; i2 < 16; ++i2)
-            split_pack2(f2_mul(f2_pack(p[c + 2 * i2], p[c + 2 * i2 + 1]),
-                               f2_add(f2_pack(__uint_as_float(rr[2 * i2]), __uint_as_float(rr[2 * i2 + 1])), nd2)),
-                        hv[c / 2 + i2], lv[c / 2 + i2]);
+          for (int i2 = 0; i2 < 16; ++i2) {
+            // dS (in its fp16 scale) = P (dP c_dp - D s_dS)
+            float g0, g1;
+            f2_unpack(f2_mul(f2_pack(p[c + 2 * i2], p[c + 2 * i2 + 1]),
+                             f2_fma(f2_pack(__uint_as_float(rr[2 * i2]), __uint_as_float(rr[2 * i2 + 1])), cdp2, nd2)),
+                      g0, g1);
+            hv[c / 2 + i2] = pack_f16(g0, g1);
+          }
         }
         tc_fence_before();
         mbar_arrive(&s.bar_dp_free);  // dP of tile J has been read: the next dP may overwrite it
-        // dS over the S_J columns this warp has read: hi -> [c0, +BN/4), lo -> [c0 + BN/4, +BN/4)
+        // dS (fp16) over the S_J columns this warp has read: [c0, +BN/4)
 #pragma unroll
-        for (int c = 0; c < kHalf / 2; c += 16) {
-          tmem_st16(tmem + lane_base + s_col + c0 + c, hv + c);
-          tmem_st16(tmem + lane_base + s_col + c0 + BN / 4 + c, lv + c);
-        }
+        for (int c = 0; c < kHalf / 2; c += 16) tmem_st16(tmem + lane_base + s_col + c0 + c, hv + c);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&s.bar_ds_ready[st]);
@@ -842,7 +935,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
           for (int i2 = 0; i2 < 32; ++i2) rr[i2] = 0u;
         }
-        if (row_valid) store_row_bf16(dqrow + c, rr, prm.scale);
+        if (row_valid) store_row_bf16(dqrow + c, rr, sc.dq_mul);
       }
       // dQ has been read: the next unit's first dQ product waits for its dS, which comes after
       tc_fence_before();
@@ -872,6 +965,31 @@ cudaError_t launch_q(const BwdParams& p, const CUtensorMap& tq, const CUtensorMa
 
 cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, const void* v, const void* out,
                            const void* dout, const float* lse, cudaStream_t st) {
+  // the scaled fp16 copies of Q, K, V, dOut (same layouts)
+  {
+    F16Copy c;
+    const long long nq8 = static_cast<long long>(a.B) * a.N1 * a.S_q * kD / 8;
+    const long long nk8 = static_cast<long long>(a.B) * a.N2 * a.S_kv * kD / 8;
+    const void* src[4] = {q, k, v, dout};
+    void* dst[4] = {a.q16, a.k16, a.v16, a.do16};
+    const long long n8[4] = {nq8, nk8, nk8, nq8};
+    for (int t = 0; t < 4; ++t) {
+      c.src[t] = static_cast<const uint4*>(src[t]);
+      c.dst[t] = static_cast<uint4*>(dst[t]);
+      c.n8[t] = n8[t];
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const dim3 grid(static_cast<unsigned>(sms * 4), 4);
+    prof_begin("bsa_bwd_f16", st);
+    cudaError_t e = launch_pdl(bwd_to_f16_kernel, grid, dim3(256), 0, st, c, a.amax);
+    if (e == cudaSuccess)
+      e = launch_pdl(bwd_f16_fixup_kernel, grid, dim3(256), 0, st, c, static_cast<const uint32_t*>(a.amax));
+    prof_end(st);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const long long n_rows = static_cast<long long>(a.B) * a.N1 * a.nqb * kT;
   {
     const long long threads = n_rows * 8;
@@ -879,12 +997,13 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     prof_begin("bsa_bwd_prep", st);
     cudaError_t e = launch_pdl(bwd_prep_kernel, dim3(static_cast<unsigned>((threads + blk - 1) / blk)), dim3(blk), 0,
                                st, static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout),
-                               lse, a.N1, a.S_q, a.bx, a.nqb, n_rows, a.qs, a.lse_s, a.dvec, a.lse2);
+                               lse, a.N1, a.S_q, a.bx, a.nqb, n_rows, a.qs, a.lse_s,
+                               static_cast<const uint32_t*>(a.amax), a.dvec, a.lse2);
     prof_end(st);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // Q, dO, K, V as (head dim, head, position, batch), whichever of BNSD / BSND is in memory
+  // the fp16 copies as (head dim, head, position, batch), whichever of BNSD / BSND is in memory
   CUtensorMap tq, tk, tv, tdo, tk128, tv128, tq64, tdo64;
   auto qmap = [&](CUtensorMap* m, const void* base, uint32_t rows) {
     return make_tmap_4d_bf16(m, base, kD, a.N1, a.S_q, a.B, a.qs.h, a.qs.s, a.qs.b, rows);
@@ -892,8 +1011,9 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
   auto kvmap = [&](CUtensorMap* m, const void* base, uint32_t rows) {
     return make_tmap_4d_bf16(m, base, kD, a.N2, a.S_kv, a.B, a.kvs.h, a.kvs.s, a.kvs.b, rows);
   };
-  if (!qmap(&tq, q, kT) || !qmap(&tdo, dout, kT) || !kvmap(&tk, k, a.by) || !kvmap(&tv, v, a.by) ||
-      !kvmap(&tk128, k, kT) || !kvmap(&tv128, v, kT) || !qmap(&tq64, q, kHalfRows) || !qmap(&tdo64, dout, kHalfRows))
+  if (!qmap(&tq, a.q16, kT) || !qmap(&tdo, a.do16, kT) || !kvmap(&tk, a.k16, a.by) || !kvmap(&tv, a.v16, a.by) ||
+      !kvmap(&tk128, a.k16, kT) || !kvmap(&tv128, a.v16, kT) || !qmap(&tq64, a.q16, kHalfRows) ||
+      !qmap(&tdo64, a.do16, kHalfRows))
     return cudaErrorInvalidValue;
   BwdParams p;
   bool kv_launched = false;
@@ -909,6 +1029,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
   p.qs = a.qs;
   p.kvs = a.kvs;
   p.amask = a.atten_mask;
+  p.amax = a.amax;
   // KV-major pass
   {
     BwdParams pk = p;

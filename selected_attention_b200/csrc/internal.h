@@ -93,6 +93,7 @@ struct BsaFwdArgs {
 struct WsHeader {
   uint32_t status;
   int32_t next_fwd, next_bwd_kv, next_bwd_q;
+  uint32_t amax[4];  // backward: max |x| (float bits) of Q, K, V, dOut
 };
 cudaError_t bsa_fwd_launch(const BsaFwdArgs& a, const void* q, const void* k, const void* v, cudaStream_t st);
 
@@ -108,6 +109,8 @@ struct BsaBwdArgs {
   const int32_t* t_col;
   float* dvec;               // scratch [B*N1*nqb*128]
   float* lse2;               // scratch [B*N1*nqb*128]
+  void *q16, *k16, *v16, *do16;  // scratch: fp16 copies of Q, K, V, dOut (same layout), scaled by powers of 2
+  uint32_t* amax;            // WsHeader::amax, zeroed before the launch
   int32_t* next_kv;          // work counters of the persistent passes, zeroed before the launch
   int32_t* next_q;
   void* dq;

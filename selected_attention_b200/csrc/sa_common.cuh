@@ -4,6 +4,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -297,6 +298,34 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// The same with f16 A and B ([7,10) and [10,13) = 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);  // RNE; .x = lo occupies the low half
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Power-of-two scale s with amax * s <= 2^14 (s = 1 for amax = 0 or a non-finite amax): an fp16
+// copy of a tensor scaled by s keeps every bf16 value exactly (8 significant bits, far from the
+// fp16 overflow at 65504) unless it falls below the fp16 normal range.
+__device__ __forceinline__ float pow2_scale(float amax) {
+  if (!(amax > 0.f) || !(amax <= 3.0e38f)) return 1.f;
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 126;  // amax < 2^e
+  int se = 14 - e;
+  se = se > 127 ? 127 : (se < -126 ? -126 : se);
+  return __uint_as_float(static_cast<uint32_t>(se + 127) << 23);
+}
+
+// Scale of a backward fp16 operand copy: 1 (a plain conversion) when 2^-8 <= amax < 2^14, else the
+// power of two pow2_scale gives (for very large or very small tensors).
+__device__ __forceinline__ float copy_scale(float amax) {
+  return (amax >= 0.00390625f && amax < 16384.f) ? 1.f : pow2_scale(amax);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes with
