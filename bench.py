@@ -67,17 +67,14 @@ def with_spec(roof):
 # capture of each kernel, valid only while the kernel's source file is unchanged (sha1 prefix of
 # the file recorded at capture time); reported as null once the source has changed.
 NCU_TRAFFIC = {
-    "bsa_bwd_kv": {"bytes": 270692864 + 105957888, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                   "src_sha1": "1b48ca31dc53"},
-    "bsa_bwd_q": {"bytes": 270671872 + 53610752, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                  "src_sha1": "1b48ca31dc53"},
-    "bsa_fwd": {"bytes": 201541888 + 51276544, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
-                "src_sha1": "90fa1eb3e002"},
-    "sfa_decode": {"bytes": 147414528 + 4740864, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
-                   "src_sha1": "b6892b780a60"},
-    # full-size launch, T = 61440
-    "nsa_bwd_dq": {"bytes": 2239617536 + 985623296, "config": 3, "src": "selected_attention_b200/csrc/nsa.cu",
-                   "src_sha1": "ea904e4aa7c6"},
+    "bsa_bwd_kv": {"bytes": 491879936 + 103701504, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                   "src_sha1": "0e7611c58dfc"},
+    "bsa_bwd_q": {"bytes": 270693632 + 51921664, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+                  "src_sha1": "0e7611c58dfc"},
+    "bsa_fwd": {"bytes": 201467648 + 52431360, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+                "src_sha1": "f1562c183dfe"},
+    "sfa_decode": {"bytes": 147508480 + 4237312, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
+                   "src_sha1": "6c80d26dac90"},
 }
 
 
