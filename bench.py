@@ -422,6 +422,9 @@ def run_reference(args, rank, world):
         cfg = config_dict_nsa(w, args)
         metric = METRIC_NSA
     elif isinstance(w, synth.BsaWorkload):
+        if world > 1:  # the same job as the GPU arm: the workload's batches times the rank count
+            import dataclasses
+            w = dataclasses.replace(w, name=f"{w.name}_x{world}", B=w.B * world)
         mask = w.block_mask()
         sample = lambda: cpu_oracle_sample(w, mask, budget_s=step_budget)  # noqa: E731
         cfg = config_dict(w, args)
@@ -454,13 +457,17 @@ def config_dict_decode(w):
 
 
 def config_dict(w, args):
+    """w: the job's workload (B already multiplied by the rank count)."""
+    world = args.gpus
     return {
         "workload": f"{w.name}: block-sparse attention fwd+bwd, BNSD B={w.B} N={w.N1} S={w.S} D={w.D}, "
                     f"{w.block}x{w.block} blocks, selection={w.selection} {w.sel_args}, causal",
         "B": w.B, "N": w.N1, "S": w.S, "D": w.D, "block": w.block, "seed": w.seed,
         "l2": "no flush: inputs (Q,K,V,dOut) exceed the 126 MB L2" if 4 * w.B * w.N1 * w.S * w.D * 2 > 126e6
         else "inputs fit in L2 (small parity workload)",
-        "parallelism": f"replicas x{args.gpus} (independent batches)",
+        "parallelism": "single GPU" if world == 1 else
+        (f"dp{world}: {w.B} batches, contiguous (batch, kv head) slice ranges per rank balanced by selected "
+         f"tiles; no collective on the data path"),
     }
 
 
@@ -483,6 +490,16 @@ def nsa_workload(args):
         lens = [int(x) for x in args.nsa_seqlens.split(",")]
         w = dataclasses.replace(w, seqlens=lens, name=f"{w.name}_seqlens_{'_'.join(map(str, lens))}")
     return w
+
+
+def sum_over_ranks(world, dev, x):
+    """Bookkeeping outside the timed region (the job's credited work): the sum of x over ranks."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t)
+    return float(t.item())
 
 
 def _dist_helpers(world, dev):
@@ -736,6 +753,31 @@ def run_decode(args, rank, world, local_rank):
         print(json.dumps(line))
 
 
+def bsa_job(w, world, rank):
+    """The rank's share of the block-sparse job.  With N ranks the job is N times the workload's
+    batches (B * N batches under the workload's seed: weak scaling); bsa_partition cuts its
+    (batch, kv head) slices into N contiguous ranges balanced by selected tiles, and each rank runs
+    its range as contiguous BNSD pieces (b0, b1, g0, g1).  The slices are independent, so no
+    collective runs on the data path.  With one rank the single piece is the whole workload.
+    Returns (job workload, job mask, pieces, the cut)."""
+    import dataclasses
+
+    from selected_attention_b200 import shard
+    wj = w if world == 1 else dataclasses.replace(w, name=f"{w.name}_x{world}", B=w.B * world)
+    mask = wj.block_mask()
+    starts, pieces = shard.split(mask, wj.N2, world, rank)
+    return wj, mask, pieces, starts
+
+
+def piece_tensor(wj, tag, b0, b1, h0, h1):
+    """bf16 bits [b1 - b0, h1 - h0, S, D] of q/k/v/dout: the job's rows for batches b0..b1-1 and
+    heads h0..h1-1, generated by row range (the same values as the whole tensor holds there)."""
+    heads = wj.N1 if tag in ("q", "dout") else wj.N2
+    rows = [synth.normal_rows_bf16(wj.seed, tag, wj.B * heads * wj.S, wj.D, wj.S, (b * heads + h0) * wj.S,
+                                   (b * heads + h1) * wj.S) for b in range(b0, b1)]
+    return np.concatenate(rows).reshape(b1 - b0, h1 - h0, wj.S, wj.D)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -743,34 +785,48 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = bsa_workload(args.config)
-    mask = w.block_mask()
-    vpairs = visible_pairs_bsa(mask, w.block, w.block, w.S, w.S)
-    flops_step = 14 * w.D * vpairs
-
-    host = {t: torch.from_numpy(w.tensor(t)).view(torch.bfloat16) for t in ("q", "k", "v", "dout")}
-    q, k, v, do = (host[t].to(dev) for t in ("q", "k", "v", "dout"))
-    dmask = torch.from_numpy(mask).to(dev)
+    w0 = bsa_workload(args.config)
+    w, mask_job, pieces, starts = bsa_job(w0, world, rank)
+    G = w.N1 // w.N2
     bx = by = w.block
-    out = torch.empty_like(q)
-    lse = torch.empty(w.B, w.N1, w.S, dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    p = sa.bsa_params(q, k, dmask, bx, by, w.mask_mode, w.scale)
-    ws_f = torch.empty(sa.bsa_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(sa.bsa_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    barrier, max_over_ranks = _dist_helpers(world, dev)
+
+    # per piece: host inputs, device inputs and outputs, workspaces
+    P = []
+    for b0, b1, g0, g1 in pieces:
+        host = {t: torch.from_numpy(piece_tensor(w, t, b0, b1, *((g0 * G, g1 * G) if t in ("q", "dout") else
+                                                                (g0, g1)))).view(torch.bfloat16)
+                for t in ("q", "k", "v", "dout")}
+        m = np.ascontiguousarray(mask_job[b0:b1, g0 * G:g1 * G])
+        d = {t: host[t].to(dev) for t in host}
+        d["mask"] = torch.from_numpy(m).to(dev)
+        o = {"out": torch.empty_like(d["q"]), "lse": torch.empty(b1 - b0, (g1 - g0) * G, w.S, dtype=torch.float32,
+                                                                  device=dev),
+             "dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"])}
+        prm = sa.bsa_params(d["q"], d["k"], d["mask"], bx, by, w.mask_mode, w.scale)
+        P.append({"host": host, "mask": m, "dev": d, "out": o, "vpairs": visible_pairs_bsa(m, bx, by, w.S, w.S),
+                  "ws_f": torch.empty(sa.bsa_fwd_workspace_size(prm), dtype=torch.uint8, device=dev),
+                  "ws_b": torch.empty(sa.bsa_bwd_workspace_size(prm), dtype=torch.uint8, device=dev)})
+    vpairs = sum(x["vpairs"] for x in P)
+    flops_rank = 14 * w.D * vpairs
+    flops_job = sum_over_ranks(world, dev, flops_rank)
     stream = torch.cuda.current_stream()
 
-    def step(qq=q, kk=k, vv=v, dd=do, mm=dmask):
-        sa.bsa_fwd(qq, kk, vv, mm, bx, by, w.mask_mode, w.scale, out=out, lse=lse, workspace=ws_f)
-        sa.bsa_bwd(qq, kk, vv, out, dd, lse, mm, bx, by, w.mask_mode, w.scale, dq=dq, dk=dk, dv=dv,
-                   workspace=ws_b)
+    def compute(x, o, pc):
+        sa.bsa_fwd(x["q"], x["k"], x["v"], x["mask"], bx, by, w.mask_mode, w.scale, out=o["out"], lse=o["lse"],
+                   workspace=pc["ws_f"])
+        sa.bsa_bwd(x["q"], x["k"], x["v"], o["out"], x["dout"], o["lse"], x["mask"], bx, by, w.mask_mode, w.scale,
+                   dq=o["dq"], dk=o["dk"], dv=o["dv"], workspace=pc["ws_b"])
 
-    barrier, max_over_ranks = _dist_helpers(world, dev)
+    def step():
+        for pc in P:
+            compute(pc["dev"], pc["out"], pc)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    assert sa.bsa_get_status(ws_f) == 0 and sa.bsa_get_status(ws_b) == 0, "device status bits set"
+    for pc in P:
+        assert sa.bsa_get_status(pc["ws_f"]) == 0 and sa.bsa_get_status(pc["ws_b"]) == 0, "device status bits set"
 
     # ---- device-timed region: inputs resident in HBM
     with ClockSampler(local_rank) as clocks:
@@ -787,26 +843,28 @@ def run_ours(args, rank, world, local_rank):
         prof = sa.bsa_profile_collect()
         sa.bsa_profile_enable(False)
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
-    value = world * flops_step / (ms * 1e-3) / 1e12
+    value = flops_job / (ms * 1e-3) / 1e12
     sched = schedule_balance(sa, torch, step, dev)  # an extra, untimed step
 
     # ---- end to end through the public API with host buffers (pinned), copies timed, each on its
     # own stream and double-buffered against the compute
-    pin = {t: host[t].pin_memory() for t in host}
-    pin["mask"] = torch.from_numpy(mask).pin_memory()
-    outs = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    pin, d0, outs = {}, {}, {}
+    for i, pc in enumerate(P):
+        for t, x in pc["host"].items():
+            pin[f"{t}{i}"] = x.pin_memory()
+        pin[f"mask{i}"] = torch.from_numpy(pc["mask"]).pin_memory()
+        d0.update({f"{t}{i}": x for t, x in pc["dev"].items()})
+        outs.update({f"{n}{i}": x for n, x in pc["out"].items()})
     h_out = {n: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n, x in outs.items()}
-    d0 = {"q": q, "k": k, "v": v, "dout": do, "mask": dmask}
     dev_in = [d0, {t: torch.empty_like(x) for t, x in d0.items()}]
     dev_out = [outs, {n: torch.empty_like(x) for n, x in outs.items()}]
     h2d = sum(x.numel() * x.element_size() for x in pin.values())
     d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
     def e2e_compute(x, o):
-        sa.bsa_fwd(x["q"], x["k"], x["v"], x["mask"], bx, by, w.mask_mode, w.scale, out=o["out"], lse=o["lse"],
-                   workspace=ws_f)
-        sa.bsa_bwd(x["q"], x["k"], x["v"], o["out"], x["dout"], o["lse"], x["mask"], bx, by, w.mask_mode, w.scale,
-                   dq=o["dq"], dk=o["dk"], dv=o["dv"], workspace=ws_b)
+        for i, pc in enumerate(P):
+            compute({t: x[f"{t}{i}"] for t in ("q", "k", "v", "dout", "mask")},
+                    {n: o[f"{n}{i}"] for n in ("out", "lse", "dq", "dk", "dv")}, pc)
 
     e2e_ms = pipelined_e2e(args.steps, pin, dev_in, dev_out, h_out, e2e_compute, barrier, max_over_ranks)
 
@@ -821,20 +879,21 @@ def run_ours(args, rank, world, local_rank):
     if dom in alg:
         launches, total = prof[dom]
         avg_ms = total / launches
-        achieved = alg[dom] / (avg_ms * 1e-3) / 1e12
+        achieved = alg[dom] / len(P) / (avg_ms * 1e-3) / 1e12  # a launch's average share of the work
         traffic = None
         tr = NCU_TRAFFIC.get(dom)
-        if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config:
+        if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config \
+                and world == 1:
             traffic = tr["bytes"]
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_source": peak_desc, "traffic": traffic, "avg_launch_ms": avg_ms,
                 "frac_of_burst": achieved / peaks["bf16_tflops"]}
-    kernels = kernel_table(prof, alg, args.steps, peak)
+    kernels = kernel_table(prof, {n: f / len(P) for n, f in alg.items()}, args.steps, peak)
     launches_total = sum(c for c, _ in prof.values())
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, t, desc = cpu_oracle_sample(w, mask, budget_s=args.cpu_seconds)
+        f, t, desc = cpu_oracle_sample(w, mask_job, budget_s=args.cpu_seconds)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
                "kind": "oracle", "sample": desc}
 
@@ -843,12 +902,14 @@ def run_ours(args, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, args),
-            "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": flops_job / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_total, "kernels": kernels, "roofline": with_spec(roof), "cpu_baseline": cpu,
-            "clocks": clocks.summary(), "visible_pairs": vpairs, "credited_flops_per_step": flops_step,
+            "clocks": clocks.summary(), "visible_pairs": vpairs, "credited_flops_per_step": flops_job,
             "schedule": sched,
         }
+        if world > 1:
+            line["shard"] = {"slice_cut": [int(x) for x in starts], "rank0_pieces": [list(x) for x in pieces]}
         print(json.dumps(line))
 
 

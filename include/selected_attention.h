@@ -9,9 +9,10 @@
  *                               varlen, GQA ("aclnnNsaSelectedAttention" page, forward formula;
  *                               the backward applies the BlockSparseAttentionGrad formulas to the
  *                               gathered blocks).
- *   sfa_sparse_decode           sparse flash attention decode over a paged KV cache with a rope
+ *   sfa_sparse_decode / _bwd    sparse flash attention decode over a paged KV cache with a rope
  *                               sub-head ("aclnnSparseFlashAttention" page, formula and
- *                               constraints).
+ *                               constraints); the backward applies the BlockSparseAttentionGrad
+ *                               formulas to the gathered keys.
  *   sparse_attn_metadata        selection -> per-unit KV lists, transposed lists and per-page
  *                               lists, consumed by the ops above ("SparseAttnSharedkvMetadata"
  *                               page, function description: a task list built ahead of the
@@ -101,6 +102,19 @@ typedef struct bsa_params {
    * nonzero = masked out; applied inside the selected blocks on top of mask_mode (the
    * Mask(., atten_mask) step of the BlockSparseAttentionGrad formulas).  NULL = none. */
   const uint8_t* atten_mask;
+  /* Optional metadata plan (SparseAttnSharedkvMetadata page: the metadata op's output is the
+   * attention ops' input), device, 256-byte aligned, written by sparse_attn_metadata with op
+   * plan_op for this same problem (the same params and the same selection tensor, unchanged since).
+   * NULL = the op builds its lists in its own workspace.  With a plan the op launches no metadata
+   * kernel and its workspace shrinks (the *_workspace_size calls see the plan).  Accepted ops:
+   *   bsa_fwd: BSA_META_BSA_KV or BSA_META_BSA_BWD;  bsa_bwd: BSA_META_BSA_BWD;
+   *   nsa_selected_fwd: BSA_META_NSA_KV or BSA_META_NSA_TOKENS;  nsa_selected_bwd: BSA_META_NSA_TOKENS.
+   * Another plan_op returns BSA_ERR_INVALID_ARG; a plan given to sfa_sparse_decode returns
+   * BSA_ERR_UNSUPPORTED (the decode builds its page lists in its own prologue).  Device status bits
+   * the metadata raised (bad ids, bad cu_seqlens) stay in the plan's status word: read them with
+   * bsa_get_status(plan).  The library cannot tell a stale plan from a current one. */
+  const void* plan;
+  int32_t plan_op; /* bsa_meta_op */
 } bsa_params;
 
 /* ---- workspace sizing (phase 1: host validation, no launch) ------------------------------ */
@@ -172,9 +186,9 @@ BSA_API bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const vo
  *   holds logical sparse-block ids (sparse_block_size tokens each, a whole number of pages;
  *   -1 = empty slot); seqused_kv [B] is each sequence's token count: keys at or past it are not
  *   attended.  Query head h uses kv head h / (N1 / N2).
- *   Cache rows past seqused_kv inside a selected page are read by the tensor-core products with
- *   weight exactly zero, so they must hold finite values (0 * NaN is NaN); rows of pages that no
- *   selected block reaches are never read.
+ *   Cache rows past seqused_kv inside a selected page are masked, and their V rows are zeroed in
+ *   shared memory before the products, so any value there (NaN included) leaves Out unchanged;
+ *   rows of pages that no selected block reaches are never read.
  *   Host errors: UNSUPPORTED for S_q != 1, D / Dv / D_rope other than 512 / 512 / 64, N1 / N2 >
  *   128, page_size not a multiple of 32, or num_pages * page_size * N2 >= 2^31; INVALID_ARG for
  *   non-positive sizes, N1 % N2 != 0, page_size not a multiple of 16 in [16, 1024],
@@ -186,12 +200,39 @@ BSA_API bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const v
                              const void* k_rope_cache, const void* v_cache, void* out, float* lse,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward of sfa_sparse_decode: the BlockSparseAttentionGrad page's backward formulas applied to
+ * the gathered keys, with the score s = scale (q.k + q_rope.k_rope) split as in the forward:
+ *   P = exp(s - LSE), D = rowsum(dOut o Out), dP = dOut v~^T, dS = P o (dP - D),
+ *   dq = scale dS k~, dq_rope = scale dS k_rope~, dk~ = scale dS^T q, dk_rope~ = scale dS^T q_rope,
+ *   dv~ = P^T dOut.
+ *   Inputs as for sfa_sparse_decode, plus out (the forward's Out, bf16 [B, 1, N1, 512]), dout
+ *   (bf16, same shape) and lse (fp32 [B, 1, N1], natural log).  Outputs (bf16): dq [B, 1, N1, 512],
+ *   dq_rope [B, 1, N1, 64], and dk_cache, dv_cache [num_pages, page_size, N2, 512], dk_rope_cache
+ *   [num_pages, page_size, N2, 64], laid out as the caches.
+ *   Every cache row the step read (a token in use of a selected page of batch b, kv head g) is SET
+ *   to the sum of its gathered rows' gradients: a page listed twice, or reached from two batches'
+ *   block tables, adds each read; the sum runs in a fixed order (deterministic).  Cache rows the
+ *   step did not read are NOT written: zero the three gradient caches first to obtain the full
+ *   cache gradient.  P and dS enter the tensor cores as bf16.
+ *   Host errors: as sfa_sparse_decode, plus BSA_ERR_UNSUPPORTED when p->plan is set or
+ *   num_pages * N2 >= 2^30.  Device status bits: as sfa_sparse_decode.  The workspace holds the
+ *   page lists, per-tile parts of dq and the gathered-order row gradients (about
+ *   B N2 sparse_count sparse_block_size x 2.2 KB). */
+BSA_API bsa_status sfa_sparse_decode_bwd_workspace_size(const bsa_params* p, size_t* bytes);
+BSA_API bsa_status sfa_sparse_decode_bwd(const bsa_params* p, const void* q, const void* q_rope, const void* k_cache,
+                                 const void* k_rope_cache, const void* v_cache, const void* out,
+                                 const void* dout, const float* lse, void* dq, void* dq_rope, void* dk_cache,
+                                 void* dk_rope_cache, void* dv_cache, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* ---- metadata (SparseAttnSharedkvMetadata page) -------------------------------------------
  * Writes the integer plan the attention kernels consume into `plan` (device, plan_bytes from
  * sparse_attn_metadata_size).  op selects the product:
  *   BSA_META_BSA_KV     int32 row_ptr[U+1] then col[...]: per (b, h, qb) unit, ascending KV
  *                       block ids of its BlockSparseMask row (U = B*N1*nqb).
  *   BSA_META_BSA_Q      transposed lists: per (b, g, kb) row, ascending h_local*nqb + qb.
+ *   BSA_META_BSA_BWD    both: offsets[1] row_ptr and [2] col as BSA_META_BSA_KV, [3] row_ptr and
+ *                       [4] col as BSA_META_BSA_Q (the backward's two passes), [5] scratch.
  *   BSA_META_NSA_KV     int32 ids[T, N2, K] (valid ids ascending, then -1) and cnt[T, N2].
  *   BSA_META_NSA_TOKENS also, per (b, g, kb) row (kb < ceil(S_q / sel_block_size)), the
  *                       ascending global token indices whose list holds kb, each token once:
@@ -215,7 +256,8 @@ typedef enum {
   BSA_META_NSA_KV = 2,
   BSA_META_NSA_TOKENS = 3,
   BSA_META_SFA_PAGES = 4,
-  BSA_META_SFA_WORK = 5
+  BSA_META_SFA_WORK = 5,
+  BSA_META_BSA_BWD = 6
 } bsa_meta_op;
 
 /* Offsets (bytes from `plan`) of the arrays an op writes: offsets[0] = status word,
@@ -230,6 +272,17 @@ typedef struct bsa_meta_layout {
 
 BSA_API bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta_layout* layout);
 BSA_API bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, size_t plan_bytes, void* stream);
+
+/* ---- multi-GPU split (host only) -----------------------------------------------------------
+ * Contiguous balanced split of n work items into `parts` ranges (SparseAttnSharedkvMetadata
+ * page, function description: each core gets the start and end of its share of the task list).
+ * Used to give each rank a contiguous range of (batch, kv head) slices weighted by their selected
+ * tiles.  With W the total weight and prefix(t) = weights[0] + ... + weights[t-1]:
+ *   starts[s] = min { t : prefix(t) >= ceil(s W / parts) } for s < parts, starts[parts] = n;
+ * part s takes items [starts[s], starts[s+1]).  weights: host int64 [n], each >= 0; starts: host
+ * int32 [parts + 1], written by the call.  Touches no device state.  Errors: NULL pointers ->
+ * BSA_ERR_NULLPTR; n < 0, parts < 1 or a negative weight -> BSA_ERR_INVALID_ARG (starts untouched). */
+BSA_API bsa_status bsa_partition(const int64_t* weights, int32_t n, int32_t parts, int32_t* starts);
 
 /* ---- status --------------------------------------------------------------------------------
  * Copies the device status word at the start of `workspace` (or of a metadata plan) to

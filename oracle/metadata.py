@@ -140,6 +140,25 @@ def work_cuts(weights: np.ndarray, n_parts: int) -> np.ndarray:
     return np.array([-(-(s * W) // n_parts) for s in range(n_parts + 1)], dtype=np.int64)
 
 
+def slice_cuts(weights, n_parts: int) -> np.ndarray:
+    """Whole-item version of work_cuts: the first item of each part when items may not be cut
+    (the multi-GPU split of (batch, kv head) slices; SparseAttnSharedkvMetadata page, each core's
+    start and end in the task list).  Part s starts at the smallest t whose prefix weight
+    w[0] + ... + w[t-1] reaches ceil(s*W/n_parts); the last cut is the item count.  Plain loops."""
+    w = [int(x) for x in weights]
+    W = sum(w)
+    starts = []
+    for s in range(n_parts):
+        target = -(-(s * W) // n_parts)
+        t, prefix = 0, 0
+        while prefix < target and t < len(w):
+            prefix += w[t]
+            t += 1
+        starts.append(t)
+    starts.append(len(w))
+    return np.array(starts, dtype=np.int32)
+
+
 def sfa_pieces_per_unit(units: int, sms: int, max_pieces: int = 4) -> int:
     """Pieces per decode unit: as many as one wave of the GPU's SMs allows, at most `max_pieces`
     (the pieces of a unit merge their partial results inside one thread-block cluster)."""

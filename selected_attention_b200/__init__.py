@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_NULLPTR", 2: "BSA_ERR_INVALID_ARG", 3: 
                 4: "BSA_ERR_WORKSPACE_TOO_SMALL", 5: "BSA_ERR_CUDA"}
 LAYOUT_BNSD, LAYOUT_TND, LAYOUT_BSND, LAYOUT_PA_ND = 0, 1, 2, 3
 MASK_NONE, MASK_CAUSAL, MASK_RIGHT_DOWN_CAUSAL, MASK_BAND = 0, 2, 3, 4
-META_BSA_KV, META_BSA_Q, META_NSA_KV, META_NSA_TOKENS, META_SFA_PAGES, META_SFA_WORK = range(6)
+META_BSA_KV, META_BSA_Q, META_NSA_KV, META_NSA_TOKENS, META_SFA_PAGES, META_SFA_WORK, META_BSA_BWD = range(7)
 DEV_BAD_INDEX, DEV_BAD_SEQLEN, DEV_TIMEOUT = 1, 2, 4
 
 EXPORTED = [
@@ -30,7 +30,8 @@ EXPORTED = [
     "nsa_selected_fwd", "nsa_selected_bwd", "sfa_sparse_decode", "sparse_attn_metadata_layout",
     "sparse_attn_metadata", "bsa_get_status", "bsa_version", "bsa_diag_mma_tile",
     "bsa_profile_enable", "bsa_profile_collect", "bsa_fwd_noalloc", "bsa_fwd_noalloc_get_status", "bsa_diag_exp2",
-    "bsa_diag_wait", "bsa_profile_cta_clock",
+    "bsa_diag_wait", "bsa_profile_cta_clock", "bsa_partition", "sfa_sparse_decode_bwd_workspace_size",
+    "sfa_sparse_decode_bwd",
 ]
 
 
@@ -60,6 +61,7 @@ class Params(ctypes.Structure):
         ("mask_mode", ctypes.c_int32), ("win_left", ctypes.c_int32), ("win_right", ctypes.c_int32),
         ("scale", ctypes.c_float),
         ("atten_mask", ctypes.c_void_p),
+        ("plan", ctypes.c_void_p), ("plan_op", ctypes.c_int32),
     ]
 
 
@@ -85,7 +87,8 @@ def lib() -> ctypes.CDLL:
         P = ctypes.POINTER(Params)
         vp, sz = ctypes.c_void_p, ctypes.c_size_t
         for name in ("bsa_fwd_workspace_size", "bsa_bwd_workspace_size", "nsa_selected_fwd_workspace_size",
-                     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size"):
+                     "nsa_selected_bwd_workspace_size", "sfa_sparse_decode_workspace_size",
+                     "sfa_sparse_decode_bwd_workspace_size"):
             getattr(L, name).argtypes = [P, ctypes.POINTER(sz)]
         L.bsa_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nsa_selected_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -94,6 +97,7 @@ def lib() -> ctypes.CDLL:
         L.bsa_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nsa_selected_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sfa_sparse_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sfa_sparse_decode_bwd.argtypes = [P] + [vp] * 14 + [sz, vp]
         L.sparse_attn_metadata_layout.argtypes = [P, ctypes.c_int32, ctypes.POINTER(MetaLayout)]
         L.sparse_attn_metadata.argtypes = [P, ctypes.c_int32, vp, sz, vp]
         L.bsa_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -102,6 +106,7 @@ def lib() -> ctypes.CDLL:
         L.bsa_diag_wait.argtypes = [vp, ctypes.c_int32, vp]
         L.bsa_profile_enable.argtypes = [ctypes.c_int32]
         L.bsa_profile_cta_clock.argtypes = [vp, ctypes.c_int32]
+        L.bsa_partition.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, vp]
         L.bsa_profile_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
         L.bsa_version.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -168,6 +173,15 @@ def bsa_params(q, k, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=
     return p
 
 
+def _set_plan(p: Params, plan):
+    """plan: None, or (plan tensor, op) as sparse_attn_metadata made it for this same problem."""
+    if plan is not None:
+        t, op = plan
+        _need_cuda(t)
+        p.plan, p.plan_op = t.data_ptr(), op
+    return p
+
+
 def _lse_shape(p: Params):
     return (p.B, p.S_q, p.N1) if p.q_layout == LAYOUT_BSND else (p.B, p.N1, p.S_q)
 
@@ -179,12 +193,15 @@ def bsa_fwd_workspace_size(p: Params) -> int:
 
 
 def bsa_fwd(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
-            win_right=0, out=None, lse=None, workspace=None, stream=None, layout=LAYOUT_BNSD, atten_mask=None):
+            win_right=0, out=None, lse=None, workspace=None, stream=None, layout=LAYOUT_BNSD, atten_mask=None,
+            plan=None):
     """Out, LSE = softmax(Mask(scale Q K_sel^T)) V_sel for BNSD (or BSND) bf16 tensors and a uint8
     BlockSparseMask [B, N1, ceil(S_q/block_x), ceil(S_kv/block_y)].  Out has q's layout; LSE is
-    [B, N1, S_q] (BNSD) or [B, S_q, N1] (BSND)."""
+    [B, N1, S_q] (BNSD) or [B, S_q, N1] (BSND).  plan: optional (tensor, META_BSA_KV or
+    META_BSA_BWD) from sparse_attn_metadata for this problem; the lists are then not rebuilt."""
     _need_cuda(q, k, v, block_mask)
     p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right, layout, atten_mask)
+    _set_plan(p, plan)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
@@ -198,12 +215,15 @@ def bsa_fwd(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=
 
 
 def bsa_fwd_noalloc(q, k, v, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None, win_left=0,
-                    win_right=0, out=None, lse=None, stream=None, layout=LAYOUT_BNSD):
+                    win_right=0, out=None, lse=None, stream=None, layout=LAYOUT_BNSD, plan=None):
     """bsa_fwd without a workspace, for callers that cannot allocate device memory: the library
     keeps the scratch in a fixed 8 MiB device array (shared by all calls on a device; calls that
-    overlap on the GPU race).  Out and LSE are still the caller's tensors."""
+    overlap on the GPU race).  Out and LSE are still the caller's tensors.  With a plan (as for
+    bsa_fwd) the lists are the plan's and the array holds only the status header, so problems
+    whose lists exceed 8 MiB run too."""
     _need_cuda(q, k, v, block_mask)
     p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right, layout)
+    _set_plan(p, plan)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
@@ -228,10 +248,12 @@ def bsa_bwd_workspace_size(p: Params) -> int:
 
 def bsa_bwd(q, k, v, out, dout, lse, block_mask, block_x, block_y, mask_mode=MASK_CAUSAL, scale=None,
             win_left=0, win_right=0, dq=None, dk=None, dv=None, workspace=None, stream=None, layout=LAYOUT_BNSD,
-            atten_mask=None):
-    """dQ, dK, dV of block-sparse attention (BNSD or BSND, the gradients in the inputs' layout)."""
+            atten_mask=None, plan=None):
+    """dQ, dK, dV of block-sparse attention (BNSD or BSND, the gradients in the inputs' layout).
+    plan: optional (tensor, META_BSA_BWD) from sparse_attn_metadata for this problem."""
     _need_cuda(q, k, v, out, dout, lse, block_mask)
     p = bsa_params(q, k, block_mask, block_x, block_y, mask_mode, scale, win_left, win_right, layout, atten_mask)
+    _set_plan(p, plan)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -304,10 +326,12 @@ def nsa_selected_bwd_workspace_size(p: Params) -> int:
 
 
 def nsa_selected_fwd(q, k, v, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode=MASK_CAUSAL,
-                     scale=None, out=None, lse=None, workspace=None, stream=None):
-    """Out [T, N1, 128] bf16, LSE [T, N1] fp32 of NSA selected attention."""
+                     scale=None, out=None, lse=None, workspace=None, stream=None, plan=None):
+    """Out [T, N1, 128] bf16, LSE [T, N1] fp32 of NSA selected attention.  plan: optional
+    (tensor, META_NSA_KV or META_NSA_TOKENS) from sparse_attn_metadata for this problem."""
     _need_cuda(q, k, v, topk_indices, cu_seqlens)
     p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale)
+    _set_plan(p, plan)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if lse is None else lse
     if workspace is None:
@@ -318,10 +342,13 @@ def nsa_selected_fwd(q, k, v, topk_indices, cu_seqlens, max_seqlen, sel_block_si
 
 
 def nsa_selected_bwd(q, k, v, out, dout, lse, topk_indices, cu_seqlens, max_seqlen, sel_block_size,
-                     mask_mode=MASK_CAUSAL, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV of NSA selected attention."""
+                     mask_mode=MASK_CAUSAL, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None,
+                     plan=None):
+    """dQ, dK, dV of NSA selected attention.  plan: optional (tensor, META_NSA_TOKENS) from
+    sparse_attn_metadata for this problem."""
     _need_cuda(q, k, v, out, dout, lse, topk_indices, cu_seqlens)
     p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale)
+    _set_plan(p, plan)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -378,6 +405,46 @@ def sfa_sparse_decode(q, q_rope, k_cache, k_rope_cache, v_cache, block_table, sp
                                                         _ptr(k_rope_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
                                                         _ptr(workspace), workspace.numel(), _stream(stream)))
     return out, lse
+
+
+def sfa_sparse_decode_bwd_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check("sfa_sparse_decode_bwd_workspace_size",
+           lib().sfa_sparse_decode_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def sfa_sparse_decode_bwd(q, q_rope, k_cache, k_rope_cache, v_cache, out, dout, lse, block_table, sparse_indices,
+                          seqused_kv, sparse_block_size, scale=None, dq=None, dq_rope=None, dk_cache=None,
+                          dk_rope_cache=None, dv_cache=None, workspace=None, stream=None):
+    """dQ, dQ_rope and the cache gradients of sparse decode attention.  The cache rows the step
+    read are set to their gradient; rows it did not read are left as they are (the caches this
+    function allocates when none are given start at zero)."""
+    _need_cuda(q, q_rope, k_cache, k_rope_cache, v_cache, out, dout, lse, block_table, sparse_indices, seqused_kv)
+    p = sfa_params(q, k_cache, block_table, sparse_indices, seqused_kv, sparse_block_size, scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dq_rope = torch.empty_like(q_rope) if dq_rope is None else dq_rope
+    dk_cache = torch.zeros_like(k_cache) if dk_cache is None else dk_cache
+    dk_rope_cache = torch.zeros_like(k_rope_cache) if dk_rope_cache is None else dk_rope_cache
+    dv_cache = torch.zeros_like(v_cache) if dv_cache is None else dv_cache
+    if workspace is None:
+        workspace = _workspace(sfa_sparse_decode_bwd_workspace_size(p), q.device)
+    _check("sfa_sparse_decode_bwd", lib().sfa_sparse_decode_bwd(
+        ctypes.byref(p), _ptr(q), _ptr(q_rope), _ptr(k_cache), _ptr(k_rope_cache), _ptr(v_cache), _ptr(out),
+        _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dq_rope), _ptr(dk_cache), _ptr(dk_rope_cache), _ptr(dv_cache),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dq_rope, dk_cache, dk_rope_cache, dv_cache
+
+
+def partition(weights, parts: int):
+    """Contiguous balanced split (the C bsa_partition): int32 starts [parts + 1], part s taking
+    items [starts[s], starts[s + 1]) of the int64 weights."""
+    import numpy as np
+    w = np.ascontiguousarray(weights, dtype=np.int64)
+    starts = np.zeros(parts + 1, dtype=np.int32)
+    _check("bsa_partition", lib().bsa_partition(w.ctypes.data_as(ctypes.c_void_p), len(w), parts,
+                                                starts.ctypes.data_as(ctypes.c_void_p)))
+    return starts
 
 
 def bsa_get_status(workspace, stream=None) -> int:

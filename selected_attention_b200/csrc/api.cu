@@ -38,6 +38,23 @@ bsa_status check_bsa(const bsa_params* p) {
   return BSA_OK;
 }
 
+// A metadata plan passed in bsa_params::plan: 256-byte aligned and made by one of the ops `a`, `b`.
+bsa_status check_plan(const bsa_params* p, int32_t a, int32_t b) {
+  if (!p->plan) return BSA_OK;
+  if (reinterpret_cast<uintptr_t>(p->plan) % 256 != 0) return BSA_ERR_INVALID_ARG;
+  return (p->plan_op == a || p->plan_op == b) ? BSA_OK : BSA_ERR_INVALID_ARG;
+}
+
+// Array `i` of a plan made by `op` for problem `p` (the layout sparse_attn_metadata_layout gives).
+template <class T>
+T* plan_array(const bsa_params* p, int32_t op, int i) {
+  bsa_meta_layout L;
+  if (sparse_attn_metadata_layout(p, op, &L) != BSA_OK) return nullptr;
+  return reinterpret_cast<T*>(static_cast<char*>(const_cast<void*>(p->plan)) + L.offsets[i]);
+}
+
+// Without a plan the forward builds its KV lists in the workspace; with one it needs only the
+// workspace header.
 struct BsaFwdWs {
   uint32_t* status;
   int32_t *counts, *row_ptr, *col;
@@ -48,9 +65,15 @@ size_t carve_bsa_fwd(const bsa_params* p, void* ws, BsaFwdWs* w) {
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
   const size_t units = static_cast<size_t>(p->B) * p->N1 * nqb;
   w->status = static_cast<uint32_t*>(ws);
-  w->counts = c.take<int32_t>(units);
-  w->row_ptr = c.take<int32_t>(units + 1);
-  w->col = c.take<int32_t>(units * nkb);
+  w->counts = w->row_ptr = w->col = nullptr;
+  if (!p->plan) {
+    w->counts = c.take<int32_t>(units);
+    w->row_ptr = c.take<int32_t>(units + 1);
+    w->col = c.take<int32_t>(units * nkb);
+  } else if (ws) {
+    w->row_ptr = plan_array<int32_t>(p, p->plan_op, 1);
+    w->col = plan_array<int32_t>(p, p->plan_op, 2);
+  }
   return c.bytes();
 }
 
@@ -69,13 +92,22 @@ size_t carve_bsa_bwd(const bsa_params* p, void* ws, BsaBwdWs* w) {
   const size_t units = static_cast<size_t>(p->B) * p->N1 * nqb;
   const size_t t_rows = static_cast<size_t>(p->B) * p->N2 * nkb;
   w->status = static_cast<uint32_t*>(ws);
-  w->counts = c.take<int32_t>(units);
-  w->row_ptr = c.take<int32_t>(units + 1);
-  w->col = c.take<int32_t>(units * nkb);
-  w->maskT = c.take<uint8_t>(units * nkb);
-  w->t_counts = c.take<int32_t>(t_rows);
-  w->t_row_ptr = c.take<int32_t>(t_rows + 1);
-  w->t_col = c.take<int32_t>(units * nkb);
+  w->counts = w->row_ptr = w->col = w->t_counts = w->t_row_ptr = w->t_col = nullptr;
+  w->maskT = nullptr;
+  if (!p->plan) {
+    w->counts = c.take<int32_t>(units);
+    w->row_ptr = c.take<int32_t>(units + 1);
+    w->col = c.take<int32_t>(units * nkb);
+    w->maskT = c.take<uint8_t>(units * nkb);
+    w->t_counts = c.take<int32_t>(t_rows);
+    w->t_row_ptr = c.take<int32_t>(t_rows + 1);
+    w->t_col = c.take<int32_t>(units * nkb);
+  } else if (ws) {  // a BSA_META_BSA_BWD plan
+    w->row_ptr = plan_array<int32_t>(p, BSA_META_BSA_BWD, 1);
+    w->col = plan_array<int32_t>(p, BSA_META_BSA_BWD, 2);
+    w->t_row_ptr = plan_array<int32_t>(p, BSA_META_BSA_BWD, 3);
+    w->t_col = plan_array<int32_t>(p, BSA_META_BSA_BWD, 4);
+  }
   w->dvec = c.take<float>(units * 128);
   w->lse2 = c.take<float>(units * 128);
   const size_t nq = static_cast<size_t>(p->B) * p->N1 * p->S_q * p->D;
@@ -139,7 +171,9 @@ struct NsaWs {
   size_t off_ids, off_cnt, off_t_row_ptr, off_t_col;  // byte offsets, for the metadata layout
 };
 
-size_t carve_nsa(const bsa_params* p, void* ws, NsaWs* w, bool bwd) {
+// The NSA workspace without a plan (and the layout of an NSA plan: the metadata op writes the
+// same arrays).
+size_t carve_nsa_lists(const bsa_params* p, void* ws, NsaWs* w, bool bwd) {
   Carver c(ws);
   w->nblk_max = div_up(p->S_q, p->sel_block_size);
   w->words = div_up(p->T_q, 32);
@@ -163,6 +197,25 @@ size_t carve_nsa(const bsa_params* p, void* ws, NsaWs* w, bool bwd) {
     w->t_row_ptr = c.take<int32_t>(trows + 1);
     w->off_t_col = c.next();
     w->t_col = c.take<int32_t>(rows * p->sel_block_count);
+    w->lse2 = c.take<float>(static_cast<size_t>(p->T_q) * p->N1);
+    w->dvec = c.take<float>(static_cast<size_t>(p->T_q) * p->N1);
+  }
+  return c.bytes();
+}
+
+// An op's workspace: with a plan the lists (and the cu_seqlens check flag) are the plan's, laid
+// out as a plan-less workspace of op plan_op, and the workspace keeps only the backward's scratch.
+size_t carve_nsa(const bsa_params* p, void* ws, NsaWs* w, bool bwd) {
+  if (!p->plan) return carve_nsa_lists(p, ws, w, bwd);
+  bsa_params lists = *p;
+  lists.plan = nullptr;
+  carve_nsa_lists(&lists, const_cast<void*>(p->plan), w, p->plan_op == BSA_META_NSA_TOKENS);
+  Carver c(ws);
+  w->status = static_cast<uint32_t*>(ws);
+  w->bitmap = nullptr;
+  w->t_counts = nullptr;
+  w->lse2 = w->dvec = nullptr;
+  if (bwd) {
     w->lse2 = c.take<float>(static_cast<size_t>(p->T_q) * p->N1);
     w->dvec = c.take<float>(static_cast<size_t>(p->T_q) * p->N1);
   }
@@ -253,6 +306,7 @@ const char* bsa_version(void) { return "selected_attention_b200 0.1 (sm_100a)"; 
 bsa_status bsa_fwd_workspace_size(const bsa_params* p, size_t* bytes) {
   if (!bytes) return BSA_ERR_NULLPTR;
   bsa_status s = check_bsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_BSA_KV, BSA_META_BSA_BWD);
   if (s != BSA_OK) return s;
   BsaFwdWs w;
   *bytes = carve_bsa_fwd(p, nullptr, &w);
@@ -262,6 +316,7 @@ bsa_status bsa_fwd_workspace_size(const bsa_params* p, size_t* bytes) {
 bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
                    void* workspace, size_t workspace_bytes, void* stream) {
   bsa_status s = check_bsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_BSA_KV, BSA_META_BSA_BWD);
   if (s != BSA_OK) return s;
   if (!q || !k || !v || !out || !lse || !p->block_mask) return BSA_ERR_NULLPTR;
   BsaFwdWs w;
@@ -272,7 +327,7 @@ bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
   const int units = p->B * p->N1 * nqb;
   cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(WsHeader), st);
-  if (e == cudaSuccess) e = bsa_kv_lists(p->block_mask, units, nkb, w.counts, w.row_ptr, w.col, st);
+  if (e == cudaSuccess && !p->plan) e = bsa_kv_lists(p->block_mask, units, nkb, w.counts, w.row_ptr, w.col, st);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   BsaFwdArgs a;
   a.next_unit = &reinterpret_cast<WsHeader*>(w.status)->next_fwd;
@@ -290,6 +345,7 @@ bsa_status bsa_fwd(const bsa_params* p, const void* q, const void* k, const void
 bsa_status bsa_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
   if (!bytes) return BSA_ERR_NULLPTR;
   bsa_status s = check_bsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_BSA_BWD, BSA_META_BSA_BWD);
   if (s != BSA_OK) return s;
   BsaBwdWs w;
   *bytes = carve_bsa_bwd(p, nullptr, &w);
@@ -300,6 +356,7 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
                    const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
                    size_t workspace_bytes, void* stream) {
   bsa_status s = check_bsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_BSA_BWD, BSA_META_BSA_BWD);
   if (s != BSA_OK) return s;
   if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !p->block_mask) return BSA_ERR_NULLPTR;
   BsaBwdWs w;
@@ -309,8 +366,9 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
   cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(WsHeader), st);
-  if (e == cudaSuccess) e = bsa_kv_lists(p->block_mask, p->B * p->N1 * nqb, nkb, w.counts, w.row_ptr, w.col, st);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && !p->plan)
+    e = bsa_kv_lists(p->block_mask, p->B * p->N1 * nqb, nkb, w.counts, w.row_ptr, w.col, st);
+  if (e == cudaSuccess && !p->plan)
     e = bsa_q_lists(p->block_mask, p->B, p->N1, p->N2, nqb, nkb, w.maskT, w.t_counts, w.t_row_ptr, w.t_col, st);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   BsaBwdArgs a;
@@ -332,6 +390,7 @@ bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, const void
 bsa_status nsa_selected_fwd_workspace_size(const bsa_params* p, size_t* bytes) {
   if (!bytes) return BSA_ERR_NULLPTR;
   bsa_status s = check_nsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_NSA_KV, BSA_META_NSA_TOKENS);
   if (s != BSA_OK) return s;
   NsaWs w;
   *bytes = carve_nsa(p, nullptr, &w, false);
@@ -341,6 +400,7 @@ bsa_status nsa_selected_fwd_workspace_size(const bsa_params* p, size_t* bytes) {
 bsa_status nsa_selected_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
   if (!bytes) return BSA_ERR_NULLPTR;
   bsa_status s = check_nsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_NSA_TOKENS, BSA_META_NSA_TOKENS);
   if (s != BSA_OK) return s;
   NsaWs w;
   *bytes = carve_nsa(p, nullptr, &w, true);
@@ -350,6 +410,7 @@ bsa_status nsa_selected_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
 bsa_status nsa_selected_fwd(const bsa_params* p, const void* q, const void* k, const void* v, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream) {
   bsa_status s = check_nsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_NSA_KV, BSA_META_NSA_TOKENS);
   if (s != BSA_OK) return s;
   if (!q || !k || !v || !out || !lse || !p->topk_indices || !p->cu_seqlens_q) return BSA_ERR_NULLPTR;
   NsaWs w;
@@ -358,8 +419,7 @@ bsa_status nsa_selected_fwd(const bsa_params* p, const void* q, const void* k, c
   carve_nsa(p, workspace, &w, false);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
-  cudaError_t e = nsa_metadata(nsa_meta_args(p, w, false), st);
-  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  if (!p->plan && nsa_metadata(nsa_meta_args(p, w, false), st) != cudaSuccess) return BSA_ERR_CUDA;
   NsaArgs a = nsa_args(p, w);
   a.q = q; a.k = k; a.v = v; a.out = out; a.lse_out = lse;
   return cuda_status(nsa_fwd_launch(a, st));
@@ -369,6 +429,7 @@ bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const void* k, c
                             const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, void* stream) {
   bsa_status s = check_nsa(p);
+  if (s == BSA_OK) s = check_plan(p, BSA_META_NSA_TOKENS, BSA_META_NSA_TOKENS);
   if (s != BSA_OK) return s;
   if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !p->topk_indices || !p->cu_seqlens_q)
     return BSA_ERR_NULLPTR;
@@ -378,8 +439,7 @@ bsa_status nsa_selected_bwd(const bsa_params* p, const void* q, const void* k, c
   carve_nsa(p, workspace, &w, true);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
-  cudaError_t e = nsa_metadata(nsa_meta_args(p, w, true), st);
-  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  if (!p->plan && nsa_metadata(nsa_meta_args(p, w, true), st) != cudaSuccess) return BSA_ERR_CUDA;
   NsaArgs a = nsa_args(p, w);
   a.q = q; a.k = k; a.v = v; a.out_in = out; a.dout = dout; a.lse_in = lse; a.dq = dq; a.dk = dk; a.dv = dv;
   return cuda_status(nsa_bwd_launch(a, st));
@@ -388,6 +448,7 @@ bsa_status sfa_sparse_decode_workspace_size(const bsa_params* p, size_t* bytes) 
   if (!bytes) return BSA_ERR_NULLPTR;
   bsa_status s = check_sfa(p);
   if (s != BSA_OK) return s;
+  if (p->plan) return BSA_ERR_UNSUPPORTED;  // the decode builds its page lists in its prologue
   SfaWs w;
   *bytes = carve_sfa(p, nullptr, &w);
   return BSA_OK;
@@ -398,6 +459,7 @@ bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_r
                              size_t workspace_bytes, void* stream) {
   bsa_status s = check_sfa(p);
   if (s != BSA_OK) return s;
+  if (p->plan) return BSA_ERR_UNSUPPORTED;
   if (!q || !q_rope || !k_cache || !k_rope_cache || !v_cache || !out || !lse || !p->block_table ||
       !p->sparse_indices || !p->seqused_kv)
     return BSA_ERR_NULLPTR;
@@ -419,10 +481,106 @@ bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_r
   return cuda_status(sfa_decode_launch(a, st));
 }
 
+// Backward of the decode: the unit's page lists, the preprocess, the per-tile dQ parts, the
+// gathered-order row gradients and the readers of every cache row-block.
+struct SfaBwdWs {
+  uint32_t* status;
+  int32_t *pages, *tokens, *count, *cnt, *ptr, *list;
+  float *lse2, *dvec, *dqp;
+  uint16_t *gk, *gv;
+};
+
+size_t carve_sfa_bwd(const bsa_params* p, void* ws, SfaBwdWs* w) {
+  Carver c(ws);
+  const size_t U = static_cast<size_t>(p->B) * p->N2;
+  const size_t cap = static_cast<size_t>(p->sparse_count) * (p->sparse_block_size / p->page_size);
+  const size_t rows = U * cap * p->page_size;
+  const size_t keys = static_cast<size_t>(p->num_pages) * p->N2;
+  const size_t T = static_cast<size_t>(sfa_bwd_tiles(static_cast<int>(cap), p->page_size));
+  w->status = static_cast<uint32_t*>(ws);
+  w->pages = c.take<int32_t>(U * cap);
+  w->tokens = c.take<int32_t>(U * cap);
+  w->count = c.take<int32_t>(U);
+  w->cnt = c.take<int32_t>(2 * keys);
+  w->ptr = c.take<int32_t>(keys + 1);
+  w->list = c.take<int32_t>(U * cap);
+  w->lse2 = c.take<float>(static_cast<size_t>(p->B) * p->N1);
+  w->dvec = c.take<float>(static_cast<size_t>(p->B) * p->N1);
+  w->dqp = c.take<float>(U * T * (p->N1 / p->N2) * 576);
+  w->gk = c.take<uint16_t>(rows * 576);
+  w->gv = c.take<uint16_t>(rows * 512);
+  return c.bytes();
+}
+
+bsa_status sfa_sparse_decode_bwd_workspace_size(const bsa_params* p, size_t* bytes) {
+  if (!bytes) return BSA_ERR_NULLPTR;
+  bsa_status s = check_sfa(p);
+  if (s != BSA_OK) return s;
+  if (p->plan) return BSA_ERR_UNSUPPORTED;
+  if (1LL * p->num_pages * p->N2 >= (1LL << 30)) return BSA_ERR_UNSUPPORTED;
+  SfaBwdWs w;
+  *bytes = carve_sfa_bwd(p, nullptr, &w);
+  return BSA_OK;
+}
+
+bsa_status sfa_sparse_decode_bwd(const bsa_params* p, const void* q, const void* q_rope, const void* k_cache,
+                                 const void* k_rope_cache, const void* v_cache, const void* out, const void* dout,
+                                 const float* lse, void* dq, void* dq_rope, void* dk_cache, void* dk_rope_cache,
+                                 void* dv_cache, void* workspace, size_t workspace_bytes, void* stream) {
+  size_t need = 0;
+  bsa_status s = sfa_sparse_decode_bwd_workspace_size(p, &need);
+  if (s != BSA_OK) return s;
+  if (!q || !q_rope || !k_cache || !k_rope_cache || !v_cache || !out || !dout || !lse || !dq || !dq_rope ||
+      !dk_cache || !dk_rope_cache || !dv_cache || !p->block_table || !p->sparse_indices || !p->seqused_kv)
+    return BSA_ERR_NULLPTR;
+  if ((s = check_ws(workspace, workspace_bytes, need)) != BSA_OK) return s;
+  SfaBwdWs w;
+  carve_sfa_bwd(p, workspace, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
+  SfaBwdArgs a;
+  a.meta = sfa_meta_args(p);
+  a.meta.pages = w.pages; a.meta.tokens = w.tokens; a.meta.count = w.count; a.meta.status = w.status;
+  a.B = p->B; a.N1 = p->N1; a.N2 = p->N2; a.page_size = p->page_size; a.num_pages = p->num_pages;
+  a.cap = p->sparse_count * (p->sparse_block_size / p->page_size);
+  a.scale = p->scale;
+  a.q = q; a.q_rope = q_rope; a.k_cache = k_cache; a.k_rope_cache = k_rope_cache; a.v_cache = v_cache;
+  a.out = out; a.dout = dout; a.lse = lse;
+  a.dq = dq; a.dq_rope = dq_rope; a.dk_cache = dk_cache; a.dk_rope_cache = dk_rope_cache; a.dv_cache = dv_cache;
+  a.lse2 = w.lse2; a.dvec = w.dvec; a.dqp = w.dqp; a.gk = w.gk; a.gv = w.gv;
+  a.cnt = w.cnt; a.ptr = w.ptr; a.list = w.list;
+  return cuda_status(sfa_bwd_launch(a, st));
+}
+
 // ---- metadata -------------------------------------------------------------------------------------
 bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta_layout* layout) {
   if (!layout) return BSA_ERR_NULLPTR;
   std::memset(layout, 0, sizeof(*layout));
+  if (op == BSA_META_BSA_BWD) {
+    bsa_status s = check_bsa(p);
+    if (s != BSA_OK) return s;
+    const int nqb = div_up(p->S_q, p->block_x), nkb = div_up(p->S_kv, p->block_y);
+    const size_t units = static_cast<size_t>(p->B) * p->N1 * nqb;
+    const size_t t_rows = static_cast<size_t>(p->B) * p->N2 * nkb;
+    const size_t ents = units * nkb;
+    Carver c(nullptr);
+    layout->offsets[0] = 0;
+    layout->offsets[1] = c.next();  // row_ptr (per (b, h, qb))
+    c.take<int32_t>(units + 1);
+    layout->offsets[2] = c.next();  // col
+    c.take<int32_t>(ents);
+    layout->offsets[3] = c.next();  // transposed row_ptr (per (b, g, kb))
+    c.take<int32_t>(t_rows + 1);
+    layout->offsets[4] = c.next();  // transposed col
+    c.take<int32_t>(ents);
+    layout->offsets[5] = c.next();  // scratch: counts, transposed counts, transposed mask
+    c.take<int32_t>(units);
+    c.take<int32_t>(t_rows);
+    c.take<uint8_t>(ents);
+    layout->count = 6;
+    layout->total_bytes = c.bytes();
+    return BSA_OK;
+  }
   if (op == BSA_META_BSA_KV || op == BSA_META_BSA_Q) {
     bsa_status s = check_bsa(p);
     if (s != BSA_OK) return s;
@@ -455,7 +613,7 @@ bsa_status sparse_attn_metadata_layout(const bsa_params* p, int32_t op, bsa_meta
     if (s != BSA_OK) return s;
     NsaWs w;
     const bool tok = op == BSA_META_NSA_TOKENS;
-    layout->total_bytes = carve_nsa(p, nullptr, &w, tok);
+    layout->total_bytes = carve_nsa_lists(p, nullptr, &w, tok);
     layout->offsets[1] = w.off_ids;
     layout->offsets[2] = w.off_cnt;
     layout->offsets[3] = w.off_t_row_ptr;
@@ -511,7 +669,7 @@ bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, siz
     if (!p->topk_indices || !p->cu_seqlens_q) return BSA_ERR_NULLPTR;
     if (cudaMemsetAsync(plan, 0, sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
     NsaWs w;
-    carve_nsa(p, plan, &w, op == BSA_META_NSA_TOKENS);
+    carve_nsa_lists(p, plan, &w, op == BSA_META_NSA_TOKENS);
     return cuda_status(nsa_metadata(nsa_meta_args(p, w, op == BSA_META_NSA_TOKENS), st));
   }
   if (op == BSA_META_SFA_PAGES || op == BSA_META_SFA_WORK) {
@@ -535,6 +693,20 @@ bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, siz
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   int32_t* row_ptr = reinterpret_cast<int32_t*>(base + L.offsets[1]);
   int32_t* col = reinterpret_cast<int32_t*>(base + L.offsets[2]);
+  if (op == BSA_META_BSA_BWD) {
+    Carver c(base + L.offsets[5]);
+    c.off = 0;
+    const size_t units = static_cast<size_t>(p->B) * p->N1 * nqb;
+    int32_t* counts = c.take<int32_t>(units);
+    int32_t* t_counts = c.take<int32_t>(static_cast<size_t>(p->B) * p->N2 * nkb);
+    uint8_t* maskT = c.take<uint8_t>(units * nkb);
+    e = bsa_kv_lists(p->block_mask, static_cast<int>(units), nkb, counts, row_ptr, col, st);
+    if (e == cudaSuccess)
+      e = bsa_q_lists(p->block_mask, p->B, p->N1, p->N2, nqb, nkb, maskT, t_counts,
+                      reinterpret_cast<int32_t*>(base + L.offsets[3]), reinterpret_cast<int32_t*>(base + L.offsets[4]),
+                      st);
+    return cuda_status(e);
+  }
   int32_t* counts = reinterpret_cast<int32_t*>(base + L.offsets[3]);
   if (op == BSA_META_BSA_KV)
     e = bsa_kv_lists(p->block_mask, p->B * p->N1 * nqb, nkb, counts, row_ptr, col, st);
@@ -542,6 +714,25 @@ bsa_status sparse_attn_metadata(const bsa_params* p, int32_t op, void* plan, siz
     e = bsa_q_lists(p->block_mask, p->B, p->N1, p->N2, nqb, nkb, reinterpret_cast<uint8_t*>(base + L.offsets[4]),
                     counts, row_ptr, col, st);
   return cuda_status(e);
+}
+
+bsa_status bsa_partition(const int64_t* weights, int32_t n, int32_t parts, int32_t* starts) {
+  if (!starts || (n > 0 && !weights)) return BSA_ERR_NULLPTR;
+  if (n < 0 || parts < 1) return BSA_ERR_INVALID_ARG;
+  __int128 total = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    if (weights[i] < 0) return BSA_ERR_INVALID_ARG;
+    total += weights[i];
+  }
+  int32_t t = 0;
+  __int128 prefix = 0;  // prefix(t)
+  for (int32_t s = 0; s < parts; ++s) {
+    const __int128 target = (static_cast<__int128>(s) * total + parts - 1) / parts;  // ceil(s W / parts)
+    while (prefix < target && t < n) prefix += weights[t++];
+    starts[s] = t;
+  }
+  starts[parts] = n;
+  return BSA_OK;
 }
 
 bsa_status bsa_get_status(const void* workspace, void* stream, uint32_t* dev_bits) {

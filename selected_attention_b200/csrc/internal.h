@@ -154,6 +154,27 @@ struct SfaDecodeArgs {
 };
 cudaError_t sfa_decode_launch(const SfaDecodeArgs& a, cudaStream_t st);
 
+// ---- SFA backward (sfa_bwd.cu) --------------------------------------------------------------------
+// Unit u = b * N2 + g (all G heads of a kv head); meta holds the page lists ([U][cap], count [U]).
+struct SfaBwdArgs {
+  SfaMetaArgs meta;
+  int B, N1, N2, page_size, num_pages, cap;  // cap = K * ppb pages per unit
+  float scale;
+  const void *q, *q_rope, *k_cache, *k_rope_cache, *v_cache, *out, *dout;
+  const float* lse;
+  void *dq, *dq_rope, *dk_cache, *dk_rope_cache, *dv_cache;
+  // workspace
+  float *lse2, *dvec;  // [B * N1]
+  float* dqp;          // [U][T][G][576], T = tiles of 128 gathered tokens per unit
+  void *gk, *gv;       // gathered-order row gradients [U][cap * page_size][576] / [..][512] bf16
+  int32_t *cnt;        // [2][num_pages * N2]: readers per cache row-block, then the fill cursor
+  int32_t *ptr;        // [num_pages * N2 + 1]
+  int32_t *list;       // [U * cap]
+};
+cudaError_t sfa_bwd_launch(const SfaBwdArgs& a, cudaStream_t st);
+// tiles of 128 gathered tokens per unit for a list of cap pages (the same rule the kernel uses)
+int sfa_bwd_tiles(int cap, int page_size);
+
 // ---- NSA selected attention (nsa_meta.cu, nsa.cu) ----------------------------------------------
 struct NsaMetaArgs {
   const int32_t* topk;        // [T, N2, K]

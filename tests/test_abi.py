@@ -167,3 +167,75 @@ def test_metadata_layouts_without_gpu():
     assert kv.offsets[2] - kv.offsets[1] >= ids_bytes and tok.total_bytes > kv.total_bytes
     assert sa.lib().sparse_attn_metadata_layout(ctypes.byref(q), 99, ctypes.byref(sa.MetaLayout())) \
         == sa.BSA_ERR_UNSUPPORTED
+
+
+def test_plan_input_validation():
+    """A metadata plan passed to an op must come from an op that holds the lists it reads, be
+    256-byte aligned, and shrinks the op's workspace to its scratch; the decode takes none."""
+    fake = 1 << 20  # an aligned address: sizing calls never dereference the plan
+    n_plain = _ws("bsa_fwd_workspace_size", _bsa())[1]
+    code, n = _ws("bsa_fwd_workspace_size", _bsa(plan=fake, plan_op=sa.META_BSA_KV))
+    assert code == sa.BSA_OK and n == 256 < n_plain
+    assert _ws("bsa_fwd_workspace_size", _bsa(plan=fake, plan_op=sa.META_BSA_BWD))[0] == sa.BSA_OK
+    assert _ws("bsa_fwd_workspace_size", _bsa(plan=fake, plan_op=sa.META_BSA_Q))[0] == sa.BSA_ERR_INVALID_ARG
+    assert _ws("bsa_fwd_workspace_size", _bsa(plan=fake + 4, plan_op=sa.META_BSA_KV))[0] == sa.BSA_ERR_INVALID_ARG
+    b_plain = _ws("bsa_bwd_workspace_size", _bsa())[1]
+    code, b = _ws("bsa_bwd_workspace_size", _bsa(plan=fake, plan_op=sa.META_BSA_BWD))
+    assert code == sa.BSA_OK and b < b_plain
+    assert _ws("bsa_bwd_workspace_size", _bsa(plan=fake, plan_op=sa.META_BSA_KV))[0] == sa.BSA_ERR_INVALID_ARG
+    q = _nsa()
+    q.plan, q.plan_op = fake, sa.META_NSA_KV
+    assert _ws("nsa_selected_fwd_workspace_size", q)[0] == sa.BSA_OK
+    assert _ws("nsa_selected_bwd_workspace_size", q)[0] == sa.BSA_ERR_INVALID_ARG
+    q.plan_op = sa.META_NSA_TOKENS
+    code, nb = _ws("nsa_selected_bwd_workspace_size", q)
+    q.plan = None
+    assert code == sa.BSA_OK and nb < _ws("nsa_selected_bwd_workspace_size", q)[1]
+    assert _ws("sfa_sparse_decode_workspace_size", _sfa(plan=fake, plan_op=sa.META_SFA_WORK))[0] \
+        == sa.BSA_ERR_UNSUPPORTED
+
+
+def test_bsa_bwd_plan_layout():
+    """The backward plan holds both list sets: forward CSR then transposed CSR, each array
+    256-byte aligned and sized like the single-op plans."""
+    p = _bsa(B=1, N1=4, N2=2, S_q=1000, S_kv=1000)
+    units, nkb, trows = 1 * 4 * 8, 8, 1 * 2 * 8
+    lay = sa.sparse_attn_metadata_layout(p, sa.META_BSA_BWD)
+    assert lay.count == 6
+    offs = [lay.offsets[i] for i in range(1, 6)]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert offs[1] - offs[0] >= 4 * (units + 1) and offs[2] - offs[1] >= 4 * units * nkb
+    assert offs[3] - offs[2] >= 4 * (trows + 1) and offs[4] - offs[3] >= 4 * units * nkb
+    assert lay.total_bytes >= offs[4] + 4 * (units + trows) + units * nkb
+
+
+def test_partition_matches_cpu_reference():
+    """bsa_partition (host code in the library, no device access) against the CPU reference's
+    slice_cuts, bit for bit, and its argument checks."""
+    from oracle import metadata as M
+    import numpy as np
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        n, parts = int(rng.integers(0, 40)), int(rng.integers(1, 10))
+        w = rng.integers(0, 1000, n) * (rng.random(n) < 0.8)
+        assert sa.partition(w, parts).tolist() == M.slice_cuts(w, parts).tolist()
+    big = np.full(1024, 2 ** 40, np.int64)  # totals past 2^32
+    assert sa.partition(big, 7).tolist() == M.slice_cuts(big, 7).tolist()
+    starts = (ctypes.c_int32 * 3)()
+    neg = (ctypes.c_int64 * 2)(1, -1)
+    assert sa.lib().bsa_partition(neg, 2, 2, starts) == sa.BSA_ERR_INVALID_ARG
+    assert sa.lib().bsa_partition(neg, 2, 0, starts) == sa.BSA_ERR_INVALID_ARG
+    assert sa.lib().bsa_partition(None, 2, 2, starts) == sa.BSA_ERR_NULLPTR
+
+
+def test_sfa_bwd_host_validation():
+    """The decode backward takes the decode's constraints; its workspace holds the gathered-order
+    row gradients (~2.2 KB per selected token) and takes no metadata plan."""
+    p = _sfa()
+    code, n = _ws("sfa_sparse_decode_bwd_workspace_size", p)
+    tokens = p.B * p.N2 * p.sparse_count * p.sparse_block_size
+    assert code == sa.BSA_OK and n >= tokens * (576 + 512) * 2
+    assert _ws("sfa_sparse_decode_bwd_workspace_size", _sfa(S_q=2))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws("sfa_sparse_decode_bwd_workspace_size", _sfa(plan=1 << 20, plan_op=sa.META_SFA_WORK))[0] \
+        == sa.BSA_ERR_UNSUPPORTED
+    assert sa.lib().sfa_sparse_decode_bwd(ctypes.byref(p), *([None] * 14), 0, None) == sa.BSA_ERR_NULLPTR

@@ -96,6 +96,37 @@ def test_work_cuts():
     assert np.all(np.diff(cuts) >= 0) and np.max(np.diff(cuts)) - np.min(np.diff(cuts)) <= 1
 
 
+def test_slice_cuts_golden():
+    with open(os.path.join(GOLDEN, "slice_cuts.json")) as f:
+        g = json.load(f)
+    for c in g["cases"]:
+        assert M.slice_cuts(np.array(c["weights"], np.int64), c["parts"]).tolist() == c["starts"], c["why"]
+
+
+def test_slice_cuts_uniform_closed_form_and_balance():
+    """Equal weights give starts ceil(s n / parts) (the textbook even split); for any weights each
+    part's total stays within one slice's weight of W / parts (brute force over small random
+    weight vectors, zeros included)."""
+    for n in range(0, 13):
+        for parts in range(1, 7):
+            got = M.slice_cuts(np.full(n, 3, np.int64), parts)
+            assert got.tolist() == [-(-(s * n) // parts) for s in range(parts)] + [n]
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        n, parts = int(rng.integers(1, 12)), int(rng.integers(1, 6))
+        w = rng.integers(0, 9, n)
+        st = M.slice_cuts(w, parts)
+        assert st[0] == 0 and st[-1] == n and np.all(np.diff(st) >= 0)
+        part_w = [int(w[st[s]:st[s + 1]].sum()) for s in range(parts)]
+        assert sum(part_w) == w.sum()
+        assert max(part_w) <= -(-int(w.sum()) // parts) + int(w.max()) if n else True
+        # each cut is the first place the running total reaches its share: no earlier cut works
+        pre = np.concatenate([[0], np.cumsum(w)])
+        for s in range(1, parts):
+            target = -(-(s * int(w.sum())) // parts)
+            assert min(t for t in range(n + 1) if pre[t] >= target or t == n) == st[s]
+
+
 def test_sfa_pieces_cover_each_unit_evenly():
     """Brute-force properties of the decode split, independent of its formula: the pieces of a
     unit are consecutive, start at 0, end at n, and their lengths differ by at most one (the
