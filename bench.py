@@ -49,6 +49,7 @@ from workloads import synth  # noqa: E402
 METRIC = "effective block-sparse attn fwd+bwd TFLOP/s (bf16)"
 METRIC_NSA = "effective NSA selected attn fwd+bwd TFLOP/s (bf16)"
 METRIC_DEC = "sparse decode gathered-KV bandwidth (paged, bf16)"
+METRIC_DEC_BWD = "sparse decode backward gathered-KV + gradient-row bandwidth (paged, bf16)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal B200 figures, reported beside the measured-peak fractions: dense bf16 and HBM3e
 SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
@@ -66,16 +67,32 @@ def with_spec(roof):
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum of one launch) from an ncu
 # capture of each kernel, valid only while the kernel's source file is unchanged (sha1 prefix of
 # the file recorded at capture time); reported as null once the source has changed.
-NCU_TRAFFIC = {
-    "bsa_bwd_kv": {"bytes": 491879936 + 103701504, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                   "src_sha1": "0e7611c58dfc"},
-    "bsa_bwd_q": {"bytes": 270693632 + 51921664, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-                  "src_sha1": "0e7611c58dfc"},
-    "bsa_fwd": {"bytes": 201467648 + 52431360, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
-                "src_sha1": "f1562c183dfe"},
-    "sfa_decode": {"bytes": 147508480 + 4237312, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
-                   "src_sha1": "6c80d26dac90"},
-}
+NCU_TRAFFIC = [
+    {"kernel": "bsa_bwd_kv", "bytes": 491879936 + 103701504, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+     "src_sha1": "0e7611c58dfc"},
+    {"kernel": "bsa_bwd_q", "bytes": 270693632 + 51921664, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+     "src_sha1": "0e7611c58dfc"},
+    {"kernel": "bsa_fwd", "bytes": 201467648 + 52431360, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+     "src_sha1": "f1562c183dfe"},
+    # full-size launches of the S=131072 workload (one-pass DRAM counters)
+    {"kernel": "bsa_bwd_kv", "bytes": 12192800256 + 2115727104, "config": 5,
+     "src": "selected_attention_b200/csrc/bsa_bwd.cu", "src_sha1": "0e7611c58dfc"},
+    {"kernel": "bsa_bwd_q", "bytes": 5642680576 + 1057762560, "config": 5, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+     "src_sha1": "0e7611c58dfc"},
+    {"kernel": "bsa_fwd", "bytes": 4284632064 + 1075282176, "config": 5, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+     "src_sha1": "f1562c183dfe"},
+    {"kernel": "sfa_decode", "bytes": 147508480 + 4237312, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
+     "src_sha1": "6c80d26dac90"},
+]
+
+
+def ncu_traffic(kernel, config):
+    """DRAM bytes of one launch of `kernel` on workload `config` from an ncu capture, or None when
+    there is none or the kernel's source has changed since."""
+    for tr in NCU_TRAFFIC:
+        if tr["kernel"] == kernel and tr["config"] == config and tr["src_sha1"] == source_sha1(tr["src"]):
+            return tr["bytes"]
+    return None
 
 
 def visible_pairs_bsa(mask: np.ndarray, bx: int, by: int, s_q: int, s_kv: int) -> int:
@@ -229,6 +246,38 @@ def cpu_oracle_sample_decode(w, budget_s: float):
         if dt >= budget_s:
             break
     return len(done) * per_batch, dt, f"oracle decode of {len(done)} of {w.B} batches"
+
+
+def decode_dout(w):
+    """The synthetic dOut of the paged decode workload: bf16 bits [B, 1, N1, D]."""
+    return synth.normal_rows_bf16(w.seed, "dout", w.B, w.N1 * w.D, 1).reshape(w.B, 1, w.N1, w.D)
+
+
+def cpu_oracle_sample_decode_bwd(w, budget_s: float):
+    """Time the fp64 oracle backward of the decode one batch at a time (the batch's selected pages
+    gathered into small caches) until budget_s of oracle time has passed; returns (bytes credited:
+    gathered rows read plus gradient rows written, seconds, description)."""
+    from oracle import attention as A
+    table, idx = w.selection()
+    seqused = np.full(w.B, w.context, np.int32)
+    q, qr, do = w.query("q"), w.query("q_rope"), decode_dout(w)
+    per_batch = 2 * w.count * w.sparse_block * (w.D + w.Dr + w.D) * 2
+    ppb = w.sparse_block // w.page
+    done, dt = [], 0.0
+    for b in range(w.B):
+        logical = sorted({int(j) * ppb + x for j in idx[b, 0, 0] if j >= 0 for x in range(ppb)})
+        phys = [int(table[b, lp]) for lp in logical]
+        small = {tag: w.pages(tag, phys) for tag in ("k", "k_rope", "v")}
+        t2 = np.zeros((1, table.shape[1]), np.int32)
+        t2[0, logical] = np.arange(len(logical), dtype=np.int32)
+        t0 = time.perf_counter()
+        A.sfa_backward(q[b:b + 1], qr[b:b + 1], small["k"], small["k_rope"], small["v"], do[b:b + 1], t2,
+                       idx[b:b + 1], seqused[b:b + 1], w.page, w.sparse_block, w.scale)
+        dt += time.perf_counter() - t0
+        done.append(b)
+        if dt >= budget_s:
+            break
+    return len(done) * per_batch, dt, f"oracle decode backward of {len(done)} of {w.B} batches"
 
 
 def visible_pairs_nsa(w, topk: np.ndarray) -> int:
@@ -428,6 +477,10 @@ def run_reference(args, rank, world):
         mask = w.block_mask()
         sample = lambda: cpu_oracle_sample(w, mask, budget_s=step_budget)  # noqa: E731
         cfg = config_dict(w, args)
+    elif getattr(args, "decode_bwd", False):  # the decode's backward: gathered and gradient bytes per second
+        sample = lambda: cpu_oracle_sample_decode_bwd(w, budget_s=step_budget)  # noqa: E731
+        cfg = dict(config_dict_decode(w), op="backward")
+        metric, unit, scale = METRIC_DEC_BWD, "GB/s", 1e9
     else:  # paged sparse decode: gathered bytes per second
         sample = lambda: cpu_oracle_sample_decode(w, budget_s=step_budget)  # noqa: E731
         cfg = config_dict_decode(w)
@@ -599,8 +652,7 @@ def run_nsa(args, rank, world, local_rank):
         launches, total = prof[dom]
         avg_ms = total / launches
         achieved = alg[dom] / (avg_ms * 1e-3) / 1e12
-        tr = NCU_TRAFFIC.get(dom)
-        traffic = tr["bytes"] if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) else None
+        traffic = ncu_traffic(dom, args.config)
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_desc, "traffic": traffic,
                 "avg_launch_ms": avg_ms, "frac_of_burst": achieved / peaks["bf16_tflops"]}
@@ -729,8 +781,7 @@ def run_decode(args, rank, world, local_rank):
     value = world * gathered / (ms * 1e-3) / 1e9  # every rank decodes its own copy of the batch
     dec_ms = prof["sfa_decode"][1] / prof["sfa_decode"][0] if "sfa_decode" in prof else None
     dec_gbs = gathered / (dec_ms * 1e-3) / 1e9 if dec_ms else None
-    tr = NCU_TRAFFIC["sfa_decode"]
-    dec_traffic = tr["bytes"] if tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config else None
+    dec_traffic = ncu_traffic("sfa_decode", args.config)
     line = {
         "metric": METRIC_DEC, "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -748,6 +799,138 @@ def run_decode(args, rank, world, local_rank):
                                "avg_launch_ms": dec_ms}),
         "kernels": {n: {"launches": c, "ms_per_call": t / c} for n, (c, t) in prof.items()},
         "cpu_baseline": cpu, "clocks": clocks.summary(), "gathered_bytes_per_step": gathered,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+
+
+def run_decode_bwd(args, rank, world, local_rank):
+    """Backward of the paged sparse decode workload: each timed rep is one CUDA-graph replay of the
+    whole backward call (page lists, readers of each cache row-block, preprocess, the token-major
+    products, the dQ sum, the cache-row scatter) after an L2 flush.  Credited bytes: the gathered
+    K, K_rope, V rows read and their gradient rows written."""
+    import torch
+
+    import selected_attention_b200 as sa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.workload(4)
+    table, idx = w.selection()
+    seqused = np.full(w.B, w.context, np.int32)
+    used = np.unique(table[np.arange(w.B)[:, None], idx[:, 0, 0, :]].ravel())
+    caches, grads = {}, {}
+    for tag, d in (("k", 512), ("k_rope", 64), ("v", 512)):
+        t = torch.zeros((w.n_pages, w.page, 1, d), dtype=torch.bfloat16, device=dev)
+        t[torch.from_numpy(used).long().to(dev)] = torch.from_numpy(w.pages(tag, used)).view(torch.bfloat16).to(dev)
+        caches[tag] = t
+        grads[tag] = torch.zeros_like(t)
+    q = torch.from_numpy(w.query("q")).view(torch.bfloat16).to(dev)
+    qr = torch.from_numpy(w.query("q_rope")).view(torch.bfloat16).to(dev)
+    do = torch.from_numpy(decode_dout(w)).view(torch.bfloat16).to(dev)
+    tb, ti, tu = (torch.from_numpy(x).to(dev) for x in (table, idx, seqused))
+    out, lse = sa.sfa_sparse_decode(q, qr, caches["k"], caches["k_rope"], caches["v"], tb, ti, tu, w.sparse_block,
+                                    w.scale)
+    p = sa.sfa_params(q, caches["k"], tb, ti, tu, w.sparse_block, w.scale)
+    ws = torch.empty(sa.sfa_sparse_decode_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    dq, dqr = torch.empty_like(q), torch.empty_like(qr)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call(qq=q, qqr=qr, dd=do, oo=out, ll=lse, t_b=tb, t_i=ti, t_u=tu):
+        sa.sfa_sparse_decode_bwd(qq, qqr, caches["k"], caches["k_rope"], caches["v"], oo, dd, ll, t_b, t_i, t_u,
+                                 w.sparse_block, w.scale, dq=dq, dq_rope=dqr, dk_cache=grads["k"],
+                                 dk_rope_cache=grads["k_rope"], dv_cache=grads["v"], workspace=ws)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    torch.cuda.synchronize()
+    tokens = int(w.B * w.count * w.sparse_block)
+    moved = 2 * tokens * (w.D + w.Dr + w.D) * 2
+    flops = tokens * w.N1 * 2 * (3 * (w.D + w.Dr) + 2 * w.D)
+    barrier, max_over_ranks = _dist_helpers(world, dev)
+    times = []
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        barrier()
+    ms = max_over_ranks(float(np.mean(times)))
+    assert sa.bsa_get_status(ws) == 0
+    sa.bsa_profile_enable(True)
+    for _ in range(3):
+        flush.fill_(1)
+        call()
+    prof = sa.bsa_profile_collect()
+    sa.bsa_profile_enable(False)
+    launches_per_call = sum(c for c, _ in prof.values()) // 3
+
+    # end to end through the API: the step's query-side inputs (q, q_rope, dOut, Out, LSE and the
+    # selection) come from pinned host memory and dQ, dQ_rope go back; the caches and their
+    # gradients are resident device state
+    named = (("q", q), ("qr", qr), ("do", do), ("o", out), ("l", lse), ("tb", tb), ("ti", ti), ("tu", tu))
+    h_in = {n_: x.cpu().pin_memory() for n_, x in named}
+    d_in = {n_: torch.empty_like(x) for n_, x in named}
+    h_dq, h_dqr = torch.empty(dq.shape, dtype=dq.dtype).pin_memory(), torch.empty(dqr.shape, dtype=dqr.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in h_in.values())
+    d2h = h_dq.numel() * h_dq.element_size() + h_dqr.numel() * h_dqr.element_size()
+
+    def e2e_step():
+        for n_ in d_in:
+            d_in[n_].copy_(h_in[n_], non_blocking=True)
+        call(d_in["q"], d_in["qr"], d_in["do"], d_in["o"], d_in["l"], d_in["tb"], d_in["ti"], d_in["tu"])
+        h_dq.copy_(dq, non_blocking=True)
+        h_dqr.copy_(dqr, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_times = []
+    barrier()
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_times.append(e0.elapsed_time(e1))
+    barrier()
+    e2e_ms = max_over_ranks(float(np.mean(e2e_times)))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f_, t_, desc = cpu_oracle_sample_decode_bwd(w, budget_s=args.cpu_seconds)
+        cpu = {"value": f_ / t_ / 1e9, "unit": "GB/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+               "kind": "oracle", "sample": desc}
+    peaks, src = measured_peaks()
+    value = world * moved / (ms * 1e-3) / 1e9
+    k_ms = prof["sfa_bwd"][1] / prof["sfa_bwd"][0] if "sfa_bwd" in prof else None
+    line = {
+        "metric": METRIC_DEC_BWD, "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_dict_decode(w), op="backward"),
+        "e2e": {"value": world * moved / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_call * args.steps,
+        "effective_tflops": world * flops / (ms * 1e-3) / 1e12,
+        # the token-major kernel reads the gathered rows; the scatter writes the gradient rows: the
+        # roofline line credits the kernel with the reads, the step with both
+        "roofline": with_spec({"bound": "hbm", "kernel": "sfa_bwd",
+                               "achieved": (moved / 2) / (k_ms * 1e-3) / 1e9 if k_ms else None,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": (moved / 2) / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"] if k_ms else None,
+                               "peak_source": f"{src} hbm_gbs (burst)", "traffic": None, "avg_launch_ms": k_ms}),
+        "kernels": {n: {"launches": c, "ms_per_call": t / c} for n, (c, t) in prof.items()},
+        "cpu_baseline": cpu, "clocks": clocks.summary(), "bytes_per_step": moved,
     }
     if rank == 0:
         print(json.dumps(line))
@@ -880,11 +1063,7 @@ def run_ours(args, rank, world, local_rank):
         launches, total = prof[dom]
         avg_ms = total / launches
         achieved = alg[dom] / len(P) / (avg_ms * 1e-3) / 1e12  # a launch's average share of the work
-        traffic = None
-        tr = NCU_TRAFFIC.get(dom)
-        if tr is not None and tr["src_sha1"] == source_sha1(tr["src"]) and tr["config"] == args.config \
-                and world == 1:
-            traffic = tr["bytes"]
+        traffic = ncu_traffic(dom, args.config) if world == 1 else None
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_source": peak_desc, "traffic": traffic, "avg_launch_ms": avg_ms,
                 "frac_of_burst": achieved / peaks["bf16_tflops"]}
@@ -929,6 +1108,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nsa-seqlens", default="", help="config 3 only: comma-separated batch lengths")
+    ap.add_argument("--decode-bwd", action="store_true", help="config 4 only: time the decode's backward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -945,7 +1125,9 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if args.config == 4:
+        if args.config == 4 and args.decode_bwd:
+            run_decode_bwd(args, rank, world, local_rank)
+        elif args.config == 4:
             run_decode(args, rank, world, local_rank)
         elif args.config == 3:
             run_nsa(args, rank, world, local_rank)
