@@ -816,6 +816,9 @@ def run_decode_bwd(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = synth.workload(4)
+    if args.decode_batches:  # a smaller batch of the same problem (profiler captures)
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}_B{args.decode_batches}", B=args.decode_batches)
     table, idx = w.selection()
     seqused = np.full(w.B, w.context, np.int32)
     used = np.unique(table[np.arange(w.B)[:, None], idx[:, 0, 0, :]].ravel())
@@ -1109,6 +1112,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nsa-seqlens", default="", help="config 3 only: comma-separated batch lengths")
     ap.add_argument("--decode-bwd", action="store_true", help="config 4 only: time the decode's backward")
+    ap.add_argument("--decode-batches", type=int, default=0, help="--decode-bwd only: fewer batches (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -25,6 +25,7 @@ std::vector<cudaEvent_t> g_pool;
 size_t g_pool_next = 0;
 std::vector<Rec> g_recs;
 int g_open = -1;
+int g_depth = 0;  // open brackets (nested ones are not recorded)
 uint64_t* g_cta_buf = nullptr;  // caller-owned device array [3][g_cta_cap][2]
 int g_cta_cap = 0;
 
@@ -39,9 +40,12 @@ cudaEvent_t take_event() {
 
 }  // namespace
 
+// A bracket opened inside another one (a launcher that times itself, called from a launcher that
+// times a group of kernels) is counted in the outer bracket only.
 void prof_begin(const char* name, cudaStream_t st) {
   if (!g_on) return;
   std::lock_guard<std::mutex> lk(g_mu);
+  if (g_depth++ > 0) return;
   Rec r{name, take_event(), take_event()};
   if (r.start && r.stop && cudaEventRecord(r.start, st) == cudaSuccess) {
     g_recs.push_back(r);
@@ -52,7 +56,8 @@ void prof_begin(const char* name, cudaStream_t st) {
 void prof_end(cudaStream_t st) {
   if (!g_on) return;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_open >= 0) cudaEventRecord(g_recs[g_open].stop, st);
+  if (g_depth > 0 && --g_depth > 0) return;
+  if (g_open >= 0 && cudaEventRecord(g_recs[g_open].stop, st) != cudaSuccess) g_recs.pop_back();
   g_open = -1;
 }
 
@@ -80,6 +85,7 @@ bsa_status bsa_profile_enable(int32_t on) {
   sa::g_recs.clear();
   sa::g_pool_next = 0;
   sa::g_open = -1;
+  sa::g_depth = 0;
   return BSA_OK;
 }
 
