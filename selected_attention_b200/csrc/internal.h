@@ -56,6 +56,11 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64
 bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                        uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2);
 
+// 3D fp32 map over [d2][d1][d0] (d0 contiguous), strides in elements, box {box0, box1, box2}
+// (box0 * 4 bytes <= 128: the 128-byte swizzle).
+bool make_tmap_3d_f32(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+                      uint64_t stride2, uint32_t box0, uint32_t box1, uint32_t box2);
+
 // 4D bf16 map over (d0 contiguous, d1, d2, d3) with strides in elements, box {64, 1, box2, 1}: a
 // [B][..][..][D] attention tensor seen as (head dim, head, position, batch) whatever the order of
 // head and position in memory (BNSD or BSND).  Rows past d2 read as zero and are not stored.

@@ -17,7 +17,9 @@
 // [0, 256); the element-wise warps turn them into P^T and dS^T (bf16) in shared memory, the
 // K-major A operands of dv~ / dk~ (and, read MN-major, of dQ_t).  The 14 column chunks of the three
 // gradient products then alternate between two 128-column TMEM buffers, so the warps write one
-// chunk out while the next is computed.  Every operand tile streams through one ring of 32 KB
+// chunk out while the next is computed: each warp stages its 32 rows x 64 columns in shared memory
+// and writes them with one TMA store (rows of the outputs are 1 KB or more apart, so the TMEM
+// layout, one row per thread, would otherwise cost a separate 32-byte sector per thread and store).  Every operand tile streams through one ring of 32 KB
 // stages (two 16 KB [128 rows][64] tiles, 128-byte swizzle) in the order the products use them;
 // q, dOut and the tile's k~ are read twice (L2-resident: one batch's q and dOut are 272 KB).
 //
@@ -43,7 +45,7 @@ constexpr int kDR = 64;        // rope dim
 constexpr int kDK = kDQ + kDR;  // q|q_rope, k|k_rope
 constexpr int kQC = 9;         // 64-wide chunks of q|q_rope
 constexpr int kVC = 8;         // 64-wide chunks of v / dOut
-constexpr int kRing = 4;       // ring stages
+constexpr int kRing = 3;       // ring stages
 constexpr int kCw = 8;         // element-wise / epilogue warps
 constexpr int kThreads = (kCw + 2) * 32;  // + producer, MMA issuer
 constexpr uint32_t kTile = kTok * 128;    // [128 rows][64 bf16], 16 KB
@@ -56,6 +58,7 @@ struct __align__(1024) BwdSmem {
   uint8_t ring[kRing][2][kTile];   // stages of two tiles
   uint8_t pt[2][kTile];            // P^T  [128 tok][2 x 64 heads] bf16 (K-major atoms of 64 heads)
   uint8_t dst[2][kTile];           // dS^T
+  uint8_t stage_out[kCw][4096];    // per epilogue warp: [32 rows][128 B] of output, then a TMA store
   float lse2[128], dvec[128];      // per head: LSE log2(e), rowsum(dOut o Out)
   int32_t vrow[kTok];              // gathered row in use (1) or masked (0)
   uint64_t full[kRing], empty[kRing];
@@ -71,9 +74,7 @@ struct BwdParams {
   const int32_t* count;
   const float* lse2;
   const float* dvec;
-  float* dqp;              // [unit][T][G][576] fp32
-  __nv_bfloat16* gk;       // [unit][cap * page_size][576]
-  __nv_bfloat16* gv;       // [unit][cap * page_size][512]
+  int rows_u;              // cap * page_size: gathered rows per unit
   uint32_t* status;
 };
 
@@ -101,7 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sfa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v,
-                   const BwdParams prm) {
+                   const __grid_constant__ CUtensorMap tm_gk, const __grid_constant__ CUtensorMap tm_gv,
+                   const __grid_constant__ CUtensorMap tm_dqp, const BwdParams prm) {
   griddep_launch_dependents();
   griddep_wait();  // page lists and the preprocess must be complete
   const int u = blockIdx.y, t = blockIdx.x;  // unit (b, g), tile
@@ -327,8 +329,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
     }
     mbar_arrive(&s.bar_ops);
-    // epilogue of the 14 column chunks
-    const size_t grow = static_cast<size_t>(u) * prm.cap * prm.page_size + static_cast<size_t>(t) * kTok + r;
+    // epilogue of the 14 column chunks: rows 32 quarter .. +31 and columns 64 half .. +63 of each
+    uint8_t* so = s.stage_out[warp];
+    const int row0 = t * kTok + quarter * 32;  // gathered row of lane 0 (dv~, dk~)
+    auto flush = [&]() {  // the staged block has been read by its TMA store; the buffer is free
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+    };
     for (int j = 0; ok && j < kChunks; ++j) {
       const int buf = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s.chunk_full[buf], (j >> 1) & 1, prm.status));
@@ -341,41 +348,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(col, v);
         tmem_ld32(col + 32, w);
         tmem_ld_wait(v);
-        if (j < 9 && s.vrow[r]) {
-          // dv~ (j < 4) or dk~ (scaled) rows in use, bf16, gathered order
+        if (j < 9) {
+          // dv~ (j < 4) or dk~ (scaled) rows, bf16, gathered order: row lane of the block
           const float mul = j < 4 ? 1.f : prm.scale;
-          __nv_bfloat16* dstp = j < 4 ? prm.gv + grow * kDQ + j * 128 + half * 64
-                                      : prm.gk + grow * kDK + (j - 4) * 128 + half * 64;
-          uint4* o = reinterpret_cast<uint4*>(dstp);
+          uint32_t pk[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            o[q] = make_uint4(pack_bf16(__uint_as_float(v[8 * q]) * mul, __uint_as_float(v[8 * q + 1]) * mul),
-                              pack_bf16(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul),
-                              pack_bf16(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul),
-                              pack_bf16(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul));
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = pack_bf16(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+            pk[16 + i] = pack_bf16(__uint_as_float(w[2 * i]) * mul, __uint_as_float(w[2 * i + 1]) * mul);
+          }
+          flush();
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            o[4 + q] = make_uint4(pack_bf16(__uint_as_float(w[8 * q]) * mul, __uint_as_float(w[8 * q + 1]) * mul),
-                                  pack_bf16(__uint_as_float(w[8 * q + 2]) * mul, __uint_as_float(w[8 * q + 3]) * mul),
-                                  pack_bf16(__uint_as_float(w[8 * q + 4]) * mul, __uint_as_float(w[8 * q + 5]) * mul),
-                                  pack_bf16(__uint_as_float(w[8 * q + 6]) * mul, __uint_as_float(w[8 * q + 7]) * mul));
-        } else if (j >= 9 && r < prm.G) {
-          // dQ_t row of head r, fp32 (the scale is applied when the tiles are summed)
-          float4* o = reinterpret_cast<float4*>(prm.dqp + ((static_cast<size_t>(u) * prm.T + t) * prm.G + r) * kDK +
-                                                (j - 9) * 128 + half * 64);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(so + sw128(lane, c)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < prm.rows_u) {
+            if (j < 4) tma_store_3d(&tm_gv, so, j * 128 + half * 64, row0, u);
+            else tma_store_3d(&tm_gk, so, (j - 4) * 128 + half * 64, row0, u);
+            bulk_commit();
+          }
+        } else if (quarter * 32 < prm.G) {
+          // dQ_t rows of heads 32 quarter .. (fp32, the scale is applied when the tiles are summed),
+          // in two blocks of 32 columns
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            o[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                               __uint_as_float(v[4 * q + 3]));
+          for (int p2 = 0; p2 < 2; ++p2) {
+            flush();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            o[8 + q] = make_float4(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1]),
-                                   __uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3]));
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* src = p2 ? w : v;
+              *reinterpret_cast<uint4*>(so + sw128(lane, c)) =
+                  make_uint4(src[4 * c], src[4 * c + 1], src[4 * c + 2], src[4 * c + 3]);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tm_dqp, so, (j - 9) * 128 + half * 64 + p2 * 32, quarter * 32, u * prm.T + t);
+              bulk_commit();
+            }
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&s.chunk_free[buf]);
     }
+    if (lane == 0) bulk_wait_all();  // the stores are complete before the CTA exits
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -580,19 +598,26 @@ cudaError_t sfa_bwd_launch(const SfaBwdArgs& a, cudaStream_t st) {
       !make_tmap_3d_bf16(&tkr, a.k_rope_cache, kDR, a.N2, tokens, kDR, static_cast<uint64_t>(a.N2) * kDR, 1, sub) ||
       !make_tmap_3d_bf16(&tv, a.v_cache, kDQ, a.N2, tokens, kDQ, static_cast<uint64_t>(a.N2) * kDQ, 1, sub))
     return cudaErrorInvalidValue;
+  // outputs: gathered rows [U][cap * page_size][576 | 512] bf16, dQ_t [U * T][G][576] fp32
+  CUtensorMap tgk, tgv, tdqp;
+  const uint64_t rows_u = static_cast<uint64_t>(cap) * a.page_size;
+  if (!make_tmap_3d_bf16(&tgk, a.gk, kDK, rows_u, U, kDK, rows_u * kDK, 32, 1) ||
+      !make_tmap_3d_bf16(&tgv, a.gv, kDQ, rows_u, U, kDQ, rows_u * kDQ, 32, 1) ||
+      !make_tmap_3d_f32(&tdqp, a.dqp, kDK, G, static_cast<uint64_t>(U) * T, kDK, static_cast<uint64_t>(G) * kDK, 32, 32,
+                        1))
+    return cudaErrorInvalidValue;
   BwdParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.G = G; p.Gp = (G + 15) / 16 * 16; p.K = a.meta.K; p.ppb = a.meta.ppb;
   p.page_size = a.page_size; p.cap = cap; p.sub_rows = sub; p.T = T;
   p.scale = a.scale; p.scale_log2 = a.scale * kLog2e;
   p.pages = a.meta.pages; p.tokens = a.meta.tokens; p.count = a.meta.count;
-  p.lse2 = a.lse2; p.dvec = a.dvec; p.dqp = a.dqp;
-  p.gk = static_cast<__nv_bfloat16*>(a.gk); p.gv = static_cast<__nv_bfloat16*>(a.gv); p.status = a.meta.status;
+  p.lse2 = a.lse2; p.dvec = a.dvec; p.rows_u = cap * a.page_size; p.status = a.meta.status;
   const size_t smem = sizeof(BwdSmem) + 1024;
   if ((e = cudaFuncSetAttribute(sfa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
     return e;
   if (T > 0 && U > 0) {
     prof_begin("sfa_bwd", st);
-    e = launch_pdl(sfa_bwd_kernel, dim3(T, U), dim3(kThreads), smem, st, tq, tqr, tdo, tk, tkr, tv, p);
+    e = launch_pdl(sfa_bwd_kernel, dim3(T, U), dim3(kThreads), smem, st, tq, tqr, tdo, tk, tkr, tv, tgk, tgv, tdqp, p);
     prof_end(st);
     if (e != cudaSuccess) return e;
   }
