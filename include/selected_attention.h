@@ -209,11 +209,12 @@ BSA_API bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const v
  *   (bf16, same shape) and lse (fp32 [B, 1, N1], natural log).  Outputs (bf16): dq [B, 1, N1, 512],
  *   dq_rope [B, 1, N1, 64], and dk_cache, dv_cache [num_pages, page_size, N2, 512], dk_rope_cache
  *   [num_pages, page_size, N2, 64], laid out as the caches.
- *   Every cache row the step read (a token in use of a selected page of batch b, kv head g) is SET
- *   to the sum of its gathered rows' gradients: a page listed twice, or reached from two batches'
- *   block tables, adds each read; the sum runs in a fixed order (deterministic).  Cache rows the
- *   step did not read are NOT written: zero the three gradient caches first to obtain the full
- *   cache gradient.  P and dS enter the tensor cores as bf16.
+ *   Every row of a page the step read (kv head g of a page holding a selected block of batch b) is
+ *   SET: a row in use gets the sum of its gathered rows' gradients (a page listed twice, or reached
+ *   from two batches' block tables, adds each read; the sum runs in a fixed order, so the result is
+ *   deterministic), a row past the sequence's end gets zero.  Rows of pages the step did not read
+ *   are NOT written: zero the three gradient caches first to obtain the full cache gradient.  P and
+ *   dS enter the tensor cores as bf16.
  *   Host errors: as sfa_sparse_decode, plus BSA_ERR_UNSUPPORTED when p->plan is set or
  *   num_pages * N2 >= 2^30.  Device status bits: as sfa_sparse_decode.  The workspace holds the
  *   page lists, per-tile parts of dq and the gathered-order row gradients (about

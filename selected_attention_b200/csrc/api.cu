@@ -486,8 +486,8 @@ bsa_status sfa_sparse_decode(const bsa_params* p, const void* q, const void* q_r
 struct SfaBwdWs {
   uint32_t* status;
   int32_t *pages, *tokens, *count, *cnt, *ptr, *list;
-  float *lse2, *dvec, *dqp;
-  uint16_t *gk, *gv;
+  float *lse2, *dvec;
+  uint16_t *ds, *gk, *gv;
 };
 
 size_t carve_sfa_bwd(const bsa_params* p, void* ws, SfaBwdWs* w) {
@@ -506,7 +506,7 @@ size_t carve_sfa_bwd(const bsa_params* p, void* ws, SfaBwdWs* w) {
   w->list = c.take<int32_t>(U * cap);
   w->lse2 = c.take<float>(static_cast<size_t>(p->B) * p->N1);
   w->dvec = c.take<float>(static_cast<size_t>(p->B) * p->N1);
-  w->dqp = c.take<float>(U * T * (p->N1 / p->N2) * 576);
+  w->ds = c.take<uint16_t>(U * T * 128 * 128);
   w->gk = c.take<uint16_t>(rows * 576);
   w->gv = c.take<uint16_t>(rows * 512);
   return c.bytes();
@@ -547,7 +547,7 @@ bsa_status sfa_sparse_decode_bwd(const bsa_params* p, const void* q, const void*
   a.q = q; a.q_rope = q_rope; a.k_cache = k_cache; a.k_rope_cache = k_rope_cache; a.v_cache = v_cache;
   a.out = out; a.dout = dout; a.lse = lse;
   a.dq = dq; a.dq_rope = dq_rope; a.dk_cache = dk_cache; a.dk_rope_cache = dk_rope_cache; a.dv_cache = dv_cache;
-  a.lse2 = w.lse2; a.dvec = w.dvec; a.dqp = w.dqp; a.gk = w.gk; a.gv = w.gv;
+  a.lse2 = w.lse2; a.dvec = w.dvec; a.ds = w.ds; a.gk = w.gk; a.gv = w.gv;
   a.cnt = w.cnt; a.ptr = w.ptr; a.list = w.list;
   return cuda_status(sfa_bwd_launch(a, st));
 }

@@ -170,7 +170,7 @@ struct SfaBwdArgs {
   void *dq, *dq_rope, *dk_cache, *dk_rope_cache, *dv_cache;
   // workspace
   float *lse2, *dvec;  // [B * N1]
-  float* dqp;          // [U][T][G][576], T = tiles of 128 gathered tokens per unit
+  void* ds;            // [U][T * 128][128] bf16: each tile's dS^T (T = tiles of 128 gathered tokens per unit)
   void *gk, *gv;       // gathered-order row gradients [U][cap * page_size][576] / [..][512] bf16
   int32_t *cnt;        // [2][num_pages * N2]: readers per cache row-block, then the fill cursor
   int32_t *ptr;        // [num_pages * N2 + 1]

@@ -12,24 +12,26 @@
 //   dP^T [128 tok][G] = v~ . dOut^T                           (8 chunks)
 //   dv~ [128 tok][512] = P^T . dOut                           (4 column chunks of 128)
 //   dk~ [128 tok][576] = dS^T . [q | q_rope]                  (4 chunks of 128 + 1 of 64)
-//   dQ_t [G][576]      = dS . [k~ | k_rope~]                   (the tile's part of dQ, 5 chunks)
 // One CTA per (batch, kv head, tile of 128 gathered tokens).  S^T and dP^T take TMEM columns
 // [0, 256); the element-wise warps turn them into P^T and dS^T (bf16) in shared memory, the
-// K-major A operands of dv~ / dk~ (and, read MN-major, of dQ_t).  The 14 column chunks of the three
-// gradient products then alternate between two 128-column TMEM buffers, so the warps write one
-// chunk out while the next is computed: each warp stages its 32 rows x 64 columns in shared memory
-// and writes them with one TMA store (rows of the outputs are 1 KB or more apart, so the TMEM
-// layout, one row per thread, would otherwise cost a separate 32-byte sector per thread and store).  Every operand tile streams through one ring of 32 KB
-// stages (two 16 KB [128 rows][64] tiles, 128-byte swizzle) in the order the products use them;
-// q, dOut and the tile's k~ are read twice (L2-resident: one batch's q and dOut are 272 KB).
+// K-major A operands of dv~ / dk~, and the tile's dS^T is also stored for the dQ kernel.  The 9
+// column chunks of the two gradient products alternate between two 128-column TMEM buffers, so the
+// warps write one chunk out while the next is computed: each warp stages its 32 rows x 64 columns
+// in shared memory and writes them with one TMA store (rows of the outputs are 1 KB or more apart,
+// so the TMEM layout, one row per thread, would otherwise cost a separate 32-byte sector per thread
+// and store).  Every operand tile streams through one ring of 32 KB stages (two 16 KB [128 rows][64]
+// tiles, 128-byte swizzle) in the order the products use them; q and dOut are read twice
+// (L2-resident: one batch's q and dOut are 272 KB).
 //
-// Outputs per tile: dv~ and dk~ rows (bf16) into a gathered-order scratch, dQ_t (fp32) into a
-// per-tile scratch.  A second kernel sums each (batch, head)'s dQ_t in tile order; a third writes
-// every cache row the step read: the sum, in a fixed order, of the gathered rows read from it (a
-// page listed twice, or reached from two batches, adds its contributions), so the result does not
-// depend on scheduling.  Rows of a page past its tokens in use are masked (P = dS = 0) and the
-// tile's k~ rows there are zeroed before dQ_t (a non-finite value in a cache tail would turn
-// 0 * x into NaN).
+// dv~ and dk~ rows (bf16) go straight into the cache gradients when their page has one reader (the
+// common case), else into a gathered-order scratch.  The dQ kernel accumulates
+//   dQ [G][64-dim chunk] = sum over the unit's tiles of dS . [k~ | k_rope~]
+// in TMEM (one CTA per (batch, kv head, 64-dim chunk), tiles in order), and a third kernel writes
+// the rows of every page with two or more readers: the sum, in a fixed order, of the gathered rows
+// read from it (a page listed twice, or reached from two batches, adds its contributions), so no
+// result depends on scheduling.  Every row of a page the step read is written (rows past the
+// sequence's end get zero).  Rows of a page past its tokens in use are masked (P = dS = 0), and the
+// dQ kernel zeroes the k~ rows there (a non-finite value in a cache tail would turn 0 * x into NaN).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -49,8 +51,8 @@ constexpr int kRing = 3;       // ring stages
 constexpr int kCw = 8;         // element-wise / epilogue warps
 constexpr int kThreads = (kCw + 2) * 32;  // + producer, MMA issuer
 constexpr uint32_t kTile = kTok * 128;    // [128 rows][64 bf16], 16 KB
-constexpr int kStages = kQC + kVC + 4 + 5 + 5;  // 31 per tile
-constexpr int kChunks = 14;                     // 4 dv~ + 5 dk~ + 5 dQ_t
+constexpr int kStages = kQC + kVC + 4 + 5;  // 26 per tile
+constexpr int kChunks = 9;                 // 4 dv~ + 5 dk~
 constexpr uint32_t kColS = 0, kColDP = 128, kColOut = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -75,6 +77,7 @@ struct BwdParams {
   const float* lse2;
   const float* dvec;
   int rows_u;              // cap * page_size: gathered rows per unit
+  const int32_t* refs;     // [num_pages * N2]: readers of each cache row-block (page, kv head)
   uint32_t* status;
 };
 
@@ -89,9 +92,7 @@ __device__ __forceinline__ StageDef stage_def(int s) {
   s -= kQC + kVC;
   if (s < 4) return {3, 2 * s, 3, 2 * s + 1};             // dv~ chunk: dOut pair
   s -= 4;
-  if (s < 5) return {2, 2 * s, 2, s < 4 ? 2 * s + 1 : -1};  // dk~ chunk: Q pair (the last: q_rope)
-  s -= 5;
-  return {0, 2 * s, 0, s < 4 ? 2 * s + 1 : -1};           // dQ_t chunk: K~ pair (the last: k_rope)
+  return {2, 2 * s, 2, s < 4 ? 2 * s + 1 : -1};           // dk~ chunk: Q pair (the last: q_rope)
 }
 
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
@@ -103,7 +104,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_gk, const __grid_constant__ CUtensorMap tm_gv,
-                   const __grid_constant__ CUtensorMap tm_dqp, const BwdParams prm) {
+                   const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_dkc,
+                   const __grid_constant__ CUtensorMap tm_dkrc, const __grid_constant__ CUtensorMap tm_dvc,
+                   const BwdParams prm) {
   griddep_launch_dependents();
   griddep_wait();  // page lists and the preprocess must be complete
   const int u = blockIdx.y, t = blockIdx.x;  // unit (b, g), tile
@@ -228,9 +231,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the three gradient products, once P^T and dS^T are in shared memory
     if (ok && lane == 0) ok = mbar_wait(&s.bar_ops, 0, prm.status);
     ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && lane == 0) {  // the tile's dS^T for the dQ kernel: two [128 tok][64 heads] boxes
+      tma_store_3d(&tm_ds, s.dst[0], 0, t * kTok, u);
+      tma_store_3d(&tm_ds, s.dst[1], 64, t * kTok, u);
+      bulk_commit();
+    }
     const uint64_t dpt = sdesc_sw128(smem_u32(s.pt[0]), 0, 1024);  // K-major A, atoms 16 KB apart
     const uint64_t dds = sdesc_sw128(smem_u32(s.dst[0]), 0, 1024);
-    const uint64_t dds_mn = sdesc_sw128(smem_u32(s.dst[0]), kTile, 1024);  // dS as MN-major A (M = heads)
     const int ksteps = prm.Gp / 16;
     for (int j = 0; ok && j < kChunks; ++j, ++st) {
       const int buf = j & 1;
@@ -239,50 +246,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (!(ok = wait_stage(st))) break;
       const int slot = st % kRing;
-      const bool rope = (j == 8 || j == 13);  // the 64-wide last chunk of dk~ / dQ_t
+      const bool rope = j == 8;  // the 64-wide last chunk of dk~
       const int n = rope ? 64 : 128;
-      if (j >= 9) {
-        // dQ_t reads the tile's k~ rows as B: zero the rows that are masked (cache tails, boxes past
-        // the unit's end), so 0 * x cannot become NaN
-        bool any = false;
-        for (int r = lane; r < kTok; r += 32) any |= s.vrow[r] == 0;
-        if (__any_sync(0xffffffffu, any)) {
-          // every lane observes the copy's completion itself before it overwrites part of it
-          ok = __all_sync(0xffffffffu, mbar_wait(&s.full[slot], (st / kRing) & 1, prm.status));
-          if (!ok) break;
-          for (int x = 0; x < (rope ? 1 : 2); ++x) {
-            uint8_t* tile = s.ring[slot][x];
-            for (int r = 0; r < kTok; ++r) {
-              if (s.vrow[r]) continue;
-              if (lane < 8) *reinterpret_cast<uint4*>(tile + r * 128 + lane * 16) = make_uint4(0u, 0u, 0u, 0u);
-            }
-          }
-          fence_async_smem();
-          __syncwarp();
-        }
-      }
       if (lane == 0) {
         tc_fence_after();
         const uint64_t bst = sdesc_sw128(smem_u32(s.ring[slot][0]), kTile, 1024);  // MN-major B, N chunks 16 KB apart
         const uint32_t d = tmem + kColOut + buf * 128;
-        if (j < 9) {
-          // dv~ / dk~: M = tokens, K = heads: A = P^T or dS^T (K-major), B = dOut / Q pair (MN-major)
-          const uint32_t id = idesc_bf16_f32(kTok, n, false, true);
-          const uint64_t a0 = j < 4 ? dpt : dds;
-          for (int ks = 0; ks < ksteps; ++ks)
-            mma_bf16_ss(d, sdesc_add(a0, (ks >> 2) * kTile + (ks & 3) * 32), sdesc_add(bst, ks * 2048), id,
-                        ks > 0 ? 1u : 0u);
-        } else {
-          // dQ_t: M = heads, K = tokens: A = dS (MN-major), B = k~ pair (MN-major)
-          const uint32_t id = idesc_bf16_f32(kTok, n, true, true);
-          for (int ks = 0; ks < kTok / 16; ++ks)
-            mma_bf16_ss(d, sdesc_add(dds_mn, ks * 2048), sdesc_add(bst, ks * 2048), id, ks > 0 ? 1u : 0u);
-        }
+        // dv~ / dk~: M = tokens, K = heads: A = P^T or dS^T (K-major), B = dOut / Q pair (MN-major)
+        const uint32_t id = idesc_bf16_f32(kTok, n, false, true);
+        const uint64_t a0 = j < 4 ? dpt : dds;
+        for (int ks = 0; ks < ksteps; ++ks)
+          mma_bf16_ss(d, sdesc_add(a0, (ks >> 2) * kTile + (ks & 3) * 32), sdesc_add(bst, ks * 2048), id,
+                      ks > 0 ? 1u : 0u);
         tc_commit(&s.empty[slot]);
         tc_commit(&s.chunk_full[buf]);
       }
       __syncwarp();
     }
+    if (lane == 0) bulk_wait_all();  // the dS^T store is complete before the CTA exits
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ element-wise and epilogue warps
     const int quarter = warp & 3, half = warp >> 2;
@@ -329,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
     }
     mbar_arrive(&s.bar_ops);
-    // epilogue of the 14 column chunks: rows 32 quarter .. +31 and columns 64 half .. +63 of each
+    // epilogue of the 9 column chunks: rows 32 quarter .. +31 and columns 64 half .. +63 of each
     uint8_t* so = s.stage_out[warp];
     const int row0 = t * kTok + quarter * 32;  // gathered row of lane 0 (dv~, dk~)
     auto flush = [&]() {  // the staged block has been read by its TMA store; the buffer is free
@@ -341,14 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.chunk_full[buf], (j >> 1) & 1, prm.status));
       if (!ok) break;
       tc_fence_after();
-      const bool rope = (j == 8 || j == 13);
+      const bool rope = j == 8;
       if (!(rope && half == 1)) {
         uint32_t v[32], w[32];
         const uint32_t col = tmem + lane_base + kColOut + buf * 128 + half * 64;
         tmem_ld32(col, v);
         tmem_ld32(col + 32, w);
         tmem_ld_wait(v);
-        if (j < 9) {
+        {
           // dv~ (j < 4) or dk~ (scaled) rows, bf16, gathered order: row lane of the block
           const float mul = j < 4 ? 1.f : prm.scale;
           uint32_t pk[32];
@@ -363,29 +345,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(so + sw128(lane, c)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
           fence_async_smem();
           __syncwarp();
-          if (lane == 0 && row0 < prm.rows_u) {
-            if (j < 4) tma_store_3d(&tm_gv, so, j * 128 + half * 64, row0, u);
-            else tma_store_3d(&tm_gk, so, (j - 4) * 128 + half * 64, row0, u);
+          // the block's 32 rows lie in one page of the unit's list (32 divides the page size)
+          const int entry = row0 / prm.page_size;
+          if (lane == 0 && entry < prm.count[u]) {
+            const int page = plist[entry];
+            if (prm.refs[page * prm.N2 + g] == 1) {
+              // the page's only reader: straight into the cache gradients
+              const int crow = page * prm.page_size + row0 % prm.page_size;
+              if (j < 4) tma_store_3d(&tm_dvc, so, j * 128 + half * 64, g, crow);
+              else if (j < 8) tma_store_3d(&tm_dkc, so, (j - 4) * 128 + half * 64, g, crow);
+              else tma_store_3d(&tm_dkrc, so, 0, g, crow);
+            } else {
+              // a page with several readers: gathered order, summed by the scatter
+              if (j < 4) tma_store_3d(&tm_gv, so, j * 128 + half * 64, row0, u);
+              else tma_store_3d(&tm_gk, so, (j - 4) * 128 + half * 64, row0, u);
+            }
             bulk_commit();
-          }
-        } else if (quarter * 32 < prm.G) {
-          // dQ_t rows of heads 32 quarter .. (fp32, the scale is applied when the tiles are summed),
-          // in two blocks of 32 columns
-#pragma unroll
-          for (int p2 = 0; p2 < 2; ++p2) {
-            flush();
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint32_t* src = p2 ? w : v;
-              *reinterpret_cast<uint4*>(so + sw128(lane, c)) =
-                  make_uint4(src[4 * c], src[4 * c + 1], src[4 * c + 2], src[4 * c + 3]);
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_3d(&tm_dqp, so, (j - 9) * 128 + half * 64 + p2 * 32, quarter * 32, u * prm.T + t);
-              bulk_commit();
-            }
           }
         }
       }
@@ -426,31 +401,154 @@ __global__ void sfa_bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const
   }
 }
 
-// dQ, dQ_rope of (unit u, head h) = scale * the sum of the unit's tiles' dQ_t rows, in tile order.
-__global__ void sfa_bwd_dq_kernel(const float* __restrict__ dqp, const int32_t* __restrict__ count, int N1, int N2,
-                                  int G, int T, int spp, int n_sub, float scale, __nv_bfloat16* __restrict__ dq,
-                                  __nv_bfloat16* __restrict__ dqr) {
-  griddep_wait();
+// dQ of one (unit, 64-dim chunk of q | q_rope): D [128 heads][64 dims] = sum over the unit's tiles
+// t (in order) of dS_t [heads][128 tok] . k~_t [128 tok][64 dims], accumulated in TMEM.  A = the
+// stored dS^T tile read MN-major (M = heads), B = the tile's gathered k~ chunk read MN-major.
+// Warps: 0-3 epilogue (TMEM lane quarter = 32 heads), 4 producer, 5 issuer (it first zeroes the k~
+// rows past a page's tokens in use: those rows have dS = 0, but a non-finite cache value would
+// still turn 0 * x into NaN).
+constexpr int kDqRing = 3;
+constexpr int kDqThreads = 6 * 32;
+
+struct __align__(1024) DqSmem {
+  uint8_t ds[kDqRing][2][kTile];  // dS^T [128 tok][2 x 64 heads]
+  uint8_t k[kDqRing][kTile];      // k~ chunk [128 tok][64 dims]
+  uint64_t full[kDqRing], empty[kDqRing], done;
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(kDqThreads, 1)
+    sfa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_kr, const BwdParams prm, __nv_bfloat16* __restrict__ dq,
+                      __nv_bfloat16* __restrict__ dqr) {
   griddep_launch_dependents();
-  const int u = blockIdx.y, h = blockIdx.x;
-  const int b = u / N2, g = u % N2;
-  const int n_tiles = (count[u] * spp + n_sub - 1) / n_sub;
-  const size_t row = static_cast<size_t>(b) * N1 + g * G + h;
-  for (int c = threadIdx.x; c < kDK / 4; c += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t = 0; t < n_tiles; ++t) {
-      const float4 v = reinterpret_cast<const float4*>(dqp + ((static_cast<size_t>(u) * T + t) * G + h) * kDK)[c];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+  griddep_wait();  // the dS^T tiles must be complete
+  const int c = blockIdx.x, u = blockIdx.y;  // 64-dim chunk (8: q_rope), unit (b, g)
+  const int b = u / prm.N2, g = u % prm.N2;
+  const int sub = prm.sub_rows, spp = prm.page_size / sub, n_sub = kTok / sub;
+  const int n_chunks = prm.count[u] * spp;
+  const int n_tiles = (n_chunks + n_sub - 1) / n_sub;
+  extern __shared__ uint8_t smem_raw[];
+  DqSmem& s = *reinterpret_cast<DqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t* plist = prm.pages + static_cast<size_t>(u) * prm.cap;
+  const int32_t* tlist = prm.tokens + static_cast<size_t>(u) * prm.cap;
+  if (tid == 0) {
+    for (int i = 0; i < kDqRing; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
     }
-    uint2 pk;
-    pk.x = pack_bf16(acc.x * scale, acc.y * scale);
-    pk.y = pack_bf16(acc.z * scale, acc.w * scale);
-    if (c < kDQ / 4) *reinterpret_cast<uint2*>(dq + row * kDQ + 4 * c) = pk;
-    else *reinterpret_cast<uint2*>(dqr + row * kDR + 4 * (c - kDQ / 4)) = pk;
+    mbar_init(&s.done, 1);
+    fence_mbar_init();
   }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  if (warp == 4) {
+    // ------------------------------------------------------------------ producer
+    bool ok = true;
+    for (int t = 0; ok && t < n_tiles; ++t) {
+      const int slot = t % kDqRing;
+      if (lane == 0 && t >= kDqRing) ok = mbar_wait(&s.empty[slot], ((t / kDqRing) - 1) & 1, prm.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&s.full[slot], 3 * kTile);
+        tma_load_3d(s.ds[slot][0], &tm_ds, &s.full[slot], 0, t * kTok, u);
+        tma_load_3d(s.ds[slot][1], &tm_ds, &s.full[slot], 64, t * kTok, u);
+      }
+      __syncwarp();
+      if (lane < n_sub) {  // box lane of the tile; a box past the unit's end repeats the first
+        const int qb0 = t * n_sub + lane;
+        const int qb = qb0 < n_chunks ? qb0 : t * n_sub;
+        const int tok = plist[qb / spp] * prm.page_size + (qb % spp) * sub;
+        uint8_t* bx = s.k[slot] + lane * sub * 128;
+        if (c < 8) tma_load_3d(bx, &tm_k, &s.full[slot], c * 64, g, tok);
+        else tma_load_3d(bx, &tm_kr, &s.full[slot], 0, g, tok);
+      }
+      __syncwarp();
+    }
+    if (lane == 0)
+      for (int t = (n_tiles > kDqRing ? n_tiles - kDqRing : 0); t < n_tiles; ++t)
+        mbar_wait(&s.full[t % kDqRing], (t / kDqRing) & 1, prm.status);
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ zeroing + issuer
+    const uint32_t id = idesc_bf16_f32(kTok, 64, true, true);
+    bool ok = true;
+    for (int t = 0; ok && t < n_tiles; ++t) {
+      const int slot = t % kDqRing;
+      // rows in use: lane covers rows lane, lane + 32, lane + 64, lane + 96
+      uint32_t masked = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane + 32 * i;
+        const int qb = t * n_sub + r / sub, off = (qb % spp) * sub + r % sub;
+        if (!(qb < n_chunks && off < tlist[qb / spp])) masked |= 1u << i;
+      }
+      const bool any = __any_sync(0xffffffffu, masked != 0);
+      // every lane observes the copy's completion itself before it may overwrite part of it
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.full[slot], (t / kDqRing) & 1, prm.status));
+      if (!ok) break;
+      if (any) {
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t rows = __ballot_sync(0xffffffffu, (masked >> i) & 1u);
+          for (uint32_t m = rows; m; m &= m - 1) {
+            const int r = (__ffs(m) - 1) + 32 * i;
+            if (lane < 8) *reinterpret_cast<uint4*>(s.k[slot] + r * 128 + lane * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0) {
+        tc_fence_after();
+        const uint64_t da = sdesc_sw128(smem_u32(s.ds[slot][0]), kTile, 1024);  // M chunks (64 heads) 16 KB apart
+        const uint64_t db = sdesc_sw128(smem_u32(s.k[slot]), kTile, 1024);
+#pragma unroll
+        for (int ks = 0; ks < kTok / 16; ++ks)
+          mma_bf16_ss(tmem, sdesc_add(da, ks * 2048), sdesc_add(db, ks * 2048), id, (t > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(&s.empty[slot]);
+      }
+      __syncwarp();
+    }
+    if (ok && lane == 0 && n_tiles > 0) tc_commit(&s.done);
+  } else {
+    // ------------------------------------------------------------------ epilogue: head h = TMEM lane
+    const int h = warp * 32 + lane;
+    uint32_t v[32], w[32];
+    bool have = false;
+    if (n_tiles > 0) {
+      have = __all_sync(0xffffffffu, mbar_wait(&s.done, 0, prm.status));
+      if (have) {
+        tc_fence_after();
+        const uint32_t lb = static_cast<uint32_t>(warp * 32) << 16;
+        tmem_ld32(tmem + lb, v);
+        tmem_ld32(tmem + lb + 32, w);
+        tmem_ld_wait(v);
+      }
+    }
+    if (h < prm.G && (have || n_tiles == 0)) {
+      const size_t row = static_cast<size_t>(b) * prm.N1 + g * prm.G + h;
+      uint4* o = c < 8 ? reinterpret_cast<uint4*>(dq + row * kDQ + c * 64) : reinterpret_cast<uint4*>(dqr + row * kDR);
+      const float sc = prm.scale;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        pk[i] = have ? pack_bf16(__uint_as_float(v[2 * i]) * sc, __uint_as_float(v[2 * i + 1]) * sc) : 0u;
+        pk[16 + i] = have ? pack_bf16(__uint_as_float(w[2 * i]) * sc, __uint_as_float(w[2 * i + 1]) * sc) : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
 // Readers of every cache row-block (physical page, kv head): entry e = u * cap + i (page i of unit
@@ -498,9 +596,10 @@ __global__ void sfa_refs_sort_kernel(const int32_t* __restrict__ ptr, int n_keys
   }
 }
 
-// One CTA per entry; the first reader of a key writes the key's rows: row x of the page gets the
-// sum, over the key's readers in order, of their gathered row x (readers whose page has fewer
-// tokens in use skip it); a row no reader has in use is not written.
+// One CTA per entry; for a key with two or more readers, the first reader writes the key's rows:
+// row x of the page gets the sum, over the key's readers in order, of their gathered row x
+// (readers whose page has fewer tokens in use skip it), and zero where no reader has the row in
+// use.  (A key with one reader was written by the backward kernel itself.)
 __global__ void sfa_scatter_kernel(const int32_t* __restrict__ pages, const int32_t* __restrict__ tokens,
                                    const int32_t* __restrict__ count, int U, int N2, int cap, int page_size,
                                    const int32_t* __restrict__ ptr, const int32_t* __restrict__ list,
@@ -515,7 +614,7 @@ __global__ void sfa_scatter_kernel(const int32_t* __restrict__ pages, const int3
   const int g = u % N2, page = pages[e];
   const int key = page * N2 + g;
   const int a = ptr[key], z = ptr[key + 1];
-  if (list[a] != e) return;  // not the key's first reader
+  if (z - a < 2 || list[a] != e) return;  // a single reader, or not the key's first reader
   // 8 bf16 per step: 72 steps of k|k_rope and 64 of v per row
   constexpr int kStepsK = kDK / 8, kStepsV = kDQ / 8;
   for (int x = threadIdx.x; x < page_size * (kStepsK + kStepsV); x += blockDim.x) {
@@ -534,9 +633,9 @@ __global__ void sfa_scatter_kernel(const int32_t* __restrict__ pages, const int3
       acc[4] += bf16lo(w.z); acc[5] += bf16hi(w.z);
       acc[6] += bf16lo(w.w); acc[7] += bf16hi(w.w);
     }
-    if (!any) continue;
-    const uint4 o = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
-                               pack_bf16(acc[6], acc[7]));
+    const uint4 o = any ? make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
+                                     pack_bf16(acc[6], acc[7]))
+                        : make_uint4(0u, 0u, 0u, 0u);
     const size_t crow = (static_cast<size_t>(page) * page_size + row) * N2 + g;
     if (c < kDQ / 8) reinterpret_cast<uint4*>(dk + crow * kDQ)[c] = o;
     else if (c < kStepsK) reinterpret_cast<uint4*>(dkr + crow * kDR)[c - kDQ / 8] = o;
@@ -555,7 +654,6 @@ int sfa_bwd_tiles(int cap, int page_size) {
 cudaError_t sfa_bwd_launch(const SfaBwdArgs& a, cudaStream_t st) {
   const int U = a.B * a.N2, cap = a.cap, G = a.N1 / a.N2;
   const int sub = a.page_size % 64 == 0 ? 64 : 32;
-  const int spp = a.page_size / sub, n_sub = kTok / sub;
   const int T = sfa_bwd_tiles(cap, a.page_size);
   const int n_keys = a.num_pages * a.N2;
   cudaError_t e = cudaSuccess;
@@ -598,36 +696,48 @@ cudaError_t sfa_bwd_launch(const SfaBwdArgs& a, cudaStream_t st) {
       !make_tmap_3d_bf16(&tkr, a.k_rope_cache, kDR, a.N2, tokens, kDR, static_cast<uint64_t>(a.N2) * kDR, 1, sub) ||
       !make_tmap_3d_bf16(&tv, a.v_cache, kDQ, a.N2, tokens, kDQ, static_cast<uint64_t>(a.N2) * kDQ, 1, sub))
     return cudaErrorInvalidValue;
-  // outputs: gathered rows [U][cap * page_size][576 | 512] bf16, dQ_t [U * T][G][576] fp32
-  CUtensorMap tgk, tgv, tdqp;
+  // outputs: gathered rows [U][cap * page_size][576 | 512] bf16, dS^T [U][T * 128 tok][128 heads] bf16
+  CUtensorMap tgk, tgv, tds;
   const uint64_t rows_u = static_cast<uint64_t>(cap) * a.page_size;
   if (!make_tmap_3d_bf16(&tgk, a.gk, kDK, rows_u, U, kDK, rows_u * kDK, 32, 1) ||
       !make_tmap_3d_bf16(&tgv, a.gv, kDQ, rows_u, U, kDQ, rows_u * kDQ, 32, 1) ||
-      !make_tmap_3d_f32(&tdqp, a.dqp, kDK, G, static_cast<uint64_t>(U) * T, kDK, static_cast<uint64_t>(G) * kDK, 32, 32,
-                        1))
+      !make_tmap_3d_bf16(&tds, a.ds, 128, static_cast<uint64_t>(T) * kTok, U, 128, static_cast<uint64_t>(T) * kTok * 128,
+                         kTok, 1))
+    return cudaErrorInvalidValue;
+  // the cache gradients, written directly for pages with one reader: boxes of 32 rows of one head
+  CUtensorMap tdkc, tdkrc, tdvc;
+  if (!make_tmap_3d_bf16(&tdkc, a.dk_cache, kDQ, a.N2, tokens, kDQ, static_cast<uint64_t>(a.N2) * kDQ, 1, 32) ||
+      !make_tmap_3d_bf16(&tdkrc, a.dk_rope_cache, kDR, a.N2, tokens, kDR, static_cast<uint64_t>(a.N2) * kDR, 1, 32) ||
+      !make_tmap_3d_bf16(&tdvc, a.dv_cache, kDQ, a.N2, tokens, kDQ, static_cast<uint64_t>(a.N2) * kDQ, 1, 32))
     return cudaErrorInvalidValue;
   BwdParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.G = G; p.Gp = (G + 15) / 16 * 16; p.K = a.meta.K; p.ppb = a.meta.ppb;
   p.page_size = a.page_size; p.cap = cap; p.sub_rows = sub; p.T = T;
   p.scale = a.scale; p.scale_log2 = a.scale * kLog2e;
   p.pages = a.meta.pages; p.tokens = a.meta.tokens; p.count = a.meta.count;
-  p.lse2 = a.lse2; p.dvec = a.dvec; p.rows_u = cap * a.page_size; p.status = a.meta.status;
+  p.lse2 = a.lse2; p.dvec = a.dvec; p.rows_u = cap * a.page_size; p.status = a.meta.status; p.refs = a.cnt;
   const size_t smem = sizeof(BwdSmem) + 1024;
   if ((e = cudaFuncSetAttribute(sfa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
     return e;
   if (T > 0 && U > 0) {
     prof_begin("sfa_bwd", st);
-    e = launch_pdl(sfa_bwd_kernel, dim3(T, U), dim3(kThreads), smem, st, tq, tqr, tdo, tk, tkr, tv, tgk, tgv, tdqp, p);
+    e = launch_pdl(sfa_bwd_kernel, dim3(T, U), dim3(kThreads), smem, st, tq, tqr, tdo, tk, tkr, tv, tgk, tgv, tds,
+                   tdkc, tdkrc, tdvc, p);
     prof_end(st);
     if (e != cudaSuccess) return e;
   }
-  // dQ, then the cache rows
-  prof_begin("sfa_bwd_dq", st);
-  e = launch_pdl(sfa_bwd_dq_kernel, dim3(G, U), dim3(160), 0, st, static_cast<const float*>(a.dqp),
-                 static_cast<const int32_t*>(a.meta.count), a.N1, a.N2, G, T, spp, n_sub, a.scale,
-                 static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dq_rope));
-  prof_end(st);
-  if (e != cudaSuccess) return e;
+  // dQ (9 chunks of 64 dims per unit), then the rows of pages with several readers
+  const size_t dq_smem = sizeof(DqSmem) + 1024;
+  if ((e = cudaFuncSetAttribute(sfa_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem)) !=
+      cudaSuccess)
+    return e;
+  if (U > 0) {
+    prof_begin("sfa_bwd_dq", st);
+    e = launch_pdl(sfa_bwd_dq_kernel, dim3(kDK / 64, U), dim3(kDqThreads), dq_smem, st, tds, tk, tkr, p,
+                   static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dq_rope));
+    prof_end(st);
+    if (e != cudaSuccess) return e;
+  }
   if (ne > 0) {
     prof_begin("sfa_bwd_scatter", st);
     e = launch_pdl(sfa_scatter_kernel, dim3(ne), dim3(256), 0, st, static_cast<const int32_t*>(a.meta.pages),
