@@ -152,19 +152,22 @@ BSA_API bsa_status bsa_bwd(const bsa_params* p, const void* q, const void* k, co
                    const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
                    size_t workspace_bytes, void* stream);
 
-/* ---- NSA selected attention (NsaSelectedAttention page), TND, GQA, D = Dv = 128 -----------
+/* ---- NSA selected attention (NsaSelectedAttention page), TND, GQA, D = 128 or 192, Dv = 128 -
  * Forward formula of the page: for token t and kv head g, selected_key/value = Gather(key/value,
  * topk_indices[t, g, i]) for the listed blocks; Out = softmax(Mask(scale q K_sel^T)) V_sel for
  * each of the group's G = N1/N2 query heads (heads g*G .. g*G+G-1); LSE per (t, head).
- *   p->q_layout = p->kv_layout = BSA_LAYOUT_TND; q/out/dout/dq [T, N1, 128], k/v/dk/dv
- *   [T, N2, 128], lse [T, N1]; T_q = T_kv = T; cu_seqlens_q (= cu_seqlens_kv) [B+1] device int32
+ *   p->q_layout = p->kv_layout = BSA_LAYOUT_TND; q/dq [T, N1, D], out/dout [T, N1, 128], k/dk
+ *   [T, N2, D], v/dv [T, N2, 128], lse [T, N1]; (D, Dv) = (128, 128), or (192, 128) (the page's
+ *   head-dim pair for query and key vs value) with G = N1 / N2 <= 16.
+ *   T_q = T_kv = T; cu_seqlens_q (= cu_seqlens_kv) [B+1] device int32
  *   with per-batch lengths (query and key lengths equal); S_q = the longest batch's length.
  *   topk_indices [T, N2, sel_block_count] int32: block ids of sel_block_size tokens, counted
  *   from the batch's first token; -1 = empty slot; a duplicated id is gathered twice.
  *   mask_mode BSA_MASK_NONE or BSA_MASK_CAUSAL (key position <= query position in the batch).
  *   Host errors (INVALID_ARG / UNSUPPORTED): sel_block_size not a multiple of 16 in [16, 128],
  *   sel_block_count not in [1, 128] or count * size > 8192, N1 % N2 != 0, N2 > 32, N1 > 128,
- *   D != 128, S_q > 128K, T_q != T_kv, scale <= 0.
+ *   (D, Dv) other than (128, 128) or (192, 128), D = 192 with G > 16, S_q > 128K, T_q != T_kv,
+ *   scale <= 0.
  *   Device status bits: SA_DEV_BAD_INDEX for an id at or past the batch's block count (the id
  *   is skipped); SA_DEV_BAD_SEQLEN if cu_seqlens is not a non-decreasing 0..T sequence or a
  *   batch is longer than S_q (nothing is computed).

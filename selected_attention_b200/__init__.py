@@ -295,8 +295,9 @@ def plan_array(plan, layout: MetaLayout, index: int, count: int, dtype=torch.int
 # NSA selected attention (TND)
 # ---------------------------------------------------------------------------------------------
 def nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode=MASK_CAUSAL,
-               scale=None) -> Params:
-    """q [T, N1, 128], k [T, N2, 128], topk_indices [T, N2, K] int32, cu_seqlens [B+1] int32 (device)."""
+               scale=None, dv=None) -> Params:
+    """q [T, N1, D], k [T, N2, D] (D = 128, or 192 with v's 128: dv), topk_indices [T, N2, K] int32,
+    cu_seqlens [B+1] int32 (device)."""
     T, N1, D = q.shape
     _, N2, _ = k.shape
     p = Params()
@@ -304,7 +305,8 @@ def nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_
     p.B, p.N1, p.N2 = cu_seqlens.shape[0] - 1, N1, N2
     p.S_q = p.S_kv = int(max_seqlen)
     p.T_q = p.T_kv = T
-    p.D = p.Dv = D
+    p.D = D
+    p.Dv = D if dv is None else dv
     p.cu_seqlens_q = p.cu_seqlens_kv = cu_seqlens.data_ptr()
     p.sel_block_size, p.sel_block_count = sel_block_size, topk_indices.shape[-1]
     p.topk_indices = topk_indices.data_ptr()
@@ -327,12 +329,13 @@ def nsa_selected_bwd_workspace_size(p: Params) -> int:
 
 def nsa_selected_fwd(q, k, v, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode=MASK_CAUSAL,
                      scale=None, out=None, lse=None, workspace=None, stream=None, plan=None):
-    """Out [T, N1, 128] bf16, LSE [T, N1] fp32 of NSA selected attention.  plan: optional
-    (tensor, META_NSA_KV or META_NSA_TOKENS) from sparse_attn_metadata for this problem."""
+    """Out [T, N1, Dv] bf16, LSE [T, N1] fp32 of NSA selected attention (q, k [.., D], v [.., Dv]).
+    plan: optional (tensor, META_NSA_KV or META_NSA_TOKENS) from sparse_attn_metadata for this
+    problem."""
     _need_cuda(q, k, v, topk_indices, cu_seqlens)
-    p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale)
+    p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale, v.shape[-1])
     _set_plan(p, plan)
-    out = torch.empty_like(q) if out is None else out
+    out = torch.empty(q.shape[0], q.shape[1], v.shape[-1], dtype=torch.bfloat16, device=q.device) if out is None else out
     lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if lse is None else lse
     if workspace is None:
         workspace = _workspace(nsa_selected_fwd_workspace_size(p), q.device)
@@ -347,7 +350,7 @@ def nsa_selected_bwd(q, k, v, out, dout, lse, topk_indices, cu_seqlens, max_seql
     """dQ, dK, dV of NSA selected attention.  plan: optional (tensor, META_NSA_TOKENS) from
     sparse_attn_metadata for this problem."""
     _need_cuda(q, k, v, out, dout, lse, topk_indices, cu_seqlens)
-    p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale)
+    p = nsa_params(q, k, topk_indices, cu_seqlens, max_seqlen, sel_block_size, mask_mode, scale, v.shape[-1])
     _set_plan(p, plan)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk

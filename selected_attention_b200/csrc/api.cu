@@ -149,7 +149,9 @@ bsa_status check_nsa(const bsa_params* p) {
   if (p->q_layout != BSA_LAYOUT_TND || p->kv_layout != BSA_LAYOUT_TND) return BSA_ERR_UNSUPPORTED;
   if (p->B < 1 || p->B > 1024 || p->N1 < 1 || p->N1 > 128 || p->N2 < 1 || p->N2 > 32) return BSA_ERR_INVALID_ARG;
   if (p->N1 < p->N2 || p->N1 % p->N2 != 0) return BSA_ERR_INVALID_ARG;
-  if (p->D != 128 || p->Dv != 128) return BSA_ERR_UNSUPPORTED;
+  // head dims: 128 / 128, or 192 for q / k with 128 for v (query groups of at most 16 heads)
+  if (p->Dv != 128 || (p->D != 128 && p->D != 192)) return BSA_ERR_UNSUPPORTED;
+  if (p->D == 192 && p->N1 / p->N2 > 16) return BSA_ERR_UNSUPPORTED;
   if (p->T_q <= 0 || p->T_q != p->T_kv) return BSA_ERR_INVALID_ARG;
   if (p->S_q <= 0 || p->S_q > 128 * 1024 || p->S_q > p->T_q) return BSA_ERR_INVALID_ARG;
   if (p->sel_block_size <= 0 || p->sel_block_size > 128 || p->sel_block_size % 16 != 0) return BSA_ERR_INVALID_ARG;
@@ -235,6 +237,7 @@ NsaMetaArgs nsa_meta_args(const bsa_params* p, const NsaWs& w, bool token_lists)
 NsaArgs nsa_args(const bsa_params* p, const NsaWs& w) {
   NsaArgs a;
   a.B = p->B; a.T = p->T_q; a.N1 = p->N1; a.N2 = p->N2; a.K = p->sel_block_count; a.sel_block = p->sel_block_size;
+  a.D = p->D;
   a.nblk_max = w.nblk_max; a.mask_mode = p->mask_mode; a.scale = p->scale;
   a.cu_seqlens = p->cu_seqlens_q; a.ok_flag = w.ok_flag; a.ids = w.ids; a.cnt = w.cnt; a.dup = w.dup;
   a.t_row_ptr = w.t_row_ptr; a.t_col = w.t_col;

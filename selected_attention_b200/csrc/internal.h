@@ -197,6 +197,7 @@ struct NsaMetaArgs {
 cudaError_t nsa_metadata(const NsaMetaArgs& a, cudaStream_t st);
 struct NsaArgs {
   int B, T, N1, N2, K, sel_block, nblk_max, mask_mode;
+  int D;  // head dim of q and k: 128, or 192 (with G <= 16); v, Out and dOut have 128
   float scale;
   const int32_t *cu_seqlens, *ok_flag, *ids, *cnt, *dup, *t_row_ptr, *t_col;
   const void *q, *k, *v, *out_in, *dout;

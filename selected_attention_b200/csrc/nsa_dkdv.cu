@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool nsa_dkdv_tc_supported(const NsaArgs& a) {
   const int G = a.N1 / a.N2;
-  return a.sel_block == kKeys && G >= 8 && G <= 128 && 128 % G == 0;
+  return a.D == kD && a.sel_block == kKeys && G >= 8 && G <= 128 && 128 % G == 0;
 }
 
 cudaError_t nsa_dkdv_tc_launch(const NsaArgs& a, cudaStream_t st) {

@@ -32,7 +32,7 @@ namespace sa {
 namespace {
 
 constexpr int kTok = 128;     // keys per tile: MMA M
-constexpr int kD = 128;       // head dim of q / k / v
+constexpr int kDV = 128;      // head dim of v, Out and dOut (q and k: DQK, 128 or 192)
 // Keys per gather chunk (one TMA box per head-dim half): 64 when the selected block size is a
 // multiple of 64 (a block's visible prefix then ends inside its last chunk and is masked there),
 // else 16.  A 128-key tile holds kTok / chunk chunks.
@@ -51,12 +51,14 @@ constexpr float kLazy = 8.f;  // log2 units a tile may exceed the running maximu
 
 // Ring depths: an operand held until the last product of its tile (V in the forward, K in the dQ
 // pass) gets the deeper ring, the one released by the first product the shallower.
-// A 32-head tile's Q, dO and P buffers take one stage of the deeper ring (227 KB per CTA).
-template <bool kDq, int NH>
+// A 32-head tile's Q, dO and P buffers take one stage of the deeper ring (227 KB per CTA); with
+// 192-dim q / k (16-head tiles only) a K stage is 48 KB and the rings are two or three deep.
+template <bool kDq, int NH, int DQK>
 struct TcCfg {
+  static constexpr int kQC = DQK / 64;  // 64-wide chunks of q / k
   static constexpr int kDeep = !kDq ? (NH == 16 ? 4 : 3) : (NH == 16 ? 3 : 2);
-  static constexpr int kKR = kDq ? kDeep : 2;  // K ring (read by S^T, and by dQ^T in the dQ pass)
-  static constexpr int kVR = kDq ? 2 : kDeep;  // V ring (read by O^T in the forward, by dP^T in the dQ pass)
+  static constexpr int kKR = DQK == 128 ? (kDq ? kDeep : 2) : 2;  // K ring (S^T, and dQ^T in the dQ pass)
+  static constexpr int kVR = DQK == 128 ? (kDq ? 2 : kDeep) : (kDq ? 2 : 3);  // V ring (O^T, or dP^T)
 };
 
 struct ItemDesc {
@@ -66,12 +68,13 @@ struct ItemDesc {
   int32_t kp0[kMaxChunks];  // first key (within the batch) of each visible chunk
 };
 
-template <bool kDq, int NH>
+template <bool kDq, int NH, int DQK>
 struct __align__(1024) TcSmem {
+  using Cfg = TcCfg<kDq, NH, DQK>;
   // operand buffers start on 1024-byte boundaries (the 128-byte swizzle's pattern)
-  alignas(1024) uint8_t k[TcCfg<kDq, NH>::kKR][2][kTileBytes];
-  alignas(1024) uint8_t v[TcCfg<kDq, NH>::kVR][2][kTileBytes];
-  alignas(1024) uint8_t q[2][2][NH * 128];   // [item slot][head-dim half][NH rows][64 dims]
+  alignas(1024) uint8_t k[Cfg::kKR][Cfg::kQC][kTileBytes];
+  alignas(1024) uint8_t v[Cfg::kVR][2][kTileBytes];
+  alignas(1024) uint8_t q[2][Cfg::kQC][NH * 128];   // [item slot][64-dim chunk][NH rows][64 dims]
   // P^T (dS^T hi, lo) per tile parity: [tile & 1][part][key half][NH rows][64 keys]
   alignas(1024) uint8_t p[2][kDq ? 2 : 1][2][NH * 128];
   alignas(1024) uint8_t dout[kDq ? 2 : 1][2][kDq ? NH * 128 : 16];  // dQ pass only
@@ -80,8 +83,8 @@ struct __align__(1024) TcSmem {
   float red_l[4][NH];
   uint64_t bar_desc_full[2], bar_desc_empty[2];
   uint64_t bar_q[2], bar_q_empty[2];
-  uint64_t bar_k[TcCfg<kDq, NH>::kKR], bar_k_empty[TcCfg<kDq, NH>::kKR];
-  uint64_t bar_v[TcCfg<kDq, NH>::kVR], bar_v_empty[TcCfg<kDq, NH>::kVR];
+  uint64_t bar_k[Cfg::kKR], bar_k_empty[Cfg::kKR];
+  uint64_t bar_v[Cfg::kVR], bar_v_empty[Cfg::kVR];
   uint64_t bar_s_full[2], bar_s_free[2];     // score buffers (S^T, and dP^T in the dQ pass)
   uint64_t bar_p_full[2], bar_pv_done[2];    // the P^T (dS^T) buffers: written / consumed, per tile parity
   uint64_t bar_x;                            // softmax warps exchange tile maxima, then sums
@@ -155,22 +158,24 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <bool kDq, int NH>
+template <bool kDq, int NH, int DQK>
 __global__ void __launch_bounds__(kThreads, 1)
     nsa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const TcParams prm) {
-  using Cfg = TcCfg<kDq, NH>;
-  constexpr int kKR = Cfg::kKR, kVR = Cfg::kVR;
+  using Cfg = TcCfg<kDq, NH, DQK>;
+  constexpr int kKR = Cfg::kKR, kVR = Cfg::kVR, kQC = Cfg::kQC;
+  // 192-dim dQ: a second accumulator over dims 64..191 (its rows 64..127 are dims 128..191)
+  constexpr bool kTwoAcc = kDq && DQK == 192;
   // TMEM columns: score buffers at [0, NH) and [NH, 2NH); dP^T buffers after them (dQ pass); the
-  // O^T / dQ^T accumulator last
+  // O^T / dQ^T accumulator(s) last
   constexpr uint32_t kColS = 0, kColDP = 2 * NH, kColAcc = kDq ? 4 * NH : 2 * NH;
-  constexpr uint32_t kTmemCols = kDq ? (5 * NH <= 128 ? 128 : 256) : 128;
+  constexpr uint32_t kTmemCols = kDq ? ((kTwoAcc ? 6 : 5) * NH <= 128 ? 128 : 256) : 128;
   griddep_launch_dependents();
   griddep_wait();  // launched early: the metadata (and the preprocess) must be complete
   extern __shared__ uint8_t smem_raw[];
-  TcSmem<kDq, NH>& s =
-      *reinterpret_cast<TcSmem<kDq, NH>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  TcSmem<kDq, NH, DQK>& s =
+      *reinterpret_cast<TcSmem<kDq, NH, DQK>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool run = *prm.ok_flag != 0;  // cu_seqlens valid (uniform)
   // this CTA's items: blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -269,10 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         if (k >= 2) ok = mbar_wait(&s.bar_q_empty[slot], ((k >> 1) - 1) & 1, prm.status);
         if (ok) {
-          mbar_arrive_expect_tx(&s.bar_q[slot], (kDq ? 4 : 2) * NH * 128);
+          mbar_arrive_expect_tx(&s.bar_q[slot], (kQC + (kDq ? 2 : 0)) * NH * 128);
           const int qrow = t * prm.N1 + h0;
-          tma_load_2d(s.q[slot][0], &tm_q, &s.bar_q[slot], 0, qrow);
-          tma_load_2d(s.q[slot][1], &tm_q, &s.bar_q[slot], 64, qrow);
+#pragma unroll
+          for (int c = 0; c < kQC; ++c) tma_load_2d(s.q[slot][c], &tm_q, &s.bar_q[slot], c * 64, qrow);
           if (kDq) {
             tma_load_2d(s.dout[kDq ? slot : 0][0], &tm_do, &s.bar_q[slot], 0, qrow);
             tma_load_2d(s.dout[kDq ? slot : 0][1], &tm_do, &s.bar_q[slot], 64, qrow);
@@ -311,12 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         uint8_t* dst = is_k ? s.k[st % kRK][0] : s.v[st % kRV][0];
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
+        const int nc = is_k ? kQC : 2;  // 64-wide chunks of a key row
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], nc * kTileBytes);
         __syncwarp();
-        if (lane < cpt) {
-          tma_load_3d(dst + lane * prm.chunk * 128, map, &full[st], 0, g, tok);
-          tma_load_3d(dst + kTileBytes + lane * prm.chunk * 128, map, &full[st], 64, g, tok);
-        }
+        if (lane < cpt)
+          for (int c = 0; c < nc; ++c)
+            tma_load_3d(dst + c * kTileBytes + lane * prm.chunk * 128, map, &full[st], c * 64, g, tok);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.bar_desc_empty[slot]);  // this warp is done with the item's list
@@ -342,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_tiles = (n_vis + (kTok >> prm.chunk_shift) - 1) / (kTok >> prm.chunk_shift);
         // every item's Q slot is loaded (and released below), with or without tiles
         if (!(ok = mbar_wait(&s.bar_q[slot], (k >> 1) & 1, prm.status))) break;
-        const uint64_t dq = dq0 + static_cast<uint64_t>(slot) * ((2 * NH * 128) >> 4);
+        const uint64_t dq = dq0 + static_cast<uint64_t>(slot) * ((kQC * NH * 128) >> 4);
         const uint64_t ddo = ddo0 + static_cast<uint64_t>(kDq ? slot : 0) * ((2 * NH * 128) >> 4);
         for (int j = 0; ok && j < n_tiles; ++j, ++J) {
           const int st = static_cast<int>(J & 1);
@@ -351,9 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ks_ = static_cast<int>(J % kKR);
           if (!(ok = mbar_wait(&s.bar_k[ks_], (J / kKR) & 1, prm.status))) break;
           tc_fence_after();
-          const uint64_t dk = dk0 + static_cast<uint64_t>(ks_) * ((2 * kTileBytes) >> 4);
+          const uint64_t dk = dk0 + static_cast<uint64_t>(ks_) * ((kQC * kTileBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk)
+          for (int kk = 0; kk < DQK / 16; ++kk)
             mma_bf16_ss(tmem + kColS + st * NH, sdesc_add(dk, (kk >> 2) * kTileBytes + (kk & 3) * 32),
                         sdesc_add(dq, (kk >> 2) * (NH * 128) + (kk & 3) * 32), id_s, kk > 0 ? 1u : 0u);
           if (!kDq) tc_commit(&s.bar_k_empty[ks_]);  // forward: K is read by S^T only
@@ -363,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint64_t dv = dv0 + static_cast<uint64_t>(vs) * ((2 * kTileBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk)
+            for (int kk = 0; kk < kDV / 16; ++kk)
               mma_bf16_ss(tmem + kColDP + st * NH, sdesc_add(dv, (kk >> 2) * kTileBytes + (kk & 3) * 32),
                           sdesc_add(ddo, (kk >> 2) * (NH * 128) + (kk & 3) * 32), id_s, kk > 0 ? 1u : 0u);
             tc_commit(&s.bar_v_empty[vs]);  // dQ pass: V is read by dP^T only
@@ -402,15 +407,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int as = static_cast<int>(J % kAR);
           if (!kDq && !(ok = mbar_wait(&s.bar_v[as], (J / kAR) & 1, prm.status))) break;
           tc_fence_after();
-          const uint64_t da = da0 + static_cast<uint64_t>(as) * ((2 * kTileBytes) >> 4);
+          const uint64_t da = da0 + static_cast<uint64_t>(as) * (((kDq ? kQC : 2) * kTileBytes) >> 4);
 #pragma unroll
-          for (int part = 0; part < (kDq ? 2 : 1); ++part) {  // dQ pass: dS^T hi, then lo
-            const uint64_t dp = dp0 + static_cast<uint64_t>(st) * kPBuf16 + static_cast<uint64_t>(part) * ((2 * NH * 128) >> 4);
+          for (int acc_i = 0; acc_i < (kTwoAcc ? 2 : 1); ++acc_i) {  // 192-dim dQ: dims 0..127, 64..191
+            const uint64_t da_i = da + static_cast<uint64_t>(acc_i) * (kTileBytes >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kTok / 16; ++kk)
-              mma_bf16_ss(tmem + kColAcc, sdesc_add(da, kk * 2048),
-                          sdesc_add(dp, (kk >> 2) * (NH * 128) + (kk & 3) * 32), id_o,
-                          (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            for (int part = 0; part < (kDq ? 2 : 1); ++part) {  // dQ pass: dS^T hi, then lo
+              const uint64_t dp = dp0 + static_cast<uint64_t>(st) * kPBuf16 + static_cast<uint64_t>(part) * ((2 * NH * 128) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kTok / 16; ++kk)
+                mma_bf16_ss(tmem + kColAcc + acc_i * NH, sdesc_add(da_i, kk * 2048),
+                            sdesc_add(dp, (kk >> 2) * (NH * 128) + (kk & 3) * 32), id_o,
+                            (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc_commit(kDq ? &s.bar_k_empty[as] : &s.bar_v_empty[as]);
           tc_commit(&s.bar_pv_done[st]);
@@ -561,32 +570,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < HW; ++h)
           L[h] = (s.red_l[0][hb + h] + s.red_l[1][hb + h]) + (s.red_l[2][hb + h] + s.red_l[3][hb + h]);
       }
-      uint32_t acc[HW];
+      uint32_t acc[HW], acc2[HW];
+      const bool hi_rows = kTwoAcc && quarter >= 2;  // this warp's rows 64..127 also hold dims 128..191
       if (n_tiles > 0) {
         const long long jl = J - 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[jl & 1], (jl >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
         tmem_ld_row<HW>(tmem + lane_base + kColAcc + hb, acc);
+        if (hi_rows) tmem_ld_row<HW>(tmem + lane_base + kColAcc + NH + hb, acc2);
         tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < HW; ++h) reg_fence(acc[h]);
+        for (int h = 0; h < HW; ++h) {
+          reg_fence(acc[h]);
+          if (hi_rows) reg_fence(acc2[h]);
+        }
         tc_fence_before();
         mbar_arrive(&s.bar_acc_free);
       } else {
 #pragma unroll
-        for (int h = 0; h < HW; ++h) acc[h] = 0u;
+        for (int h = 0; h < HW; ++h) acc[h] = acc2[h] = 0u;
       }
       // the descriptor slot is no longer needed
       mbar_arrive(&s.bar_desc_empty[slot]);
-      __nv_bfloat16* base = prm.out + static_cast<size_t>(t) * prm.N1 * kD;
+      constexpr int kDO = kDq ? DQK : kDV;  // row length of the output (dQ or Out)
+      __nv_bfloat16* base = prm.out + static_cast<size_t>(t) * prm.N1 * kDO;
 #pragma unroll
       for (int h = 0; h < HW; ++h) {
         if (hb + h >= rows) break;
         float mul;
         if (kDq) mul = prm.scale;
         else mul = L[h] > 0.f ? 1.f / L[h] : 0.f;
-        base[static_cast<size_t>(h0 + hb + h) * kD + r] = __float2bfloat16_rn(__uint_as_float(acc[h]) * mul);
+        base[static_cast<size_t>(h0 + hb + h) * kDO + r] = __float2bfloat16_rn(__uint_as_float(acc[h]) * mul);
+        if (hi_rows)
+          base[static_cast<size_t>(h0 + hb + h) * kDO + 64 + r] = __float2bfloat16_rn(__uint_as_float(acc2[h]) * mul);
       }
       if (!kDq && quarter == 0 && lane < HW && hb + lane < rows) {
         float mh = m[0], lh = L[0];
@@ -605,19 +622,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <bool kDq, int NH>
+template <bool kDq, int NH, int DQK>
 cudaError_t launch_tc(const NsaArgs& a, const TcParams& p, const char* name, cudaStream_t st) {
   CUtensorMap tq, tdo, tk, tv;
   const uint64_t qrows = static_cast<uint64_t>(a.T) * a.N1;
-  const uint64_t hs = static_cast<uint64_t>(a.N2) * kD;
-  if (!make_tmap_2d_bf16(&tq, a.q, qrows, kD, kD, NH) ||
-      !make_tmap_2d_bf16(&tdo, kDq ? a.dout : a.q, qrows, kD, kD, NH) ||
-      !make_tmap_3d_bf16(&tk, a.k, kD, a.N2, a.T, kD, hs, 1, p.chunk) ||
-      !make_tmap_3d_bf16(&tv, a.v, kD, a.N2, a.T, kD, hs, 1, p.chunk))
+  if (!make_tmap_2d_bf16(&tq, a.q, qrows, DQK, DQK, NH) ||
+      (kDq && !make_tmap_2d_bf16(&tdo, a.dout, qrows, kDV, kDV, NH)) || (!kDq && !make_tmap_2d_bf16(&tdo, a.q, qrows, DQK, DQK, NH)) ||
+      !make_tmap_3d_bf16(&tk, a.k, DQK, a.N2, a.T, DQK, static_cast<uint64_t>(a.N2) * DQK, 1, p.chunk) ||
+      !make_tmap_3d_bf16(&tv, a.v, kDV, a.N2, a.T, kDV, static_cast<uint64_t>(a.N2) * kDV, 1, p.chunk))
     return cudaErrorInvalidValue;
-  static_assert(sizeof(TcSmem<kDq, NH>) + 1024 <= 227 * 1024, "shared memory of one CTA (227 KB on sm_100)");
-  const size_t smem = sizeof(TcSmem<kDq, NH>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(nsa_tc_kernel<kDq, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static_assert(sizeof(TcSmem<kDq, NH, DQK>) + 1024 <= 227 * 1024, "shared memory of one CTA (227 KB on sm_100)");
+  const size_t smem = sizeof(TcSmem<kDq, NH, DQK>) + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(nsa_tc_kernel<kDq, NH, DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -625,7 +642,7 @@ cudaError_t launch_tc(const NsaArgs& a, const TcParams& p, const char* name, cud
   const int grid = static_cast<int>(p.items < sms ? p.items : sms);
   if (grid == 0) return cudaSuccess;
   prof_begin(name, st);
-  e = launch_pdl(nsa_tc_kernel<kDq, NH>, dim3(grid), dim3(kThreads), smem, st, tq, tdo, tk, tv, p);
+  e = launch_pdl(nsa_tc_kernel<kDq, NH, DQK>, dim3(grid), dim3(kThreads), smem, st, tq, tdo, tk, tv, p);
   prof_end(st);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -650,8 +667,9 @@ cudaError_t nsa_fwd_tc_launch(const NsaArgs& a, cudaStream_t st) {
   TcParams p = tc_params(a, G <= 16 ? 16 : 32);
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse_out = a.lse_out;
-  if (G <= 16) return launch_tc<false, 16>(a, p, "nsa_fwd", st);
-  return launch_tc<false, 32>(a, p, "nsa_fwd", st);
+  if (a.D == 192) return G <= 16 ? launch_tc<false, 16, 192>(a, p, "nsa_fwd", st) : cudaErrorNotSupported;
+  if (G <= 16) return launch_tc<false, 16, 128>(a, p, "nsa_fwd", st);
+  return launch_tc<false, 32, 128>(a, p, "nsa_fwd", st);
 }
 
 cudaError_t nsa_dq_tc_launch(const NsaArgs& a, cudaStream_t st) {
@@ -659,8 +677,9 @@ cudaError_t nsa_dq_tc_launch(const NsaArgs& a, cudaStream_t st) {
   TcParams p = tc_params(a, G <= 16 ? 16 : 32);
   p.out = static_cast<__nv_bfloat16*>(a.dq);
   p.lse_out = nullptr;
-  if (G <= 16) return launch_tc<true, 16>(a, p, "nsa_bwd_dq", st);
-  return launch_tc<true, 32>(a, p, "nsa_bwd_dq", st);
+  if (a.D == 192) return G <= 16 ? launch_tc<true, 16, 192>(a, p, "nsa_bwd_dq", st) : cudaErrorNotSupported;
+  if (G <= 16) return launch_tc<true, 16, 128>(a, p, "nsa_bwd_dq", st);
+  return launch_tc<true, 32, 128>(a, p, "nsa_bwd_dq", st);
 }
 
 }  // namespace sa

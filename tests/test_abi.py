@@ -239,3 +239,12 @@ def test_sfa_bwd_host_validation():
     assert _ws("sfa_sparse_decode_bwd_workspace_size", _sfa(plan=1 << 20, plan_op=sa.META_SFA_WORK))[0] \
         == sa.BSA_ERR_UNSUPPORTED
     assert sa.lib().sfa_sparse_decode_bwd(ctypes.byref(p), *([None] * 14), 0, None) == sa.BSA_ERR_NULLPTR
+
+
+def test_nsa_head_dim_pairs():
+    """q / k / v head dims 128 / 128, or 192 / 128 with query groups of at most 16 heads."""
+    fn = "nsa_selected_fwd_workspace_size"
+    assert _ws(fn, _nsa(D=192, Dv=128, N1=64, N2=4))[0] == sa.BSA_OK          # G = 16
+    assert _ws(fn, _nsa(D=192, Dv=128, N1=64, N2=2))[0] == sa.BSA_ERR_UNSUPPORTED  # G = 32
+    assert _ws(fn, _nsa(D=192, Dv=192))[0] == sa.BSA_ERR_UNSUPPORTED
+    assert _ws(fn, _nsa(D=64, Dv=128))[0] == sa.BSA_ERR_UNSUPPORTED

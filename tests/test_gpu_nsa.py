@@ -40,14 +40,16 @@ def _topk(rng, seqlens, N2, bs, K, causal, dup=False, past=False):
     return np.asarray(rows, np.int32).reshape(T, N2, K)
 
 
-def _problem(seqlens, N1, N2, bs, K, mode, seed, dup=False, past=False):
+def _problem(seqlens, N1, N2, bs, K, mode, seed, dup=False, past=False, dqk=D):
+    """dqk: head dim of q and k (v, Out and dOut keep D = 128)."""
     rng = np.random.default_rng(seed)
     T = sum(seqlens)
     bits = lambda *s: synth.f32_to_bf16_bits(rng.standard_normal(s, dtype=np.float32))  # noqa: E731
-    q, k, v, do = bits(T, N1, D), bits(T, N2, D), bits(T, N2, D), bits(T, N1, D)
+    q, k, v, do = bits(T, N1, dqk), bits(T, N2, dqk), bits(T, N2, D), bits(T, N1, D)
     topk = _topk(rng, seqlens, N2, bs, K, causal=(mode == 2), dup=dup, past=past)
     cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
-    return dict(q=q, k=k, v=v, do=do, topk=topk, cu=cu, S=max(seqlens), bs=bs, mode=mode, scale=1 / np.sqrt(D))
+    return dict(q=q, k=k, v=v, do=do, topk=topk, cu=cu, S=max(seqlens), bs=bs, mode=mode,
+                scale=1 / np.sqrt(dqk))
 
 
 def _dev(pb):
@@ -87,6 +89,9 @@ CASES = [
     dict(seqlens=[200], N1=64, N2=2, bs=64, K=3, mode=2),                    # G = 32
     dict(seqlens=[130, 70], N1=64, N2=1, bs=64, K=3, mode=0),                # G = 64
     dict(seqlens=[130, 70], N1=128, N2=1, bs=64, K=3, mode=2),               # G = 128
+    # 192-dim q / k with 128-dim v (NsaSelectedAttention constraints: a head-dim pair)
+    dict(seqlens=[200, 77], N1=16, N2=1, bs=64, K=4, mode=2, dqk=192),       # G = 16
+    dict(seqlens=[130, 256, 33], N1=16, N2=2, bs=32, K=6, mode=0, dup=True, dqk=192),  # G = 8, 32-token blocks
 ]
 
 
