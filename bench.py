@@ -327,7 +327,7 @@ def cpu_oracle_sample_nsa(w, topk, budget_s: float, chunk: int = 32):
             if w.mask_mode == 2:
                 hi = np.minimum(hi, pos + 1)
             vis = int(np.where(sub >= 0, np.clip(hi - sub.astype(np.int64) * w.sel_block, 0, None), 0).sum())
-            flops += 14 * w.D * vis * G
+            flops += (8 * w.D + 6 * w.dv) * vis * G
             done.append((b, g, len(toks)))
             if time.perf_counter() - t_start >= budget_s:
                 n = sum(x[2] for x in done)
@@ -527,8 +527,8 @@ def config_dict(w, args):
 def config_dict_nsa(w, args):
     return {
         "workload": f"{w.name}: NSA selected attention fwd+bwd, TND seqlens={w.seqlens} (T={w.T}), N1={w.N1} "
-                    f"N2={w.N2} D={w.D}, {w.sel_count} blocks of {w.sel_block} per (token, kv head), causal",
-        "T": w.T, "N1": w.N1, "N2": w.N2, "D": w.D, "sel_block": w.sel_block, "sel_count": w.sel_count,
+                    f"N2={w.N2} D={w.D} Dv={w.dv}, {w.sel_count} blocks of {w.sel_block} per (token, kv head), causal",
+        "T": w.T, "N1": w.N1, "N2": w.N2, "D": w.D, "Dv": w.dv, "sel_block": w.sel_block, "sel_count": w.sel_count,
         "seed": w.seed, "l2": "no flush: inputs (Q, dOut 1 GiB each) exceed the 126 MB L2",
         "parallelism": f"replicas x{args.gpus} (independent batches)",
     }
@@ -542,6 +542,8 @@ def nsa_workload(args):
     if args.nsa_seqlens:
         lens = [int(x) for x in args.nsa_seqlens.split(",")]
         w = dataclasses.replace(w, seqlens=lens, name=f"{w.name}_seqlens_{'_'.join(map(str, lens))}")
+    if getattr(args, "nsa_dqk", 128) != 128:  # q / k head dim 192 with v's 128 (the page's head-dim pair)
+        w = dataclasses.replace(w, D=args.nsa_dqk, Dv=w.D, name=f"{w.name}_dqk{args.nsa_dqk}")
     return w
 
 
@@ -584,15 +586,16 @@ def run_nsa(args, rank, world, local_rank):
     topk = w.topk()
     cu = w.cu_seqlens()
     vpairs = visible_pairs_nsa(w, topk)
-    flops_step = 14 * w.D * vpairs
+    # forward 2 (D + Dv) per visible pair (S, O); backward S, dQ, dK 2 D each and dP, dV 2 Dv each
+    flops_step = (8 * w.D + 6 * w.dv) * vpairs
     S = max(w.seqlens)
     host = {t: torch.from_numpy(w.tensor(t)).view(torch.bfloat16) for t in ("q", "k", "v", "dout")}
     host["topk"], host["cu"] = torch.from_numpy(topk), torch.from_numpy(cu)
     d = {t: x.to(dev) for t, x in host.items()}
-    out = torch.empty_like(d["q"])
+    out = torch.empty(w.T, w.N1, w.dv, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(w.T, w.N1, dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
-    p = sa.nsa_params(d["q"], d["k"], d["topk"], d["cu"], S, w.sel_block, w.mask_mode, w.scale)
+    p = sa.nsa_params(d["q"], d["k"], d["topk"], d["cu"], S, w.sel_block, w.mask_mode, w.scale, w.dv)
     ws_f = torch.empty(sa.nsa_selected_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(sa.nsa_selected_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -644,7 +647,11 @@ def run_nsa(args, rank, world, local_rank):
     peaks, peak_src = measured_peaks()
     # forward 4*D per visible pair; dK/dV pass 8*D (S^T, dP^T, dV, dK); dQ pass 2*D (dQ; its S and dP
     # recompute what the dK/dV pass is credited with)
-    alg = {"nsa_fwd": 4 * w.D * vpairs, "nsa_bwd_dkdv": 8 * w.D * vpairs, "nsa_bwd_dq": 2 * w.D * vpairs}
+    # forward S, O; dK/dV pass S^T, dP^T, dV, dK; dQ pass dQ (its S and dP are recomputations)
+    alg = {"nsa_fwd": 2 * (w.D + w.dv) * vpairs, "nsa_bwd_dkdv": (4 * w.D + 4 * w.dv) * vpairs,
+           "nsa_bwd_dq": 2 * w.D * vpairs}
+    if w.D != w.dv:  # 192-dim q / k: dK / dV run on the warp-level kernel
+        alg["nsa_bwd_dkdv_warp"] = alg["nsa_bwd_dkdv"]
     peak, peak_desc = tensor_peak(peaks, peak_src, ms * args.steps)
     dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
     roof = None
@@ -1112,6 +1119,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nsa-seqlens", default="", help="config 3 only: comma-separated batch lengths")
     ap.add_argument("--decode-bwd", action="store_true", help="config 4 only: time the decode's backward")
+    ap.add_argument("--nsa-dqk", type=int, default=128, choices=[128, 192],
+                    help="config 3 only: head dim of q / k (v keeps 128)")
     ap.add_argument("--decode-batches", type=int, default=0, help="--decode-bwd only: fewer batches (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:

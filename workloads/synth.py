@@ -226,10 +226,15 @@ class NsaWorkload:
     sel_block: int
     sel_count: int
     mask_mode: int = MASK_CAUSAL
+    Dv: int = 0  # head dim of v / Out / dOut; 0: the same as q / k (D)
 
     @property
     def scale(self) -> float:
         return 1.0 / float(np.sqrt(self.D))
+
+    @property
+    def dv(self) -> int:
+        return self.Dv or self.D
 
     @property
     def T(self) -> int:
@@ -248,9 +253,10 @@ class NsaWorkload:
     def tensor(self, tag: str, lo: int = 0, hi: int | None = None) -> np.ndarray:
         """bf16 bits of q/k/v/dout, TND, tokens [lo, hi)."""
         heads = self.N1 if tag in ("q", "dout") else self.N2
+        d = self.D if tag in ("q", "k") else self.dv
         hi = self.T if hi is None else hi
-        rows = normal_rows_bf16(self.seed, tag, self.T, heads * self.D, 64, lo, hi)
-        return rows.reshape(hi - lo, heads, self.D)
+        rows = normal_rows_bf16(self.seed, tag, self.T, heads * d, 64, lo, hi)
+        return rows.reshape(hi - lo, heads, d)
 
 
 @dataclass
