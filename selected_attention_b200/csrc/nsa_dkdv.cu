@@ -14,8 +14,13 @@
 //
 // Warps 0-7 compute P and dS (TMEM lane quarter = warp % 4, key half = warp / 4), warp 8 issues
 // the TMA loads, warp 9 issues the MMAs.  Every wait is bounded (SA_DEV_TIMEOUT).
+// With 192-dim q / k (v and dO keep 128) the Q rows of a step are three 64-dim chunks, Q / dO have
+// one stage instead of two (227 KB), and dK^T takes two M = 128 accumulators over dims 0-127 and
+// 64-191, the second's rows 64-127 giving dims 128-191.
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "internal.h"
 #include "sa_common.cuh"
@@ -25,20 +30,23 @@ namespace {
 
 constexpr int kRows = 128;  // (token, head) rows of a step
 constexpr int kKeys = 64;   // keys of a block
-constexpr int kD = 128;
+constexpr int kDV = 128;    // head dim of v / dO (q / k: DQK)
 constexpr int kEw = 8;      // element-wise warps
 constexpr int kThreads = (kEw + 2) * 32;
-constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 192;  // TMEM columns
+constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 192, kColDK2 = 256;  // TMEM columns
 constexpr float kLog2e = 1.4426950408889634f;
 
+template <int DQK>
 struct __align__(1024) DkdvSmem {
-  uint8_t k[2][kKeys * 128];          // K block: [64 keys][64 d] per head-dim half
+  static constexpr int kQC = DQK / 64;             // 64-dim chunks of q / k
+  static constexpr int kNst = DQK == 128 ? 2 : 1;  // Q / dO stages
+  uint8_t k[kQC][kKeys * 128];        // K block: [64 keys][64 d] per head-dim chunk
   uint8_t v[2][kKeys * 128];
-  uint8_t q[2][2][kRows * 128];       // [stage][half] [128 rows][64 d]
-  uint8_t dout[2][2][kRows * 128];
+  uint8_t q[kNst][kQC][kRows * 128];  // [stage][chunk] [128 rows][64 d]
+  uint8_t dout[kNst][2][kRows * 128];
   uint8_t p[2][kRows * 128];          // P hi, lo: [128 rows][64 keys]
   uint8_t ds[2][kRows * 128];         // dS hi, lo
-  uint64_t bar_kv, bar_qdo[2], bar_qdo_empty[2];
+  uint64_t bar_kv, bar_qdo[kNst], bar_qdo_empty[kNst];
   uint64_t bar_s_full, bar_p_ready, bar_p_free, bar_done;
   uint32_t tmem_base;
 };
@@ -69,12 +77,17 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+template <int DQK>
 __global__ void __launch_bounds__(kThreads, 1)
     nsa_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DkdvParams prm) {
+  using Sm = DkdvSmem<DQK>;
+  constexpr int kQC = Sm::kQC, kNst = Sm::kNst;
+  constexpr bool kTwoAcc = DQK == 192;
+  constexpr uint32_t kTmemCols = kTwoAcc ? 512 : 256;
   extern __shared__ uint8_t smem_raw[];
-  DkdvSmem& s = *reinterpret_cast<DkdvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // CTA order: batches from the last one (longest lists first in causal workloads), kv head,
   // then blocks ascending; CTAs that run together share the batch's Q / dO rows in L2
@@ -95,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&s.bar_kv, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNst; ++i) {
       mbar_init(&s.bar_qdo[i], 1);
       mbar_init(&s.bar_qdo_empty[i], 1);
     }
@@ -106,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&s.tmem_base, 256);
+    tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -119,27 +132,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Lane j < tps loads the token of slot j and issues that slot's four row copies, so the token
     // reads of a step are one round trip, not tps dependent ones.
     if (lane == 0) {
-      mbar_arrive_expect_tx(&s.bar_kv, 4 * kKeys * 128);
-      tma_load_3d(s.k[0], &tm_k, &s.bar_kv, 0, g, key_tok0);
-      tma_load_3d(s.k[1], &tm_k, &s.bar_kv, 64, g, key_tok0);
+      mbar_arrive_expect_tx(&s.bar_kv, (kQC + 2) * kKeys * 128);
+      for (int c = 0; c < kQC; ++c) tma_load_3d(s.k[c], &tm_k, &s.bar_kv, c * 64, g, key_tok0);
       tma_load_3d(s.v[0], &tm_v, &s.bar_kv, 0, g, key_tok0);
       tma_load_3d(s.v[1], &tm_v, &s.bar_kv, 64, g, key_tok0);
     }
     int issued = 0;
     for (int i = 0; i < steps; ++i) {
-      const int st = i & 1;
+      const int st = i % kNst;
       // slots past the list repeat its last token (finite data; their rows are masked)
       const int qrow = lane < tps ? prm.t_col[rp + min(i * tps + lane, n_tok - 1)] * prm.N1 + g * prm.G : 0;
       bool ok = true;
       if (lane == 0) {
-        if (i >= 2) ok = mbar_wait(&s.bar_qdo_empty[st], ((i - 2) >> 1) & 1, prm.status);
-        if (ok) mbar_arrive_expect_tx(&s.bar_qdo[st], 4 * kRows * 128);
+        if (i >= kNst) ok = mbar_wait(&s.bar_qdo_empty[st], ((i - kNst) / kNst) & 1, prm.status);
+        if (ok) mbar_arrive_expect_tx(&s.bar_qdo[st], (kQC + 2) * kRows * 128);
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // the expected bytes are set before any copy
       if (lane < tps) {
         const uint32_t off = static_cast<uint32_t>(lane * prm.G * 128);
-        tma_load_2d(s.q[st][0] + off, &tm_q, &s.bar_qdo[st], 0, qrow);
-        tma_load_2d(s.q[st][1] + off, &tm_q, &s.bar_qdo[st], 64, qrow);
+        for (int c = 0; c < kQC; ++c) tma_load_2d(s.q[st][c] + off, &tm_q, &s.bar_qdo[st], c * 64, qrow);
         tma_load_2d(s.dout[st][0] + off, &tm_do, &s.bar_qdo[st], 0, qrow);
         tma_load_2d(s.dout[st][1] + off, &tm_do, &s.bar_qdo[st], 64, qrow);
       }
@@ -147,15 +158,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // wait for this CTA's own copies still in flight before it may exit
     if (lane == 0) {
-      for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
-        mbar_wait(&s.bar_qdo[i & 1], (i >> 1) & 1, prm.status);
+      for (int i = (issued > kNst ? issued - kNst : 0); i < issued; ++i)
+        mbar_wait(&s.bar_qdo[i % kNst], (i / kNst) & 1, prm.status);
       mbar_wait(&s.bar_kv, 0, prm.status);
     }
   } else if (warp == kEw + 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(kRows, kKeys, false, false);  // S, dP
-      const uint32_t id_g = idesc_bf16_f32(kD, kKeys, true, true);       // dV^T, dK^T
+      const uint32_t id_g = idesc_bf16_f32(128, kKeys, true, true);      // dV^T, dK^T (M = 128 dims)
       // descriptors of stage 0 / sub-tile 0; stages, sub-tiles and K steps are added offsets
       const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0][0]), 0, 1024);
       const uint64_t ddo0 = sdesc_sw128(smem_u32(s.dout[0][0]), 0, 1024);
@@ -165,11 +176,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0][0]), kRows * 128, 1024);
       const uint64_t dph = sdesc_sw128(smem_u32(s.p[0]), kRows * 128, 1024), dpl = sdesc_add(dph, kRows * 128);
       const uint64_t dsh = sdesc_sw128(smem_u32(s.ds[0]), kRows * 128, 1024), dsl = sdesc_add(dsh, kRows * 128);
-      constexpr uint32_t kStage16 = (2 * kRows * 128) >> 4;  // one Q / dO stage, in 16-byte units
-      // [128 rows] x [64 keys] += A [128 rows][128 d] . B [64 keys][128 d]^T, both K-major
-      auto mma_s = [&](uint32_t d, uint64_t a, uint64_t b) {
+      constexpr uint32_t kStageQ16 = (kQC * kRows * 128) >> 4;  // one Q stage, in 16-byte units
+      constexpr uint32_t kStageD16 = (2 * kRows * 128) >> 4;    // one dO stage
+      // [128 rows] x [64 keys] += A [128 rows][KD] . B [64 keys][KD]^T, both K-major (KD = DQK for S,
+      // 128 for dP)
+      auto mma_s = [&](uint32_t d, uint64_t a, uint64_t b, auto kd) {
+        constexpr int KD = decltype(kd)::value;
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks)
+        for (int ks = 0; ks < KD / 16; ++ks)
           mma_bf16_ss(d, sdesc_add(a, (ks >> 2) * (kRows * 128) + (ks & 3) * 32),
                       sdesc_add(b, (ks >> 2) * (kKeys * 128) + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
       };
@@ -183,27 +197,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&s.bar_kv, 0, prm.status) && mbar_wait(&s.bar_qdo[0], 0, prm.status);
       if (ok) {
         tc_fence_after();
-        mma_s(tmem + kColS, dq0, dk);
-        mma_s(tmem + kColDP, ddo0, dv);
+        mma_s(tmem + kColS, dq0, dk, std::integral_constant<int, DQK>{});
+        mma_s(tmem + kColDP, ddo0, dv, std::integral_constant<int, kDV>{});
         tc_commit(&s.bar_s_full);
       }
       for (int i = 0; ok && i < steps; ++i) {
-        const int st = i & 1;
+        const int st = i % kNst;
         if (!(ok = mbar_wait(&s.bar_p_ready, i & 1, prm.status))) break;
         tc_fence_after();
-        const uint64_t ddom = ddom0 + static_cast<uint64_t>(st) * kStage16;
-        const uint64_t dqm = dqm0 + static_cast<uint64_t>(st) * kStage16;
+        const uint64_t ddom = ddom0 + static_cast<uint64_t>(st) * kStageD16;
+        const uint64_t dqm = dqm0 + static_cast<uint64_t>(st) * kStageQ16;
         mma_g(tmem + kColDV, ddom, dph, i > 0);   // dV^T += dO^T P_hi
         mma_g(tmem + kColDV, ddom, dpl, true);    // dV^T += dO^T P_lo
-        mma_g(tmem + kColDK, dqm, dsh, i > 0);    // dK^T += Q^T dS_hi
+        mma_g(tmem + kColDK, dqm, dsh, i > 0);    // dK^T += Q^T dS_hi  (dims 0..127)
         mma_g(tmem + kColDK, dqm, dsl, true);     // dK^T += Q^T dS_lo
+        if (kTwoAcc) {                             // dims 64..191: Q^T from chunks 1 and 2
+          const uint64_t dqm1 = sdesc_add(dqm, kRows * 128);
+          mma_g(tmem + kColDK2, dqm1, dsh, i > 0);
+          mma_g(tmem + kColDK2, dqm1, dsl, true);
+        }
         tc_commit(&s.bar_p_free);
         tc_commit(&s.bar_qdo_empty[st]);
         if (i + 1 < steps) {
-          if (!(ok = mbar_wait(&s.bar_qdo[st ^ 1], ((i + 1) >> 1) & 1, prm.status))) break;
+          const int sn = (i + 1) % kNst;
+          if (!(ok = mbar_wait(&s.bar_qdo[sn], ((i + 1) / kNst) & 1, prm.status))) break;
           tc_fence_after();
-          mma_s(tmem + kColS, dq0 + static_cast<uint64_t>(st ^ 1) * kStage16, dk);
-          mma_s(tmem + kColDP, ddo0 + static_cast<uint64_t>(st ^ 1) * kStage16, dv);
+          mma_s(tmem + kColS, dq0 + static_cast<uint64_t>(sn) * kStageQ16, dk, std::integral_constant<int, DQK>{});
+          mma_s(tmem + kColDP, ddo0 + static_cast<uint64_t>(sn) * kStageD16, dv, std::integral_constant<int, kDV>{});
           tc_commit(&s.bar_s_full);
         }
       }
@@ -293,22 +313,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         if (c0 + c >= nkeys) break;
-        const size_t o = (static_cast<size_t>(key_tok0 + c0 + c) * prm.N2 + g) * kD + r;
-        prm.dk[o] = __float2bfloat16_rn(__uint_as_float(rk[c]) * prm.scale);
-        prm.dv[o] = __float2bfloat16_rn(__uint_as_float(rv[c]));
+        const size_t krow = static_cast<size_t>(key_tok0 + c0 + c) * prm.N2 + g;
+        prm.dk[krow * DQK + r] = __float2bfloat16_rn(__uint_as_float(rk[c]) * prm.scale);
+        prm.dv[krow * kDV + r] = __float2bfloat16_rn(__uint_as_float(rv[c]));
+      }
+      if (kTwoAcc && quarter >= 2) {  // rows 64..127 of the second accumulator: dims 128..191
+        tmem_ld32(tmem + lane_base + kColDK2 + c0, rk);
+        tmem_ld_wait(rk);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (c0 + c >= nkeys) break;
+          const size_t krow = static_cast<size_t>(key_tok0 + c0 + c) * prm.N2 + g;
+          prm.dk[krow * DQK + 64 + r] = __float2bfloat16_rn(__uint_as_float(rk[c]) * prm.scale);
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
 
 bool nsa_dkdv_tc_supported(const NsaArgs& a) {
   const int G = a.N1 / a.N2;
-  return a.D == kD && a.sel_block == kKeys && G >= 8 && G <= 128 && 128 % G == 0;
+  return (a.D == 128 || a.D == 192) && a.sel_block == kKeys && G >= 8 && G <= 128 && 128 % G == 0;
 }
 
 cudaError_t nsa_dkdv_tc_launch(const NsaArgs& a, cudaStream_t st) {
@@ -318,9 +348,10 @@ cudaError_t nsa_dkdv_tc_launch(const NsaArgs& a, cudaStream_t st) {
   if (rows == 0 || a.T == 0) return cudaSuccess;
   CUtensorMap tq, tdo, tk, tv;
   const uint64_t qrows = static_cast<uint64_t>(a.T) * a.N1;
-  if (!make_tmap_2d_bf16(&tq, a.q, qrows, kD, kD, G) || !make_tmap_2d_bf16(&tdo, a.dout, qrows, kD, kD, G) ||
-      !make_tmap_3d_bf16(&tk, a.k, kD, a.N2, a.T, kD, static_cast<uint64_t>(a.N2) * kD, 1, kKeys) ||
-      !make_tmap_3d_bf16(&tv, a.v, kD, a.N2, a.T, kD, static_cast<uint64_t>(a.N2) * kD, 1, kKeys))
+  const int D = a.D;
+  if (!make_tmap_2d_bf16(&tq, a.q, qrows, D, D, G) || !make_tmap_2d_bf16(&tdo, a.dout, qrows, kDV, kDV, G) ||
+      !make_tmap_3d_bf16(&tk, a.k, D, a.N2, a.T, D, static_cast<uint64_t>(a.N2) * D, 1, kKeys) ||
+      !make_tmap_3d_bf16(&tv, a.v, kDV, a.N2, a.T, kDV, static_cast<uint64_t>(a.N2) * kDV, 1, kKeys))
     return cudaErrorInvalidValue;
   DkdvParams p;
   p.B = a.B; p.N1 = a.N1; p.N2 = a.N2; p.G = G; p.K = a.K; p.nblk_max = a.nblk_max; p.mask_mode = a.mask_mode;
@@ -331,11 +362,14 @@ cudaError_t nsa_dkdv_tc_launch(const NsaArgs& a, cudaStream_t st) {
   p.lse2 = a.lse2; p.dvec = a.dvec;
   p.dk = static_cast<__nv_bfloat16*>(a.dk); p.dv = static_cast<__nv_bfloat16*>(a.dv);
   p.status = a.status;
-  const size_t smem = sizeof(DkdvSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(nsa_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static_assert(sizeof(DkdvSmem<192>) + 1024 <= 227 * 1024, "shared memory of one CTA (227 KB on sm_100)");
+  static_assert(sizeof(DkdvSmem<128>) + 1024 <= 227 * 1024, "shared memory of one CTA (227 KB on sm_100)");
+  const size_t smem = (D == 192 ? sizeof(DkdvSmem<192>) : sizeof(DkdvSmem<128>)) + 1024;
+  auto kern = D == 192 ? nsa_dkdv_tc_kernel<192> : nsa_dkdv_tc_kernel<128>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   prof_begin("nsa_bwd_dkdv", st);
-  nsa_dkdv_tc_kernel<<<rows, kThreads, smem, st>>>(tq, tdo, tk, tv, p);
+  kern<<<rows, kThreads, smem, st>>>(tq, tdo, tk, tv, p);
   prof_end(st);
   return cudaGetLastError();
 }
