@@ -8,20 +8,25 @@
 // and the query side is only NH rows: the products are taken transposed, with 128 gathered keys as
 // the MMA's M and the heads as N (the form the paged decode uses):
 //   forward  S^T [128 keys][NH] = K~ . Q^T          O^T [128 dv][NH] += V~^T . P^T
-//   dQ pass  S^T = K~ . Q^T, dP^T = V~ . dO^T        dQ^T [128 d][NH] += K~^T . dS^T (bf16 hi + lo)
+//   dQ pass  S^T = K~ . Q^T, dP^T = V~ . dO^T        dQ^T [d][NH] += K~^T . dS^T (bf16 hi + lo)
 // P^T (dS^T) is written to shared memory as the B operand, K-major ([NH heads][128 keys]).
+// q / k have DQK = 128 or 192 dims (v, Out, dO 128): with 192 a K tile is three 64-dim chunks and
+// dQ^T takes two M = 128 accumulators, over dims 0-127 and 64-191 (the second's rows 64-127 are
+// dims 128-191).
 //
-// Gather: the visible 16-key chunks of the token's listed blocks (a block's chunks past the last
-// visible key, the query under the causal mask or the batch end, are skipped; a block listed twice
-// is gathered twice) are laid out in order by the producer warp into a per-item list in shared
-// memory; 8 chunks make a 128-key tile, loaded by TMA ({64 dims, 1 head, 16 tokens} boxes, 128-byte
-// swizzle) into K and V rings.  A tile's unused chunk slots repeat its first chunk and are masked.
+// Gather: the visible chunks (16 keys, or 64 when the block size is a multiple of 64) of the
+// token's listed blocks (a block's chunks past the last visible key, the query under the causal
+// mask or the batch end, are skipped; a block listed twice is gathered twice) are laid out in
+// order by the list warp into a per-item list in shared memory; a 128-key tile is loaded by TMA
+// ({64 dims, 1 head, chunk tokens} boxes, 128-byte swizzle) into K and V rings.  A tile's unused
+// chunk slots repeat its first chunk and are masked.
 //
 // Warps: 0-15 softmax (TMEM lane quarter = 32 keys, or 32 rows of the accumulator in the epilogue,
 // and a quarter of the tile's heads), 16 builds the item lists (up to two items ahead) and loads Q
 // (dO), 17 and 18 load the K and V tiles (each on its own ring, so K runs ahead of the V slots the
-// later products still hold), 19 issues S^T (and dP^T), 20 issues O^T (dQ^T).  Persistent CTAs take items round-robin.  Every wait is
-// bounded; on a timeout the kernel sets SA_DEV_TIMEOUT and stops.
+// later products still hold), 19 issues S^T (and dP^T), 20 issues O^T (dQ^T).  Persistent CTAs
+// take items round-robin.  Every wait is bounded; on a timeout the kernel sets SA_DEV_TIMEOUT and
+// stops.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
