@@ -220,12 +220,15 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 // walks each block's transposed list.  Every entry (a 128-row Q tile of one of the group's heads)
 // runs as two 64-row halves, so the element-wise work on one half overlaps the tensor-core work of
 // the neighbouring halves:
-//   TMEM columns: scores S^T [0,64) | dP^T [64,128) of one half (128 keys x 64 query rows); the
-//   fp16 A operands of the products P^T [128,160) and dS^T [192,224) (64 query rows -> 32 packed
-//   columns); dV [256,384), dK [384,512).
-//   The score buffer is released as soon as the 8 element-wise warps have loaded it into
-//   registers, so S^T / dP^T of half x + 1 run on the tensor cores while the warps turn half x into
-//   P and dS; those go to the operand buffer once the products of half x - 1 have read it.
+//   TMEM columns: two score buffers, b = half % 2, each S^T [128b, 128b+64) | dP^T [128b+64,
+//   128b+128) of one half (128 keys x 64 query rows); dV [256,384), dK [384,512).  The fp16 A
+//   operands of the products are written in place: each element-wise thread, which loaded the
+//   32 query columns [32h, 32h+32) of S^T and of dP^T, writes its 16 packed columns of P^T over
+//   [128b+32h, +16) and of dS^T over [128b+64+32h, +16), so no thread overwrites columns another
+//   thread still has to load.  The products of half x read buffer x % 2 and release it for the
+//   scores of half x + 2, so those of half x + 1 are already in the other buffer when the warps
+//   finish half x: the chain "warps load half x, then the scores of x + 1 start" of a single
+//   score buffer is gone, and the score MMAs of x + 1 overlap the warps' work on x.
 //   Shared memory: the block's K and V tiles, and a 4-stage ring of half entries (64 rows of Q
 //   and dO with their D and LSE*log2e values), so loads run two half-steps ahead.
 // ------------------------------------------------------------------------------------------------
@@ -247,10 +250,12 @@ struct __align__(1024) KvSmem {
   int32_t sched[kSchedKv];
   uint64_t bar_kv, bar_kv_empty;
   uint64_t bar_qdo[kKvRing], bar_qdo_empty[kKvRing];
-  uint64_t bar_sdp_full;    // S^T / dP^T of the current half are in the score buffer
-  uint64_t bar_sdp_free;    // the element-wise warps have loaded them (256 arrivals)
-  uint64_t bar_pds_ready;   // P^T / dS^T of the half are in the operand buffer (256 arrivals)
-  uint64_t bar_grads_done;  // the products of the half have completed (operand buffer reusable)
+  uint64_t bar_sdp_full[2];  // S^T / dP^T of a half are in score buffer b (one phase per half of b)
+  uint64_t bar_pds_ready[2];  // P^T / dS^T of a half are written in place in buffer b (256 arrivals).
+                              // One per buffer: a warp may start half x + 1 before a slower one
+                              // has arrived for half x (never x + 2, whose scores need the
+                              // products of x), so its arrival must not count toward x's phase
+  uint64_t bar_grads_done[2];  // the products of a half in buffer b have completed (b reusable)
   uint64_t bar_done;
   uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
   uint32_t tmem_base;
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   griddep_launch_dependents();  // after the wait: the dQ pass then starts only once its inputs exist
   if (prm.cta_clock && threadIdx.x == 0) prm.cta_clock[2 * blockIdx.x] = globaltimer_ns();
   const BwdScales sc = bwd_scales(prm.amax, prm.scale, prm.scale_log2);
-  constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDV = 256, kColDK = 384;
+  constexpr uint32_t kColBuf = 128, kColDP = 64, kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   KvSmem& s = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -279,10 +284,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&s.bar_qdo[i], 1);
       mbar_init(&s.bar_qdo_empty[i], 1);
     }
-    mbar_init(&s.bar_sdp_full, 1);
-    mbar_init(&s.bar_sdp_free, kVecWarps * 32);
-    mbar_init(&s.bar_pds_ready, kVecWarps * 32);
-    mbar_init(&s.bar_grads_done, 1);
+    mbar_init(&s.bar_sdp_full[0], 1);
+    mbar_init(&s.bar_sdp_full[1], 1);
+    mbar_init(&s.bar_pds_ready[0], kVecWarps * 32);
+    mbar_init(&s.bar_pds_ready[1], kVecWarps * 32);
+    mbar_init(&s.bar_grads_done[0], 1);
+    mbar_init(&s.bar_grads_done[1], 1);
     mbar_init(&s.bar_done, 1);
     for (int i = 0; i < kSchedKv; ++i) {
       mbar_init(&s.bar_sched_full[i], 1);
@@ -398,12 +405,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0][0]), kHalfRows * 128, 1024);      // MN-major
       const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0][0]), kHalfRows * 128, 1024);
       constexpr uint32_t kStage16 = (2 * kHalfRows * 128) >> 4;  // one ring stage, in 16-byte units
-      // S^T = K Q_h^T and dP^T = V dO_h^T of global half hx into the score buffer
+      // S^T = K Q_h^T and dP^T = V dO_h^T of global half hx into score buffer hx % 2
       auto sdp = [&](int hx) -> bool {
         const int hs = hx % kKvRing;
         if (!mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status)) return false;
         tc_fence_after();
-        const uint32_t d = tmem + kColS;
+        const uint32_t d = tmem + (hx & 1) * kColBuf;
         const uint64_t dq = dq0 + static_cast<uint64_t>(hs) * kStage16;
         const uint64_t ddo = ddo0 + static_cast<uint64_t>(hs) * kStage16;
 #pragma unroll
@@ -414,16 +421,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
-          mma_bf16_ss(d + (kColDP - kColS), sdesc_add(dv0, ko), sdesc_add(ddo, qo), id_sdp, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(d + kColDP, sdesc_add(dv0, ko), sdesc_add(ddo, qo), id_sdp, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&s.bar_sdp_full);
+        tc_commit(&s.bar_sdp_full[hx & 1]);
         return true;
       };
-      // acc += A (TMEM, 128 keys x 64 query rows) . B (the half's [64 rows][128 d], MN-major)
+      // acc += A (TMEM, 128 keys x 64 query rows) . B (the half's [64 rows][128 d], MN-major).  A's
+      // query rows 16 ks .. 16 ks + 15 sit in columns a_col + 8 (ks & 1) + 32 (ks >> 1): the 16
+      // packed columns of query rows [0,32) start at a_col, those of [32,64) at a_col + 32.
       auto grad = [&](uint32_t d, uint32_t a_col, uint64_t bdesc, bool acc) {
 #pragma unroll
         for (int ks = 0; ks < kHalfRows / 16; ++ks)
-          mma_bf16_ts(d, tmem + a_col + ks * 8, sdesc_add(bdesc, ks * 2048), id_mnb, (acc || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(d, tmem + a_col + (ks & 1) * 8 + (ks >> 1) * 32, sdesc_add(bdesc, ks * 2048), id_mnb,
+                      (acc || ks > 0) ? 1u : 0u);
       };
       for (int k = 0; ok; ++k) {
         const int i = next_from_ring(k);
@@ -436,26 +446,30 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           // dV += P^T dO and dK += dS^T Q as soon as the element-wise warps have a half
           for (int x = 0; ok && x < nh; ++x) {
             const int hx = G0 + x, hs = hx % kKvRing;
-            // exact parity: the next phase needs the warps' P / dS of half hx + 1, which wait for
-            // the grads_done commit below
-            if (!(ok = mbar_wait(&s.bar_pds_ready, hx & 1, prm.status))) break;
+            // exact parity: the next phase of pds_ready[hx % 2] needs the warps' P / dS of half
+            // hx + 2, whose scores wait for the products of half hx, issued after this wait
+            if (!(ok = mbar_wait(&s.bar_pds_ready[hx & 1], (hx >> 1) & 1, prm.status))) break;
             tc_fence_after();
             const uint64_t ddom = ddom0 + static_cast<uint64_t>(hs) * kStage16;
             const uint64_t dqm = dqm0 + static_cast<uint64_t>(hs) * kStage16;
-            grad(tmem + kColDV, kColP, ddom, x > 0);        // dV += P^T dO
-            grad(tmem + kColDK, kColP + 64, dqm, x > 0);    // dK += dS^T Q
+            const uint32_t buf = (hx & 1) * kColBuf;
+            grad(tmem + kColDV, buf, ddom, x > 0);            // dV += P^T dO
+            grad(tmem + kColDK, buf + kColDP, dqm, x > 0);    // dK += dS^T Q
             tc_commit(&s.bar_qdo_empty[hs]);
-            tc_commit(&s.bar_grads_done);                   // the operand buffer may be rewritten
+            tc_commit(&s.bar_grads_done[hx & 1]);             // score buffer hx % 2 may be rewritten
           }
           if (ok) tc_commit(&s.bar_done);
         } else {
-          // S^T / dP^T of each half once the warps have loaded the previous half's scores.  Exact
-          // parity: the next phase of sdp_free needs the scores of half hx, issued after the wait.
+          // S^T / dP^T of each half once the products of half hx - 2 have released its score
+          // buffer.  Exact parity: the next phase of grads_done[hx % 2] (the products of half hx)
+          // needs the scores this thread issues after the wait.  (With one barrier for both
+          // buffers the products of half hx - 1 could complete while this thread waits for the
+          // next block's K / V, two phases past the one it waits for.)
           if (!(ok = mbar_wait(&s.bar_kv, ucount & 1, prm.status))) break;
           ++ucount;
           for (int x = 0; ok && x < nh; ++x) {
             const int hx = G0 + x;
-            if (hx >= 1 && !(ok = mbar_wait(&s.bar_sdp_free, (hx - 1) & 1, prm.status))) break;
+            if (hx >= 2 && !(ok = mbar_wait(&s.bar_grads_done[hx & 1], ((hx - 2) >> 1) & 1, prm.status))) break;
             if (!(ok = sdp(hx))) break;
             if (x + 1 == nh) tc_commit(&s.bar_kv_empty);  // the block's last read of K and V
           }
@@ -490,20 +504,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         int qh, tile, qpos0;
         entry_rows(bg, prm.col[rp + (x >> 1)], qh, tile, qpos0);
         const int qp0 = qpos0 + (x & 1) * kHalfRows + c0;  // query position of column c0
-        // exact parity: the next phase of sdp_full needs the sdp_free arrival below
+        // exact parity: the next phase of sdp_full[hx % 2] (the scores of half hx + 2) waits for
+        // the products of half hx, which need the pds_ready arrival below
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status) &&
-                                         mbar_wait(&s.bar_sdp_full, hx & 1, prm.status));
+                                         mbar_wait(&s.bar_sdp_full[hx & 1], (hx >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
+        const uint32_t buf = tmem + lane_base + (hx & 1) * kColBuf + c0;  // this thread's S^T columns
         uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_base + kColS + c0, sr);
-        tmem_ld32(tmem + lane_base + kColDP + c0, dr);
+        tmem_ld32(buf, sr);
+        tmem_ld32(buf + kColDP, dr);
         tmem_ld_wait(sr);
 #pragma unroll
         for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
-        // the score buffer is free for the next half's S^T / dP^T
-        tc_fence_before();
-        mbar_arrive(&s.bar_sdp_free);
         const float4* nl2 = reinterpret_cast<const float4*>(s.lse2[hs] + c0);  // -LSE*log2e per query row
         const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D s_dS per query row
         const uint64_t sc2 = f2_pack(sc.c_s, sc.c_s), cdp2 = f2_pack(sc.c_dp, sc.c_dp);
@@ -542,19 +555,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             dh[c / 2] = pack_f16(g0, g1);
           }
         }
-        // the operand buffer is free once the previous half's products have completed (exact
-        // parity: grads_done's next phase needs the pds_ready arrival below)
-        if (hx >= 1) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_grads_done, (hx - 1) & 1, prm.status));
-          if (!ok) break;
-          tc_fence_after();
-        }
-        const uint32_t base = tmem + lane_base + kColP + hf * 16;
-        tmem_st16(base, ph);       // P^T: columns [128, 160)
-        tmem_st16(base + 64, dh);  // dS^T: columns [192, 224)
+        // in place, over the first 16 of the 32 columns this thread loaded
+        tmem_st16(buf, ph);           // P^T
+        tmem_st16(buf + kColDP, dh);  // dS^T
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&s.bar_pds_ready);
+        mbar_arrive(&s.bar_pds_ready[hx & 1]);
       }
       if (!ok) break;
       // ---- epilogue: dK = scale * acc, dV = acc (this thread: head-dim columns [hf*64, +64))
