@@ -235,10 +235,14 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 constexpr int kHalfRows = 64;
 constexpr int kKvRing = 4;
 constexpr int kSchedKv = 4;
-// warps: 0-7 element-wise, 8 scheduler + TMA, 9 issues dV / dK products, 10 issues S^T / dP^T.
-// Two issuing threads: tcgen05.mma issue blocks while the tensor pipe's queue is full, so with one
-// thread the next half's products would wait behind the previous half's score MMAs.
-constexpr int kKvThreads = (kVecWarps + 3) * 32;
+// warps: 0-7 element-wise, 8 scheduler + TMA, 9 issues dV / dK products, 10 issues S^T, 11 dP^T.
+// One thread issues a tcgen05.mma about every 70 clocks whatever its shape (measured: chains of
+// M = 128 MMAs with N = 64 or 128 from one thread run at 70-77 clocks each, two threads together
+// at 55), while an N = 64 MMA with both operands in shared memory occupies the tensor pipe ~48
+// clocks: the 16 score MMAs of a half from one thread would pace the whole pass, so S^T and dP^T
+// have a thread each.  The dQ pass's MMAs are N = 128 (64 clocks), and two issuers keep up there.
+constexpr int kKvThreads = (kVecWarps + 3) * 32;       // the Q-major pass
+constexpr int kKvPassThreads = (kVecWarps + 4) * 32;   // the KV-major pass
 
 struct __align__(1024) KvSmem {
   uint8_t k[2][kT * 128];                 // K tile [128 keys][64 d] x 2
@@ -262,7 +266,7 @@ struct __align__(1024) KvSmem {
 };
 
 template <bool kMask>  // kMask: a dense atten_mask is applied
-__global__ void __launch_bounds__(kKvThreads, 1)
+__global__ void __launch_bounds__(kKvPassThreads, 1)
     bsa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
                       const BwdParams prm) {
@@ -279,13 +283,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 
   if (tid == 0) {
     mbar_init(&s.bar_kv, 1);
-    mbar_init(&s.bar_kv_empty, 1);
+    mbar_init(&s.bar_kv_empty, 2);  // the block's last S^T and last dP^T
     for (int i = 0; i < kKvRing; ++i) {
       mbar_init(&s.bar_qdo[i], 1);
       mbar_init(&s.bar_qdo_empty[i], 1);
     }
-    mbar_init(&s.bar_sdp_full[0], 1);
-    mbar_init(&s.bar_sdp_full[1], 1);
+    mbar_init(&s.bar_sdp_full[0], 2);  // one commit each from the S^T and the dP^T thread
+    mbar_init(&s.bar_sdp_full[1], 2);
     mbar_init(&s.bar_pds_ready[0], kVecWarps * 32);
     mbar_init(&s.bar_pds_ready[1], kVecWarps * 32);
     mbar_init(&s.bar_grads_done[0], 1);
@@ -293,7 +297,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     mbar_init(&s.bar_done, 1);
     for (int i = 0; i < kSchedKv; ++i) {
       mbar_init(&s.bar_sched_full[i], 1);
-      mbar_init(&s.bar_sched_empty[i], 2 + kVecWarps * 32);
+      mbar_init(&s.bar_sched_empty[i], 3 + kVecWarps * 32);
     }
     fence_mbar_init();
   }
@@ -389,10 +393,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         mbar_wait(&s.bar_qdo[j % kKvRing], (j / kKvRing) & 1, prm.status);
       if (ucount > 0) mbar_wait(&s.bar_kv, (ucount - 1) & 1, prm.status);
     }
-  } else if (warp == kVecWarps + 1 || warp == kVecWarps + 2) {
+  } else if (warp >= kVecWarps + 1) {
     // ------------------------------------------------------------------ MMA issuers
     if (lane == 0) {
       const bool grads_thread = warp == kVecWarps + 1;
+      const bool dp_thread = warp == kVecWarps + 3;  // else S^T
       const uint32_t id_sdp = idesc_f16_f32(kT, kHalfRows, false, false);  // S^T, dP^T of a half
       const uint32_t id_mnb = idesc_f16_f32(kT, kD, false, true);          // dV, dK (B = [queries][d])
       int G0 = 0, ucount = 0;
@@ -405,23 +410,20 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0][0]), kHalfRows * 128, 1024);      // MN-major
       const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0][0]), kHalfRows * 128, 1024);
       constexpr uint32_t kStage16 = (2 * kHalfRows * 128) >> 4;  // one ring stage, in 16-byte units
-      // S^T = K Q_h^T and dP^T = V dO_h^T of global half hx into score buffer hx % 2
+      // S^T = K Q_h^T (the S^T thread) or dP^T = V dO_h^T (the dP^T thread) of global half hx into
+      // score buffer hx % 2
+      const uint64_t da0 = dp_thread ? dv0 : dk0, db0 = dp_thread ? ddo0 : dq0;
+      const uint32_t dcol = dp_thread ? kColDP : 0u;
       auto sdp = [&](int hx) -> bool {
         const int hs = hx % kKvRing;
         if (!mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status)) return false;
         tc_fence_after();
-        const uint32_t d = tmem + (hx & 1) * kColBuf;
-        const uint64_t dq = dq0 + static_cast<uint64_t>(hs) * kStage16;
-        const uint64_t ddo = ddo0 + static_cast<uint64_t>(hs) * kStage16;
+        const uint32_t d = tmem + (hx & 1) * kColBuf + dcol;
+        const uint64_t db = db0 + static_cast<uint64_t>(hs) * kStage16;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
-          mma_bf16_ss(d, sdesc_add(dk0, ko), sdesc_add(dq, qo), id_sdp, ks > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
-          mma_bf16_ss(d + kColDP, sdesc_add(dv0, ko), sdesc_add(ddo, qo), id_sdp, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(d, sdesc_add(da0, ko), sdesc_add(db, qo), id_sdp, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_sdp_full[hx & 1]);
         return true;
@@ -460,7 +462,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           }
           if (ok) tc_commit(&s.bar_done);
         } else {
-          // S^T / dP^T of each half once the products of half hx - 2 have released its score
+          // S^T (or dP^T) of each half once the products of half hx - 2 have released its score
           // buffer.  Exact parity: the next phase of grads_done[hx % 2] (the products of half hx)
           // needs the scores this thread issues after the wait.  (With one barrier for both
           // buffers the products of half hx - 1 could complete while this thread waits for the
@@ -471,7 +473,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const int hx = G0 + x;
             if (hx >= 2 && !(ok = mbar_wait(&s.bar_grads_done[hx & 1], ((hx - 2) >> 1) & 1, prm.status))) break;
             if (!(ok = sdp(hx))) break;
-            if (x + 1 == nh) tc_commit(&s.bar_kv_empty);  // the block's last read of K and V
+            if (x + 1 == nh) tc_commit(&s.bar_kv_empty);  // the block's last read of K (or V)
           }
         }
         G0 += nh;
@@ -1054,7 +1056,7 @@ cudaError_t bsa_bwd_launch(const BsaBwdArgs& a, const void* q, const void* k, co
     prof_begin("bsa_bwd_kv", st);
     pk.pdl_wait = 1;
     pk.cta_clock = prof_cta_clock(1, grid);
-    if (grid > 0) e = launch_pdl(kv_kernel, dim3(grid), dim3(kKvThreads), smem, st, tq64, tk128, tv128, tdo64, pk);
+    if (grid > 0) e = launch_pdl(kv_kernel, dim3(grid), dim3(kKvPassThreads), smem, st, tq64, tk128, tv128, tdo64, pk);
     prof_end(st);
     if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
     kv_launched = grid > 0;
