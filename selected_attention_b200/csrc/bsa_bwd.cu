@@ -229,6 +229,11 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 //   scores of half x + 2, so those of half x + 1 are already in the other buffer when the warps
 //   finish half x: the chain "warps load half x, then the scores of x + 1 start" of a single
 //   score buffer is gone, and the score MMAs of x + 1 overlap the warps' work on x.
+//   Each hand-off is split in two, so the critical loop (products of x -> scores of x + 2 ->
+//   element-wise work on x + 2 -> its products) moves in smaller steps: the warps turn S^T into
+//   P^T and store it as soon as S^T has landed (dV += P^T dO may start), then wait for dP^T and
+//   write dS^T (dK += dS^T Q); S^T of half x + 2 waits only for dV of half x (which read the S^T
+//   columns), dP^T of x + 2 only for dK of x.
 //   Shared memory: the block's K and V tiles, and a 4-stage ring of half entries (64 rows of Q
 //   and dO with their D and LSE*log2e values), so loads run two half-steps ahead.
 // ------------------------------------------------------------------------------------------------
@@ -254,12 +259,16 @@ struct __align__(1024) KvSmem {
   int32_t sched[kSchedKv];
   uint64_t bar_kv, bar_kv_empty;
   uint64_t bar_qdo[kKvRing], bar_qdo_empty[kKvRing];
-  uint64_t bar_sdp_full[2];  // S^T / dP^T of a half are in score buffer b (one phase per half of b)
-  uint64_t bar_pds_ready[2];  // P^T / dS^T of a half are written in place in buffer b (256 arrivals).
-                              // One per buffer: a warp may start half x + 1 before a slower one
-                              // has arrived for half x (never x + 2, whose scores need the
-                              // products of x), so its arrival must not count toward x's phase
-  uint64_t bar_grads_done[2];  // the products of a half in buffer b have completed (b reusable)
+  // one of each per score buffer b (one phase per half of b): a warp may start half x + 1 before a
+  // slower one has arrived for half x (never x + 2, whose scores need the products of x), so its
+  // arrivals must not count toward x's phase; and a score thread may wait for the next block's K / V
+  // between two halves, so its release barrier must not run two phases past it
+  uint64_t bar_s_full[2];    // S^T of a half has landed in buffer b
+  uint64_t bar_dp_full[2];   // dP^T of a half has landed
+  uint64_t bar_p_ready[2];   // P^T written in place (256 arrivals)
+  uint64_t bar_ds_ready[2];  // dS^T written in place (256 arrivals)
+  uint64_t bar_dv_done[2];   // dV += P^T dO of the half has completed (the S^T columns are free)
+  uint64_t bar_dk_done[2];   // dK += dS^T Q has completed (the dP^T columns are free)
   uint64_t bar_done;
   uint64_t bar_sched_full[kSchedKv], bar_sched_empty[kSchedKv];
   uint32_t tmem_base;
@@ -288,12 +297,14 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
       mbar_init(&s.bar_qdo[i], 1);
       mbar_init(&s.bar_qdo_empty[i], 1);
     }
-    mbar_init(&s.bar_sdp_full[0], 2);  // one commit each from the S^T and the dP^T thread
-    mbar_init(&s.bar_sdp_full[1], 2);
-    mbar_init(&s.bar_pds_ready[0], kVecWarps * 32);
-    mbar_init(&s.bar_pds_ready[1], kVecWarps * 32);
-    mbar_init(&s.bar_grads_done[0], 1);
-    mbar_init(&s.bar_grads_done[1], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s.bar_s_full[b], 1);
+      mbar_init(&s.bar_dp_full[b], 1);
+      mbar_init(&s.bar_p_ready[b], kVecWarps * 32);
+      mbar_init(&s.bar_ds_ready[b], kVecWarps * 32);
+      mbar_init(&s.bar_dv_done[b], 1);
+      mbar_init(&s.bar_dk_done[b], 1);
+    }
     mbar_init(&s.bar_done, 1);
     for (int i = 0; i < kSchedKv; ++i) {
       mbar_init(&s.bar_sched_full[i], 1);
@@ -425,7 +436,7 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
           const uint32_t ko = (ks >> 2) * (kT * 128) + (ks & 3) * 32, qo = (ks >> 2) * (kHalfRows * 128) + (ks & 3) * 32;
           mma_bf16_ss(d, sdesc_add(da0, ko), sdesc_add(db, qo), id_sdp, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&s.bar_sdp_full[hx & 1]);
+        tc_commit(dp_thread ? &s.bar_dp_full[hx & 1] : &s.bar_s_full[hx & 1]);
         return true;
       };
       // acc += A (TMEM, 128 keys x 64 query rows) . B (the half's [64 rows][128 d], MN-major).  A's
@@ -448,30 +459,32 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
           // dV += P^T dO and dK += dS^T Q as soon as the element-wise warps have a half
           for (int x = 0; ok && x < nh; ++x) {
             const int hx = G0 + x, hs = hx % kKvRing;
-            // exact parity: the next phase of pds_ready[hx % 2] needs the warps' P / dS of half
-            // hx + 2, whose scores wait for the products of half hx, issued after this wait
-            if (!(ok = mbar_wait(&s.bar_pds_ready[hx & 1], (hx >> 1) & 1, prm.status))) break;
-            tc_fence_after();
-            const uint64_t ddom = ddom0 + static_cast<uint64_t>(hs) * kStage16;
-            const uint64_t dqm = dqm0 + static_cast<uint64_t>(hs) * kStage16;
+            // exact parity: the next phase of p_ready[hx % 2] needs the warps' P of half hx + 2,
+            // whose S^T waits for the dV product of half hx, issued after this wait (the same for
+            // ds_ready, dP^T and dK)
             const uint32_t buf = (hx & 1) * kColBuf;
-            grad(tmem + kColDV, buf, ddom, x > 0);            // dV += P^T dO
-            grad(tmem + kColDK, buf + kColDP, dqm, x > 0);    // dK += dS^T Q
+            if (!(ok = mbar_wait(&s.bar_p_ready[hx & 1], (hx >> 1) & 1, prm.status))) break;
+            tc_fence_after();
+            grad(tmem + kColDV, buf, ddom0 + static_cast<uint64_t>(hs) * kStage16, x > 0);  // dV += P^T dO
+            tc_commit(&s.bar_dv_done[hx & 1]);
+            if (!(ok = mbar_wait(&s.bar_ds_ready[hx & 1], (hx >> 1) & 1, prm.status))) break;
+            tc_fence_after();
+            grad(tmem + kColDK, buf + kColDP, dqm0 + static_cast<uint64_t>(hs) * kStage16, x > 0);  // dK += dS^T Q
             tc_commit(&s.bar_qdo_empty[hs]);
-            tc_commit(&s.bar_grads_done[hx & 1]);             // score buffer hx % 2 may be rewritten
+            tc_commit(&s.bar_dk_done[hx & 1]);
           }
           if (ok) tc_commit(&s.bar_done);
         } else {
-          // S^T (or dP^T) of each half once the products of half hx - 2 have released its score
-          // buffer.  Exact parity: the next phase of grads_done[hx % 2] (the products of half hx)
-          // needs the scores this thread issues after the wait.  (With one barrier for both
-          // buffers the products of half hx - 1 could complete while this thread waits for the
-          // next block's K / V, two phases past the one it waits for.)
+          // S^T (dP^T) of each half once the dV (dK) product of half hx - 2 has released its
+          // columns of the score buffer.  Exact parity: the next phase of dv_done[hx % 2] (dV of
+          // half hx) needs the scores this thread issues after the wait.
           if (!(ok = mbar_wait(&s.bar_kv, ucount & 1, prm.status))) break;
           ++ucount;
           for (int x = 0; ok && x < nh; ++x) {
             const int hx = G0 + x;
-            if (hx >= 2 && !(ok = mbar_wait(&s.bar_grads_done[hx & 1], ((hx - 2) >> 1) & 1, prm.status))) break;
+            if (hx >= 2 && !(ok = mbar_wait(dp_thread ? &s.bar_dk_done[hx & 1] : &s.bar_dv_done[hx & 1],
+                                            ((hx - 2) >> 1) & 1, prm.status)))
+              break;
             if (!(ok = sdp(hx))) break;
             if (x + 1 == nh) tc_commit(&s.bar_kv_empty);  // the block's last read of K (or V)
           }
@@ -506,19 +519,16 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
         int qh, tile, qpos0;
         entry_rows(bg, prm.col[rp + (x >> 1)], qh, tile, qpos0);
         const int qp0 = qpos0 + (x & 1) * kHalfRows + c0;  // query position of column c0
-        // exact parity: the next phase of sdp_full[hx % 2] (the scores of half hx + 2) waits for
-        // the products of half hx, which need the pds_ready arrival below
+        // exact parity: the next phase of s_full[hx % 2] (S^T of half hx + 2) waits for the dV
+        // product of half hx, which needs the p_ready arrival below (the same for dp_full)
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_qdo[hs], (hx / kKvRing) & 1, prm.status) &&
-                                         mbar_wait(&s.bar_sdp_full[hx & 1], (hx >> 1) & 1, prm.status));
+                                         mbar_wait(&s.bar_s_full[hx & 1], (hx >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
         const uint32_t buf = tmem + lane_base + (hx & 1) * kColBuf + c0;  // this thread's S^T columns
         uint32_t sr[32], dr[32];
         tmem_ld32(buf, sr);
-        tmem_ld32(buf + kColDP, dr);
         tmem_ld_wait(sr);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
         const float4* nl2 = reinterpret_cast<const float4*>(s.lse2[hs] + c0);  // -LSE*log2e per query row
         const float4* nd = reinterpret_cast<const float4*>(s.dvec[hs] + c0);   // -D s_dS per query row
         const uint64_t sc2 = f2_pack(sc.c_s, sc.c_s), cdp2 = f2_pack(sc.c_dp, sc.c_dp);
@@ -533,9 +543,10 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
         }
         const bool full = qp0 >= qlo && qp0 + 31 <= qhi && mbits == 0;
         uint32_t ph[16], dh[16];
+        // P = exp2(S c_s - LSE log2e), kept in fp32 (over the scores) for dS
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 L = nl2[c4], Dn = nd[c4];
+          const float4 L = nl2[c4];
 #pragma unroll
           for (int hp = 0; hp < 2; ++hp) {
             const int c = c4 * 4 + hp * 2;
@@ -548,21 +559,40 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
               if (qp0 + c < qlo || qp0 + c > qhi || ((mbits >> c) & 1u)) p0 = 0.f;
               if (qp0 + c + 1 < qlo || qp0 + c + 1 > qhi || ((mbits >> (c + 1)) & 1u)) p1 = 0.f;
             }
-            // dS (in its fp16 scale) = P (dP c_dp - D s_dS)
-            float g0, g1;
-            f2_unpack(f2_mul(f2_pack(p0, p1), f2_fma(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), cdp2,
-                                                    hp ? f2_pack(Dn.z, Dn.w) : f2_pack(Dn.x, Dn.y))),
-                      g0, g1);
+            sr[c] = __float_as_uint(p0);
+            sr[c + 1] = __float_as_uint(p1);
             ph[c / 2] = pack_f16(p0, p1);
+          }
+        }
+        // in place, over the first 16 of the 32 S^T columns this thread loaded
+        tmem_st16(buf, ph);  // P^T
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&s.bar_p_ready[hx & 1]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_dp_full[hx & 1], (hx >> 1) & 1, prm.status));
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld32(buf + kColDP, dr);
+        tmem_ld_wait(dr);
+        // dS (in its fp16 scale) = P (dP c_dp - D s_dS)
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 Dn = nd[c4];
+#pragma unroll
+          for (int hp = 0; hp < 2; ++hp) {
+            const int c = c4 * 4 + hp * 2;
+            float g0, g1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                             f2_fma(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), cdp2,
+                                    hp ? f2_pack(Dn.z, Dn.w) : f2_pack(Dn.x, Dn.y))),
+                      g0, g1);
             dh[c / 2] = pack_f16(g0, g1);
           }
         }
-        // in place, over the first 16 of the 32 columns this thread loaded
-        tmem_st16(buf, ph);           // P^T
-        tmem_st16(buf + kColDP, dh);  // dS^T
+        tmem_st16(buf + kColDP, dh);  // dS^T, over the first 16 of this thread's dP^T columns
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&s.bar_pds_ready[hx & 1]);
+        mbar_arrive(&s.bar_ds_ready[hx & 1]);
       }
       if (!ok) break;
       // ---- epilogue: dK = scale * acc, dV = acc (this thread: head-dim columns [hf*64, +64))
