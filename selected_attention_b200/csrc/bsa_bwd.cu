@@ -514,10 +514,15 @@ __global__ void __launch_bounds__(kKvPassThreads, 1)
       else if (prm.mask_mode == 3) qlo = kpos - shift;
       else if (prm.mask_mode == 4) { qlo = kpos - shift - prm.win_right; qhi = kpos - shift + prm.win_left; }
       if (!key_valid) { qlo = 1; qhi = 0; }
+      // the list entry of the next half is read one half ahead: a global load on this loop's
+      // critical path otherwise (~350 clocks per half)
+      int code_next = n > 0 ? prm.col[rp] : 0;
       for (int x = 0; x < 2 * n; ++x) {
         const int hx = G0 + x, hs = hx % kKvRing;
+        const int code = code_next;
+        if (x + 1 < 2 * n) code_next = prm.col[rp + ((x + 1) >> 1)];
         int qh, tile, qpos0;
-        entry_rows(bg, prm.col[rp + (x >> 1)], qh, tile, qpos0);
+        entry_rows(bg, code, qh, tile, qpos0);
         const int qp0 = qpos0 + (x & 1) * kHalfRows + c0;  // query position of column c0
         // exact parity: the next phase of s_full[hx % 2] (S^T of half hx + 2) waits for the dV
         // product of half hx, which needs the p_ready arrival below (the same for dp_full)
@@ -884,13 +889,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const size_t trow = static_cast<size_t>(bh * prm.nqb + qb) * kT + r;
       const uint64_t nl2 = f2_pack(prm.lse2[trow], prm.lse2[trow]);  // -LSE*log2e of the row, twice
       const uint64_t nd2 = f2_pack(prm.dvec[trow], prm.dvec[trow]);  // -D s_dS of the row, twice
+      int col_next = n > 0 ? prm.col[rp] : 0;  // read one tile ahead, before the wait
       for (int j = 0; j < n; ++j) {
         const int J = J0 + j, st = J & 1;
         const uint32_t s_col = st ? kColS1 : kColS0;
+        const int cj = col_next;
+        if (j + 1 < n) col_next = prm.col[rp + j + 1];
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (J >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
-        const int kpos0 = prm.col[rp + j] * prm.by + c0;
+        const int kpos0 = cj * prm.by + c0;
         const bool full = kpos0 >= lo && kpos0 + kHalf - 1 <= hi;
         float p[kHalf];
 #pragma unroll

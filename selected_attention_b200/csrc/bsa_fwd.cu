@@ -308,14 +308,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       else if (prm.mask_mode == 4) { lo = qq - prm.win_left; hi = min(hi, qq + prm.win_right); }
       if (!row_valid) { lo = 1; hi = 0; }
       float m = -INFINITY, l = 0.f;  // l: partial sum over this thread's columns
+      int col_next = n > 0 ? prm.col[rp] : 0;  // read one tile ahead, before the wait
       for (int j = 0; j < n; ++j) {
         const int J = J0 + j;
         const int st = J & 1;
+        const int cj = col_next;
+        if (j + 1 < n) col_next = prm.col[rp + j + 1];
         ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[st], (J >> 1) & 1, prm.status));
         if (!ok) break;
         tc_fence_after();
         const uint32_t s_col = st ? kColS1 : kColS0;
-        const int kpos0 = prm.col[rp + j] * prm.by + hf * kHalf;
+        const int kpos0 = cj * prm.by + hf * kHalf;
         // the dense atten_mask inside the selected block: bit c = this row may not see column c
         const uint64_t mbits = kMask && row_valid
                                    ? dense_mask_bits<kHalf>(prm.amask + static_cast<size_t>(qpos) * prm.S_kv, kpos0,
