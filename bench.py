@@ -68,19 +68,19 @@ def with_spec(roof):
 # capture of each kernel, valid only while the kernel's source file is unchanged (sha1 prefix of
 # the file recorded at capture time); reported as null once the source has changed.
 NCU_TRAFFIC = [
-    {"kernel": "bsa_bwd_kv", "bytes": 491879936 + 103701504, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-     "src_sha1": "0e7611c58dfc"},
-    {"kernel": "bsa_bwd_q", "bytes": 270693632 + 51921664, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-     "src_sha1": "0e7611c58dfc"},
-    {"kernel": "bsa_fwd", "bytes": 201467648 + 52431360, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
-     "src_sha1": "f1562c183dfe"},
+    {"kernel": "bsa_bwd_kv", "bytes": 492699648 + 103334144, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+     "src_sha1": "0143e70727d3"},
+    {"kernel": "bsa_bwd_q", "bytes": 270674688 + 52001024, "config": 2, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+     "src_sha1": "0143e70727d3"},
+    {"kernel": "bsa_fwd", "bytes": 201507840 + 52752640, "config": 2, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+     "src_sha1": "3b1165691fa4"},
     # full-size launches of the S=131072 workload (one-pass DRAM counters)
-    {"kernel": "bsa_bwd_kv", "bytes": 12192800256 + 2115727104, "config": 5,
-     "src": "selected_attention_b200/csrc/bsa_bwd.cu", "src_sha1": "0e7611c58dfc"},
-    {"kernel": "bsa_bwd_q", "bytes": 5642680576 + 1057762560, "config": 5, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
-     "src_sha1": "0e7611c58dfc"},
-    {"kernel": "bsa_fwd", "bytes": 4284632064 + 1075282176, "config": 5, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
-     "src_sha1": "f1562c183dfe"},
+    {"kernel": "bsa_bwd_kv", "bytes": 12216385024 + 2114009088, "config": 5,
+     "src": "selected_attention_b200/csrc/bsa_bwd.cu", "src_sha1": "0143e70727d3"},
+    {"kernel": "bsa_bwd_q", "bytes": 5664402432 + 1057575936, "config": 5, "src": "selected_attention_b200/csrc/bsa_bwd.cu",
+     "src_sha1": "0143e70727d3"},
+    {"kernel": "bsa_fwd", "bytes": 4296163840 + 1075880960, "config": 5, "src": "selected_attention_b200/csrc/bsa_fwd.cu",
+     "src_sha1": "3b1165691fa4"},
     {"kernel": "sfa_decode", "bytes": 147508480 + 4237312, "config": 4, "src": "selected_attention_b200/csrc/sfa_decode.cu",
      "src_sha1": "6c80d26dac90"},
 ]
